@@ -1,0 +1,443 @@
+"""Pins of the oracle against things other than itself: hand-derived values
+(tests/golden), closed forms, invariants, library routines run as a
+cross-check (torch's float8_e4m3fn and bfloat16 casts, numpy's fp64 matmul),
+and brute force on tiny inputs.  Each pin is chosen so that a plausible slip in
+the oracle (a dropped term, a wrong sign or index, a transposed operand, a
+wrong tie rule) fails at least one of them.  CPU only."""
+
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "e4m3_hand.txt")
+
+
+def _golden(kind):
+    rows = []
+    with open(GOLDEN) as f:
+        for line in f:
+            if line.startswith(kind + " "):
+                rows.append(line.split()[1:])
+    assert rows
+    return rows
+
+
+def bits_of(t: torch.Tensor) -> np.ndarray:
+    """BF16 torch tensor -> uint16 numpy bit patterns."""
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def torch_e4m3(values_f32: np.ndarray) -> np.ndarray:
+    """Library cross-check: clamp to +-448 ourselves, then let torch cast."""
+    t = torch.from_numpy(np.clip(values_f32, -448.0, 448.0).astype(np.float32))
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def bitfield_decode(c: int) -> float:
+    """Independent decode of one code from its bit fields with ldexp."""
+    s = -1.0 if c & 0x80 else 1.0
+    e = (c >> 3) & 0xF
+    m = c & 7
+    if e == 15 and m == 7:
+        return math.nan
+    if e == 0:
+        return s * math.ldexp(m, -9)
+    return s * math.ldexp(8 + m, e - 10)
+
+
+# ------------------------------------------------------------------ codebook
+
+
+def test_codebook_closed_form():
+    cb = oracle.codebook()
+    assert cb.shape == (256,)
+    assert np.isnan(cb).sum() == 2 and np.isnan(cb[0x7F]) and np.isnan(cb[0xFF])
+    assert np.isfinite(cb).sum() == 254
+    assert cb[0x7E] == 448.0 and cb[0xFE] == -448.0
+    assert np.nanmax(cb) == 448.0
+    assert cb[0x08] == 2.0 ** -6 and cb[0x01] == 2.0 ** -9
+    # magnitude strictly increasing in the low 7 bits
+    pos = cb[0:0x7F]
+    assert np.all(np.diff(pos) > 0)
+    # the negative half mirrors the positive half
+    assert np.array_equal(cb[0x80:0xFF], -cb[0:0x7F])
+
+
+def test_codebook_bitfield_decode():
+    cb = oracle.codebook()
+    for c in range(256):
+        v = bitfield_decode(c)
+        if math.isnan(v):
+            assert np.isnan(cb[c])
+        else:
+            assert cb[c] == v, hex(c)
+
+
+def test_codebook_matches_torch_float8():
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    tv = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    cb = oracle.codebook()
+    same = (tv == cb) | (np.isnan(tv) & np.isnan(cb))
+    assert same.all()
+
+
+def test_golden_decode():
+    cb = oracle.codebook()
+    for code, val in _golden("decode"):
+        assert cb[int(code, 16)] == float(val), code
+
+
+# ------------------------------------------------------------------ quantize
+
+
+def test_golden_quant():
+    for v, s, code in _golden("quant"):
+        assert oracle.quant_f32(float(v), float(s)) == int(code, 16), (v, s)
+
+
+@pytest.mark.parametrize("s", [1.0, 2.0 ** -5, 8.0])
+def test_roundtrip_every_finite_code(s):
+    cb = oracle.codebook()
+    for c in range(256):
+        if np.isnan(cb[c]):
+            continue
+        v = np.float32(cb[c] * s)
+        assert oracle.quant_f32(float(v), s) == c, hex(c)
+
+
+def test_idempotence_and_saturation():
+    rng = np.random.default_rng(0)
+    x = (rng.standard_t(3, size=20000) * 50).astype(np.float32)
+    xb = bits_of(torch.from_numpy(x).to(torch.bfloat16))
+    s = oracle.f32(0.37)
+    q = oracle.quantize(xb, s)
+    deq = oracle.dequant(q)
+    # q(deq(q(x)) * s) == q(x)
+    re = np.array([oracle.quant_f32(float(np.float32(d * s)), s) for d in deq])
+    # (the fp32 product d*s is off by at most 2^-24 relative, far from any
+    # rounding midpoint, which sits at least 1/16 of a value away)
+    assert np.array_equal(re, q)
+    xv = oracle.bf16_to_f64(xb)
+    big = np.abs(xv) >= 448.0 * s * (1 + 1e-6)
+    assert big.any()
+    assert np.all(q[big & (xv > 0)] == 0x7E)
+    assert np.all(q[big & (xv < 0)] == 0xFE)
+
+
+def test_ties_go_to_even_codes():
+    cb = oracle.codebook()
+    for c in range(0, 0x7E):
+        mid = (cb[c] + cb[c + 1]) / 2.0  # exact in fp32 for E4M3 neighbours
+        assert np.float32(mid) == mid
+        want = c if c % 2 == 0 else c + 1
+        assert oracle.quant_f32(mid, 1.0) == want, hex(c)
+        assert oracle.quant_f32(-mid, 1.0) == (0x80 | want)
+
+
+def test_quantize_matches_torch_cast_after_clamp():
+    rng = np.random.default_rng(1)
+    x = np.concatenate([
+        rng.standard_normal(50000) * 3,
+        rng.standard_t(4, size=50000) * 100,
+        rng.standard_normal(5000) * 1e-3,
+    ]).astype(np.float32)
+    xb = bits_of(torch.from_numpy(x).to(torch.bfloat16))
+    for s in (1.0, oracle.f32(0.0123), oracle.f32(1.7)):
+        q = oracle.quantize(xb, s)
+        xf = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).float()
+        t = (xf / torch.tensor(s, dtype=torch.float32)).numpy()  # IEEE fp32 divide
+        assert np.array_equal(q, torch_e4m3(t)), s
+
+
+def test_zero_sign_and_nan():
+    assert oracle.quant_f32(0.0, 1.0) == 0x00
+    assert oracle.quant_f32(-0.0, 1.0) == 0x80
+    assert oracle.quant_f32(-1e-12, 1.0) == 0x80
+    assert oracle.quant_f32(float("nan"), 1.0) & 0x7F == 0x7F
+
+
+def test_fp32_divide_not_reciprocal():
+    """The scale is a divisor: find a case where x * (1/s) and x / s round to
+    different fp32 values and check the oracle follows the divide."""
+    rng = np.random.default_rng(2)
+    s = np.float32(0.3)
+    xs = rng.standard_normal(200000).astype(np.float32) * 100
+    div = xs / s
+    mul = xs * (np.float32(1.0) / s)
+    idx = np.nonzero(div != mul)[0]
+    assert idx.size > 0
+    got = np.array([oracle.quant_f32(float(xs[i]), float(s)) for i in idx[:200]])
+    want = torch_e4m3(div[idx[:200]])
+    assert np.array_equal(got, want)
+
+
+# --------------------------------------------------------------- bf16 round
+
+
+def test_round_bf16_matches_torch_on_fp32_inputs():
+    rng = np.random.default_rng(3)
+    f = np.concatenate([
+        rng.standard_normal(100000).astype(np.float32) * 1e3,
+        (rng.standard_normal(20000) * 1e-38).astype(np.float32),  # subnormals
+        np.array([3.3e38, -3.3e38, 3.39e38, 1.0, 1.00390625, 1.01171875], dtype=np.float32),
+    ])
+    got = oracle.round_bf16(f.astype(np.float64))
+    want = bits_of(torch.from_numpy(f).to(torch.bfloat16))
+    assert np.array_equal(got, want)
+
+
+def test_round_bf16_single_rounding():
+    # 1 + 2^-8 + 2^-40 is just above the midpoint of 1 and 1+2^-7: must go up,
+    # while rounding through fp32 first would land on the tie and go to even (1.0).
+    x = 1.0 + 2.0 ** -8 + 2.0 ** -40
+    assert oracle.round_bf16(np.array([x]))[0] == 0x3F81
+    assert oracle.round_bf16(np.array([1.0 + 2.0 ** -8]))[0] == 0x3F80
+
+
+# ---------------------------------------------------------------- observer
+
+
+def test_golden_observer():
+    for maxima, want in _golden("observer"):
+        a = [float(v) for v in maxima.split(",")]
+        assert abs(oracle.moving_average(a) - float(want)) < 1e-12
+
+
+def test_observer_closed_forms():
+    assert oracle.moving_average([5.0] * 16) == 5.0
+    a1, a2 = 3.0, 7.5
+    assert abs(oracle.moving_average([a1, a2]) - (0.99 * a1 + 0.01 * a2)) < 1e-15
+    # geometric closed form: a_1 = 0 then constant a gives A_B = a (1 - 0.99^(B-1))
+    B, a = 16, 2.0
+    got = oracle.moving_average([0.0] + [a] * (B - 1))
+    assert abs(got - a * (1 - 0.99 ** (B - 1))) < 1e-12
+    assert oracle.scale_from_amax(448.0) == 1.0
+    assert oracle.scale_from_amax(4.04) == np.float32(4.04 / 448.0)
+
+
+def test_observer_clips_heavy_tails():
+    """With heavy-tailed batches the moving average sits below the largest
+    batch maximum, so the rarest activations saturate."""
+    data = synth.c1_linear(256, 2048, n_calib=16, calib_rows=64)
+    s = oracle.observer_scale([bits_of(b) for b in data["calib"]])
+    maxima = [oracle.absmax(bits_of(b)) for b in data["calib"]]
+    assert s * 448.0 < max(maxima)
+    q = oracle.quantize(bits_of(data["x"]), s)
+    assert ((q & 0x7F) == 0x7E).any()
+
+
+def test_rtn_weight():
+    w = synth.normal((64, 96), 0.02, 123)
+    wb = bits_of(w)
+    wq, sw = oracle.rtn_weight(wb)
+    amax = np.abs(oracle.bf16_to_f64(wb)).max()
+    assert sw == np.float32(np.float32(amax) / np.float32(448.0))
+    # the largest weight maps to the largest code
+    i = np.argmax(np.abs(oracle.bf16_to_f64(wb)))
+    assert wq.ravel()[i] & 0x7F == 0x7E
+    # dequantized error within half a step of the grid around each value
+    err = np.abs(oracle.dequant(wq) * sw - oracle.bf16_to_f64(wb))
+    assert np.all(err <= np.abs(oracle.bf16_to_f64(wb)) * 2.0 ** -4 + 2.0 ** -10 * sw)
+
+
+# ------------------------------------------------------------------- linear
+
+
+def test_linear_integer_exact():
+    """Integer-valued codes with unit scales: exact integer arithmetic."""
+    rng = np.random.default_rng(4)
+    ints = {int(c): v for c, v in enumerate(oracle.codebook()) if np.isfinite(v) and v == int(v) and abs(v) <= 4}
+    codes = np.array(list(ints.keys()), dtype=np.uint8)
+    M, N, K = 5, 7, 15
+    xq = rng.choice(codes, size=(M, K)).astype(np.uint8)
+    wq = rng.choice(codes, size=(N, K)).astype(np.uint8)
+    y = oracle.linear(xq, wq, 1.0, 1.0)
+    xi = np.vectorize(ints.get)(xq).astype(np.int64)
+    wi = np.vectorize(ints.get)(wq).astype(np.int64)
+    ref = xi @ wi.T
+    assert np.all(np.abs(ref) < 256)  # exact in bf16 (8 significant bits)
+    assert np.array_equal(oracle.bf16_to_f64(y), ref.astype(np.float64))
+
+
+def test_linear_matches_numpy_fp64_matmul():
+    rng = np.random.default_rng(5)
+    M, N, K = 9, 13, 160
+    xq = rng.integers(0, 256, size=(M, K), dtype=np.uint8)
+    wq = rng.integers(0, 256, size=(N, K), dtype=np.uint8)
+    xq[(xq & 0x7F) == 0x7F] = 0x3A
+    wq[(wq & 0x7F) == 0x7F] = 0xB1
+    s_in, s_w = oracle.f32(0.0137), oracle.f32(0.00021)
+    y = oracle.linear(xq, wq, s_in, s_w)
+    cb = oracle.codebook()
+    acc = cb[xq] @ cb[wq].T  # exact: every partial sum fits in fp64
+    ref = oracle.round_bf16((float(s_in) * float(s_w)) * acc)
+    assert np.array_equal(y, ref)
+    # and the orientation matters: Y[m, n] uses row n of W
+    assert not np.array_equal(y[:, :M], oracle.round_bf16((float(s_in) * float(s_w)) * (cb[xq] @ cb[wq][:M].T).T[:M]))
+
+
+def test_linear_torch_cross_check():
+    """Library cross-check through torch: fp64 matmul then torch's bf16 cast
+    (which may round twice, so allow one BF16 ulp on a tiny fraction)."""
+    rng = np.random.default_rng(6)
+    M, N, K = 16, 24, 256
+    xq = rng.integers(0, 0x7E, size=(M, K), dtype=np.uint8) | (rng.integers(0, 2, size=(M, K), dtype=np.uint8) << 7)
+    wq = rng.integers(0, 0x7E, size=(N, K), dtype=np.uint8) | (rng.integers(0, 2, size=(N, K), dtype=np.uint8) << 7)
+    y = oracle.linear(xq, wq, 0.5, 0.25)
+    xt = torch.from_numpy(xq).view(torch.float8_e4m3fn).double()
+    wt = torch.from_numpy(wq).view(torch.float8_e4m3fn).double()
+    ref = bits_of(((xt @ wt.T) * 0.125).to(torch.bfloat16))
+    diff = np.abs(y.astype(np.int32) - ref.astype(np.int32))
+    assert diff.max() <= 1 and (diff > 0).mean() < 1e-2
+
+
+# ------------------------------------------------------------------- swiglu
+
+
+def test_swiglu_2in_equals_fused_split_form():
+    d = synth.c2_swiglu(1024, 8192, device="cpu", n_calib=0)
+    g = bits_of(d["g"][:32, :704].contiguous())
+    u = bits_of(d["u"][:32, :704].contiguous())
+    s = oracle.f32(0.031)
+    h2 = oracle.silu_mul_2in(g, u, s)
+    gu = np.concatenate([g, u], axis=1)
+    hf = oracle.silu_and_mul_fused(gu, s)
+    assert np.array_equal(h2, hf)
+    # swapping gate and up is a different function: the pin can tell them apart
+    assert not np.array_equal(h2, oracle.silu_mul_2in(u, g, s))
+
+
+def test_swiglu_special_cases():
+    s = 1.0
+    zero = bits_of(torch.zeros(8, dtype=torch.bfloat16))
+    u = bits_of(torch.linspace(-4, 4, 8).to(torch.bfloat16))
+    h = oracle.silu_mul_2in(zero, u, s)
+    assert np.all((h & 0x7F) == 0)  # SiLU(0) = 0
+    # large positive g: SiLU(g) * u -> g * u; large negative g: -> 0
+    g = bits_of(torch.full((8,), 40.0).to(torch.bfloat16))
+    u = bits_of(torch.tensor([0.5, 1, 2, 3, -1, -2, 0.25, 5]).to(torch.bfloat16))
+    h = oracle.silu_mul_2in(g, u, s)
+    want = [oracle.quant_f64(40.0 * float(v), 1.0) for v in oracle.bf16_to_f64(u)]
+    assert list(h) == want
+    gneg = bits_of(torch.full((8,), -60.0).to(torch.bfloat16))
+    assert np.all((oracle.silu_mul_2in(gneg, u, s) & 0x7F) == 0)
+
+
+def test_swiglu_independent_sigmoid_form():
+    """SiLU written another way: g * (1 + tanh(g/2)) / 2.  Codes agree except
+    where the fp64 value lies within rounding noise of a code boundary."""
+    d = synth.c2_swiglu(1024, 8192, device="cpu", n_calib=0)
+    g = bits_of(d["g"][:16, :1024].contiguous())
+    u = bits_of(d["u"][:16, :1024].contiguous())
+    s = oracle.f32(0.02)
+    h = oracle.silu_mul_2in(g, u, s)
+    gv, uv = oracle.bf16_to_f64(g), oracle.bf16_to_f64(u)
+    v = gv * (1.0 + np.tanh(gv / 2.0)) / 2.0 * uv / float(s)
+    want = torch_e4m3(np.clip(v, -448, 448).astype(np.float32))
+    # fp32 rounding of v may move a value across a tie; allow 1e-4 of elements
+    assert (h != want).mean() < 1e-4
+
+
+def test_swiglu_quantize_saturates():
+    g = bits_of(torch.full((4,), 8.0).to(torch.bfloat16))
+    u = bits_of(torch.tensor([100.0, -100.0, 1.0, -1.0]).to(torch.bfloat16))
+    h = oracle.silu_mul_2in(g, u, 0.5)
+    assert list(h[:2]) == [0x7E, 0xFE]
+
+
+# ---------------------------------------------------- shared quant and groups
+
+
+def test_shared_quant_equals_three_separate_quantizations():
+    d = synth.c3_qkv(n_calib=0)
+    x = bits_of(d["x"][:48].contiguous())
+    s = oracle.f32(0.05)
+    wqs = []
+    for name in ("wq", "wk", "wv"):
+        wq, sw = oracle.rtn_weight(bits_of(d[name][:40].contiguous()))
+        wqs.append((wq, sw))
+    shared = oracle.qkv_shared_quant(x, s, wqs)
+    separate = [oracle.linear(oracle.quantize(x, s), wq, s, sw) for wq, sw in wqs]
+    for a, b in zip(shared, separate):
+        assert np.array_equal(a, b)
+
+
+def test_shared_scale_invariant():
+    s = np.float32(0.0123)
+    assert oracle.shared_scales_equal([s, s, s])
+    one_ulp = np.nextafter(s, np.float32(1))
+    assert not oracle.shared_scales_equal([s, s, one_ulp])
+    assert not oracle.shared_scales_equal([0.0, 0.0])
+    assert not oracle.shared_scales_equal([np.inf, np.inf])
+    assert not oracle.shared_scales_equal([-s, -s])
+
+
+def test_fused_group_requant_changes_codes_split_keeps_them():
+    """Group with genuinely different weight scales (asserted first): the
+    fused loader's second rounding changes codes; the split path keeps the
+    calibrated codes exactly."""
+    wg = bits_of(synth.normal((64, 128), 0.02, 7))
+    wu = bits_of(synth.normal((64, 128), 0.05, 8))
+    qg, sg = oracle.rtn_weight(wg)
+    qu, su = oracle.rtn_weight(wu)
+    assert sg != su
+    smax = max(sg, su)
+    smin_q = qg if sg < su else qu
+    s_small = min(sg, su)
+    re = oracle.requant_group_member(smin_q, s_small, smax)
+    assert (re != smin_q).any()
+    # re-quantizing onto its own scale is the identity (the split path)
+    assert np.array_equal(oracle.requant_group_member(smin_q, s_small, s_small), smin_q)
+
+
+# --------------------------------------------------------------- gated MLP
+
+
+def _c0_weights():
+    d = synth.c0_mlp()
+    wgq, swg = oracle.rtn_weight(bits_of(d["wg"]))
+    wuq, swu = oracle.rtn_weight(bits_of(d["wu"]))
+    wdq, swd = oracle.rtn_weight(bits_of(d["wd"]))
+    calib = [bits_of(b) for b in d["calib"]]
+    s_in = oracle.observer_scale(calib)
+    s_down = oracle.down_scale(calib, bits_of(d["wg"]), bits_of(d["wu"]))
+    return d, (s_in, wgq, swg, wuq, swu, s_down, wdq, swd)
+
+
+def test_gated_mlp_row_independence():
+    d, args = _c0_weights()
+    x = bits_of(d["x"])
+    y = oracle.gated_mlp(x, *args)
+    rows = [0, 5, 17, 63]
+    y_rows = oracle.gated_mlp(np.ascontiguousarray(x[rows]), *args)
+    assert np.array_equal(y[rows], y_rows)
+
+
+def test_gated_mlp_brute_force_tiny():
+    """Independent composition from library routines on a tiny slice: torch
+    casts for the quantizers, numpy fp64 matmuls, tanh-form SiLU.  Equal up to
+    rare one-step differences of H near code boundaries."""
+    d, (s_in, wgq, swg, wuq, swu, s_down, wdq, swd) = _c0_weights()
+    x = bits_of(d["x"][:8].contiguous())
+    y = oracle.gated_mlp(x, s_in, wgq, swg, wuq, swu, s_down, wdq, swd)
+    cb = oracle.codebook()
+    xf = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).float()
+    xq = torch_e4m3((xf / torch.tensor(s_in)).numpy())
+    g = ((cb[xq] @ cb[wgq].T) * (float(s_in) * float(swg)))
+    u = ((cb[xq] @ cb[wuq].T) * (float(s_in) * float(swu)))
+    g = torch.from_numpy(g).to(torch.bfloat16).double().numpy()
+    u = torch.from_numpy(u).to(torch.bfloat16).double().numpy()
+    hv = g * (1 + np.tanh(g / 2)) / 2 * u / float(s_down)
+    hq = torch_e4m3(np.clip(hv, -448, 448).astype(np.float32))
+    ref = torch.from_numpy((cb[hq] @ cb[wdq].T) * (float(s_down) * float(swd))).to(torch.bfloat16)
+    ref = ref.double().numpy()
+    yv = oracle.bf16_to_f64(y)
+    rel = np.linalg.norm(yv - ref) / np.linalg.norm(ref)
+    assert rel < 1e-2
+    assert np.isfinite(yv).all() and np.abs(yv).max() > 0
