@@ -1,0 +1,551 @@
+"""Benchmark of the static FP8 W8A8 hot path on B200.
+
+Workload (one step): the two-tower decoder-MLP pass -- 36 layers, each with
+an understanding-tower gated MLP over 1024 tokens and a generation-tower gated
+MLP over 4096 tokens, d=3072, I=12288, every layer and tower with its own FP8
+weights and static scales.  One gated MLP = quantize X once, gate and up FP8
+GEMMs, two-input SwiGLU quantized to FP8, FP8 down GEMM.  Metric: tokens/s of
+the whole pass, (1024 + 4096) tokens per step per GPU.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun with N>1 every rank runs an independent replica of the pass on
+its own GPU (no data-path collective; weak scaling).  Rank 0 prints one JSON
+line.  The timed region issues the path's kernels through the C ABI with CUDA
+events between them, so the same run yields the pass time and each kernel's
+average duration (for the roofline of the dominant kernel).  The end-to-end
+number goes through the composite gated-MLP call with host buffers: every
+layer's input is copied from pinned host memory and its output copied back
+inside the timed region.
+
+`--impl reference` times the CPU oracle (the only other implementation there
+is) on a bounded sample of rows of the same pass on the host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "gated-MLP tokens/s + FP8 GEMM TFLOP/s & SwiGLU-quant GB/s vs roofline"
+UNIT = "tokens/s"
+LAYERS = synth.C4["layers"]
+D, I = synth.C4["d"], synth.C4["I"]
+TOWERS = (("und", synth.C4["M_und"]), ("gen", synth.C4["M_gen"]))
+TOKENS_PER_STEP = sum(m for _, m in TOWERS)
+CALIB_BATCHES = 16
+CALIB_ROWS = 256
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sustained=float(p["bf16_tflops_sustained"]), source="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# ------------------------------------------------------------------ clocks
+
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.flush()
+        self.out.seek(0)
+        rows = [ln.split(",") for ln in self.out.read().splitlines() if ln.strip()]
+        os.unlink(self.out.name)
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+                for name, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(name)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- set-up
+
+
+class Layer:
+    pass
+
+
+def prepare(fw, device, n_layers, log):
+    """Synthetic checkpoint of the two-tower pass, made on the GPU with the
+    library's own load-time calls: RTN FP8 weights (s_w = max|W|/448) and
+    static input scales from the moving-average observer over 16 calibration
+    batches (s_in over the batches' inputs; s_down over SiLU(G)*U of the same
+    batches, with G and U taken from the FP8 gate/up GEMMs)."""
+    layers = []
+    t0 = time.time()
+    for l in range(n_layers):
+        for tower, M in TOWERS:
+            src = synth.c4_layer(l, tower, device=device, n_calib=CALIB_BATCHES,
+                                 calib_rows=CALIB_ROWS)
+            L = Layer()
+            L.tower, L.M, L.index = tower, M, l
+            L.x = src["x"]
+            L.wg, L.s_wg = fw.fp8_rtn_quantize_weight(src["wg"])
+            L.wu, L.s_wu = fw.fp8_rtn_quantize_weight(src["wu"])
+            L.wd, L.s_wd = fw.fp8_rtn_quantize_weight(src["wd"])
+            amax_in = torch.cat([fw.fp8_absmax_bf16(b) for b in src["calib"]])
+            L.s_in = fw.fp8_observer_scale(amax_in)
+            amax_h = []
+            for b in src["calib"]:
+                bq = fw.fp8_quant_static(b, L.s_in)
+                g = fw.fp8_linear_static(bq, L.wg, L.s_in, L.s_wg)
+                u = fw.fp8_linear_static(bq, L.wu, L.s_in, L.s_wu)
+                amax_h.append(fw.fp8_silu_mul_absmax(g, u))
+            L.s_down = fw.fp8_observer_scale(torch.cat(amax_h))
+            del src
+            layers.append(L)
+    torch.cuda.synchronize()
+    # gate and up share one quantized activation: the load-time invariant
+    for L in layers:
+        st = fw.fp8_check_shared_input_scale([L.s_in, L.s_in])
+        if st != 0:
+            raise RuntimeError(f"shared input scale check failed: {st}")
+    log(f"prepared {len(layers)} layer-towers in {time.time() - t0:.1f}s")
+    return layers
+
+
+def make_buffers(fw, layers, device):
+    ws = {}
+    bufs = {}
+    for tower, M in TOWERS:
+        nbytes = fw.gated_mlp_static_fp8_workspace(M, D, I)
+        ws[tower] = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        bufs[tower] = fw.gated_mlp_workspace_views(ws[tower], M, D, I)
+    for L in layers:
+        L.y = torch.empty((L.M, D), dtype=torch.bfloat16, device=device)
+    return ws, bufs
+
+
+# ---------------------------------------------------------- timed region
+
+
+def build_plan(fw, layers, bufs, stream_handle):
+    """The pass as a flat list of direct C-ABI calls (kind, fn, args), in the
+    same order the composite gated-MLP call issues them."""
+    lib = fw.load()
+    plan = []
+    for L in layers:
+        b = bufs[L.tower]
+        M = L.M
+        xq, g, u, h = b["xq"].data_ptr(), b["g"].data_ptr(), b["u"].data_ptr(), b["h"].data_ptr()
+        s_in, s_down = L.s_in.data_ptr(), L.s_down.data_ptr()
+        plan.append(("quant", lib.fp8_quant_static,
+                     (L.x.data_ptr(), M * D, s_in, xq, stream_handle), 3 * M * D, 0))
+        plan.append(("gemm", lib.fp8_linear_static,
+                     (xq, L.wg.data_ptr(), M, I, D, s_in, L.s_wg.data_ptr(), g, stream_handle),
+                     M * D + I * D + 2 * M * I, 2 * M * I * D))
+        plan.append(("gemm", lib.fp8_linear_static,
+                     (xq, L.wu.data_ptr(), M, I, D, s_in, L.s_wu.data_ptr(), u, stream_handle),
+                     M * D + I * D + 2 * M * I, 2 * M * I * D))
+        plan.append(("swiglu", lib.silu_mul_2in_fp8, (g, u, M * I, s_down, h, stream_handle),
+                     5 * M * I, 0))
+        plan.append(("gemm", lib.fp8_linear_static,
+                     (h, L.wd.data_ptr(), M, D, I, s_down, L.s_wd.data_ptr(), L.y.data_ptr(),
+                      stream_handle),
+                     M * I + D * I + 2 * M * D, 2 * M * D * I))
+    return plan
+
+
+def run_plan(plan, events=None):
+    if events is None:
+        for _, fn, args, _, _ in plan:
+            if fn(*args) != 0:
+                raise RuntimeError("launch failed")
+        return
+    for i, (_, fn, args, _, _) in enumerate(plan):
+        events[i].record()
+        if fn(*args) != 0:
+            raise RuntimeError("launch failed")
+    events[len(plan)].record()
+
+
+def time_device(plan, steps, warmup, dist_ctx, sampler=None):
+    """W untimed steps, then K timed steps between a barrier + synchronize on
+    both sides; per-kernel events inside the timed region."""
+    for _ in range(warmup):
+        run_plan(plan)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(plan) + 1)]
+          for _ in range(steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist_ctx.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    start.record()
+    for k in range(steps):
+        run_plan(plan, ev[k])
+    stop.record()
+    torch.cuda.synchronize()
+    if sampler:
+        clocks = sampler.stop()
+    else:
+        clocks = None
+    dist_ctx.barrier()
+    total_ms = start.elapsed_time(stop)
+    per_kind = {}
+    for k in range(steps):
+        for i, (kind, _, _, nbytes, flops) in enumerate(plan):
+            dt = ev[k][i].elapsed_time(ev[k][i + 1])
+            acc = per_kind.setdefault(kind, [0.0, 0, 0, 0])
+            acc[0] += dt
+            acc[1] += 1
+            acc[2] += nbytes
+            acc[3] += flops
+    return total_ms, per_kind, clocks
+
+
+def time_e2e(fw, layers, steps, warmup, device, dist_ctx):
+    """The pass through the composite C-ABI call with host buffers: each
+    layer's X is copied from pinned host memory on a copy stream, the gated
+    MLP runs on the compute stream, Y is copied back to pinned host memory on
+    a third stream; two device buffer sets per tower let copies overlap the
+    previous layer's compute."""
+    h_x = [L.x.cpu().pin_memory() for L in layers]
+    h_y = [torch.empty((L.M, D), dtype=torch.bfloat16).pin_memory() for L in layers]
+    dx = {t: [torch.empty((M, D), dtype=torch.bfloat16, device=device) for _ in range(2)]
+          for t, M in TOWERS}
+    dy = {t: [torch.empty((M, D), dtype=torch.bfloat16, device=device) for _ in range(2)]
+          for t, M in TOWERS}
+    ws = {t: torch.empty(fw.gated_mlp_static_fp8_workspace(M, D, I), dtype=torch.uint8,
+                         device=device) for t, M in TOWERS}
+    comp = torch.cuda.Stream(device)
+    h2d = torch.cuda.Stream(device)
+    d2h = torch.cuda.Stream(device)
+    n = len(layers)
+
+    def one_pass():
+        # a pass starts once the previous one is complete (slots are reused)
+        h2d.wait_stream(comp)
+        d2h.wait_stream(comp)
+        ready = [torch.cuda.Event() for _ in range(n)]
+        done = [torch.cuda.Event() for _ in range(n)]
+        copied_out = [torch.cuda.Event() for _ in range(n)]
+        for i, L in enumerate(layers):
+            slot = (i // 2) % 2  # layers alternate towers; two slots per tower
+            with torch.cuda.stream(h2d):
+                if i >= 4:
+                    h2d.wait_event(done[i - 4])  # slot's previous user finished compute
+                dx[L.tower][slot].copy_(h_x[i], non_blocking=True)
+                ready[i].record(h2d)
+            with torch.cuda.stream(comp):
+                comp.wait_event(ready[i])
+                if i >= 4:
+                    comp.wait_event(copied_out[i - 4])  # slot's previous output copied out
+                fw.gated_mlp_static_fp8(dx[L.tower][slot], L.s_in, L.wg, L.s_wg, L.wu, L.s_wu,
+                                        L.s_down, L.wd, L.s_wd, workspace=ws[L.tower],
+                                        out=dy[L.tower][slot], stream=comp)
+                done[i].record(comp)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(done[i])
+                h_y[i].copy_(dy[L.tower][slot], non_blocking=True)
+                copied_out[i].record(d2h)
+        # the step ends when its last result is in host memory
+        comp.wait_stream(d2h)
+        comp.wait_stream(h2d)
+
+    for _ in range(warmup):
+        one_pass()
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist_ctx.barrier()
+    torch.cuda.synchronize()
+    comp.wait_stream(torch.cuda.current_stream())
+    start.record(comp)
+    for _ in range(steps):
+        one_pass()
+    stop.record(comp)
+    torch.cuda.synchronize()
+    dist_ctx.barrier()
+    ms = start.elapsed_time(stop)
+    h2d_bytes = sum(t.numel() * t.element_size() for t in h_x)
+    d2h_bytes = sum(t.numel() * t.element_size() for t in h_y)
+    # check one output against the device-path result of the same layer
+    return ms, h2d_bytes, d2h_bytes, h_y
+
+
+# ------------------------------------------------------------- CPU oracle
+
+
+class OracleSample:
+    """The oracle on a bounded sample of the same pass: rows of one layer of
+    each tower, on all host cores.  Rows are independent under static scales,
+    so the time per row extrapolates to the whole pass.  The weights are
+    quantized once up front (load time, not timed); the scale values do not
+    change the oracle's cost."""
+
+    def __init__(self, layer: int = 0):
+        import oracle  # the CPU-baseline leg is the one place the benchmark runs it
+
+        self.oracle = oracle
+        self.cores = len(os.sched_getaffinity(0))
+        oracle.set_num_threads(self.cores)
+        self.layer = layer
+        self.towers = []
+        for tower, M in TOWERS:
+            src = synth.c4_layer(layer, tower, device="cpu", n_calib=0)
+            b = {k: src[k].view(torch.int16).numpy().view(np.uint16) for k in ("x", "wg", "wu", "wd")}
+            wgq, swg = oracle.rtn_weight(b["wg"])
+            wuq, swu = oracle.rtn_weight(b["wu"])
+            wdq, swd = oracle.rtn_weight(b["wd"])
+            s_in = oracle.scale_from_amax(oracle.absmax(b["x"]))
+            self.towers.append((tower, b["x"], (s_in, wgq, swg, wuq, swu, oracle.f32(4 * s_in),
+                                                wdq, swd)))
+
+    def run(self, rows_per_tower: int):
+        """Seconds per token-layer, averaged over both towers."""
+        per_row = []
+        for _, x, args in self.towers:
+            rows = np.ascontiguousarray(x[:rows_per_tower])
+            t0 = time.perf_counter()
+            self.oracle.gated_mlp(rows, *args)
+            per_row.append((time.perf_counter() - t0) / rows_per_tower)
+        return statistics.mean(per_row)
+
+    def tokens_per_s(self, sec_per_token_layer: float) -> float:
+        return 1.0 / (sec_per_token_layer * LAYERS)
+
+    def describe(self, rows_per_tower: int, wall: float) -> str:
+        return (f"oracle gated MLP (d=3072, I=12288) on {rows_per_tower} rows of layer {self.layer} "
+                f"of each tower, {wall:.1f}s wall on {self.cores} threads; rows are independent, "
+                f"time per row extrapolated to the 36-layer pass")
+
+
+def cpu_baseline(rows_per_tower: int = 96):
+    o = OracleSample()
+    t0 = time.perf_counter()
+    spt = o.run(rows_per_tower)
+    wall = time.perf_counter() - t0
+    return o.tokens_per_s(spt), o.cores, o.describe(rows_per_tower, wall)
+
+
+# -------------------------------------------------------------- dist glue
+
+
+class DistCtx:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, backend="nccl"):
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            if backend == "nccl":
+                torch.cuda.set_device(self.local_rank)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg is not None:
+            if self.pg.get_backend() == "nccl":
+                self.pg.barrier(device_ids=[self.local_rank])
+            else:
+                self.pg.barrier()
+
+    def max(self, v: float) -> float:
+        if self.pg is None:
+            return v
+        dev = torch.device("cuda", self.local_rank) if self.pg.get_backend() == "nccl" else "cpu"
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+def aggregate_value(tokens_per_rank: int, world: int, max_seconds: float) -> float:
+    """Whole-job throughput: tokens of every rank over the slowest rank's time."""
+    return tokens_per_rank * world / max_seconds
+
+
+# ------------------------------------------------------------------ main
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--layers", type=int, default=LAYERS)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    log = lambda m: print(m, file=sys.stderr, flush=True)  # noqa: E731
+
+    ctx = DistCtx()
+    if args.impl == "reference":
+        if ctx.rank != 0:
+            return 0
+        o = OracleSample()
+        rows = 16
+        for _ in range(args.warmup):
+            o.run(2)
+        step_times = []
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            step_times.append(o.tokens_per_s(o.run(rows)))
+        wall = time.perf_counter() - t0
+        cores, sample = o.cores, o.describe(rows, wall / max(args.steps, 1)) + " (per step)"
+        value = statistics.median(step_times)
+        line = {
+            "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": TOKENS_PER_STEP / value * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": "two-tower MoT decoder-MLP pass, 36 layers x {und M=1024, gen M=4096}, d=3072, I=12288",
+                       "global_batch": TOKENS_PER_STEP, "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+        return 0
+
+    import fp8_w8a8_static_b200 as fw
+
+    ctx.init("nccl")
+    device = torch.device("cuda", ctx.local_rank)
+    torch.cuda.set_device(device)
+    fw.load()
+    if fw.device_check() != 0:
+        raise RuntimeError("not an sm_100 device")
+    pk = peaks()
+    layers = prepare(fw, device, args.layers, log)
+    ws, bufs = make_buffers(fw, layers, device)
+    stream = torch.cuda.current_stream(device)
+    plan = build_plan(fw, layers, bufs, stream.cuda_stream)
+
+    launches_before = fw.launch_count()
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    total_ms, per_kind, clocks = time_device(plan, args.steps, max(args.warmup, 3), ctx, sampler)
+    launches = (fw.launch_count() - launches_before) // (args.steps + max(args.warmup, 3)) * args.steps
+    st, where = fw.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} at wait site {where}")
+
+    max_ms = ctx.max(total_ms)
+    tokens = TOKENS_PER_STEP * args.steps * args.layers / LAYERS
+    value = aggregate_value(tokens, ctx.world, max_ms / 1e3)
+
+    # per-kernel achieved rates from the events inside the timed region
+    comp = {}
+    for kind, (ms, n, nbytes, flops) in per_kind.items():
+        d = {"launches_per_step": n // args.steps, "ms_per_step": ms / args.steps,
+             "share": ms / sum(v[0] for v in per_kind.values())}
+        if flops:
+            d["tflops"] = flops / (ms / 1e3) / 1e12
+        d["gbs"] = nbytes / (ms / 1e3) / 1e9
+        comp[kind] = d
+    gemm = per_kind["gemm"]
+    fp8_peak = 2.0 * pk["bf16_sustained"]
+    achieved = gemm[3] / (gemm[0] / 1e3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
+                "frac": achieved / fp8_peak, "traffic": None,
+                "kernel": "fp8_gemm_kernel (all GEMM launches of the pass, flop-weighted)",
+                "peak_source": f"{pk['source']}: bf16 sustained {pk['bf16_sustained']} TFLOP/s x 2 (nominal fp8/bf16 ratio)"}
+    comp["swiglu"]["hbm_frac"] = comp["swiglu"]["gbs"] / pk["hbm"]
+    comp["quant"]["hbm_frac"] = comp["quant"]["gbs"] / pk["hbm"]
+
+    e2e = None
+    if not args.no_e2e:
+        ms, hb, db, h_y = time_e2e(fw, layers, max(1, args.steps // 2), 1, device, ctx)
+        ms = ctx.max(ms)
+        torch.cuda.synchronize()
+        same = torch.equal(h_y[-1], layers[-1].y.cpu())
+        e2e = {"value": aggregate_value(TOKENS_PER_STEP * max(1, args.steps // 2) * args.layers / LAYERS,
+                                        ctx.world, ms / 1e3),
+               "unit": UNIT, "h2d_bytes_per_step": hb, "d2h_bytes_per_step": db,
+               "matches_device_path": bool(same)}
+
+    cpu = None
+    if ctx.rank == 0 and ctx.world == 1 and not args.no_cpu_baseline:
+        tps, cores, sample = cpu_baseline()
+        cpu = {"value": tps, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+
+    if ctx.rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ctx.world,
+            "steps": args.steps, "warmup": max(args.warmup, 3),
+            "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp8-e4m3 MMA, fp32 accumulate, bf16 out",
+            "data": "synthetic",
+            "config": {"workload": "two-tower MoT decoder-MLP pass, 36 layers x {und M=1024, gen M=4096}, d=3072, I=12288",
+                       "layers": args.layers, "global_batch": TOKENS_PER_STEP * ctx.world,
+                       "parallelism": f"replicas x{ctx.world}",
+                       "l2": "inputs larger than L2 (8.15 GB of FP8 weights per pass)"},
+            "roofline": roofline, "components": comp, "e2e": e2e, "cpu_baseline": cpu,
+            "gpu_launches": launches, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    ctx.close()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,380 @@
+"""Static per-tensor FP8 E4M3 W8A8 Linear blocks on B200 (sm_100a).
+
+A thin ctypes binding over the C ABI in ``include/fp8ws.h``.  The functions
+keep the C names; they check the torch tensors they are given (device, dtype,
+contiguity, alignment), pass raw pointers and the current CUDA stream, and
+raise :class:`FP8WSError` on a nonzero status.  Every step of the path runs in
+the library's own sm_100a kernels; there is no fallback.  If the compiled
+library is missing, the first call raises with the command that builds it.
+
+Pages the operations follow: the TensorRT-LLM pull request "Load static FP8
+Cosmos3 Nano/Super checkpoints without re-quantizing them" (What changed) and
+the Hugging Face model card "Cosmos3-Nano-Policy-DROID, FP8 + RTN +
+moving-average activation observer (ModelOpt W8A8, per-tensor static)"
+(Scheme table).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+__all__ = [
+    "FP8WSError", "library_path", "load",
+    "fp8_quant_static", "fp8_linear_static", "silu_mul_2in_fp8",
+    "gated_mlp_static_fp8", "gated_mlp_static_fp8_workspace",
+    "qkv_shared_quant", "qkv_shared_quant_workspace",
+    "fp8_check_shared_input_scale", "fp8_absmax_bf16", "fp8_silu_mul_absmax",
+    "fp8_observer_scale", "fp8_rtn_quantize_weight",
+    "device_check", "device_status", "launch_count", "launch_log", "launch_log_clear",
+    "FP8", "OBSERVER_CONSTANT", "EXPORTED_SYMBOLS",
+]
+
+FP8 = torch.float8_e4m3fn
+OBSERVER_CONSTANT = 0.01
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "_lib", "libfp8ws.so")
+
+STATUS = {
+    0: "ok", 1: "null pointer", 2: "unsupported size", 3: "pointer not 16-byte aligned",
+    4: "group input scales differ", 5: "scale not finite or not positive",
+    6: "CUDA runtime error", 7: "bounded wait in a kernel ran out",
+    8: "device is not sm_100", 9: "workspace NULL or not 256-byte aligned",
+}
+OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_SCALE_MISMATCH, ERR_BAD_SCALE, ERR_CUDA, \
+    ERR_DEVICE_TIMEOUT, ERR_UNSUPPORTED, ERR_WORKSPACE = range(10)
+
+KIND_QUANT, KIND_GEMM, KIND_SWIGLU, KIND_CALIB = 1, 2, 3, 4
+
+
+class FP8WSError(RuntimeError):
+    def __init__(self, status: int, call: str):
+        self.status = status
+        super().__init__(f"{call}: status {status} ({STATUS.get(status, 'unknown')})")
+
+
+class LaunchRecord(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("pad", ctypes.c_int32), ("in0", ctypes.c_void_p),
+                ("in1", ctypes.c_void_p), ("out", ctypes.c_void_p)]
+
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_SIGS = {
+    "fp8_quant_static": (ctypes.c_int, [_P, _I64, _P, _P, _P]),
+    "fp8_linear_static": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _P, _P]),
+    "silu_mul_2in_fp8": (ctypes.c_int, [_P, _P, _I64, _P, _P, _P]),
+    "gated_mlp_static_fp8_workspace": (ctypes.c_size_t, [_I64, _I64, _I64]),
+    "gated_mlp_static_fp8": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _P,
+                                            _P, _P, _P]),
+    "qkv_shared_quant_workspace": (ctypes.c_size_t, [_I64, _I64]),
+    "qkv_shared_quant": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _I64, _P, _P, _I64, _P, _P, _I64,
+                                        _P, _P, _P, _P, _P, _P]),
+    "fp8_check_shared_input_scale": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int,
+                                                    _P]),
+    "fp8_absmax_bf16": (ctypes.c_int, [_P, _I64, _P, _P]),
+    "fp8_silu_mul_absmax": (ctypes.c_int, [_P, _P, _I64, _P, _P]),
+    "fp8_observer_scale": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_double, _P, _P]),
+    "fp8_rtn_quantize_weight": (ctypes.c_int, [_P, _I64, _P, _P, _P]),
+    "fp8ws_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "fp8ws_device_check": (ctypes.c_int, []),
+    "fp8ws_device_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int),
+                                           ctypes.POINTER(ctypes.c_int)]),
+    "fp8ws_launch_count": (ctypes.c_int64, []),
+    "fp8ws_launch_log": (ctypes.c_int, [ctypes.POINTER(LaunchRecord), ctypes.c_int]),
+    "fp8ws_launch_log_clear": (None, []),
+}
+EXPORTED_SYMBOLS = tuple(_SIGS)
+
+_lib = None
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """Load the compiled library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(
+                f"{_LIB_PATH} is missing: build it with `python -m fp8_w8a8_static_b200.build`")
+        lib = ctypes.CDLL(_LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+# ------------------------------------------------------------------ helpers
+
+
+def _check(status: int, call: str) -> None:
+    if status != OK:
+        raise FP8WSError(status, call)
+
+
+def _dev_ptr(t: torch.Tensor, name: str, dtypes) -> int:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor (got {t.device})")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} is not contiguous; strided tensors are refused, not copied")
+    return t.data_ptr()
+
+
+def _bf16(t, name):
+    return _dev_ptr(t, name, (torch.bfloat16,))
+
+
+def _fp8(t, name):
+    return _dev_ptr(t, name, (FP8, torch.uint8))
+
+
+def _f32(t, name):
+    p = _dev_ptr(t, name, (torch.float32,))
+    if t.numel() < 1:
+        raise ValueError(f"{name} must hold at least one fp32 value")
+    return p
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _device_of(t: torch.Tensor):
+    return torch.cuda.device(t.device)
+
+
+# ---------------------------------------------------------------- hot path
+
+
+def fp8_quant_static(x: torch.Tensor, s_in: torch.Tensor, out: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """Xq = E4M3_satRNE(x / s_in), any shape, BF16 in, FP8 out."""
+    lib = load()
+    if out is None:
+        out = torch.empty(x.shape, dtype=FP8, device=x.device)
+    if out.numel() != x.numel():
+        raise ValueError("out size differs from x")
+    with _device_of(x):
+        _check(lib.fp8_quant_static(_bf16(x, "x"), x.numel(), _f32(s_in, "s_in"),
+                                    _fp8(out, "out"), _stream(stream)), "fp8_quant_static")
+    return out
+
+
+def fp8_linear_static(xq: torch.Tensor, wq: torch.Tensor, s_in: torch.Tensor, s_w: torch.Tensor,
+                      out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Y[M,N] = bf16((s_in*s_w) * Xq[M,K] . Wq[N,K]^T)."""
+    lib = load()
+    if xq.dim() != 2 or wq.dim() != 2 or xq.shape[1] != wq.shape[1]:
+        raise ValueError(f"shapes {tuple(xq.shape)} x {tuple(wq.shape)}^T do not match")
+    M, K = xq.shape
+    N = wq.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    if tuple(out.shape) != (M, N):
+        raise ValueError("out must be [M, N]")
+    with _device_of(xq):
+        _check(lib.fp8_linear_static(_fp8(xq, "xq"), _fp8(wq, "wq"), M, N, K, _f32(s_in, "s_in"),
+                                     _f32(s_w, "s_w"), _bf16(out, "out"), _stream(stream)),
+               "fp8_linear_static")
+    return out
+
+
+def silu_mul_2in_fp8(g: torch.Tensor, u: torch.Tensor, s_down: torch.Tensor,
+                     out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """H = E4M3_satRNE(SiLU(G) * U / s_down) from two separate BF16 tensors (any rank)."""
+    lib = load()
+    if g.shape != u.shape:
+        raise ValueError("G and U shapes differ")
+    if out is None:
+        out = torch.empty(g.shape, dtype=FP8, device=g.device)
+    if out.numel() != g.numel():
+        raise ValueError("out size differs from G")
+    with _device_of(g):
+        _check(lib.silu_mul_2in_fp8(_bf16(g, "g"), _bf16(u, "u"), g.numel(),
+                                    _f32(s_down, "s_down"), _fp8(out, "out"), _stream(stream)),
+               "silu_mul_2in_fp8")
+    return out
+
+
+def gated_mlp_static_fp8_workspace(M: int, d: int, I: int) -> int:
+    return load().gated_mlp_static_fp8_workspace(M, d, I)
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    # torch's caching allocator hands out 512-byte aligned blocks
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def gated_mlp_static_fp8(x, s_in, wg, s_wg, wu, s_wu, s_down, wd, s_wd, workspace=None, out=None,
+                         stream=None) -> torch.Tensor:
+    """Split gated MLP: quantize X once, gate and up FP8 GEMMs, two-input
+    SwiGLU to FP8, FP8 down GEMM.  x [M,d] BF16; wg, wu [I,d], wd [d,I] FP8."""
+    lib = load()
+    if x.dim() != 2:
+        raise ValueError("x must be [M, d]")
+    M, d = x.shape
+    I = wg.shape[0]
+    if tuple(wg.shape) != (I, d) or tuple(wu.shape) != (I, d) or tuple(wd.shape) != (d, I):
+        raise ValueError("weight shapes must be Wg, Wu [I,d] and Wd [d,I]")
+    need = lib.gated_mlp_static_fp8_workspace(M, d, I)
+    if workspace is None:
+        workspace = _workspace(need, x.device)
+    if workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace needs {need} bytes")
+    if out is None:
+        out = torch.empty((M, d), dtype=torch.bfloat16, device=x.device)
+    with _device_of(x):
+        _check(lib.gated_mlp_static_fp8(
+            _bf16(x, "x"), M, d, I, _f32(s_in, "s_in"), _fp8(wg, "wg"), _f32(s_wg, "s_wg"),
+            _fp8(wu, "wu"), _f32(s_wu, "s_wu"), _f32(s_down, "s_down"), _fp8(wd, "wd"),
+            _f32(s_wd, "s_wd"), _dev_ptr(workspace, "workspace", (torch.uint8,)),
+            _bf16(out, "out"), _stream(stream)), "gated_mlp_static_fp8")
+    return out
+
+
+def gated_mlp_workspace_views(workspace: torch.Tensor, M: int, d: int, I: int):
+    """Views of the regions gated_mlp_static_fp8 writes: Xq [M,d], G [M,I],
+    U [M,I] (BF16) and H [M,I] (FP8)."""
+    def r256(v):
+        return (v + 255) // 256 * 256
+    o_g = r256(M * d)
+    o_u = o_g + r256(M * I * 2)
+    o_h = o_u + r256(M * I * 2)
+    ws = workspace.view(torch.uint8)
+    xq = ws[:M * d].view(FP8).view(M, d)
+    g = ws[o_g:o_g + M * I * 2].view(torch.bfloat16).view(M, I)
+    u = ws[o_u:o_u + M * I * 2].view(torch.bfloat16).view(M, I)
+    h = ws[o_h:o_h + M * I].view(FP8).view(M, I)
+    return dict(xq=xq, g=g, u=u, h=h)
+
+
+def qkv_shared_quant_workspace(M: int, d: int) -> int:
+    return load().qkv_shared_quant_workspace(M, d)
+
+
+def qkv_shared_quant(x, s_in, wq, s_wq, wk, s_wk, wv, s_wv, workspace=None, out=None, stream=None):
+    """Q, K, V = three FP8 GEMMs over one shared quantization of x [M,d]."""
+    lib = load()
+    M, d = x.shape
+    Nq, Nk, Nv = wq.shape[0], wk.shape[0], wv.shape[0]
+    for w, n in ((wq, "wq"), (wk, "wk"), (wv, "wv")):
+        if w.dim() != 2 or w.shape[1] != d:
+            raise ValueError(f"{n} must be [N, {d}]")
+    need = lib.qkv_shared_quant_workspace(M, d)
+    if workspace is None:
+        workspace = _workspace(need, x.device)
+    if workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace needs {need} bytes")
+    if out is None:
+        out = tuple(torch.empty((M, n), dtype=torch.bfloat16, device=x.device) for n in (Nq, Nk, Nv))
+    q, k, v = out
+    with _device_of(x):
+        _check(lib.qkv_shared_quant(
+            _bf16(x, "x"), M, d, _f32(s_in, "s_in"), _fp8(wq, "wq"), Nq, _f32(s_wq, "s_wq"),
+            _fp8(wk, "wk"), Nk, _f32(s_wk, "s_wk"), _fp8(wv, "wv"), Nv, _f32(s_wv, "s_wv"),
+            _dev_ptr(workspace, "workspace", (torch.uint8,)), _bf16(q, "q"), _bf16(k, "k"),
+            _bf16(v, "v"), _stream(stream)), "qkv_shared_quant")
+    return q, k, v
+
+
+# ---------------------------------------------------------------- load time
+
+
+def fp8_check_shared_input_scale(scales: Sequence[torch.Tensor], stream=None) -> int:
+    """Status of the equal-input-scale invariant of a group (0 = holds).  Syncs."""
+    lib = load()
+    ptrs = (ctypes.c_void_p * len(scales))(*[_f32(s, f"scales[{i}]") for i, s in enumerate(scales)])
+    with _device_of(scales[0]):
+        return lib.fp8_check_shared_input_scale(ptrs, len(scales), _stream(stream))
+
+
+def fp8_absmax_bf16(x, out=None, stream=None) -> torch.Tensor:
+    lib = load()
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=x.device)
+    with _device_of(x):
+        _check(lib.fp8_absmax_bf16(_bf16(x, "x"), x.numel(), _f32(out, "out"), _stream(stream)),
+               "fp8_absmax_bf16")
+    return out
+
+
+def fp8_silu_mul_absmax(g, u, out=None, stream=None) -> torch.Tensor:
+    lib = load()
+    if g.shape != u.shape:
+        raise ValueError("G and U shapes differ")
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=g.device)
+    with _device_of(g):
+        _check(lib.fp8_silu_mul_absmax(_bf16(g, "g"), _bf16(u, "u"), g.numel(), _f32(out, "out"),
+                                       _stream(stream)), "fp8_silu_mul_absmax")
+    return out
+
+
+def fp8_observer_scale(amaxes: torch.Tensor, c: float = OBSERVER_CONSTANT, out=None,
+                       stream=None) -> torch.Tensor:
+    lib = load()
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=amaxes.device)
+    with _device_of(amaxes):
+        _check(lib.fp8_observer_scale(_f32(amaxes, "amaxes"), amaxes.numel(), float(c),
+                                      _f32(out, "out"), _stream(stream)), "fp8_observer_scale")
+    return out
+
+
+def fp8_rtn_quantize_weight(w: torch.Tensor, wq=None, s_w=None, stream=None):
+    """(Wq, s_w): RTN per-tensor weight quantization with s_w = max|W| / 448."""
+    lib = load()
+    if wq is None:
+        wq = torch.empty(w.shape, dtype=FP8, device=w.device)
+    if s_w is None:
+        s_w = torch.empty(1, dtype=torch.float32, device=w.device)
+    with _device_of(w):
+        _check(lib.fp8_rtn_quantize_weight(_bf16(w, "w"), w.numel(), _f32(s_w, "s_w"),
+                                           _fp8(wq, "wq"), _stream(stream)),
+               "fp8_rtn_quantize_weight")
+    return wq, s_w
+
+
+# ------------------------------------------------------------- diagnostics
+
+
+def device_check() -> int:
+    return load().fp8ws_device_check()
+
+
+def device_status():
+    """(status, where): reads and clears the device status word (syncs)."""
+    st, wh = ctypes.c_int(0), ctypes.c_int(0)
+    _check(load().fp8ws_device_status(ctypes.byref(st), ctypes.byref(wh)), "fp8ws_device_status")
+    return st.value, wh.value
+
+
+def launch_count() -> int:
+    return load().fp8ws_launch_count()
+
+
+def launch_log(max_records: int = 64):
+    buf = (LaunchRecord * max_records)()
+    n = load().fp8ws_launch_log(buf, max_records)
+    return [(r.kind, r.in0 or 0, r.in1 or 0, r.out or 0) for r in buf[:n]]
+
+
+def launch_log_clear() -> None:
+    load().fp8ws_launch_log_clear()

@@ -1,0 +1,211 @@
+// HBM-bound kernels of the static FP8 path: the activation quantizer, the
+// two-input SwiGLU with FP8 output, and the calibration reductions.
+//
+// All of them stream flat contiguous runs: each thread moves 16-byte vectors
+// (8 BF16 values) with several vectors in flight, grids are sized to fill every
+// SM, and the ragged tail (numel not a multiple of 8) is finished by the first
+// threads of the grid one element at a time.
+#pragma once
+
+#include "common.cuh"
+
+namespace fp8ws {
+
+constexpr int kEwThreads = 256;  // threads per block of the streaming kernels
+constexpr int kEwUnroll = 4;     // 16-byte vectors in flight per thread and input
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Two fp32 values -> two E4M3 codes (first value in the low byte), rounded to
+// nearest even with saturation to +-448 (NaN stays NaN).
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float a, float b) {
+  return static_cast<uint32_t>(
+      __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
+}
+
+__device__ __forceinline__ uint32_t pack4(uint32_t p01, uint32_t p23) {
+  return (p01 & 0xFFFFu) | (p23 << 16);
+}
+
+// Streaming loads/stores: every byte is touched once.
+__device__ __forceinline__ uint4 ld_stream(const uint4 *p) { return __ldcs(p); }
+__device__ __forceinline__ void st_stream(uint2 *p, uint2 v) { __stcs(p, v); }
+
+// ------------------------------------------------------------- quantize
+// q = E4M3_satRNE(x / s) with IEEE fp32 division.
+__device__ __forceinline__ uint2 quant8(uint4 v, float s) {
+  uint2 o;
+  o.x = pack4(cvt_e4m3x2(__fdiv_rn(bf16_lo(v.x), s), __fdiv_rn(bf16_hi(v.x), s)),
+              cvt_e4m3x2(__fdiv_rn(bf16_lo(v.y), s), __fdiv_rn(bf16_hi(v.y), s)));
+  o.y = pack4(cvt_e4m3x2(__fdiv_rn(bf16_lo(v.z), s), __fdiv_rn(bf16_hi(v.z), s)),
+              cvt_e4m3x2(__fdiv_rn(bf16_lo(v.w), s), __fdiv_rn(bf16_hi(v.w), s)));
+  return o;
+}
+
+__global__ void __launch_bounds__(kEwThreads) quant_static_kernel(
+    const uint16_t *__restrict__ x, int64_t numel, const float *__restrict__ s_in,
+    uint8_t *__restrict__ xq) {
+  const float s = __ldg(s_in);
+  const int64_t nvec = numel >> 3;
+  const uint4 *xv = reinterpret_cast<const uint4 *>(x);
+  uint2 *qv = reinterpret_cast<uint2 *>(xq);
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  int64_t i = tid;
+  for (; i + (kEwUnroll - 1) * stride < nvec; i += kEwUnroll * stride) {
+    uint4 v[kEwUnroll];
+#pragma unroll
+    for (int u = 0; u < kEwUnroll; ++u) v[u] = ld_stream(xv + i + u * stride);
+#pragma unroll
+    for (int u = 0; u < kEwUnroll; ++u) st_stream(qv + i + u * stride, quant8(v[u], s));
+  }
+  for (; i < nvec; i += stride) st_stream(qv + i, quant8(ld_stream(xv + i), s));
+  const int64_t t = (nvec << 3) + tid;
+  if (t < numel) {
+    float a = __uint_as_float(static_cast<uint32_t>(x[t]) << 16);
+    xq[t] = static_cast<uint8_t>(cvt_e4m3x2(__fdiv_rn(a, s), 0.0f) & 0xFFu);
+  }
+}
+
+// ------------------------------------------------------ SwiGLU -> FP8
+// SiLU(g) * u * (1/s) in fp32 with the fast exponential and divide.
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  return __fdividef(g, 1.0f + __expf(-g)) * u;
+}
+
+__device__ __forceinline__ uint2 silu_mul_quant8(uint4 g, uint4 u, float inv_s) {
+  uint2 o;
+  o.x = pack4(cvt_e4m3x2(silu_mul(bf16_lo(g.x), bf16_lo(u.x)) * inv_s,
+                         silu_mul(bf16_hi(g.x), bf16_hi(u.x)) * inv_s),
+              cvt_e4m3x2(silu_mul(bf16_lo(g.y), bf16_lo(u.y)) * inv_s,
+                         silu_mul(bf16_hi(g.y), bf16_hi(u.y)) * inv_s));
+  o.y = pack4(cvt_e4m3x2(silu_mul(bf16_lo(g.z), bf16_lo(u.z)) * inv_s,
+                         silu_mul(bf16_hi(g.z), bf16_hi(u.z)) * inv_s),
+              cvt_e4m3x2(silu_mul(bf16_lo(g.w), bf16_lo(u.w)) * inv_s,
+                         silu_mul(bf16_hi(g.w), bf16_hi(u.w)) * inv_s));
+  return o;
+}
+
+__global__ void __launch_bounds__(kEwThreads) silu_mul_2in_kernel(
+    const uint16_t *__restrict__ g, const uint16_t *__restrict__ u, int64_t numel,
+    const float *__restrict__ s_down, uint8_t *__restrict__ h) {
+  const float inv_s = __frcp_rn(__ldg(s_down));
+  const int64_t nvec = numel >> 3;
+  const uint4 *gv = reinterpret_cast<const uint4 *>(g);
+  const uint4 *uv = reinterpret_cast<const uint4 *>(u);
+  uint2 *hv = reinterpret_cast<uint2 *>(h);
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  int64_t i = tid;
+  for (; i + (kEwUnroll - 1) * stride < nvec; i += kEwUnroll * stride) {
+    uint4 a[kEwUnroll], b[kEwUnroll];
+#pragma unroll
+    for (int k = 0; k < kEwUnroll; ++k) {
+      a[k] = ld_stream(gv + i + k * stride);
+      b[k] = ld_stream(uv + i + k * stride);
+    }
+#pragma unroll
+    for (int k = 0; k < kEwUnroll; ++k) st_stream(hv + i + k * stride, silu_mul_quant8(a[k], b[k], inv_s));
+  }
+  for (; i < nvec; i += stride) st_stream(hv + i, silu_mul_quant8(ld_stream(gv + i), ld_stream(uv + i), inv_s));
+  const int64_t t = (nvec << 3) + tid;
+  if (t < numel) {
+    float a = __uint_as_float(static_cast<uint32_t>(g[t]) << 16);
+    float b = __uint_as_float(static_cast<uint32_t>(u[t]) << 16);
+    h[t] = static_cast<uint8_t>(cvt_e4m3x2(silu_mul(a, b) * inv_s, 0.0f) & 0xFFu);
+  }
+}
+
+// -------------------------------------------------------- calibration
+__device__ __forceinline__ float block_max(float m) {
+  __shared__ float red[kEwThreads / 32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = threadIdx.x < (kEwThreads / 32) ? red[threadIdx.x] : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  }
+  return m;
+}
+
+__device__ __forceinline__ float absmax8(uint4 v, float m) {
+  m = fmaxf(m, fabsf(bf16_lo(v.x)));
+  m = fmaxf(m, fabsf(bf16_hi(v.x)));
+  m = fmaxf(m, fabsf(bf16_lo(v.y)));
+  m = fmaxf(m, fabsf(bf16_hi(v.y)));
+  m = fmaxf(m, fabsf(bf16_lo(v.z)));
+  m = fmaxf(m, fabsf(bf16_hi(v.z)));
+  m = fmaxf(m, fabsf(bf16_lo(v.w)));
+  m = fmaxf(m, fabsf(bf16_hi(v.w)));
+  return m;
+}
+
+// *amax_bits must be zero before the launch; non-negative floats order like
+// their bit patterns, so an unsigned atomicMax on the bits is a float max.
+__global__ void __launch_bounds__(kEwThreads) absmax_bf16_kernel(
+    const uint16_t *__restrict__ x, int64_t numel, unsigned int *__restrict__ amax_bits) {
+  const int64_t nvec = numel >> 3;
+  const uint4 *xv = reinterpret_cast<const uint4 *>(x);
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  float m = 0.0f;
+  for (int64_t i = tid; i < nvec; i += stride) m = absmax8(ld_stream(xv + i), m);
+  const int64_t t = (nvec << 3) + tid;
+  if (t < numel) m = fmaxf(m, fabsf(__uint_as_float(static_cast<uint32_t>(x[t]) << 16)));
+  m = block_max(m);
+  if (threadIdx.x == 0) atomicMax(amax_bits, __float_as_uint(m));
+}
+
+__global__ void __launch_bounds__(kEwThreads) silu_mul_absmax_kernel(
+    const uint16_t *__restrict__ g, const uint16_t *__restrict__ u, int64_t numel,
+    unsigned int *__restrict__ amax_bits) {
+  const int64_t nvec = numel >> 3;
+  const uint4 *gv = reinterpret_cast<const uint4 *>(g);
+  const uint4 *uv = reinterpret_cast<const uint4 *>(u);
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  float m = 0.0f;
+  for (int64_t i = tid; i < nvec; i += stride) {
+    uint4 a = ld_stream(gv + i), b = ld_stream(uv + i);
+    m = fmaxf(m, fabsf(silu_mul(bf16_lo(a.x), bf16_lo(b.x))));
+    m = fmaxf(m, fabsf(silu_mul(bf16_hi(a.x), bf16_hi(b.x))));
+    m = fmaxf(m, fabsf(silu_mul(bf16_lo(a.y), bf16_lo(b.y))));
+    m = fmaxf(m, fabsf(silu_mul(bf16_hi(a.y), bf16_hi(b.y))));
+    m = fmaxf(m, fabsf(silu_mul(bf16_lo(a.z), bf16_lo(b.z))));
+    m = fmaxf(m, fabsf(silu_mul(bf16_hi(a.z), bf16_hi(b.z))));
+    m = fmaxf(m, fabsf(silu_mul(bf16_lo(a.w), bf16_lo(b.w))));
+    m = fmaxf(m, fabsf(silu_mul(bf16_hi(a.w), bf16_hi(b.w))));
+  }
+  const int64_t t = (nvec << 3) + tid;
+  if (t < numel) {
+    float a = __uint_as_float(static_cast<uint32_t>(g[t]) << 16);
+    float b = __uint_as_float(static_cast<uint32_t>(u[t]) << 16);
+    m = fmaxf(m, fabsf(silu_mul(a, b)));
+  }
+  m = block_max(m);
+  if (threadIdx.x == 0) atomicMax(amax_bits, __float_as_uint(m));
+}
+
+// Moving average of per-batch maxima in fp64, written without fused
+// multiply-adds so that every step rounds exactly as the definition reads:
+// A_1 = a_1, A_b = A_{b-1} + c (a_b - A_{b-1}); scale = fp32(A / 448).
+__global__ void observer_scale_kernel(const float *__restrict__ amaxes, int nbatch, double c,
+                                      float *__restrict__ scale) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  double A = static_cast<double>(amaxes[0]);
+  for (int b = 1; b < nbatch; ++b)
+    A = __dadd_rn(A, __dmul_rn(c, __dsub_rn(static_cast<double>(amaxes[b]), A)));
+  *scale = __double2float_rn(__ddiv_rn(A, 448.0));
+}
+
+// RTN weight scale in place: s = amax / 448 (IEEE fp32 division).
+__global__ void rtn_scale_kernel(float *__restrict__ s) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  *s = __fdiv_rn(*s, 448.0f);
+}
+
+}  // namespace fp8ws

@@ -1,0 +1,460 @@
+// C ABI of the static FP8 W8A8 Linear-block library (declared in fp8ws.h).
+//
+// One translation unit: the kernels are included here so that the device
+// status word has a single definition without relocatable device code.
+// Host code validates every argument before enqueueing anything, builds the
+// TMA tensor maps of each GEMM on the host (they travel as kernel
+// parameters, so the calls stay free of device allocations and host syncs),
+// picks the GEMM tile width from the problem shape and records every launch
+// in a small ring for tests and benchmarks.
+#include "../../include/fp8ws.h"
+
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "elementwise.cuh"
+#include "gemm_sm100.cuh"
+
+namespace fp8ws {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kWaitLimitNs = 4ull * 1000 * 1000 * 1000;  // bounded mbarrier waits
+
+// ---------------------------------------------------------------- launch log
+std::mutex g_log_mu;
+fp8ws_launch_record g_log[FP8WS_LOG_CAPACITY];
+int64_t g_log_head = 0;  // records written since the last clear
+int64_t g_launch_total = 0;
+
+void log_launch(int kind, const void *in0, const void *in1, const void *out) {
+  std::lock_guard<std::mutex> lk(g_log_mu);
+  fp8ws_launch_record &r = g_log[g_log_head % FP8WS_LOG_CAPACITY];
+  r.kind = kind;
+  r.pad = 0;
+  r.in0 = in0;
+  r.in1 = in1;
+  r.out = out;
+  ++g_log_head;
+  ++g_launch_total;
+}
+
+enum { kKindQuant = 1, kKindGemm = 2, kKindSwiglu = 3, kKindCalib = 4 };
+
+// --------------------------------------------------------------- device info
+struct DeviceInfo {
+  int checked = 0;  // 0 unknown, 1 sm_100, -1 other
+  int sms = 0;
+  unsigned gemm_attr_set = 0;  // bit per GEMM instantiation
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+int current_device(int *dev) {
+  if (cudaGetDevice(dev) != cudaSuccess) return FP8WS_ERR_CUDA;
+  if (*dev < 0 || *dev >= kMaxDevices) return FP8WS_ERR_UNSUPPORTED;
+  return FP8WS_OK;
+}
+
+int device_info(DeviceInfo **out) {
+  int dev;
+  int st = current_device(&dev);
+  if (st) return st;
+  DeviceInfo &d = g_dev[dev];
+  if (d.checked == 0) {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (d.checked == 0) {
+      int major = 0, minor = 0, sms = 0;
+      if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return FP8WS_ERR_CUDA;
+      d.sms = sms;
+      d.checked = (major == 10 && minor == 0) ? 1 : -1;
+    }
+  }
+  if (d.checked != 1) return FP8WS_ERR_UNSUPPORTED;
+  *out = &d;
+  return FP8WS_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int launch_status() {
+  return cudaGetLastError() == cudaSuccess ? FP8WS_OK : FP8WS_ERR_CUDA;
+}
+
+cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Grid of a streaming kernel: enough blocks for every vector to be visited
+// once by an unrolled iteration, capped at what all SMs hold at once (the
+// kernels loop over the rest with a grid stride).
+template <typename Kernel>
+int ew_grid(const DeviceInfo *d, Kernel kern, int64_t nvec) {
+  static int resident = 0;  // blocks per SM; same on every B200
+  if (resident == 0) {
+    int r = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&r, kern, kEwThreads, 0) != cudaSuccess ||
+        r < 1)
+      r = 1;
+    resident = r;
+  }
+  int64_t per_block = static_cast<int64_t>(kEwThreads) * kEwUnroll;
+  int64_t want = (nvec + per_block - 1) / per_block;
+  int64_t cap = static_cast<int64_t>(d->sms) * resident;
+  if (want > cap) want = cap;
+  if (want < 1) want = 1;
+  return static_cast<int>(want);
+}
+
+// ------------------------------------------------------------- tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Row-major [rows, cols] matrix, 128-byte swizzled boxes of box_cols x box_rows.
+int make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, int elem_bytes, const void *base,
+                int64_t rows, int64_t cols, int box_cols, int box_rows, bool for_load) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return FP8WS_ERR_CUDA;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * elem_bytes};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  for_load ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8WS_OK : FP8WS_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------- GEMM
+template <int BN, int STAGES, int BIT>
+int launch_gemm_cfg(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int M, int N, int K,
+                    const float *s_in, const float *s_w, uint16_t *y, cudaStream_t st) {
+  using C = GemmCfg<BN, STAGES>;
+  auto kern = fp8_gemm_kernel<BN, STAGES>;
+  if (!(d->gemm_attr_set & (1u << BIT))) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+        cudaSuccess)
+      return FP8WS_ERR_CUDA;
+    d->gemm_attr_set |= 1u << BIT;
+  }
+  CUtensorMap ma, mb, md;
+  int rc = make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, xq, M, K, kGemmBK, kGemmBM, true);
+  if (!rc) rc = make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, wq, N, K, kGemmBK, BN, true);
+  if (!rc)
+    rc = make_map_2d(&md, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, M, N, C::EPI_COLS, 32, false);
+  if (rc) return rc;
+  const int tiles = ((M + kGemmBM - 1) / kGemmBM) * ((N + BN - 1) / BN);
+  const int grid = tiles < d->sms ? tiles : d->sms;
+  kern<<<grid, kGemmThreads, C::SMEM_BYTES, st>>>(ma, mb, md, s_in, s_w, M, N, K, kWaitLimitNs);
+  log_launch(kKindGemm, xq, wq, y);
+  return launch_status();
+}
+
+int check_gemm_args(const void *xq, const void *wq, int64_t M, int64_t N, int64_t K,
+                    const float *s_in, const float *s_w, const void *y) {
+  if (!xq || !wq || !s_in || !s_w || !y) return FP8WS_ERR_NULL;
+  if (M < 0 || N < 8 || K < 16 || (N % 8) != 0 || (K % 16) != 0) return FP8WS_ERR_SHAPE;
+  if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+    return FP8WS_ERR_SHAPE;
+  if (!aligned16(xq) || !aligned16(wq) || !aligned16(y)) return FP8WS_ERR_ALIGN;
+  return FP8WS_OK;
+}
+
+// Tile width: the widest of 256/128/64 columns that still gives every SM at
+// least one tile; narrower tiles only when the problem is too small to fill
+// the GPU otherwise.
+int gemm_dispatch(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int64_t M, int64_t N,
+                  int64_t K, const float *s_in, const float *s_w, uint16_t *y, cudaStream_t st) {
+  if (M == 0) return FP8WS_OK;
+  const int64_t num_m = (M + kGemmBM - 1) / kGemmBM;
+  const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
+  if (num_m * ((N + 255) / 256) >= d->sms)
+    return launch_gemm_cfg<256, 4, 0>(d, xq, wq, m, n, k, s_in, s_w, y, st);
+  if (num_m * ((N + 127) / 128) >= d->sms)
+    return launch_gemm_cfg<128, 6, 1>(d, xq, wq, m, n, k, s_in, s_w, y, st);
+  return launch_gemm_cfg<64, 8, 2>(d, xq, wq, m, n, k, s_in, s_w, y, st);
+}
+
+// ----------------------------------------------------------- elementwise
+int quant_launch(DeviceInfo *d, const uint16_t *x, int64_t numel, const float *s, uint8_t *xq,
+                 cudaStream_t st) {
+  if (numel == 0) return FP8WS_OK;
+  quant_static_kernel<<<ew_grid(d, quant_static_kernel, numel >> 3), kEwThreads, 0, st>>>(x, numel, s, xq);
+  log_launch(kKindQuant, x, nullptr, xq);
+  return launch_status();
+}
+
+int silu_launch(DeviceInfo *d, const uint16_t *g, const uint16_t *u, int64_t numel,
+                const float *s, uint8_t *h, cudaStream_t st) {
+  if (numel == 0) return FP8WS_OK;
+  silu_mul_2in_kernel<<<ew_grid(d, silu_mul_2in_kernel, numel >> 3), kEwThreads, 0, st>>>(g, u, numel, s, h);
+  log_launch(kKindSwiglu, g, u, h);
+  return launch_status();
+}
+
+size_t round256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+}  // namespace fp8ws
+
+using namespace fp8ws;
+
+extern "C" {
+
+int fp8_quant_static(const uint16_t *x, int64_t numel, const float *s_in, uint8_t *xq,
+                     void *stream) {
+  if (!x || !s_in || !xq) return FP8WS_ERR_NULL;
+  if (numel < 0) return FP8WS_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(xq)) return FP8WS_ERR_ALIGN;
+  DeviceInfo *d;
+  int rc = device_info(&d);
+  if (rc) return rc;
+  return quant_launch(d, x, numel, s_in, xq, as_stream(stream));
+}
+
+int fp8_linear_static(const uint8_t *xq, const uint8_t *wq, int64_t M, int64_t N, int64_t K,
+                      const float *s_in, const float *s_w, uint16_t *y, void *stream) {
+  int rc = check_gemm_args(xq, wq, M, N, K, s_in, s_w, y);
+  if (rc) return rc;
+  DeviceInfo *d;
+  rc = device_info(&d);
+  if (rc) return rc;
+  return gemm_dispatch(d, xq, wq, M, N, K, s_in, s_w, y, as_stream(stream));
+}
+
+int silu_mul_2in_fp8(const uint16_t *g, const uint16_t *u, int64_t numel, const float *s_down,
+                     uint8_t *h, void *stream) {
+  if (!g || !u || !s_down || !h) return FP8WS_ERR_NULL;
+  if (numel < 0) return FP8WS_ERR_SHAPE;
+  if (!aligned16(g) || !aligned16(u) || !aligned16(h)) return FP8WS_ERR_ALIGN;
+  DeviceInfo *d;
+  int rc = device_info(&d);
+  if (rc) return rc;
+  return silu_launch(d, g, u, numel, s_down, h, as_stream(stream));
+}
+
+size_t gated_mlp_static_fp8_workspace(int64_t M, int64_t d, int64_t I) {
+  if (M < 0 || d < 0 || I < 0) return 0;
+  const size_t m = static_cast<size_t>(M), dd = static_cast<size_t>(d), ii = static_cast<size_t>(I);
+  return round256(m * dd) + 2 * round256(m * ii * 2) + round256(m * ii);
+}
+
+int gated_mlp_static_fp8(const uint16_t *x, int64_t M, int64_t dm, int64_t I, const float *s_in,
+                         const uint8_t *Wg, const float *s_wg, const uint8_t *Wu,
+                         const float *s_wu, const float *s_down, const uint8_t *Wd,
+                         const float *s_wd, void *workspace, uint16_t *y, void *stream) {
+  if (!x || !s_in || !Wg || !s_wg || !Wu || !s_wu || !s_down || !Wd || !s_wd || !y)
+    return FP8WS_ERR_NULL;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FP8WS_ERR_WORKSPACE;
+  if (!aligned16(x)) return FP8WS_ERR_ALIGN;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  const size_t m = static_cast<size_t>(M < 0 ? 0 : M);
+  uint8_t *xq = ws;
+  uint16_t *G = reinterpret_cast<uint16_t *>(ws + round256(m * dm));
+  uint16_t *U = reinterpret_cast<uint16_t *>(reinterpret_cast<uint8_t *>(G) + round256(m * I * 2));
+  uint8_t *H = reinterpret_cast<uint8_t *>(U) + round256(m * I * 2);
+  int rc = check_gemm_args(xq, Wg, M, I, dm, s_in, s_wg, G);
+  if (!rc) rc = check_gemm_args(xq, Wu, M, I, dm, s_in, s_wu, U);
+  if (!rc) rc = check_gemm_args(H, Wd, M, dm, I, s_down, s_wd, y);
+  if (rc) return rc;
+  DeviceInfo *d;
+  rc = device_info(&d);
+  if (rc) return rc;
+  if (M == 0) return FP8WS_OK;
+  cudaStream_t st = as_stream(stream);
+  rc = quant_launch(d, x, M * dm, s_in, xq, st);
+  if (!rc) rc = gemm_dispatch(d, xq, Wg, M, I, dm, s_in, s_wg, G, st);
+  if (!rc) rc = gemm_dispatch(d, xq, Wu, M, I, dm, s_in, s_wu, U, st);
+  if (!rc) rc = silu_launch(d, G, U, M * I, s_down, H, st);
+  if (!rc) rc = gemm_dispatch(d, H, Wd, M, dm, I, s_down, s_wd, y, st);
+  return rc;
+}
+
+size_t qkv_shared_quant_workspace(int64_t M, int64_t d) {
+  if (M < 0 || d < 0) return 0;
+  return round256(static_cast<size_t>(M) * static_cast<size_t>(d));
+}
+
+int qkv_shared_quant(const uint16_t *x, int64_t M, int64_t dm, const float *s_in,
+                     const uint8_t *Wq, int64_t Nq, const float *s_wq, const uint8_t *Wk,
+                     int64_t Nk, const float *s_wk, const uint8_t *Wv, int64_t Nv,
+                     const float *s_wv, void *workspace, uint16_t *q, uint16_t *k, uint16_t *v,
+                     void *stream) {
+  if (!x || !s_in) return FP8WS_ERR_NULL;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FP8WS_ERR_WORKSPACE;
+  if (!aligned16(x)) return FP8WS_ERR_ALIGN;
+  uint8_t *xq = static_cast<uint8_t *>(workspace);
+  int rc = check_gemm_args(xq, Wq, M, Nq, dm, s_in, s_wq, q);
+  if (!rc) rc = check_gemm_args(xq, Wk, M, Nk, dm, s_in, s_wk, k);
+  if (!rc) rc = check_gemm_args(xq, Wv, M, Nv, dm, s_in, s_wv, v);
+  if (rc) return rc;
+  DeviceInfo *d;
+  rc = device_info(&d);
+  if (rc) return rc;
+  if (M == 0) return FP8WS_OK;
+  cudaStream_t st = as_stream(stream);
+  rc = quant_launch(d, x, M * dm, s_in, xq, st);
+  if (!rc) rc = gemm_dispatch(d, xq, Wq, M, Nq, dm, s_in, s_wq, q, st);
+  if (!rc) rc = gemm_dispatch(d, xq, Wk, M, Nk, dm, s_in, s_wk, k, st);
+  if (!rc) rc = gemm_dispatch(d, xq, Wv, M, Nv, dm, s_in, s_wv, v, st);
+  return rc;
+}
+
+int fp8_check_shared_input_scale(const float *const *d_scales, int n, void *stream) {
+  if (!d_scales) return FP8WS_ERR_NULL;
+  if (n < 1 || n > 4096) return FP8WS_ERR_SHAPE;
+  for (int i = 0; i < n; ++i)
+    if (!d_scales[i]) return FP8WS_ERR_NULL;
+  cudaStream_t st = as_stream(stream);
+  float vals[4096];
+  for (int i = 0; i < n; ++i)
+    if (cudaMemcpyAsync(&vals[i], d_scales[i], sizeof(float), cudaMemcpyDeviceToHost, st) !=
+        cudaSuccess)
+      return FP8WS_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return FP8WS_ERR_CUDA;
+  for (int i = 0; i < n; ++i)
+    if (!isfinite(vals[i]) || !(vals[i] > 0.0f)) return FP8WS_ERR_BAD_SCALE;
+  uint32_t b0;
+  memcpy(&b0, &vals[0], 4);
+  for (int i = 1; i < n; ++i) {
+    uint32_t bi;
+    memcpy(&bi, &vals[i], 4);
+    if (bi != b0) return FP8WS_ERR_SCALE_MISMATCH;
+  }
+  return FP8WS_OK;
+}
+
+int fp8_absmax_bf16(const uint16_t *x, int64_t numel, float *amax, void *stream) {
+  if (!x || !amax) return FP8WS_ERR_NULL;
+  if (numel < 0) return FP8WS_ERR_SHAPE;
+  if (!aligned16(x)) return FP8WS_ERR_ALIGN;
+  DeviceInfo *d;
+  int rc = device_info(&d);
+  if (rc) return rc;
+  cudaStream_t st = as_stream(stream);
+  if (cudaMemsetAsync(amax, 0, sizeof(float), st) != cudaSuccess) return FP8WS_ERR_CUDA;
+  if (numel == 0) return FP8WS_OK;
+  absmax_bf16_kernel<<<ew_grid(d, absmax_bf16_kernel, numel >> 3), kEwThreads, 0, st>>>(
+      x, numel, reinterpret_cast<unsigned int *>(amax));
+  log_launch(kKindCalib, x, nullptr, amax);
+  return launch_status();
+}
+
+int fp8_silu_mul_absmax(const uint16_t *g, const uint16_t *u, int64_t numel, float *amax,
+                        void *stream) {
+  if (!g || !u || !amax) return FP8WS_ERR_NULL;
+  if (numel < 0) return FP8WS_ERR_SHAPE;
+  if (!aligned16(g) || !aligned16(u)) return FP8WS_ERR_ALIGN;
+  DeviceInfo *d;
+  int rc = device_info(&d);
+  if (rc) return rc;
+  cudaStream_t st = as_stream(stream);
+  if (cudaMemsetAsync(amax, 0, sizeof(float), st) != cudaSuccess) return FP8WS_ERR_CUDA;
+  if (numel == 0) return FP8WS_OK;
+  silu_mul_absmax_kernel<<<ew_grid(d, silu_mul_absmax_kernel, numel >> 3), kEwThreads, 0, st>>>(
+      g, u, numel, reinterpret_cast<unsigned int *>(amax));
+  log_launch(kKindCalib, g, u, amax);
+  return launch_status();
+}
+
+int fp8_observer_scale(const float *amaxes, int nbatch, double c, float *scale, void *stream) {
+  if (!amaxes || !scale) return FP8WS_ERR_NULL;
+  if (nbatch < 1) return FP8WS_ERR_SHAPE;
+  if (!isfinite(c)) return FP8WS_ERR_BAD_SCALE;
+  DeviceInfo *d;
+  int rc = device_info(&d);
+  if (rc) return rc;
+  observer_scale_kernel<<<1, 32, 0, as_stream(stream)>>>(amaxes, nbatch, c, scale);
+  log_launch(kKindCalib, amaxes, nullptr, scale);
+  return launch_status();
+}
+
+int fp8_rtn_quantize_weight(const uint16_t *w, int64_t numel, float *s_w, uint8_t *wq,
+                            void *stream) {
+  if (!w || !s_w || !wq) return FP8WS_ERR_NULL;
+  if (numel < 1) return FP8WS_ERR_SHAPE;
+  if (!aligned16(w) || !aligned16(wq)) return FP8WS_ERR_ALIGN;
+  int rc = fp8_absmax_bf16(w, numel, s_w, stream);
+  if (rc) return rc;
+  cudaStream_t st = as_stream(stream);
+  rtn_scale_kernel<<<1, 32, 0, st>>>(s_w);
+  log_launch(kKindCalib, s_w, nullptr, s_w);
+  rc = launch_status();
+  if (rc) return rc;
+  return fp8_quant_static(w, numel, s_w, wq, stream);
+}
+
+const char *fp8ws_status_string(int status) {
+  switch (status) {
+    case FP8WS_OK: return "ok";
+    case FP8WS_ERR_NULL: return "null pointer";
+    case FP8WS_ERR_SHAPE: return "unsupported size";
+    case FP8WS_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case FP8WS_ERR_SCALE_MISMATCH: return "group input scales differ";
+    case FP8WS_ERR_BAD_SCALE: return "scale not finite or not positive";
+    case FP8WS_ERR_CUDA: return "CUDA runtime error";
+    case FP8WS_ERR_DEVICE_TIMEOUT: return "bounded wait in a kernel ran out";
+    case FP8WS_ERR_UNSUPPORTED: return "device is not sm_100";
+    case FP8WS_ERR_WORKSPACE: return "workspace NULL or not 256-byte aligned";
+    default: return "unknown status";
+  }
+}
+
+int fp8ws_device_check(void) {
+  DeviceInfo *d;
+  return device_info(&d);
+}
+
+int fp8ws_device_status(int *status, int *where) {
+  if (!status || !where) return FP8WS_ERR_NULL;
+  if (cudaDeviceSynchronize() != cudaSuccess) return FP8WS_ERR_CUDA;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return FP8WS_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return FP8WS_ERR_CUDA;
+  *where = v;
+  *status = v ? FP8WS_ERR_DEVICE_TIMEOUT : FP8WS_OK;
+  return FP8WS_OK;
+}
+
+int64_t fp8ws_launch_count(void) {
+  std::lock_guard<std::mutex> lk(g_log_mu);
+  return g_launch_total;
+}
+
+int fp8ws_launch_log(fp8ws_launch_record *out, int max) {
+  if (!out || max <= 0) return 0;
+  std::lock_guard<std::mutex> lk(g_log_mu);
+  int64_t n = g_log_head < FP8WS_LOG_CAPACITY ? g_log_head : FP8WS_LOG_CAPACITY;
+  if (n > max) n = max;
+  for (int64_t i = 0; i < n; ++i) out[i] = g_log[(g_log_head - n + i) % FP8WS_LOG_CAPACITY];
+  return static_cast<int>(n);
+}
+
+void fp8ws_launch_log_clear(void) {
+  std::lock_guard<std::mutex> lk(g_log_mu);
+  g_log_head = 0;
+}
+
+}  // extern "C"

@@ -1,0 +1,235 @@
+/*
+ * fp8ws: static per-tensor FP8 E4M3 W8A8 Linear blocks for B200 (sm_100a).
+ *
+ * C ABI.  Plain pointers and sizes only; no CUDA or torch types appear in the
+ * signatures.  `stream` is a cudaStream_t passed as void* (NULL = the legacy
+ * default stream).
+ *
+ * Conventions for every entry point:
+ *  - Return value: FP8WS_OK (0) or one of the FP8WS_ERR_* codes below.  No
+ *    call aborts or throws.  Argument checks happen before any work is
+ *    enqueued, so a call that returns an argument error has launched nothing.
+ *  - Memory: the caller owns every buffer.  The hot-path calls allocate
+ *    nothing, never synchronize the device and never read a scale on the host;
+ *    they enqueue kernels on `stream` and return.
+ *  - Tensors are dense and row-major ("contiguous").  BF16 data is passed as
+ *    uint16_t bit patterns, FP8 E4M3 data as uint8_t codes, scales as pointers
+ *    to one device fp32 value each.
+ *  - Alignment: every tensor pointer must be 16-byte aligned
+ *    (FP8WS_ERR_ALIGN otherwise).
+ *  - FP8 E4M3: 1 sign, 4 exponent (bias 7), 3 mantissa bits; largest finite
+ *    value 448; quantization divides by the scale, saturates to +-448 and
+ *    rounds to nearest, ties to even.
+ *  - Errors found inside a kernel (a bounded wait that ran out) are recorded
+ *    in a device status word; fp8ws_device_status() reads and clears it.
+ *
+ * Sources of the operations (the pages this library implements):
+ *  [MC] Hugging Face model card "Cosmos3-Nano-Policy-DROID, FP8 + RTN +
+ *       moving-average activation observer (ModelOpt W8A8, per-tensor
+ *       static)", Scheme table.
+ *  [PR] TensorRT-LLM pull request "Load static FP8 Cosmos3 Nano/Super
+ *       checkpoints without re-quantizing them", sections Description and
+ *       What changed.
+ */
+#ifndef FP8WS_H
+#define FP8WS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FP8WS_API __attribute__((visibility("default")))
+#else
+#define FP8WS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  FP8WS_OK = 0,
+  FP8WS_ERR_NULL = 1,           /* a required pointer is NULL */
+  FP8WS_ERR_SHAPE = 2,          /* a size is negative, zero where not allowed, or unsupported */
+  FP8WS_ERR_ALIGN = 3,          /* a pointer is not 16-byte aligned */
+  FP8WS_ERR_SCALE_MISMATCH = 4, /* group members carry different input scales */
+  FP8WS_ERR_BAD_SCALE = 5,      /* a scale is not finite or not > 0 */
+  FP8WS_ERR_CUDA = 6,           /* a CUDA runtime call failed */
+  FP8WS_ERR_DEVICE_TIMEOUT = 7, /* a bounded wait inside a kernel ran out */
+  FP8WS_ERR_UNSUPPORTED = 8,    /* the current device is not sm_100 */
+  FP8WS_ERR_WORKSPACE = 9       /* workspace NULL or misaligned */
+};
+
+/* ---------------------------------------------------------------- hot path */
+
+/*
+ * fp8_quant_static -- quantize an activation once with its static scale.
+ * [MC] Scheme table (activations FP8 E4M3 with one static scale per tensor);
+ * [PR] What changed (the shared activation is quantized once and handed to
+ * every projection of the group).
+ *
+ *   xq[i] = E4M3_satRNE( fp32(x[i]) / s_in[0] )   (IEEE fp32 division)
+ *
+ * x: device, numel BF16 values, any rank, read as one flat run.
+ * s_in: device, one fp32 value.
+ * xq: device, numel FP8 codes (written).
+ * numel >= 0 (0 launches nothing).
+ */
+FP8WS_API int fp8_quant_static(const uint16_t *x, int64_t numel, const float *s_in, uint8_t *xq,
+                     void *stream);
+
+/*
+ * fp8_linear_static -- W8A8 Linear with the dequant in the GEMM epilogue.
+ * [PR] What changed (each Linear applies its own scale in the GEMM epilogue;
+ * split projections are contiguous Linear outputs); Description (static FP8
+ * keeps one scale per projection).
+ *
+ *   y[m,n] = bf16_RN( (s_in[0]*s_w[0]) * sum_k deq(xq[m,k]) * deq(wq[n,k]) ),
+ *   fp32 accumulation on the tensor cores.
+ *
+ * xq: device [M,K] FP8 codes, row-major.
+ * wq: device [N,K] FP8 codes, row-major (the Linear's [out,in] weight).
+ * s_in, s_w: device, one fp32 value each.
+ * y: device [M,N] BF16, row-major, contiguous (row stride N).
+ * Sizes: M >= 0 (0 launches nothing), N >= 8 with N % 8 == 0, K >= 16 with
+ * K % 16 == 0; M, N, K < 2^31.
+ */
+FP8WS_API int fp8_linear_static(const uint8_t *xq, const uint8_t *wq, int64_t M, int64_t N, int64_t K,
+                      const float *s_in, const float *s_w, uint16_t *y, void *stream);
+
+/*
+ * silu_mul_2in_fp8 -- two-input SwiGLU quantized straight to FP8 for the
+ * down projection.  [PR] What changed (SiLU(G)*U from two separate tensors,
+ * quantized directly for the FP8 down_proj; flat indexing over a 1-D grid, so
+ * any rank works; strided inputs are refused, not copied).
+ *
+ *   h[i] = E4M3_satRNE( SiLU(g[i]) * u[i] / s_down[0] ),  SiLU(g) = g/(1+e^-g),
+ *   computed in fp32 (fast exp and reciprocal; the result may differ from an
+ *   exact evaluation by one E4M3 step on values within rounding noise of a
+ *   code boundary).
+ *
+ * g, u: device, numel BF16 values each, contiguous.  s_down: device fp32.
+ * h: device, numel FP8 codes.  numel >= 0.
+ */
+FP8WS_API int silu_mul_2in_fp8(const uint16_t *g, const uint16_t *u, int64_t numel, const float *s_down,
+                     uint8_t *h, void *stream);
+
+/*
+ * gated_mlp_static_fp8 -- the split gated MLP on the static FP8 path.
+ * [PR] What changed (GatedMLP with split gate/up: quantize the shared
+ * activation once, hand the FP8 tensor to both projections, two-input SwiGLU
+ * to FP8, FP8 down projection).
+ *
+ *   Xq = fp8_quant_static(x, s_in)
+ *   G  = fp8_linear_static(Xq, Wg, s_in, s_wg)      [M,I] BF16
+ *   U  = fp8_linear_static(Xq, Wu, s_in, s_wu)      [M,I] BF16
+ *   H  = silu_mul_2in_fp8(G, U, s_down)             [M,I] FP8
+ *   y  = fp8_linear_static(H, Wd, s_down, s_wd)     [M,d] BF16
+ *
+ * Gate and up share s_in; fp8_check_shared_input_scale proves at load time
+ * that their calibrated input scales are equal.
+ * x: device [M,d] BF16.  Wg, Wu: device [I,d] FP8.  Wd: device [d,I] FP8.
+ * workspace: device, at least gated_mlp_static_fp8_workspace(M,d,I) bytes,
+ * 256-byte aligned; holds Xq, G, U and H (in that order, each region 256-byte
+ * aligned) and is overwritten.  y: device [M,d] BF16.
+ * Sizes: as fp8_linear_static for (M, I, d) and (M, d, I).
+ */
+FP8WS_API size_t gated_mlp_static_fp8_workspace(int64_t M, int64_t d, int64_t I);
+FP8WS_API int gated_mlp_static_fp8(const uint16_t *x, int64_t M, int64_t d, int64_t I, const float *s_in,
+                         const uint8_t *Wg, const float *s_wg, const uint8_t *Wu,
+                         const float *s_wu, const float *s_down, const uint8_t *Wd,
+                         const float *s_wd, void *workspace, uint16_t *y, void *stream);
+
+/*
+ * qkv_shared_quant -- Q/K/V projections from one shared quantization.
+ * [PR] What changed (Attention with shared Q/K/V input quantization: the
+ * activation is quantized once for all three projections; each projection
+ * writes its own contiguous output).
+ *
+ * x: device [M,d] BF16.  Wq [Nq,d], Wk [Nk,d], Wv [Nv,d]: device FP8.
+ * workspace: device, at least qkv_shared_quant_workspace(M,d) bytes, 256-byte
+ * aligned (holds Xq).  q [M,Nq], k [M,Nk], v [M,Nv]: device BF16, contiguous.
+ * Cross-attention, where K/V come from another tensor, must not use this call.
+ */
+FP8WS_API size_t qkv_shared_quant_workspace(int64_t M, int64_t d);
+FP8WS_API int qkv_shared_quant(const uint16_t *x, int64_t M, int64_t d, const float *s_in,
+                     const uint8_t *Wq, int64_t Nq, const float *s_wq, const uint8_t *Wk,
+                     int64_t Nk, const float *s_wk, const uint8_t *Wv, int64_t Nv,
+                     const float *s_wv, void *workspace, uint16_t *q, uint16_t *k, uint16_t *v,
+                     void *stream);
+
+/* ------------------------------------------------------------- load time */
+
+/*
+ * fp8_check_shared_input_scale -- the invariant that shared quantization rests
+ * on: every member of a group carries the same calibrated input scale.
+ * [PR] What changed (post_load_weights validates it at load, never in forward,
+ * because reading a scale on the host synchronizes the device).
+ *
+ * d_scales: host array of n device pointers, each to one fp32 input scale.
+ * n >= 1.  Copies the n values to the host (synchronizes `stream`) and returns
+ * FP8WS_OK if all are finite, > 0 and bitwise equal; FP8WS_ERR_BAD_SCALE if
+ * one is not finite or not > 0; FP8WS_ERR_SCALE_MISMATCH if two differ.
+ */
+FP8WS_API int fp8_check_shared_input_scale(const float *const *d_scales, int n, void *stream);
+
+/*
+ * Calibration helpers (load time; asynchronous on `stream`).
+ * [MC] Scheme table: RTN weights with one scale per tensor; activation scales
+ * from the MOVING_AVERAGE_MINMAX observer with averaging constant 0.01.
+ *
+ * fp8_absmax_bf16: amax[0] = max |x[i]| over numel BF16 values (exact; NaN
+ *   values are ignored; 0 for numel == 0).  amax: device fp32, overwritten.
+ * fp8_silu_mul_absmax: amax[0] = max |SiLU(g[i]) * u[i]| in fp32.
+ * fp8_observer_scale: A_1 = amaxes[0], A_b = A_{b-1} + c (amaxes[b-1] -
+ *   A_{b-1}) in fp64 (no fused multiply-add), then scale[0] = fp32(A / 448).
+ *   amaxes: device, nbatch fp32 values; nbatch >= 1.
+ * fp8_rtn_quantize_weight: s_w[0] = fp32(max|w|) / 448 (fp32 division), then
+ *   wq = fp8_quant_static(w, s_w).  w: device numel BF16; wq: numel FP8.
+ */
+FP8WS_API int fp8_absmax_bf16(const uint16_t *x, int64_t numel, float *amax, void *stream);
+FP8WS_API int fp8_silu_mul_absmax(const uint16_t *g, const uint16_t *u, int64_t numel, float *amax,
+                        void *stream);
+FP8WS_API int fp8_observer_scale(const float *amaxes, int nbatch, double c, float *scale, void *stream);
+FP8WS_API int fp8_rtn_quantize_weight(const uint16_t *w, int64_t numel, float *s_w, uint8_t *wq,
+                            void *stream);
+
+/* ------------------------------------------------------------ diagnostics */
+
+/* Human-readable name of a status code (static string). */
+FP8WS_API const char *fp8ws_status_string(int status);
+
+/* FP8WS_OK if the current device is sm_100 (B200), FP8WS_ERR_UNSUPPORTED
+ * otherwise, FP8WS_ERR_CUDA if no device can be queried. */
+FP8WS_API int fp8ws_device_check(void);
+
+/* Read and clear the device status word of the current device (synchronizes
+ * the device).  *status receives FP8WS_OK or FP8WS_ERR_DEVICE_TIMEOUT;
+ * *where receives a code naming the wait that ran out (0 if none). */
+FP8WS_API int fp8ws_device_status(int *status, int *where);
+
+/* Launch log.  Every kernel the library enqueues is counted and recorded in a
+ * small ring (the most recent FP8WS_LOG_CAPACITY launches).  kind: 1 quant,
+ * 2 GEMM, 3 SwiGLU-quant, 4 calibration.  in0/in1 are the primary input
+ * pointers (for a GEMM: activation and weight), out the output pointer. */
+#define FP8WS_LOG_CAPACITY 64
+typedef struct {
+  int32_t kind;
+  int32_t pad;
+  const void *in0;
+  const void *in1;
+  const void *out;
+} fp8ws_launch_record;
+
+/* Total kernels launched by this library since load (all devices). */
+FP8WS_API int64_t fp8ws_launch_count(void);
+/* Copy up to max most recent records, oldest first; returns how many. */
+FP8WS_API int fp8ws_launch_log(fp8ws_launch_record *out, int max);
+/* Empty the ring (the total count keeps running). */
+FP8WS_API void fp8ws_launch_log_clear(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8WS_H */
