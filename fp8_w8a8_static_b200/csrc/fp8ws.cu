@@ -172,9 +172,11 @@ int launch_gemm_cfg(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int M, 
   return launch_status();
 }
 
+// With M == 0 there is nothing to read or write, so xq and y may be NULL
+// (an empty tensor's data pointer).
 int check_gemm_args(const void *xq, const void *wq, int64_t M, int64_t N, int64_t K,
                     const float *s_in, const float *s_w, const void *y) {
-  if (!xq || !wq || !s_in || !s_w || !y) return FP8WS_ERR_NULL;
+  if (!wq || !s_in || !s_w || (M != 0 && (!xq || !y))) return FP8WS_ERR_NULL;
   if (M < 0 || N < 8 || K < 16 || (N % 8) != 0 || (K % 16) != 0) return FP8WS_ERR_SHAPE;
   if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
     return FP8WS_ERR_SHAPE;
@@ -225,8 +227,9 @@ extern "C" {
 
 int fp8_quant_static(const uint16_t *x, int64_t numel, const float *s_in, uint8_t *xq,
                      void *stream) {
-  if (!x || !s_in || !xq) return FP8WS_ERR_NULL;
   if (numel < 0) return FP8WS_ERR_SHAPE;
+  if (numel == 0) return FP8WS_OK;  // empty tensors may carry NULL pointers
+  if (!x || !s_in || !xq) return FP8WS_ERR_NULL;
   if (!aligned16(x) || !aligned16(xq)) return FP8WS_ERR_ALIGN;
   DeviceInfo *d;
   int rc = device_info(&d);
@@ -246,8 +249,9 @@ int fp8_linear_static(const uint8_t *xq, const uint8_t *wq, int64_t M, int64_t N
 
 int silu_mul_2in_fp8(const uint16_t *g, const uint16_t *u, int64_t numel, const float *s_down,
                      uint8_t *h, void *stream) {
-  if (!g || !u || !s_down || !h) return FP8WS_ERR_NULL;
   if (numel < 0) return FP8WS_ERR_SHAPE;
+  if (numel == 0) return FP8WS_OK;  // empty tensors may carry NULL pointers
+  if (!g || !u || !s_down || !h) return FP8WS_ERR_NULL;
   if (!aligned16(g) || !aligned16(u) || !aligned16(h)) return FP8WS_ERR_ALIGN;
   DeviceInfo *d;
   int rc = device_info(&d);
@@ -265,7 +269,8 @@ int gated_mlp_static_fp8(const uint16_t *x, int64_t M, int64_t dm, int64_t I, co
                          const uint8_t *Wg, const float *s_wg, const uint8_t *Wu,
                          const float *s_wu, const float *s_down, const uint8_t *Wd,
                          const float *s_wd, void *workspace, uint16_t *y, void *stream) {
-  if (!x || !s_in || !Wg || !s_wg || !Wu || !s_wu || !s_down || !Wd || !s_wd || !y)
+  if (!s_in || !Wg || !s_wg || !Wu || !s_wu || !s_down || !Wd || !s_wd ||
+      (M != 0 && (!x || !y)))
     return FP8WS_ERR_NULL;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FP8WS_ERR_WORKSPACE;
   if (!aligned16(x)) return FP8WS_ERR_ALIGN;
@@ -302,7 +307,7 @@ int qkv_shared_quant(const uint16_t *x, int64_t M, int64_t dm, const float *s_in
                      int64_t Nk, const float *s_wk, const uint8_t *Wv, int64_t Nv,
                      const float *s_wv, void *workspace, uint16_t *q, uint16_t *k, uint16_t *v,
                      void *stream) {
-  if (!x || !s_in) return FP8WS_ERR_NULL;
+  if (!s_in || (M != 0 && !x)) return FP8WS_ERR_NULL;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FP8WS_ERR_WORKSPACE;
   if (!aligned16(x)) return FP8WS_ERR_ALIGN;
   uint8_t *xq = static_cast<uint8_t *>(workspace);
@@ -347,7 +352,7 @@ int fp8_check_shared_input_scale(const float *const *d_scales, int n, void *stre
 }
 
 int fp8_absmax_bf16(const uint16_t *x, int64_t numel, float *amax, void *stream) {
-  if (!x || !amax) return FP8WS_ERR_NULL;
+  if (!amax || (numel != 0 && !x)) return FP8WS_ERR_NULL;
   if (numel < 0) return FP8WS_ERR_SHAPE;
   if (!aligned16(x)) return FP8WS_ERR_ALIGN;
   DeviceInfo *d;
@@ -364,7 +369,7 @@ int fp8_absmax_bf16(const uint16_t *x, int64_t numel, float *amax, void *stream)
 
 int fp8_silu_mul_absmax(const uint16_t *g, const uint16_t *u, int64_t numel, float *amax,
                         void *stream) {
-  if (!g || !u || !amax) return FP8WS_ERR_NULL;
+  if (!amax || (numel != 0 && (!g || !u))) return FP8WS_ERR_NULL;
   if (numel < 0) return FP8WS_ERR_SHAPE;
   if (!aligned16(g) || !aligned16(u)) return FP8WS_ERR_ALIGN;
   DeviceInfo *d;

@@ -16,7 +16,8 @@
  *    uint16_t bit patterns, FP8 E4M3 data as uint8_t codes, scales as pointers
  *    to one device fp32 value each.
  *  - Alignment: every tensor pointer must be 16-byte aligned
- *    (FP8WS_ERR_ALIGN otherwise).
+ *    (FP8WS_ERR_ALIGN otherwise).  A tensor with no elements (numel == 0,
+ *    M == 0) may be passed as NULL; such a call succeeds and launches nothing.
  *  - FP8 E4M3: 1 sign, 4 exponent (bias 7), 3 mantissa bits; largest finite
  *    value 448; quantization divides by the scale, saturates to +-448 and
  *    rounds to nearest, ties to even.

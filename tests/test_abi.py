@@ -82,6 +82,9 @@ def test_argument_checks_before_cuda(lib):
     assert lib.fp8_observer_scale(a, 0, 0.01, a, None) == fw.ERR_SHAPE
     assert lib.fp8_rtn_quantize_weight(a, 0, a, a, None) == fw.ERR_SHAPE
     assert lib.fp8_check_shared_input_scale(None, 2, None) == fw.ERR_NULL
+    # empty tensors carry NULL data pointers: nothing to do, nothing launched
+    assert lib.fp8_quant_static(None, 0, None, None, None) == fw.OK
+    assert lib.silu_mul_2in_fp8(None, None, 0, None, None, None) == fw.OK
     assert fw.launch_count() == n0
 
 
