@@ -71,6 +71,8 @@ _SIGS = {
     "gated_mlp_static_fp8_workspace": (ctypes.c_size_t, [_I64, _I64, _I64]),
     "gated_mlp_static_fp8": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _P,
                                             _P, _P, _P]),
+    "gated_mlp_static_fp8_noalloc": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P,
+                                                    _P, _P, _P, _P]),
     "qkv_shared_quant_workspace": (ctypes.c_size_t, [_I64, _I64]),
     "qkv_shared_quant": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _I64, _P, _P, _I64, _P, _P, _I64,
                                         _P, _P, _P, _P, _P, _P]),

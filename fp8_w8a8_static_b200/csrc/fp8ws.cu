@@ -327,6 +327,51 @@ int qkv_shared_quant(const uint16_t *x, int64_t M, int64_t dm, const float *s_in
   return rc;
 }
 
+}  // extern "C"
+
+// Scratch area of gated_mlp_static_fp8_noalloc, for callers that cannot
+// allocate device memory per call.  Reserved in every GPU's memory when the
+// library's module is loaded there and kept until the process exits.  Host
+// code must not pass the array's name to a kernel: on the host it is only a
+// stand-in, and the real device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[FP8WS_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[fp8ws::kMaxDevices];  // device address per device, looked up once
+
+// Device address of the scratch area on the current device; the first call
+// per device looks it up with that device current.
+int noalloc_scratch(void **out) {
+  int dev;
+  int rc = fp8ws::current_device(&dev);
+  if (rc) return rc;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return FP8WS_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FP8WS_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int gated_mlp_static_fp8_noalloc(const uint16_t *x, int64_t M, int64_t d, int64_t I,
+                                 const float *s_in, const uint8_t *Wg, const float *s_wg,
+                                 const uint8_t *Wu, const float *s_wu, const float *s_down,
+                                 const uint8_t *Wd, const float *s_wd, uint16_t *y, void *stream) {
+  if (M < 0 || d < 0 || I < 0) return FP8WS_ERR_SHAPE;
+  if (gated_mlp_static_fp8_workspace(M, d, I) > FP8WS_NOALLOC_SCRATCH_BYTES) return FP8WS_ERR_SHAPE;
+  void *scratch = nullptr;
+  int rc = noalloc_scratch(&scratch);
+  if (rc) return rc;
+  return gated_mlp_static_fp8(x, M, d, I, s_in, Wg, s_wg, Wu, s_wu, s_down, Wd, s_wd, scratch, y,
+                              stream);
+}
+
 int fp8_check_shared_input_scale(const float *const *d_scales, int n, void *stream) {
   if (!d_scales) return FP8WS_ERR_NULL;
   if (n < 1 || n > 4096) return FP8WS_ERR_SHAPE;

@@ -159,6 +159,46 @@ FP8WS_API int qkv_shared_quant(const uint16_t *x, int64_t M, int64_t d, const fl
                      const float *s_wv, void *workspace, uint16_t *q, uint16_t *k, uint16_t *v,
                      void *stream);
 
+/*
+ * gated_mlp_static_fp8_noalloc -- the same gated MLP as gated_mlp_static_fp8,
+ * for callers that cannot allocate device memory when they call it.  The pages
+ * have no counterpart to this entry point; it exists for the caller, not the
+ * method.
+ *
+ * Who needs it: code whose device memory is fixed before it runs, so that a
+ * workspace cannot be obtained per call -- a plugin inside an inference engine
+ * whose enqueue step may not allocate, or a process that hands all device
+ * memory to its own pool at start-up (a robot's policy server, say), where a
+ * cudaMalloc would fail or stall the control loop.
+ *
+ * Instead of a caller-supplied workspace, the call uses one scratch area that
+ * the library reserves as a static device array of
+ * FP8WS_NOALLOC_SCRATCH_BYTES (64 MiB) on every GPU that loads the library,
+ * held until the process exits.  The call itself allocates nothing: no
+ * cudaMalloc, no cudaFree, no allocating library routine.
+ *
+ * Limits and behaviour:
+ *  - Sizes whose gated_mlp_static_fp8_workspace(M, d, I) exceeds
+ *    FP8WS_NOALLOC_SCRATCH_BYTES are refused with FP8WS_ERR_SHAPE before any
+ *    launch (for d = 3072, I = 12288 this allows up to M = 1024 rows).
+ *  - The first call on each device looks up the scratch area's device
+ *    address on that device (cudaGetSymbolAddress, with the device current);
+ *    make that first call before any stream capture.
+ *  - Every call on a device shares the one scratch area, which keeps the
+ *    previous call's contents.  Each call overwrites every byte it reads, so
+ *    nothing needs clearing, but calls that overlap on the GPU (different
+ *    streams without ordering, or different host threads) race on the scratch
+ *    and give wrong results.  Order them on one stream.
+ * Arguments are those of gated_mlp_static_fp8 without the workspace.
+ */
+#define FP8WS_NOALLOC_SCRATCH_BYTES (64ull * 1024 * 1024)
+FP8WS_API int gated_mlp_static_fp8_noalloc(const uint16_t *x, int64_t M, int64_t d, int64_t I,
+                                           const float *s_in, const uint8_t *Wg,
+                                           const float *s_wg, const uint8_t *Wu,
+                                           const float *s_wu, const float *s_down,
+                                           const uint8_t *Wd, const float *s_wd, uint16_t *y,
+                                           void *stream);
+
 /* ------------------------------------------------------------- load time */
 
 /*
