@@ -371,12 +371,92 @@ class OracleSample:
                 f"time per row extrapolated to the 36-layer pass")
 
 
-def cpu_baseline(rows_per_tower: int = 96):
+def cpu_baseline(rows_per_tower: int = 1024):
     o = OracleSample()
     t0 = time.perf_counter()
     spt = o.run(rows_per_tower)
     wall = time.perf_counter() - t0
     return o.tokens_per_s(spt), o.cores, o.describe(rows_per_tower, wall)
+
+
+# ------------------------------------------------------- single kernels
+
+
+L2_FLUSH_BYTES = 256 * 1024 * 1024  # twice the 126 MB L2
+
+
+def kernel_bench(fw, kind, shape, steps, warmup, device):
+    """One kernel on synthetic data shaped like the pages' workloads, timed
+    launch by launch with CUDA events; L2 is flushed (256 MB memset) between
+    launches, outside the timed interval.  Returns a dict for one JSON line."""
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    pk = peaks()
+    if kind == "gemm":
+        M, N, K = shape
+        x = synth.student_t((M, K), 4, synth.seed(1, 90, 0), device)
+        w = synth.normal((N, K), synth.W_STD, synth.seed(1, 90, 10), device)
+        s_in = fw.fp8_observer_scale(fw.fp8_absmax_bf16(x))
+        xq = fw.fp8_quant_static(x, s_in)
+        wq, s_w = fw.fp8_rtn_quantize_weight(w)
+        del x, w
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        fn = lambda: fw.fp8_linear_static(xq, wq, s_in, s_w, out=y)  # noqa: E731
+        work = 2.0 * M * N * K
+        nbytes = M * K + N * K + 2 * M * N
+    elif kind == "swiglu":
+        M, Ii = shape
+        g = synth.normal((M, Ii), 2.0, synth.seed(2, 90, 7), device)
+        u = synth.normal((M, Ii), 1.0, synth.seed(2, 90, 8), device)
+        s = fw.fp8_observer_scale(fw.fp8_silu_mul_absmax(g, u))
+        h = torch.empty((M, Ii), dtype=fw.FP8, device=device)
+        fn = lambda: fw.silu_mul_2in_fp8(g, u, s, out=h)  # noqa: E731
+        work = None
+        nbytes = 5 * M * Ii
+    elif kind == "quant":
+        M, K = shape
+        x = synth.activation_with_outliers(M, K, 9, 0, 0, device)
+        s = fw.fp8_observer_scale(fw.fp8_absmax_bf16(x))
+        xq = torch.empty((M, K), dtype=fw.FP8, device=device)
+        fn = lambda: fw.fp8_quant_static(x, s, out=xq)  # noqa: E731
+        work = None
+        nbytes = 3 * M * K
+    else:
+        raise ValueError(kind)
+    for _ in range(warmup):
+        fn()
+    times = []
+    for _ in range(steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    ms = statistics.median(times)
+    out = {"kernel": kind, "shape": list(shape), "us": ms * 1e3, "steps": steps,
+           "gbs": nbytes / (ms / 1e3) / 1e9, "hbm_frac": nbytes / (ms / 1e3) / 1e9 / pk["hbm"],
+           "l2": "flushed between launches"}
+    if work:
+        out["tflops"] = work / (ms / 1e3) / 1e12
+        out["fp8_peak_frac"] = out["tflops"] / (2.0 * pk["bf16"])
+        out["fp8_peak"] = f"{2.0 * pk['bf16']:.0f} TFLOP/s ({pk['source']} bf16 burst x 2)"
+    st, where = fw.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} at wait site {where}")
+    return out
+
+
+SWEEPS = {
+    "c1": [("gemm", (m, n, synth.C1_K)) for m in synth.C1_M for n in synth.C1_N],
+    "c2": [("swiglu", (m, i)) for m in synth.C2_M for i in synth.C2_I],
+    "c3": [("quant", (synth.C3["M"], synth.C3["d"]))] +
+          [("gemm", (synth.C3["M"], n, synth.C3["d"])) for n in (synth.C3["Nq"], synth.C3["Nk"], synth.C3["Nv"])],
+    "c4": [("gemm", (m, synth.C4["I"], synth.C4["d"])) for m in (1024, 4096)] +
+          [("gemm", (m, synth.C4["d"], synth.C4["I"])) for m in (1024, 4096)] +
+          [("swiglu", (m, synth.C4["I"])) for m in (1024, 4096)] +
+          [("quant", (m, synth.C4["d"])) for m in (1024, 4096)],
+}
 
 
 # -------------------------------------------------------------- dist glue
@@ -429,14 +509,31 @@ def aggregate_value(tokens_per_rank: int, world: int, max_seconds: float) -> flo
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", choices=("gemm", "swiglu", "quant"),
+                    help="time one kernel on one shape instead of the pass")
+    ap.add_argument("--shape", help="M,N,K for gemm; M,I for swiglu; M,K for quant")
+    ap.add_argument("--sweep", choices=tuple(SWEEPS), help="time every kernel shape of a workload")
     args = ap.parse_args()
     log = lambda m: print(m, file=sys.stderr, flush=True)  # noqa: E731
+
+    if args.kernel or args.sweep:
+        import fp8_w8a8_static_b200 as fw
+        device = torch.device("cuda", 0)
+        torch.cuda.set_device(device)
+        fw.load()
+        jobs = ([(args.kernel, tuple(int(v) for v in args.shape.split(",")))] if args.kernel
+                else SWEEPS[args.sweep])
+        for kind, shape in jobs:
+            print(json.dumps(kernel_bench(fw, kind, shape, args.steps, max(args.warmup, 3), device)),
+                  flush=True)
+            torch.cuda.empty_cache()
+        return 0
 
     ctx = DistCtx()
     if args.impl == "reference":
