@@ -387,9 +387,11 @@ L2_FLUSH_BYTES = 256 * 1024 * 1024  # twice the 126 MB L2
 
 def kernel_bench(fw, kind, shape, steps, warmup, device):
     """One kernel on synthetic data shaped like the pages' workloads, timed
-    launch by launch with CUDA events; L2 is flushed (256 MB memset) between
-    launches, outside the timed interval.  Returns a dict for one JSON line."""
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    launch by launch with CUDA events.  Between launches, outside the timed
+    interval, L2 is flushed by reading a 256 MB buffer (a read leaves no dirty
+    lines to be written back inside the next timed launch).  Returns a dict for
+    one JSON line."""
+    flush = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     pk = peaks()
     if kind == "gemm":
         M, N, K = shape
@@ -426,7 +428,7 @@ def kernel_bench(fw, kind, shape, steps, warmup, device):
         fn()
     times = []
     for _ in range(steps):
-        flush.zero_()
+        flush.sum()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         fn()

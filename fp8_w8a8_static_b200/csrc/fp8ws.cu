@@ -17,6 +17,7 @@
 
 #include "common.cuh"
 #include "elementwise.cuh"
+#include "gemm_pair_sm100.cuh"
 #include "gemm_sm100.cuh"
 
 namespace fp8ws {
@@ -50,6 +51,7 @@ struct DeviceInfo {
   int checked = 0;  // 0 unknown, 1 sm_100, -1 other
   int sms = 0;
   unsigned gemm_attr_set = 0;  // bit per GEMM instantiation
+  int pair_clusters = 0;       // CTA pairs of the pair GEMM resident at once
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -174,6 +176,50 @@ int launch_gemm_cfg(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int M, 
 
 // With M == 0 there is nothing to read or write, so xq and y may be NULL
 // (an empty tensor's data pointer).
+// CTA-pair GEMM: one cluster of two CTAs per TPC, persistent over 256 x 256
+// tiles.  The grid holds as many pairs as can be resident at once.
+template <int STAGES, int BIT>
+int launch_gemm_pair(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int M, int N, int K,
+                     const float *s_in, const float *s_w, uint16_t *y, cudaStream_t st) {
+  using C = PairCfg<STAGES>;
+  auto kern = fp8_gemm_pair_kernel<STAGES>;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (!(d->gemm_attr_set & (1u << BIT))) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+        cudaSuccess)
+      return FP8WS_ERR_CUDA;
+    int clusters = 0;
+    cfg.gridDim = dim3(2 * (d->sms / 2));
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1)
+      return FP8WS_ERR_CUDA;
+    d->pair_clusters = clusters;
+    d->gemm_attr_set |= 1u << BIT;
+  }
+  CUtensorMap ma, mb, md;
+  int rc = make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, xq, M, K, kGemmBK, 128, true);
+  if (!rc) rc = make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, wq, N, K, kGemmBK, 128, true);
+  if (!rc)
+    rc = make_map_2d(&md, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, M, N, C::EPI_COLS, 32, false);
+  if (rc) return rc;
+  const int tiles = ((M + kPairTile - 1) / kPairTile) * ((N + kPairTile - 1) / kPairTile);
+  const int clusters = tiles < d->pair_clusters ? tiles : d->pair_clusters;
+  cfg.gridDim = dim3(2 * clusters);
+  if (cudaLaunchKernelEx(&cfg, kern, ma, mb, md, s_in, s_w, M, N, K, kWaitLimitNs) != cudaSuccess)
+    return FP8WS_ERR_CUDA;
+  log_launch(kKindGemm, xq, wq, y);
+  return launch_status();
+}
+
 int check_gemm_args(const void *xq, const void *wq, int64_t M, int64_t N, int64_t K,
                     const float *s_in, const float *s_w, const void *y) {
   if (!wq || !s_in || !s_w || (M != 0 && (!xq || !y))) return FP8WS_ERR_NULL;
@@ -184,14 +230,16 @@ int check_gemm_args(const void *xq, const void *wq, int64_t M, int64_t N, int64_
   return FP8WS_OK;
 }
 
-// Tile width: the widest of 256/128/64 columns that still gives every SM at
-// least one tile; narrower tiles only when the problem is too small to fill
-// the GPU otherwise.
+// Tile shape: CTA-pair 256 x 256 tiles when there is at least one per TPC;
+// otherwise one CTA per tile with the widest of 256/128/64 columns that still
+// gives every SM a tile (narrower only when the problem is too small).
 int gemm_dispatch(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int64_t M, int64_t N,
                   int64_t K, const float *s_in, const float *s_w, uint16_t *y, cudaStream_t st) {
   if (M == 0) return FP8WS_OK;
   const int64_t num_m = (M + kGemmBM - 1) / kGemmBM;
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
+  if (((M + 255) / 256) * ((N + 255) / 256) >= d->sms / 2)
+    return launch_gemm_pair<6, 3>(d, xq, wq, m, n, k, s_in, s_w, y, st);
   if (num_m * ((N + 255) / 256) >= d->sms)
     return launch_gemm_cfg<256, 4, 0>(d, xq, wq, m, n, k, s_in, s_w, y, st);
   if (num_m * ((N + 127) / 128) >= d->sms)

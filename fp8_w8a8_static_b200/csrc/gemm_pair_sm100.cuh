@@ -1,0 +1,263 @@
+// FP8 E4M3 W8A8 GEMM on CTA pairs (tcgen05 cta_group::2), for sm_100a.
+//
+//   Y[M,N] = bf16( (s_in * s_w) * Xq[M,K] . Wq[N,K]^T ),  fp32 accumulation
+//
+// Same contract as fp8_gemm_kernel, with 256 x 256 output tiles computed by a
+// cluster of two CTAs on the two SMs of a TPC.  Each CTA loads 128 rows of A
+// and 128 rows of B per 128-byte K step (32 KB instead of 48 KB per SM for the
+// same tensor work), both CTAs' loads count on the leader CTA's barrier, and
+// the leader issues one M=256, N=256 tcgen05.mma over both CTAs' shared
+// memory.  Each CTA's TMEM holds the accumulator of its own 128 rows; both
+// CTAs run the epilogue on their own rows.
+//   warp 0      TMA producer (both CTAs; no cluster multicast)
+//   warp 1      TMEM allocation (both CTAs, cta_group::2); MMA issue (leader)
+//   warps 2..5  epilogue (both CTAs)
+// Bounded waits as in fp8_gemm_kernel.  Both CTAs always reach the final
+// cluster barrier, so neither leaves while its peer may still touch its
+// shared memory or TMEM.
+#pragma once
+
+#include "common.cuh"
+#include "gemm_sm100.cuh"
+
+namespace fp8ws {
+
+constexpr int kPairTile = 256;  // output rows and columns per CTA pair
+
+template <int STAGES_>
+struct PairCfg {
+  static constexpr int STAGES = STAGES_;
+  static constexpr int A_BYTES = 128 * kGemmBK;   // this CTA's half of A
+  static constexpr int B_BYTES = 128 * kGemmBK;   // this CTA's half of B
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TX_BYTES = 2 * STAGE_BYTES;  // both CTAs, counted at the leader
+  static constexpr int EPI_COLS = 64;
+  static constexpr int EPI_BUF_BYTES = 32 * EPI_COLS * 2;
+  static constexpr int EPI_BYTES = 4 * 2 * EPI_BUF_BYTES;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;  // two 256-column accumulators
+  static_assert((2 * STAGES + 5) * 8 + 8 <= BAR_BYTES, "barrier area");
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+
+template <int STAGES>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
+                         const __grid_constant__ CUtensorMap tm_b,
+                         const __grid_constant__ CUtensorMap tm_d, const float *__restrict__ s_in,
+                         const float *__restrict__ s_w, int M, int N, int K,
+                         uint64_t timeout_ns) {
+  using C = PairCfg<STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sA = smem;
+  uint8_t *sB = smem + STAGES * C::A_BYTES;
+  uint8_t *sEpi = sB + STAGES * C::B_BYTES;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sEpi + C::EPI_BYTES);
+  uint64_t *full = bars;              // leader: both CTAs' loads of a stage landed
+  uint64_t *empty = bars + STAGES;    // both: the leader's MMAs finished with a stage
+  uint64_t *tfull = bars + 2 * STAGES;  // both: an accumulator is complete
+  uint64_t *tempty = tfull + 2;       // leader: both CTAs' epilogues read an accumulator
+  uint64_t *drain = tempty + 2;       // leader: every MMA retired
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cluster = blockIdx.x >> 1;
+  const int nclusters = gridDim.x >> 1;
+  const int num_m = (M + kPairTile - 1) / kPairTile;
+  const int num_n = (N + kPairTile - 1) / kPairTile;
+  const int num_tiles = num_m * num_n;
+  const int num_kb = (K + kGemmBK - 1) / kGemmBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 8);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+    tma_prefetch_desc(&tm_d);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      uint32_t issued_mask = 0, issued_parity = 0;
+      bool ok = true;
+      for (int t = cluster; t < num_tiles && ok; t += nclusters) {
+        const TileCoord tc = tile_coord(t, num_m, num_n);
+        const int a_row = tc.m * kPairTile + static_cast<int>(rank) * 128;
+        const int b_row = tc.n * kPairTile + static_cast<int>(rank) * 128;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, timeout_ns)) {
+            record_timeout(kSiteProducerEmpty);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          const uint32_t full_leader = map_shared_rank(smem_u32(&full[stage]), 0);
+          if (leader) mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
+          tma_load_2d_pair(sA + stage * C::A_BYTES, &tm_a, full_leader, kb * kGemmBK, a_row);
+          tma_load_2d_pair(sB + stage * C::B_BYTES, &tm_b, full_leader, kb * kGemmBK, b_row);
+          issued_mask |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok && leader) {
+        // Let the loads of the rounds this CTA started land before leaving.
+        int zero = 0;
+        for (int s = 0; s < STAGES; ++s)
+          if (issued_mask & (1u << s))
+            mbar_wait_bounded(&full[s], (issued_parity >> s) & 1u, &zero, timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------- MMA issue (leader)
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(kPairTile, kPairTile);
+      uint32_t stage = 0, phase = 0;
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = cluster; t < num_tiles && ok; t += nclusters, ++it) {
+        const uint32_t acc = it & 1u;
+        const uint32_t acc_phase = (it >> 1) & 1u;
+        if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, timeout_ns)) {
+          record_timeout(kSiteMmaTmemEmpty);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * kPairTile;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, timeout_ns)) {
+            record_timeout(kSiteMmaFull);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * C::A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * C::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < kGemmBK / 32; ++k) {
+            umma_f8_pair(d_tmem, smem_desc_k_sw128(a_addr + k * 32),
+                         smem_desc_k_sw128(b_addr + k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          umma_commit_pair(&empty[stage], 0x3);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) umma_commit_pair(&tfull[acc], 0x3);
+      }
+      umma_commit_pair(drain, 0x1);
+      int zero = 0;
+      if (!mbar_wait_bounded(drain, 0, &zero, timeout_ns)) record_timeout(kSiteDrain);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ epilogue (both CTAs)
+    const int ew = warp - 2;
+    const int quarter = warp & 3;
+    const float scale = __ldg(s_in) * __ldg(s_w);
+    uint32_t it = 0, chunk = 0;
+    for (int t = cluster; t < num_tiles; t += nclusters, ++it) {
+      const TileCoord tc = tile_coord(t, num_m, num_n);
+      const uint32_t acc = it & 1u;
+      const uint32_t acc_phase = (it >> 1) & 1u;
+      if (!mbar_wait_bounded_warp(&tfull[acc], acc_phase, abort_flag, timeout_ns)) {
+        if (lane == 0) {
+          record_timeout(kSiteEpiTmemFull);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      tc_fence_after();
+      const int row0 = tc.m * kPairTile + static_cast<int>(rank) * 128 + quarter * 32;
+      const uint32_t t_row =
+          tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kPairTile;
+      constexpr int NCHUNK = kPairTile / C::EPI_COLS;
+#pragma unroll 1
+      for (int c = 0; c < NCHUNK; ++c) {
+        uint32_t r0[32], r1[32];
+        tmem_ld_32x32b_x32(t_row + c * C::EPI_COLS, r0);
+        tmem_ld_32x32b_x32(t_row + c * C::EPI_COLS + 32, r1);
+        tmem_ld_wait();
+        if (c == NCHUNK - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(map_shared_rank(smem_u32(&tempty[acc]), 0));
+        }
+        const int col0 = tc.n * kPairTile + c * C::EPI_COLS;
+        if (col0 >= N || row0 >= M) continue;  // whole chunk outside Y
+        uint8_t *buf = sEpi + (ew * 2 + (chunk & 1u)) * C::EPI_BUF_BYTES;
+        if (lane == 0) tma_store_wait_read<1>();
+        __syncwarp();
+        uint8_t *row = buf + lane * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t *src = (j < 4) ? &r0[j * 8] : &r1[(j - 4) * 8];
+          uint4 v;
+          __nv_bfloat162 p0 = __floats2bfloat162_rn(__uint_as_float(src[0]) * scale,
+                                                    __uint_as_float(src[1]) * scale);
+          __nv_bfloat162 p1 = __floats2bfloat162_rn(__uint_as_float(src[2]) * scale,
+                                                    __uint_as_float(src[3]) * scale);
+          __nv_bfloat162 p2 = __floats2bfloat162_rn(__uint_as_float(src[4]) * scale,
+                                                    __uint_as_float(src[5]) * scale);
+          __nv_bfloat162 p3 = __floats2bfloat162_rn(__uint_as_float(src[6]) * scale,
+                                                    __uint_as_float(src[7]) * scale);
+          v.x = *reinterpret_cast<uint32_t *>(&p0);
+          v.y = *reinterpret_cast<uint32_t *>(&p1);
+          v.z = *reinterpret_cast<uint32_t *>(&p2);
+          v.w = *reinterpret_cast<uint32_t *>(&p3);
+          *reinterpret_cast<uint4 *>(row + ((j ^ (lane & 7)) << 4)) = v;
+        }
+        fence_async_shared();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tm_d, buf, col0, row0);
+          tma_store_commit();
+        }
+        ++chunk;
+      }
+    }
+    if (lane == 0) tma_store_wait_all<0>();
+  }
+
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace fp8ws
