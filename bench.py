@@ -164,13 +164,18 @@ def prepare(fw, device, n_layers, log):
     return layers
 
 
-def make_buffers(fw, layers, device):
+def make_buffers(fw, layers, device, fused):
     ws = {}
     bufs = {}
     for tower, M in TOWERS:
-        nbytes = fw.gated_mlp_static_fp8_workspace(M, D, I)
-        ws[tower] = torch.empty(nbytes, dtype=torch.uint8, device=device)
-        bufs[tower] = fw.gated_mlp_workspace_views(ws[tower], M, D, I)
+        if fused:
+            nbytes = fw.gated_mlp_static_fp8_fused_workspace(M, D, I)
+            ws[tower] = torch.empty(nbytes, dtype=torch.uint8, device=device)
+            bufs[tower] = fw.fused_workspace_views(ws[tower], M, D, I)
+        else:
+            nbytes = fw.gated_mlp_static_fp8_workspace(M, D, I)
+            ws[tower] = torch.empty(nbytes, dtype=torch.uint8, device=device)
+            bufs[tower] = fw.gated_mlp_workspace_views(ws[tower], M, D, I)
     for L in layers:
         L.y = torch.empty((L.M, D), dtype=torch.bfloat16, device=device)
     return ws, bufs
@@ -179,26 +184,35 @@ def make_buffers(fw, layers, device):
 # ---------------------------------------------------------- timed region
 
 
-def build_plan(fw, layers, bufs, stream_handle):
-    """The pass as a flat list of direct C-ABI calls (kind, fn, args), in the
-    same order the composite gated-MLP call issues them."""
+def build_plan(fw, layers, bufs, stream_handle, fused):
+    """The pass as a flat list of direct C-ABI calls (kind, fn, args,
+    algorithmic bytes, flops), in the order the composite gated-MLP call
+    issues them.  Fused: quantize X, fused gate/up GEMM + SwiGLU-quant, down
+    GEMM.  Unfused: quantize X, gate GEMM, up GEMM, SwiGLU-quant, down GEMM."""
     lib = fw.load()
     plan = []
     for L in layers:
         b = bufs[L.tower]
         M = L.M
-        xq, g, u, h = b["xq"].data_ptr(), b["g"].data_ptr(), b["u"].data_ptr(), b["h"].data_ptr()
+        xq, h = b["xq"].data_ptr(), b["h"].data_ptr()
         s_in, s_down = L.s_in.data_ptr(), L.s_down.data_ptr()
         plan.append(("quant", lib.fp8_quant_static,
                      (L.x.data_ptr(), M * D, s_in, xq, stream_handle), 3 * M * D, 0))
-        plan.append(("gemm", lib.fp8_linear_static,
-                     (xq, L.wg.data_ptr(), M, I, D, s_in, L.s_wg.data_ptr(), g, stream_handle),
-                     M * D + I * D + 2 * M * I, 2 * M * I * D))
-        plan.append(("gemm", lib.fp8_linear_static,
-                     (xq, L.wu.data_ptr(), M, I, D, s_in, L.s_wu.data_ptr(), u, stream_handle),
-                     M * D + I * D + 2 * M * I, 2 * M * I * D))
-        plan.append(("swiglu", lib.silu_mul_2in_fp8, (g, u, M * I, s_down, h, stream_handle),
-                     5 * M * I, 0))
+        if fused:
+            plan.append(("gate_up_swiglu", lib.fp8_gate_up_swiglu_static,
+                         (xq, L.wg.data_ptr(), L.wu.data_ptr(), M, I, D, s_in, L.s_wg.data_ptr(),
+                          L.s_wu.data_ptr(), s_down, h, stream_handle),
+                         M * D + 2 * I * D + M * I, 4 * M * I * D))
+        else:
+            g, u = b["g"].data_ptr(), b["u"].data_ptr()
+            plan.append(("gemm", lib.fp8_linear_static,
+                         (xq, L.wg.data_ptr(), M, I, D, s_in, L.s_wg.data_ptr(), g, stream_handle),
+                         M * D + I * D + 2 * M * I, 2 * M * I * D))
+            plan.append(("gemm", lib.fp8_linear_static,
+                         (xq, L.wu.data_ptr(), M, I, D, s_in, L.s_wu.data_ptr(), u, stream_handle),
+                         M * D + I * D + 2 * M * I, 2 * M * I * D))
+            plan.append(("swiglu", lib.silu_mul_2in_fp8, (g, u, M * I, s_down, h, stream_handle),
+                         5 * M * I, 0))
         plan.append(("gemm", lib.fp8_linear_static,
                      (h, L.wd.data_ptr(), M, D, I, s_down, L.s_wd.data_ptr(), L.y.data_ptr(),
                       stream_handle),
@@ -255,7 +269,7 @@ def time_device(plan, steps, warmup, dist_ctx, sampler=None):
     return total_ms, per_kind, clocks
 
 
-def time_e2e(fw, layers, steps, warmup, device, dist_ctx):
+def time_e2e(fw, layers, steps, warmup, device, dist_ctx, fused):
     """The pass through the composite C-ABI call with host buffers: each
     layer's X is copied from pinned host memory on a copy stream, the gated
     MLP runs on the compute stream, Y is copied back to pinned host memory on
@@ -267,8 +281,9 @@ def time_e2e(fw, layers, steps, warmup, device, dist_ctx):
           for t, M in TOWERS}
     dy = {t: [torch.empty((M, D), dtype=torch.bfloat16, device=device) for _ in range(2)]
           for t, M in TOWERS}
-    ws = {t: torch.empty(fw.gated_mlp_static_fp8_workspace(M, D, I), dtype=torch.uint8,
-                         device=device) for t, M in TOWERS}
+    wsize = fw.gated_mlp_static_fp8_fused_workspace if fused else fw.gated_mlp_static_fp8_workspace
+    mlp = fw.gated_mlp_static_fp8_fused if fused else fw.gated_mlp_static_fp8
+    ws = {t: torch.empty(wsize(M, D, I), dtype=torch.uint8, device=device) for t, M in TOWERS}
     comp = torch.cuda.Stream(device)
     h2d = torch.cuda.Stream(device)
     d2h = torch.cuda.Stream(device)
@@ -292,7 +307,7 @@ def time_e2e(fw, layers, steps, warmup, device, dist_ctx):
                 comp.wait_event(ready[i])
                 if i >= 4:
                     comp.wait_event(copied_out[i - 4])  # slot's previous output copied out
-                fw.gated_mlp_static_fp8(dx[L.tower][slot], L.s_in, L.wg, L.s_wg, L.wu, L.s_wu,
+                mlp(dx[L.tower][slot], L.s_in, L.wg, L.s_wg, L.wu, L.s_wu,
                                         L.s_down, L.wd, L.s_wd, workspace=ws[L.tower],
                                         out=dy[L.tower][slot], stream=comp)
                 done[i].record(comp)
@@ -405,6 +420,19 @@ def kernel_bench(fw, kind, shape, steps, warmup, device):
         fn = lambda: fw.fp8_linear_static(xq, wq, s_in, s_w, out=y)  # noqa: E731
         work = 2.0 * M * N * K
         nbytes = M * K + N * K + 2 * M * N
+    elif kind == "dual":
+        M, N, K = shape
+        x = synth.activation_with_outliers(M, K, 9, 1, 0, device)
+        s_in = fw.fp8_observer_scale(fw.fp8_absmax_bf16(x))
+        xq = fw.fp8_quant_static(x, s_in)
+        wg, s_wg = fw.fp8_rtn_quantize_weight(synth.normal((N, K), synth.W_STD, synth.seed(4, 90, 1), device))
+        wu, s_wu = fw.fp8_rtn_quantize_weight(synth.normal((N, K), synth.W_STD, synth.seed(4, 90, 2), device))
+        s_down = torch.tensor([0.003], dtype=torch.float32, device=device)
+        del x
+        h = torch.empty((M, N), dtype=fw.FP8, device=device)
+        fn = lambda: fw.fp8_gate_up_swiglu_static(xq, wg, wu, s_in, s_wg, s_wu, s_down, out=h)  # noqa: E731
+        work = 4.0 * M * N * K
+        nbytes = M * K + 2 * N * K + M * N
     elif kind == "swiglu":
         M, Ii = shape
         g = synth.normal((M, Ii), 2.0, synth.seed(2, 90, 7), device)
@@ -454,7 +482,8 @@ SWEEPS = {
     "c2": [("swiglu", (m, i)) for m in synth.C2_M for i in synth.C2_I],
     "c3": [("quant", (synth.C3["M"], synth.C3["d"]))] +
           [("gemm", (synth.C3["M"], n, synth.C3["d"])) for n in (synth.C3["Nq"], synth.C3["Nk"], synth.C3["Nv"])],
-    "c4": [("gemm", (m, synth.C4["I"], synth.C4["d"])) for m in (1024, 4096)] +
+    "c4": [("dual", (m, synth.C4["I"], synth.C4["d"])) for m in (1024, 4096)] +
+          [("gemm", (m, synth.C4["I"], synth.C4["d"])) for m in (1024, 4096)] +
           [("gemm", (m, synth.C4["d"], synth.C4["I"])) for m in (1024, 4096)] +
           [("swiglu", (m, synth.C4["I"])) for m in (1024, 4096)] +
           [("quant", (m, synth.C4["d"])) for m in (1024, 4096)],
@@ -517,9 +546,11 @@ def main():
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=("gemm", "swiglu", "quant"),
+    ap.add_argument("--unfused", action="store_true",
+                    help="time the five-kernel composition (separate gate/up GEMMs and SwiGLU-quant)")
+    ap.add_argument("--kernel", choices=("gemm", "dual", "swiglu", "quant"),
                     help="time one kernel on one shape instead of the pass")
-    ap.add_argument("--shape", help="M,N,K for gemm; M,I for swiglu; M,K for quant")
+    ap.add_argument("--shape", help="M,N,K for gemm; M,I,K for dual; M,I for swiglu; M,K for quant")
     ap.add_argument("--sweep", choices=tuple(SWEEPS), help="time every kernel shape of a workload")
     args = ap.parse_args()
     log = lambda m: print(m, file=sys.stderr, flush=True)  # noqa: E731
@@ -576,9 +607,10 @@ def main():
         raise RuntimeError("not an sm_100 device")
     pk = peaks()
     layers = prepare(fw, device, args.layers, log)
-    ws, bufs = make_buffers(fw, layers, device)
+    fused = not args.unfused
+    ws, bufs = make_buffers(fw, layers, device, fused)
     stream = torch.cuda.current_stream(device)
-    plan = build_plan(fw, layers, bufs, stream.cuda_stream)
+    plan = build_plan(fw, layers, bufs, stream.cuda_stream, fused)
 
     launches_before = fw.launch_count()
     sampler = ClockSampler(device.index if device.index is not None else 0)
@@ -601,19 +633,27 @@ def main():
             d["tflops"] = flops / (ms / 1e3) / 1e12
         d["gbs"] = nbytes / (ms / 1e3) / 1e9
         comp[kind] = d
-    gemm = per_kind["gemm"]
+    # the dominant kernel: largest share of the pass; all its launches, flop-weighted
+    tensor_kinds = [k for k in per_kind if per_kind[k][3]]
+    dom = max(tensor_kinds, key=lambda k: per_kind[k][0])
     fp8_peak = 2.0 * pk["bf16_sustained"]
-    achieved = gemm[3] / (gemm[0] / 1e3) / 1e12
+    achieved = per_kind[dom][3] / (per_kind[dom][0] / 1e3) / 1e12
+    names = {"gemm": "fp8_gemm_kernel / fp8_gemm_pair_kernel",
+             "gate_up_swiglu": "fp8_dual_swiglu_pair_kernel (gate/up GEMMs + SwiGLU-quant)"}
     roofline = {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
                 "frac": achieved / fp8_peak, "traffic": None,
-                "kernel": "fp8_gemm_kernel (all GEMM launches of the pass, flop-weighted)",
+                "kernel": f"{names[dom]}, all launches of the pass, flop-weighted",
                 "peak_source": f"{pk['source']}: bf16 sustained {pk['bf16_sustained']} TFLOP/s x 2 (nominal fp8/bf16 ratio)"}
-    comp["swiglu"]["hbm_frac"] = comp["swiglu"]["gbs"] / pk["hbm"]
-    comp["quant"]["hbm_frac"] = comp["quant"]["gbs"] / pk["hbm"]
+    for k in ("swiglu", "quant"):
+        if k in comp:
+            comp[k]["hbm_frac"] = comp[k]["gbs"] / pk["hbm"]
+    all_flops = sum(v[3] for v in per_kind.values())
+    all_tensor_ms = sum(per_kind[k][0] for k in tensor_kinds)
+    comp["all_tensor_kernels_tflops"] = all_flops / (all_tensor_ms / 1e3) / 1e12
 
     e2e = None
     if not args.no_e2e:
-        ms, hb, db, h_y = time_e2e(fw, layers, max(1, args.steps // 2), 1, device, ctx)
+        ms, hb, db, h_y = time_e2e(fw, layers, max(1, args.steps // 2), 1, device, ctx, fused)
         ms = ctx.max(ms)
         torch.cuda.synchronize()
         same = torch.equal(h_y[-1], layers[-1].y.cpu())
@@ -635,6 +675,8 @@ def main():
             "vs_baseline": None, "dtype": "fp8-e4m3 MMA, fp32 accumulate, bf16 out",
             "data": "synthetic",
             "config": {"workload": "two-tower MoT decoder-MLP pass, 36 layers x {und M=1024, gen M=4096}, d=3072, I=12288",
+                       "path": ("fused: quantize X -> gate/up GEMM with SwiGLU-quant epilogue -> down GEMM"
+                                if fused else "unfused: quantize X -> gate GEMM -> up GEMM -> SwiGLU-quant -> down GEMM"),
                        "layers": args.layers, "global_batch": TOKENS_PER_STEP * ctx.world,
                        "parallelism": f"replicas x{ctx.world}",
                        "l2": "inputs larger than L2 (8.15 GB of FP8 weights per pass)"},

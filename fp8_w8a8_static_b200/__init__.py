@@ -26,6 +26,8 @@ __all__ = [
     "FP8WSError", "library_path", "load",
     "fp8_quant_static", "fp8_linear_static", "silu_mul_2in_fp8",
     "gated_mlp_static_fp8", "gated_mlp_static_fp8_workspace",
+    "fp8_gate_up_swiglu_static", "gated_mlp_static_fp8_fused",
+    "gated_mlp_static_fp8_fused_workspace",
     "qkv_shared_quant", "qkv_shared_quant_workspace",
     "fp8_check_shared_input_scale", "fp8_absmax_bf16", "fp8_silu_mul_absmax",
     "fp8_observer_scale", "fp8_rtn_quantize_weight",
@@ -48,7 +50,7 @@ STATUS = {
 OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_SCALE_MISMATCH, ERR_BAD_SCALE, ERR_CUDA, \
     ERR_DEVICE_TIMEOUT, ERR_UNSUPPORTED, ERR_WORKSPACE = range(10)
 
-KIND_QUANT, KIND_GEMM, KIND_SWIGLU, KIND_CALIB = 1, 2, 3, 4
+KIND_QUANT, KIND_GEMM, KIND_SWIGLU, KIND_CALIB, KIND_DUAL = 1, 2, 3, 4, 5
 
 
 class FP8WSError(RuntimeError):
@@ -71,6 +73,11 @@ _SIGS = {
     "gated_mlp_static_fp8_workspace": (ctypes.c_size_t, [_I64, _I64, _I64]),
     "gated_mlp_static_fp8": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _P,
                                             _P, _P, _P]),
+    "fp8_gate_up_swiglu_static": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P,
+                                                 _P, _P]),
+    "gated_mlp_static_fp8_fused_workspace": (ctypes.c_size_t, [_I64, _I64, _I64]),
+    "gated_mlp_static_fp8_fused": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P,
+                                                  _P, _P, _P, _P, _P]),
     "gated_mlp_static_fp8_noalloc": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P,
                                                     _P, _P, _P, _P]),
     "qkv_shared_quant_workspace": (ctypes.c_size_t, [_I64, _I64]),
@@ -265,6 +272,64 @@ def gated_mlp_workspace_views(workspace: torch.Tensor, M: int, d: int, I: int):
     u = ws[o_u:o_u + M * I * 2].view(torch.bfloat16).view(M, I)
     h = ws[o_h:o_h + M * I].view(FP8).view(M, I)
     return dict(xq=xq, g=g, u=u, h=h)
+
+
+def fp8_gate_up_swiglu_static(xq, wg, wu, s_in, s_wg, s_wu, s_down, out=None,
+                              stream=None) -> torch.Tensor:
+    """H = E4M3(SiLU(bf16(G)) * bf16(U) / s_down) with G, U the gate and up
+    projections of xq [M,K] (Wg, Wu [I,K]), computed in one kernel."""
+    lib = load()
+    M, K = xq.shape
+    I = wg.shape[0]
+    if tuple(wg.shape) != (I, K) or tuple(wu.shape) != (I, K):
+        raise ValueError("Wg and Wu must both be [I, K]")
+    if out is None:
+        out = torch.empty((M, I), dtype=FP8, device=xq.device)
+    with _device_of(xq):
+        _check(lib.fp8_gate_up_swiglu_static(
+            _fp8(xq, "xq"), _fp8(wg, "wg"), _fp8(wu, "wu"), M, I, K, _f32(s_in, "s_in"),
+            _f32(s_wg, "s_wg"), _f32(s_wu, "s_wu"), _f32(s_down, "s_down"), _fp8(out, "out"),
+            _stream(stream)), "fp8_gate_up_swiglu_static")
+    return out
+
+
+def gated_mlp_static_fp8_fused_workspace(M: int, d: int, I: int) -> int:
+    return load().gated_mlp_static_fp8_fused_workspace(M, d, I)
+
+
+def gated_mlp_static_fp8_fused(x, s_in, wg, s_wg, wu, s_wu, s_down, wd, s_wd, workspace=None,
+                               out=None, stream=None) -> torch.Tensor:
+    """The gated MLP with gate/up and the SwiGLU-quant fused: quantize X, one
+    fused gate/up/SwiGLU kernel, the down GEMM.  Same result as
+    gated_mlp_static_fp8, bit for bit."""
+    lib = load()
+    if x.dim() != 2:
+        raise ValueError("x must be [M, d]")
+    M, d = x.shape
+    I = wg.shape[0]
+    if tuple(wg.shape) != (I, d) or tuple(wu.shape) != (I, d) or tuple(wd.shape) != (d, I):
+        raise ValueError("weight shapes must be Wg, Wu [I,d] and Wd [d,I]")
+    need = lib.gated_mlp_static_fp8_fused_workspace(M, d, I)
+    if workspace is None:
+        workspace = _workspace(need, x.device)
+    if workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace needs {need} bytes")
+    if out is None:
+        out = torch.empty((M, d), dtype=torch.bfloat16, device=x.device)
+    with _device_of(x):
+        _check(lib.gated_mlp_static_fp8_fused(
+            _bf16(x, "x"), M, d, I, _f32(s_in, "s_in"), _fp8(wg, "wg"), _f32(s_wg, "s_wg"),
+            _fp8(wu, "wu"), _f32(s_wu, "s_wu"), _f32(s_down, "s_down"), _fp8(wd, "wd"),
+            _f32(s_wd, "s_wd"), _dev_ptr(workspace, "workspace", (torch.uint8,)),
+            _bf16(out, "out"), _stream(stream)), "gated_mlp_static_fp8_fused")
+    return out
+
+
+def fused_workspace_views(workspace: torch.Tensor, M: int, d: int, I: int):
+    """Views of the regions gated_mlp_static_fp8_fused writes: Xq [M,d], H [M,I]."""
+    o_h = (M * d + 255) // 256 * 256
+    ws = workspace.view(torch.uint8)
+    return dict(xq=ws[:M * d].view(FP8).view(M, d), h=ws[o_h:o_h + M * I].view(FP8).view(M, I))
 
 
 def qkv_shared_quant_workspace(M: int, d: int) -> int:

@@ -17,6 +17,7 @@
 
 #include "common.cuh"
 #include "elementwise.cuh"
+#include "gemm_dual_sm100.cuh"
 #include "gemm_pair_sm100.cuh"
 #include "gemm_sm100.cuh"
 
@@ -44,7 +45,7 @@ void log_launch(int kind, const void *in0, const void *in1, const void *out) {
   ++g_launch_total;
 }
 
-enum { kKindQuant = 1, kKindGemm = 2, kKindSwiglu = 3, kKindCalib = 4 };
+enum { kKindQuant = 1, kKindGemm = 2, kKindSwiglu = 3, kKindCalib = 4, kKindDual = 5 };
 
 // --------------------------------------------------------------- device info
 struct DeviceInfo {
@@ -52,6 +53,7 @@ struct DeviceInfo {
   int sms = 0;
   unsigned gemm_attr_set = 0;  // bit per GEMM instantiation
   int pair_clusters = 0;       // CTA pairs of the pair GEMM resident at once
+  int dual_clusters = 0;       // CTA pairs of the gate/up dual GEMM resident at once
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -220,6 +222,51 @@ int launch_gemm_pair(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int M,
   return launch_status();
 }
 
+// Gate/up dual GEMM with the SwiGLU-quant epilogue, on CTA pairs.
+template <int STAGES, int BIT>
+int launch_dual_swiglu(DeviceInfo *d, const uint8_t *xq, const uint8_t *wg, const uint8_t *wu,
+                       int M, int N, int K, const float *s_in, const float *s_wg,
+                       const float *s_wu, const float *s_down, uint8_t *h, cudaStream_t st) {
+  using C = DualCfg<STAGES>;
+  auto kern = fp8_dual_swiglu_pair_kernel<STAGES>;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (!(d->gemm_attr_set & (1u << BIT))) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+        cudaSuccess)
+      return FP8WS_ERR_CUDA;
+    int clusters = 0;
+    cfg.gridDim = dim3(2 * (d->sms / 2));
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1)
+      return FP8WS_ERR_CUDA;
+    d->dual_clusters = clusters;
+    d->gemm_attr_set |= 1u << BIT;
+  }
+  CUtensorMap ma, mg, mu, mh;
+  int rc = make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, xq, M, K, kGemmBK, 128, true);
+  if (!rc) rc = make_map_2d(&mg, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, wg, N, K, kGemmBK, 64, true);
+  if (!rc) rc = make_map_2d(&mu, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, wu, N, K, kGemmBK, 64, true);
+  if (!rc) rc = make_map_2d(&mh, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h, M, N, 128, 32, false);
+  if (rc) return rc;
+  const int tiles = ((M + kDualTileM - 1) / kDualTileM) * ((N + kDualTileN - 1) / kDualTileN);
+  const int clusters = tiles < d->dual_clusters ? tiles : d->dual_clusters;
+  cfg.gridDim = dim3(2 * clusters);
+  if (cudaLaunchKernelEx(&cfg, kern, ma, mg, mu, mh, s_in, s_wg, s_wu, s_down, M, N, K,
+                         kWaitLimitNs) != cudaSuccess)
+    return FP8WS_ERR_CUDA;
+  log_launch(kKindDual, xq, wg, h);
+  return launch_status();
+}
+
 int check_gemm_args(const void *xq, const void *wq, int64_t M, int64_t N, int64_t K,
                     const float *s_in, const float *s_w, const void *y) {
   if (!wq || !s_in || !s_w || (M != 0 && (!xq || !y))) return FP8WS_ERR_NULL;
@@ -372,6 +419,61 @@ int qkv_shared_quant(const uint16_t *x, int64_t M, int64_t dm, const float *s_in
   if (!rc) rc = gemm_dispatch(d, xq, Wq, M, Nq, dm, s_in, s_wq, q, st);
   if (!rc) rc = gemm_dispatch(d, xq, Wk, M, Nk, dm, s_in, s_wk, k, st);
   if (!rc) rc = gemm_dispatch(d, xq, Wv, M, Nv, dm, s_in, s_wv, v, st);
+  return rc;
+}
+
+int fp8_gate_up_swiglu_static(const uint8_t *xq, const uint8_t *Wg, const uint8_t *Wu,
+                              int64_t M, int64_t I, int64_t K, const float *s_in,
+                              const float *s_wg, const float *s_wu, const float *s_down,
+                              uint8_t *h, void *stream) {
+  if (!s_down || !Wu || !s_wu) return FP8WS_ERR_NULL;
+  int rc = check_gemm_args(xq, Wg, M, I, K, s_in, s_wg, h);
+  if (rc) return rc;
+  if (I % 16 != 0) return FP8WS_ERR_SHAPE;  // FP8 rows of H must be 16-byte multiples
+  if (!aligned16(Wu)) return FP8WS_ERR_ALIGN;
+  DeviceInfo *d;
+  rc = device_info(&d);
+  if (rc) return rc;
+  if (M == 0) return FP8WS_OK;
+  return launch_dual_swiglu<6, 4>(d, xq, Wg, Wu, static_cast<int>(M), static_cast<int>(I),
+                                  static_cast<int>(K), s_in, s_wg, s_wu, s_down, h,
+                                  as_stream(stream));
+}
+
+size_t gated_mlp_static_fp8_fused_workspace(int64_t M, int64_t d, int64_t I) {
+  if (M < 0 || d < 0 || I < 0) return 0;
+  const size_t m = static_cast<size_t>(M);
+  return round256(m * static_cast<size_t>(d)) + round256(m * static_cast<size_t>(I));
+}
+
+int gated_mlp_static_fp8_fused(const uint16_t *x, int64_t M, int64_t dm, int64_t I,
+                               const float *s_in, const uint8_t *Wg, const float *s_wg,
+                               const uint8_t *Wu, const float *s_wu, const float *s_down,
+                               const uint8_t *Wd, const float *s_wd, void *workspace, uint16_t *y,
+                               void *stream) {
+  if (!s_in || !Wg || !s_wg || !Wu || !s_wu || !s_down || !Wd || !s_wd ||
+      (M != 0 && (!x || !y)))
+    return FP8WS_ERR_NULL;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FP8WS_ERR_WORKSPACE;
+  if (!aligned16(x) || !aligned16(Wu)) return FP8WS_ERR_ALIGN;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  const size_t m = static_cast<size_t>(M < 0 ? 0 : M);
+  uint8_t *xq = ws;
+  uint8_t *H = ws + round256(m * dm);
+  int rc = check_gemm_args(xq, Wg, M, I, dm, s_in, s_wg, H);
+  if (!rc) rc = check_gemm_args(H, Wd, M, dm, I, s_down, s_wd, y);
+  if (rc) return rc;
+  if (I % 16 != 0) return FP8WS_ERR_SHAPE;
+  DeviceInfo *d;
+  rc = device_info(&d);
+  if (rc) return rc;
+  if (M == 0) return FP8WS_OK;
+  cudaStream_t st = as_stream(stream);
+  rc = quant_launch(d, x, M * dm, s_in, xq, st);
+  if (!rc)
+    rc = launch_dual_swiglu<6, 4>(d, xq, Wg, Wu, static_cast<int>(M), static_cast<int>(I),
+                                  static_cast<int>(dm), s_in, s_wg, s_wu, s_down, H, st);
+  if (!rc) rc = gemm_dispatch(d, H, Wd, M, dm, I, s_down, s_wd, y, st);
   return rc;
 }
 

@@ -1,0 +1,276 @@
+// Gate/up dual FP8 GEMM with the two-input SwiGLU and the FP8 quantization of
+// its result in the epilogue, on CTA pairs (tcgen05 cta_group::2), sm_100a.
+//
+//   G = bf16((s_in*s_wg) * Xq . Wg^T),  U = bf16((s_in*s_wu) * Xq . Wu^T)
+//   H = E4M3_satRNE( SiLU(G) * U * (1/s_down) )            [M, I] FP8
+//
+// The BF16 rounding of G and U and the fp32 SwiGLU arithmetic are the very
+// operations of fp8_gemm_kernel's epilogue followed by silu_mul_2in_kernel, so
+// H is bit-identical to the unfused path, while G and U never leave the chip.
+//
+// A cluster of two CTAs computes a 256 x 128 tile of both G and U: each CTA
+// loads 128 rows of Xq and 64 rows each of Wg and Wu per 128-byte K step
+// (32 KB per SM), and the leader issues two M=256, N=128 tcgen05.mma per K
+// slice, one into the G accumulator and one into the U accumulator.  TMEM per
+// CTA holds two buffers of (G 128 columns | U 128 columns), so the epilogue of
+// a tile overlaps the main loop of the next.  Epilogue warps read 32 columns of
+// G and of U per step, write 32 FP8 codes of each row into a 128-byte swizzled
+// row and TMA-store 32 x 128-byte boxes.  Roles, bounded waits and teardown
+// follow fp8_gemm_pair_kernel.
+#pragma once
+
+#include "common.cuh"
+#include "elementwise.cuh"
+#include "gemm_pair_sm100.cuh"
+
+namespace fp8ws {
+
+constexpr int kDualTileM = 256;  // rows per CTA pair
+constexpr int kDualTileN = 128;  // columns of G and of U per tile
+
+template <int STAGES_>
+struct DualCfg {
+  static constexpr int STAGES = STAGES_;
+  static constexpr int A_BYTES = 128 * kGemmBK;   // this CTA's 128 rows of Xq
+  static constexpr int BH_BYTES = 64 * kGemmBK;   // this CTA's 64 rows of Wg (or Wu)
+  static constexpr int STAGE_BYTES = A_BYTES + 2 * BH_BYTES;
+  static constexpr int TX_BYTES = 2 * STAGE_BYTES;
+  static constexpr int EPI_BUF_BYTES = 32 * 128;   // 32 rows x 128 FP8 codes
+  static constexpr int EPI_BYTES = 4 * 2 * EPI_BUF_BYTES;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
+  static constexpr uint32_t ACC_COLS = 2 * kDualTileN;  // G | U
+  static constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;   // two buffers
+  static_assert((2 * STAGES + 5) * 8 + 8 <= BAR_BYTES, "barrier area");
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+  static_assert(TMEM_COLS == 512, "tmem");
+};
+
+template <int STAGES>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    fp8_dual_swiglu_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
+                                const __grid_constant__ CUtensorMap tm_bg,
+                                const __grid_constant__ CUtensorMap tm_bu,
+                                const __grid_constant__ CUtensorMap tm_h,
+                                const float *__restrict__ s_in, const float *__restrict__ s_wg,
+                                const float *__restrict__ s_wu,
+                                const float *__restrict__ s_down, int M, int N, int K,
+                                uint64_t timeout_ns) {
+  using C = DualCfg<STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sA = smem;
+  uint8_t *sBg = smem + STAGES * C::A_BYTES;
+  uint8_t *sBu = sBg + STAGES * C::BH_BYTES;
+  uint8_t *sEpi = sBu + STAGES * C::BH_BYTES;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sEpi + C::EPI_BYTES);
+  uint64_t *full = bars;
+  uint64_t *empty = bars + STAGES;
+  uint64_t *tfull = bars + 2 * STAGES;
+  uint64_t *tempty = tfull + 2;
+  uint64_t *drain = tempty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cluster = blockIdx.x >> 1;
+  const int nclusters = gridDim.x >> 1;
+  const int num_m = (M + kDualTileM - 1) / kDualTileM;
+  const int num_n = (N + kDualTileN - 1) / kDualTileN;
+  const int num_tiles = num_m * num_n;
+  const int num_kb = (K + kGemmBK - 1) / kGemmBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 8);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_bg);
+    tma_prefetch_desc(&tm_bu);
+    tma_prefetch_desc(&tm_h);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      uint32_t issued_mask = 0, issued_parity = 0;
+      bool ok = true;
+      for (int t = cluster; t < num_tiles && ok; t += nclusters) {
+        const TileCoord tc = tile_coord(t, num_m, num_n);
+        const int a_row = tc.m * kDualTileM + static_cast<int>(rank) * 128;
+        const int b_row = tc.n * kDualTileN + static_cast<int>(rank) * 64;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, timeout_ns)) {
+            record_timeout(kSiteProducerEmpty);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          const uint32_t full_leader = map_shared_rank(smem_u32(&full[stage]), 0);
+          if (leader) mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
+          tma_load_2d_pair(sA + stage * C::A_BYTES, &tm_a, full_leader, kb * kGemmBK, a_row);
+          tma_load_2d_pair(sBg + stage * C::BH_BYTES, &tm_bg, full_leader, kb * kGemmBK, b_row);
+          tma_load_2d_pair(sBu + stage * C::BH_BYTES, &tm_bu, full_leader, kb * kGemmBK, b_row);
+          issued_mask |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok && leader) {
+        int zero = 0;
+        for (int s = 0; s < STAGES; ++s)
+          if (issued_mask & (1u << s))
+            mbar_wait_bounded(&full[s], (issued_parity >> s) & 1u, &zero, timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------- MMA issue (leader)
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(kDualTileM, kDualTileN);
+      uint32_t stage = 0, phase = 0;
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = cluster; t < num_tiles && ok; t += nclusters, ++it) {
+        const uint32_t acc = it & 1u;
+        const uint32_t acc_phase = (it >> 1) & 1u;
+        if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, timeout_ns)) {
+          record_timeout(kSiteMmaTmemEmpty);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_g = tmem_base + acc * C::ACC_COLS;
+        const uint32_t d_u = d_g + kDualTileN;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, timeout_ns)) {
+            record_timeout(kSiteMmaFull);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * C::A_BYTES);
+          const uint32_t g_addr = smem_u32(sBg + stage * C::BH_BYTES);
+          const uint32_t u_addr = smem_u32(sBu + stage * C::BH_BYTES);
+#pragma unroll
+          for (int k = 0; k < kGemmBK / 32; ++k) {
+            const uint64_t da = smem_desc_k_sw128(a_addr + k * 32);
+            const uint32_t accum = (kb | k) != 0 ? 1u : 0u;
+            umma_f8_pair(d_g, da, smem_desc_k_sw128(g_addr + k * 32), idesc, accum);
+            umma_f8_pair(d_u, da, smem_desc_k_sw128(u_addr + k * 32), idesc, accum);
+          }
+          umma_commit_pair(&empty[stage], 0x3);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) umma_commit_pair(&tfull[acc], 0x3);
+      }
+      umma_commit_pair(drain, 0x1);
+      int zero = 0;
+      if (!mbar_wait_bounded(drain, 0, &zero, timeout_ns)) record_timeout(kSiteDrain);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ epilogue (both CTAs)
+    const int ew = warp - 2;
+    const int quarter = warp & 3;
+    const float scale_g = __ldg(s_in) * __ldg(s_wg);
+    const float scale_u = __ldg(s_in) * __ldg(s_wu);
+    const float inv_s = __frcp_rn(__ldg(s_down));
+    uint32_t it = 0;
+    for (int t = cluster; t < num_tiles; t += nclusters, ++it) {
+      const TileCoord tc = tile_coord(t, num_m, num_n);
+      const uint32_t acc = it & 1u;
+      const uint32_t acc_phase = (it >> 1) & 1u;
+      if (!mbar_wait_bounded_warp(&tfull[acc], acc_phase, abort_flag, timeout_ns)) {
+        if (lane == 0) {
+          record_timeout(kSiteEpiTmemFull);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      tc_fence_after();
+      const int row0 = tc.m * kDualTileM + static_cast<int>(rank) * 128 + quarter * 32;
+      const int col0 = tc.n * kDualTileN;
+      const bool store = row0 < M && col0 < N;
+      const uint32_t t_g =
+          tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * C::ACC_COLS;
+      uint8_t *buf = sEpi + (ew * 2 + (it & 1u)) * C::EPI_BUF_BYTES;
+      if (lane == 0) tma_store_wait_read<1>();  // this buffer's previous store has read it
+      __syncwarp();
+      uint8_t *row = buf + lane * 128;
+#pragma unroll 1
+      for (int c = 0; c < kDualTileN / 32; ++c) {
+        uint32_t g[32], u[32];
+        tmem_ld_32x32b_x32(t_g + c * 32, g);
+        tmem_ld_32x32b_x32(t_g + kDualTileN + c * 32, u);
+        tmem_ld_wait();
+        if (c == kDualTileN / 32 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(map_shared_rank(smem_u32(&tempty[acc]), 0));
+        }
+        uint32_t q[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float h[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float gv = __bfloat162float(__float2bfloat16_rn(__uint_as_float(g[4 * j + e]) * scale_g));
+            const float uv = __bfloat162float(__float2bfloat16_rn(__uint_as_float(u[4 * j + e]) * scale_u));
+            h[e] = silu_mul(gv, uv) * inv_s;
+          }
+          q[j] = pack4(cvt_e4m3x2(h[0], h[1]), cvt_e4m3x2(h[2], h[3]));
+        }
+        // 32 codes = two 16-byte units (2c, 2c+1) of this row, swizzled
+        *reinterpret_cast<uint4 *>(row + (((2 * c) ^ (lane & 7)) << 4)) =
+            make_uint4(q[0], q[1], q[2], q[3]);
+        *reinterpret_cast<uint4 *>(row + (((2 * c + 1) ^ (lane & 7)) << 4)) =
+            make_uint4(q[4], q[5], q[6], q[7]);
+      }
+      fence_async_shared();
+      __syncwarp();
+      if (lane == 0 && store) {
+        tma_store_2d(&tm_h, buf, col0, row0);
+      }
+      if (lane == 0) tma_store_commit();
+    }
+    if (lane == 0) tma_store_wait_all<0>();
+  }
+
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace fp8ws

@@ -142,6 +142,42 @@ FP8WS_API int gated_mlp_static_fp8(const uint16_t *x, int64_t M, int64_t d, int6
                          const float *s_wd, void *workspace, uint16_t *y, void *stream);
 
 /*
+ * fp8_gate_up_swiglu_static -- gate and up projections and the two-input
+ * SwiGLU-quant in one kernel (the fusion of fp8_linear_static x 2 and
+ * silu_mul_2in_fp8 on the MLP path; [PR] What changed describes the three
+ * steps, this call runs them without writing G and U to memory).
+ *
+ *   G = bf16((s_in*s_wg) . Xq Wg^T),  U = bf16((s_in*s_wu) . Xq Wu^T)   (kept on chip)
+ *   h = E4M3_satRNE( SiLU(G) * U / s_down )   in fp32 as silu_mul_2in_fp8
+ *
+ * Bit-identical to fp8_linear_static (gate), fp8_linear_static (up) and
+ * silu_mul_2in_fp8 run one after the other on the same inputs.
+ * xq: device [M,K] FP8.  Wg, Wu: device [I,K] FP8.  Scales: device fp32.
+ * h: device [M,I] FP8.  Sizes: as fp8_linear_static with N = I, and I % 16 == 0.
+ */
+FP8WS_API int fp8_gate_up_swiglu_static(const uint8_t *xq, const uint8_t *Wg, const uint8_t *Wu,
+                                        int64_t M, int64_t I, int64_t K, const float *s_in,
+                                        const float *s_wg, const float *s_wu,
+                                        const float *s_down, uint8_t *h, void *stream);
+
+/*
+ * gated_mlp_static_fp8_fused -- gated_mlp_static_fp8 with the gate/up GEMMs
+ * and the SwiGLU-quant fused (fp8_gate_up_swiglu_static): three launches
+ * (quantize X, fused gate/up/SwiGLU, down GEMM) instead of five, and no G or U
+ * round trip through memory.  Same result, bit for bit.
+ * workspace: device, gated_mlp_static_fp8_fused_workspace(M,d,I) bytes,
+ * 256-byte aligned; holds Xq [M,d] then H [M,I] (each region 256-byte
+ * aligned).  Other arguments as gated_mlp_static_fp8.
+ */
+FP8WS_API size_t gated_mlp_static_fp8_fused_workspace(int64_t M, int64_t d, int64_t I);
+FP8WS_API int gated_mlp_static_fp8_fused(const uint16_t *x, int64_t M, int64_t d, int64_t I,
+                                         const float *s_in, const uint8_t *Wg, const float *s_wg,
+                                         const uint8_t *Wu, const float *s_wu,
+                                         const float *s_down, const uint8_t *Wd,
+                                         const float *s_wd, void *workspace, uint16_t *y,
+                                         void *stream);
+
+/*
  * qkv_shared_quant -- Q/K/V projections from one shared quantization.
  * [PR] What changed (Attention with shared Q/K/V input quantization: the
  * activation is quantized once for all three projections; each projection
@@ -251,7 +287,7 @@ FP8WS_API int fp8ws_device_status(int *status, int *where);
 
 /* Launch log.  Every kernel the library enqueues is counted and recorded in a
  * small ring (the most recent FP8WS_LOG_CAPACITY launches).  kind: 1 quant,
- * 2 GEMM, 3 SwiGLU-quant, 4 calibration.  in0/in1 are the primary input
+ * 2 GEMM, 3 SwiGLU-quant, 4 calibration, 5 fused gate/up SwiGLU-quant.  in0/in1 are the primary input
  * pointers (for a GEMM: activation and weight), out the output pointer. */
 #define FP8WS_LOG_CAPACITY 64
 typedef struct {
