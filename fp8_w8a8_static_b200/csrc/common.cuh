@@ -330,3 +330,20 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t *bar, uint16_t cta_mas
 }
 
 }  // namespace fp8ws
+
+// ------------------------------------------- programmatic dependent launch
+namespace fp8ws {
+
+// Let the next kernel on the stream be scheduled now; it still waits in
+// pdl_wait() until this grid has finished and its writes are visible.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Block until the previous kernel on the stream has completed and its memory
+// operations are visible (returns at once when launched without the
+// programmatic-serialization attribute).  Every kernel here calls it before
+// its first global-memory access, so stream order is preserved exactly.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+}  // namespace fp8ws

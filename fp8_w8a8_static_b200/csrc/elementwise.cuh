@@ -33,20 +33,43 @@ __device__ __forceinline__ uint4 ld_stream(const uint4 *p) { return __ldcs(p); }
 __device__ __forceinline__ void st_stream(uint2 *p, uint2 v) { __stcs(p, v); }
 
 // ------------------------------------------------------------- quantize
-// q = E4M3_satRNE(x / s) with IEEE fp32 division.
-__device__ __forceinline__ uint2 quant8(uint4 v, float s) {
+// q = E4M3_satRNE(fl32(x / s)), the code of the IEEE fp32 quotient.
+//
+// The code only depends on which E4M3 rounding interval fl32(x / s) falls in.
+// With r = fl32(1/s), t = fl32(x * r) = (x/s)(1 + d) with |d| <= 2^-23 + 2^-48,
+// and fl32(x/s) = (x/s)(1 + e) with |e| <= 2^-24, so the two differ by less
+// than 3 ulp of t (an ulp is at least 2^-24 |t|).  Rounding to E4M3 is
+// monotone, so when the floats 4 ulp below and above t (adjacent bit
+// patterns, across a binade boundary too) give the same code, that is the
+// code of the quotient.  Otherwise (t near an E4M3 rounding boundary, near
+// zero, or not finite) the quotient is computed with IEEE division.
+__device__ __forceinline__ uint32_t quant1(float x, float s, float r) {
+  const float t = x * r;
+  const uint32_t b = __float_as_uint(t);
+  const uint32_t lohi = cvt_e4m3x2(__uint_as_float(b - 4u), __uint_as_float(b + 4u));
+  if ((lohi & 0xFFu) == (lohi >> 8)) return lohi & 0xFFu;
+  return cvt_e4m3x2(__fdiv_rn(x, s), 0.0f) & 0xFFu;
+}
+
+__device__ __forceinline__ uint32_t quant4(uint32_t w0, uint32_t w1, float s, float r) {
+  return quant1(bf16_lo(w0), s, r) | (quant1(bf16_hi(w0), s, r) << 8) |
+         (quant1(bf16_lo(w1), s, r) << 16) | (quant1(bf16_hi(w1), s, r) << 24);
+}
+
+__device__ __forceinline__ uint2 quant8(uint4 v, float s, float r) {
   uint2 o;
-  o.x = pack4(cvt_e4m3x2(__fdiv_rn(bf16_lo(v.x), s), __fdiv_rn(bf16_hi(v.x), s)),
-              cvt_e4m3x2(__fdiv_rn(bf16_lo(v.y), s), __fdiv_rn(bf16_hi(v.y), s)));
-  o.y = pack4(cvt_e4m3x2(__fdiv_rn(bf16_lo(v.z), s), __fdiv_rn(bf16_hi(v.z), s)),
-              cvt_e4m3x2(__fdiv_rn(bf16_lo(v.w), s), __fdiv_rn(bf16_hi(v.w), s)));
+  o.x = quant4(v.x, v.y, s, r);
+  o.y = quant4(v.z, v.w, s, r);
   return o;
 }
 
 __global__ void __launch_bounds__(kEwThreads) quant_static_kernel(
     const uint16_t *__restrict__ x, int64_t numel, const float *__restrict__ s_in,
     uint8_t *__restrict__ xq) {
+  pdl_launch_dependents();
+  pdl_wait();
   const float s = __ldg(s_in);
+  const float r = __frcp_rn(s);
   const int64_t nvec = numel >> 3;
   const uint4 *xv = reinterpret_cast<const uint4 *>(x);
   uint2 *qv = reinterpret_cast<uint2 *>(xq);
@@ -58,13 +81,13 @@ __global__ void __launch_bounds__(kEwThreads) quant_static_kernel(
 #pragma unroll
     for (int u = 0; u < kEwUnroll; ++u) v[u] = ld_stream(xv + i + u * stride);
 #pragma unroll
-    for (int u = 0; u < kEwUnroll; ++u) st_stream(qv + i + u * stride, quant8(v[u], s));
+    for (int u = 0; u < kEwUnroll; ++u) st_stream(qv + i + u * stride, quant8(v[u], s, r));
   }
-  for (; i < nvec; i += stride) st_stream(qv + i, quant8(ld_stream(xv + i), s));
+  for (; i < nvec; i += stride) st_stream(qv + i, quant8(ld_stream(xv + i), s, r));
   const int64_t t = (nvec << 3) + tid;
   if (t < numel) {
     float a = __uint_as_float(static_cast<uint32_t>(x[t]) << 16);
-    xq[t] = static_cast<uint8_t>(cvt_e4m3x2(__fdiv_rn(a, s), 0.0f) & 0xFFu);
+    xq[t] = static_cast<uint8_t>(quant1(a, s, r));
   }
 }
 
@@ -90,6 +113,8 @@ __device__ __forceinline__ uint2 silu_mul_quant8(uint4 g, uint4 u, float inv_s) 
 __global__ void __launch_bounds__(kEwThreads) silu_mul_2in_kernel(
     const uint16_t *__restrict__ g, const uint16_t *__restrict__ u, int64_t numel,
     const float *__restrict__ s_down, uint8_t *__restrict__ h) {
+  pdl_launch_dependents();
+  pdl_wait();
   const float inv_s = __frcp_rn(__ldg(s_down));
   const int64_t nvec = numel >> 3;
   const uint4 *gv = reinterpret_cast<const uint4 *>(g);

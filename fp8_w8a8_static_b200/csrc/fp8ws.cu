@@ -11,6 +11,7 @@
 
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
@@ -115,6 +116,45 @@ int ew_grid(const DeviceInfo *d, Kernel kern, int64_t nvec) {
   return static_cast<int>(want);
 }
 
+// Kernels are launched with programmatic stream serialization: the next
+// kernel on the stream may be scheduled while this one finishes, and waits in
+// griddepcontrol.wait before touching memory.  FP8WS_PDL=0 turns it off.
+bool use_pdl() {
+  static int v = -1;
+  if (v < 0) {
+    const char *e = getenv("FP8WS_PDL");
+    v = (e && e[0] == '0') ? 0 : 1;
+  }
+  return v == 1;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                      int cluster_x, Args... args) {
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (use_pdl()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // ------------------------------------------------------------- tensor maps
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
@@ -171,7 +211,9 @@ int launch_gemm_cfg(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int M, 
   if (rc) return rc;
   const int tiles = ((M + kGemmBM - 1) / kGemmBM) * ((N + BN - 1) / BN);
   const int grid = tiles < d->sms ? tiles : d->sms;
-  kern<<<grid, kGemmThreads, C::SMEM_BYTES, st>>>(ma, mb, md, s_in, s_w, M, N, K, kWaitLimitNs);
+  if (launch_ex(kern, dim3(grid), dim3(kGemmThreads), C::SMEM_BYTES, st, 1, ma, mb, md, s_in, s_w,
+                M, N, K, kWaitLimitNs) != cudaSuccess)
+    return FP8WS_ERR_CUDA;
   log_launch(kKindGemm, xq, wq, y);
   return launch_status();
 }
@@ -215,8 +257,8 @@ int launch_gemm_pair(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int M,
   if (rc) return rc;
   const int tiles = ((M + kPairTile - 1) / kPairTile) * ((N + kPairTile - 1) / kPairTile);
   const int clusters = tiles < d->pair_clusters ? tiles : d->pair_clusters;
-  cfg.gridDim = dim3(2 * clusters);
-  if (cudaLaunchKernelEx(&cfg, kern, ma, mb, md, s_in, s_w, M, N, K, kWaitLimitNs) != cudaSuccess)
+  if (launch_ex(kern, dim3(2 * clusters), dim3(kGemmThreads), C::SMEM_BYTES, st, 2, ma, mb, md,
+                s_in, s_w, M, N, K, kWaitLimitNs) != cudaSuccess)
     return FP8WS_ERR_CUDA;
   log_launch(kKindGemm, xq, wq, y);
   return launch_status();
@@ -253,15 +295,14 @@ int launch_dual_swiglu(DeviceInfo *d, const uint8_t *xq, const uint8_t *wg, cons
   }
   CUtensorMap ma, mg, mu, mh;
   int rc = make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, xq, M, K, kGemmBK, 128, true);
-  if (!rc) rc = make_map_2d(&mg, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, wg, N, K, kGemmBK, 64, true);
-  if (!rc) rc = make_map_2d(&mu, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, wu, N, K, kGemmBK, 64, true);
+  if (!rc) rc = make_map_2d(&mg, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, wg, N, K, kGemmBK, 128, true);
+  if (!rc) rc = make_map_2d(&mu, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, wu, N, K, kGemmBK, 128, true);
   if (!rc) rc = make_map_2d(&mh, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h, M, N, 128, 32, false);
   if (rc) return rc;
   const int tiles = ((M + kDualTileM - 1) / kDualTileM) * ((N + kDualTileN - 1) / kDualTileN);
   const int clusters = tiles < d->dual_clusters ? tiles : d->dual_clusters;
-  cfg.gridDim = dim3(2 * clusters);
-  if (cudaLaunchKernelEx(&cfg, kern, ma, mg, mu, mh, s_in, s_wg, s_wu, s_down, M, N, K,
-                         kWaitLimitNs) != cudaSuccess)
+  if (launch_ex(kern, dim3(2 * clusters), dim3(kGemmThreads), C::SMEM_BYTES, st, 2, ma, mg, mu, mh,
+                s_in, s_wg, s_wu, s_down, M, N, K, kWaitLimitNs) != cudaSuccess)
     return FP8WS_ERR_CUDA;
   log_launch(kKindDual, xq, wg, h);
   return launch_status();
@@ -298,7 +339,9 @@ int gemm_dispatch(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int64_t M
 int quant_launch(DeviceInfo *d, const uint16_t *x, int64_t numel, const float *s, uint8_t *xq,
                  cudaStream_t st) {
   if (numel == 0) return FP8WS_OK;
-  quant_static_kernel<<<ew_grid(d, quant_static_kernel, numel >> 3), kEwThreads, 0, st>>>(x, numel, s, xq);
+  if (launch_ex(quant_static_kernel, dim3(ew_grid(d, quant_static_kernel, numel >> 3)),
+                dim3(kEwThreads), 0, st, 1, x, numel, s, xq) != cudaSuccess)
+    return FP8WS_ERR_CUDA;
   log_launch(kKindQuant, x, nullptr, xq);
   return launch_status();
 }
@@ -306,7 +349,9 @@ int quant_launch(DeviceInfo *d, const uint16_t *x, int64_t numel, const float *s
 int silu_launch(DeviceInfo *d, const uint16_t *g, const uint16_t *u, int64_t numel,
                 const float *s, uint8_t *h, cudaStream_t st) {
   if (numel == 0) return FP8WS_OK;
-  silu_mul_2in_kernel<<<ew_grid(d, silu_mul_2in_kernel, numel >> 3), kEwThreads, 0, st>>>(g, u, numel, s, h);
+  if (launch_ex(silu_mul_2in_kernel, dim3(ew_grid(d, silu_mul_2in_kernel, numel >> 3)),
+                dim3(kEwThreads), 0, st, 1, g, u, numel, s, h) != cudaSuccess)
+    return FP8WS_ERR_CUDA;
   log_launch(kKindSwiglu, g, u, h);
   return launch_status();
 }

@@ -8,12 +8,14 @@
 // operations of fp8_gemm_kernel's epilogue followed by silu_mul_2in_kernel, so
 // H is bit-identical to the unfused path, while G and U never leave the chip.
 //
-// A cluster of two CTAs computes a 256 x 128 tile of both G and U: each CTA
-// loads 128 rows of Xq and 64 rows each of Wg and Wu per 128-byte K step
-// (32 KB per SM), and the leader issues two M=256, N=128 tcgen05.mma per K
-// slice, one into the G accumulator and one into the U accumulator.  TMEM per
-// CTA holds two buffers of (G 128 columns | U 128 columns), so the epilogue of
-// a tile overlaps the main loop of the next.  Epilogue warps read 32 columns of
+// A cluster of two CTAs computes a 256 x 128 tile of both G and U with one
+// M=256, N=256 tcgen05.mma per K slice: the B operand's 256 rows are 128 rows
+// of Wg held by the leader CTA and the same 128 rows of Wu held by the peer, so
+// accumulator columns 0..127 are G and 128..255 are U.  Each CTA loads 128
+// rows of Xq and 128 rows of its weight per 128-byte K step (32 KB per SM, the
+// same operand traffic per flop as the plain CTA-pair GEMM).  TMEM per CTA
+// holds two buffers of (G 128 columns | U 128 columns), so the epilogue of a
+// tile overlaps the main loop of the next.  Epilogue warps read 32 columns of
 // G and of U per step, write 32 FP8 codes of each row into a 128-byte swizzled
 // row and TMA-store 32 x 128-byte boxes.  Roles, bounded waits and teardown
 // follow fp8_gemm_pair_kernel.
@@ -32,8 +34,8 @@ template <int STAGES_>
 struct DualCfg {
   static constexpr int STAGES = STAGES_;
   static constexpr int A_BYTES = 128 * kGemmBK;   // this CTA's 128 rows of Xq
-  static constexpr int BH_BYTES = 64 * kGemmBK;   // this CTA's 64 rows of Wg (or Wu)
-  static constexpr int STAGE_BYTES = A_BYTES + 2 * BH_BYTES;
+  static constexpr int B_BYTES = 128 * kGemmBK;   // 128 rows of Wg (leader) or Wu (peer)
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TX_BYTES = 2 * STAGE_BYTES;
   static constexpr int EPI_BUF_BYTES = 32 * 128;   // 32 rows x 128 FP8 codes
   static constexpr int EPI_BYTES = 4 * 2 * EPI_BUF_BYTES;
@@ -61,9 +63,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t *sA = smem;
-  uint8_t *sBg = smem + STAGES * C::A_BYTES;
-  uint8_t *sBu = sBg + STAGES * C::BH_BYTES;
-  uint8_t *sEpi = sBu + STAGES * C::BH_BYTES;
+  uint8_t *sB = smem + STAGES * C::A_BYTES;
+  uint8_t *sEpi = sB + STAGES * C::B_BYTES;
   uint64_t *bars = reinterpret_cast<uint64_t *>(sEpi + C::EPI_BYTES);
   uint64_t *full = bars;
   uint64_t *empty = bars + STAGES;
@@ -105,6 +106,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
     tmem_relinquish_pair();
   }
+  pdl_launch_dependents();
+  pdl_wait();  // the previous kernel's outputs (our inputs) are complete from here on
   tc_fence_before();
   cluster_sync();
   tc_fence_after();
@@ -119,7 +122,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int t = cluster; t < num_tiles && ok; t += nclusters) {
         const TileCoord tc = tile_coord(t, num_m, num_n);
         const int a_row = tc.m * kDualTileM + static_cast<int>(rank) * 128;
-        const int b_row = tc.n * kDualTileN + static_cast<int>(rank) * 64;
+        const int b_row = tc.n * kDualTileN;
+        const CUtensorMap *tm_b = leader ? &tm_bg : &tm_bu;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, timeout_ns)) {
             record_timeout(kSiteProducerEmpty);
@@ -130,8 +134,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t full_leader = map_shared_rank(smem_u32(&full[stage]), 0);
           if (leader) mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
           tma_load_2d_pair(sA + stage * C::A_BYTES, &tm_a, full_leader, kb * kGemmBK, a_row);
-          tma_load_2d_pair(sBg + stage * C::BH_BYTES, &tm_bg, full_leader, kb * kGemmBK, b_row);
-          tma_load_2d_pair(sBu + stage * C::BH_BYTES, &tm_bu, full_leader, kb * kGemmBK, b_row);
+          tma_load_2d_pair(sB + stage * C::B_BYTES, tm_b, full_leader, kb * kGemmBK, b_row);
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -151,7 +154,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------- MMA issue (leader)
     if (lane == 0 && leader) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(kDualTileM, kDualTileN);
+      constexpr uint32_t idesc = idesc_e4m3_f32(kDualTileM, 2 * kDualTileN);
       uint32_t stage = 0, phase = 0;
       uint32_t it = 0;
       bool ok = true;
@@ -164,8 +167,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t d_g = tmem_base + acc * C::ACC_COLS;
-        const uint32_t d_u = d_g + kDualTileN;
+        const uint32_t d_gu = tmem_base + acc * C::ACC_COLS;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait_bounded(&full[stage], phase, abort_flag, timeout_ns)) {
             record_timeout(kSiteMmaFull);
@@ -175,14 +177,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(sA + stage * C::A_BYTES);
-          const uint32_t g_addr = smem_u32(sBg + stage * C::BH_BYTES);
-          const uint32_t u_addr = smem_u32(sBu + stage * C::BH_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * C::B_BYTES);
 #pragma unroll
           for (int k = 0; k < kGemmBK / 32; ++k) {
-            const uint64_t da = smem_desc_k_sw128(a_addr + k * 32);
-            const uint32_t accum = (kb | k) != 0 ? 1u : 0u;
-            umma_f8_pair(d_g, da, smem_desc_k_sw128(g_addr + k * 32), idesc, accum);
-            umma_f8_pair(d_u, da, smem_desc_k_sw128(u_addr + k * 32), idesc, accum);
+            umma_f8_pair(d_gu, smem_desc_k_sw128(a_addr + k * 32),
+                         smem_desc_k_sw128(b_addr + k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
           }
           umma_commit_pair(&empty[stage], 0x3);
           if (++stage == STAGES) {

@@ -95,6 +95,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
     tmem_relinquish_pair();
   }
+  pdl_launch_dependents();
+  pdl_wait();  // the previous kernel's outputs (our inputs) are complete from here on
   tc_fence_before();
   cluster_sync();
   tc_fence_after();

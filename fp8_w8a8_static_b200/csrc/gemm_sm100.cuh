@@ -109,6 +109,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
+  pdl_launch_dependents();
+  pdl_wait();  // the previous kernel's outputs (our inputs) are complete from here on
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
