@@ -93,6 +93,7 @@ _SIGS = {
     "fp8ws_device_check": (ctypes.c_int, []),
     "fp8ws_device_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int),
                                            ctypes.POINTER(ctypes.c_int)]),
+    "fp8ws_set_gemm_config": (ctypes.c_int, [ctypes.c_int]),
     "fp8ws_launch_count": (ctypes.c_int64, []),
     "fp8ws_launch_log": (ctypes.c_int, [ctypes.POINTER(LaunchRecord), ctypes.c_int]),
     "fp8ws_launch_log_clear": (None, []),
@@ -431,6 +432,14 @@ def device_status():
     st, wh = ctypes.c_int(0), ctypes.c_int(0)
     _check(load().fp8ws_device_status(ctypes.byref(st), ctypes.byref(wh)), "fp8ws_device_status")
     return st.value, wh.value
+
+
+GEMM_CONFIGS = {"auto": 0, "pair256": 1, "cta256": 2, "cta128": 3, "cta64": 4}
+
+
+def set_gemm_config(name: str = "auto") -> None:
+    """Force a GEMM tile configuration (see GEMM_CONFIGS); "auto" = cost model."""
+    _check(load().fp8ws_set_gemm_config(GEMM_CONFIGS[name]), "fp8ws_set_gemm_config")
 
 
 def launch_count() -> int:

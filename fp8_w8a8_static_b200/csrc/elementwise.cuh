@@ -51,9 +51,20 @@ __device__ __forceinline__ uint32_t quant1(float x, float s, float r) {
   return cvt_e4m3x2(__fdiv_rn(x, s), 0.0f) & 0xFFu;
 }
 
+// The same test for the two BF16 values of one 32-bit word at once: one
+// conversion of the pair 4 ulp below, one 4 ulp above; if the two code pairs
+// agree they are the codes of both quotients.
+__device__ __forceinline__ uint32_t quant2(uint32_t w, float s, float r) {
+  const float a = bf16_lo(w), c = bf16_hi(w);
+  const uint32_t ba = __float_as_uint(a * r), bc = __float_as_uint(c * r);
+  const uint32_t lo = cvt_e4m3x2(__uint_as_float(ba - 4u), __uint_as_float(bc - 4u));
+  const uint32_t hi = cvt_e4m3x2(__uint_as_float(ba + 4u), __uint_as_float(bc + 4u));
+  if (lo == hi) return lo;
+  return cvt_e4m3x2(__fdiv_rn(a, s), __fdiv_rn(c, s));
+}
+
 __device__ __forceinline__ uint32_t quant4(uint32_t w0, uint32_t w1, float s, float r) {
-  return quant1(bf16_lo(w0), s, r) | (quant1(bf16_hi(w0), s, r) << 8) |
-         (quant1(bf16_lo(w1), s, r) << 16) | (quant1(bf16_hi(w1), s, r) << 24);
+  return pack4(quant2(w0, s, r), quant2(w1, s, r));
 }
 
 __device__ __forceinline__ uint2 quant8(uint4 v, float s, float r) {

@@ -318,20 +318,35 @@ int check_gemm_args(const void *xq, const void *wq, int64_t M, int64_t N, int64_
   return FP8WS_OK;
 }
 
-// Tile shape: CTA-pair 256 x 256 tiles when there is at least one per TPC;
-// otherwise one CTA per tile with the widest of 256/128/64 columns that still
-// gives every SM a tile (narrower only when the problem is too small).
+// Tile shape from a cost model: time ~ waves x (output area per SM per tile)
+// / efficiency, where waves = ceil(tiles / tiles resident at once).  The
+// efficiencies are the measured throughput of each configuration on large
+// problems relative to the CTA-pair kernel: narrower one-CTA tiles move more
+// operand bytes per tensor cycle and become L2-bandwidth bound.
+int g_forced_gemm_config = 0;  // fp8ws_set_gemm_config: 0 = cost model
+
 int gemm_dispatch(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int64_t M, int64_t N,
                   int64_t K, const float *s_in, const float *s_w, uint16_t *y, cudaStream_t st) {
   if (M == 0) return FP8WS_OK;
-  const int64_t num_m = (M + kGemmBM - 1) / kGemmBM;
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
-  if (((M + 255) / 256) * ((N + 255) / 256) >= d->sms / 2)
-    return launch_gemm_pair<6, 3>(d, xq, wq, m, n, k, s_in, s_w, y, st);
-  if (num_m * ((N + 255) / 256) >= d->sms)
-    return launch_gemm_cfg<256, 4, 0>(d, xq, wq, m, n, k, s_in, s_w, y, st);
-  if (num_m * ((N + 127) / 128) >= d->sms)
-    return launch_gemm_cfg<128, 6, 1>(d, xq, wq, m, n, k, s_in, s_w, y, st);
+  switch (g_forced_gemm_config) {
+    case 1: return launch_gemm_pair<6, 3>(d, xq, wq, m, n, k, s_in, s_w, y, st);
+    case 2: return launch_gemm_cfg<256, 4, 0>(d, xq, wq, m, n, k, s_in, s_w, y, st);
+    case 3: return launch_gemm_cfg<128, 6, 1>(d, xq, wq, m, n, k, s_in, s_w, y, st);
+    case 4: return launch_gemm_cfg<64, 8, 2>(d, xq, wq, m, n, k, s_in, s_w, y, st);
+    default: break;
+  }
+  const int pairs = d->pair_clusters > 0 ? d->pair_clusters : d->sms / 2;
+  auto waves = [](int64_t tiles, int64_t slots) { return (tiles + slots - 1) / slots; };
+  const int64_t m128 = (M + 127) / 128, m256 = (M + 255) / 256;
+  const double est_pair = waves(m256 * ((N + 255) / 256), pairs) * (128.0 * 256) / 1.0;
+  const double est_256 = waves(m128 * ((N + 255) / 256), d->sms) * (128.0 * 256) / 0.85;
+  const double est_128 = waves(m128 * ((N + 127) / 128), d->sms) * (128.0 * 128) / 0.45;
+  const double est_64 = waves(m128 * ((N + 63) / 64), d->sms) * (128.0 * 64) / 0.25;
+  const double best = fmin(fmin(est_pair, est_256), fmin(est_128, est_64));
+  if (est_pair == best) return launch_gemm_pair<6, 3>(d, xq, wq, m, n, k, s_in, s_w, y, st);
+  if (est_256 == best) return launch_gemm_cfg<256, 4, 0>(d, xq, wq, m, n, k, s_in, s_w, y, st);
+  if (est_128 == best) return launch_gemm_cfg<128, 6, 1>(d, xq, wq, m, n, k, s_in, s_w, y, st);
   return launch_gemm_cfg<64, 8, 2>(d, xq, wq, m, n, k, s_in, s_w, y, st);
 }
 
@@ -680,6 +695,12 @@ int fp8ws_device_status(int *status, int *where) {
   if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return FP8WS_ERR_CUDA;
   *where = v;
   *status = v ? FP8WS_ERR_DEVICE_TIMEOUT : FP8WS_OK;
+  return FP8WS_OK;
+}
+
+int fp8ws_set_gemm_config(int config) {
+  if (config < 0 || config > 4) return FP8WS_ERR_SHAPE;
+  g_forced_gemm_config = config;
   return FP8WS_OK;
 }
 

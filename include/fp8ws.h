@@ -285,6 +285,13 @@ FP8WS_API int fp8ws_device_check(void);
  * *where receives a code naming the wait that ran out (0 if none). */
 FP8WS_API int fp8ws_device_status(int *status, int *where);
 
+/* Tile configuration of fp8_linear_static and of the down projection of the
+ * gated MLPs, for tuning and tests: 0 = chosen per shape by the cost model
+ * (default), 1 = CTA-pair 256x256 tiles, 2/3/4 = one CTA with 128x256,
+ * 128x128 or 128x64 tiles.  Applies to later calls from every thread;
+ * FP8WS_ERR_SHAPE for other values. */
+FP8WS_API int fp8ws_set_gemm_config(int config);
+
 /* Launch log.  Every kernel the library enqueues is counted and recorded in a
  * small ring (the most recent FP8WS_LOG_CAPACITY launches).  kind: 1 quant,
  * 2 GEMM, 3 SwiGLU-quant, 4 calibration, 5 fused gate/up SwiGLU-quant.  in0/in1 are the primary input

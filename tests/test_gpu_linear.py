@@ -40,6 +40,13 @@ def _run(xq, wq, s_in, s_w, rows=None):
     return yb, ref
 
 
+@pytest.fixture(params=["auto", "pair256", "cta256", "cta128", "cta64"])
+def gemm_config(request):
+    fw.set_gemm_config(request.param)
+    yield request.param
+    fw.set_gemm_config("auto")
+
+
 @pytest.mark.parametrize("M,N,K", [
     (1, 8, 16),          # smallest legal problem
     (64, 704, 256),      # tiny-MLP gate/up
@@ -50,7 +57,7 @@ def _run(xq, wq, s_in, s_w, rows=None):
     (300, 1000, 272),
     (1024, 4096, 512),   # widest-tile dispatch
 ])
-def test_shapes(M, N, K):
+def test_shapes(M, N, K, gemm_config):
     rng = np.random.default_rng(M * 7 + N * 3 + K)
     xq = _random_codes(rng, (M, K))
     wq = _random_codes(rng, (N, K), 0.5)
@@ -64,7 +71,7 @@ def test_zero_rows():
     assert y.shape == (0, 16)
 
 
-def test_extreme_codes_no_overflow():
+def test_extreme_codes_no_overflow(gemm_config):
     """Largest codes everywhere: 448*448*K stays finite in fp32."""
     M, N, K = 128, 256, 512
     xq = np.full((M, K), 0x7E, np.uint8)
