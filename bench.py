@@ -201,7 +201,7 @@ def build_plan(fw, layers, bufs, stream_handle, fused):
         if fused:
             plan.append(("gate_up_swiglu", lib.fp8_gate_up_swiglu_static,
                          (xq, L.wg.data_ptr(), L.wu.data_ptr(), M, I, D, s_in, L.s_wg.data_ptr(),
-                          L.s_wu.data_ptr(), s_down, h, stream_handle),
+                          L.s_wu.data_ptr(), s_down, None, h, stream_handle),
                          M * D + 2 * I * D + M * I, 4 * M * I * D))
         else:
             g, u = b["g"].data_ptr(), b["u"].data_ptr()

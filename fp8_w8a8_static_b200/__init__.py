@@ -26,9 +26,10 @@ __all__ = [
     "FP8WSError", "library_path", "load",
     "fp8_quant_static", "fp8_linear_static", "silu_mul_2in_fp8",
     "gated_mlp_static_fp8", "gated_mlp_static_fp8_workspace",
-    "fp8_gate_up_swiglu_static", "gated_mlp_static_fp8_fused",
+    "fp8_gate_up_swiglu_static", "gated_mlp_static_fp8_fused", "swiglu_2in_fp8", "swiglu",
     "gated_mlp_static_fp8_fused_workspace",
-    "qkv_shared_quant", "qkv_shared_quant_workspace",
+    "qkv_shared_quant", "qkv_shared_quant_workspace", "fp8_shared_quant_linears",
+    "cross_attention_qkv_static_fp8",
     "fp8_check_shared_input_scale", "fp8_absmax_bf16", "fp8_silu_mul_absmax",
     "fp8_observer_scale", "fp8_rtn_quantize_weight",
     "device_check", "device_status", "launch_count", "launch_log", "launch_log_clear",
@@ -59,6 +60,21 @@ class FP8WSError(RuntimeError):
         super().__init__(f"{call}: status {status} ({STATUS.get(status, 'unknown')})")
 
 
+class Swiglu(ctypes.Structure):
+    """SwiGLU variant descriptor: g' sigmoid(alpha g') (u' + beta), with the
+    clamp g' <= limit, |u'| <= limit when has_limit."""
+    _fields_ = [("alpha", ctypes.c_float), ("beta", ctypes.c_float), ("limit", ctypes.c_float),
+                ("has_limit", ctypes.c_int32)]
+
+
+def swiglu(alpha: float = 1.0, beta: float = 0.0, limit=None) -> "Swiglu":
+    return Swiglu(alpha, beta, 0.0 if limit is None else limit, int(limit is not None))
+
+
+def _act(act):
+    return None if act is None else ctypes.byref(act)
+
+
 class LaunchRecord(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int32), ("pad", ctypes.c_int32), ("in0", ctypes.c_void_p),
                 ("in1", ctypes.c_void_p), ("out", ctypes.c_void_p)]
@@ -73,14 +89,25 @@ _SIGS = {
     "gated_mlp_static_fp8_workspace": (ctypes.c_size_t, [_I64, _I64, _I64]),
     "gated_mlp_static_fp8": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _P,
                                             _P, _P, _P]),
+    "swiglu_2in_fp8": (ctypes.c_int, [_P, _P, _I64, _P, _P, _P, _P]),
     "fp8_gate_up_swiglu_static": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P,
-                                                 _P, _P]),
+                                                 _P, _P, _P]),
     "gated_mlp_static_fp8_fused_workspace": (ctypes.c_size_t, [_I64, _I64, _I64]),
     "gated_mlp_static_fp8_fused": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P,
-                                                  _P, _P, _P, _P, _P]),
+                                                  _P, _P, _P, _P, _P, _P]),
     "gated_mlp_static_fp8_noalloc": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P,
                                                     _P, _P, _P, _P]),
     "qkv_shared_quant_workspace": (ctypes.c_size_t, [_I64, _I64]),
+    "fp8_shared_quant_linears_workspace": (ctypes.c_size_t, [_I64, _I64]),
+    "fp8_shared_quant_linears": (ctypes.c_int, [_P, _I64, _I64, _P, ctypes.c_int,
+                                                ctypes.POINTER(ctypes.c_void_p),
+                                                ctypes.POINTER(ctypes.c_int64),
+                                                ctypes.POINTER(ctypes.c_void_p),
+                                                ctypes.POINTER(ctypes.c_void_p), _P, _P]),
+    "cross_attention_qkv_static_fp8_workspace": (ctypes.c_size_t, [_I64, _I64, _I64]),
+    "cross_attention_qkv_static_fp8": (ctypes.c_int, [_P, _I64, _P, _I64, _I64, _P, _P, _I64, _P,
+                                                      _P, _P, _I64, _P, _P, _I64, _P, _P, _P, _P,
+                                                      _P, _P]),
     "qkv_shared_quant": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _I64, _P, _P, _I64, _P, _P, _I64,
                                         _P, _P, _P, _P, _P, _P]),
     "fp8_check_shared_input_scale": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int,
@@ -275,7 +302,21 @@ def gated_mlp_workspace_views(workspace: torch.Tensor, M: int, d: int, I: int):
     return dict(xq=xq, g=g, u=u, h=h)
 
 
-def fp8_gate_up_swiglu_static(xq, wg, wu, s_in, s_wg, s_wu, s_down, out=None,
+def swiglu_2in_fp8(g: torch.Tensor, u: torch.Tensor, s_down: torch.Tensor, act=None,
+                   out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """silu_mul_2in_fp8 with an optional variant descriptor (see swiglu())."""
+    lib = load()
+    if g.shape != u.shape:
+        raise ValueError("G and U shapes differ")
+    if out is None:
+        out = torch.empty(g.shape, dtype=FP8, device=g.device)
+    with _device_of(g):
+        _check(lib.swiglu_2in_fp8(_bf16(g, "g"), _bf16(u, "u"), g.numel(), _f32(s_down, "s_down"),
+                                  _act(act), _fp8(out, "out"), _stream(stream)), "swiglu_2in_fp8")
+    return out
+
+
+def fp8_gate_up_swiglu_static(xq, wg, wu, s_in, s_wg, s_wu, s_down, act=None, out=None,
                               stream=None) -> torch.Tensor:
     """H = E4M3(SiLU(bf16(G)) * bf16(U) / s_down) with G, U the gate and up
     projections of xq [M,K] (Wg, Wu [I,K]), computed in one kernel."""
@@ -289,8 +330,8 @@ def fp8_gate_up_swiglu_static(xq, wg, wu, s_in, s_wg, s_wu, s_down, out=None,
     with _device_of(xq):
         _check(lib.fp8_gate_up_swiglu_static(
             _fp8(xq, "xq"), _fp8(wg, "wg"), _fp8(wu, "wu"), M, I, K, _f32(s_in, "s_in"),
-            _f32(s_wg, "s_wg"), _f32(s_wu, "s_wu"), _f32(s_down, "s_down"), _fp8(out, "out"),
-            _stream(stream)), "fp8_gate_up_swiglu_static")
+            _f32(s_wg, "s_wg"), _f32(s_wu, "s_wu"), _f32(s_down, "s_down"), _act(act),
+            _fp8(out, "out"), _stream(stream)), "fp8_gate_up_swiglu_static")
     return out
 
 
@@ -299,7 +340,7 @@ def gated_mlp_static_fp8_fused_workspace(M: int, d: int, I: int) -> int:
 
 
 def gated_mlp_static_fp8_fused(x, s_in, wg, s_wg, wu, s_wu, s_down, wd, s_wd, workspace=None,
-                               out=None, stream=None) -> torch.Tensor:
+                               out=None, stream=None, act=None) -> torch.Tensor:
     """The gated MLP with gate/up and the SwiGLU-quant fused: quantize X, one
     fused gate/up/SwiGLU kernel, the down GEMM.  Same result as
     gated_mlp_static_fp8, bit for bit."""
@@ -320,8 +361,8 @@ def gated_mlp_static_fp8_fused(x, s_in, wg, s_wg, wu, s_wu, s_down, wd, s_wd, wo
     with _device_of(x):
         _check(lib.gated_mlp_static_fp8_fused(
             _bf16(x, "x"), M, d, I, _f32(s_in, "s_in"), _fp8(wg, "wg"), _f32(s_wg, "s_wg"),
-            _fp8(wu, "wu"), _f32(s_wu, "s_wu"), _f32(s_down, "s_down"), _fp8(wd, "wd"),
-            _f32(s_wd, "s_wd"), _dev_ptr(workspace, "workspace", (torch.uint8,)),
+            _fp8(wu, "wu"), _f32(s_wu, "s_wu"), _f32(s_down, "s_down"), _act(act),
+            _fp8(wd, "wd"), _f32(s_wd, "s_wd"), _dev_ptr(workspace, "workspace", (torch.uint8,)),
             _bf16(out, "out"), _stream(stream)), "gated_mlp_static_fp8_fused")
     return out
 
@@ -359,6 +400,57 @@ def qkv_shared_quant(x, s_in, wq, s_wq, wk, s_wk, wv, s_wv, workspace=None, out=
             _fp8(wk, "wk"), Nk, _f32(s_wk, "s_wk"), _fp8(wv, "wv"), Nv, _f32(s_wv, "s_wv"),
             _dev_ptr(workspace, "workspace", (torch.uint8,)), _bf16(q, "q"), _bf16(k, "k"),
             _bf16(v, "v"), _stream(stream)), "qkv_shared_quant")
+    return q, k, v
+
+
+def fp8_shared_quant_linears(x, s_in, projections, workspace=None, out=None, stream=None):
+    """Quantize x [M,d] once, then one Linear per (W [N,d] FP8, s_w) in
+    projections; returns the BF16 outputs [M,N] (n = 1 is e.g. o_proj)."""
+    lib = load()
+    M, d = x.shape
+    n = len(projections)
+    for i, (w, _) in enumerate(projections):
+        if w.dim() != 2 or w.shape[1] != d:
+            raise ValueError(f"projection {i} must be [N, {d}]")
+    if out is None:
+        out = [torch.empty((M, w.shape[0]), dtype=torch.bfloat16, device=x.device)
+               for w, _ in projections]
+    need = lib.fp8_shared_quant_linears_workspace(M, d)
+    if workspace is None:
+        workspace = _workspace(need, x.device)
+    W = (ctypes.c_void_p * n)(*[_fp8(w, f"W[{i}]") for i, (w, _) in enumerate(projections)])
+    N = (ctypes.c_int64 * n)(*[w.shape[0] for w, _ in projections])
+    S = (ctypes.c_void_p * n)(*[_f32(sw, f"s_w[{i}]") for i, (_, sw) in enumerate(projections)])
+    Y = (ctypes.c_void_p * n)(*[_bf16(y, f"y[{i}]") for i, y in enumerate(out)])
+    with _device_of(x):
+        _check(lib.fp8_shared_quant_linears(_bf16(x, "x"), M, d, _f32(s_in, "s_in"), n, W, N, S, Y,
+                                            _dev_ptr(workspace, "workspace", (torch.uint8,)),
+                                            _stream(stream)), "fp8_shared_quant_linears")
+    return out
+
+
+def cross_attention_qkv_static_fp8(x, ctx, s_q, wq, s_wq, s_kv, wk, s_wk, wv, s_wv,
+                                   workspace=None, out=None, stream=None):
+    """Q from x (own quantization at s_q); K and V from ctx (one shared
+    quantization at s_kv).  Returns contiguous BF16 q, k, v."""
+    lib = load()
+    Mq, d = x.shape
+    Mkv = ctx.shape[0]
+    if out is None:
+        out = (torch.empty((Mq, wq.shape[0]), dtype=torch.bfloat16, device=x.device),
+               torch.empty((Mkv, wk.shape[0]), dtype=torch.bfloat16, device=x.device),
+               torch.empty((Mkv, wv.shape[0]), dtype=torch.bfloat16, device=x.device))
+    q, k, v = out
+    need = lib.cross_attention_qkv_static_fp8_workspace(Mq, Mkv, d)
+    if workspace is None:
+        workspace = _workspace(need, x.device)
+    with _device_of(x):
+        _check(lib.cross_attention_qkv_static_fp8(
+            _bf16(x, "x"), Mq, _bf16(ctx, "ctx"), Mkv, d, _f32(s_q, "s_q"), _fp8(wq, "wq"),
+            wq.shape[0], _f32(s_wq, "s_wq"), _f32(s_kv, "s_kv"), _fp8(wk, "wk"), wk.shape[0],
+            _f32(s_wk, "s_wk"), _fp8(wv, "wv"), wv.shape[0], _f32(s_wv, "s_wv"),
+            _dev_ptr(workspace, "workspace", (torch.uint8,)), _bf16(q, "q"), _bf16(k, "k"),
+            _bf16(v, "v"), _stream(stream)), "cross_attention_qkv_static_fp8")
     return q, k, v
 
 

@@ -108,6 +108,72 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
   return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
+// SwiGLU variant: g' sigmoid(alpha g') (u' + beta), with the clamp g' <= limit,
+// |u'| <= limit when has_limit, and the offset only when beta != 0.  With
+// alpha = 1, beta = 0 and no limit this performs exactly silu_mul's
+// operations (alpha * g == g), so the results are bit-identical.
+struct SwigluParams {
+  float alpha, beta, limit;
+  int has_limit;
+};
+
+__device__ __forceinline__ float swiglu_mul(float g, float u, const SwigluParams &p) {
+  if (p.has_limit) {
+    g = fminf(g, p.limit);
+    u = fminf(fmaxf(u, -p.limit), p.limit);
+  }
+  const float up = p.beta != 0.0f ? u + p.beta : u;
+  return __fdividef(g, 1.0f + __expf(-(p.alpha * g))) * up;
+}
+
+__device__ __forceinline__ uint2 swiglu_quant8(uint4 g, uint4 u, float inv_s,
+                                               const SwigluParams &p) {
+  uint2 o;
+  o.x = pack4(cvt_e4m3x2(swiglu_mul(bf16_lo(g.x), bf16_lo(u.x), p) * inv_s,
+                         swiglu_mul(bf16_hi(g.x), bf16_hi(u.x), p) * inv_s),
+              cvt_e4m3x2(swiglu_mul(bf16_lo(g.y), bf16_lo(u.y), p) * inv_s,
+                         swiglu_mul(bf16_hi(g.y), bf16_hi(u.y), p) * inv_s));
+  o.y = pack4(cvt_e4m3x2(swiglu_mul(bf16_lo(g.z), bf16_lo(u.z), p) * inv_s,
+                         swiglu_mul(bf16_hi(g.z), bf16_hi(u.z), p) * inv_s),
+              cvt_e4m3x2(swiglu_mul(bf16_lo(g.w), bf16_lo(u.w), p) * inv_s,
+                         swiglu_mul(bf16_hi(g.w), bf16_hi(u.w), p) * inv_s));
+  return o;
+}
+
+__global__ void __launch_bounds__(kEwThreads) swiglu_2in_kernel(
+    const uint16_t *__restrict__ g, const uint16_t *__restrict__ u, int64_t numel,
+    const float *__restrict__ s_down, SwigluParams p, uint8_t *__restrict__ h) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const float inv_s = __frcp_rn(__ldg(s_down));
+  const int64_t nvec = numel >> 3;
+  const uint4 *gv = reinterpret_cast<const uint4 *>(g);
+  const uint4 *uv = reinterpret_cast<const uint4 *>(u);
+  uint2 *hv = reinterpret_cast<uint2 *>(h);
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  int64_t i = tid;
+  for (; i + (kEwUnroll - 1) * stride < nvec; i += kEwUnroll * stride) {
+    uint4 a[kEwUnroll], b[kEwUnroll];
+#pragma unroll
+    for (int k = 0; k < kEwUnroll; ++k) {
+      a[k] = ld_stream(gv + i + k * stride);
+      b[k] = ld_stream(uv + i + k * stride);
+    }
+#pragma unroll
+    for (int k = 0; k < kEwUnroll; ++k)
+      st_stream(hv + i + k * stride, swiglu_quant8(a[k], b[k], inv_s, p));
+  }
+  for (; i < nvec; i += stride)
+    st_stream(hv + i, swiglu_quant8(ld_stream(gv + i), ld_stream(uv + i), inv_s, p));
+  const int64_t t = (nvec << 3) + tid;
+  if (t < numel) {
+    float a = __uint_as_float(static_cast<uint32_t>(g[t]) << 16);
+    float b = __uint_as_float(static_cast<uint32_t>(u[t]) << 16);
+    h[t] = static_cast<uint8_t>(cvt_e4m3x2(swiglu_mul(a, b, p) * inv_s, 0.0f) & 0xFFu);
+  }
+}
+
 __device__ __forceinline__ uint2 silu_mul_quant8(uint4 g, uint4 u, float inv_s) {
   uint2 o;
   o.x = pack4(cvt_e4m3x2(silu_mul(bf16_lo(g.x), bf16_lo(u.x)) * inv_s,

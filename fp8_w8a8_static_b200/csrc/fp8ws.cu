@@ -268,7 +268,8 @@ int launch_gemm_pair(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int M,
 template <int STAGES, int BIT>
 int launch_dual_swiglu(DeviceInfo *d, const uint8_t *xq, const uint8_t *wg, const uint8_t *wu,
                        int M, int N, int K, const float *s_in, const float *s_wg,
-                       const float *s_wu, const float *s_down, uint8_t *h, cudaStream_t st) {
+                       const float *s_wu, const float *s_down, SwigluParams act, uint8_t *h,
+                       cudaStream_t st) {
   using C = DualCfg<STAGES>;
   auto kern = fp8_dual_swiglu_pair_kernel<STAGES>;
   cudaLaunchAttribute attr[1];
@@ -302,7 +303,7 @@ int launch_dual_swiglu(DeviceInfo *d, const uint8_t *xq, const uint8_t *wg, cons
   const int tiles = ((M + kDualTileM - 1) / kDualTileM) * ((N + kDualTileN - 1) / kDualTileN);
   const int clusters = tiles < d->dual_clusters ? tiles : d->dual_clusters;
   if (launch_ex(kern, dim3(2 * clusters), dim3(kGemmThreads), C::SMEM_BYTES, st, 2, ma, mg, mu, mh,
-                s_in, s_wg, s_wu, s_down, M, N, K, kWaitLimitNs) != cudaSuccess)
+                s_in, s_wg, s_wu, s_down, act, M, N, K, kWaitLimitNs) != cudaSuccess)
     return FP8WS_ERR_CUDA;
   log_launch(kKindDual, xq, wg, h);
   return launch_status();
@@ -373,6 +374,22 @@ int silu_launch(DeviceInfo *d, const uint16_t *g, const uint16_t *u, int64_t num
 
 size_t round256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
+// NULL = plain SwiGLU (alpha 1, no offset, no clamp).
+int swiglu_params(const fp8ws_swiglu *act, SwigluParams *p) {
+  p->alpha = 1.0f;
+  p->beta = 0.0f;
+  p->limit = 0.0f;
+  p->has_limit = 0;
+  if (!act) return FP8WS_OK;
+  if (!isfinite(act->alpha) || !isfinite(act->beta)) return FP8WS_ERR_BAD_SCALE;
+  if (act->has_limit && !(act->limit > 0.0f)) return FP8WS_ERR_BAD_SCALE;
+  p->alpha = act->alpha;
+  p->beta = act->beta;
+  p->limit = act->limit;
+  p->has_limit = act->has_limit ? 1 : 0;
+  return FP8WS_OK;
+}
+
 }  // namespace
 }  // namespace fp8ws
 
@@ -412,6 +429,26 @@ int silu_mul_2in_fp8(const uint16_t *g, const uint16_t *u, int64_t numel, const 
   int rc = device_info(&d);
   if (rc) return rc;
   return silu_launch(d, g, u, numel, s_down, h, as_stream(stream));
+}
+
+int swiglu_2in_fp8(const uint16_t *g, const uint16_t *u, int64_t numel, const float *s_down,
+                   const fp8ws_swiglu *act, uint8_t *h, void *stream) {
+  if (numel < 0) return FP8WS_ERR_SHAPE;
+  SwigluParams ap;
+  int rc = swiglu_params(act, &ap);
+  if (rc) return rc;
+  if (numel == 0) return FP8WS_OK;
+  if (!g || !u || !s_down || !h) return FP8WS_ERR_NULL;
+  if (!aligned16(g) || !aligned16(u) || !aligned16(h)) return FP8WS_ERR_ALIGN;
+  DeviceInfo *d;
+  rc = device_info(&d);
+  if (rc) return rc;
+  cudaStream_t st = as_stream(stream);
+  if (launch_ex(swiglu_2in_kernel, dim3(ew_grid(d, swiglu_2in_kernel, numel >> 3)),
+                dim3(kEwThreads), 0, st, 1, g, u, numel, s_down, ap, h) != cudaSuccess)
+    return FP8WS_ERR_CUDA;
+  log_launch(kKindSwiglu, g, u, h);
+  return launch_status();
 }
 
 size_t gated_mlp_static_fp8_workspace(int64_t M, int64_t d, int64_t I) {
@@ -485,9 +522,12 @@ int qkv_shared_quant(const uint16_t *x, int64_t M, int64_t dm, const float *s_in
 int fp8_gate_up_swiglu_static(const uint8_t *xq, const uint8_t *Wg, const uint8_t *Wu,
                               int64_t M, int64_t I, int64_t K, const float *s_in,
                               const float *s_wg, const float *s_wu, const float *s_down,
-                              uint8_t *h, void *stream) {
+                              const fp8ws_swiglu *act, uint8_t *h, void *stream) {
   if (!s_down || !Wu || !s_wu) return FP8WS_ERR_NULL;
   int rc = check_gemm_args(xq, Wg, M, I, K, s_in, s_wg, h);
+  if (rc) return rc;
+  SwigluParams ap;
+  rc = swiglu_params(act, &ap);
   if (rc) return rc;
   if (I % 16 != 0) return FP8WS_ERR_SHAPE;  // FP8 rows of H must be 16-byte multiples
   if (!aligned16(Wu)) return FP8WS_ERR_ALIGN;
@@ -496,7 +536,7 @@ int fp8_gate_up_swiglu_static(const uint8_t *xq, const uint8_t *Wg, const uint8_
   if (rc) return rc;
   if (M == 0) return FP8WS_OK;
   return launch_dual_swiglu<6, 4>(d, xq, Wg, Wu, static_cast<int>(M), static_cast<int>(I),
-                                  static_cast<int>(K), s_in, s_wg, s_wu, s_down, h,
+                                  static_cast<int>(K), s_in, s_wg, s_wu, s_down, ap, h,
                                   as_stream(stream));
 }
 
@@ -509,11 +549,14 @@ size_t gated_mlp_static_fp8_fused_workspace(int64_t M, int64_t d, int64_t I) {
 int gated_mlp_static_fp8_fused(const uint16_t *x, int64_t M, int64_t dm, int64_t I,
                                const float *s_in, const uint8_t *Wg, const float *s_wg,
                                const uint8_t *Wu, const float *s_wu, const float *s_down,
-                               const uint8_t *Wd, const float *s_wd, void *workspace, uint16_t *y,
-                               void *stream) {
+                               const fp8ws_swiglu *act, const uint8_t *Wd, const float *s_wd,
+                               void *workspace, uint16_t *y, void *stream) {
   if (!s_in || !Wg || !s_wg || !Wu || !s_wu || !s_down || !Wd || !s_wd ||
       (M != 0 && (!x || !y)))
     return FP8WS_ERR_NULL;
+  SwigluParams ap;
+  int rca = swiglu_params(act, &ap);
+  if (rca) return rca;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FP8WS_ERR_WORKSPACE;
   if (!aligned16(x) || !aligned16(Wu)) return FP8WS_ERR_ALIGN;
   uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -532,7 +575,7 @@ int gated_mlp_static_fp8_fused(const uint16_t *x, int64_t M, int64_t dm, int64_t
   rc = quant_launch(d, x, M * dm, s_in, xq, st);
   if (!rc)
     rc = launch_dual_swiglu<6, 4>(d, xq, Wg, Wu, static_cast<int>(M), static_cast<int>(I),
-                                  static_cast<int>(dm), s_in, s_wg, s_wu, s_down, H, st);
+                                  static_cast<int>(dm), s_in, s_wg, s_wu, s_down, ap, H, st);
   if (!rc) rc = gemm_dispatch(d, H, Wd, M, dm, I, s_down, s_wd, y, st);
   return rc;
 }
@@ -580,6 +623,68 @@ int gated_mlp_static_fp8_noalloc(const uint16_t *x, int64_t M, int64_t d, int64_
   if (rc) return rc;
   return gated_mlp_static_fp8(x, M, d, I, s_in, Wg, s_wg, Wu, s_wu, s_down, Wd, s_wd, scratch, y,
                               stream);
+}
+
+size_t fp8_shared_quant_linears_workspace(int64_t M, int64_t d) {
+  if (M < 0 || d < 0) return 0;
+  return round256(static_cast<size_t>(M) * static_cast<size_t>(d));
+}
+
+int fp8_shared_quant_linears(const uint16_t *x, int64_t M, int64_t dm, const float *s_in, int n,
+                             const uint8_t *const *W, const int64_t *N, const float *const *s_w,
+                             uint16_t *const *y, void *workspace, void *stream) {
+  if (n < 1 || n > FP8WS_MAX_PROJECTIONS) return FP8WS_ERR_SHAPE;
+  if (!W || !N || !s_w || !y || !s_in || (M != 0 && !x)) return FP8WS_ERR_NULL;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FP8WS_ERR_WORKSPACE;
+  if (!aligned16(x)) return FP8WS_ERR_ALIGN;
+  uint8_t *xq = static_cast<uint8_t *>(workspace);
+  int rc = FP8WS_OK;
+  for (int i = 0; i < n && !rc; ++i) rc = check_gemm_args(xq, W[i], M, N[i], dm, s_in, s_w[i], y[i]);
+  if (rc) return rc;
+  DeviceInfo *d;
+  rc = device_info(&d);
+  if (rc) return rc;
+  if (M == 0) return FP8WS_OK;
+  cudaStream_t st = as_stream(stream);
+  rc = quant_launch(d, x, M * dm, s_in, xq, st);
+  for (int i = 0; i < n && !rc; ++i) rc = gemm_dispatch(d, xq, W[i], M, N[i], dm, s_in, s_w[i], y[i], st);
+  return rc;
+}
+
+size_t cross_attention_qkv_static_fp8_workspace(int64_t Mq, int64_t Mkv, int64_t d) {
+  if (Mq < 0 || Mkv < 0 || d < 0) return 0;
+  return round256(static_cast<size_t>(Mq) * d) + round256(static_cast<size_t>(Mkv) * d);
+}
+
+int cross_attention_qkv_static_fp8(const uint16_t *x, int64_t Mq, const uint16_t *ctx,
+                                   int64_t Mkv, int64_t dm, const float *s_q, const uint8_t *Wq,
+                                   int64_t Nq, const float *s_wq, const float *s_kv,
+                                   const uint8_t *Wk, int64_t Nk, const float *s_wk,
+                                   const uint8_t *Wv, int64_t Nv, const float *s_wv,
+                                   void *workspace, uint16_t *q, uint16_t *k, uint16_t *v,
+                                   void *stream) {
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FP8WS_ERR_WORKSPACE;
+  if (Mq < 0 || Mkv < 0 || dm < 0) return FP8WS_ERR_SHAPE;
+  uint8_t *ws_kv = static_cast<uint8_t *>(workspace) + round256(static_cast<size_t>(Mq) * dm);
+  // validate both halves before enqueueing either
+  uint8_t *probe = static_cast<uint8_t *>(workspace);
+  int rc = check_gemm_args(probe, Wq, Mq, Nq, dm, s_q, s_wq, q);
+  if (!rc) rc = check_gemm_args(ws_kv, Wk, Mkv, Nk, dm, s_kv, s_wk, k);
+  if (!rc) rc = check_gemm_args(ws_kv, Wv, Mkv, Nv, dm, s_kv, s_wv, v);
+  if (!rc && ((Mq != 0 && !x) || (Mkv != 0 && !ctx))) rc = FP8WS_ERR_NULL;
+  if (!rc && (!aligned16(x) || !aligned16(ctx))) rc = FP8WS_ERR_ALIGN;
+  if (rc) return rc;
+  const uint8_t *wq1[1] = {Wq};
+  const int64_t nq1[1] = {Nq};
+  const float *sq1[1] = {s_wq};
+  uint16_t *yq1[1] = {q};
+  rc = fp8_shared_quant_linears(x, Mq, dm, s_q, 1, wq1, nq1, sq1, yq1, workspace, stream);
+  if (rc) return rc;
+  const uint8_t *wkv[2] = {Wk, Wv};
+  const int64_t nkv[2] = {Nk, Nv};
+  const float *skv[2] = {s_wk, s_wv};
+  uint16_t *ykv[2] = {k, v};
+  return fp8_shared_quant_linears(ctx, Mkv, dm, s_kv, 2, wkv, nkv, skv, ykv, ws_kv, stream);
 }
 
 int fp8_check_shared_input_scale(const float *const *d_scales, int n, void *stream) {

@@ -3,6 +3,7 @@
 //
 //   G = bf16((s_in*s_wg) * Xq . Wg^T),  U = bf16((s_in*s_wu) * Xq . Wu^T)
 //   H = E4M3_satRNE( SiLU(G) * U * (1/s_down) )            [M, I] FP8
+//   (or the alpha/beta/limit SwiGLU variant of swiglu_mul)
 //
 // The BF16 rounding of G and U and the fp32 SwiGLU arithmetic are the very
 // operations of fp8_gemm_kernel's epilogue followed by silu_mul_2in_kernel, so
@@ -56,8 +57,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                 const __grid_constant__ CUtensorMap tm_h,
                                 const float *__restrict__ s_in, const float *__restrict__ s_wg,
                                 const float *__restrict__ s_wu,
-                                const float *__restrict__ s_down, int M, int N, int K,
-                                uint64_t timeout_ns) {
+                                const float *__restrict__ s_down, SwigluParams act, int M,
+                                int N, int K, uint64_t timeout_ns) {
   using C = DualCfg<STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -244,7 +245,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int e = 0; e < 4; ++e) {
             const float gv = __bfloat162float(__float2bfloat16_rn(__uint_as_float(g[4 * j + e]) * scale_g));
             const float uv = __bfloat162float(__float2bfloat16_rn(__uint_as_float(u[4 * j + e]) * scale_u));
-            h[e] = silu_mul(gv, uv) * inv_s;
+            h[e] = swiglu_mul(gv, uv, act) * inv_s;
           }
           q[j] = pack4(cvt_e4m3x2(h[0], h[1]), cvt_e4m3x2(h[2], h[3]));
         }

@@ -116,6 +116,31 @@ FP8WS_API int silu_mul_2in_fp8(const uint16_t *g, const uint16_t *u, int64_t num
                      uint8_t *h, void *stream);
 
 /*
+ * SwiGLU variants.  [PR] commit notes on the two-input SwiGLU: the activation
+ * may carry swiglu_alpha (a gain inside the sigmoid), swiglu_beta (an offset
+ * on up) and swiglu_limit; omitting all of them is plain SwiGLU.  The limit is
+ * read as the clamp of the "swigluoai" shape: gate <= limit and
+ * -limit <= up <= limit.
+ *
+ *   h = E4M3_satRNE( g' * sigmoid(alpha * g') * (u' + beta) / s_down )
+ *
+ * A NULL descriptor, or alpha = 1, beta = 0, has_limit = 0, gives exactly the
+ * results of silu_mul_2in_fp8.  alpha and beta must be finite and limit > 0
+ * when has_limit (FP8WS_ERR_BAD_SCALE otherwise).
+ */
+typedef struct {
+  float alpha;
+  float beta;
+  float limit;
+  int32_t has_limit;
+} fp8ws_swiglu;
+
+/* swiglu_2in_fp8 -- silu_mul_2in_fp8 with an optional variant descriptor. */
+FP8WS_API int swiglu_2in_fp8(const uint16_t *g, const uint16_t *u, int64_t numel,
+                             const float *s_down, const fp8ws_swiglu *act, uint8_t *h,
+                             void *stream);
+
+/*
  * gated_mlp_static_fp8 -- the split gated MLP on the static FP8 path.
  * [PR] What changed (GatedMLP with split gate/up: quantize the shared
  * activation once, hand the FP8 tensor to both projections, two-input SwiGLU
@@ -153,12 +178,14 @@ FP8WS_API int gated_mlp_static_fp8(const uint16_t *x, int64_t M, int64_t d, int6
  * Bit-identical to fp8_linear_static (gate), fp8_linear_static (up) and
  * silu_mul_2in_fp8 run one after the other on the same inputs.
  * xq: device [M,K] FP8.  Wg, Wu: device [I,K] FP8.  Scales: device fp32.
+ * act: SwiGLU variant (NULL = plain), as swiglu_2in_fp8.
  * h: device [M,I] FP8.  Sizes: as fp8_linear_static with N = I, and I % 16 == 0.
  */
 FP8WS_API int fp8_gate_up_swiglu_static(const uint8_t *xq, const uint8_t *Wg, const uint8_t *Wu,
                                         int64_t M, int64_t I, int64_t K, const float *s_in,
                                         const float *s_wg, const float *s_wu,
-                                        const float *s_down, uint8_t *h, void *stream);
+                                        const float *s_down, const fp8ws_swiglu *act,
+                                        uint8_t *h, void *stream);
 
 /*
  * gated_mlp_static_fp8_fused -- gated_mlp_static_fp8 with the gate/up GEMMs
@@ -167,15 +194,16 @@ FP8WS_API int fp8_gate_up_swiglu_static(const uint8_t *xq, const uint8_t *Wg, co
  * round trip through memory.  Same result, bit for bit.
  * workspace: device, gated_mlp_static_fp8_fused_workspace(M,d,I) bytes,
  * 256-byte aligned; holds Xq [M,d] then H [M,I] (each region 256-byte
- * aligned).  Other arguments as gated_mlp_static_fp8.
+ * aligned).  act: SwiGLU variant (NULL = plain).  Other arguments as
+ * gated_mlp_static_fp8.
  */
 FP8WS_API size_t gated_mlp_static_fp8_fused_workspace(int64_t M, int64_t d, int64_t I);
 FP8WS_API int gated_mlp_static_fp8_fused(const uint16_t *x, int64_t M, int64_t d, int64_t I,
                                          const float *s_in, const uint8_t *Wg, const float *s_wg,
                                          const uint8_t *Wu, const float *s_wu,
-                                         const float *s_down, const uint8_t *Wd,
-                                         const float *s_wd, void *workspace, uint16_t *y,
-                                         void *stream);
+                                         const float *s_down, const fp8ws_swiglu *act,
+                                         const uint8_t *Wd, const float *s_wd, void *workspace,
+                                         uint16_t *y, void *stream);
 
 /*
  * qkv_shared_quant -- Q/K/V projections from one shared quantization.
@@ -234,6 +262,48 @@ FP8WS_API int gated_mlp_static_fp8_noalloc(const uint16_t *x, int64_t M, int64_t
                                            const float *s_wu, const float *s_down,
                                            const uint8_t *Wd, const float *s_wd, uint16_t *y,
                                            void *stream);
+
+/*
+ * fp8_shared_quant_linears -- quantize one activation once and run n Linears
+ * on that single FP8 copy (the general form of qkv_shared_quant; with n = 1 it
+ * is a standalone projection such as o_proj).  [PR] What changed: members of
+ * a formerly fused group consume one quantized activation, which is only
+ * sound while their calibrated input scales agree (checked at load with
+ * fp8_check_shared_input_scale).
+ *
+ * x: device [M,d] BF16.  n: 1..FP8WS_MAX_PROJECTIONS.  W, N, s_w, y: host
+ * arrays of n entries: device [N[i],d] FP8 weights, output widths, device fp32
+ * weight scales and device [M,N[i]] BF16 outputs (each contiguous).
+ * workspace: device, fp8_shared_quant_linears_workspace(M,d) bytes, 256-byte
+ * aligned (holds Xq).
+ */
+#define FP8WS_MAX_PROJECTIONS 16
+FP8WS_API size_t fp8_shared_quant_linears_workspace(int64_t M, int64_t d);
+FP8WS_API int fp8_shared_quant_linears(const uint16_t *x, int64_t M, int64_t d, const float *s_in,
+                                       int n, const uint8_t *const *W, const int64_t *N,
+                                       const float *const *s_w, uint16_t *const *y,
+                                       void *workspace, void *stream);
+
+/*
+ * cross_attention_qkv_static_fp8 -- projections of a cross-attention: Q from
+ * the query-side activation x, K and V from a different tensor ctx.  [PR] Test
+ * Coverage: where K/V come from another tensor, sharing must not engage
+ * between Q and K/V.  So x is quantized with its own s_q for Q, and ctx is
+ * quantized once with s_kv and shared by K and V (whose calibrated input
+ * scales must agree).
+ * x: device [Mq,d] BF16; ctx: device [Mkv,d] BF16; Wq [Nq,d], Wk [Nk,d],
+ * Wv [Nv,d] FP8; q [Mq,Nq], k [Mkv,Nk], v [Mkv,Nv] BF16, contiguous.
+ * workspace: cross_attention_qkv_static_fp8_workspace(Mq,Mkv,d) bytes,
+ * 256-byte aligned: Xq [Mq,d] then the quantized context [Mkv,d].
+ */
+FP8WS_API size_t cross_attention_qkv_static_fp8_workspace(int64_t Mq, int64_t Mkv, int64_t d);
+FP8WS_API int cross_attention_qkv_static_fp8(const uint16_t *x, int64_t Mq, const uint16_t *ctx,
+                                             int64_t Mkv, int64_t d, const float *s_q,
+                                             const uint8_t *Wq, int64_t Nq, const float *s_wq,
+                                             const float *s_kv, const uint8_t *Wk, int64_t Nk,
+                                             const float *s_wk, const uint8_t *Wv, int64_t Nv,
+                                             const float *s_wv, void *workspace, uint16_t *q,
+                                             uint16_t *k, uint16_t *v, void *stream);
 
 /* ------------------------------------------------------------- load time */
 

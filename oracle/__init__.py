@@ -84,6 +84,8 @@ def lib():
             "oracle_silu_mul_2in": (None, [u16p, u16p, i64, f32, u8p]),
             "oracle_silu_and_mul_fused": (None, [u16p, i64, i64, f32, u8p]),
             "oracle_silu_mul_f64": (None, [dp, dp, i64, dp]),
+            "oracle_swiglu_2in": (None, [u16p, u16p, i64, f32, f32, f32, ctypes.c_int, f32, u8p]),
+            "oracle_swiglu_fused": (None, [u16p, i64, i64, f32, f32, f32, ctypes.c_int, f32, u8p]),
             "oracle_requant_group_member": (None, [u8p, i64, f32, f32, u8p]),
             "oracle_dequant": (None, [u8p, i64, dp]),
             "oracle_num_threads": (ctypes.c_int, []),
@@ -210,6 +212,34 @@ def silu_and_mul_fused(gu_bf16, s_down: float) -> np.ndarray:
     return h
 
 
+def swiglu_2in(g_bf16, u_bf16, s_down: float, alpha: float = 1.0, beta: float = 0.0,
+               limit=None) -> np.ndarray:
+    """Two-input SwiGLU variant quantized to FP8: g' sigmoid(alpha g') (u' + beta),
+    with the optional clamp g' = min(g, limit), u' = clamp(u, -limit, limit)."""
+    g = _u16(g_bf16)
+    u = _u16(u_bf16)
+    if g.shape != u.shape:
+        raise ValueError("G and U shapes differ")
+    h = np.empty(g.shape, dtype=np.uint8)
+    lib().oracle_swiglu_2in(_p(g, ctypes.c_uint16), _p(u, ctypes.c_uint16), g.size, s_down,
+                            alpha, beta, int(limit is not None),
+                            0.0 if limit is None else limit, _p(h, ctypes.c_uint8))
+    return h
+
+
+def swiglu_fused(gu_bf16, s_down: float, alpha: float = 1.0, beta: float = 0.0,
+                 limit=None) -> np.ndarray:
+    """The variant on one [..., 2I] tensor (gate = first half, up = second half)."""
+    gu = _u16(gu_bf16)
+    I2 = gu.shape[-1]
+    rows = gu.size // I2
+    h = np.empty(gu.shape[:-1] + (I2 // 2,), dtype=np.uint8)
+    lib().oracle_swiglu_fused(_p(gu, ctypes.c_uint16), rows, I2 // 2, s_down, alpha, beta,
+                              int(limit is not None), 0.0 if limit is None else limit,
+                              _p(h, ctypes.c_uint8))
+    return h
+
+
 def requant_group_member(qw, s_i: float, s_max: float) -> np.ndarray:
     """The fused loader's second rounding: q64(s_i * deq(qW) / s_max)."""
     qw = _u8(qw)
@@ -316,6 +346,15 @@ def qkv_shared_quant(x_bf16, s_in, projections):
     """Quantize X once, then one Linear per (Wq, s_w) in projections."""
     xq = quantize(x_bf16, s_in)
     return [linear(xq, wq, s_in, sw) for wq, sw in projections]
+
+
+def cross_attention_qkv(x_bf16, ctx_bf16, s_q, q_proj, s_kv, k_proj, v_proj):
+    """Cross-attention projections: Q from x at its own scale s_q; K and V
+    from ctx through one shared quantization at s_kv (sharing between Q and
+    K/V must not engage, since they read different tensors)."""
+    (q,) = qkv_shared_quant(x_bf16, s_q, [q_proj])
+    k, v = qkv_shared_quant(ctx_bf16, s_kv, [k_proj, v_proj])
+    return q, k, v
 
 
 def num_threads() -> int:

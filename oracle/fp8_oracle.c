@@ -265,6 +265,45 @@ void oracle_silu_and_mul_fused(const uint16_t *gu, int64_t rows, int64_t I,
       h[r * I + i] = silu_mul_code(gu[r * 2 * I + i], gu[r * 2 * I + I + i], s);
 }
 
+/* ------------------------------------------------------------------------ */
+/* SwiGLU variants ([PR] commit notes on the two-input SwiGLU: alpha is a gain */
+/* inside the sigmoid, beta an offset on up; swiglu_limit is named there and  */
+/* read here as the clamp of the "swigluoai" shape: gate <= limit,            */
+/* -limit <= up <= limit).                                                   */
+/*   h = q64( g' * sigmoid(alpha g') * (u' + beta), s_down )                 */
+/* with g' = min(g, limit), u' = clamp(u, -limit, limit) when has_limit,     */
+/* and the offset added only when beta != 0 (so that alpha = 1, beta = 0 and */
+/* no limit is the plain two-input SwiGLU, bit for bit).                     */
+/* ------------------------------------------------------------------------ */
+static uint8_t swiglu_code(uint16_t gb, uint16_t ub, double s, double alpha, double beta,
+                           int has_limit, double limit) {
+  double g = bf16_to_double(gb);
+  double u = bf16_to_double(ub);
+  if (has_limit) {
+    if (g > limit) g = limit;
+    if (u > limit) u = limit;
+    if (u < -limit) u = -limit;
+  }
+  double act = g / (1.0 + exp(-(alpha * g)));
+  double up = (beta != 0.0) ? u + beta : u;
+  return oracle_quant_f64(act * up, s);
+}
+
+void oracle_swiglu_2in(const uint16_t *g, const uint16_t *u, int64_t n, float s_down,
+                       float alpha, float beta, int has_limit, float limit, uint8_t *h) {
+  for (int64_t i = 0; i < n; ++i)
+    h[i] = swiglu_code(g[i], u[i], (double)s_down, (double)alpha, (double)beta, has_limit,
+                       (double)limit);
+}
+
+void oracle_swiglu_fused(const uint16_t *gu, int64_t rows, int64_t I, float s_down, float alpha,
+                         float beta, int has_limit, float limit, uint8_t *h) {
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t i = 0; i < I; ++i)
+      h[r * I + i] = swiglu_code(gu[r * 2 * I + i], gu[r * 2 * I + I + i], (double)s_down,
+                                 (double)alpha, (double)beta, has_limit, (double)limit);
+}
+
 /* Unquantized SiLU(g) * u in fp64 (the value the down_proj input observer
  * sees), for calibration of s_down. */
 void oracle_silu_mul_f64(const double *g, const double *u, int64_t n, double *out) {

@@ -1,0 +1,83 @@
+"""Attention projections on the static FP8 path: o_proj (one Linear over its
+own quantization), the general shared-quant projection call, and
+cross-attention Q/K/V, where Q reads the query-side activation and K/V a
+different tensor, so Q does not share their quantization."""
+
+import numpy as np
+import pytest
+import torch
+
+import fp8_w8a8_static_b200 as fw
+import oracle
+import synth
+from _util import GEMM_REL_FRO, bits, codes, rel_fro, scalar
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _proj(N, d, seed):
+    return fw.fp8_rtn_quantize_weight(synth.normal((N, d), 0.02, seed, DEV))
+
+
+def _ref(p):
+    return codes(p[0]), p[1].item()
+
+
+def test_o_proj_single_linear():
+    M, d = 2048, 3072
+    x = synth.activation_with_outliers(M, d, 5, 3, 0, DEV)
+    s = oracle.f32(0.03)
+    wo = _proj(d, d, 501)
+    (y,) = fw.fp8_shared_quant_linears(x, scalar(s, DEV), [wo])
+    rows = np.random.default_rng(5).choice(M, 8, replace=False)
+    ref = oracle.qkv_shared_quant(bits(x[rows]), s, [_ref(wo)])[0]
+    assert rel_fro(bits(y[rows]), ref) <= GEMM_REL_FRO
+
+
+def test_general_call_matches_qkv_shared_quant_bitwise():
+    M, d = 512, 3072
+    x = synth.activation_with_outliers(M, d, 5, 4, 0, DEV)
+    s = scalar(0.03, DEV)
+    wq, wk, wv = _proj(3072, d, 511), _proj(1024, d, 512), _proj(1024, d, 513)
+    a = fw.fp8_shared_quant_linears(x, s, [wq, wk, wv])
+    b = fw.qkv_shared_quant(x, s, *wq, *wk, *wv)
+    for t, r in zip(a, b):
+        assert torch.equal(t, r)
+
+
+def test_cross_attention_projections():
+    Mq, Mkv, d = 4096, 1024, 3072   # generation-tower queries over understanding-tower context
+    x = synth.activation_with_outliers(Mq, d, 5, 5, 0, DEV)
+    ctx = synth.activation_with_outliers(Mkv, d, 5, 6, 0, DEV)
+    s_q, s_kv = oracle.f32(0.031), oracle.f32(0.027)
+    wq, wk, wv = _proj(3072, d, 521), _proj(1024, d, 522), _proj(1024, d, 523)
+    ws = torch.empty(fw.load().cross_attention_qkv_static_fp8_workspace(Mq, Mkv, d),
+                     dtype=torch.uint8, device=DEV)
+    fw.launch_log_clear()
+    q, k, v = fw.cross_attention_qkv_static_fp8(x, ctx, scalar(s_q, DEV), *wq, scalar(s_kv, DEV),
+                                                *wk, *wv, workspace=ws)
+    log = fw.launch_log()
+    kinds = [r[0] for r in log]
+    assert kinds == [fw.KIND_QUANT, fw.KIND_GEMM, fw.KIND_QUANT, fw.KIND_GEMM, fw.KIND_GEMM]
+    xq_ptr, ctxq_ptr = log[0][3], log[2][3]
+    assert log[0][1] == x.data_ptr() and log[2][1] == ctx.data_ptr()
+    assert xq_ptr != ctxq_ptr                        # Q does not share K/V's quantization
+    assert log[1][1] == xq_ptr
+    assert log[3][1] == ctxq_ptr and log[4][1] == ctxq_ptr   # K and V share one
+    rq = np.random.default_rng(6).choice(Mq, 6, replace=False)
+    rk = np.random.default_rng(7).choice(Mkv, 6, replace=False)
+    ref_q = oracle.qkv_shared_quant(bits(x[rq]), s_q, [_ref(wq)])[0]
+    ref_k, ref_v = oracle.qkv_shared_quant(bits(ctx[rk]), s_kv, [_ref(wk), _ref(wv)])
+    assert rel_fro(bits(q[rq]), ref_q) <= GEMM_REL_FRO
+    assert rel_fro(bits(k[rk]), ref_k) <= GEMM_REL_FRO
+    assert rel_fro(bits(v[rk]), ref_v) <= GEMM_REL_FRO
+    for t in (q, k, v):
+        assert t.is_contiguous()
+
+
+def test_kv_input_scales_checked_at_load():
+    s = scalar(0.027, DEV)
+    assert fw.fp8_check_shared_input_scale([s, s.clone()]) == fw.OK
+    other = scalar(0.031, DEV)
+    assert fw.fp8_check_shared_input_scale([s, other]) == fw.ERR_SCALE_MISMATCH

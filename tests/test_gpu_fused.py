@@ -99,3 +99,20 @@ def test_fused_mlp_c0_against_oracle():
                            codes(w["wu"][0]), w["wu"][1].item(), s_down, codes(w["wd"][0]),
                            w["wd"][1].item())
     assert rel_fro(bits(y), ref) <= GEMM_REL_FRO
+
+
+@pytest.mark.parametrize("alpha,beta,limit", [(1.702, 1.0, 7.0), (1.0, 1.0, None)])
+def test_fused_variant_equals_unfused_variant(alpha, beta, limit):
+    M, K, I = 1024, 3072, 1024
+    x, s_in, xq, wg, s_wg, wu, s_wu = _inputs(M, K, I, 77)
+    s_down = scalar(0.004, DEV)
+    act = fw.swiglu(alpha, beta, limit)
+    g = fw.fp8_linear_static(xq, wg, s_in, s_wg)
+    u = fw.fp8_linear_static(xq, wu, s_in, s_wu)
+    h_ref = fw.swiglu_2in_fp8(g, u, s_down, act)
+    h = fw.fp8_gate_up_swiglu_static(xq, wg, wu, s_in, s_wg, s_wu, s_down, act)
+    torch.cuda.synchronize()
+    assert torch.equal(h.view(torch.uint8), h_ref.view(torch.uint8))
+    # and differs from plain SwiGLU, so the descriptor reached the kernel
+    h_plain = fw.fp8_gate_up_swiglu_static(xq, wg, wu, s_in, s_wg, s_wu, s_down)
+    assert not torch.equal(h.view(torch.uint8), h_plain.view(torch.uint8))

@@ -88,3 +88,39 @@ def test_noncontiguous_refused():
 def test_empty():
     g = torch.empty(0, dtype=torch.bfloat16, device=DEV)
     assert fw.silu_mul_2in_fp8(g, g, scalar(1.0, DEV)).numel() == 0
+
+
+# ------------------------------------------------------------------ variants
+
+VARIANTS = [(1.702, 1.0, 7.0), (1.702, 0.0, None), (1.0, 1.0, None), (1.0, 0.0, 2.0)]
+
+
+def test_variant_defaults_bitwise_equal_plain():
+    g = synth.normal((256, 704), 2.0, 21, DEV)
+    u = synth.normal((256, 704), 1.0, 22, DEV)
+    s = scalar(0.0213, DEV)
+    plain = fw.silu_mul_2in_fp8(g, u, s)
+    assert torch.equal(fw.swiglu_2in_fp8(g, u, s).view(torch.uint8), plain.view(torch.uint8))
+    assert torch.equal(fw.swiglu_2in_fp8(g, u, s, fw.swiglu()).view(torch.uint8),
+                       plain.view(torch.uint8))
+
+
+@pytest.mark.parametrize("alpha,beta,limit", VARIANTS)
+def test_variant_against_oracle(alpha, beta, limit):
+    g = synth.normal((512, 1000), 4.0, 23, DEV)
+    u = synth.normal((512, 1000), 3.0, 24, DEV)
+    s = oracle.f32(0.05)
+    h = codes(fw.swiglu_2in_fp8(g, u, scalar(s, DEV), fw.swiglu(alpha, beta, limit)))
+    ref = oracle.swiglu_2in(bits(g), bits(u), s, alpha, beta, limit)
+    _compare(h, ref)
+    # the fused [M, 2I] form of the oracle agrees too
+    gu = np.concatenate([bits(g), bits(u)], axis=1)
+    _compare(h, oracle.swiglu_fused(gu, s, alpha, beta, limit))
+
+
+def test_variant_bad_descriptor_refused():
+    g = synth.normal((8, 16), 1.0, 25, DEV)
+    with pytest.raises(fw.FP8WSError):
+        fw.swiglu_2in_fp8(g, g, scalar(1.0, DEV), fw.swiglu(1.0, 0.0, -1.0))
+    with pytest.raises(fw.FP8WSError):
+        fw.swiglu_2in_fp8(g, g, scalar(1.0, DEV), fw.swiglu(float("nan"), 0.0, None))

@@ -441,3 +441,80 @@ def test_gated_mlp_brute_force_tiny():
     rel = np.linalg.norm(yv - ref) / np.linalg.norm(ref)
     assert rel < 1e-2
     assert np.isfinite(yv).all() and np.abs(yv).max() > 0
+
+
+# ---------------------------------------------------------- SwiGLU variants
+
+
+def _gu(seed, rows=16, cols=512, gstd=3.0):
+    g = bits_of(synth.normal((rows, cols), gstd, seed))
+    u = bits_of(synth.normal((rows, cols), 2.0, seed + 1))
+    return g, u
+
+
+def test_swiglu_variant_defaults_equal_plain():
+    """alpha = 1, beta = 0 and no limit is plain SwiGLU, bit for bit."""
+    g, u = _gu(40)
+    s = oracle.f32(0.017)
+    assert np.array_equal(oracle.swiglu_2in(g, u, s), oracle.silu_mul_2in(g, u, s))
+
+
+@pytest.mark.parametrize("alpha,beta,limit", [(1.702, 1.0, 7.0), (1.702, 0.0, None),
+                                              (1.0, 1.0, None), (1.0, 0.0, 2.0)])
+def test_swiglu_variant_two_input_equals_fused(alpha, beta, limit):
+    g, u = _gu(41)
+    s = oracle.f32(0.031)
+    h2 = oracle.swiglu_2in(g, u, s, alpha, beta, limit)
+    hf = oracle.swiglu_fused(np.concatenate([g, u], axis=1), s, alpha, beta, limit)
+    assert np.array_equal(h2, hf)
+
+
+def test_swiglu_variant_independent_form():
+    """Same variant written another way (tanh-form sigmoid, numpy clamps)."""
+    g, u = _gu(42)
+    alpha, beta, limit, s = 1.702, 1.0, 7.0, oracle.f32(0.05)
+    h = oracle.swiglu_2in(g, u, s, alpha, beta, limit)
+    gv = np.minimum(oracle.bf16_to_f64(g), limit)
+    uv = np.clip(oracle.bf16_to_f64(u), -limit, limit)
+    v = gv * (1.0 + np.tanh(alpha * gv / 2.0)) / 2.0 * (uv + beta) / float(s)
+    want = torch_e4m3(np.clip(v, -448, 448).astype(np.float32))
+    assert (h != want).mean() < 1e-3
+    # and each term matters: dropping the offset, the gain or the clamp changes codes
+    assert not np.array_equal(h, oracle.swiglu_2in(g, u, s, alpha, 0.0, limit))
+    assert not np.array_equal(h, oracle.swiglu_2in(g, u, s, 1.0, beta, limit))
+    assert not np.array_equal(h, oracle.swiglu_2in(g, u, s, alpha, beta, None))
+
+
+def test_swiglu_variant_closed_forms():
+    s = 1.0
+    big = bits_of(torch.full((4,), 20.0).to(torch.bfloat16))
+    one = bits_of(torch.full((4,), 1.0).to(torch.bfloat16))
+    # the clamp: gate 20 limited to 7, up 1: 7 sigmoid(7 alpha) (1 + beta)
+    h = oracle.swiglu_2in(big, one, s, 1.702, 1.0, 7.0)
+    want = oracle.quant_f64(7.0 / (1.0 + np.exp(-7.0 * np.float32(1.702).item())) * 2.0, 1.0)
+    assert np.all(h == want)
+    # up equal to -beta gives zero
+    neg = bits_of(torch.full((4,), -1.0).to(torch.bfloat16))
+    assert np.all((oracle.swiglu_2in(one, neg, s, 1.0, 1.0, None) & 0x7F) == 0)
+
+
+# ------------------------------------------------------ attention projections
+
+
+def test_cross_attention_reduces_to_self_attention():
+    """With ctx = x and equal scales the cross-attention projections are the
+    shared-quant Q/K/V; with a different context K and V change, Q does not."""
+    d = synth.c3_qkv(n_calib=0)
+    x = bits_of(d["x"][:24].contiguous())
+    ctx = bits_of(d["x"][100:124].contiguous())
+    s = oracle.f32(0.04)
+    proj = [oracle.rtn_weight(bits_of(d[n][:32].contiguous())) for n in ("wq", "wk", "wv")]
+    self_q, self_k, self_v = oracle.qkv_shared_quant(x, s, proj)
+    q, k, v = oracle.cross_attention_qkv(x, x, s, proj[0], s, proj[1], proj[2])
+    assert np.array_equal(q, self_q) and np.array_equal(k, self_k) and np.array_equal(v, self_v)
+    q2, k2, v2 = oracle.cross_attention_qkv(x, ctx, s, proj[0], oracle.f32(0.05), proj[1], proj[2])
+    assert np.array_equal(q2, self_q)
+    assert not np.array_equal(k2, self_k) and not np.array_equal(v2, self_v)
+    # K from ctx equals a plain quantize-then-Linear of ctx at s_kv
+    assert np.array_equal(k2, oracle.linear(oracle.quantize(ctx, oracle.f32(0.05)), *proj[1][:1],
+                                            oracle.f32(0.05), proj[1][1]))
