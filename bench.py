@@ -54,6 +54,12 @@ CALIB_BATCHES = 16
 CALIB_ROWS = 256
 
 
+# DRAM bytes (read + write) per launch of the dominant kernel, from an ncu
+# capture of the same kernel build on the same shape (profiles/).  None when
+# the kernel has changed since the capture.
+TRAFFIC = {}
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -196,24 +202,25 @@ def build_plan(fw, layers, bufs, stream_handle, fused):
         M = L.M
         xq, h = b["xq"].data_ptr(), b["h"].data_ptr()
         s_in, s_down = L.s_in.data_ptr(), L.s_down.data_ptr()
-        plan.append(("quant", lib.fp8_quant_static,
+        tw = "@" + L.tower
+        plan.append(("quant" + tw, lib.fp8_quant_static,
                      (L.x.data_ptr(), M * D, s_in, xq, stream_handle), 3 * M * D, 0))
         if fused:
-            plan.append(("gate_up_swiglu", lib.fp8_gate_up_swiglu_static,
+            plan.append(("gate_up_swiglu" + tw, lib.fp8_gate_up_swiglu_static,
                          (xq, L.wg.data_ptr(), L.wu.data_ptr(), M, I, D, s_in, L.s_wg.data_ptr(),
                           L.s_wu.data_ptr(), s_down, None, h, stream_handle),
                          M * D + 2 * I * D + M * I, 4 * M * I * D))
         else:
             g, u = b["g"].data_ptr(), b["u"].data_ptr()
-            plan.append(("gemm", lib.fp8_linear_static,
+            plan.append(("gemm_gate" + tw, lib.fp8_linear_static,
                          (xq, L.wg.data_ptr(), M, I, D, s_in, L.s_wg.data_ptr(), g, stream_handle),
                          M * D + I * D + 2 * M * I, 2 * M * I * D))
-            plan.append(("gemm", lib.fp8_linear_static,
+            plan.append(("gemm_up" + tw, lib.fp8_linear_static,
                          (xq, L.wu.data_ptr(), M, I, D, s_in, L.s_wu.data_ptr(), u, stream_handle),
                          M * D + I * D + 2 * M * I, 2 * M * I * D))
-            plan.append(("swiglu", lib.silu_mul_2in_fp8, (g, u, M * I, s_down, h, stream_handle),
+            plan.append(("swiglu" + tw, lib.silu_mul_2in_fp8, (g, u, M * I, s_down, h, stream_handle),
                          5 * M * I, 0))
-        plan.append(("gemm", lib.fp8_linear_static,
+        plan.append(("gemm_down" + tw, lib.fp8_linear_static,
                      (h, L.wd.data_ptr(), M, D, I, s_down, L.s_wd.data_ptr(), L.y.data_ptr(),
                       stream_handle),
                      M * I + D * I + 2 * M * D, 2 * M * D * I))
@@ -640,19 +647,28 @@ def main():
             d["tflops"] = flops / (ms / 1e3) / 1e12
         d["gbs"] = nbytes / (ms / 1e3) / 1e9
         comp[kind] = d
-    # the dominant kernel: largest share of the pass; all its launches, flop-weighted
+    # the dominant kernel: the launch shape with the largest share of the pass
     tensor_kinds = [k for k in per_kind if per_kind[k][3]]
     dom = max(tensor_kinds, key=lambda k: per_kind[k][0])
     fp8_peak = 2.0 * pk["bf16_sustained"]
-    achieved = per_kind[dom][3] / (per_kind[dom][0] / 1e3) / 1e12
-    names = {"gemm": "fp8_gemm_kernel / fp8_gemm_pair_kernel",
-             "gate_up_swiglu": "fp8_dual_swiglu_pair_kernel (gate/up GEMMs + SwiGLU-quant)"}
+    ms, n, _, flops = per_kind[dom]
+    achieved = (flops / n) / (ms / n / 1e3) / 1e12
+    kind, tower = dom.split("@")
+    mrows = dict(TOWERS)[tower]
+    names = {"gemm_down": f"fp8_gemm_pair_kernel, down projection M={mrows} N={D} K={I}",
+             "gemm_gate": f"fp8_gemm_pair_kernel, gate projection M={mrows} N={I} K={D}",
+             "gemm_up": f"fp8_gemm_pair_kernel, up projection M={mrows} N={I} K={D}",
+             "gate_up_swiglu": f"fp8_dual_swiglu_pair_kernel (gate/up GEMMs + SwiGLU-quant), "
+                               f"M={mrows} I={I} K={D}"}
     roofline = {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
-                "frac": achieved / fp8_peak, "traffic": None,
-                "kernel": f"{names[dom]}, all launches of the pass, flop-weighted",
+                "frac": achieved / fp8_peak, "traffic": TRAFFIC.get(dom),
+                "kernel": f"{names[kind]}, {tower} tower, {n // args.steps} launches per step, "
+                          f"{flops / n / 1e9:.1f} GFLOP and {per_kind[dom][2] / n / 1e6:.1f} MB "
+                          "algorithmic per launch",
+                "launch_us": ms / n * 1e3,
                 "peak_source": f"{pk['source']}: bf16 sustained {pk['bf16_sustained']} TFLOP/s x 2 (nominal fp8/bf16 ratio)"}
-    for k in ("swiglu", "quant"):
-        if k in comp:
+    for k in list(comp):
+        if k.startswith(("swiglu", "quant")) and isinstance(comp[k], dict):
             comp[k]["hbm_frac"] = comp[k]["gbs"] / pk["hbm"]
     all_flops = sum(v[3] for v in per_kind.values())
     all_tensor_ms = sum(per_kind[k][0] for k in tensor_kinds)

@@ -29,7 +29,8 @@ __all__ = [
     "fp8_gate_up_swiglu_static", "gated_mlp_static_fp8_fused", "swiglu_2in_fp8", "swiglu",
     "gated_mlp_static_fp8_fused_workspace",
     "qkv_shared_quant", "qkv_shared_quant_workspace", "fp8_shared_quant_linears",
-    "cross_attention_qkv_static_fp8",
+    "cross_attention_qkv_static_fp8", "fp8_quant_per_token", "fp8_linear_scaled",
+    "silu_mul_2in_fp8_per_token", "gated_mlp_per_token_fp8",
     "fp8_check_shared_input_scale", "fp8_absmax_bf16", "fp8_silu_mul_absmax",
     "fp8_observer_scale", "fp8_rtn_quantize_weight",
     "device_check", "device_status", "launch_count", "launch_log", "launch_log_clear",
@@ -110,6 +111,13 @@ _SIGS = {
                                                       _P, _P]),
     "qkv_shared_quant": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _I64, _P, _P, _I64, _P, _P, _I64,
                                         _P, _P, _P, _P, _P, _P]),
+    "fp8_quant_per_token": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P]),
+    "fp8_linear_scaled": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, ctypes.c_int, _P,
+                                         ctypes.c_int, _P, _P]),
+    "silu_mul_2in_fp8_per_token": (ctypes.c_int, [_P, _P, _I64, _I64, _P, _P, _P]),
+    "gated_mlp_per_token_fp8_workspace": (ctypes.c_size_t, [_I64, _I64, _I64]),
+    "gated_mlp_per_token_fp8": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P,
+                                               _P, _P]),
     "fp8_check_shared_input_scale": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int,
                                                     _P]),
     "fp8_absmax_bf16": (ctypes.c_int, [_P, _I64, _P, _P]),
@@ -452,6 +460,78 @@ def cross_attention_qkv_static_fp8(x, ctx, s_q, wq, s_wq, s_kv, wk, s_wk, wv, s_
             _dev_ptr(workspace, "workspace", (torch.uint8,)), _bf16(q, "q"), _bf16(k, "k"),
             _bf16(v, "v"), _stream(stream)), "cross_attention_qkv_static_fp8")
     return q, k, v
+
+
+# -------------------------------------------- per-channel / per-token scales
+
+
+def fp8_quant_per_token(x: torch.Tensor, out=None, scales=None, stream=None):
+    """(xq, s): one scale per row of x [rows, K], computed at run time
+    (per-token for activations, per-channel RTN for weights [N, K])."""
+    lib = load()
+    rows, K = x.shape
+    if out is None:
+        out = torch.empty((rows, K), dtype=FP8, device=x.device)
+    if scales is None:
+        scales = torch.empty(rows, dtype=torch.float32, device=x.device)
+    with _device_of(x):
+        _check(lib.fp8_quant_per_token(_bf16(x, "x"), rows, K, _dev_ptr(scales, "s", (torch.float32,)),
+                                       _fp8(out, "out"), _stream(stream)), "fp8_quant_per_token")
+    return out, scales
+
+
+def fp8_linear_scaled(xq, wq, s_x, s_w, out=None, stream=None) -> torch.Tensor:
+    """Linear with vector scales: s_x of M values (per token) or 1, s_w of N
+    values (per output channel) or 1."""
+    lib = load()
+    M, K = xq.shape
+    N = wq.shape[0]
+    if s_x.numel() not in (1, M) or s_w.numel() not in (1, N):
+        raise ValueError("s_x must hold 1 or M values, s_w 1 or N values")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    with _device_of(xq):
+        _check(lib.fp8_linear_scaled(_fp8(xq, "xq"), _fp8(wq, "wq"), M, N, K, _f32(s_x, "s_x"),
+                                     int(s_x.numel() == M and M > 1), _f32(s_w, "s_w"),
+                                     int(s_w.numel() == N and N > 1), _bf16(out, "out"),
+                                     _stream(stream)), "fp8_linear_scaled")
+    return out
+
+
+def silu_mul_2in_fp8_per_token(g, u, out=None, scales=None, stream=None):
+    """(h, s): SiLU(G) * U quantized with one scale per row, computed at run time."""
+    lib = load()
+    rows, I = g.shape
+    if out is None:
+        out = torch.empty((rows, I), dtype=FP8, device=g.device)
+    if scales is None:
+        scales = torch.empty(rows, dtype=torch.float32, device=g.device)
+    with _device_of(g):
+        _check(lib.silu_mul_2in_fp8_per_token(_bf16(g, "g"), _bf16(u, "u"), rows, I,
+                                              _dev_ptr(scales, "s", (torch.float32,)),
+                                              _fp8(out, "out"), _stream(stream)),
+               "silu_mul_2in_fp8_per_token")
+    return out, scales
+
+
+def gated_mlp_per_token_fp8(x, wg, s_wg, wu, s_wu, wd, s_wd, workspace=None, out=None,
+                            stream=None) -> torch.Tensor:
+    """Gated MLP with per-channel weight scales and per-token activation scales."""
+    lib = load()
+    M, d = x.shape
+    I = wg.shape[0]
+    need = lib.gated_mlp_per_token_fp8_workspace(M, d, I)
+    if workspace is None:
+        workspace = _workspace(need, x.device)
+    if out is None:
+        out = torch.empty((M, d), dtype=torch.bfloat16, device=x.device)
+    with _device_of(x):
+        _check(lib.gated_mlp_per_token_fp8(
+            _bf16(x, "x"), M, d, I, _fp8(wg, "wg"), _f32(s_wg, "s_wg"), _fp8(wu, "wu"),
+            _f32(s_wu, "s_wu"), _fp8(wd, "wd"), _f32(s_wd, "s_wd"),
+            _dev_ptr(workspace, "workspace", (torch.uint8,)), _bf16(out, "out"), _stream(stream)),
+            "gated_mlp_per_token_fp8")
+    return out
 
 
 # ---------------------------------------------------------------- load time

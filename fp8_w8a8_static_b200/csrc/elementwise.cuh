@@ -311,3 +311,85 @@ __global__ void rtn_scale_kernel(float *__restrict__ s) {
 }
 
 }  // namespace fp8ws
+
+// --------------------------------------------- per-token / per-channel rows
+namespace fp8ws {
+
+constexpr int kRowThreads = 256;
+
+__device__ __forceinline__ float block_max_rows(float m, float *red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  m = red[0];
+#pragma unroll
+  for (int w = 1; w < kRowThreads / 32; ++w) m = fmaxf(m, red[w]);
+  return m;
+}
+
+// One block per row of a [rows, K] BF16 tensor (K % 8 == 0): s[r] = max|x| /
+// 448 (1 for an all-zero row), codes q(x, s[r]) as the static quantizer.
+// Per-token scales for activations, per-channel scales for weights.
+__global__ void __launch_bounds__(kRowThreads) quant_rows_kernel(
+    const uint16_t *__restrict__ x, int K, float *__restrict__ s_out, uint8_t *__restrict__ q) {
+  __shared__ float red[kRowThreads / 32];
+  pdl_launch_dependents();
+  pdl_wait();
+  const int64_t row = blockIdx.x;
+  const uint4 *xv = reinterpret_cast<const uint4 *>(x + row * K);
+  uint2 *qv = reinterpret_cast<uint2 *>(q + row * K);
+  const int nvec = K >> 3;
+  float m = 0.0f;
+  for (int i = threadIdx.x; i < nvec; i += kRowThreads) m = absmax8(__ldg(xv + i), m);
+  m = block_max_rows(m, red);
+  const float s = m > 0.0f ? __fdiv_rn(m, 448.0f) : 1.0f;
+  const float r = __frcp_rn(s);
+  if (threadIdx.x == 0) s_out[row] = s;
+  for (int i = threadIdx.x; i < nvec; i += kRowThreads) qv[i] = quant8(__ldg(xv + i), s, r);
+}
+
+// One block per row of G, U [rows, I] (I % 8 == 0, I <= kMaxRowI): v =
+// SiLU(g) * u in fp32 kept in shared memory, s[r] = max|v| / 448 (1 for an
+// all-zero row), h = E4M3(v * (1/s)).
+constexpr int kMaxRowI = 16384;
+
+__global__ void __launch_bounds__(kRowThreads) silu_mul_rows_kernel(
+    const uint16_t *__restrict__ g, const uint16_t *__restrict__ u, int I,
+    float *__restrict__ s_out, uint8_t *__restrict__ h) {
+  extern __shared__ float vrow[];
+  __shared__ float red[kRowThreads / 32];
+  pdl_launch_dependents();
+  pdl_wait();
+  const int64_t row = blockIdx.x;
+  const uint4 *gv = reinterpret_cast<const uint4 *>(g + row * I);
+  const uint4 *uv = reinterpret_cast<const uint4 *>(u + row * I);
+  const int nvec = I >> 3;
+  float m = 0.0f;
+  for (int i = threadIdx.x; i < nvec; i += kRowThreads) {
+    const uint4 a = ld_stream(gv + i), b = ld_stream(uv + i);
+    float v[8] = {silu_mul(bf16_lo(a.x), bf16_lo(b.x)), silu_mul(bf16_hi(a.x), bf16_hi(b.x)),
+                  silu_mul(bf16_lo(a.y), bf16_lo(b.y)), silu_mul(bf16_hi(a.y), bf16_hi(b.y)),
+                  silu_mul(bf16_lo(a.z), bf16_lo(b.z)), silu_mul(bf16_hi(a.z), bf16_hi(b.z)),
+                  silu_mul(bf16_lo(a.w), bf16_lo(b.w)), silu_mul(bf16_hi(a.w), bf16_hi(b.w))};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      vrow[i * 8 + e] = v[e];
+      m = fmaxf(m, fabsf(v[e]));
+    }
+  }
+  m = block_max_rows(m, red);
+  const float s = m > 0.0f ? __fdiv_rn(m, 448.0f) : 1.0f;
+  const float inv = __frcp_rn(s);
+  if (threadIdx.x == 0) s_out[row] = s;
+  uint2 *hv = reinterpret_cast<uint2 *>(h + row * I);
+  for (int i = threadIdx.x; i < nvec; i += kRowThreads) {
+    const float *v = vrow + i * 8;
+    uint2 o;
+    o.x = pack4(cvt_e4m3x2(v[0] * inv, v[1] * inv), cvt_e4m3x2(v[2] * inv, v[3] * inv));
+    o.y = pack4(cvt_e4m3x2(v[4] * inv, v[5] * inv), cvt_e4m3x2(v[6] * inv, v[7] * inv));
+    st_stream(hv + i, o);
+  }
+}
+
+}  // namespace fp8ws

@@ -52,7 +52,7 @@ enum { kKindQuant = 1, kKindGemm = 2, kKindSwiglu = 3, kKindCalib = 4, kKindDual
 struct DeviceInfo {
   int checked = 0;  // 0 unknown, 1 sm_100, -1 other
   int sms = 0;
-  unsigned gemm_attr_set = 0;  // bit per GEMM instantiation
+  unsigned gemm_attr_set = 0;  // bit per kernel whose attributes were set on this device
   int pair_clusters = 0;       // CTA pairs of the pair GEMM resident at once
   int dual_clusters = 0;       // CTA pairs of the gate/up dual GEMM resident at once
 };
@@ -222,11 +222,11 @@ int launch_gemm_cfg(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int M, 
 // (an empty tensor's data pointer).
 // CTA-pair GEMM: one cluster of two CTAs per TPC, persistent over 256 x 256
 // tiles.  The grid holds as many pairs as can be resident at once.
-template <int STAGES, int BIT>
+template <int STAGES, int BIT, int SCALE_MODE = 0>
 int launch_gemm_pair(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int M, int N, int K,
                      const float *s_in, const float *s_w, uint16_t *y, cudaStream_t st) {
   using C = PairCfg<STAGES>;
-  auto kern = fp8_gemm_pair_kernel<STAGES>;
+  auto kern = fp8_gemm_pair_kernel<STAGES, SCALE_MODE>;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -685,6 +685,105 @@ int cross_attention_qkv_static_fp8(const uint16_t *x, int64_t Mq, const uint16_t
   const float *skv[2] = {s_wk, s_wv};
   uint16_t *ykv[2] = {k, v};
   return fp8_shared_quant_linears(ctx, Mkv, dm, s_kv, 2, wkv, nkv, skv, ykv, ws_kv, stream);
+}
+
+int fp8_quant_per_token(const uint16_t *x, int64_t rows, int64_t K, float *s, uint8_t *xq,
+                        void *stream) {
+  if (rows < 0 || K < 0 || K % 8 != 0 || rows >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+    return FP8WS_ERR_SHAPE;
+  if (rows == 0 || K == 0) return FP8WS_OK;
+  if (!x || !s || !xq) return FP8WS_ERR_NULL;
+  if (!aligned16(x) || !aligned16(xq)) return FP8WS_ERR_ALIGN;
+  DeviceInfo *d;
+  int rc = device_info(&d);
+  if (rc) return rc;
+  cudaStream_t st = as_stream(stream);
+  if (launch_ex(quant_rows_kernel, dim3(static_cast<unsigned>(rows)), dim3(kRowThreads), 0, st, 1,
+                x, static_cast<int>(K), s, xq) != cudaSuccess)
+    return FP8WS_ERR_CUDA;
+  log_launch(kKindQuant, x, nullptr, xq);
+  return launch_status();
+}
+
+int fp8_linear_scaled(const uint8_t *xq, const uint8_t *wq, int64_t M, int64_t N, int64_t K,
+                      const float *s_x, int x_per_row, const float *s_w, int w_per_col,
+                      uint16_t *y, void *stream) {
+  int rc = check_gemm_args(xq, wq, M, N, K, s_x, s_w, y);
+  if (rc) return rc;
+  DeviceInfo *d;
+  rc = device_info(&d);
+  if (rc) return rc;
+  if (M == 0) return FP8WS_OK;
+  cudaStream_t st = as_stream(stream);
+  const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
+  const int mode = (x_per_row ? kScaleRowVec : 0) | (w_per_col ? kScaleColVec : 0);
+  switch (mode) {
+    case 0: return launch_gemm_pair<6, 3, 0>(d, xq, wq, m, n, k, s_x, s_w, y, st);
+    case 1: return launch_gemm_pair<6, 5, 1>(d, xq, wq, m, n, k, s_x, s_w, y, st);
+    case 2: return launch_gemm_pair<6, 6, 2>(d, xq, wq, m, n, k, s_x, s_w, y, st);
+    default: return launch_gemm_pair<6, 7, 3>(d, xq, wq, m, n, k, s_x, s_w, y, st);
+  }
+}
+
+int silu_mul_2in_fp8_per_token(const uint16_t *g, const uint16_t *u, int64_t rows, int64_t I,
+                               float *s, uint8_t *h, void *stream) {
+  if (rows < 0 || I < 0 || I % 8 != 0 || I > kMaxRowI || rows >= (int64_t(1) << 31))
+    return FP8WS_ERR_SHAPE;
+  if (rows == 0 || I == 0) return FP8WS_OK;
+  if (!g || !u || !s || !h) return FP8WS_ERR_NULL;
+  if (!aligned16(g) || !aligned16(u) || !aligned16(h)) return FP8WS_ERR_ALIGN;
+  DeviceInfo *d;
+  int rc = device_info(&d);
+  if (rc) return rc;
+  const size_t smem = static_cast<size_t>(I) * sizeof(float);
+  if (!(d->gemm_attr_set & (1u << 8))) {
+    if (cudaFuncSetAttribute(silu_mul_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kMaxRowI * sizeof(float)) != cudaSuccess)
+      return FP8WS_ERR_CUDA;
+    d->gemm_attr_set |= 1u << 8;
+  }
+  cudaStream_t st = as_stream(stream);
+  if (launch_ex(silu_mul_rows_kernel, dim3(static_cast<unsigned>(rows)), dim3(kRowThreads), smem,
+                st, 1, g, u, static_cast<int>(I), s, h) != cudaSuccess)
+    return FP8WS_ERR_CUDA;
+  log_launch(kKindSwiglu, g, u, h);
+  return launch_status();
+}
+
+size_t gated_mlp_per_token_fp8_workspace(int64_t M, int64_t d, int64_t I) {
+  if (M < 0 || d < 0 || I < 0) return 0;
+  const size_t m = static_cast<size_t>(M);
+  return round256(m * d) + round256(m * 4) + 2 * round256(m * I * 2) + round256(m * I) +
+         round256(m * 4);
+}
+
+int gated_mlp_per_token_fp8(const uint16_t *x, int64_t M, int64_t dm, int64_t I,
+                            const uint8_t *Wg, const float *s_wg, const uint8_t *Wu,
+                            const float *s_wu, const uint8_t *Wd, const float *s_wd,
+                            void *workspace, uint16_t *y, void *stream) {
+  if (!Wg || !s_wg || !Wu || !s_wu || !Wd || !s_wd || (M != 0 && (!x || !y))) return FP8WS_ERR_NULL;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FP8WS_ERR_WORKSPACE;
+  if (M < 0 || dm % 16 != 0 || I % 16 != 0 || I > kMaxRowI) return FP8WS_ERR_SHAPE;
+  if (!aligned16(x)) return FP8WS_ERR_ALIGN;
+  const size_t m = static_cast<size_t>(M);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  uint8_t *xq = ws;
+  float *sx = reinterpret_cast<float *>(ws + round256(m * dm));
+  uint16_t *G = reinterpret_cast<uint16_t *>(reinterpret_cast<uint8_t *>(sx) + round256(m * 4));
+  uint16_t *U = reinterpret_cast<uint16_t *>(reinterpret_cast<uint8_t *>(G) + round256(m * I * 2));
+  uint8_t *H = reinterpret_cast<uint8_t *>(U) + round256(m * I * 2);
+  float *sh = reinterpret_cast<float *>(H + round256(m * I));
+  int rc = check_gemm_args(xq, Wg, M, I, dm, sx, s_wg, G);
+  if (!rc) rc = check_gemm_args(xq, Wu, M, I, dm, sx, s_wu, U);
+  if (!rc) rc = check_gemm_args(H, Wd, M, dm, I, sh, s_wd, y);
+  if (rc) return rc;
+  if (M == 0) return FP8WS_OK;
+  rc = fp8_quant_per_token(x, M, dm, sx, xq, stream);
+  if (!rc) rc = fp8_linear_scaled(xq, Wg, M, I, dm, sx, 1, s_wg, 1, G, stream);
+  if (!rc) rc = fp8_linear_scaled(xq, Wu, M, I, dm, sx, 1, s_wu, 1, U, stream);
+  if (!rc) rc = silu_mul_2in_fp8_per_token(G, U, M, I, sh, H, stream);
+  if (!rc) rc = fp8_linear_scaled(H, Wd, M, dm, I, sh, 1, s_wd, 1, y, stream);
+  return rc;
 }
 
 int fp8_check_shared_input_scale(const float *const *d_scales, int n, void *stream) {

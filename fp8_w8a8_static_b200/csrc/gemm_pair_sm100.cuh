@@ -24,6 +24,12 @@ namespace fp8ws {
 
 constexpr int kPairTile = 256;  // output rows and columns per CTA pair
 
+// Scale modes of the epilogue: bit 0 = one activation scale per row
+// (s_in[M], per token), bit 1 = one weight scale per column (s_w[N], per
+// channel); 0 = the static per-tensor scalars.
+constexpr int kScaleRowVec = 1;
+constexpr int kScaleColVec = 2;
+
 template <int STAGES_>
 struct PairCfg {
   static constexpr int STAGES = STAGES_;
@@ -41,7 +47,7 @@ struct PairCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
-template <int STAGES>
+template <int STAGES, int SCALE_MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
                          const __grid_constant__ CUtensorMap tm_b,
@@ -189,7 +195,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------ epilogue (both CTAs)
     const int ew = warp - 2;
     const int quarter = warp & 3;
-    const float scale = __ldg(s_in) * __ldg(s_w);
+    const float scale = (SCALE_MODE == 0) ? __ldg(s_in) * __ldg(s_w) : 0.0f;
     uint32_t it = 0, chunk = 0;
     for (int t = cluster; t < num_tiles; t += nclusters, ++it) {
       const TileCoord tc = tile_coord(t, num_m, num_n);
@@ -204,6 +210,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_after();
       const int row0 = tc.m * kPairTile + static_cast<int>(rank) * 128 + quarter * 32;
+      float row_scale = 0.0f;  // this thread's row factor (row0 + lane)
+      if (SCALE_MODE != 0) {
+        const int my_row = row0 + lane;
+        row_scale = (SCALE_MODE & kScaleRowVec) ? (my_row < M ? __ldg(s_in + my_row) : 0.0f)
+                                                : __ldg(s_in);
+        if (!(SCALE_MODE & kScaleColVec)) row_scale *= __ldg(s_w);
+      }
       const uint32_t t_row =
           tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kPairTile;
       constexpr int NCHUNK = kPairTile / C::EPI_COLS;
@@ -220,6 +233,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         const int col0 = tc.n * kPairTile + c * C::EPI_COLS;
         if (col0 >= N || row0 >= M) continue;  // whole chunk outside Y
+        // per-column scales of this chunk: lane l holds columns l and 32 + l
+        float cs0 = 0.0f, cs1 = 0.0f;
+        if (SCALE_MODE & kScaleColVec) {
+          cs0 = col0 + lane < N ? __ldg(s_w + col0 + lane) : 0.0f;
+          cs1 = col0 + 32 + lane < N ? __ldg(s_w + col0 + 32 + lane) : 0.0f;
+        }
         uint8_t *buf = sEpi + (ew * 2 + (chunk & 1u)) * C::EPI_BUF_BYTES;
         if (lane == 0) tma_store_wait_read<1>();
         __syncwarp();
@@ -227,15 +246,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const uint32_t *src = (j < 4) ? &r0[j * 8] : &r1[(j - 4) * 8];
+          float sc[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if (SCALE_MODE == 0) {
+              sc[e] = scale;
+            } else if (SCALE_MODE & kScaleColVec) {
+              const int cc = j * 8 + e;  // column within the chunk
+              sc[e] = row_scale * __shfl_sync(0xFFFFFFFFu, cc < 32 ? cs0 : cs1, cc & 31);
+            } else {
+              sc[e] = row_scale;
+            }
+          }
           uint4 v;
-          __nv_bfloat162 p0 = __floats2bfloat162_rn(__uint_as_float(src[0]) * scale,
-                                                    __uint_as_float(src[1]) * scale);
-          __nv_bfloat162 p1 = __floats2bfloat162_rn(__uint_as_float(src[2]) * scale,
-                                                    __uint_as_float(src[3]) * scale);
-          __nv_bfloat162 p2 = __floats2bfloat162_rn(__uint_as_float(src[4]) * scale,
-                                                    __uint_as_float(src[5]) * scale);
-          __nv_bfloat162 p3 = __floats2bfloat162_rn(__uint_as_float(src[6]) * scale,
-                                                    __uint_as_float(src[7]) * scale);
+          __nv_bfloat162 p0 = __floats2bfloat162_rn(__uint_as_float(src[0]) * sc[0],
+                                                    __uint_as_float(src[1]) * sc[1]);
+          __nv_bfloat162 p1 = __floats2bfloat162_rn(__uint_as_float(src[2]) * sc[2],
+                                                    __uint_as_float(src[3]) * sc[3]);
+          __nv_bfloat162 p2 = __floats2bfloat162_rn(__uint_as_float(src[4]) * sc[4],
+                                                    __uint_as_float(src[5]) * sc[5]);
+          __nv_bfloat162 p3 = __floats2bfloat162_rn(__uint_as_float(src[6]) * sc[6],
+                                                    __uint_as_float(src[7]) * sc[7]);
           v.x = *reinterpret_cast<uint32_t *>(&p0);
           v.y = *reinterpret_cast<uint32_t *>(&p1);
           v.z = *reinterpret_cast<uint32_t *>(&p2);

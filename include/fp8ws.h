@@ -305,6 +305,45 @@ FP8WS_API int cross_attention_qkv_static_fp8(const uint16_t *x, int64_t Mq, cons
                                              const float *s_wv, void *workspace, uint16_t *q,
                                              uint16_t *k, uint16_t *v, void *stream);
 
+/* ----------------------------------- per-channel / per-token scales (rows) */
+
+/*
+ * The finer-grained FP8 scheme of the exploratory builds ([MC] comparison
+ * report, table 3.2: per-channel weight, per-token activation scales).
+ *
+ * fp8_quant_per_token -- one scale per row of x [rows,K] BF16 (K % 8 == 0),
+ *   computed at run time: s[r] = max_k |x[r,k]| / 448 (IEEE fp32; 1 for an
+ *   all-zero row), xq[r,k] = E4M3_satRNE(x[r,k] / s[r]).  For activations the
+ *   rows are tokens; for weights [N,K] the rows are output channels (per-channel
+ *   RTN).  s: device, rows fp32 (written).  xq: device [rows,K] FP8.
+ * fp8_linear_scaled -- fp8_linear_static with vector scales:
+ *   y[m,n] = bf16( sx * sw * sum_k deq(xq[m,k]) deq(wq[n,k]) ), where sx is
+ *   s_x[m] if x_per_row else s_x[0], and sw is s_w[n] if w_per_col else s_w[0].
+ * silu_mul_2in_fp8_per_token -- SiLU(G) * U quantized with one scale per row,
+ *   computed at run time: v = SiLU(g) * u in fp32, s[r] = max |v| / 448 (1 for
+ *   an all-zero row), h = E4M3_satRNE(v / s[r]).  G, U: device [rows,I] BF16,
+ *   I % 8 == 0, I <= 16384.  s: device, rows fp32 (written).  h: [rows,I] FP8.
+ * gated_mlp_per_token_fp8 -- the gated MLP on this scheme: per-token X
+ *   quantization, gate and up GEMMs with (per-token x per-channel) scales,
+ *   per-token SwiGLU quantization, down GEMM likewise.  s_wg, s_wu: device [I]
+ *   fp32, s_wd: device [d] fp32 (per-channel).  workspace:
+ *   gated_mlp_per_token_fp8_workspace(M,d,I) bytes, 256-byte aligned:
+ *   Xq [M,d] | s_x [M] | G [M,I] | U [M,I] | H [M,I] | s_h [M], each region
+ *   256-byte aligned.
+ */
+FP8WS_API int fp8_quant_per_token(const uint16_t *x, int64_t rows, int64_t K, float *s,
+                                  uint8_t *xq, void *stream);
+FP8WS_API int fp8_linear_scaled(const uint8_t *xq, const uint8_t *wq, int64_t M, int64_t N,
+                                int64_t K, const float *s_x, int x_per_row, const float *s_w,
+                                int w_per_col, uint16_t *y, void *stream);
+FP8WS_API int silu_mul_2in_fp8_per_token(const uint16_t *g, const uint16_t *u, int64_t rows,
+                                         int64_t I, float *s, uint8_t *h, void *stream);
+FP8WS_API size_t gated_mlp_per_token_fp8_workspace(int64_t M, int64_t d, int64_t I);
+FP8WS_API int gated_mlp_per_token_fp8(const uint16_t *x, int64_t M, int64_t d, int64_t I,
+                                      const uint8_t *Wg, const float *s_wg, const uint8_t *Wu,
+                                      const float *s_wu, const uint8_t *Wd, const float *s_wd,
+                                      void *workspace, uint16_t *y, void *stream);
+
 /* ------------------------------------------------------------- load time */
 
 /*

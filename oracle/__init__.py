@@ -84,6 +84,12 @@ def lib():
             "oracle_silu_mul_2in": (None, [u16p, u16p, i64, f32, u8p]),
             "oracle_silu_and_mul_fused": (None, [u16p, i64, i64, f32, u8p]),
             "oracle_silu_mul_f64": (None, [dp, dp, i64, dp]),
+            "oracle_quantize_rows": (None, [u16p, i64, i64, ctypes.POINTER(ctypes.c_float), u8p]),
+            "oracle_linear_scaled": (None, [u8p, u8p, i64, i64, i64, ctypes.POINTER(ctypes.c_float),
+                                            ctypes.c_int, ctypes.POINTER(ctypes.c_float),
+                                            ctypes.c_int, u16p]),
+            "oracle_silu_mul_2in_rows": (None, [u16p, u16p, i64, i64, ctypes.POINTER(ctypes.c_float),
+                                                u8p]),
             "oracle_swiglu_2in": (None, [u16p, u16p, i64, f32, f32, f32, ctypes.c_int, f32, u8p]),
             "oracle_swiglu_fused": (None, [u16p, i64, i64, f32, f32, f32, ctypes.c_int, f32, u8p]),
             "oracle_requant_group_member": (None, [u8p, i64, f32, f32, u8p]),
@@ -238,6 +244,56 @@ def swiglu_fused(gu_bf16, s_down: float, alpha: float = 1.0, beta: float = 0.0,
                               int(limit is not None), 0.0 if limit is None else limit,
                               _p(h, ctypes.c_uint8))
     return h
+
+
+def quantize_rows(x_bf16):
+    """Per-row (per-token / per-channel) quantization of a [rows, K] tensor:
+    returns (codes, fp32 scales[rows])."""
+    x = _u16(x_bf16)
+    rows, K = x.shape
+    q = np.empty(x.shape, dtype=np.uint8)
+    s = np.empty(rows, dtype=np.float32)
+    lib().oracle_quantize_rows(_p(x, ctypes.c_uint16), rows, K, _p(s, ctypes.c_float),
+                               _p(q, ctypes.c_uint8))
+    return q, s
+
+
+def linear_scaled(xq, wq, sx, sw) -> np.ndarray:
+    """Linear with vector scales: sx per token (length M) or one value, sw per
+    output channel (length N) or one value."""
+    xq = _u8(xq)
+    wq = _u8(wq)
+    M, K = xq.shape
+    N = wq.shape[0]
+    sx = np.ascontiguousarray(np.atleast_1d(np.asarray(sx, dtype=np.float32)))
+    sw = np.ascontiguousarray(np.atleast_1d(np.asarray(sw, dtype=np.float32)))
+    y = np.empty((M, N), dtype=np.uint16)
+    lib().oracle_linear_scaled(_p(xq, ctypes.c_uint8), _p(wq, ctypes.c_uint8), M, N, K,
+                               _p(sx, ctypes.c_float), int(sx.size > 1), _p(sw, ctypes.c_float),
+                               int(sw.size > 1), _p(y, ctypes.c_uint16))
+    return y
+
+
+def silu_mul_2in_rows(g_bf16, u_bf16):
+    """Two-input SwiGLU with per-token FP8 output: (codes, fp32 scales[rows])."""
+    g = _u16(g_bf16)
+    u = _u16(u_bf16)
+    rows, I = g.shape
+    h = np.empty(g.shape, dtype=np.uint8)
+    s = np.empty(rows, dtype=np.float32)
+    lib().oracle_silu_mul_2in_rows(_p(g, ctypes.c_uint16), _p(u, ctypes.c_uint16), rows, I,
+                                   _p(s, ctypes.c_float), _p(h, ctypes.c_uint8))
+    return h, s
+
+
+def gated_mlp_per_token(x_bf16, wgq, s_wg, wuq, s_wu, wdq, s_wd):
+    """Gated MLP with per-channel weight scales (vectors) and per-token
+    activation scales computed at run time for X and for H."""
+    xq, sx = quantize_rows(x_bf16)
+    g = linear_scaled(xq, wgq, sx, s_wg)
+    u = linear_scaled(xq, wuq, sx, s_wu)
+    h, sh = silu_mul_2in_rows(g, u)
+    return linear_scaled(h, wdq, sh, s_wd)
 
 
 def requant_group_member(qw, s_i: float, s_max: float) -> np.ndarray:

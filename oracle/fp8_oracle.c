@@ -311,6 +311,61 @@ void oracle_silu_mul_f64(const double *g, const double *u, int64_t n, double *ou
 }
 
 /* ------------------------------------------------------------------------ */
+/* Per-channel weight / per-token activation scales ([MC] comparison report, */
+/* table 3.2: the exploratory per-row builds).  One scale per row of a       */
+/* [rows, K] tensor: s[r] = fp32(max_k |x[r,k]|) / 448 in fp32 (1 for an     */
+/* all-zero row, where every code is 0 whatever the scale), codes            */
+/* q(x[r,k], s[r]).  For weights the rows are output channels; for           */
+/* activations they are tokens, computed at run time.                       */
+/* ------------------------------------------------------------------------ */
+void oracle_quantize_rows(const uint16_t *x, int64_t rows, int64_t K, float *s, uint8_t *q) {
+  for (int64_t r = 0; r < rows; ++r) {
+    float amax = (float)oracle_absmax_bf16(x + r * K, K);
+    volatile float sr = amax / 448.0f;
+    float sv = (amax > 0.0f) ? (float)sr : 1.0f;
+    s[r] = sv;
+    oracle_quantize_bf16(x + r * K, K, sv, q + r * K);
+  }
+}
+
+/* Linear with vector scales: y[m,n] = bf16( sx[m] * sw[n] * sum_k ... ),    */
+/* sx of length M (per token) or 1, sw of length N (per channel) or 1.       */
+void oracle_linear_scaled(const uint8_t *xq, const uint8_t *wq, int64_t M, int64_t N, int64_t K,
+                          const float *sx, int x_per_row, const float *sw, int w_per_col,
+                          uint16_t *y) {
+  const double *cb = codebook();
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t m = 0; m < M; ++m) {
+    const uint8_t *xr = xq + m * K;
+    double a = (double)sx[x_per_row ? m : 0];
+    for (int64_t n = 0; n < N; ++n) {
+      const uint8_t *wr = wq + n * K;
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; ++k) acc += cb[xr[k]] * cb[wr[k]];
+      double scale = a * (double)sw[w_per_col ? n : 0]; /* exact: 24 x 24 bits */
+      y[m * N + n] = oracle_round_bf16(scale * acc);
+    }
+  }
+}
+
+/* Two-input SwiGLU with per-token FP8 output: v = SiLU(g) * u in fp64 per   */
+/* row, s[r] = fp32(max |v| / 448) (1 for an all-zero row), codes q64(v, s).  */
+void oracle_silu_mul_2in_rows(const uint16_t *g, const uint16_t *u, int64_t rows, int64_t I,
+                              float *s, uint8_t *h) {
+  for (int64_t r = 0; r < rows; ++r) {
+    double amax = 0.0;
+    for (int64_t i = 0; i < I; ++i) {
+      double gv = bf16_to_double(g[r * I + i]), uv = bf16_to_double(u[r * I + i]);
+      double v = fabs(gv / (1.0 + exp(-gv)) * uv);
+      if (v > amax) amax = v;
+    }
+    float sv = (amax > 0.0) ? (float)(amax / 448.0) : 1.0f;
+    s[r] = sv;
+    for (int64_t i = 0; i < I; ++i) h[r * I + i] = silu_mul_code(g[r * I + i], u[r * I + i], (double)sv);
+  }
+}
+
+/* ------------------------------------------------------------------------ */
 /* The re-quantization the fused loader did ([PR] Description):              */
 /*   qW' = FP8-round((s_i * deq(qW_i)) / max(s))                             */
 /* ------------------------------------------------------------------------ */

@@ -1,0 +1,84 @@
+"""Per-channel weight and per-token activation scales on the GPU against the
+oracle: row-wise quantization bit-exact (codes and scales), Linear with vector
+scales and the gated MLP on this scheme within the GEMM bar, per-token
+SwiGLU-quant within the SwiGLU bar."""
+
+import numpy as np
+import pytest
+import torch
+
+import fp8_w8a8_static_b200 as fw
+import oracle
+import synth
+from _util import (GEMM_REL_FRO, SWIGLU_MAX_FRAC, bits, code_step_diff, codes, from_codes,
+                   rel_fro, scalar)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.mark.parametrize("rows,K", [(1, 8), (7, 264), (300, 3072), (4096, 3072)])
+def test_quant_rows_bitexact(rows, K):
+    x = synth.activation_with_outliers(rows, K, 6, rows, 0, DEV)
+    if rows > 3:
+        x[2] = 0  # an all-zero row
+    q, s = fw.fp8_quant_per_token(x)
+    sample = np.arange(rows) if rows <= 300 else np.random.default_rng(1).choice(rows, 64, replace=False)
+    rq, rs = oracle.quantize_rows(bits(x[sample]))
+    assert np.array_equal(s.cpu().numpy()[sample], rs)
+    assert np.array_equal(codes(q[sample]), rq)
+
+
+def test_per_channel_weights_bitexact():
+    w = synth.normal((1024, 3072), 0.02, 71, DEV)
+    q, s = fw.fp8_quant_per_token(w)
+    rq, rs = oracle.quantize_rows(bits(w))
+    assert np.array_equal(s.cpu().numpy(), rs)
+    assert np.array_equal(codes(q), rq)
+
+
+@pytest.mark.parametrize("x_vec,w_vec", [(True, True), (True, False), (False, True), (False, False)])
+def test_linear_scaled(x_vec, w_vec):
+    M, N, K = 520, 776, 1024
+    x = synth.activation_with_outliers(M, K, 6, 9, 0, DEV)
+    w = synth.normal((N, K), 0.02, 72, DEV)
+    if x_vec:
+        xq, sx = fw.fp8_quant_per_token(x)
+    else:
+        sx = fw.fp8_observer_scale(fw.fp8_absmax_bf16(x))
+        xq = fw.fp8_quant_static(x, sx)
+    if w_vec:
+        wq, sw = fw.fp8_quant_per_token(w)
+    else:
+        wq, sw = fw.fp8_rtn_quantize_weight(w)
+    y = fw.fp8_linear_scaled(xq, wq, sx, sw)
+    ref = oracle.linear_scaled(codes(xq), codes(wq), sx.cpu().numpy(), sw.cpu().numpy())
+    assert rel_fro(bits(y), ref) <= GEMM_REL_FRO
+    if not x_vec and not w_vec:
+        assert torch.equal(y, fw.fp8_linear_static(xq, wq, sx, sw))
+
+
+def test_silu_mul_per_token():
+    g = synth.normal((256, 12288), 2.0, 73, DEV)
+    u = synth.normal((256, 12288), 1.0, 74, DEV)
+    g[5] = 0
+    h, s = fw.silu_mul_2in_fp8_per_token(g, u)
+    rh, rs = oracle.silu_mul_2in_rows(bits(g), bits(u))
+    assert np.allclose(s.cpu().numpy(), rs, rtol=1e-6, atol=0)
+    diff = code_step_diff(codes(h), rh)
+    assert diff.max() <= 1 and (diff > 0).mean() <= SWIGLU_MAX_FRAC
+
+
+@pytest.mark.parametrize("M", [64, 1024])
+def test_gated_mlp_per_token(M):
+    d, I = 3072, 12288
+    x = synth.activation_with_outliers(M, d, 6, 10 + M, 0, DEV)
+    wg, s_wg = fw.fp8_quant_per_token(synth.normal((I, d), 0.02, 75, DEV))
+    wu, s_wu = fw.fp8_quant_per_token(synth.normal((I, d), 0.02, 76, DEV))
+    wd, s_wd = fw.fp8_quant_per_token(synth.normal((d, I), 0.02, 77, DEV))
+    y = fw.gated_mlp_per_token_fp8(x, wg, s_wg, wu, s_wu, wd, s_wd)
+    rows = np.arange(M) if M <= 64 else np.random.default_rng(3).choice(M, 4, replace=False)
+    ref = oracle.gated_mlp_per_token(bits(x[rows]), codes(wg), s_wg.cpu().numpy(), codes(wu),
+                                     s_wu.cpu().numpy(), codes(wd), s_wd.cpu().numpy())
+    assert rel_fro(bits(y[rows]), ref) <= GEMM_REL_FRO
+    assert fw.device_status()[0] == fw.OK

@@ -518,3 +518,54 @@ def test_cross_attention_reduces_to_self_attention():
     # K from ctx equals a plain quantize-then-Linear of ctx at s_kv
     assert np.array_equal(k2, oracle.linear(oracle.quantize(ctx, oracle.f32(0.05)), *proj[1][:1],
                                             oracle.f32(0.05), proj[1][1]))
+
+
+# ------------------------------------------- per-channel / per-token scales
+
+
+def test_quantize_rows_is_per_row_rtn():
+    """Each row is its own RTN tensor: same codes and scale as rtn_weight on
+    that row alone; an all-zero row gets scale 1 and zero codes."""
+    w = bits_of(synth.normal((12, 200), 0.3, 61))
+    w[5] = 0
+    q, s = oracle.quantize_rows(w)
+    for r in range(12):
+        if r == 5:
+            assert s[r] == 1.0 and np.all(q[r] == 0)
+            continue
+        qr, sr = oracle.rtn_weight(np.ascontiguousarray(w[r]))
+        assert sr == s[r] and np.array_equal(qr, q[r])
+        assert (q[r] & 0x7F).max() == 0x7E   # each row reaches the largest code
+
+
+def test_linear_scaled_reduces_to_per_tensor():
+    rng = np.random.default_rng(62)
+    xq = rng.integers(0, 0x7E, size=(7, 64), dtype=np.uint8)
+    wq = rng.integers(0, 0x7E, size=(9, 64), dtype=np.uint8) | 0x80
+    a, b = oracle.f32(0.3), oracle.f32(0.002)
+    ref = oracle.linear(xq, wq, a, b)
+    assert np.array_equal(oracle.linear_scaled(xq, wq, a, b), ref)
+    assert np.array_equal(oracle.linear_scaled(xq, wq, np.full(7, a, np.float32),
+                                               np.full(9, b, np.float32)), ref)
+    # a per-row scale multiplies that row only; a per-column scale that column only
+    sx = np.full(7, a, np.float32)
+    sx[3] *= 2
+    y = oracle.linear_scaled(xq, wq, sx, b)
+    assert np.array_equal(y[:3], ref[:3]) and np.array_equal(y[4:], ref[4:])
+    assert np.array_equal(oracle.bf16_to_f64(y[3]), 2 * oracle.bf16_to_f64(ref[3]))
+    sw = np.full(9, b, np.float32)
+    sw[6] *= 4
+    y = oracle.linear_scaled(xq, wq, a, sw)
+    assert np.array_equal(oracle.bf16_to_f64(y[:, 6]), 4 * oracle.bf16_to_f64(ref[:, 6]))
+    assert np.array_equal(np.delete(y, 6, axis=1), np.delete(ref, 6, axis=1))
+
+
+def test_silu_mul_rows_uses_each_rows_maximum():
+    g, u = _gu(63, rows=6, cols=300)
+    h, s = oracle.silu_mul_2in_rows(g, u)
+    v = oracle.silu_mul_f64(oracle.bf16_to_f64(g), oracle.bf16_to_f64(u))
+    for r in range(6):
+        assert s[r] == np.float32(np.abs(v[r]).max() / 448.0)
+        assert np.array_equal(h[r], oracle.silu_mul_2in(np.ascontiguousarray(g[r]),
+                                                        np.ascontiguousarray(u[r]), float(s[r])))
+        assert (h[r] & 0x7F).max() == 0x7E
