@@ -240,14 +240,55 @@ def run_plan(plan, events=None):
     events[len(plan)].record()
 
 
-def time_device(plan, steps, warmup, dist_ctx, sampler=None):
+def make_stream_runner(plan, device):
+    """The pass with the two towers of each layer on two streams.  Within a
+    layer the understanding-tower and generation-tower MLPs are independent,
+    so they run concurrently (each stream keeps its own kernel order); at
+    every layer boundary the streams join, as the next layer's inputs would
+    depend on both towers."""
+    main = torch.cuda.current_stream(device)
+    side = torch.cuda.Stream(device)
+    # group plan entries by layer: each layer is und entries then gen entries
+    n_layers = sum(1 for e in plan if e[0] == "quant@und")
+    step = len(plan) // n_layers
+    groups = [plan[i:i + step] for i in range(0, len(plan), step)]
+    side_handle = side.cuda_stream
+    main_handle = main.cuda_stream
+    # rebind the stream argument (the last one) of every call
+    bound = []
+    for g in groups:
+        und = [(fn, args[:-1] + (side_handle,)) for k, fn, args, _, _ in g if k.endswith("@und")]
+        gen = [(fn, args[:-1] + (main_handle,)) for k, fn, args, _, _ in g if k.endswith("@gen")]
+        bound.append((und, gen))
+    ev_main = [torch.cuda.Event() for _ in bound]
+    ev_side = [torch.cuda.Event() for _ in bound]
+
+    def run():
+        side.wait_stream(main)
+        for li, (und, gen) in enumerate(bound):
+            for fn, args in und:
+                if fn(*args) != 0:
+                    raise RuntimeError("launch failed")
+            for fn, args in gen:
+                if fn(*args) != 0:
+                    raise RuntimeError("launch failed")
+            ev_side[li].record(side)
+            ev_main[li].record(main)
+            main.wait_event(ev_side[li])
+            side.wait_event(ev_main[li])
+        main.wait_stream(side)
+    return run
+
+
+def time_device(plan, steps, warmup, dist_ctx, sampler=None, runner=None):
     """W untimed steps, then K timed steps between a barrier + synchronize on
     both sides, with CUDA events on the launching stream around the region
     only (an event between two kernels would stop the next kernel from being
     scheduled early).  Then K more steps with events between every launch,
     for each kernel's average duration."""
+    run = runner if runner is not None else (lambda: run_plan(plan))
     for _ in range(warmup):
-        run_plan(plan)
+        run()
     torch.cuda.synchronize()
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     dist_ctx.barrier()
@@ -256,7 +297,7 @@ def time_device(plan, steps, warmup, dist_ctx, sampler=None):
         sampler.start()
     start.record()
     for k in range(steps):
-        run_plan(plan)
+        run()
     stop.record()
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
@@ -558,6 +599,8 @@ def main():
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--streams", type=int, choices=(1, 2), default=1,
+                    help="2: the two towers of each layer on two streams, joined per layer")
     ap.add_argument("--unfused", action="store_true",
                     help="time the five-kernel composition (separate gate/up GEMMs and SwiGLU-quant)")
     ap.add_argument("--kernel", choices=("gemm", "dual", "swiglu", "quant"),
@@ -626,8 +669,9 @@ def main():
 
     launches_before = fw.launch_count()
     sampler = ClockSampler(device.index if device.index is not None else 0)
+    runner = make_stream_runner(plan, device) if args.streams == 2 else None
     total_ms, per_kind, clocks, instrumented_ms = time_device(plan, args.steps, max(args.warmup, 3),
-                                                              ctx, sampler)
+                                                              ctx, sampler, runner)
     launches = (fw.launch_count() - launches_before) // (2 * args.steps + max(args.warmup, 3)) * args.steps
     st, where = fw.device_status()
     if st != 0:
@@ -700,7 +744,7 @@ def main():
             "config": {"workload": "two-tower MoT decoder-MLP pass, 36 layers x {und M=1024, gen M=4096}, d=3072, I=12288",
                        "path": ("fused: quantize X -> gate/up GEMM with SwiGLU-quant epilogue -> down GEMM"
                                 if fused else "unfused: quantize X -> gate GEMM -> up GEMM -> SwiGLU-quant -> down GEMM"),
-                       "layers": args.layers, "global_batch": TOKENS_PER_STEP * ctx.world,
+                       "layers": args.layers, "streams": args.streams, "global_batch": TOKENS_PER_STEP * ctx.world,
                        "parallelism": f"replicas x{ctx.world}",
                        "l2": "inputs larger than L2 (8.15 GB of FP8 weights per pass)"},
             "roofline": roofline, "components": comp, "e2e": e2e, "cpu_baseline": cpu,

@@ -55,6 +55,7 @@ struct DeviceInfo {
   unsigned gemm_attr_set = 0;  // bit per kernel whose attributes were set on this device
   int pair_clusters = 0;       // CTA pairs of the pair GEMM resident at once
   int dual_clusters = 0;       // CTA pairs of the gate/up dual GEMM resident at once
+  // (the same for every epilogue variant: one CTA per SM either way)
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -222,11 +223,12 @@ int launch_gemm_cfg(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int M, 
 // (an empty tensor's data pointer).
 // CTA-pair GEMM: one cluster of two CTAs per TPC, persistent over 256 x 256
 // tiles.  The grid holds as many pairs as can be resident at once.
-template <int STAGES, int BIT, int SCALE_MODE = 0>
-int launch_gemm_pair(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int M, int N, int K,
-                     const float *s_in, const float *s_w, uint16_t *y, cudaStream_t st) {
-  using C = PairCfg<STAGES>;
-  auto kern = fp8_gemm_pair_kernel<STAGES, SCALE_MODE>;
+template <int STAGES, int BIT, int SCALE_MODE = 0, bool DIRECT = false>
+int launch_gemm_pair_cfg(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int M, int N,
+                         int K, const float *s_in, const float *s_w, uint16_t *y,
+                         cudaStream_t st) {
+  using C = PairCfg<STAGES, DIRECT>;
+  auto kern = fp8_gemm_pair_kernel<STAGES, SCALE_MODE, DIRECT>;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -258,20 +260,41 @@ int launch_gemm_pair(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int M,
   const int tiles = ((M + kPairTile - 1) / kPairTile) * ((N + kPairTile - 1) / kPairTile);
   const int clusters = tiles < d->pair_clusters ? tiles : d->pair_clusters;
   if (launch_ex(kern, dim3(2 * clusters), dim3(kGemmThreads), C::SMEM_BYTES, st, 2, ma, mb, md,
-                s_in, s_w, M, N, K, kWaitLimitNs) != cudaSuccess)
+                s_in, s_w, M, N, K, kWaitLimitNs, y) != cudaSuccess)
     return FP8WS_ERR_CUDA;
   log_launch(kKindGemm, xq, wq, y);
   return launch_status();
 }
 
+// Epilogue of the CTA-pair kernels: TMA stores from shared-memory tiles with
+// six pipeline stages (default), or 16-byte global stores from registers with
+// seven stages (FP8WS_EPILOGUE=direct).
+bool direct_epilogue() {
+  static int v = -1;
+  if (v < 0) {
+    const char *e = getenv("FP8WS_EPILOGUE");
+    v = (e && e[0] == 'd') ? 1 : 0;
+  }
+  return v == 1;
+}
+
+template <int BIT, int SCALE_MODE = 0>
+int launch_gemm_pair(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int M, int N, int K,
+                     const float *s_in, const float *s_w, uint16_t *y, cudaStream_t st) {
+  if (direct_epilogue())
+    return launch_gemm_pair_cfg<7, BIT + 16, SCALE_MODE, true>(d, xq, wq, M, N, K, s_in, s_w, y,
+                                                               st);
+  return launch_gemm_pair_cfg<6, BIT, SCALE_MODE, false>(d, xq, wq, M, N, K, s_in, s_w, y, st);
+}
+
 // Gate/up dual GEMM with the SwiGLU-quant epilogue, on CTA pairs.
-template <int STAGES, int BIT>
-int launch_dual_swiglu(DeviceInfo *d, const uint8_t *xq, const uint8_t *wg, const uint8_t *wu,
-                       int M, int N, int K, const float *s_in, const float *s_wg,
-                       const float *s_wu, const float *s_down, SwigluParams act, uint8_t *h,
-                       cudaStream_t st) {
-  using C = DualCfg<STAGES>;
-  auto kern = fp8_dual_swiglu_pair_kernel<STAGES>;
+template <int STAGES, int BIT, bool DIRECT>
+int launch_dual_swiglu_cfg(DeviceInfo *d, const uint8_t *xq, const uint8_t *wg,
+                           const uint8_t *wu, int M, int N, int K, const float *s_in,
+                           const float *s_wg, const float *s_wu, const float *s_down,
+                           SwigluParams act, uint8_t *h, cudaStream_t st) {
+  using C = DualCfg<STAGES, DIRECT>;
+  auto kern = fp8_dual_swiglu_pair_kernel<STAGES, DIRECT>;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -303,10 +326,22 @@ int launch_dual_swiglu(DeviceInfo *d, const uint8_t *xq, const uint8_t *wg, cons
   const int tiles = ((M + kDualTileM - 1) / kDualTileM) * ((N + kDualTileN - 1) / kDualTileN);
   const int clusters = tiles < d->dual_clusters ? tiles : d->dual_clusters;
   if (launch_ex(kern, dim3(2 * clusters), dim3(kGemmThreads), C::SMEM_BYTES, st, 2, ma, mg, mu, mh,
-                s_in, s_wg, s_wu, s_down, act, M, N, K, kWaitLimitNs) != cudaSuccess)
+                s_in, s_wg, s_wu, s_down, act, M, N, K, kWaitLimitNs, h) != cudaSuccess)
     return FP8WS_ERR_CUDA;
   log_launch(kKindDual, xq, wg, h);
   return launch_status();
+}
+
+template <int STAGES_UNUSED, int BIT>
+int launch_dual_swiglu(DeviceInfo *d, const uint8_t *xq, const uint8_t *wg, const uint8_t *wu,
+                       int M, int N, int K, const float *s_in, const float *s_wg,
+                       const float *s_wu, const float *s_down, SwigluParams act, uint8_t *h,
+                       cudaStream_t st) {
+  if (direct_epilogue())
+    return launch_dual_swiglu_cfg<7, BIT + 16, true>(d, xq, wg, wu, M, N, K, s_in, s_wg, s_wu,
+                                                     s_down, act, h, st);
+  return launch_dual_swiglu_cfg<6, BIT, false>(d, xq, wg, wu, M, N, K, s_in, s_wg, s_wu, s_down,
+                                               act, h, st);
 }
 
 int check_gemm_args(const void *xq, const void *wq, int64_t M, int64_t N, int64_t K,
@@ -331,7 +366,7 @@ int gemm_dispatch(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int64_t M
   if (M == 0) return FP8WS_OK;
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
   switch (g_forced_gemm_config) {
-    case 1: return launch_gemm_pair<6, 3>(d, xq, wq, m, n, k, s_in, s_w, y, st);
+    case 1: return launch_gemm_pair<3>(d, xq, wq, m, n, k, s_in, s_w, y, st);
     case 2: return launch_gemm_cfg<256, 4, 0>(d, xq, wq, m, n, k, s_in, s_w, y, st);
     case 3: return launch_gemm_cfg<128, 6, 1>(d, xq, wq, m, n, k, s_in, s_w, y, st);
     case 4: return launch_gemm_cfg<64, 8, 2>(d, xq, wq, m, n, k, s_in, s_w, y, st);
@@ -345,7 +380,7 @@ int gemm_dispatch(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int64_t M
   const double est_128 = waves(m128 * ((N + 127) / 128), d->sms) * (128.0 * 128) / 0.45;
   const double est_64 = waves(m128 * ((N + 63) / 64), d->sms) * (128.0 * 64) / 0.25;
   const double best = fmin(fmin(est_pair, est_256), fmin(est_128, est_64));
-  if (est_pair == best) return launch_gemm_pair<6, 3>(d, xq, wq, m, n, k, s_in, s_w, y, st);
+  if (est_pair == best) return launch_gemm_pair<3>(d, xq, wq, m, n, k, s_in, s_w, y, st);
   if (est_256 == best) return launch_gemm_cfg<256, 4, 0>(d, xq, wq, m, n, k, s_in, s_w, y, st);
   if (est_128 == best) return launch_gemm_cfg<128, 6, 1>(d, xq, wq, m, n, k, s_in, s_w, y, st);
   return launch_gemm_cfg<64, 8, 2>(d, xq, wq, m, n, k, s_in, s_w, y, st);
@@ -718,10 +753,10 @@ int fp8_linear_scaled(const uint8_t *xq, const uint8_t *wq, int64_t M, int64_t N
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
   const int mode = (x_per_row ? kScaleRowVec : 0) | (w_per_col ? kScaleColVec : 0);
   switch (mode) {
-    case 0: return launch_gemm_pair<6, 3, 0>(d, xq, wq, m, n, k, s_x, s_w, y, st);
-    case 1: return launch_gemm_pair<6, 5, 1>(d, xq, wq, m, n, k, s_x, s_w, y, st);
-    case 2: return launch_gemm_pair<6, 6, 2>(d, xq, wq, m, n, k, s_x, s_w, y, st);
-    default: return launch_gemm_pair<6, 7, 3>(d, xq, wq, m, n, k, s_x, s_w, y, st);
+    case 0: return launch_gemm_pair<3, 0>(d, xq, wq, m, n, k, s_x, s_w, y, st);
+    case 1: return launch_gemm_pair<5, 1>(d, xq, wq, m, n, k, s_x, s_w, y, st);
+    case 2: return launch_gemm_pair<6, 2>(d, xq, wq, m, n, k, s_x, s_w, y, st);
+    default: return launch_gemm_pair<7, 3>(d, xq, wq, m, n, k, s_x, s_w, y, st);
   }
 }
 

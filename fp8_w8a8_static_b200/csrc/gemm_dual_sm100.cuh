@@ -31,15 +31,18 @@ namespace fp8ws {
 constexpr int kDualTileM = 256;  // rows per CTA pair
 constexpr int kDualTileN = 128;  // columns of G and of U per tile
 
-template <int STAGES_>
+// DIRECT_: H written with 16-byte global stores from registers instead of
+// TMA stores of shared-memory tiles; the freed 32 KB hold a seventh stage.
+template <int STAGES_, bool DIRECT_ = false>
 struct DualCfg {
   static constexpr int STAGES = STAGES_;
+  static constexpr bool DIRECT = DIRECT_;
   static constexpr int A_BYTES = 128 * kGemmBK;   // this CTA's 128 rows of Xq
   static constexpr int B_BYTES = 128 * kGemmBK;   // 128 rows of Wg (leader) or Wu (peer)
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TX_BYTES = 2 * STAGE_BYTES;
   static constexpr int EPI_BUF_BYTES = 32 * 128;   // 32 rows x 128 FP8 codes
-  static constexpr int EPI_BYTES = 4 * 2 * EPI_BUF_BYTES;
+  static constexpr int EPI_BYTES = DIRECT ? 0 : 4 * 2 * EPI_BUF_BYTES;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
   static constexpr uint32_t ACC_COLS = 2 * kDualTileN;  // G | U
@@ -49,7 +52,7 @@ struct DualCfg {
   static_assert(TMEM_COLS == 512, "tmem");
 };
 
-template <int STAGES>
+template <int STAGES, bool DIRECT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     fp8_dual_swiglu_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
                                 const __grid_constant__ CUtensorMap tm_bg,
@@ -58,8 +61,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                 const float *__restrict__ s_in, const float *__restrict__ s_wg,
                                 const float *__restrict__ s_wu,
                                 const float *__restrict__ s_down, SwigluParams act, int M,
-                                int N, int K, uint64_t timeout_ns) {
-  using C = DualCfg<STAGES>;
+                                int N, int K, uint64_t timeout_ns, uint8_t *__restrict__ h_out) {
+  using C = DualCfg<STAGES, DIRECT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -223,9 +226,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t t_g =
           tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * C::ACC_COLS;
       uint8_t *buf = sEpi + (ew * 2 + (it & 1u)) * C::EPI_BUF_BYTES;
-      if (lane == 0) tma_store_wait_read<1>();  // this buffer's previous store has read it
-      __syncwarp();
+      if (!DIRECT) {
+        if (lane == 0) tma_store_wait_read<1>();  // this buffer's previous store has read it
+        __syncwarp();
+      }
       uint8_t *row = buf + lane * 128;
+      uint8_t *hrow = h_out + static_cast<int64_t>(row0 + lane) * N + col0;
+      const bool row_ok = row0 + lane < M;
 #pragma unroll 1
       for (int c = 0; c < kDualTileN / 32; ++c) {
         uint32_t g[32], u[32];
@@ -249,18 +256,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           q[j] = pack4(cvt_e4m3x2(h[0], h[1]), cvt_e4m3x2(h[2], h[3]));
         }
-        // 32 codes = two 16-byte units (2c, 2c+1) of this row, swizzled
-        *reinterpret_cast<uint4 *>(row + (((2 * c) ^ (lane & 7)) << 4)) =
-            make_uint4(q[0], q[1], q[2], q[3]);
-        *reinterpret_cast<uint4 *>(row + (((2 * c + 1) ^ (lane & 7)) << 4)) =
-            make_uint4(q[4], q[5], q[6], q[7]);
+        if (DIRECT) {
+          // columns col0 + 32c .. +31 of this thread's row (N % 16 == 0)
+          if (row_ok && col0 + 32 * c < N)
+            *reinterpret_cast<uint4 *>(hrow + 32 * c) = make_uint4(q[0], q[1], q[2], q[3]);
+          if (row_ok && col0 + 32 * c + 16 < N)
+            *reinterpret_cast<uint4 *>(hrow + 32 * c + 16) = make_uint4(q[4], q[5], q[6], q[7]);
+        } else {
+          // 32 codes = two 16-byte units (2c, 2c+1) of this row, swizzled
+          *reinterpret_cast<uint4 *>(row + (((2 * c) ^ (lane & 7)) << 4)) =
+              make_uint4(q[0], q[1], q[2], q[3]);
+          *reinterpret_cast<uint4 *>(row + (((2 * c + 1) ^ (lane & 7)) << 4)) =
+              make_uint4(q[4], q[5], q[6], q[7]);
+        }
       }
-      fence_async_shared();
-      __syncwarp();
-      if (lane == 0 && store) {
-        tma_store_2d(&tm_h, buf, col0, row0);
+      if (!DIRECT) {
+        fence_async_shared();
+        __syncwarp();
+        if (lane == 0 && store) {
+          tma_store_2d(&tm_h, buf, col0, row0);
+        }
+        if (lane == 0) tma_store_commit();
       }
-      if (lane == 0) tma_store_commit();
     }
     if (lane == 0) tma_store_wait_all<0>();
   }

@@ -30,16 +30,20 @@ constexpr int kPairTile = 256;  // output rows and columns per CTA pair
 constexpr int kScaleRowVec = 1;
 constexpr int kScaleColVec = 2;
 
-template <int STAGES_>
+// DIRECT_: the epilogue writes Y with 16-byte global stores from registers
+// instead of staging 32 x 64 tiles in shared memory for TMA stores; the 32 KB
+// this frees hold a seventh pipeline stage.
+template <int STAGES_, bool DIRECT_ = false>
 struct PairCfg {
   static constexpr int STAGES = STAGES_;
+  static constexpr bool DIRECT = DIRECT_;
   static constexpr int A_BYTES = 128 * kGemmBK;   // this CTA's half of A
   static constexpr int B_BYTES = 128 * kGemmBK;   // this CTA's half of B
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TX_BYTES = 2 * STAGE_BYTES;  // both CTAs, counted at the leader
   static constexpr int EPI_COLS = 64;
   static constexpr int EPI_BUF_BYTES = 32 * EPI_COLS * 2;
-  static constexpr int EPI_BYTES = 4 * 2 * EPI_BUF_BYTES;
+  static constexpr int EPI_BYTES = DIRECT ? 0 : 4 * 2 * EPI_BUF_BYTES;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;  // two 256-column accumulators
@@ -47,14 +51,14 @@ struct PairCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
-template <int STAGES, int SCALE_MODE>
+template <int STAGES, int SCALE_MODE, bool DIRECT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
                          const __grid_constant__ CUtensorMap tm_b,
                          const __grid_constant__ CUtensorMap tm_d, const float *__restrict__ s_in,
                          const float *__restrict__ s_w, int M, int N, int K,
-                         uint64_t timeout_ns) {
-  using C = PairCfg<STAGES>;
+                         uint64_t timeout_ns, uint16_t *__restrict__ y_out) {
+  using C = PairCfg<STAGES, DIRECT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -240,9 +244,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           cs1 = col0 + 32 + lane < N ? __ldg(s_w + col0 + 32 + lane) : 0.0f;
         }
         uint8_t *buf = sEpi + (ew * 2 + (chunk & 1u)) * C::EPI_BUF_BYTES;
-        if (lane == 0) tma_store_wait_read<1>();
-        __syncwarp();
+        if (!DIRECT) {
+          if (lane == 0) tma_store_wait_read<1>();
+          __syncwarp();
+        }
         uint8_t *row = buf + lane * 128;
+        // direct stores: this thread's row of Y, 64 columns from col0
+        uint16_t *yrow = y_out + static_cast<int64_t>(row0 + lane) * N + col0;
+        const bool row_ok = row0 + lane < M;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const uint32_t *src = (j < 4) ? &r0[j * 8] : &r1[(j - 4) * 8];
@@ -271,13 +280,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           v.y = *reinterpret_cast<uint32_t *>(&p1);
           v.z = *reinterpret_cast<uint32_t *>(&p2);
           v.w = *reinterpret_cast<uint32_t *>(&p3);
-          *reinterpret_cast<uint4 *>(row + ((j ^ (lane & 7)) << 4)) = v;
+          if (DIRECT) {
+            if (row_ok && col0 + j * 8 < N) *reinterpret_cast<uint4 *>(yrow + j * 8) = v;
+          } else {
+            *reinterpret_cast<uint4 *>(row + ((j ^ (lane & 7)) << 4)) = v;
+          }
         }
-        fence_async_shared();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&tm_d, buf, col0, row0);
-          tma_store_commit();
+        if (!DIRECT) {
+          fence_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tm_d, buf, col0, row0);
+            tma_store_commit();
+          }
         }
         ++chunk;
       }
