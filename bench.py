@@ -599,7 +599,7 @@ def main():
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--streams", type=int, choices=(1, 2), default=1,
+    ap.add_argument("--streams", type=int, choices=(1, 2), default=2,
                     help="2: the two towers of each layer on two streams, joined per layer")
     ap.add_argument("--unfused", action="store_true",
                     help="time the five-kernel composition (separate gate/up GEMMs and SwiGLU-quant)")
@@ -628,7 +628,7 @@ def main():
         if ctx.rank != 0:
             return 0
         o = OracleSample()
-        rows = 16
+        rows = 64
         for _ in range(args.warmup):
             o.run(2)
         step_times = []
