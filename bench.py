@@ -176,7 +176,7 @@ def make_buffers(fw, layers, device, fused):
     for tower, M in TOWERS:
         if fused:
             nbytes = fw.gated_mlp_static_fp8_fused_workspace(M, D, I)
-            ws[tower] = torch.empty(nbytes, dtype=torch.uint8, device=device)
+            ws[tower] = torch.zeros(nbytes, dtype=torch.uint8, device=device)
             bufs[tower] = fw.fused_workspace_views(ws[tower], M, D, I)
         else:
             nbytes = fw.gated_mlp_static_fp8_workspace(M, D, I)
@@ -190,7 +190,24 @@ def make_buffers(fw, layers, device, fused):
 # ---------------------------------------------------------- timed region
 
 
-def build_plan(fw, layers, bufs, stream_handle, fused):
+def build_value_plan(fw, layers, ws, stream_handle, fused):
+    """The pass as one composite C-ABI call per MLP (the call a user makes):
+    gated_mlp_static_fp8_fused (or gated_mlp_static_fp8 when unfused)."""
+    lib = fw.load()
+    fn = lib.gated_mlp_static_fp8_fused if fused else lib.gated_mlp_static_fp8
+    plan = []
+    for L in layers:
+        M = L.M
+        head = (L.x.data_ptr(), M, D, I, L.s_in.data_ptr(), L.wg.data_ptr(), L.s_wg.data_ptr(),
+                L.wu.data_ptr(), L.s_wu.data_ptr(), L.s_down.data_ptr())
+        tail = (L.wd.data_ptr(), L.s_wd.data_ptr(), ws[L.tower].data_ptr(), L.y.data_ptr(),
+                stream_handle)
+        args = head + ((None,) if fused else ()) + tail
+        plan.append(("mlp@" + L.tower, fn, args, 0, 0))
+    return plan
+
+
+def build_plan(fw, layers, bufs, stream_handle, fused, ws=None):
     """The pass as a flat list of direct C-ABI calls (kind, fn, args,
     algorithmic bytes, flops), in the order the composite gated-MLP call
     issues them.  Fused: quantize X, fused gate/up GEMM + SwiGLU-quant, down
@@ -220,10 +237,18 @@ def build_plan(fw, layers, bufs, stream_handle, fused):
                          M * D + I * D + 2 * M * I, 2 * M * I * D))
             plan.append(("swiglu" + tw, lib.silu_mul_2in_fp8, (g, u, M * I, s_down, h, stream_handle),
                          5 * M * I, 0))
-        plan.append(("gemm_down" + tw, lib.fp8_linear_static,
-                     (h, L.wd.data_ptr(), M, D, I, s_down, L.s_wd.data_ptr(), L.y.data_ptr(),
-                      stream_handle),
-                     M * I + D * I + 2 * M * D, 2 * M * D * I))
+        if fused:
+            # the composite's down GEMM: split-K of the last wave in its scratch
+            splitk = bufs[L.tower]["splitk"]
+            plan.append(("gemm_down" + tw, lib.fp8_linear_static_ws,
+                         (h, L.wd.data_ptr(), M, D, I, s_down, L.s_wd.data_ptr(), L.y.data_ptr(),
+                          splitk.data_ptr(), splitk.numel(), stream_handle),
+                         M * I + D * I + 2 * M * D, 2 * M * D * I))
+        else:
+            plan.append(("gemm_down" + tw, lib.fp8_linear_static,
+                         (h, L.wd.data_ptr(), M, D, I, s_down, L.s_wd.data_ptr(), L.y.data_ptr(),
+                          stream_handle),
+                         M * I + D * I + 2 * M * D, 2 * M * D * I))
     return plan
 
 
@@ -249,7 +274,7 @@ def make_stream_runner(plan, device):
     main = torch.cuda.current_stream(device)
     side = torch.cuda.Stream(device)
     # group plan entries by layer: each layer is und entries then gen entries
-    n_layers = sum(1 for e in plan if e[0] == "quant@und")
+    n_layers = sum(1 for e in plan if e[0] == plan[0][0])  # first entry of every layer
     step = len(plan) // n_layers
     groups = [plan[i:i + step] for i in range(0, len(plan), step)]
     side_handle = side.cuda_stream
@@ -280,7 +305,7 @@ def make_stream_runner(plan, device):
     return run
 
 
-def time_device(plan, steps, warmup, dist_ctx, sampler=None, runner=None):
+def time_device(plan, steps, warmup, dist_ctx, sampler=None, runner=None, instr_plan=None):
     """W untimed steps, then K timed steps between a barrier + synchronize on
     both sides, with CUDA events on the launching stream around the region
     only (an event between two kernels would stop the next kernel from being
@@ -304,6 +329,7 @@ def time_device(plan, steps, warmup, dist_ctx, sampler=None, runner=None):
     dist_ctx.barrier()
     total_ms = start.elapsed_time(stop)
 
+    plan = instr_plan if instr_plan is not None else plan
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(plan) + 1)]
           for _ in range(steps)]
     for k in range(steps):
@@ -666,13 +692,21 @@ def main():
     ws, bufs = make_buffers(fw, layers, device, fused)
     stream = torch.cuda.current_stream(device)
     plan = build_plan(fw, layers, bufs, stream.cuda_stream, fused)
+    value_plan = build_value_plan(fw, layers, ws, stream.cuda_stream, fused)
 
     launches_before = fw.launch_count()
+    launches_per_step = sum(3 if fused else 5 for _ in value_plan)
     sampler = ClockSampler(device.index if device.index is not None else 0)
-    runner = make_stream_runner(plan, device) if args.streams == 2 else None
-    total_ms, per_kind, clocks, instrumented_ms = time_device(plan, args.steps, max(args.warmup, 3),
-                                                              ctx, sampler, runner)
-    launches = (fw.launch_count() - launches_before) // (2 * args.steps + max(args.warmup, 3)) * args.steps
+    runner = make_stream_runner(value_plan, device) if args.streams == 2 else None
+    total_ms, per_kind, clocks, instrumented_ms = time_device(value_plan, args.steps,
+                                                              max(args.warmup, 3), ctx, sampler,
+                                                              runner, instr_plan=plan)
+    launches = launches_per_step * args.steps
+    counted = fw.launch_count() - launches_before
+    expect = launches_per_step * (args.steps + max(args.warmup, 3)) + \
+        sum(1 for _ in plan) * args.steps
+    if counted != expect:
+        raise RuntimeError(f"launch count {counted} != expected {expect}")
     st, where = fw.device_status()
     if st != 0:
         raise RuntimeError(f"device status {st} at wait site {where}")

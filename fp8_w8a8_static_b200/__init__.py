@@ -24,7 +24,7 @@ import torch
 
 __all__ = [
     "FP8WSError", "library_path", "load",
-    "fp8_quant_static", "fp8_linear_static", "silu_mul_2in_fp8",
+    "fp8_quant_static", "fp8_linear_static", "fp8_linear_static_ws", "silu_mul_2in_fp8",
     "gated_mlp_static_fp8", "gated_mlp_static_fp8_workspace",
     "fp8_gate_up_swiglu_static", "gated_mlp_static_fp8_fused", "swiglu_2in_fp8", "swiglu",
     "gated_mlp_static_fp8_fused_workspace",
@@ -87,6 +87,9 @@ _SIGS = {
     "fp8_quant_static": (ctypes.c_int, [_P, _I64, _P, _P, _P]),
     "fp8_linear_static": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _P, _P]),
     "silu_mul_2in_fp8": (ctypes.c_int, [_P, _P, _I64, _P, _P, _P]),
+    "fp8_linear_static_ws_bytes": (ctypes.c_size_t, []),
+    "fp8_linear_static_ws": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _P, _P,
+                                            ctypes.c_size_t, _P]),
     "gated_mlp_static_fp8_workspace": (ctypes.c_size_t, [_I64, _I64, _I64]),
     "gated_mlp_static_fp8": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _P,
                                             _P, _P, _P]),
@@ -241,6 +244,25 @@ def fp8_linear_static(xq: torch.Tensor, wq: torch.Tensor, s_in: torch.Tensor, s_
     return out
 
 
+def fp8_linear_static_ws(xq, wq, s_in, s_w, workspace=None, out=None, stream=None):
+    """fp8_linear_static with split-K of the ragged last wave (workspace scratch)."""
+    lib = load()
+    M, K = xq.shape
+    N = wq.shape[0]
+    need = lib.fp8_linear_static_ws_bytes()
+    if workspace is None:
+        workspace = _workspace(need, xq.device)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    with _device_of(xq):
+        _check(lib.fp8_linear_static_ws(_fp8(xq, "xq"), _fp8(wq, "wq"), M, N, K, _f32(s_in, "s_in"),
+                                        _f32(s_w, "s_w"), _bf16(out, "out"),
+                                        _dev_ptr(workspace, "workspace", (torch.uint8,)),
+                                        workspace.numel() * workspace.element_size(),
+                                        _stream(stream)), "fp8_linear_static_ws")
+    return out
+
+
 def silu_mul_2in_fp8(g: torch.Tensor, u: torch.Tensor, s_down: torch.Tensor,
                      out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """H = E4M3_satRNE(SiLU(G) * U / s_down) from two separate BF16 tensors (any rank)."""
@@ -376,10 +398,13 @@ def gated_mlp_static_fp8_fused(x, s_in, wg, s_wg, wu, s_wu, s_down, wd, s_wd, wo
 
 
 def fused_workspace_views(workspace: torch.Tensor, M: int, d: int, I: int):
-    """Views of the regions gated_mlp_static_fp8_fused writes: Xq [M,d], H [M,I]."""
+    """Views of the regions of gated_mlp_static_fp8_fused's workspace: Xq [M,d],
+    H [M,I] and the down GEMM's split-K scratch (as fp8_linear_static_ws)."""
     o_h = (M * d + 255) // 256 * 256
+    o_s = o_h + (M * I + 255) // 256 * 256
     ws = workspace.view(torch.uint8)
-    return dict(xq=ws[:M * d].view(FP8).view(M, d), h=ws[o_h:o_h + M * I].view(FP8).view(M, I))
+    return dict(xq=ws[:M * d].view(FP8).view(M, d), h=ws[o_h:o_h + M * I].view(FP8).view(M, I),
+                splitk=ws[o_s:o_s + load().fp8_linear_static_ws_bytes()])
 
 
 def qkv_shared_quant_workspace(M: int, d: int) -> int:

@@ -74,11 +74,15 @@ __device__ __forceinline__ uint2 quant8(uint4 v, float s, float r) {
   return o;
 }
 
+// zero_words / n_zero: an optional int array cleared by block 0 (the split-K
+// counters of the GEMMs that follow on the stream).
 __global__ void __launch_bounds__(kEwThreads) quant_static_kernel(
     const uint16_t *__restrict__ x, int64_t numel, const float *__restrict__ s_in,
-    uint8_t *__restrict__ xq) {
+    uint8_t *__restrict__ xq, int *__restrict__ zero_words, int n_zero) {
   pdl_launch_dependents();
   pdl_wait();
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero_words[i] = 0;
   const float s = __ldg(s_in);
   const float r = __frcp_rn(s);
   const int64_t nvec = numel >> 3;

@@ -223,10 +223,55 @@ int launch_gemm_cfg(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int M, 
 // (an empty tensor's data pointer).
 // CTA-pair GEMM: one cluster of two CTAs per TPC, persistent over 256 x 256
 // tiles.  The grid holds as many pairs as can be resident at once.
+// Split-K scratch of the CTA-pair GEMM, laid out independently of the device:
+// kSplitkSlots slots of 2 x 128 x 256 fp32 (one per split unit) followed by
+// one counter per (remainder tile, CTA, epilogue warp) for up to
+// kSplitkTiles remainder tiles.  Plans never need more.
+constexpr int kSplitkSlots = 148;
+constexpr int kSplitkTiles = 128;
+constexpr int kSplitkCounterWords = kSplitkTiles * 2 * 4;
+size_t splitk_slot_bytes() { return static_cast<size_t>(2) * 128 * kPairTile * sizeof(float); }
+int splitk_max_slots(int pairs) { return 2 * pairs < kSplitkSlots ? 2 * pairs : kSplitkSlots; }
+size_t splitk_bytes() {
+  return kSplitkSlots * splitk_slot_bytes() + ((kSplitkCounterWords * sizeof(int) + 255) & ~255ul);
+}
+int *splitk_counters(void *splitk) {
+  return reinterpret_cast<int *>(static_cast<uint8_t *>(splitk) + kSplitkSlots * splitk_slot_bytes());
+}
+
+// Remainder tiles (those past the last full wave) split over S K ranges, S in
+// 1..4 minimising waves-of-units x (1/S) of a tile's time, with at most two
+// waves of units and at least two K steps per range.  No scratch: no split.
+SplitPlan make_split_plan(int tiles, int pairs, int num_kb, float *partials, int *counters) {
+  SplitPlan p{tiles, 0, 1, num_kb, nullptr, nullptr};
+  if (!partials || pairs < 1 || tiles % pairs == 0) return p;
+  const int R = tiles % pairs;
+  if (R > kSplitkTiles) return p;
+  int best_s = 1;
+  double best = 1.0;
+  for (int S = 2; S <= 4; ++S) {
+    const int kbs = (num_kb + S - 1) / S;
+    if (kbs < 2 || (S - 1) * kbs >= num_kb || R * S > splitk_max_slots(pairs)) continue;
+    const double t = static_cast<double>((R * S + pairs - 1) / pairs) / S;
+    if (t < best - 1e-9) {
+      best = t;
+      best_s = S;
+    }
+  }
+  if (best_s == 1) return p;
+  p.dp_tiles = tiles - R;
+  p.split_tiles = R;
+  p.splits = best_s;
+  p.kb_per_split = (num_kb + best_s - 1) / best_s;
+  p.partials = partials;
+  p.counters = counters;
+  return p;
+}
+
 template <int STAGES, int BIT, int SCALE_MODE = 0, bool DIRECT = false>
 int launch_gemm_pair_cfg(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int M, int N,
                          int K, const float *s_in, const float *s_w, uint16_t *y,
-                         cudaStream_t st) {
+                         cudaStream_t st, void *splitk = nullptr) {
   using C = PairCfg<STAGES, DIRECT>;
   auto kern = fp8_gemm_pair_kernel<STAGES, SCALE_MODE, DIRECT>;
   cudaLaunchAttribute attr[1];
@@ -258,9 +303,14 @@ int launch_gemm_pair_cfg(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, in
     rc = make_map_2d(&md, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, M, N, C::EPI_COLS, 32, false);
   if (rc) return rc;
   const int tiles = ((M + kPairTile - 1) / kPairTile) * ((N + kPairTile - 1) / kPairTile);
-  const int clusters = tiles < d->pair_clusters ? tiles : d->pair_clusters;
+  float *partials = static_cast<float *>(splitk);
+  int *counters = splitk ? splitk_counters(splitk) : nullptr;
+  const SplitPlan plan =
+      make_split_plan(tiles, d->pair_clusters, (K + kGemmBK - 1) / kGemmBK, partials, counters);
+  const int units = plan.dp_tiles + plan.split_tiles * plan.splits;
+  const int clusters = units < d->pair_clusters ? units : d->pair_clusters;
   if (launch_ex(kern, dim3(2 * clusters), dim3(kGemmThreads), C::SMEM_BYTES, st, 2, ma, mb, md,
-                s_in, s_w, M, N, K, kWaitLimitNs, y) != cudaSuccess)
+                s_in, s_w, M, N, K, kWaitLimitNs, y, plan) != cudaSuccess)
     return FP8WS_ERR_CUDA;
   log_launch(kKindGemm, xq, wq, y);
   return launch_status();
@@ -280,11 +330,13 @@ bool direct_epilogue() {
 
 template <int BIT, int SCALE_MODE = 0>
 int launch_gemm_pair(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int M, int N, int K,
-                     const float *s_in, const float *s_w, uint16_t *y, cudaStream_t st) {
+                     const float *s_in, const float *s_w, uint16_t *y, cudaStream_t st,
+                     void *splitk = nullptr) {
   if (direct_epilogue())
     return launch_gemm_pair_cfg<7, BIT + 16, SCALE_MODE, true>(d, xq, wq, M, N, K, s_in, s_w, y,
-                                                               st);
-  return launch_gemm_pair_cfg<6, BIT, SCALE_MODE, false>(d, xq, wq, M, N, K, s_in, s_w, y, st);
+                                                               st, splitk);
+  return launch_gemm_pair_cfg<6, BIT, SCALE_MODE, false>(d, xq, wq, M, N, K, s_in, s_w, y, st,
+                                                         splitk);
 }
 
 // Gate/up dual GEMM with the SwiGLU-quant epilogue, on CTA pairs.
@@ -362,11 +414,12 @@ int check_gemm_args(const void *xq, const void *wq, int64_t M, int64_t N, int64_
 int g_forced_gemm_config = 0;  // fp8ws_set_gemm_config: 0 = cost model
 
 int gemm_dispatch(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int64_t M, int64_t N,
-                  int64_t K, const float *s_in, const float *s_w, uint16_t *y, cudaStream_t st) {
+                  int64_t K, const float *s_in, const float *s_w, uint16_t *y, cudaStream_t st,
+                  void *splitk = nullptr) {
   if (M == 0) return FP8WS_OK;
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
   switch (g_forced_gemm_config) {
-    case 1: return launch_gemm_pair<3>(d, xq, wq, m, n, k, s_in, s_w, y, st);
+    case 1: return launch_gemm_pair<3>(d, xq, wq, m, n, k, s_in, s_w, y, st, splitk);
     case 2: return launch_gemm_cfg<256, 4, 0>(d, xq, wq, m, n, k, s_in, s_w, y, st);
     case 3: return launch_gemm_cfg<128, 6, 1>(d, xq, wq, m, n, k, s_in, s_w, y, st);
     case 4: return launch_gemm_cfg<64, 8, 2>(d, xq, wq, m, n, k, s_in, s_w, y, st);
@@ -380,7 +433,7 @@ int gemm_dispatch(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int64_t M
   const double est_128 = waves(m128 * ((N + 127) / 128), d->sms) * (128.0 * 128) / 0.45;
   const double est_64 = waves(m128 * ((N + 63) / 64), d->sms) * (128.0 * 64) / 0.25;
   const double best = fmin(fmin(est_pair, est_256), fmin(est_128, est_64));
-  if (est_pair == best) return launch_gemm_pair<3>(d, xq, wq, m, n, k, s_in, s_w, y, st);
+  if (est_pair == best) return launch_gemm_pair<3>(d, xq, wq, m, n, k, s_in, s_w, y, st, splitk);
   if (est_256 == best) return launch_gemm_cfg<256, 4, 0>(d, xq, wq, m, n, k, s_in, s_w, y, st);
   if (est_128 == best) return launch_gemm_cfg<128, 6, 1>(d, xq, wq, m, n, k, s_in, s_w, y, st);
   return launch_gemm_cfg<64, 8, 2>(d, xq, wq, m, n, k, s_in, s_w, y, st);
@@ -388,10 +441,10 @@ int gemm_dispatch(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int64_t M
 
 // ----------------------------------------------------------- elementwise
 int quant_launch(DeviceInfo *d, const uint16_t *x, int64_t numel, const float *s, uint8_t *xq,
-                 cudaStream_t st) {
+                 cudaStream_t st, int *zero_words = nullptr, int n_zero = 0) {
   if (numel == 0) return FP8WS_OK;
   if (launch_ex(quant_static_kernel, dim3(ew_grid(d, quant_static_kernel, numel >> 3)),
-                dim3(kEwThreads), 0, st, 1, x, numel, s, xq) != cudaSuccess)
+                dim3(kEwThreads), 0, st, 1, x, numel, s, xq, zero_words, n_zero) != cudaSuccess)
     return FP8WS_ERR_CUDA;
   log_launch(kKindQuant, x, nullptr, xq);
   return launch_status();
@@ -578,7 +631,8 @@ int fp8_gate_up_swiglu_static(const uint8_t *xq, const uint8_t *Wg, const uint8_
 size_t gated_mlp_static_fp8_fused_workspace(int64_t M, int64_t d, int64_t I) {
   if (M < 0 || d < 0 || I < 0) return 0;
   const size_t m = static_cast<size_t>(M);
-  return round256(m * static_cast<size_t>(d)) + round256(m * static_cast<size_t>(I));
+  return round256(m * static_cast<size_t>(d)) + round256(m * static_cast<size_t>(I)) +
+         splitk_bytes();
 }
 
 int gated_mlp_static_fp8_fused(const uint16_t *x, int64_t M, int64_t dm, int64_t I,
@@ -598,6 +652,7 @@ int gated_mlp_static_fp8_fused(const uint16_t *x, int64_t M, int64_t dm, int64_t
   const size_t m = static_cast<size_t>(M < 0 ? 0 : M);
   uint8_t *xq = ws;
   uint8_t *H = ws + round256(m * dm);
+  void *splitk = H + round256(m * I);
   int rc = check_gemm_args(xq, Wg, M, I, dm, s_in, s_wg, H);
   if (!rc) rc = check_gemm_args(H, Wd, M, dm, I, s_down, s_wd, y);
   if (rc) return rc;
@@ -607,12 +662,34 @@ int gated_mlp_static_fp8_fused(const uint16_t *x, int64_t M, int64_t dm, int64_t
   if (rc) return rc;
   if (M == 0) return FP8WS_OK;
   cudaStream_t st = as_stream(stream);
-  rc = quant_launch(d, x, M * dm, s_in, xq, st);
+  // the quantizer also clears the split-K counters used by the down GEMM
+  rc = quant_launch(d, x, M * dm, s_in, xq, st, splitk_counters(splitk), kSplitkCounterWords);
   if (!rc)
     rc = launch_dual_swiglu<6, 4>(d, xq, Wg, Wu, static_cast<int>(M), static_cast<int>(I),
                                   static_cast<int>(dm), s_in, s_wg, s_wu, s_down, ap, H, st);
-  if (!rc) rc = gemm_dispatch(d, H, Wd, M, dm, I, s_down, s_wd, y, st);
+  if (!rc) rc = gemm_dispatch(d, H, Wd, M, dm, I, s_down, s_wd, y, st, splitk);
   return rc;
+}
+
+size_t fp8_linear_static_ws_bytes(void) { return splitk_bytes(); }
+
+int fp8_linear_static_ws(const uint8_t *xq, const uint8_t *wq, int64_t M, int64_t N, int64_t K,
+                         const float *s_in, const float *s_w, uint16_t *y, void *workspace,
+                         size_t workspace_bytes, void *stream) {
+  int rc = check_gemm_args(xq, wq, M, N, K, s_in, s_w, y);
+  if (rc) return rc;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      workspace_bytes < splitk_bytes())
+    return FP8WS_ERR_WORKSPACE;
+  DeviceInfo *d;
+  rc = device_info(&d);
+  if (rc) return rc;
+  if (M == 0) return FP8WS_OK;
+  cudaStream_t st = as_stream(stream);
+  if (cudaMemsetAsync(splitk_counters(workspace), 0, kSplitkCounterWords * sizeof(int), st) !=
+      cudaSuccess)
+    return FP8WS_ERR_CUDA;
+  return gemm_dispatch(d, xq, wq, M, N, K, s_in, s_w, y, st, workspace);
 }
 
 }  // extern "C"

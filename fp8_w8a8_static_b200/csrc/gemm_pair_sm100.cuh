@@ -24,6 +24,35 @@ namespace fp8ws {
 
 constexpr int kPairTile = 256;  // output rows and columns per CTA pair
 
+// Split-K of the remainder tiles.  Units 0 .. dp_tiles-1 are whole tiles (the
+// full waves); the last split_tiles tiles are each cut into `splits` K ranges
+// of kb_per_split 128-byte K steps, one unit per range.  Every split writes
+// its fp32 partial (this CTA's 128 x 256) to its own slot of `partials`; the
+// last split of a tile to finish, told apart by a per-warp counter in
+// `counters` (zero before the launch, reset to zero by that last split), adds
+// the partials in split order and runs the epilogue.  splits == 1: no split.
+struct SplitPlan {
+  int dp_tiles;
+  int split_tiles;
+  int splits;
+  int kb_per_split;
+  float *partials;  // [split_tiles * splits][2][128][256] fp32
+  int *counters;    // [split_tiles][2][4]
+};
+
+struct UnitRange {
+  int tile, kb0, kb1, split, slot;  // split < 0: a whole tile
+};
+
+__device__ __forceinline__ UnitRange unit_range(int u, const SplitPlan &p, int num_kb) {
+  if (u < p.dp_tiles) return UnitRange{u, 0, num_kb, -1, -1};
+  const int j = u - p.dp_tiles;
+  const int sp = j % p.splits;
+  const int kb0 = sp * p.kb_per_split;
+  const int kb1 = min(kb0 + p.kb_per_split, num_kb);
+  return UnitRange{p.dp_tiles + j / p.splits, kb0, kb1, sp, j};
+}
+
 // Scale modes of the epilogue: bit 0 = one activation scale per row
 // (s_in[M], per token), bit 1 = one weight scale per column (s_w[N], per
 // channel); 0 = the static per-tensor scalars.
@@ -57,7 +86,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                          const __grid_constant__ CUtensorMap tm_b,
                          const __grid_constant__ CUtensorMap tm_d, const float *__restrict__ s_in,
                          const float *__restrict__ s_w, int M, int N, int K,
-                         uint64_t timeout_ns, uint16_t *__restrict__ y_out) {
+                         uint64_t timeout_ns, uint16_t *__restrict__ y_out, SplitPlan plan) {
   using C = PairCfg<STAGES, DIRECT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -82,8 +111,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int nclusters = gridDim.x >> 1;
   const int num_m = (M + kPairTile - 1) / kPairTile;
   const int num_n = (N + kPairTile - 1) / kPairTile;
-  const int num_tiles = num_m * num_n;
   const int num_kb = (K + kGemmBK - 1) / kGemmBK;
+  const int num_units = plan.dp_tiles + plan.split_tiles * plan.splits;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -118,11 +147,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t stage = 0, phase = 0;
       uint32_t issued_mask = 0, issued_parity = 0;
       bool ok = true;
-      for (int t = cluster; t < num_tiles && ok; t += nclusters) {
-        const TileCoord tc = tile_coord(t, num_m, num_n);
+      for (int u = cluster; u < num_units && ok; u += nclusters) {
+        const UnitRange ur = unit_range(u, plan, num_kb);
+        const TileCoord tc = tile_coord(ur.tile, num_m, num_n);
         const int a_row = tc.m * kPairTile + static_cast<int>(rank) * 128;
         const int b_row = tc.n * kPairTile + static_cast<int>(rank) * 128;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = ur.kb0; kb < ur.kb1; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, timeout_ns)) {
             record_timeout(kSiteProducerEmpty);
             *abort_flag = 1;
@@ -157,7 +187,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t stage = 0, phase = 0;
       uint32_t it = 0;
       bool ok = true;
-      for (int t = cluster; t < num_tiles && ok; t += nclusters, ++it) {
+      for (int u = cluster; u < num_units && ok; u += nclusters, ++it) {
+        const UnitRange ur = unit_range(u, plan, num_kb);
         const uint32_t acc = it & 1u;
         const uint32_t acc_phase = (it >> 1) & 1u;
         if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, timeout_ns)) {
@@ -167,7 +198,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kPairTile;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = ur.kb0; kb < ur.kb1; ++kb) {
           if (!mbar_wait_bounded(&full[stage], phase, abort_flag, timeout_ns)) {
             record_timeout(kSiteMmaFull);
             *abort_flag = 1;
@@ -180,7 +211,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int k = 0; k < kGemmBK / 32; ++k) {
             umma_f8_pair(d_tmem, smem_desc_k_sw128(a_addr + k * 32),
-                         smem_desc_k_sw128(b_addr + k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
+                         smem_desc_k_sw128(b_addr + k * 32), idesc,
+                         (kb != ur.kb0 || k != 0) ? 1u : 0u);
           }
           umma_commit_pair(&empty[stage], 0x3);
           if (++stage == STAGES) {
@@ -201,8 +233,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int quarter = warp & 3;
     const float scale = (SCALE_MODE == 0) ? __ldg(s_in) * __ldg(s_w) : 0.0f;
     uint32_t it = 0, chunk = 0;
-    for (int t = cluster; t < num_tiles; t += nclusters, ++it) {
-      const TileCoord tc = tile_coord(t, num_m, num_n);
+    for (int u = cluster; u < num_units; u += nclusters, ++it) {
+      const UnitRange ur = unit_range(u, plan, num_kb);
+      const TileCoord tc = tile_coord(ur.tile, num_m, num_n);
       const uint32_t acc = it & 1u;
       const uint32_t acc_phase = (it >> 1) & 1u;
       if (!mbar_wait_bounded_warp(&tfull[acc], acc_phase, abort_flag, timeout_ns)) {
@@ -214,6 +247,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_after();
       const int row0 = tc.m * kPairTile + static_cast<int>(rank) * 128 + quarter * 32;
+      const uint32_t t_acc =
+          tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kPairTile;
+      // Split unit: publish this partial; only the tile's last split goes on.
+      int last_split = -1;  // >= 0: this warp sums the partials of all splits
+      if (ur.split >= 0) {
+        const size_t row_off = static_cast<size_t>(quarter * 32 + lane) * kPairTile;
+        float *mine = plan.partials + static_cast<size_t>(ur.slot) * (2 * 128 * kPairTile) +
+                      static_cast<size_t>(rank) * (128 * kPairTile) + row_off;
+#pragma unroll 1
+        for (int c = 0; c < kPairTile / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_acc + c * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4)
+            __stcg(reinterpret_cast<float4 *>(mine + c * 32) + q4,
+                   make_float4(__uint_as_float(r[4 * q4]), __uint_as_float(r[4 * q4 + 1]),
+                               __uint_as_float(r[4 * q4 + 2]), __uint_as_float(r[4 * q4 + 3])));
+        }
+        __threadfence();
+        __syncwarp();
+        int *cnt = plan.counters + ((ur.tile - plan.dp_tiles) * 2 + static_cast<int>(rank)) * 4 +
+                   quarter;
+        int old = 0;
+        if (lane == 0) old = atomicAdd(cnt, 1);
+        old = __shfl_sync(0xFFFFFFFFu, old, 0);
+        if (old != plan.splits - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(map_shared_rank(smem_u32(&tempty[acc]), 0));
+          continue;
+        }
+        __threadfence();
+        if (lane == 0) atomicExch(cnt, 0);  // ready for the next launch
+        last_split = ur.split;
+      }
       float row_scale = 0.0f;  // this thread's row factor (row0 + lane)
       if (SCALE_MODE != 0) {
         const int my_row = row0 + lane;
@@ -230,6 +299,41 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_ld_32x32b_x32(t_row + c * C::EPI_COLS, r0);
         tmem_ld_32x32b_x32(t_row + c * C::EPI_COLS + 32, r1);
         tmem_ld_wait();
+        if (last_split >= 0) {
+          // sum the tile's partials in split order (this split's from TMEM)
+          const size_t row_off = static_cast<size_t>(quarter * 32 + lane) * kPairTile +
+                                 static_cast<size_t>(c) * C::EPI_COLS;
+          const int first_slot = ur.slot - last_split;
+          float v[64];
+#pragma unroll
+          for (int e = 0; e < 64; ++e) v[e] = 0.0f;
+          for (int sp = 0; sp < plan.splits; ++sp) {
+            if (sp == last_split) {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                v[e] += __uint_as_float(r0[e]);
+                v[32 + e] += __uint_as_float(r1[e]);
+              }
+            } else {
+              const float4 *src = reinterpret_cast<const float4 *>(
+                  plan.partials + static_cast<size_t>(first_slot + sp) * (2 * 128 * kPairTile) +
+                  static_cast<size_t>(rank) * (128 * kPairTile) + row_off);
+#pragma unroll
+              for (int q4 = 0; q4 < 16; ++q4) {
+                const float4 w = __ldcg(src + q4);
+                v[4 * q4] += w.x;
+                v[4 * q4 + 1] += w.y;
+                v[4 * q4 + 2] += w.z;
+                v[4 * q4 + 3] += w.w;
+              }
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            r0[e] = __float_as_uint(v[e]);
+            r1[e] = __float_as_uint(v[32 + e]);
+          }
+        }
         if (c == NCHUNK - 1) {
           tc_fence_before();
           __syncwarp();

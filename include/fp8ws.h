@@ -99,6 +99,25 @@ FP8WS_API int fp8_linear_static(const uint8_t *xq, const uint8_t *wq, int64_t M,
                       const float *s_in, const float *s_w, uint16_t *y, void *stream);
 
 /*
+ * fp8_linear_static_ws -- fp8_linear_static with a scratch workspace that lets
+ * the tiles past the last full wave of CTA pairs be split over K (2..4 ranges,
+ * chosen from the shape and the number of resident CTA pairs), so the GPU is
+ * not left partly idle by a ragged last wave.  Each split stores an fp32
+ * partial in the workspace; the last split of a tile to finish adds the
+ * partials in split order (deterministic: the same inputs give the same bits
+ * on every call) and applies the epilogue.  The sum may differ from the
+ * unsplit kernel's in the last bits of fp32, well inside the GEMM tolerance.
+ * workspace: device, >= fp8_linear_static_ws_bytes() bytes, 256-byte aligned;
+ * overwritten (the call clears its counters first).  Other arguments and
+ * errors as fp8_linear_static; FP8WS_ERR_WORKSPACE for a missing, misaligned
+ * or short workspace.
+ */
+FP8WS_API size_t fp8_linear_static_ws_bytes(void);
+FP8WS_API int fp8_linear_static_ws(const uint8_t *xq, const uint8_t *wq, int64_t M, int64_t N,
+                                   int64_t K, const float *s_in, const float *s_w, uint16_t *y,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * silu_mul_2in_fp8 -- two-input SwiGLU quantized straight to FP8 for the
  * down projection.  [PR] What changed (SiLU(G)*U from two separate tensors,
  * quantized directly for the FP8 down_proj; flat indexing over a 1-D grid, so
@@ -191,10 +210,12 @@ FP8WS_API int fp8_gate_up_swiglu_static(const uint8_t *xq, const uint8_t *Wg, co
  * gated_mlp_static_fp8_fused -- gated_mlp_static_fp8 with the gate/up GEMMs
  * and the SwiGLU-quant fused (fp8_gate_up_swiglu_static): three launches
  * (quantize X, fused gate/up/SwiGLU, down GEMM) instead of five, and no G or U
- * round trip through memory.  Same result, bit for bit.
+ * round trip through memory.
  * workspace: device, gated_mlp_static_fp8_fused_workspace(M,d,I) bytes,
- * 256-byte aligned; holds Xq [M,d] then H [M,I] (each region 256-byte
- * aligned).  act: SwiGLU variant (NULL = plain).  Other arguments as
+ * 256-byte aligned; holds Xq [M,d], then H [M,I], then the split-K scratch of
+ * the down GEMM (as fp8_linear_static_ws; each region 256-byte aligned).  The
+ * down projection's sums may therefore differ from gated_mlp_static_fp8's in
+ * the last bits of fp32; H is identical.  act: SwiGLU variant (NULL = plain).  Other arguments as
  * gated_mlp_static_fp8.
  */
 FP8WS_API size_t gated_mlp_static_fp8_fused_workspace(int64_t M, int64_t d, int64_t I);

@@ -73,7 +73,10 @@ def test_fused_mlp_equals_unfused_mlp(M, d, I):
     x, s_in, xq, wg, s_wg, wu, s_wu = _inputs(M, d, I, 11 + M)
     wd, s_wd = fw.fp8_rtn_quantize_weight(synth.normal((d, I), 0.02, 99 + M, DEV))
     s_down = scalar(0.0029, DEV)
-    y_ref = fw.gated_mlp_static_fp8(x, s_in, wg, s_wg, wu, s_wu, s_down, wd, s_wd)
+    ws_ref = torch.empty(fw.gated_mlp_static_fp8_workspace(M, d, I), dtype=torch.uint8,
+                         device=DEV)
+    y_ref = fw.gated_mlp_static_fp8(x, s_in, wg, s_wg, wu, s_wu, s_down, wd, s_wd,
+                                    workspace=ws_ref)
     ws = torch.empty(fw.gated_mlp_static_fp8_fused_workspace(M, d, I), dtype=torch.uint8,
                      device=DEV)
     fw.launch_log_clear()
@@ -81,7 +84,14 @@ def test_fused_mlp_equals_unfused_mlp(M, d, I):
                                       workspace=ws)
     log = fw.launch_log()
     torch.cuda.synchronize()
-    assert torch.equal(y, y_ref)
+    # H is bit-identical; the down GEMM of the fused call may split its last
+    # wave over K, so Y equals the split-K GEMM of that H bit for bit and the
+    # unsplit path within the GEMM tolerance
+    h = fw.fused_workspace_views(ws, M, d, I)["h"]
+    h_ref = fw.gated_mlp_workspace_views(ws_ref, M, d, I)["h"]
+    assert torch.equal(h.view(torch.uint8), h_ref.view(torch.uint8))
+    assert torch.equal(y, fw.fp8_linear_static_ws(h, wd, s_down, s_wd))
+    assert rel_fro(bits(y), bits(y_ref)) <= GEMM_REL_FRO
     assert [r[0] for r in log] == [fw.KIND_QUANT, fw.KIND_DUAL, fw.KIND_GEMM]
     assert log[0][3] == ws.data_ptr() and log[1][1] == ws.data_ptr()   # one shared Xq
     assert log[2][1] == log[1][3]                                       # down reads H
