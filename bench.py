@@ -487,7 +487,7 @@ def kernel_bench(fw, kind, shape, steps, warmup, device):
     one JSON line."""
     flush = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     pk = peaks()
-    if kind == "gemm":
+    if kind in ("gemm", "gemm_ws"):
         M, N, K = shape
         x = synth.student_t((M, K), 4, synth.seed(1, 90, 0), device)
         w = synth.normal((N, K), synth.W_STD, synth.seed(1, 90, 10), device)
@@ -496,7 +496,12 @@ def kernel_bench(fw, kind, shape, steps, warmup, device):
         wq, s_w = fw.fp8_rtn_quantize_weight(w)
         del x, w
         y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
-        fn = lambda: fw.fp8_linear_static(xq, wq, s_in, s_w, out=y)  # noqa: E731
+        if kind == "gemm_ws":
+            wsb = torch.zeros(fw.load().fp8_linear_static_ws_bytes(), dtype=torch.uint8,
+                              device=device)
+            fn = lambda: fw.fp8_linear_static_ws(xq, wq, s_in, s_w, workspace=wsb, out=y)  # noqa: E731
+        else:
+            fn = lambda: fw.fp8_linear_static(xq, wq, s_in, s_w, out=y)  # noqa: E731
         work = 2.0 * M * N * K
         nbytes = M * K + N * K + 2 * M * N
     elif kind == "dual":
@@ -629,7 +634,7 @@ def main():
                     help="2: the two towers of each layer on two streams, joined per layer")
     ap.add_argument("--unfused", action="store_true",
                     help="time the five-kernel composition (separate gate/up GEMMs and SwiGLU-quant)")
-    ap.add_argument("--kernel", choices=("gemm", "dual", "swiglu", "quant"),
+    ap.add_argument("--kernel", choices=("gemm", "gemm_ws", "dual", "swiglu", "quant"),
                     help="time one kernel on one shape instead of the pass")
     ap.add_argument("--shape", help="M,N,K for gemm; M,I,K for dual; M,I for swiglu; M,K for quant")
     ap.add_argument("--sweep", choices=tuple(SWEEPS), help="time every kernel shape of a workload")

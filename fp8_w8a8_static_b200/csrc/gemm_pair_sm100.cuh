@@ -36,13 +36,21 @@ struct SplitPlan {
   int split_tiles;
   int splits;
   int kb_per_split;
-  float *partials;  // [split_tiles * splits][2][128][256] fp32
+  float *partials;  // [split_tiles * splits] slots, see partial_index
+  
   int *counters;    // [split_tiles][2][4]
 };
 
 struct UnitRange {
   int tile, kb0, kb1, split, slot;  // split < 0: a whole tile
 };
+
+// A slot holds one CTA pair's 2 x 128 x 256 fp32 partial as float4s indexed
+// [CTA][32-column chunk][float4 within the chunk][row], so that the 32 lanes
+// of an epilogue warp (32 consecutive rows) touch 512 contiguous bytes.
+__device__ __forceinline__ size_t partial_index(int slot, int rank, int chunk, int q4, int row) {
+  return (((static_cast<size_t>(slot) * 2 + rank) * 8 + chunk) * 8 + q4) * 128 + row;
+}
 
 __device__ __forceinline__ UnitRange unit_range(int u, const SplitPlan &p, int num_kb) {
   if (u < p.dp_tiles) return UnitRange{u, 0, num_kb, -1, -1};
@@ -252,9 +260,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // Split unit: publish this partial; only the tile's last split goes on.
       int last_split = -1;  // >= 0: this warp sums the partials of all splits
       if (ur.split >= 0) {
-        const size_t row_off = static_cast<size_t>(quarter * 32 + lane) * kPairTile;
-        float *mine = plan.partials + static_cast<size_t>(ur.slot) * (2 * 128 * kPairTile) +
-                      static_cast<size_t>(rank) * (128 * kPairTile) + row_off;
+        float4 *slots = reinterpret_cast<float4 *>(plan.partials);
+        const int prow = quarter * 32 + lane;
 #pragma unroll 1
         for (int c = 0; c < kPairTile / 32; ++c) {
           uint32_t r[32];
@@ -262,7 +269,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_ld_wait();
 #pragma unroll
           for (int q4 = 0; q4 < 8; ++q4)
-            __stcg(reinterpret_cast<float4 *>(mine + c * 32) + q4,
+            __stcg(slots + partial_index(ur.slot, static_cast<int>(rank), c, q4, prow),
                    make_float4(__uint_as_float(r[4 * q4]), __uint_as_float(r[4 * q4 + 1]),
                                __uint_as_float(r[4 * q4 + 2]), __uint_as_float(r[4 * q4 + 3])));
         }
@@ -301,8 +308,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_ld_wait();
         if (last_split >= 0) {
           // sum the tile's partials in split order (this split's from TMEM)
-          const size_t row_off = static_cast<size_t>(quarter * 32 + lane) * kPairTile +
-                                 static_cast<size_t>(c) * C::EPI_COLS;
+          const float4 *slots = reinterpret_cast<const float4 *>(plan.partials);
+          const int prow = quarter * 32 + lane;
           const int first_slot = ur.slot - last_split;
           float v[64];
 #pragma unroll
@@ -315,12 +322,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 v[32 + e] += __uint_as_float(r1[e]);
               }
             } else {
-              const float4 *src = reinterpret_cast<const float4 *>(
-                  plan.partials + static_cast<size_t>(first_slot + sp) * (2 * 128 * kPairTile) +
-                  static_cast<size_t>(rank) * (128 * kPairTile) + row_off);
 #pragma unroll
               for (int q4 = 0; q4 < 16; ++q4) {
-                const float4 w = __ldcg(src + q4);
+                // 64 columns of this chunk = 32-column chunks 2c and 2c + 1
+                const float4 w = __ldcg(slots + partial_index(first_slot + sp,
+                                                              static_cast<int>(rank),
+                                                              2 * c + q4 / 8, q4 % 8, prow));
                 v[4 * q4] += w.x;
                 v[4 * q4 + 1] += w.y;
                 v[4 * q4 + 2] += w.z;
