@@ -237,18 +237,10 @@ def build_plan(fw, layers, bufs, stream_handle, fused, ws=None):
                          M * D + I * D + 2 * M * I, 2 * M * I * D))
             plan.append(("swiglu" + tw, lib.silu_mul_2in_fp8, (g, u, M * I, s_down, h, stream_handle),
                          5 * M * I, 0))
-        if fused:
-            # the composite's down GEMM: split-K of the last wave in its scratch
-            splitk = bufs[L.tower]["splitk"]
-            plan.append(("gemm_down" + tw, lib.fp8_linear_static_ws,
-                         (h, L.wd.data_ptr(), M, D, I, s_down, L.s_wd.data_ptr(), L.y.data_ptr(),
-                          splitk.data_ptr(), splitk.numel(), stream_handle),
-                         M * I + D * I + 2 * M * D, 2 * M * D * I))
-        else:
-            plan.append(("gemm_down" + tw, lib.fp8_linear_static,
-                         (h, L.wd.data_ptr(), M, D, I, s_down, L.s_wd.data_ptr(), L.y.data_ptr(),
-                          stream_handle),
-                         M * I + D * I + 2 * M * D, 2 * M * D * I))
+        plan.append(("gemm_down" + tw, lib.fp8_linear_static,
+                     (h, L.wd.data_ptr(), M, D, I, s_down, L.s_wd.data_ptr(), L.y.data_ptr(),
+                      stream_handle),
+                     M * I + D * I + 2 * M * D, 2 * M * D * I))
     return plan
 
 

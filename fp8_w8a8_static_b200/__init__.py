@@ -398,13 +398,10 @@ def gated_mlp_static_fp8_fused(x, s_in, wg, s_wg, wu, s_wu, s_down, wd, s_wd, wo
 
 
 def fused_workspace_views(workspace: torch.Tensor, M: int, d: int, I: int):
-    """Views of the regions of gated_mlp_static_fp8_fused's workspace: Xq [M,d],
-    H [M,I] and the down GEMM's split-K scratch (as fp8_linear_static_ws)."""
+    """Views of the regions gated_mlp_static_fp8_fused writes: Xq [M,d], H [M,I]."""
     o_h = (M * d + 255) // 256 * 256
-    o_s = o_h + (M * I + 255) // 256 * 256
     ws = workspace.view(torch.uint8)
-    return dict(xq=ws[:M * d].view(FP8).view(M, d), h=ws[o_h:o_h + M * I].view(FP8).view(M, I),
-                splitk=ws[o_s:o_s + load().fp8_linear_static_ws_bytes()])
+    return dict(xq=ws[:M * d].view(FP8).view(M, d), h=ws[o_h:o_h + M * I].view(FP8).view(M, I))
 
 
 def qkv_shared_quant_workspace(M: int, d: int) -> int:

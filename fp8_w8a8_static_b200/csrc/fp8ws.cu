@@ -631,8 +631,7 @@ int fp8_gate_up_swiglu_static(const uint8_t *xq, const uint8_t *Wg, const uint8_
 size_t gated_mlp_static_fp8_fused_workspace(int64_t M, int64_t d, int64_t I) {
   if (M < 0 || d < 0 || I < 0) return 0;
   const size_t m = static_cast<size_t>(M);
-  return round256(m * static_cast<size_t>(d)) + round256(m * static_cast<size_t>(I)) +
-         splitk_bytes();
+  return round256(m * static_cast<size_t>(d)) + round256(m * static_cast<size_t>(I));
 }
 
 int gated_mlp_static_fp8_fused(const uint16_t *x, int64_t M, int64_t dm, int64_t I,
@@ -652,7 +651,6 @@ int gated_mlp_static_fp8_fused(const uint16_t *x, int64_t M, int64_t dm, int64_t
   const size_t m = static_cast<size_t>(M < 0 ? 0 : M);
   uint8_t *xq = ws;
   uint8_t *H = ws + round256(m * dm);
-  void *splitk = H + round256(m * I);
   int rc = check_gemm_args(xq, Wg, M, I, dm, s_in, s_wg, H);
   if (!rc) rc = check_gemm_args(H, Wd, M, dm, I, s_down, s_wd, y);
   if (rc) return rc;
@@ -662,12 +660,11 @@ int gated_mlp_static_fp8_fused(const uint16_t *x, int64_t M, int64_t dm, int64_t
   if (rc) return rc;
   if (M == 0) return FP8WS_OK;
   cudaStream_t st = as_stream(stream);
-  // the quantizer also clears the split-K counters used by the down GEMM
-  rc = quant_launch(d, x, M * dm, s_in, xq, st, splitk_counters(splitk), kSplitkCounterWords);
+  rc = quant_launch(d, x, M * dm, s_in, xq, st);
   if (!rc)
     rc = launch_dual_swiglu<6, 4>(d, xq, Wg, Wu, static_cast<int>(M), static_cast<int>(I),
                                   static_cast<int>(dm), s_in, s_wg, s_wu, s_down, ap, H, st);
-  if (!rc) rc = gemm_dispatch(d, H, Wd, M, dm, I, s_down, s_wd, y, st, splitk);
+  if (!rc) rc = gemm_dispatch(d, H, Wd, M, dm, I, s_down, s_wd, y, st);
   return rc;
 }
 

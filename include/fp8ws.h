@@ -107,6 +107,10 @@ FP8WS_API int fp8_linear_static(const uint8_t *xq, const uint8_t *wq, int64_t M,
  * partials in split order (deterministic: the same inputs give the same bits
  * on every call) and applies the epilogue.  The sum may differ from the
  * unsplit kernel's in the last bits of fp32, well inside the GEMM tolerance.
+ * It pays only when the tile count is far below one wave and K is long: on
+ * the two-tower down projections (48 and 192 tiles of 256 x 256 for 74 CTA
+ * pairs, K = 12288) the partial traffic and reduction cost more than the idle
+ * tail they remove, so the composite calls do not use it.
  * workspace: device, >= fp8_linear_static_ws_bytes() bytes, 256-byte aligned;
  * overwritten (the call clears its counters first).  Other arguments and
  * errors as fp8_linear_static; FP8WS_ERR_WORKSPACE for a missing, misaligned
@@ -210,12 +214,10 @@ FP8WS_API int fp8_gate_up_swiglu_static(const uint8_t *xq, const uint8_t *Wg, co
  * gated_mlp_static_fp8_fused -- gated_mlp_static_fp8 with the gate/up GEMMs
  * and the SwiGLU-quant fused (fp8_gate_up_swiglu_static): three launches
  * (quantize X, fused gate/up/SwiGLU, down GEMM) instead of five, and no G or U
- * round trip through memory.
+ * round trip through memory.  Same result, bit for bit.
  * workspace: device, gated_mlp_static_fp8_fused_workspace(M,d,I) bytes,
- * 256-byte aligned; holds Xq [M,d], then H [M,I], then the split-K scratch of
- * the down GEMM (as fp8_linear_static_ws; each region 256-byte aligned).  The
- * down projection's sums may therefore differ from gated_mlp_static_fp8's in
- * the last bits of fp32; H is identical.  act: SwiGLU variant (NULL = plain).  Other arguments as
+ * 256-byte aligned; holds Xq [M,d] then H [M,I] (each region 256-byte
+ * aligned).  act: SwiGLU variant (NULL = plain).  Other arguments as
  * gated_mlp_static_fp8.
  */
 FP8WS_API size_t gated_mlp_static_fp8_fused_workspace(int64_t M, int64_t d, int64_t I);

@@ -84,14 +84,10 @@ def test_fused_mlp_equals_unfused_mlp(M, d, I):
                                       workspace=ws)
     log = fw.launch_log()
     torch.cuda.synchronize()
-    # H is bit-identical; the down GEMM of the fused call may split its last
-    # wave over K, so Y equals the split-K GEMM of that H bit for bit and the
-    # unsplit path within the GEMM tolerance
     h = fw.fused_workspace_views(ws, M, d, I)["h"]
     h_ref = fw.gated_mlp_workspace_views(ws_ref, M, d, I)["h"]
     assert torch.equal(h.view(torch.uint8), h_ref.view(torch.uint8))
-    assert torch.equal(y, fw.fp8_linear_static_ws(h, wd, s_down, s_wd))
-    assert rel_fro(bits(y), bits(y_ref)) <= GEMM_REL_FRO
+    assert torch.equal(y, y_ref)
     assert [r[0] for r in log] == [fw.KIND_QUANT, fw.KIND_DUAL, fw.KIND_GEMM]
     assert log[0][3] == ws.data_ptr() and log[1][1] == ws.data_ptr()   # one shared Xq
     assert log[2][1] == log[1][3]                                       # down reads H
