@@ -52,7 +52,10 @@ enum { kKindQuant = 1, kKindGemm = 2, kKindSwiglu = 3, kKindCalib = 4, kKindDual
 struct DeviceInfo {
   int checked = 0;  // 0 unknown, 1 sm_100, -1 other
   int sms = 0;
-  unsigned gemm_attr_set = 0;  // bit per kernel whose attributes were set on this device
+  // bit per kernel whose attributes were set on this device: 0-2 one-CTA GEMMs,
+  // 3/5/6/7 pair GEMM scale modes (+16 direct-store), 4 dual (+8 variant,
+  // +16 direct variant, +24 direct plain), 8 per-token SwiGLU
+  unsigned gemm_attr_set = 0;
   int pair_clusters = 0;       // CTA pairs of the pair GEMM resident at once
   int dual_clusters = 0;       // CTA pairs of the gate/up dual GEMM resident at once
   // (the same for every epilogue variant: one CTA per SM either way)
@@ -340,13 +343,13 @@ int launch_gemm_pair(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int M,
 }
 
 // Gate/up dual GEMM with the SwiGLU-quant epilogue, on CTA pairs.
-template <int STAGES, int BIT, bool DIRECT>
+template <int STAGES, int BIT, bool DIRECT, bool VARIANT>
 int launch_dual_swiglu_cfg(DeviceInfo *d, const uint8_t *xq, const uint8_t *wg,
                            const uint8_t *wu, int M, int N, int K, const float *s_in,
                            const float *s_wg, const float *s_wu, const float *s_down,
                            SwigluParams act, uint8_t *h, cudaStream_t st) {
   using C = DualCfg<STAGES, DIRECT>;
-  auto kern = fp8_dual_swiglu_pair_kernel<STAGES, DIRECT>;
+  auto kern = fp8_dual_swiglu_pair_kernel<STAGES, DIRECT, VARIANT>;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -389,11 +392,21 @@ int launch_dual_swiglu(DeviceInfo *d, const uint8_t *xq, const uint8_t *wg, cons
                        int M, int N, int K, const float *s_in, const float *s_wg,
                        const float *s_wu, const float *s_down, SwigluParams act, uint8_t *h,
                        cudaStream_t st) {
-  if (direct_epilogue())
-    return launch_dual_swiglu_cfg<7, BIT + 16, true>(d, xq, wg, wu, M, N, K, s_in, s_wg, s_wu,
-                                                     s_down, act, h, st);
-  return launch_dual_swiglu_cfg<6, BIT, false>(d, xq, wg, wu, M, N, K, s_in, s_wg, s_wu, s_down,
-                                               act, h, st);
+  // the plain activation (alpha 1, no offset, no clamp) takes the kernel
+  // without the variant's per-element tests
+  const bool variant = act.alpha != 1.0f || act.beta != 0.0f || act.has_limit;
+  if (direct_epilogue()) {
+    if (variant)
+      return launch_dual_swiglu_cfg<7, BIT + 16, true, true>(d, xq, wg, wu, M, N, K, s_in, s_wg,
+                                                             s_wu, s_down, act, h, st);
+    return launch_dual_swiglu_cfg<7, BIT + 24, true, false>(d, xq, wg, wu, M, N, K, s_in, s_wg,
+                                                            s_wu, s_down, act, h, st);
+  }
+  if (variant)
+    return launch_dual_swiglu_cfg<6, BIT + 8, false, true>(d, xq, wg, wu, M, N, K, s_in, s_wg,
+                                                           s_wu, s_down, act, h, st);
+  return launch_dual_swiglu_cfg<6, BIT, false, false>(d, xq, wg, wu, M, N, K, s_in, s_wg, s_wu,
+                                                      s_down, act, h, st);
 }
 
 int check_gemm_args(const void *xq, const void *wq, int64_t M, int64_t N, int64_t K,

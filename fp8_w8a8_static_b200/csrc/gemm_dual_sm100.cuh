@@ -52,7 +52,7 @@ struct DualCfg {
   static_assert(TMEM_COLS == 512, "tmem");
 };
 
-template <int STAGES, bool DIRECT>
+template <int STAGES, bool DIRECT, bool VARIANT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     fp8_dual_swiglu_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
                                 const __grid_constant__ CUtensorMap tm_bg,
@@ -252,7 +252,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int e = 0; e < 4; ++e) {
             const float gv = __bfloat162float(__float2bfloat16_rn(__uint_as_float(g[4 * j + e]) * scale_g));
             const float uv = __bfloat162float(__float2bfloat16_rn(__uint_as_float(u[4 * j + e]) * scale_u));
-            h[e] = swiglu_mul(gv, uv, act) * inv_s;
+            h[e] = (VARIANT ? swiglu_mul(gv, uv, act) : silu_mul(gv, uv)) * inv_s;
           }
           q[j] = pack4(cvt_e4m3x2(h[0], h[1]), cvt_e4m3x2(h[2], h[3]));
         }
