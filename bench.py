@@ -55,9 +55,10 @@ CALIB_ROWS = 256
 
 
 # DRAM bytes (read + write) per launch of the dominant kernel, from an ncu
-# capture of the same kernel build on the same shape (profiles/).  None when
-# the kernel has changed since the capture.
-TRAFFIC = {}
+# capture of the same kernel build on the same shape, L2 flushed before the
+# launch (profiles/fp8_dual_swiglu_4096x12288x3072.md: 88.11 MB read + 30.05 MB
+# written).  Remove an entry when its kernel changes.
+TRAFFIC = {"gate_up_swiglu@gen": 118_168_832}
 
 
 def peaks():
@@ -737,6 +738,7 @@ def main():
                                f"M={mrows} I={I} K={D}"}
     roofline = {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
                 "frac": achieved / fp8_peak, "traffic": TRAFFIC.get(dom),
+                "traffic_unit": "DRAM bytes per launch (ncu)",
                 "kernel": f"{names[kind]}, {tower} tower, {n // args.steps} launches per step, "
                           f"{flops / n / 1e9:.1f} GFLOP and {per_kind[dom][2] / n / 1e6:.1f} MB "
                           "algorithmic per launch",
