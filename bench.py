@@ -50,15 +50,17 @@ LAYERS = synth.C4["layers"]
 D, I = synth.C4["d"], synth.C4["I"]
 TOWERS = (("und", synth.C4["M_und"]), ("gen", synth.C4["M_gen"]))
 TOKENS_PER_STEP = sum(m for _, m in TOWERS)
+# order of the towers inside a grouped launch: the generation tower's tiles
+# first, the understanding tower's fill the ragged last wave
+GROUP_ORDER = (TOWERS[1], TOWERS[0])
 CALIB_BATCHES = 16
 CALIB_ROWS = 256
 
 
 # DRAM bytes (read + write) per launch of the dominant kernel, from an ncu
 # capture of the same kernel build on the same shape, L2 flushed before the
-# launch (profiles/fp8_dual_swiglu_4096x12288x3072.md: 88.11 MB read + 30.05 MB
-# written).  Remove an entry when its kernel changes.
-TRAFFIC = {"gate_up_swiglu@gen": 118_168_832}
+# launch.  Remove an entry when its kernel changes.
+TRAFFIC = {}
 
 
 def peaks():
@@ -171,9 +173,18 @@ def prepare(fw, device, n_layers, log):
     return layers
 
 
-def make_buffers(fw, layers, device, fused):
+def make_buffers(fw, layers, device, fused, grouped=False):
     ws = {}
     bufs = {}
+    if grouped:
+        Ms = [M for _, M in GROUP_ORDER]
+        nbytes = fw.gated_mlp_static_fp8_group_workspace(Ms, D, I)
+        ws["group"] = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+        for (tower, _), v in zip(GROUP_ORDER, fw.group_workspace_views(ws["group"], Ms, D, I)):
+            bufs[tower] = v
+        for L in layers:
+            L.y = torch.empty((L.M, D), dtype=torch.bfloat16, device=device)
+        return ws, bufs
     for tower, M in TOWERS:
         if fused:
             nbytes = fw.gated_mlp_static_fp8_fused_workspace(M, D, I)
@@ -206,6 +217,71 @@ def build_value_plan(fw, layers, ws, stream_handle, fused):
         args = head + ((None,) if fused else ()) + tail
         plan.append(("mlp@" + L.tower, fn, args, 0, 0))
     return plan
+
+
+def layer_pairs(layers):
+    """The layer-towers of the pass as (generation, understanding) pairs, one per layer."""
+    by = {}
+    for L in layers:
+        by.setdefault(L.index, {})[L.tower] = L
+    return [tuple(by[l][t] for t, _ in GROUP_ORDER) for l in sorted(by)]
+
+
+def _tower_struct(fw, L, x=None, y=None):
+    x = L.x if x is None else x
+    y = L.y if y is None else y
+    return fw.MlpTower(x.data_ptr(), L.M, L.s_in.data_ptr(), L.wg.data_ptr(), L.s_wg.data_ptr(),
+                       L.wu.data_ptr(), L.s_wu.data_ptr(), L.s_down.data_ptr(), L.wd.data_ptr(),
+                       L.s_wd.data_ptr(), y.data_ptr())
+
+
+def build_group_value_plan(fw, layers, ws, stream_handle):
+    """The pass as one grouped composite call per layer (both towers):
+    gated_mlp_static_fp8_group -- three launches per layer."""
+    lib = fw.load()
+    w = ws["group"]
+    plan, keep = [], []
+    for pair in layer_pairs(layers):
+        arr = (fw.MlpTower * len(pair))(*[_tower_struct(fw, L) for L in pair])
+        keep.append(arr)  # the call reads the array: keep it alive with the plan
+        args = (ctypes.byref(arr), len(pair), D, I, None, w.data_ptr(), w.numel(), stream_handle)
+        plan.append(("mlp@group", lib.gated_mlp_static_fp8_group, args, 0, 0))
+    return plan, keep
+
+
+def build_group_plan(fw, layers, bufs, ws, stream_handle):
+    """The grouped pass as a flat list of the three grouped C-ABI calls per
+    layer, as gated_mlp_static_fp8_group issues them: quantize both towers'
+    X, the fused gate/up GEMM + SwiGLU-quant of both, the down GEMM of both
+    with the same split-K scratch (the tail of the group workspace), so that
+    the outputs are the composite call's, bit for bit."""
+    lib = fw.load()
+    w = ws["group"]
+    off = sum(fw.gated_mlp_static_fp8_fused_workspace(M, D, I) for _, M in GROUP_ORDER)
+    splitk, splitk_bytes = w.data_ptr() + off, w.numel() - off
+    plan, keep = [], []
+    for pair in layer_pairs(layers):
+        Msum = sum(L.M for L in pair)
+        q = (fw.QuantProblem * len(pair))(*[
+            fw.QuantProblem(L.x.data_ptr(), L.M * D, L.s_in.data_ptr(), bufs[L.tower]["xq"].data_ptr())
+            for L in pair])
+        g = (fw.GateUpProblem * len(pair))(*[
+            fw.GateUpProblem(bufs[L.tower]["xq"].data_ptr(), L.wg.data_ptr(), L.wu.data_ptr(), L.M,
+                             L.s_in.data_ptr(), L.s_wg.data_ptr(), L.s_wu.data_ptr(),
+                             L.s_down.data_ptr(), bufs[L.tower]["h"].data_ptr()) for L in pair])
+        dn = (fw.LinearProblem * len(pair))(*[
+            fw.LinearProblem(bufs[L.tower]["h"].data_ptr(), L.wd.data_ptr(), L.M,
+                             L.s_down.data_ptr(), L.s_wd.data_ptr(), L.y.data_ptr()) for L in pair])
+        keep += [q, g, dn]
+        plan.append(("quant@group", lib.fp8_quant_static_group,
+                     (ctypes.byref(q), len(pair), stream_handle), 3 * Msum * D, 0))
+        plan.append(("gate_up_swiglu@group", lib.fp8_gate_up_swiglu_static_group,
+                     (ctypes.byref(g), len(pair), I, D, None, stream_handle),
+                     Msum * D + 2 * len(pair) * I * D + Msum * I, 4 * Msum * I * D))
+        plan.append(("gemm_down@group", lib.fp8_linear_static_group,
+                     (ctypes.byref(dn), len(pair), D, I, splitk, splitk_bytes, stream_handle),
+                     Msum * I + len(pair) * D * I + 2 * Msum * D, 2 * Msum * D * I))
+    return plan, keep
 
 
 def build_plan(fw, layers, bufs, stream_handle, fused, ws=None):
@@ -411,6 +487,77 @@ def time_e2e(fw, layers, steps, warmup, device, dist_ctx, fused):
     return ms, h2d_bytes, d2h_bytes, h_y
 
 
+def time_e2e_group(fw, layers, steps, warmup, device, dist_ctx):
+    """time_e2e for the grouped pass: per layer, both towers' X are copied in
+    from pinned host memory, one gated_mlp_static_fp8_group call runs both
+    towers, and both Y are copied back; two device buffer sets per tower let
+    the copies of one layer overlap the compute of the previous one."""
+    pairs = layer_pairs(layers)
+    h_x = [[L.x.cpu().pin_memory() for L in pair] for pair in pairs]
+    h_y = [[torch.empty((L.M, D), dtype=torch.bfloat16).pin_memory() for L in pair]
+           for pair in pairs]
+    dx = {t: [torch.empty((M, D), dtype=torch.bfloat16, device=device) for _ in range(2)]
+          for t, M in TOWERS}
+    dy = {t: [torch.empty((M, D), dtype=torch.bfloat16, device=device) for _ in range(2)]
+          for t, M in TOWERS}
+    ws = torch.empty(fw.gated_mlp_static_fp8_group_workspace([M for _, M in GROUP_ORDER], D, I),
+                     dtype=torch.uint8, device=device)
+    comp = torch.cuda.Stream(device)
+    h2d = torch.cuda.Stream(device)
+    d2h = torch.cuda.Stream(device)
+    n = len(pairs)
+
+    def one_pass():
+        h2d.wait_stream(comp)
+        d2h.wait_stream(comp)
+        ready = [torch.cuda.Event() for _ in range(n)]
+        done = [torch.cuda.Event() for _ in range(n)]
+        copied_out = [torch.cuda.Event() for _ in range(n)]
+        for i, pair in enumerate(pairs):
+            slot = i % 2
+            with torch.cuda.stream(h2d):
+                if i >= 2:
+                    h2d.wait_event(done[i - 2])  # slot's previous user finished compute
+                for L, hx in zip(pair, h_x[i]):
+                    dx[L.tower][slot].copy_(hx, non_blocking=True)
+                ready[i].record(h2d)
+            with torch.cuda.stream(comp):
+                comp.wait_event(ready[i])
+                if i >= 2:
+                    comp.wait_event(copied_out[i - 2])  # slot's previous output copied out
+                towers = [dict(x=dx[L.tower][slot], s_in=L.s_in, wg=L.wg, s_wg=L.s_wg, wu=L.wu,
+                               s_wu=L.s_wu, s_down=L.s_down, wd=L.wd, s_wd=L.s_wd) for L in pair]
+                fw.gated_mlp_static_fp8_group(towers, workspace=ws,
+                                              outs=[dy[L.tower][slot] for L in pair], stream=comp)
+                done[i].record(comp)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(done[i])
+                for L, hy in zip(pair, h_y[i]):
+                    hy.copy_(dy[L.tower][slot], non_blocking=True)
+                copied_out[i].record(d2h)
+        comp.wait_stream(d2h)
+        comp.wait_stream(h2d)
+
+    for _ in range(warmup):
+        one_pass()
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist_ctx.barrier()
+    torch.cuda.synchronize()
+    comp.wait_stream(torch.cuda.current_stream())
+    start.record(comp)
+    for _ in range(steps):
+        one_pass()
+    stop.record(comp)
+    torch.cuda.synchronize()
+    dist_ctx.barrier()
+    ms = start.elapsed_time(stop)
+    h2d_bytes = sum(t.numel() * t.element_size() for row in h_x for t in row)
+    d2h_bytes = sum(t.numel() * t.element_size() for row in h_y for t in row)
+    return ms, h2d_bytes, d2h_bytes, [t for row in h_y for t in row], \
+        [L for pair in pairs for L in pair]
+
+
 # ------------------------------------------------------------- CPU oracle
 
 
@@ -510,6 +657,49 @@ def kernel_bench(fw, kind, shape, steps, warmup, device):
         fn = lambda: fw.fp8_gate_up_swiglu_static(xq, wg, wu, s_in, s_wg, s_wu, s_down, out=h)  # noqa: E731
         work = 4.0 * M * N * K
         nbytes = M * K + 2 * N * K + M * N
+    elif kind in ("gemm_group", "gemm_group_ws"):
+        M0, M1, N, K = shape
+        probs = []
+        for p, M in enumerate((M0, M1)):
+            x = synth.student_t((M, K), 4, synth.seed(1, 91, p), device)
+            s_in = fw.fp8_observer_scale(fw.fp8_absmax_bf16(x))
+            xq = fw.fp8_quant_static(x, s_in)
+            wq, s_w = fw.fp8_rtn_quantize_weight(
+                synth.normal((N, K), synth.W_STD, synth.seed(1, 91, 10 + p), device))
+            probs.append((xq, wq, s_in, s_w))
+            del x
+        ys = [torch.empty((M, N), dtype=torch.bfloat16, device=device) for M in (M0, M1)]
+        wsb = torch.zeros(fw.load().fp8_linear_static_ws_bytes(), dtype=torch.uint8, device=device)
+        split = kind == "gemm_group_ws"
+        fn = lambda: fw.fp8_linear_static_group(probs, outs=ys, split_k=split, workspace=wsb)  # noqa: E731
+        work = 2.0 * (M0 + M1) * N * K
+        nbytes = (M0 + M1) * K + 2 * N * K + 2 * (M0 + M1) * N
+    elif kind == "dual_group":
+        M0, M1, N, K = shape
+        probs = []
+        for p, M in enumerate((M0, M1)):
+            x = synth.activation_with_outliers(M, K, 9, 2 + p, 0, device)
+            s_in = fw.fp8_observer_scale(fw.fp8_absmax_bf16(x))
+            xq = fw.fp8_quant_static(x, s_in)
+            wg, s_wg = fw.fp8_rtn_quantize_weight(
+                synth.normal((N, K), synth.W_STD, synth.seed(4, 91, 1 + 2 * p), device))
+            wu, s_wu = fw.fp8_rtn_quantize_weight(
+                synth.normal((N, K), synth.W_STD, synth.seed(4, 91, 2 + 2 * p), device))
+            s_down = torch.tensor([0.003], dtype=torch.float32, device=device)
+            probs.append((xq, wg, wu, s_in, s_wg, s_wu, s_down))
+            del x
+        hs = [torch.empty((M, N), dtype=fw.FP8, device=device) for M in (M0, M1)]
+        fn = lambda: fw.fp8_gate_up_swiglu_static_group(probs, outs=hs)  # noqa: E731
+        work = 4.0 * (M0 + M1) * N * K
+        nbytes = (M0 + M1) * K + 4 * N * K + (M0 + M1) * N
+    elif kind == "quant_group":
+        M0, M1, K = shape
+        xs = [synth.activation_with_outliers(M, K, 9, p, 0, device) for p, M in enumerate((M0, M1))]
+        ss = [fw.fp8_observer_scale(fw.fp8_absmax_bf16(x)) for x in xs]
+        qs = [torch.empty((M, K), dtype=fw.FP8, device=device) for M in (M0, M1)]
+        fn = lambda: fw.fp8_quant_static_group(xs, ss, outs=qs)  # noqa: E731
+        work = None
+        nbytes = 3 * (M0 + M1) * K
     elif kind == "swiglu":
         M, Ii = shape
         g = synth.normal((M, Ii), 2.0, synth.seed(2, 90, 7), device)
@@ -564,6 +754,11 @@ SWEEPS = {
           [("gemm", (m, synth.C4["d"], synth.C4["I"])) for m in (1024, 4096)] +
           [("swiglu", (m, synth.C4["I"])) for m in (1024, 4096)] +
           [("quant", (m, synth.C4["d"])) for m in (1024, 4096)],
+    # the grouped launches of the same layer (generation tower first)
+    "c4g": [("dual_group", (4096, 1024, synth.C4["I"], synth.C4["d"])),
+            ("gemm_group", (4096, 1024, synth.C4["d"], synth.C4["I"])),
+            ("gemm_group_ws", (4096, 1024, synth.C4["d"], synth.C4["I"])),
+            ("quant_group", (4096, 1024, synth.C4["d"]))],
 }
 
 
@@ -624,12 +819,18 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--streams", type=int, choices=(1, 2), default=2,
-                    help="2: the two towers of each layer on two streams, joined per layer")
+                    help="towers mode: 2 runs the two towers of each layer on two streams, "
+                         "joined per layer")
     ap.add_argument("--unfused", action="store_true",
                     help="time the five-kernel composition (separate gate/up GEMMs and SwiGLU-quant)")
-    ap.add_argument("--kernel", choices=("gemm", "gemm_ws", "dual", "swiglu", "quant"),
+    ap.add_argument("--kernel", choices=("gemm", "gemm_ws", "dual", "swiglu", "quant", "gemm_group",
+                                         "gemm_group_ws", "dual_group", "quant_group"),
                     help="time one kernel on one shape instead of the pass")
-    ap.add_argument("--shape", help="M,N,K for gemm; M,I,K for dual; M,I for swiglu; M,K for quant")
+    ap.add_argument("--shape", help="M,N,K for gemm; M,I,K for dual; M,I for swiglu; M,K for quant; "
+                                    "M0,M1,N,K / M0,M1,I,K / M0,M1,K for the group kinds")
+    ap.add_argument("--mode", choices=("group", "towers"), default="group",
+                    help="group: one grouped launch per step covers both towers of a layer; "
+                         "towers: one launch per tower (see --streams)")
     ap.add_argument("--sweep", choices=tuple(SWEEPS), help="time every kernel shape of a workload")
     args = ap.parse_args()
     log = lambda m: print(m, file=sys.stderr, flush=True)  # noqa: E731
@@ -687,15 +888,20 @@ def main():
     pk = peaks()
     layers = prepare(fw, device, args.layers, log)
     fused = not args.unfused
-    ws, bufs = make_buffers(fw, layers, device, fused)
+    grouped = fused and args.mode == "group"
+    ws, bufs = make_buffers(fw, layers, device, fused, grouped)
     stream = torch.cuda.current_stream(device)
-    plan = build_plan(fw, layers, bufs, stream.cuda_stream, fused)
-    value_plan = build_value_plan(fw, layers, ws, stream.cuda_stream, fused)
+    if grouped:
+        plan, keep_plan = build_group_plan(fw, layers, bufs, ws, stream.cuda_stream)
+        value_plan, keep_value = build_group_value_plan(fw, layers, ws, stream.cuda_stream)
+    else:
+        plan = build_plan(fw, layers, bufs, stream.cuda_stream, fused)
+        value_plan = build_value_plan(fw, layers, ws, stream.cuda_stream, fused)
 
     launches_before = fw.launch_count()
     launches_per_step = sum(3 if fused else 5 for _ in value_plan)
     sampler = ClockSampler(device.index if device.index is not None else 0)
-    runner = make_stream_runner(value_plan, device) if args.streams == 2 else None
+    runner = make_stream_runner(value_plan, device) if (args.streams == 2 and not grouped) else None
     total_ms, per_kind, clocks, instrumented_ms = time_device(value_plan, args.steps,
                                                               max(args.warmup, 3), ctx, sampler,
                                                               runner, instr_plan=plan)
@@ -730,7 +936,12 @@ def main():
     ms, n, _, flops = per_kind[dom]
     achieved = (flops / n) / (ms / n / 1e3) / 1e12
     kind, tower = dom.split("@")
-    mrows = dict(TOWERS)[tower]
+    if tower == "group":
+        mrows = "+".join(f"{M} ({t})" for t, M in GROUP_ORDER)
+        tower_desc = "both towers in one launch"
+    else:
+        mrows = dict(TOWERS)[tower]
+        tower_desc = f"{tower} tower"
     names = {"gemm_down": f"fp8_gemm_pair_kernel, down projection M={mrows} N={D} K={I}",
              "gemm_gate": f"fp8_gemm_pair_kernel, gate projection M={mrows} N={I} K={D}",
              "gemm_up": f"fp8_gemm_pair_kernel, up projection M={mrows} N={I} K={D}",
@@ -739,7 +950,7 @@ def main():
     roofline = {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
                 "frac": achieved / fp8_peak, "traffic": TRAFFIC.get(dom),
                 "traffic_unit": "DRAM bytes per launch (ncu)",
-                "kernel": f"{names[kind]}, {tower} tower, {n // args.steps} launches per step, "
+                "kernel": f"{names[kind]}, {tower_desc}, {n // args.steps} launches per step, "
                           f"{flops / n / 1e9:.1f} GFLOP and {per_kind[dom][2] / n / 1e6:.1f} MB "
                           "algorithmic per launch",
                 "launch_us": ms / n * 1e3,
@@ -753,10 +964,15 @@ def main():
 
     e2e = None
     if not args.no_e2e:
-        ms, hb, db, h_y = time_e2e(fw, layers, max(1, args.steps // 2), 1, device, ctx, fused)
+        if grouped:
+            ms, hb, db, h_y, order = time_e2e_group(fw, layers, max(1, args.steps // 2), 1,
+                                                    device, ctx)
+        else:
+            ms, hb, db, h_y = time_e2e(fw, layers, max(1, args.steps // 2), 1, device, ctx, fused)
+            order = layers
         ms = ctx.max(ms)
         torch.cuda.synchronize()
-        same = torch.equal(h_y[-1], layers[-1].y.cpu())
+        same = torch.equal(h_y[-1], order[-1].y.cpu())
         e2e = {"value": aggregate_value(TOKENS_PER_STEP * max(1, args.steps // 2) * args.layers / LAYERS,
                                         ctx.world, ms / 1e3),
                "unit": UNIT, "h2d_bytes_per_step": hb, "d2h_bytes_per_step": db,
@@ -777,7 +993,9 @@ def main():
             "config": {"workload": "two-tower MoT decoder-MLP pass, 36 layers x {und M=1024, gen M=4096}, d=3072, I=12288",
                        "path": ("fused: quantize X -> gate/up GEMM with SwiGLU-quant epilogue -> down GEMM"
                                 if fused else "unfused: quantize X -> gate GEMM -> up GEMM -> SwiGLU-quant -> down GEMM"),
-                       "layers": args.layers, "streams": args.streams, "global_batch": TOKENS_PER_STEP * ctx.world,
+                       "launch": ("grouped: one launch per step covers both towers of a layer"
+                                  if grouped else f"per tower, {args.streams} stream(s)"),
+                       "layers": args.layers, "global_batch": TOKENS_PER_STEP * ctx.world,
                        "parallelism": f"replicas x{ctx.world}",
                        "l2": "inputs larger than L2 (8.15 GB of FP8 weights per pass)"},
             "roofline": roofline, "components": comp, "e2e": e2e, "cpu_baseline": cpu,

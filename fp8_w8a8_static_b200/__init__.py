@@ -28,6 +28,9 @@ __all__ = [
     "gated_mlp_static_fp8", "gated_mlp_static_fp8_workspace",
     "fp8_gate_up_swiglu_static", "gated_mlp_static_fp8_fused", "swiglu_2in_fp8", "swiglu",
     "gated_mlp_static_fp8_fused_workspace",
+    "MAX_GROUP", "QuantProblem", "LinearProblem", "GateUpProblem", "MlpTower",
+    "fp8_quant_static_group", "fp8_linear_static_group", "fp8_gate_up_swiglu_static_group",
+    "gated_mlp_static_fp8_group", "gated_mlp_static_fp8_group_workspace", "group_workspace_views",
     "qkv_shared_quant", "qkv_shared_quant_workspace", "fp8_shared_quant_linears",
     "cross_attention_qkv_static_fp8", "fp8_quant_per_token", "fp8_linear_scaled",
     "silu_mul_2in_fp8_per_token", "gated_mlp_per_token_fp8",
@@ -83,6 +86,27 @@ class LaunchRecord(ctypes.Structure):
 
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
+
+MAX_GROUP = 2  # problems per grouped call (the towers of a decoder layer)
+
+
+class QuantProblem(ctypes.Structure):
+    _fields_ = [("x", _P), ("numel", _I64), ("s_in", _P), ("xq", _P)]
+
+
+class LinearProblem(ctypes.Structure):
+    _fields_ = [("xq", _P), ("wq", _P), ("M", _I64), ("s_in", _P), ("s_w", _P), ("y", _P)]
+
+
+class GateUpProblem(ctypes.Structure):
+    _fields_ = [("xq", _P), ("Wg", _P), ("Wu", _P), ("M", _I64), ("s_in", _P), ("s_wg", _P),
+                ("s_wu", _P), ("s_down", _P), ("h", _P)]
+
+
+class MlpTower(ctypes.Structure):
+    _fields_ = [("x", _P), ("M", _I64), ("s_in", _P), ("Wg", _P), ("s_wg", _P), ("Wu", _P),
+                ("s_wu", _P), ("s_down", _P), ("Wd", _P), ("s_wd", _P), ("y", _P)]
+
 _SIGS = {
     "fp8_quant_static": (ctypes.c_int, [_P, _I64, _P, _P, _P]),
     "fp8_linear_static": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _P, _P]),
@@ -99,6 +123,13 @@ _SIGS = {
     "gated_mlp_static_fp8_fused_workspace": (ctypes.c_size_t, [_I64, _I64, _I64]),
     "gated_mlp_static_fp8_fused": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P,
                                                   _P, _P, _P, _P, _P, _P]),
+    "fp8_quant_static_group": (ctypes.c_int, [_P, ctypes.c_int, _P]),
+    "fp8_linear_static_group": (ctypes.c_int, [_P, ctypes.c_int, _I64, _I64, _P, ctypes.c_size_t,
+                                               _P]),
+    "fp8_gate_up_swiglu_static_group": (ctypes.c_int, [_P, ctypes.c_int, _I64, _I64, _P, _P]),
+    "gated_mlp_static_fp8_group_workspace": (ctypes.c_size_t, [_P, ctypes.c_int, _I64, _I64]),
+    "gated_mlp_static_fp8_group": (ctypes.c_int, [_P, ctypes.c_int, _I64, _I64, _P, _P,
+                                                  ctypes.c_size_t, _P]),
     "gated_mlp_static_fp8_noalloc": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P,
                                                     _P, _P, _P, _P]),
     "qkv_shared_quant_workspace": (ctypes.c_size_t, [_I64, _I64]),
@@ -402,6 +433,150 @@ def fused_workspace_views(workspace: torch.Tensor, M: int, d: int, I: int):
     o_h = (M * d + 255) // 256 * 256
     ws = workspace.view(torch.uint8)
     return dict(xq=ws[:M * d].view(FP8).view(M, d), h=ws[o_h:o_h + M * I].view(FP8).view(M, I))
+
+
+# ------------------------------------------------------ grouped (two towers)
+
+
+def _group_array(cls, items):
+    if not 1 <= len(items) <= MAX_GROUP:
+        raise ValueError(f"a group holds 1..{MAX_GROUP} problems, got {len(items)}")
+    return (cls * len(items))(*items)
+
+
+def fp8_quant_static_group(xs, scales, outs=None, stream=None):
+    """[E4M3_satRNE(x_p / s_p)] for up to two activations, in one launch."""
+    lib = load()
+    if len(xs) != len(scales):
+        raise ValueError("one scale per activation")
+    if outs is None:
+        outs = [torch.empty(x.shape, dtype=FP8, device=x.device) for x in xs]
+    for x, o in zip(xs, outs):
+        if o.numel() != x.numel():
+            raise ValueError("out size differs from x")
+    arr = _group_array(QuantProblem, [
+        QuantProblem(_bf16(x, "x"), x.numel(), _f32(s, "s_in"), _fp8(o, "out"))
+        for x, s, o in zip(xs, scales, outs)])
+    with _device_of(xs[0]):
+        _check(lib.fp8_quant_static_group(ctypes.byref(arr), len(arr), _stream(stream)),
+               "fp8_quant_static_group")
+    return outs
+
+
+def fp8_linear_static_group(problems, outs=None, split_k=False, workspace=None, stream=None):
+    """fp8_linear_static for up to two problems (xq [M_p,K], wq [N,K], s_in,
+    s_w) sharing N and K, in one launch; split_k lets the tiles of the last
+    partial wave be split over K (workspace scratch)."""
+    lib = load()
+    N, K = problems[0][1].shape
+    if outs is None:
+        outs = [torch.empty((xq.shape[0], N), dtype=torch.bfloat16, device=xq.device)
+                for xq, *_ in problems]
+    items = []
+    for (xq, wq, s_in, s_w), y in zip(problems, outs):
+        if xq.dim() != 2 or tuple(wq.shape) != (N, K) or xq.shape[1] != K:
+            raise ValueError("every problem must be xq [M,K] x wq [N,K]^T with shared N, K")
+        if tuple(y.shape) != (xq.shape[0], N):
+            raise ValueError("out must be [M, N]")
+        items.append(LinearProblem(_fp8(xq, "xq"), _fp8(wq, "wq"), xq.shape[0],
+                                   _f32(s_in, "s_in"), _f32(s_w, "s_w"), _bf16(y, "out")))
+    arr = _group_array(LinearProblem, items)
+    ws_ptr, ws_bytes = None, 0
+    if split_k:
+        if workspace is None:
+            workspace = _workspace(lib.fp8_linear_static_ws_bytes(), problems[0][0].device)
+        ws_ptr = _dev_ptr(workspace, "workspace", (torch.uint8,))
+        ws_bytes = workspace.numel() * workspace.element_size()
+    with _device_of(problems[0][0]):
+        _check(lib.fp8_linear_static_group(ctypes.byref(arr), len(arr), N, K, ws_ptr, ws_bytes,
+                                           _stream(stream)), "fp8_linear_static_group")
+    return outs
+
+
+def fp8_gate_up_swiglu_static_group(problems, act=None, outs=None, stream=None):
+    """fp8_gate_up_swiglu_static for up to two problems (xq [M_p,K], wg, wu
+    [I,K], s_in, s_wg, s_wu, s_down) sharing I and K, in one launch."""
+    lib = load()
+    I, K = problems[0][1].shape
+    if outs is None:
+        outs = [torch.empty((p[0].shape[0], I), dtype=FP8, device=p[0].device) for p in problems]
+    items = []
+    for (xq, wg, wu, s_in, s_wg, s_wu, s_down), h in zip(problems, outs):
+        if tuple(wg.shape) != (I, K) or tuple(wu.shape) != (I, K) or xq.shape[1] != K:
+            raise ValueError("Wg and Wu must be [I, K], shared by the group")
+        if tuple(h.shape) != (xq.shape[0], I):
+            raise ValueError("out must be [M, I]")
+        items.append(GateUpProblem(_fp8(xq, "xq"), _fp8(wg, "wg"), _fp8(wu, "wu"), xq.shape[0],
+                                   _f32(s_in, "s_in"), _f32(s_wg, "s_wg"), _f32(s_wu, "s_wu"),
+                                   _f32(s_down, "s_down"), _fp8(h, "out")))
+    arr = _group_array(GateUpProblem, items)
+    with _device_of(problems[0][0]):
+        _check(lib.fp8_gate_up_swiglu_static_group(ctypes.byref(arr), len(arr), I, K, _act(act),
+                                                   _stream(stream)),
+               "fp8_gate_up_swiglu_static_group")
+    return outs
+
+
+def gated_mlp_static_fp8_group_workspace(Ms, d: int, I: int) -> int:
+    rows = (ctypes.c_int64 * len(Ms))(*Ms)
+    return load().gated_mlp_static_fp8_group_workspace(ctypes.byref(rows), len(Ms), d, I)
+
+
+_TOWER_KEYS = ("x", "s_in", "wg", "s_wg", "wu", "s_wu", "s_down", "wd", "s_wd")
+
+
+def gated_mlp_static_fp8_group(towers, act=None, workspace=None, outs=None, stream=None):
+    """The fused gated MLP of up to two towers sharing d and I (dicts with
+    keys x, s_in, wg, s_wg, wu, s_wu, s_down, wd, s_wd) in three launches:
+    grouped quantize, grouped gate/up/SwiGLU, grouped down GEMM."""
+    lib = load()
+    for t in towers:
+        missing = [k for k in _TOWER_KEYS if k not in t]
+        if missing:
+            raise ValueError(f"tower lacks {missing}")
+    d = towers[0]["x"].shape[1]
+    I = towers[0]["wg"].shape[0]
+    Ms = [t["x"].shape[0] for t in towers]
+    for t in towers:
+        if t["x"].dim() != 2 or t["x"].shape[1] != d:
+            raise ValueError("every x must be [M, d] with the shared d")
+        if (tuple(t["wg"].shape) != (I, d) or tuple(t["wu"].shape) != (I, d)
+                or tuple(t["wd"].shape) != (d, I)):
+            raise ValueError("weight shapes must be Wg, Wu [I,d] and Wd [d,I], shared d and I")
+    need = gated_mlp_static_fp8_group_workspace(Ms, d, I)
+    if workspace is None:
+        workspace = _workspace(need, towers[0]["x"].device)
+    if outs is None:
+        outs = [torch.empty((M, d), dtype=torch.bfloat16, device=t["x"].device)
+                for M, t in zip(Ms, towers)]
+    items = []
+    for t, y in zip(towers, outs):
+        if tuple(y.shape) != (t["x"].shape[0], d):
+            raise ValueError("out must be [M, d]")
+        items.append(MlpTower(_bf16(t["x"], "x"), t["x"].shape[0], _f32(t["s_in"], "s_in"),
+                              _fp8(t["wg"], "wg"), _f32(t["s_wg"], "s_wg"), _fp8(t["wu"], "wu"),
+                              _f32(t["s_wu"], "s_wu"), _f32(t["s_down"], "s_down"),
+                              _fp8(t["wd"], "wd"), _f32(t["s_wd"], "s_wd"), _bf16(y, "out")))
+    arr = _group_array(MlpTower, items)
+    with _device_of(towers[0]["x"]):
+        _check(lib.gated_mlp_static_fp8_group(
+            ctypes.byref(arr), len(arr), d, I, _act(act),
+            _dev_ptr(workspace, "workspace", (torch.uint8,)),
+            workspace.numel() * workspace.element_size(), _stream(stream)),
+            "gated_mlp_static_fp8_group")
+    return outs
+
+
+def group_workspace_views(workspace: torch.Tensor, Ms, d: int, I: int):
+    """Per tower, views of the regions gated_mlp_static_fp8_group writes:
+    Xq [M,d] and H [M,I] (FP8)."""
+    views, off = [], 0
+    ws = workspace.view(torch.uint8)
+    for M in Ms:
+        size = gated_mlp_static_fp8_fused_workspace(M, d, I)
+        views.append(fused_workspace_views(ws[off:off + size], M, d, I))
+        off += size
+    return views
 
 
 def qkv_shared_quant_workspace(M: int, d: int) -> int:

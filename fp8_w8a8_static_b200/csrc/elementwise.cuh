@@ -76,20 +76,20 @@ __device__ __forceinline__ uint2 quant8(uint4 v, float s, float r) {
 
 // zero_words / n_zero: an optional int array cleared by block 0 (the split-K
 // counters of the GEMMs that follow on the stream).
-__global__ void __launch_bounds__(kEwThreads) quant_static_kernel(
-    const uint16_t *__restrict__ x, int64_t numel, const float *__restrict__ s_in,
-    uint8_t *__restrict__ xq, int *__restrict__ zero_words, int n_zero) {
-  pdl_launch_dependents();
-  pdl_wait();
-  if (blockIdx.x == 0)
-    for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero_words[i] = 0;
+// The blocks block0 .. block0 + nblocks - 1 of a launch quantize x, each
+// vector visited by one thread with a stride of the blocks' thread count.
+__device__ __forceinline__ void quant_static_range(const uint16_t *__restrict__ x, int64_t numel,
+                                                   const float *__restrict__ s_in,
+                                                   uint8_t *__restrict__ xq, int block,
+                                                   int nblocks) {
+  if (numel <= 0) return;
   const float s = __ldg(s_in);
   const float r = __frcp_rn(s);
   const int64_t nvec = numel >> 3;
   const uint4 *xv = reinterpret_cast<const uint4 *>(x);
   uint2 *qv = reinterpret_cast<uint2 *>(xq);
-  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t tid = static_cast<int64_t>(block) * blockDim.x + threadIdx.x;
+  const int64_t stride = static_cast<int64_t>(nblocks) * blockDim.x;
   int64_t i = tid;
   for (; i + (kEwUnroll - 1) * stride < nvec; i += kEwUnroll * stride) {
     uint4 v[kEwUnroll];
@@ -104,6 +104,40 @@ __global__ void __launch_bounds__(kEwThreads) quant_static_kernel(
     float a = __uint_as_float(static_cast<uint32_t>(x[t]) << 16);
     xq[t] = static_cast<uint8_t>(quant1(a, s, r));
   }
+}
+
+__global__ void __launch_bounds__(kEwThreads) quant_static_kernel(
+    const uint16_t *__restrict__ x, int64_t numel, const float *__restrict__ s_in,
+    uint8_t *__restrict__ xq, int *__restrict__ zero_words, int n_zero) {
+  pdl_launch_dependents();
+  pdl_wait();
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero_words[i] = 0;
+  quant_static_range(x, numel, s_in, xq, blockIdx.x, gridDim.x);
+}
+
+// Two activations, each with its own scale, quantized by one launch (the two
+// towers of a layer): blocks 0 .. split - 1 take the first, the rest the
+// second.  Block 0 also clears n_zero words at zero_words (split-K counters of
+// a later kernel), as quant_static_kernel does.
+struct QuantSeg {
+  const uint16_t *x;
+  int64_t numel;
+  const float *s_in;
+  uint8_t *xq;
+};
+
+__global__ void __launch_bounds__(kEwThreads)
+    quant_static_pair_kernel(const QuantSeg a, const QuantSeg b, int split,
+                             int *__restrict__ zero_words, int n_zero) {
+  pdl_launch_dependents();
+  pdl_wait();
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero_words[i] = 0;
+  if (static_cast<int>(blockIdx.x) < split)
+    quant_static_range(a.x, a.numel, a.s_in, a.xq, blockIdx.x, split);
+  else
+    quant_static_range(b.x, b.numel, b.s_in, b.xq, blockIdx.x - split, gridDim.x - split);
 }
 
 // ------------------------------------------------------ SwiGLU -> FP8

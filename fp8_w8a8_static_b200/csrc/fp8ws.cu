@@ -271,51 +271,106 @@ SplitPlan make_split_plan(int tiles, int pairs, int num_kb, float *partials, int
   return p;
 }
 
+// One problem of a grouped CTA-pair launch.  b2 and s_w2 (the up weight) and
+// s_down are read by the dual gate/up kernel only; out is Y (BF16) for the
+// GEMM and H (FP8) for the dual kernel.  Every problem has M >= 1.
+struct PairProblem {
+  const uint8_t *a;
+  const uint8_t *b;
+  const uint8_t *b2;
+  void *out;
+  int M;
+  const float *s_in;
+  const float *s_w;
+  const float *s_w2;
+  const float *s_down;
+};
+
+// Kernel-side description of a group whose tiles are tile_m x tile_n.
+PairGroup make_pair_group(const PairProblem *pp, int np, int N, int tile_m, int tile_n,
+                          int *tiles) {
+  PairGroup G = {};
+  G.n = np;
+  const int num_n = (N + tile_n - 1) / tile_n;
+  int total = 0;
+  for (int p = 0; p < kMaxGroup; ++p) {
+    const PairProblem &q = pp[p < np ? p : 0];
+    G.M[p] = q.M;
+    G.num_m[p] = (q.M + tile_m - 1) / tile_m;
+    G.s_in[p] = q.s_in;
+    G.s_w[p] = q.s_w;
+    G.s_w2[p] = q.s_w2;
+    G.s_down[p] = q.s_down;
+    G.out[p] = q.out;
+    if (p == 1) G.tile_start1 = total;
+    if (p < np) total += G.num_m[p] * num_n;
+  }
+  *tiles = total;
+  return G;
+}
+
+// Grid of a CTA-pair kernel: as many clusters of two as can be resident at
+// once, found by the occupancy query on the first launch of each variant.
+template <typename Kernel>
+int pair_clusters(DeviceInfo *d, Kernel kern, int smem, int bit, int *clusters_out) {
+  if (!(d->gemm_attr_set & (1u << bit))) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return FP8WS_ERR_CUDA;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (d->sms / 2));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1)
+      return FP8WS_ERR_CUDA;
+    *clusters_out = clusters;
+    d->gemm_attr_set |= 1u << bit;
+  }
+  return FP8WS_OK;
+}
+
 template <int STAGES, int BIT, int SCALE_MODE = 0, bool DIRECT = false>
-int launch_gemm_pair_cfg(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int M, int N,
-                         int K, const float *s_in, const float *s_w, uint16_t *y,
+int launch_gemm_pair_cfg(DeviceInfo *d, const PairProblem *pp, int np, int N, int K,
                          cudaStream_t st, void *splitk = nullptr) {
   using C = PairCfg<STAGES, DIRECT>;
   auto kern = fp8_gemm_pair_kernel<STAGES, SCALE_MODE, DIRECT>;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(kGemmThreads);
-  cfg.dynamicSmemBytes = C::SMEM_BYTES;
-  cfg.stream = st;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (!(d->gemm_attr_set & (1u << BIT))) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
-        cudaSuccess)
-      return FP8WS_ERR_CUDA;
-    int clusters = 0;
-    cfg.gridDim = dim3(2 * (d->sms / 2));
-    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1)
-      return FP8WS_ERR_CUDA;
-    d->pair_clusters = clusters;
-    d->gemm_attr_set |= 1u << BIT;
-  }
-  CUtensorMap ma, mb, md;
-  int rc = make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, xq, M, K, kGemmBK, 128, true);
-  if (!rc) rc = make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, wq, N, K, kGemmBK, 128, true);
-  if (!rc)
-    rc = make_map_2d(&md, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, M, N, C::EPI_COLS, 32, false);
+  int rc = pair_clusters(d, kern, C::SMEM_BYTES, BIT, &d->pair_clusters);
   if (rc) return rc;
-  const int tiles = ((M + kPairTile - 1) / kPairTile) * ((N + kPairTile - 1) / kPairTile);
+  CUtensorMap ma[kMaxGroup], mb[kMaxGroup], md[kMaxGroup];
+  for (int p = 0; p < np && !rc; ++p) {
+    const PairProblem &q = pp[p];
+    rc = make_map_2d(&ma[p], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.a, q.M, K, kGemmBK, 128, true);
+    if (!rc) rc = make_map_2d(&mb[p], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.b, N, K, kGemmBK, 128, true);
+    if (!rc)
+      rc = make_map_2d(&md[p], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q.out, q.M, N, C::EPI_COLS, 32,
+                       false);
+  }
+  if (rc) return rc;
+  if (np == 1) {
+    ma[1] = ma[0];
+    mb[1] = mb[0];
+    md[1] = md[0];
+  }
+  int tiles = 0;
+  const PairGroup G = make_pair_group(pp, np, N, kPairTile, kPairTile, &tiles);
   float *partials = static_cast<float *>(splitk);
   int *counters = splitk ? splitk_counters(splitk) : nullptr;
   const SplitPlan plan =
       make_split_plan(tiles, d->pair_clusters, (K + kGemmBK - 1) / kGemmBK, partials, counters);
   const int units = plan.dp_tiles + plan.split_tiles * plan.splits;
   const int clusters = units < d->pair_clusters ? units : d->pair_clusters;
-  if (launch_ex(kern, dim3(2 * clusters), dim3(kGemmThreads), C::SMEM_BYTES, st, 2, ma, mb, md,
-                s_in, s_w, M, N, K, kWaitLimitNs, y, plan) != cudaSuccess)
+  if (launch_ex(kern, dim3(2 * clusters), dim3(kGemmThreads), C::SMEM_BYTES, st, 2, ma[0], ma[1],
+                mb[0], mb[1], md[0], md[1], G, N, K, kWaitLimitNs, plan) != cudaSuccess)
     return FP8WS_ERR_CUDA;
-  log_launch(kKindGemm, xq, wq, y);
+  log_launch(kKindGemm, pp[0].a, pp[0].b, pp[0].out);
   return launch_status();
 }
 
@@ -332,81 +387,76 @@ bool direct_epilogue() {
 }
 
 template <int BIT, int SCALE_MODE = 0>
+int launch_gemm_pair(DeviceInfo *d, const PairProblem *pp, int np, int N, int K, cudaStream_t st,
+                     void *splitk = nullptr) {
+  if (direct_epilogue())
+    return launch_gemm_pair_cfg<7, BIT + 16, SCALE_MODE, true>(d, pp, np, N, K, st, splitk);
+  return launch_gemm_pair_cfg<6, BIT, SCALE_MODE, false>(d, pp, np, N, K, st, splitk);
+}
+
+template <int BIT, int SCALE_MODE = 0>
 int launch_gemm_pair(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int M, int N, int K,
                      const float *s_in, const float *s_w, uint16_t *y, cudaStream_t st,
                      void *splitk = nullptr) {
-  if (direct_epilogue())
-    return launch_gemm_pair_cfg<7, BIT + 16, SCALE_MODE, true>(d, xq, wq, M, N, K, s_in, s_w, y,
-                                                               st, splitk);
-  return launch_gemm_pair_cfg<6, BIT, SCALE_MODE, false>(d, xq, wq, M, N, K, s_in, s_w, y, st,
-                                                         splitk);
+  const PairProblem p = {xq, wq, nullptr, y, M, s_in, s_w, nullptr, nullptr};
+  return launch_gemm_pair<BIT, SCALE_MODE>(d, &p, 1, N, K, st, splitk);
 }
 
 // Gate/up dual GEMM with the SwiGLU-quant epilogue, on CTA pairs.
 template <int STAGES, int BIT, bool DIRECT, bool VARIANT>
-int launch_dual_swiglu_cfg(DeviceInfo *d, const uint8_t *xq, const uint8_t *wg,
-                           const uint8_t *wu, int M, int N, int K, const float *s_in,
-                           const float *s_wg, const float *s_wu, const float *s_down,
-                           SwigluParams act, uint8_t *h, cudaStream_t st) {
+int launch_dual_swiglu_cfg(DeviceInfo *d, const PairProblem *pp, int np, int N, int K,
+                           SwigluParams act, cudaStream_t st) {
   using C = DualCfg<STAGES, DIRECT>;
   auto kern = fp8_dual_swiglu_pair_kernel<STAGES, DIRECT, VARIANT>;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(kGemmThreads);
-  cfg.dynamicSmemBytes = C::SMEM_BYTES;
-  cfg.stream = st;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (!(d->gemm_attr_set & (1u << BIT))) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
-        cudaSuccess)
-      return FP8WS_ERR_CUDA;
-    int clusters = 0;
-    cfg.gridDim = dim3(2 * (d->sms / 2));
-    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1)
-      return FP8WS_ERR_CUDA;
-    d->dual_clusters = clusters;
-    d->gemm_attr_set |= 1u << BIT;
-  }
-  CUtensorMap ma, mg, mu, mh;
-  int rc = make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, xq, M, K, kGemmBK, 128, true);
-  if (!rc) rc = make_map_2d(&mg, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, wg, N, K, kGemmBK, 128, true);
-  if (!rc) rc = make_map_2d(&mu, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, wu, N, K, kGemmBK, 128, true);
-  if (!rc) rc = make_map_2d(&mh, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h, M, N, 128, 32, false);
+  int rc = pair_clusters(d, kern, C::SMEM_BYTES, BIT, &d->dual_clusters);
   if (rc) return rc;
-  const int tiles = ((M + kDualTileM - 1) / kDualTileM) * ((N + kDualTileN - 1) / kDualTileN);
+  CUtensorMap ma[kMaxGroup], mg[kMaxGroup], mu[kMaxGroup], mh[kMaxGroup];
+  for (int p = 0; p < np && !rc; ++p) {
+    const PairProblem &q = pp[p];
+    rc = make_map_2d(&ma[p], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.a, q.M, K, kGemmBK, 128, true);
+    if (!rc) rc = make_map_2d(&mg[p], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.b, N, K, kGemmBK, 128, true);
+    if (!rc)
+      rc = make_map_2d(&mu[p], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.b2, N, K, kGemmBK, 128, true);
+    if (!rc) rc = make_map_2d(&mh[p], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.out, q.M, N, 128, 32, false);
+  }
+  if (rc) return rc;
+  if (np == 1) {
+    ma[1] = ma[0];
+    mg[1] = mg[0];
+    mu[1] = mu[0];
+    mh[1] = mh[0];
+  }
+  int tiles = 0;
+  const PairGroup G = make_pair_group(pp, np, N, kDualTileM, kDualTileN, &tiles);
   const int clusters = tiles < d->dual_clusters ? tiles : d->dual_clusters;
-  if (launch_ex(kern, dim3(2 * clusters), dim3(kGemmThreads), C::SMEM_BYTES, st, 2, ma, mg, mu, mh,
-                s_in, s_wg, s_wu, s_down, act, M, N, K, kWaitLimitNs, h) != cudaSuccess)
+  if (launch_ex(kern, dim3(2 * clusters), dim3(kGemmThreads), C::SMEM_BYTES, st, 2, ma[0], mg[0],
+                mu[0], mh[0], ma[1], mg[1], mu[1], mh[1], G, act, N, K,
+                kWaitLimitNs) != cudaSuccess)
     return FP8WS_ERR_CUDA;
-  log_launch(kKindDual, xq, wg, h);
+  log_launch(kKindDual, pp[0].a, pp[0].b, pp[0].out);
   return launch_status();
 }
 
-template <int STAGES_UNUSED, int BIT>
-int launch_dual_swiglu(DeviceInfo *d, const uint8_t *xq, const uint8_t *wg, const uint8_t *wu,
-                       int M, int N, int K, const float *s_in, const float *s_wg,
-                       const float *s_wu, const float *s_down, SwigluParams act, uint8_t *h,
-                       cudaStream_t st) {
+int launch_dual_swiglu(DeviceInfo *d, const PairProblem *pp, int np, int N, int K,
+                       SwigluParams act, cudaStream_t st) {
+  constexpr int BIT = 4;
   // the plain activation (alpha 1, no offset, no clamp) takes the kernel
   // without the variant's per-element tests
   const bool variant = act.alpha != 1.0f || act.beta != 0.0f || act.has_limit;
   if (direct_epilogue()) {
-    if (variant)
-      return launch_dual_swiglu_cfg<7, BIT + 16, true, true>(d, xq, wg, wu, M, N, K, s_in, s_wg,
-                                                             s_wu, s_down, act, h, st);
-    return launch_dual_swiglu_cfg<7, BIT + 24, true, false>(d, xq, wg, wu, M, N, K, s_in, s_wg,
-                                                            s_wu, s_down, act, h, st);
+    if (variant) return launch_dual_swiglu_cfg<7, BIT + 16, true, true>(d, pp, np, N, K, act, st);
+    return launch_dual_swiglu_cfg<7, BIT + 24, true, false>(d, pp, np, N, K, act, st);
   }
-  if (variant)
-    return launch_dual_swiglu_cfg<6, BIT + 8, false, true>(d, xq, wg, wu, M, N, K, s_in, s_wg,
-                                                           s_wu, s_down, act, h, st);
-  return launch_dual_swiglu_cfg<6, BIT, false, false>(d, xq, wg, wu, M, N, K, s_in, s_wg, s_wu,
-                                                      s_down, act, h, st);
+  if (variant) return launch_dual_swiglu_cfg<6, BIT + 8, false, true>(d, pp, np, N, K, act, st);
+  return launch_dual_swiglu_cfg<6, BIT, false, false>(d, pp, np, N, K, act, st);
+}
+
+int launch_dual_swiglu(DeviceInfo *d, const uint8_t *xq, const uint8_t *wg, const uint8_t *wu,
+                       int M, int N, int K, const float *s_in, const float *s_wg,
+                       const float *s_wu, const float *s_down, SwigluParams act, uint8_t *h,
+                       cudaStream_t st) {
+  const PairProblem p = {xq, wg, wu, h, M, s_in, s_wg, s_wu, s_down};
+  return launch_dual_swiglu(d, &p, 1, N, K, act, st);
 }
 
 int check_gemm_args(const void *xq, const void *wq, int64_t M, int64_t N, int64_t K,
@@ -426,30 +476,61 @@ int check_gemm_args(const void *xq, const void *wq, int64_t M, int64_t N, int64_
 // operand bytes per tensor cycle and become L2-bandwidth bound.
 int g_forced_gemm_config = 0;  // fp8ws_set_gemm_config: 0 = cost model
 
-int gemm_dispatch(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int64_t M, int64_t N,
-                  int64_t K, const float *s_in, const float *s_w, uint16_t *y, cudaStream_t st,
-                  void *splitk = nullptr) {
-  if (M == 0) return FP8WS_OK;
-  const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
-  switch (g_forced_gemm_config) {
-    case 1: return launch_gemm_pair<3>(d, xq, wq, m, n, k, s_in, s_w, y, st, splitk);
-    case 2: return launch_gemm_cfg<256, 4, 0>(d, xq, wq, m, n, k, s_in, s_w, y, st);
-    case 3: return launch_gemm_cfg<128, 6, 1>(d, xq, wq, m, n, k, s_in, s_w, y, st);
-    case 4: return launch_gemm_cfg<64, 8, 2>(d, xq, wq, m, n, k, s_in, s_w, y, st);
-    default: break;
-  }
+// 1 = CTA pair 256 x 256, 2 = one CTA 128 x 256, 3 = 128 x 128, 4 = 128 x 64,
+// for the np problems of rows M[p] sharing N that one launch would cover.
+int gemm_choice(const DeviceInfo *d, const int64_t *M, int np, int64_t N) {
+  if (g_forced_gemm_config) return g_forced_gemm_config;
   const int pairs = d->pair_clusters > 0 ? d->pair_clusters : d->sms / 2;
   auto waves = [](int64_t tiles, int64_t slots) { return (tiles + slots - 1) / slots; };
-  const int64_t m128 = (M + 127) / 128, m256 = (M + 255) / 256;
+  int64_t m128 = 0, m256 = 0;
+  for (int p = 0; p < np; ++p) {
+    m128 += (M[p] + 127) / 128;
+    m256 += (M[p] + 255) / 256;
+  }
   const double est_pair = waves(m256 * ((N + 255) / 256), pairs) * (128.0 * 256) / 1.0;
   const double est_256 = waves(m128 * ((N + 255) / 256), d->sms) * (128.0 * 256) / 0.85;
   const double est_128 = waves(m128 * ((N + 127) / 128), d->sms) * (128.0 * 128) / 0.45;
   const double est_64 = waves(m128 * ((N + 63) / 64), d->sms) * (128.0 * 64) / 0.25;
   const double best = fmin(fmin(est_pair, est_256), fmin(est_128, est_64));
-  if (est_pair == best) return launch_gemm_pair<3>(d, xq, wq, m, n, k, s_in, s_w, y, st, splitk);
-  if (est_256 == best) return launch_gemm_cfg<256, 4, 0>(d, xq, wq, m, n, k, s_in, s_w, y, st);
-  if (est_128 == best) return launch_gemm_cfg<128, 6, 1>(d, xq, wq, m, n, k, s_in, s_w, y, st);
-  return launch_gemm_cfg<64, 8, 2>(d, xq, wq, m, n, k, s_in, s_w, y, st);
+  if (est_pair == best) return 1;
+  if (est_256 == best) return 2;
+  if (est_128 == best) return 3;
+  return 4;
+}
+
+int gemm_dispatch(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int64_t M, int64_t N,
+                  int64_t K, const float *s_in, const float *s_w, uint16_t *y, cudaStream_t st,
+                  void *splitk = nullptr) {
+  if (M == 0) return FP8WS_OK;
+  const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
+  switch (gemm_choice(d, &M, 1, N)) {
+    case 1: return launch_gemm_pair<3>(d, xq, wq, m, n, k, s_in, s_w, y, st, splitk);
+    case 2: return launch_gemm_cfg<256, 4, 0>(d, xq, wq, m, n, k, s_in, s_w, y, st);
+    case 3: return launch_gemm_cfg<128, 6, 1>(d, xq, wq, m, n, k, s_in, s_w, y, st);
+    default: return launch_gemm_cfg<64, 8, 2>(d, xq, wq, m, n, k, s_in, s_w, y, st);
+  }
+}
+
+// A group of GEMMs sharing N and K: one CTA-pair launch over all their tiles
+// when the cost model picks CTA pairs for the group, else one launch each.
+// Problems with M == 0 are skipped.
+int gemm_group_dispatch(DeviceInfo *d, const PairProblem *pp, int np, int N, int K,
+                        cudaStream_t st, void *splitk = nullptr) {
+  PairProblem live[kMaxGroup];
+  int64_t rows[kMaxGroup];
+  int n = 0;
+  for (int p = 0; p < np; ++p)
+    if (pp[p].M > 0) {
+      live[n] = pp[p];
+      rows[n++] = pp[p].M;
+    }
+  if (n == 0) return FP8WS_OK;
+  if (gemm_choice(d, rows, n, N) == 1) return launch_gemm_pair<3>(d, live, n, N, K, st, splitk);
+  int rc = FP8WS_OK;
+  for (int p = 0; p < n && !rc; ++p)
+    rc = gemm_dispatch(d, live[p].a, live[p].b, live[p].M, N, K, live[p].s_in, live[p].s_w,
+                       static_cast<uint16_t *>(live[p].out), st, splitk);
+  return rc;
 }
 
 // ----------------------------------------------------------- elementwise
@@ -460,6 +541,30 @@ int quant_launch(DeviceInfo *d, const uint16_t *x, int64_t numel, const float *s
                 dim3(kEwThreads), 0, st, 1, x, numel, s, xq, zero_words, n_zero) != cudaSuccess)
     return FP8WS_ERR_CUDA;
   log_launch(kKindQuant, x, nullptr, xq);
+  return launch_status();
+}
+
+// Two activations in one launch, the blocks shared in proportion to their
+// sizes; a single non-empty one goes to quant_launch.
+int quant_pair_launch(DeviceInfo *d, const QuantSeg *q, int nq, cudaStream_t st,
+                      int *zero_words = nullptr, int n_zero = 0) {
+  QuantSeg live[2];
+  int n = 0;
+  for (int i = 0; i < nq; ++i)
+    if (q[i].numel > 0) live[n++] = q[i];
+  if (n == 0) return FP8WS_OK;
+  if (n == 1)
+    return quant_launch(d, live[0].x, live[0].numel, live[0].s_in, live[0].xq, st, zero_words,
+                        n_zero);
+  const int64_t total = live[0].numel + live[1].numel;
+  int grid = ew_grid(d, quant_static_pair_kernel, total >> 3);
+  if (grid < 2) grid = 2;
+  int split = static_cast<int>((static_cast<double>(grid) * live[0].numel) / total + 0.5);
+  split = split < 1 ? 1 : (split > grid - 1 ? grid - 1 : split);
+  if (launch_ex(quant_static_pair_kernel, dim3(grid), dim3(kEwThreads), 0, st, 1, live[0],
+                live[1], split, zero_words, n_zero) != cudaSuccess)
+    return FP8WS_ERR_CUDA;
+  log_launch(kKindQuant, live[0].x, live[1].x, live[0].xq);
   return launch_status();
 }
 
@@ -636,7 +741,7 @@ int fp8_gate_up_swiglu_static(const uint8_t *xq, const uint8_t *Wg, const uint8_
   rc = device_info(&d);
   if (rc) return rc;
   if (M == 0) return FP8WS_OK;
-  return launch_dual_swiglu<6, 4>(d, xq, Wg, Wu, static_cast<int>(M), static_cast<int>(I),
+  return launch_dual_swiglu(d, xq, Wg, Wu, static_cast<int>(M), static_cast<int>(I),
                                   static_cast<int>(K), s_in, s_wg, s_wu, s_down, ap, h,
                                   as_stream(stream));
 }
@@ -675,7 +780,7 @@ int gated_mlp_static_fp8_fused(const uint16_t *x, int64_t M, int64_t dm, int64_t
   cudaStream_t st = as_stream(stream);
   rc = quant_launch(d, x, M * dm, s_in, xq, st);
   if (!rc)
-    rc = launch_dual_swiglu<6, 4>(d, xq, Wg, Wu, static_cast<int>(M), static_cast<int>(I),
+    rc = launch_dual_swiglu(d, xq, Wg, Wu, static_cast<int>(M), static_cast<int>(I),
                                   static_cast<int>(dm), s_in, s_wg, s_wu, s_down, ap, H, st);
   if (!rc) rc = gemm_dispatch(d, H, Wd, M, dm, I, s_down, s_wd, y, st);
   return rc;
@@ -700,6 +805,152 @@ int fp8_linear_static_ws(const uint8_t *xq, const uint8_t *wq, int64_t M, int64_
       cudaSuccess)
     return FP8WS_ERR_CUDA;
   return gemm_dispatch(d, xq, wq, M, N, K, s_in, s_w, y, st, workspace);
+}
+
+int fp8_quant_static_group(const fp8ws_quant_problem *problems, int count, void *stream) {
+  if (count < 1 || count > FP8WS_MAX_GROUP) return FP8WS_ERR_SHAPE;
+  if (!problems) return FP8WS_ERR_NULL;
+  QuantSeg seg[FP8WS_MAX_GROUP];
+  for (int p = 0; p < count; ++p) {
+    const fp8ws_quant_problem &q = problems[p];
+    if (q.numel < 0) return FP8WS_ERR_SHAPE;
+    if (q.numel > 0) {
+      if (!q.x || !q.s_in || !q.xq) return FP8WS_ERR_NULL;
+      if (!aligned16(q.x) || !aligned16(q.xq)) return FP8WS_ERR_ALIGN;
+    }
+    seg[p] = QuantSeg{q.x, q.numel, q.s_in, q.xq};
+  }
+  if (seg[0].numel == 0 && (count < 2 || seg[1].numel == 0)) return FP8WS_OK;
+  DeviceInfo *d;
+  int rc = device_info(&d);
+  if (rc) return rc;
+  return quant_pair_launch(d, seg, count, as_stream(stream));
+}
+
+int fp8_linear_static_group(const fp8ws_linear_problem *problems, int count, int64_t N,
+                            int64_t K, void *workspace, size_t workspace_bytes, void *stream) {
+  if (count < 1 || count > FP8WS_MAX_GROUP) return FP8WS_ERR_SHAPE;
+  if (!problems) return FP8WS_ERR_NULL;
+  PairProblem pp[FP8WS_MAX_GROUP];
+  int64_t rows = 0;
+  for (int p = 0; p < count; ++p) {
+    const fp8ws_linear_problem &q = problems[p];
+    const int rc = check_gemm_args(q.xq, q.wq, q.M, N, K, q.s_in, q.s_w, q.y);
+    if (rc) return rc;
+    pp[p] = PairProblem{q.xq, q.wq, nullptr, q.y, static_cast<int>(q.M), q.s_in, q.s_w,
+                        nullptr, nullptr};
+    rows += q.M;
+  }
+  if (workspace && ((reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+                    workspace_bytes < splitk_bytes()))
+    return FP8WS_ERR_WORKSPACE;
+  if (rows == 0) return FP8WS_OK;
+  DeviceInfo *d;
+  int rc = device_info(&d);
+  if (rc) return rc;
+  cudaStream_t st = as_stream(stream);
+  if (workspace &&
+      cudaMemsetAsync(splitk_counters(workspace), 0, kSplitkCounterWords * sizeof(int), st) !=
+          cudaSuccess)
+    return FP8WS_ERR_CUDA;
+  return gemm_group_dispatch(d, pp, count, static_cast<int>(N), static_cast<int>(K), st,
+                             workspace);
+}
+
+int fp8_gate_up_swiglu_static_group(const fp8ws_gate_up_problem *problems, int count,
+                                    int64_t I, int64_t K, const fp8ws_swiglu *act,
+                                    void *stream) {
+  if (count < 1 || count > FP8WS_MAX_GROUP) return FP8WS_ERR_SHAPE;
+  if (!problems) return FP8WS_ERR_NULL;
+  SwigluParams ap;
+  int rc = swiglu_params(act, &ap);
+  if (rc) return rc;
+  PairProblem live[FP8WS_MAX_GROUP];
+  int n = 0;
+  for (int p = 0; p < count; ++p) {
+    const fp8ws_gate_up_problem &q = problems[p];
+    if (!q.s_down || !q.Wu || !q.s_wu) return FP8WS_ERR_NULL;
+    rc = check_gemm_args(q.xq, q.Wg, q.M, I, K, q.s_in, q.s_wg, q.h);
+    if (rc) return rc;
+    if (!aligned16(q.Wu)) return FP8WS_ERR_ALIGN;
+    if (q.M > 0)
+      live[n++] = PairProblem{q.xq, q.Wg, q.Wu, q.h, static_cast<int>(q.M), q.s_in, q.s_wg,
+                              q.s_wu, q.s_down};
+  }
+  if (I % 16 != 0) return FP8WS_ERR_SHAPE;  // FP8 rows of H must be 16-byte multiples
+  if (n == 0) return FP8WS_OK;
+  DeviceInfo *d;
+  rc = device_info(&d);
+  if (rc) return rc;
+  return launch_dual_swiglu(d, live, n, static_cast<int>(I), static_cast<int>(K), ap,
+                            as_stream(stream));
+}
+
+size_t gated_mlp_static_fp8_group_workspace(const int64_t *M, int count, int64_t d, int64_t I) {
+  if (!M || count < 1 || count > FP8WS_MAX_GROUP || d < 0 || I < 0) return 0;
+  size_t total = 0;
+  for (int p = 0; p < count; ++p) {
+    if (M[p] < 0) return 0;
+    total += gated_mlp_static_fp8_fused_workspace(M[p], d, I);
+  }
+  return total + splitk_bytes();
+}
+
+int gated_mlp_static_fp8_group(const fp8ws_mlp_tower *towers, int count, int64_t dm, int64_t I,
+                               const fp8ws_swiglu *act, void *workspace, size_t workspace_bytes,
+                               void *stream) {
+  if (count < 1 || count > FP8WS_MAX_GROUP) return FP8WS_ERR_SHAPE;
+  if (!towers) return FP8WS_ERR_NULL;
+  SwigluParams ap;
+  int rc = swiglu_params(act, &ap);
+  if (rc) return rc;
+  int64_t rows[FP8WS_MAX_GROUP];
+  for (int p = 0; p < count; ++p) {
+    const fp8ws_mlp_tower &t = towers[p];
+    if (t.M < 0) return FP8WS_ERR_SHAPE;
+    rows[p] = t.M;
+    if (!t.s_in || !t.Wg || !t.s_wg || !t.Wu || !t.s_wu || !t.s_down || !t.Wd || !t.s_wd ||
+        (t.M != 0 && (!t.x || !t.y)))
+      return FP8WS_ERR_NULL;
+  }
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      workspace_bytes < gated_mlp_static_fp8_group_workspace(rows, count, dm, I))
+    return FP8WS_ERR_WORKSPACE;
+  // workspace: Xq_0, H_0, Xq_1, H_1 (each 256-byte aligned), then the split-K scratch
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  QuantSeg qs[FP8WS_MAX_GROUP];
+  PairProblem up[FP8WS_MAX_GROUP], down[FP8WS_MAX_GROUP];
+  int n = 0;
+  for (int p = 0; p < count; ++p) {
+    const fp8ws_mlp_tower &t = towers[p];
+    const size_t m = static_cast<size_t>(t.M);
+    uint8_t *xq = ws;
+    uint8_t *H = ws + round256(m * dm);
+    ws += gated_mlp_static_fp8_fused_workspace(t.M, dm, I);
+    if (!aligned16(t.x) || !aligned16(t.Wu)) return FP8WS_ERR_ALIGN;
+    rc = check_gemm_args(xq, t.Wg, t.M, I, dm, t.s_in, t.s_wg, H);
+    if (!rc) rc = check_gemm_args(H, t.Wd, t.M, dm, I, t.s_down, t.s_wd, t.y);
+    if (rc) return rc;
+    if (t.M == 0) continue;
+    qs[n] = QuantSeg{t.x, t.M * dm, t.s_in, xq};
+    up[n] = PairProblem{xq, t.Wg, t.Wu, H, static_cast<int>(t.M), t.s_in, t.s_wg, t.s_wu,
+                        t.s_down};
+    down[n] = PairProblem{H, t.Wd, nullptr, t.y, static_cast<int>(t.M), t.s_down, t.s_wd,
+                          nullptr, nullptr};
+    ++n;
+  }
+  if (I % 16 != 0) return FP8WS_ERR_SHAPE;
+  if (n == 0) return FP8WS_OK;  // no rows: nothing to do, nothing launched
+  DeviceInfo *d;
+  rc = device_info(&d);
+  if (rc) return rc;
+  cudaStream_t st = as_stream(stream);
+  void *splitk = ws;  // 256-byte aligned: every region above is a multiple of 256 bytes
+  rc = quant_pair_launch(d, qs, n, st, splitk_counters(splitk), kSplitkCounterWords);
+  if (!rc) rc = launch_dual_swiglu(d, up, n, static_cast<int>(I), static_cast<int>(dm), ap, st);
+  if (!rc)
+    rc = gemm_group_dispatch(d, down, n, static_cast<int>(dm), static_cast<int>(I), st, splitk);
+  return rc;
 }
 
 }  // extern "C"

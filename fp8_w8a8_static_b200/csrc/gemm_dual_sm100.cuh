@@ -19,7 +19,10 @@
 // tile overlaps the main loop of the next.  Epilogue warps read 32 columns of
 // G and of U per step, write 32 FP8 codes of each row into a 128-byte swizzled
 // row and TMA-store 32 x 128-byte boxes.  Roles, bounded waits and teardown
-// follow fp8_gemm_pair_kernel.
+// follow fp8_gemm_pair_kernel, and so does the problem group: one launch can
+// cover the gate/up projections of both towers of a Mixture-of-Transformers
+// layer (shared d and I, per-tower rows, weights and scales), their tiles
+// dealt as one sequence.
 #pragma once
 
 #include "common.cuh"
@@ -54,14 +57,15 @@ struct DualCfg {
 
 template <int STAGES, bool DIRECT, bool VARIANT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    fp8_dual_swiglu_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
-                                const __grid_constant__ CUtensorMap tm_bg,
-                                const __grid_constant__ CUtensorMap tm_bu,
-                                const __grid_constant__ CUtensorMap tm_h,
-                                const float *__restrict__ s_in, const float *__restrict__ s_wg,
-                                const float *__restrict__ s_wu,
-                                const float *__restrict__ s_down, SwigluParams act, int M,
-                                int N, int K, uint64_t timeout_ns, uint8_t *__restrict__ h_out) {
+    fp8_dual_swiglu_pair_kernel(const __grid_constant__ CUtensorMap tm_a0,
+                                const __grid_constant__ CUtensorMap tm_bg0,
+                                const __grid_constant__ CUtensorMap tm_bu0,
+                                const __grid_constant__ CUtensorMap tm_h0,
+                                const __grid_constant__ CUtensorMap tm_a1,
+                                const __grid_constant__ CUtensorMap tm_bg1,
+                                const __grid_constant__ CUtensorMap tm_bu1,
+                                const __grid_constant__ CUtensorMap tm_h1, const PairGroup G,
+                                SwigluParams act, int N, int K, uint64_t timeout_ns) {
   using C = DualCfg<STAGES, DIRECT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -84,9 +88,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const bool leader = rank == 0;
   const int cluster = blockIdx.x >> 1;
   const int nclusters = gridDim.x >> 1;
-  const int num_m = (M + kDualTileM - 1) / kDualTileM;
   const int num_n = (N + kDualTileN - 1) / kDualTileN;
-  const int num_tiles = num_m * num_n;
+  const int num_tiles = G.n > 1 ? G.tile_start1 + G.num_m[1] * num_n : G.num_m[0] * num_n;
   const int num_kb = (K + kGemmBK - 1) / kGemmBK;
 
   if (threadIdx.x == 0) {
@@ -101,10 +104,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&tm_a);
-    tma_prefetch_desc(&tm_bg);
-    tma_prefetch_desc(&tm_bu);
-    tma_prefetch_desc(&tm_h);
+    tma_prefetch_desc(&tm_a0);
+    tma_prefetch_desc(leader ? &tm_bg0 : &tm_bu0);
+    tma_prefetch_desc(&tm_h0);
+    if (G.n > 1) {
+      tma_prefetch_desc(&tm_a1);
+      tma_prefetch_desc(leader ? &tm_bg1 : &tm_bu1);
+      tma_prefetch_desc(&tm_h1);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
@@ -124,10 +131,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t issued_mask = 0, issued_parity = 0;
       bool ok = true;
       for (int t = cluster; t < num_tiles && ok; t += nclusters) {
-        const TileCoord tc = tile_coord(t, num_m, num_n);
-        const int a_row = tc.m * kDualTileM + static_cast<int>(rank) * 128;
-        const int b_row = tc.n * kDualTileN;
-        const CUtensorMap *tm_b = leader ? &tm_bg : &tm_bu;
+        const GroupTile gt = group_tile(t, G, num_n);
+        const int a_row = gt.tc.m * kDualTileM + static_cast<int>(rank) * 128;
+        const int b_row = gt.tc.n * kDualTileN;
+        const CUtensorMap *tm_a = gt.p ? &tm_a1 : &tm_a0;
+        const CUtensorMap *tm_b =
+            gt.p ? (leader ? &tm_bg1 : &tm_bu1) : (leader ? &tm_bg0 : &tm_bu0);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, timeout_ns)) {
             record_timeout(kSiteProducerEmpty);
@@ -137,7 +146,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           const uint32_t full_leader = map_shared_rank(smem_u32(&full[stage]), 0);
           if (leader) mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
-          tma_load_2d_pair(sA + stage * C::A_BYTES, &tm_a, full_leader, kb * kGemmBK, a_row);
+          tma_load_2d_pair(sA + stage * C::A_BYTES, tm_a, full_leader, kb * kGemmBK, a_row);
           tma_load_2d_pair(sB + stage * C::B_BYTES, tm_b, full_leader, kb * kGemmBK, b_row);
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -204,12 +213,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------ epilogue (both CTAs)
     const int ew = warp - 2;
     const int quarter = warp & 3;
-    const float scale_g = __ldg(s_in) * __ldg(s_wg);
-    const float scale_u = __ldg(s_in) * __ldg(s_wu);
-    const float inv_s = __frcp_rn(__ldg(s_down));
+    float scale_g[kMaxGroup], scale_u[kMaxGroup], inv_s[kMaxGroup];
+#pragma unroll
+    for (int p = 0; p < kMaxGroup; ++p) {
+      const int q = p < G.n ? p : 0;
+      scale_g[p] = __ldg(pick(G.s_in, q)) * __ldg(pick(G.s_w, q));
+      scale_u[p] = __ldg(pick(G.s_in, q)) * __ldg(pick(G.s_w2, q));
+      inv_s[p] = __frcp_rn(__ldg(pick(G.s_down, q)));
+    }
     uint32_t it = 0;
     for (int t = cluster; t < num_tiles; t += nclusters, ++it) {
-      const TileCoord tc = tile_coord(t, num_m, num_n);
+      const GroupTile gt = group_tile(t, G, num_n);
+      const TileCoord tc = gt.tc;
+      const int M = pick(G.M, gt.p);
+      const float sg = gt.p ? scale_g[1] : scale_g[0];
+      const float su = gt.p ? scale_u[1] : scale_u[0];
+      const float is = gt.p ? inv_s[1] : inv_s[0];
+      const CUtensorMap *tm_h = gt.p ? &tm_h1 : &tm_h0;
+      uint8_t *h_out = static_cast<uint8_t *>(pick(G.out, gt.p));
       const uint32_t acc = it & 1u;
       const uint32_t acc_phase = (it >> 1) & 1u;
       if (!mbar_wait_bounded_warp(&tfull[acc], acc_phase, abort_flag, timeout_ns)) {
@@ -250,9 +271,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           float h[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float gv = __bfloat162float(__float2bfloat16_rn(__uint_as_float(g[4 * j + e]) * scale_g));
-            const float uv = __bfloat162float(__float2bfloat16_rn(__uint_as_float(u[4 * j + e]) * scale_u));
-            h[e] = (VARIANT ? swiglu_mul(gv, uv, act) : silu_mul(gv, uv)) * inv_s;
+            const float gv = __bfloat162float(__float2bfloat16_rn(__uint_as_float(g[4 * j + e]) * sg));
+            const float uv = __bfloat162float(__float2bfloat16_rn(__uint_as_float(u[4 * j + e]) * su));
+            h[e] = (VARIANT ? swiglu_mul(gv, uv, act) : silu_mul(gv, uv)) * is;
           }
           q[j] = pack4(cvt_e4m3x2(h[0], h[1]), cvt_e4m3x2(h[2], h[3]));
         }
@@ -274,7 +295,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         fence_async_shared();
         __syncwarp();
         if (lane == 0 && store) {
-          tma_store_2d(&tm_h, buf, col0, row0);
+          tma_store_2d(tm_h, buf, col0, row0);
         }
         if (lane == 0) tma_store_commit();
       }

@@ -1,18 +1,21 @@
 // FP8 E4M3 W8A8 GEMM on CTA pairs (tcgen05 cta_group::2), for sm_100a.
 //
-//   Y[M,N] = bf16( (s_in * s_w) * Xq[M,K] . Wq[N,K]^T ),  fp32 accumulation
+//   Y_p[M_p,N] = bf16( (s_in_p * s_w_p) * Xq_p[M_p,K] . Wq_p[N,K]^T ),  fp32 accumulation
 //
-// Same contract as fp8_gemm_kernel, with 256 x 256 output tiles computed by a
-// cluster of two CTAs on the two SMs of a TPC.  Each CTA loads 128 rows of A
-// and 128 rows of B per 128-byte K step (32 KB instead of 48 KB per SM for the
-// same tensor work), both CTAs' loads count on the leader CTA's barrier, and
-// the leader issues one M=256, N=256 tcgen05.mma over both CTAs' shared
-// memory.  Each CTA's TMEM holds the accumulator of its own 128 rows; both
-// CTAs run the epilogue on their own rows.
+// for a group of one or two problems p that share N and K (the two towers of a
+// Mixture-of-Transformers layer), in one persistent launch.  256 x 256 output
+// tiles are computed by a cluster of two CTAs on the two SMs of a TPC.  Each
+// CTA loads 128 rows of A and 128 rows of B per 128-byte K step (32 KB instead
+// of 48 KB per SM for the same tensor work), both CTAs' loads count on the
+// leader CTA's barrier, and the leader issues one M=256, N=256 tcgen05.mma over
+// both CTAs' shared memory.  Each CTA's TMEM holds the accumulator of its own
+// 128 rows; both CTAs run the epilogue on their own rows.
 //   warp 0      TMA producer (both CTAs; no cluster multicast)
 //   warp 1      TMEM allocation (both CTAs, cta_group::2); MMA issue (leader)
 //   warps 2..5  epilogue (both CTAs)
-// Bounded waits as in fp8_gemm_kernel.  Both CTAs always reach the final
+// The tiles of the group form one sequence (problem 0's, then problem 1's),
+// dealt round-robin to the clusters, so the second problem fills the ragged
+// last wave of the first.  Bounded waits as in fp8_gemm_kernel.  Both CTAs always reach the final
 // cluster barrier, so neither leaves while its peer may still touch its
 // shared memory or TMEM.
 #pragma once
@@ -23,6 +26,40 @@
 namespace fp8ws {
 
 constexpr int kPairTile = 256;  // output rows and columns per CTA pair
+constexpr int kMaxGroup = 2;    // problems per grouped launch
+
+// The problems of one launch.  Global tile g belongs to problem 1 when n == 2
+// and g >= tile_start1.  s_w2 and s_down are read by the dual gate/up kernel
+// only; out[p] is Y_p (BF16) or H_p (FP8) for the register-store epilogues.
+struct PairGroup {
+  int n;
+  int tile_start1;
+  int M[kMaxGroup];
+  int num_m[kMaxGroup];
+  const float *s_in[kMaxGroup];
+  const float *s_w[kMaxGroup];
+  const float *s_w2[kMaxGroup];
+  const float *s_down[kMaxGroup];
+  void *out[kMaxGroup];
+};
+
+struct GroupTile {
+  int p;
+  TileCoord tc;
+};
+
+// Member p of a group array, by selection rather than indexing, so that the
+// kernel parameter block is not copied to local memory.
+template <typename T>
+__device__ __forceinline__ T pick(const T (&a)[kMaxGroup], int p) {
+  return p ? a[1] : a[0];
+}
+
+__device__ __forceinline__ GroupTile group_tile(int g, const PairGroup &G, int num_n) {
+  const int p = (G.n > 1 && g >= G.tile_start1) ? 1 : 0;
+  const int local = p ? g - G.tile_start1 : g;
+  return GroupTile{p, tile_coord(local, pick(G.num_m, p), num_n)};
+}
 
 // Split-K of the remainder tiles.  Units 0 .. dp_tiles-1 are whole tiles (the
 // full waves); the last split_tiles tiles are each cut into `splits` K ranges
@@ -37,7 +74,6 @@ struct SplitPlan {
   int splits;
   int kb_per_split;
   float *partials;  // [split_tiles * splits] slots, see partial_index
-  
   int *counters;    // [split_tiles][2][4]
 };
 
@@ -90,11 +126,13 @@ struct PairCfg {
 
 template <int STAGES, int SCALE_MODE, bool DIRECT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
-                         const __grid_constant__ CUtensorMap tm_b,
-                         const __grid_constant__ CUtensorMap tm_d, const float *__restrict__ s_in,
-                         const float *__restrict__ s_w, int M, int N, int K,
-                         uint64_t timeout_ns, uint16_t *__restrict__ y_out, SplitPlan plan) {
+    fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a0,
+                         const __grid_constant__ CUtensorMap tm_a1,
+                         const __grid_constant__ CUtensorMap tm_b0,
+                         const __grid_constant__ CUtensorMap tm_b1,
+                         const __grid_constant__ CUtensorMap tm_d0,
+                         const __grid_constant__ CUtensorMap tm_d1, const PairGroup G, int N,
+                         int K, uint64_t timeout_ns, SplitPlan plan) {
   using C = PairCfg<STAGES, DIRECT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -117,7 +155,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const bool leader = rank == 0;
   const int cluster = blockIdx.x >> 1;
   const int nclusters = gridDim.x >> 1;
-  const int num_m = (M + kPairTile - 1) / kPairTile;
   const int num_n = (N + kPairTile - 1) / kPairTile;
   const int num_kb = (K + kGemmBK - 1) / kGemmBK;
   const int num_units = plan.dp_tiles + plan.split_tiles * plan.splits;
@@ -134,9 +171,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&tm_a);
-    tma_prefetch_desc(&tm_b);
-    tma_prefetch_desc(&tm_d);
+    tma_prefetch_desc(&tm_a0);
+    tma_prefetch_desc(&tm_b0);
+    tma_prefetch_desc(&tm_d0);
+    if (G.n > 1) {
+      tma_prefetch_desc(&tm_a1);
+      tma_prefetch_desc(&tm_b1);
+      tma_prefetch_desc(&tm_d1);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
@@ -157,9 +199,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       for (int u = cluster; u < num_units && ok; u += nclusters) {
         const UnitRange ur = unit_range(u, plan, num_kb);
-        const TileCoord tc = tile_coord(ur.tile, num_m, num_n);
-        const int a_row = tc.m * kPairTile + static_cast<int>(rank) * 128;
-        const int b_row = tc.n * kPairTile + static_cast<int>(rank) * 128;
+        const GroupTile gt = group_tile(ur.tile, G, num_n);
+        const CUtensorMap *tm_a = gt.p ? &tm_a1 : &tm_a0;
+        const CUtensorMap *tm_b = gt.p ? &tm_b1 : &tm_b0;
+        const int a_row = gt.tc.m * kPairTile + static_cast<int>(rank) * 128;
+        const int b_row = gt.tc.n * kPairTile + static_cast<int>(rank) * 128;
         for (int kb = ur.kb0; kb < ur.kb1; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, timeout_ns)) {
             record_timeout(kSiteProducerEmpty);
@@ -169,8 +213,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           const uint32_t full_leader = map_shared_rank(smem_u32(&full[stage]), 0);
           if (leader) mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
-          tma_load_2d_pair(sA + stage * C::A_BYTES, &tm_a, full_leader, kb * kGemmBK, a_row);
-          tma_load_2d_pair(sB + stage * C::B_BYTES, &tm_b, full_leader, kb * kGemmBK, b_row);
+          tma_load_2d_pair(sA + stage * C::A_BYTES, tm_a, full_leader, kb * kGemmBK, a_row);
+          tma_load_2d_pair(sB + stage * C::B_BYTES, tm_b, full_leader, kb * kGemmBK, b_row);
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -239,11 +283,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------ epilogue (both CTAs)
     const int ew = warp - 2;
     const int quarter = warp & 3;
-    const float scale = (SCALE_MODE == 0) ? __ldg(s_in) * __ldg(s_w) : 0.0f;
     uint32_t it = 0, chunk = 0;
     for (int u = cluster; u < num_units; u += nclusters, ++it) {
       const UnitRange ur = unit_range(u, plan, num_kb);
-      const TileCoord tc = tile_coord(ur.tile, num_m, num_n);
+      const GroupTile gt = group_tile(ur.tile, G, num_n);
+      const TileCoord tc = gt.tc;
+      const int M = pick(G.M, gt.p);
+      const CUtensorMap *tm_d = gt.p ? &tm_d1 : &tm_d0;
+      const float *s_in = pick(G.s_in, gt.p);
+      const float *s_w = pick(G.s_w, gt.p);
+      uint16_t *y_out = static_cast<uint16_t *>(pick(G.out, gt.p));
       const uint32_t acc = it & 1u;
       const uint32_t acc_phase = (it >> 1) & 1u;
       if (!mbar_wait_bounded_warp(&tfull[acc], acc_phase, abort_flag, timeout_ns)) {
@@ -290,6 +339,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (lane == 0) atomicExch(cnt, 0);  // ready for the next launch
         last_split = ur.split;
       }
+      const float scale = (SCALE_MODE == 0) ? __ldg(s_in) * __ldg(s_w) : 0.0f;
       float row_scale = 0.0f;  // this thread's row factor (row0 + lane)
       if (SCALE_MODE != 0) {
         const int my_row = row0 + lane;
@@ -401,7 +451,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           fence_async_shared();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&tm_d, buf, col0, row0);
+            tma_store_2d(tm_d, buf, col0, row0);
             tma_store_commit();
           }
         }

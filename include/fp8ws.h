@@ -31,6 +31,8 @@
  *  [PR] TensorRT-LLM pull request "Load static FP8 Cosmos3 Nano/Super
  *       checkpoints without re-quantizing them", sections Description and
  *       What changed.
+ *  [BLOG] "Running Cosmos 3 Robot Policies on a Single RTX 4090", section
+ *       "Make it fit via quantization".
  */
 #ifndef FP8WS_H
 #define FP8WS_H
@@ -227,6 +229,116 @@ FP8WS_API int gated_mlp_static_fp8_fused(const uint16_t *x, int64_t M, int64_t d
                                          const float *s_down, const fp8ws_swiglu *act,
                                          const uint8_t *Wd, const float *s_wd, void *workspace,
                                          uint16_t *y, void *stream);
+
+/* ------------------------------------------------- grouped (two-tower) calls
+ *
+ * A Mixture-of-Transformers decoder layer has two towers, an understanding and
+ * a generation branch, with the same Linear shapes but their own token counts,
+ * weights and calibrated scales ([BLOG] Make it fit via quantization: the two
+ * branches are quantized separately; [MC] Scheme table: one static scale per
+ * tensor).  A grouped call runs the same step for up to FP8WS_MAX_GROUP such
+ * problems in ONE kernel launch: their tiles form one sequence dealt to the
+ * persistent CTAs, so the smaller tower fills the last, partly idle wave of
+ * the larger one.  Each problem's result is the one the single-problem call
+ * gives, bit for bit (the split-K variant excepted, as fp8_linear_static_ws).
+ * Problems with no rows (M == 0, numel == 0) are skipped and may carry NULL
+ * tensor pointers.  count: 1..FP8WS_MAX_GROUP (FP8WS_ERR_SHAPE otherwise).
+ * The problem arrays live in host memory and are read during the call only.
+ */
+#define FP8WS_MAX_GROUP 2
+
+typedef struct {
+  const uint16_t *x; /* device, numel BF16 values */
+  int64_t numel;     /* >= 0 */
+  const float *s_in; /* device fp32 scale of this tensor */
+  uint8_t *xq;       /* device, numel FP8 codes (written) */
+} fp8ws_quant_problem;
+
+typedef struct {
+  const uint8_t *xq; /* device [M,K] FP8 */
+  const uint8_t *wq; /* device [N,K] FP8 */
+  int64_t M;         /* >= 0 */
+  const float *s_in; /* device fp32 */
+  const float *s_w;  /* device fp32 */
+  uint16_t *y;       /* device [M,N] BF16 (written) */
+} fp8ws_linear_problem;
+
+typedef struct {
+  const uint8_t *xq;   /* device [M,K] FP8 */
+  const uint8_t *Wg;   /* device [I,K] FP8 */
+  const uint8_t *Wu;   /* device [I,K] FP8 */
+  int64_t M;           /* >= 0 */
+  const float *s_in;   /* device fp32, shared by gate and up */
+  const float *s_wg;   /* device fp32 */
+  const float *s_wu;   /* device fp32 */
+  const float *s_down; /* device fp32, down_proj's input scale */
+  uint8_t *h;          /* device [M,I] FP8 (written) */
+} fp8ws_gate_up_problem;
+
+typedef struct {
+  const uint16_t *x;   /* device [M,d] BF16 */
+  int64_t M;           /* >= 0 */
+  const float *s_in;   /* device fp32, gate/up input scale */
+  const uint8_t *Wg;   /* device [I,d] FP8 */
+  const float *s_wg;
+  const uint8_t *Wu;   /* device [I,d] FP8 */
+  const float *s_wu;
+  const float *s_down; /* device fp32, down_proj's input scale */
+  const uint8_t *Wd;   /* device [d,I] FP8 */
+  const float *s_wd;
+  uint16_t *y;         /* device [M,d] BF16 (written) */
+} fp8ws_mlp_tower;
+
+/*
+ * fp8_quant_static_group -- fp8_quant_static for count activations, each
+ * with its own scale, in one launch.  Errors as fp8_quant_static.
+ */
+FP8WS_API int fp8_quant_static_group(const fp8ws_quant_problem *problems, int count,
+                                     void *stream);
+
+/*
+ * fp8_linear_static_group -- fp8_linear_static for count problems sharing N
+ * and K, in one CTA-pair launch when the tile cost model picks CTA pairs for
+ * the group's combined tiles, else one launch per problem.
+ * workspace: NULL (no split), or >= fp8_linear_static_ws_bytes() bytes,
+ * 256-byte aligned, for splitting the tiles of the group's last partial wave
+ * over K as fp8_linear_static_ws does (deterministic; the call clears its
+ * counters first).  Sizes and errors as fp8_linear_static, per problem;
+ * FP8WS_ERR_WORKSPACE for a misaligned or short workspace.
+ */
+FP8WS_API int fp8_linear_static_group(const fp8ws_linear_problem *problems, int count,
+                                      int64_t N, int64_t K, void *workspace,
+                                      size_t workspace_bytes, void *stream);
+
+/*
+ * fp8_gate_up_swiglu_static_group -- fp8_gate_up_swiglu_static for count
+ * problems sharing I and K (each with its own rows, weights and scales) in
+ * one launch; act (NULL = plain SwiGLU) applies to all.  Bit-identical per
+ * problem to fp8_gate_up_swiglu_static.  Sizes and errors as that call.
+ */
+FP8WS_API int fp8_gate_up_swiglu_static_group(const fp8ws_gate_up_problem *problems, int count,
+                                              int64_t I, int64_t K, const fp8ws_swiglu *act,
+                                              void *stream);
+
+/*
+ * gated_mlp_static_fp8_group -- gated_mlp_static_fp8_fused for the towers of
+ * one decoder layer (shared d and I) in three launches in all:
+ * fp8_quant_static_group, fp8_gate_up_swiglu_static_group and
+ * fp8_linear_static_group (down projections; split-K scratch in the
+ * workspace).  Each tower's y equals gated_mlp_static_fp8_fused's for that
+ * tower within the GEMM tolerance; with no tile of the down group split over
+ * K (the plan splits only a ragged last wave) the two are identical bit for
+ * bit.
+ * workspace: device, gated_mlp_static_fp8_group_workspace(M, count, d, I)
+ * bytes, 256-byte aligned; holds Xq and H of each tower and the split-K
+ * scratch, and is overwritten.  M: host array of the towers' row counts.
+ * Sizes: as gated_mlp_static_fp8_fused per tower.
+ */
+FP8WS_API size_t gated_mlp_static_fp8_group_workspace(const int64_t *M, int count, int64_t d,
+                                                      int64_t I);
+FP8WS_API int gated_mlp_static_fp8_group(const fp8ws_mlp_tower *towers, int count, int64_t d,
+                                         int64_t I, const fp8ws_swiglu *act, void *workspace,
+                                         size_t workspace_bytes, void *stream);
 
 /*
  * qkv_shared_quant -- Q/K/V projections from one shared quantization.

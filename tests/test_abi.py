@@ -110,3 +110,80 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(fw, "_LIB_PATH", str(tmp_path / "absent.so"))
     with pytest.raises(RuntimeError, match="missing"):
         fw.load()
+
+
+def _header_struct_fields(name):
+    """Field names of `typedef struct { ... } name;` in the header, in order."""
+    text = open(HEADER).read()
+    body = re.search(r"typedef struct \{([^{}]*)\}\s*" + name + r"\s*;", text).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    fields = []
+    for decl in body.split(";"):
+        decl = decl.strip()
+        if decl:
+            fields += [part.strip().lstrip("*").split()[-1].lstrip("*")
+                       for part in decl.split(",")]
+    return fields
+
+
+@pytest.mark.parametrize("cname,pyname", [
+    ("fp8ws_quant_problem", "QuantProblem"), ("fp8ws_linear_problem", "LinearProblem"),
+    ("fp8ws_gate_up_problem", "GateUpProblem"), ("fp8ws_mlp_tower", "MlpTower"),
+    ("fp8ws_swiglu", "Swiglu")])
+def test_group_structs_match_header(cname, pyname):
+    """The ctypes layouts follow the header's fields in order.  The group
+    structs hold only pointers and 64-bit integers, and the SwiGLU descriptor
+    only 4-byte fields, so matching names in order fixes the layout."""
+    cls = getattr(fw, pyname)
+    assert [f for f, _ in cls._fields_] == _header_struct_fields(cname)
+
+
+def test_group_argument_checks_before_cuda(lib):
+    import ctypes
+    a = 1 << 20
+    n0 = fw.launch_count()
+    q = (fw.QuantProblem * 2)(fw.QuantProblem(a, 64, a, a), fw.QuantProblem(a + 2, 64, a, a))
+    assert lib.fp8_quant_static_group(ctypes.byref(q), 2, None) == fw.ERR_ALIGN
+    assert lib.fp8_quant_static_group(ctypes.byref(q), 3, None) == fw.ERR_SHAPE
+    assert lib.fp8_quant_static_group(ctypes.byref(q), 0, None) == fw.ERR_SHAPE
+    assert lib.fp8_quant_static_group(None, 1, None) == fw.ERR_NULL
+    lp = (fw.LinearProblem * 2)(fw.LinearProblem(a, a, 64, a, a, a),
+                                fw.LinearProblem(a, a, 64, None, a, a))
+    assert lib.fp8_linear_static_group(ctypes.byref(lp), 2, 256, 512, None, 0, None) == fw.ERR_NULL
+    assert lib.fp8_linear_static_group(ctypes.byref(lp), 1, 260, 512, None, 0, None) == fw.ERR_SHAPE
+    assert lib.fp8_linear_static_group(ctypes.byref(lp), 1, 256, 512, a + 16, 1 << 30,
+                                       None) == fw.ERR_WORKSPACE
+    assert lib.fp8_linear_static_group(ctypes.byref(lp), 1, 256, 512, a, 1024,
+                                       None) == fw.ERR_WORKSPACE
+    gp = (fw.GateUpProblem * 1)(fw.GateUpProblem(a, a, a, 64, a, a, a, a, a))
+    assert lib.fp8_gate_up_swiglu_static_group(ctypes.byref(gp), 1, 264, 512, None,
+                                               None) == fw.ERR_SHAPE   # I % 16
+    bad = fw.swiglu(1.0, 0.0, -1.0)
+    assert lib.fp8_gate_up_swiglu_static_group(ctypes.byref(gp), 1, 256, 512, ctypes.byref(bad),
+                                               None) == fw.ERR_BAD_SCALE
+    t = fw.MlpTower(a, 64, a, a, a, a, a, a, a, a, a)
+    tw = (fw.MlpTower * 2)(t, t)
+    rows = (ctypes.c_int64 * 2)(64, 64)
+    need = lib.gated_mlp_static_fp8_group_workspace(ctypes.byref(rows), 2, 256, 704)
+    assert need == 2 * lib.gated_mlp_static_fp8_fused_workspace(64, 256, 704) + \
+        lib.fp8_linear_static_ws_bytes()
+    assert lib.gated_mlp_static_fp8_group(ctypes.byref(tw), 2, 256, 704, None, a, need - 256,
+                                          None) == fw.ERR_WORKSPACE
+    assert lib.gated_mlp_static_fp8_group(ctypes.byref(tw), 2, 256, 700, None, a, 1 << 40,
+                                          None) == fw.ERR_SHAPE
+    assert lib.gated_mlp_static_fp8_group_workspace(None, 2, 256, 704) == 0
+    # towers with no rows: nothing to do, nothing launched
+    e = fw.MlpTower(None, 0, a, a, a, a, a, a, a, a, None)
+    te = (fw.MlpTower * 2)(e, e)
+    assert lib.gated_mlp_static_fp8_group(ctypes.byref(te), 2, 256, 704, None, a, 1 << 30,
+                                          None) == fw.OK
+    assert fw.launch_count() == n0
+    eq = (fw.QuantProblem * 2)(fw.QuantProblem(None, 0, None, None),
+                               fw.QuantProblem(None, 0, None, None))
+    assert lib.fp8_quant_static_group(ctypes.byref(eq), 2, None) == fw.OK
+    el = (fw.LinearProblem * 1)(fw.LinearProblem(None, a, 0, a, a, None))
+    assert lib.fp8_linear_static_group(ctypes.byref(el), 1, 256, 512, None, 0, None) == fw.OK
+    eg = (fw.GateUpProblem * 1)(fw.GateUpProblem(None, a, a, 0, a, a, a, a, None))
+    assert lib.fp8_gate_up_swiglu_static_group(ctypes.byref(eg), 1, 256, 512, None,
+                                               None) == fw.OK
+    assert fw.launch_count() == n0
