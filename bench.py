@@ -59,8 +59,9 @@ CALIB_ROWS = 256
 
 # DRAM bytes (read + write) per launch of the dominant kernel, from an ncu
 # capture of the same kernel build on the same shape, L2 flushed before the
-# launch.  Remove an entry when its kernel changes.
-TRAFFIC = {}
+# launch (profiles/fp8_dual_swiglu_group_4096_1024x12288x3072.md: 166.78 MB read
+# + 55.44 MB written).  Remove an entry when its kernel changes.
+TRAFFIC = {"gate_up_swiglu@group": 222_221_568}
 
 
 def peaks():
@@ -487,68 +488,95 @@ def time_e2e(fw, layers, steps, warmup, device, dist_ctx, fused):
     return ms, h2d_bytes, d2h_bytes, h_y
 
 
-def time_e2e_group(fw, layers, steps, warmup, device, dist_ctx):
-    """time_e2e for the grouped pass: per layer, both towers' X are copied in
-    from pinned host memory, one gated_mlp_static_fp8_group call runs both
-    towers, and both Y are copied back; two device buffer sets per tower let
-    the copies of one layer overlap the compute of the previous one."""
+def time_e2e_group(fw, layers, steps, warmup, device, dist_ctx, slots=4, copy_streams=2):
+    """time_e2e for the grouped pass, as a stream of steps: per layer, both
+    towers' X are copied in from pinned host memory on a copy stream, one
+    gated_mlp_static_fp8_group call runs both towers on the compute stream,
+    and both Y are copied back on a third stream.  `slots` device buffer sets
+    per tower rotate over the layers of consecutive steps, and each copy or
+    call waits only for the earlier users of its slot, so the copies of one
+    layer overlap the compute of others across step boundaries too (a later
+    step's inputs stream in while the earlier step's last results stream out).
+    copy_streams=2 gives each tower its own pair of copy streams.  Four slots
+    and per-tower copy streams measured 24.4-24.9 ms per step against 27.0 ms
+    for two slots, one copy stream per direction and a full join between
+    steps (same box); the copies alone take about 24 ms.  The timed region
+    ends when the last step's last result is in host memory."""
     pairs = layer_pairs(layers)
     h_x = [[L.x.cpu().pin_memory() for L in pair] for pair in pairs]
     h_y = [[torch.empty((L.M, D), dtype=torch.bfloat16).pin_memory() for L in pair]
            for pair in pairs]
-    dx = {t: [torch.empty((M, D), dtype=torch.bfloat16, device=device) for _ in range(2)]
+    dx = {t: [torch.empty((M, D), dtype=torch.bfloat16, device=device) for _ in range(slots)]
           for t, M in TOWERS}
-    dy = {t: [torch.empty((M, D), dtype=torch.bfloat16, device=device) for _ in range(2)]
+    dy = {t: [torch.empty((M, D), dtype=torch.bfloat16, device=device) for _ in range(slots)]
           for t, M in TOWERS}
     ws = torch.empty(fw.gated_mlp_static_fp8_group_workspace([M for _, M in GROUP_ORDER], D, I),
                      dtype=torch.uint8, device=device)
     comp = torch.cuda.Stream(device)
-    h2d = torch.cuda.Stream(device)
-    d2h = torch.cuda.Stream(device)
-    n = len(pairs)
+    h2d_s = [torch.cuda.Stream(device) for _ in range(copy_streams)]
+    d2h_s = [torch.cuda.Stream(device) for _ in range(copy_streams)]
+    done, copied_out = {}, {}  # per layer-pair issue index k: compute done, results copied out
+    counter = [0]
 
     def one_pass():
-        h2d.wait_stream(comp)
-        d2h.wait_stream(comp)
-        ready = [torch.cuda.Event() for _ in range(n)]
-        done = [torch.cuda.Event() for _ in range(n)]
-        copied_out = [torch.cuda.Event() for _ in range(n)]
         for i, pair in enumerate(pairs):
-            slot = i % 2
-            with torch.cuda.stream(h2d):
-                if i >= 2:
-                    h2d.wait_event(done[i - 2])  # slot's previous user finished compute
-                for L, hx in zip(pair, h_x[i]):
+            k = counter[0]
+            counter[0] += 1
+            slot = k % slots
+            prev = k - slots  # the previous user of this slot
+            prev_done = done.pop(prev, None)
+            ready = []
+            for t, (L, hx) in enumerate(zip(pair, h_x[i])):
+                st = h2d_s[t % copy_streams]
+                with torch.cuda.stream(st):
+                    if prev_done is not None:
+                        st.wait_event(prev_done)  # its compute has read the slot's X
                     dx[L.tower][slot].copy_(hx, non_blocking=True)
-                ready[i].record(h2d)
+                    ev = torch.cuda.Event()
+                    ev.record(st)
+                    ready.append(ev)
             with torch.cuda.stream(comp):
-                comp.wait_event(ready[i])
-                if i >= 2:
-                    comp.wait_event(copied_out[i - 2])  # slot's previous output copied out
+                for ev in ready:
+                    comp.wait_event(ev)
+                for ev in copied_out.pop(prev, ()):
+                    comp.wait_event(ev)  # its Y has left the slot
                 towers = [dict(x=dx[L.tower][slot], s_in=L.s_in, wg=L.wg, s_wg=L.s_wg, wu=L.wu,
                                s_wu=L.s_wu, s_down=L.s_down, wd=L.wd, s_wd=L.s_wd) for L in pair]
                 fw.gated_mlp_static_fp8_group(towers, workspace=ws,
                                               outs=[dy[L.tower][slot] for L in pair], stream=comp)
-                done[i].record(comp)
-            with torch.cuda.stream(d2h):
-                d2h.wait_event(done[i])
-                for L, hy in zip(pair, h_y[i]):
+                done[k] = torch.cuda.Event()
+                done[k].record(comp)
+            copied_out[k] = []
+            for t, (L, hy) in enumerate(zip(pair, h_y[i])):
+                st = d2h_s[t % copy_streams]
+                with torch.cuda.stream(st):
+                    st.wait_event(done[k])
                     hy.copy_(dy[L.tower][slot], non_blocking=True)
-                copied_out[i].record(d2h)
-        comp.wait_stream(d2h)
-        comp.wait_stream(h2d)
+                    ev = torch.cuda.Event()
+                    ev.record(st)
+                    copied_out[k].append(ev)
+
+    cur = torch.cuda.current_stream()
+    streams = [comp] + h2d_s + d2h_s
+
+    def join():
+        for st in streams:
+            cur.wait_stream(st)
 
     for _ in range(warmup):
         one_pass()
+    join()
     torch.cuda.synchronize()
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     dist_ctx.barrier()
     torch.cuda.synchronize()
-    comp.wait_stream(torch.cuda.current_stream())
-    start.record(comp)
+    start.record(cur)
+    for st in streams:
+        st.wait_stream(cur)
     for _ in range(steps):
         one_pass()
-    stop.record(comp)
+    join()
+    stop.record(cur)
     torch.cuda.synchronize()
     dist_ctx.barrier()
     ms = start.elapsed_time(stop)
@@ -619,12 +647,15 @@ def cpu_baseline(rows_per_tower: int = 1024):
 L2_FLUSH_BYTES = 256 * 1024 * 1024  # twice the 126 MB L2
 
 
-def kernel_bench(fw, kind, shape, steps, warmup, device):
+def kernel_bench(fw, kind, shape, steps, warmup, device, sustain_s=0.0):
     """One kernel on synthetic data shaped like the pages' workloads, timed
     launch by launch with CUDA events.  Between launches, outside the timed
     interval, L2 is flushed by reading a 256 MB buffer (a read leaves no dirty
-    lines to be written back inside the next timed launch).  Returns a dict for
-    one JSON line."""
+    lines to be written back inside the next timed launch).  With sustain_s >
+    0 the kernel also runs back to back for that many seconds (no flush), the
+    power-capped figure.  Kind "scaled_mm" is torch._scaled_mm (cuBLASLt FP8
+    with per-tensor scales, BF16 out): the library ceiling our FP8 GEMM is
+    compared with, not part of the path.  Returns a dict for one JSON line."""
     flush = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     pk = peaks()
     if kind in ("gemm", "gemm_ws"):
@@ -657,6 +688,18 @@ def kernel_bench(fw, kind, shape, steps, warmup, device):
         fn = lambda: fw.fp8_gate_up_swiglu_static(xq, wg, wu, s_in, s_wg, s_wu, s_down, out=h)  # noqa: E731
         work = 4.0 * M * N * K
         nbytes = M * K + 2 * N * K + M * N
+    elif kind == "scaled_mm":
+        M, N, K = shape
+        x = synth.student_t((M, K), 4, synth.seed(1, 92, 0), device)
+        w = synth.normal((N, K), synth.W_STD, synth.seed(1, 92, 10), device)
+        s_in = fw.fp8_observer_scale(fw.fp8_absmax_bf16(x))
+        xq = fw.fp8_quant_static(x, s_in)
+        wq, s_w = fw.fp8_rtn_quantize_weight(w)
+        del x, w
+        fn = lambda: torch._scaled_mm(xq, wq.t(), scale_a=s_in, scale_b=s_w,  # noqa: E731
+                                      out_dtype=torch.bfloat16)
+        work = 2.0 * M * N * K
+        nbytes = M * K + N * K + 2 * M * N
     elif kind in ("gemm_group", "gemm_group_ws"):
         M0, M1, N, K = shape
         probs = []
@@ -738,6 +781,24 @@ def kernel_bench(fw, kind, shape, steps, warmup, device):
         out["tflops"] = work / (ms / 1e3) / 1e12
         out["fp8_peak_frac"] = out["tflops"] / (2.0 * pk["bf16"])
         out["fp8_peak"] = f"{2.0 * pk['bf16']:.0f} TFLOP/s ({pk['source']} bf16 burst x 2)"
+    if sustain_s > 0:
+        fn()
+        torch.cuda.synchronize()
+        n, t0 = 0, time.perf_counter()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        while time.perf_counter() - t0 < sustain_s:
+            for _ in range(20):
+                fn()
+            n += 20
+            torch.cuda.synchronize()
+        b.record()
+        b.synchronize()
+        sus_ms = a.elapsed_time(b) / n
+        out["sustained_us"] = sus_ms * 1e3
+        out["sustained_launches"] = n
+        if work:
+            out["sustained_tflops"] = work / (sus_ms / 1e3) / 1e12
     st, where = fw.device_status()
     if st != 0:
         raise RuntimeError(f"device status {st} at wait site {where}")
@@ -754,6 +815,9 @@ SWEEPS = {
           [("gemm", (m, synth.C4["d"], synth.C4["I"])) for m in (1024, 4096)] +
           [("swiglu", (m, synth.C4["I"])) for m in (1024, 4096)] +
           [("quant", (m, synth.C4["d"])) for m in (1024, 4096)],
+    # our FP8 GEMM against cuBLASLt FP8 (torch._scaled_mm) at the same shapes
+    "fp8ceil": [(k, shp) for shp in ((8192, 8192, 8192), (4096, 12288, 3072), (4096, 3072, 12288))
+                for k in ("gemm", "scaled_mm")],
     # the grouped launches of the same layer (generation tower first)
     "c4g": [("dual_group", (4096, 1024, synth.C4["I"], synth.C4["d"])),
             ("gemm_group", (4096, 1024, synth.C4["d"], synth.C4["I"])),
@@ -824,7 +888,7 @@ def main():
     ap.add_argument("--unfused", action="store_true",
                     help="time the five-kernel composition (separate gate/up GEMMs and SwiGLU-quant)")
     ap.add_argument("--kernel", choices=("gemm", "gemm_ws", "dual", "swiglu", "quant", "gemm_group",
-                                         "gemm_group_ws", "dual_group", "quant_group"),
+                                         "gemm_group_ws", "dual_group", "quant_group", "scaled_mm"),
                     help="time one kernel on one shape instead of the pass")
     ap.add_argument("--shape", help="M,N,K for gemm; M,I,K for dual; M,I for swiglu; M,K for quant; "
                                     "M0,M1,N,K / M0,M1,I,K / M0,M1,K for the group kinds")
@@ -832,6 +896,9 @@ def main():
                     help="group: one grouped launch per step covers both towers of a layer; "
                          "towers: one launch per tower (see --streams)")
     ap.add_argument("--sweep", choices=tuple(SWEEPS), help="time every kernel shape of a workload")
+    ap.add_argument("--sustain", type=float, default=0.0,
+                    help="with --kernel/--sweep: also run each kernel back to back for this many "
+                         "seconds and report the power-capped rate")
     args = ap.parse_args()
     log = lambda m: print(m, file=sys.stderr, flush=True)  # noqa: E731
 
@@ -843,8 +910,8 @@ def main():
         jobs = ([(args.kernel, tuple(int(v) for v in args.shape.split(",")))] if args.kernel
                 else SWEEPS[args.sweep])
         for kind, shape in jobs:
-            print(json.dumps(kernel_bench(fw, kind, shape, args.steps, max(args.warmup, 3), device)),
-                  flush=True)
+            print(json.dumps(kernel_bench(fw, kind, shape, args.steps, max(args.warmup, 3), device,
+                                          args.sustain)), flush=True)
             torch.cuda.empty_cache()
         return 0
 
