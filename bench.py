@@ -375,6 +375,23 @@ def make_stream_runner(plan, device):
     return run
 
 
+def capture_graph(run):
+    """One step captured into a CUDA graph (after one eager step outside the
+    capture, which does the library's per-device set-up); returns the graph's
+    replay."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        run()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run()
+    torch.cuda.synchronize()
+    return g
+
+
 def time_device(plan, steps, warmup, dist_ctx, sampler=None, runner=None, instr_plan=None):
     """W untimed steps, then K timed steps between a barrier + synchronize on
     both sides, with CUDA events on the launching stream around the region
@@ -885,6 +902,9 @@ def main():
     ap.add_argument("--streams", type=int, choices=(1, 2), default=2,
                     help="towers mode: 2 runs the two towers of each layer on two streams, "
                          "joined per layer")
+    ap.add_argument("--eager", action="store_true",
+                    help="issue the grouped pass's calls eagerly instead of replaying one step "
+                         "captured as a CUDA graph")
     ap.add_argument("--unfused", action="store_true",
                     help="time the five-kernel composition (separate gate/up GEMMs and SwiGLU-quant)")
     ap.add_argument("--kernel", choices=("gemm", "gemm_ws", "dual", "swiglu", "quant", "gemm_group",
@@ -969,13 +989,27 @@ def main():
     launches_per_step = sum(3 if fused else 5 for _ in value_plan)
     sampler = ClockSampler(device.index if device.index is not None else 0)
     runner = make_stream_runner(value_plan, device) if (args.streams == 2 and not grouped) else None
+    graph = None
+    if grouped and not args.eager:
+        # the plan's calls name the stream they launch on: rebind them to the
+        # capture stream, which torch makes current inside the capture
+        def run_current():
+            h = torch.cuda.current_stream().cuda_stream
+            for _, fn, a, _, _ in value_plan:
+                if fn(*(a[:-1] + (h,))) != 0:
+                    raise RuntimeError("launch failed")
+        graph = capture_graph(run_current)
+        runner = graph.replay
     total_ms, per_kind, clocks, instrumented_ms = time_device(value_plan, args.steps,
                                                               max(args.warmup, 3), ctx, sampler,
                                                               runner, instr_plan=plan)
     launches = launches_per_step * args.steps
     counted = fw.launch_count() - launches_before
-    expect = launches_per_step * (args.steps + max(args.warmup, 3)) + \
-        sum(1 for _ in plan) * args.steps
+    if graph is not None:  # launches are counted when issued: the eager step and the capture
+        expect = 2 * launches_per_step + sum(1 for _ in plan) * args.steps
+    else:
+        expect = launches_per_step * (args.steps + max(args.warmup, 3)) + \
+            sum(1 for _ in plan) * args.steps
     if counted != expect:
         raise RuntimeError(f"launch count {counted} != expected {expect}")
     st, where = fw.device_status()
@@ -1061,7 +1095,8 @@ def main():
                        "path": ("fused: quantize X -> gate/up GEMM with SwiGLU-quant epilogue -> down GEMM"
                                 if fused else "unfused: quantize X -> gate GEMM -> up GEMM -> SwiGLU-quant -> down GEMM"),
                        "launch": ("grouped: one launch per step covers both towers of a layer"
-                                  if grouped else f"per tower, {args.streams} stream(s)"),
+                                  if grouped else f"per tower, {args.streams} stream(s)")
+                                 + ("; the step replayed as one CUDA graph" if graph else ""),
                        "layers": args.layers, "global_batch": TOKENS_PER_STEP * ctx.world,
                        "parallelism": f"replicas x{ctx.world}",
                        "l2": "inputs larger than L2 (8.15 GB of FP8 weights per pass)"},
@@ -1069,6 +1104,7 @@ def main():
             "gpu_launches": launches, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
+    del graph
     ctx.close()
     return 0
 
