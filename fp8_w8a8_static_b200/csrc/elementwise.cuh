@@ -141,40 +141,59 @@ __global__ void __launch_bounds__(kEwThreads)
 }
 
 // ------------------------------------------------------ SwiGLU -> FP8
-// SiLU(g) * u * (1/s) in fp32 with the fast exponential and divide.
-__device__ __forceinline__ float silu_mul(float g, float u) {
-  return __fdividef(g, 1.0f + __expf(-g)) * u;
+// SiLU(g) u (1/s) in fp32, with e^-g written as 2^(-g log2 e) (the ex2.approx
+// instruction) and the sigmoid as rcp.approx(1 + e^-g):
+//   e = 2^(g * -log2 e);  r = 1 / (1 + e);  h = ((g * u) * (1/s)) * r
+// every product and sum rounded to nearest.  The element-wise kernels and
+// the fused GEMM epilogue run exactly these operations, so their codes agree
+// bit for bit.
+constexpr float kNegLog2e = -1.44269504088896341f;
+
+// 1 / (1 + e^-x)
+__device__ __forceinline__ float sigmoid_f(float x) {
+  return rcp_approx(__fadd_rn(1.0f, ex2_approx(__fmul_rn(x, kNegLog2e))));
 }
 
-// SwiGLU variant: g' sigmoid(alpha g') (u' + beta), with the clamp g' <= limit,
-// |u'| <= limit when has_limit, and the offset only when beta != 0.  With
-// alpha = 1, beta = 0 and no limit this performs exactly silu_mul's
-// operations (alpha * g == g), so the results are bit-identical.
+// SiLU(g) * u * inv_s
+__device__ __forceinline__ float silu_mul_scaled(float g, float u, float inv_s) {
+  return __fmul_rn(__fmul_rn(__fmul_rn(g, u), inv_s), sigmoid_f(g));
+}
+
+// SiLU(g) * u, unscaled (calibration maxima and the per-row scales)
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  return __fmul_rn(__fmul_rn(g, u), sigmoid_f(g));
+}
+
+// SwiGLU variant: g' sigmoid(alpha g') (u' + beta) * inv_s, with the clamp
+// g' <= limit, |u'| <= limit when has_limit, and the offset only when beta !=
+// 0.  With alpha = 1, beta = 0 and no limit this performs exactly
+// silu_mul_scaled's operations (alpha * g == g), so the codes are identical.
 struct SwigluParams {
   float alpha, beta, limit;
   int has_limit;
 };
 
-__device__ __forceinline__ float swiglu_mul(float g, float u, const SwigluParams &p) {
+__device__ __forceinline__ float swiglu_mul_scaled(float g, float u, float inv_s,
+                                                   const SwigluParams &p) {
   if (p.has_limit) {
     g = fminf(g, p.limit);
     u = fminf(fmaxf(u, -p.limit), p.limit);
   }
-  const float up = p.beta != 0.0f ? u + p.beta : u;
-  return __fdividef(g, 1.0f + __expf(-(p.alpha * g))) * up;
+  const float up = p.beta != 0.0f ? __fadd_rn(u, p.beta) : u;
+  return __fmul_rn(__fmul_rn(__fmul_rn(g, up), inv_s), sigmoid_f(__fmul_rn(p.alpha, g)));
+}
+
+__device__ __forceinline__ uint32_t swiglu_quant2(uint32_t g, uint32_t u, float inv_s,
+                                                  const SwigluParams &p) {
+  return cvt_e4m3x2(swiglu_mul_scaled(bf16_lo(g), bf16_lo(u), inv_s, p),
+                    swiglu_mul_scaled(bf16_hi(g), bf16_hi(u), inv_s, p));
 }
 
 __device__ __forceinline__ uint2 swiglu_quant8(uint4 g, uint4 u, float inv_s,
                                                const SwigluParams &p) {
   uint2 o;
-  o.x = pack4(cvt_e4m3x2(swiglu_mul(bf16_lo(g.x), bf16_lo(u.x), p) * inv_s,
-                         swiglu_mul(bf16_hi(g.x), bf16_hi(u.x), p) * inv_s),
-              cvt_e4m3x2(swiglu_mul(bf16_lo(g.y), bf16_lo(u.y), p) * inv_s,
-                         swiglu_mul(bf16_hi(g.y), bf16_hi(u.y), p) * inv_s));
-  o.y = pack4(cvt_e4m3x2(swiglu_mul(bf16_lo(g.z), bf16_lo(u.z), p) * inv_s,
-                         swiglu_mul(bf16_hi(g.z), bf16_hi(u.z), p) * inv_s),
-              cvt_e4m3x2(swiglu_mul(bf16_lo(g.w), bf16_lo(u.w), p) * inv_s,
-                         swiglu_mul(bf16_hi(g.w), bf16_hi(u.w), p) * inv_s));
+  o.x = pack4(swiglu_quant2(g.x, u.x, inv_s, p), swiglu_quant2(g.y, u.y, inv_s, p));
+  o.y = pack4(swiglu_quant2(g.z, u.z, inv_s, p), swiglu_quant2(g.w, u.w, inv_s, p));
   return o;
 }
 
@@ -208,20 +227,21 @@ __global__ void __launch_bounds__(kEwThreads) swiglu_2in_kernel(
   if (t < numel) {
     float a = __uint_as_float(static_cast<uint32_t>(g[t]) << 16);
     float b = __uint_as_float(static_cast<uint32_t>(u[t]) << 16);
-    h[t] = static_cast<uint8_t>(cvt_e4m3x2(swiglu_mul(a, b, p) * inv_s, 0.0f) & 0xFFu);
+    h[t] = static_cast<uint8_t>(cvt_e4m3x2(swiglu_mul_scaled(a, b, inv_s, p), 0.0f) & 0xFFu);
   }
 }
 
+// one 32-bit word (two BF16 values) of G and of U -> two codes
+__device__ __forceinline__ uint32_t silu_quant2(uint32_t g, uint32_t u, float inv_s) {
+  return cvt_e4m3x2(silu_mul_scaled(bf16_lo(g), bf16_lo(u), inv_s),
+                    silu_mul_scaled(bf16_hi(g), bf16_hi(u), inv_s));
+}
+
 __device__ __forceinline__ uint2 silu_mul_quant8(uint4 g, uint4 u, float inv_s) {
+  const float is = inv_s;
   uint2 o;
-  o.x = pack4(cvt_e4m3x2(silu_mul(bf16_lo(g.x), bf16_lo(u.x)) * inv_s,
-                         silu_mul(bf16_hi(g.x), bf16_hi(u.x)) * inv_s),
-              cvt_e4m3x2(silu_mul(bf16_lo(g.y), bf16_lo(u.y)) * inv_s,
-                         silu_mul(bf16_hi(g.y), bf16_hi(u.y)) * inv_s));
-  o.y = pack4(cvt_e4m3x2(silu_mul(bf16_lo(g.z), bf16_lo(u.z)) * inv_s,
-                         silu_mul(bf16_hi(g.z), bf16_hi(u.z)) * inv_s),
-              cvt_e4m3x2(silu_mul(bf16_lo(g.w), bf16_lo(u.w)) * inv_s,
-                         silu_mul(bf16_hi(g.w), bf16_hi(u.w)) * inv_s));
+  o.x = pack4(silu_quant2(g.x, u.x, is), silu_quant2(g.y, u.y, is));
+  o.y = pack4(silu_quant2(g.z, u.z, is), silu_quant2(g.w, u.w, is));
   return o;
 }
 
@@ -253,7 +273,7 @@ __global__ void __launch_bounds__(kEwThreads) silu_mul_2in_kernel(
   if (t < numel) {
     float a = __uint_as_float(static_cast<uint32_t>(g[t]) << 16);
     float b = __uint_as_float(static_cast<uint32_t>(u[t]) << 16);
-    h[t] = static_cast<uint8_t>(cvt_e4m3x2(silu_mul(a, b) * inv_s, 0.0f) & 0xFFu);
+    h[t] = static_cast<uint8_t>(cvt_e4m3x2(silu_mul_scaled(a, b, inv_s), 0.0f) & 0xFFu);
   }
 }
 

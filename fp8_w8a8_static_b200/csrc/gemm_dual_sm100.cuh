@@ -273,7 +273,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int e = 0; e < 4; ++e) {
             const float gv = __bfloat162float(__float2bfloat16_rn(__uint_as_float(g[4 * j + e]) * sg));
             const float uv = __bfloat162float(__float2bfloat16_rn(__uint_as_float(u[4 * j + e]) * su));
-            h[e] = (VARIANT ? swiglu_mul(gv, uv, act) : silu_mul(gv, uv)) * is;
+            h[e] = VARIANT ? swiglu_mul_scaled(gv, uv, is, act) : silu_mul_scaled(gv, uv, is);
           }
           q[j] = pack4(cvt_e4m3x2(h[0], h[1]), cvt_e4m3x2(h[2], h[3]));
         }
