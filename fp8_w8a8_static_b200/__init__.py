@@ -37,6 +37,7 @@ __all__ = [
     "fp8_check_shared_input_scale", "fp8_absmax_bf16", "fp8_silu_mul_absmax",
     "fp8_observer_scale", "fp8_rtn_quantize_weight",
     "device_check", "device_status", "launch_count", "launch_log", "launch_log_clear",
+    "selftest_bounded_wait", "SITE_SELFTEST",
     "FP8", "OBSERVER_CONSTANT", "EXPORTED_SYMBOLS",
 ]
 
@@ -56,6 +57,7 @@ OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_SCALE_MISMATCH, ERR_BAD_SCALE, ERR_CUDA,
     ERR_DEVICE_TIMEOUT, ERR_UNSUPPORTED, ERR_WORKSPACE = range(10)
 
 KIND_QUANT, KIND_GEMM, KIND_SWIGLU, KIND_CALIB, KIND_DUAL = 1, 2, 3, 4, 5
+SITE_SELFTEST = 6  # wait site recorded by the bounded-wait self-test
 
 
 class FP8WSError(RuntimeError):
@@ -163,6 +165,8 @@ _SIGS = {
     "fp8ws_device_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int),
                                            ctypes.POINTER(ctypes.c_int)]),
     "fp8ws_set_gemm_config": (ctypes.c_int, [ctypes.c_int]),
+    "fp8ws_selftest_bounded_wait": (ctypes.c_int, [_I64, ctypes.c_int,
+                                                   ctypes.POINTER(ctypes.c_int64), _P]),
     "fp8ws_launch_count": (ctypes.c_int64, []),
     "fp8ws_launch_log": (ctypes.c_int, [ctypes.POINTER(LaunchRecord), ctypes.c_int]),
     "fp8ws_launch_log_clear": (None, []),
@@ -804,6 +808,16 @@ def device_status():
 
 
 GEMM_CONFIGS = {"auto": 0, "pair256": 1, "cta256": 2, "cta128": 3, "cta64": 4}
+
+
+def selftest_bounded_wait(limit_ns: int, mode: int = 0, stream=None) -> int:
+    """Run the bounded-wait self-test kernel (mode 0: the wait runs out and
+    records site 6; mode 1: the abort flag ends it early).  Returns the wait's
+    duration in ns, measured on the device."""
+    out = ctypes.c_int64(0)
+    _check(load().fp8ws_selftest_bounded_wait(limit_ns, mode, ctypes.byref(out), _stream(stream)),
+           "fp8ws_selftest_bounded_wait")
+    return out.value
 
 
 def set_gemm_config(name: str = "auto") -> None:

@@ -23,6 +23,7 @@ enum WaitSite : int {
   kSiteMmaTmemEmpty = 3,
   kSiteEpiTmemFull = 4,
   kSiteDrain = 5,
+  kSiteSelfTest = 6,  // fp8ws_selftest_bounded_wait
 };
 
 __device__ __forceinline__ void record_timeout(int site) {

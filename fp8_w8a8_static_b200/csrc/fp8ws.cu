@@ -580,6 +580,38 @@ int silu_launch(DeviceInfo *d, const uint16_t *g, const uint16_t *u, int64_t num
 
 size_t round256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
+// Self-test of the bounded wait (fp8ws_selftest_bounded_wait): lane 0 of warp 0
+// waits on an mbarrier that nothing arrives at.  Mode 0: the wait runs out
+// after limit_ns and records kSiteSelfTest in the status word.  Mode 1: warp 1
+// raises the abort flag after a quarter of the limit and the wait returns
+// then, recording nothing.  Either way the kernel returns; the time the wait
+// took goes to g_selftest_elapsed_ns.
+__device__ long long g_selftest_elapsed_ns = 0;
+
+__global__ void selftest_wait_kernel(uint64_t limit_ns, int mode) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ volatile int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint64_t t0 = global_timer_ns();
+    const bool ok = mbar_wait_bounded(&bar, 0, &abort_flag, limit_ns);
+    const uint64_t t1 = global_timer_ns();
+    if (!ok && mode == 0) record_timeout(kSiteSelfTest);
+    g_selftest_elapsed_ns = static_cast<long long>(t1 - t0);
+    mbar_arrive(&bar);  // complete the phase before the block exits
+  } else if (threadIdx.x == 32 && mode == 1) {
+    const uint64_t t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < limit_ns / 4) {
+    }
+    abort_flag = 1;
+  }
+}
+
 // NULL = plain SwiGLU (alpha 1, no offset, no clamp).
 int swiglu_params(const fp8ws_swiglu *act, SwigluParams *p) {
   p->alpha = 1.0f;
@@ -1257,6 +1289,24 @@ const char *fp8ws_status_string(int status) {
     case FP8WS_ERR_WORKSPACE: return "workspace NULL or not 256-byte aligned";
     default: return "unknown status";
   }
+}
+
+int fp8ws_selftest_bounded_wait(int64_t limit_ns, int mode, int64_t *elapsed_ns, void *stream) {
+  if (!elapsed_ns) return FP8WS_ERR_NULL;
+  if (limit_ns <= 0 || limit_ns > static_cast<int64_t>(kWaitLimitNs) || (mode != 0 && mode != 1))
+    return FP8WS_ERR_SHAPE;
+  DeviceInfo *d;
+  int rc = device_info(&d);
+  if (rc) return rc;
+  cudaStream_t st = as_stream(stream);
+  selftest_wait_kernel<<<1, 64, 0, st>>>(static_cast<uint64_t>(limit_ns), mode);
+  if (cudaGetLastError() != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess)
+    return FP8WS_ERR_CUDA;
+  long long v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_selftest_elapsed_ns, sizeof(v)) != cudaSuccess)
+    return FP8WS_ERR_CUDA;
+  *elapsed_ns = v;
+  return FP8WS_OK;
 }
 
 int fp8ws_device_check(void) {

@@ -529,6 +529,17 @@ FP8WS_API int fp8ws_device_check(void);
  * *where receives a code naming the wait that ran out (0 if none). */
 FP8WS_API int fp8ws_device_status(int *status, int *where);
 
+/* Self-test of the bounded waits every GEMM kernel uses (failure detection
+ * without a GPU fault): one small kernel waits on an mbarrier that nothing
+ * arrives at.  mode 0: the wait runs out after limit_ns, the kernel records
+ * wait site 6 in the device status word (read it with fp8ws_device_status)
+ * and returns.  mode 1: a second warp raises the kernel's abort flag after
+ * limit_ns / 4; the wait returns then and records nothing.  Synchronizes
+ * `stream`; *elapsed_ns (host) receives how long the wait took, measured on
+ * the device.  limit_ns: 1 .. 4e9 (FP8WS_ERR_SHAPE otherwise). */
+FP8WS_API int fp8ws_selftest_bounded_wait(int64_t limit_ns, int mode, int64_t *elapsed_ns,
+                                          void *stream);
+
 /* Tile configuration of fp8_linear_static and of the down projection of the
  * gated MLPs, for tuning and tests: 0 = chosen per shape by the cost model
  * (default), 1 = CTA-pair 256x256 tiles, 2/3/4 = one CTA with 128x256,

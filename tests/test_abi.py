@@ -187,3 +187,12 @@ def test_group_argument_checks_before_cuda(lib):
     assert lib.fp8_gate_up_swiglu_static_group(ctypes.byref(eg), 1, 256, 512, None,
                                                None) == fw.OK
     assert fw.launch_count() == n0
+
+
+def test_selftest_argument_checks(lib):
+    import ctypes
+    out = ctypes.c_int64(0)
+    assert lib.fp8ws_selftest_bounded_wait(1000, 0, None, None) == fw.ERR_NULL
+    assert lib.fp8ws_selftest_bounded_wait(0, 0, ctypes.byref(out), None) == fw.ERR_SHAPE
+    assert lib.fp8ws_selftest_bounded_wait(5_000_000_000, 0, ctypes.byref(out), None) == fw.ERR_SHAPE
+    assert lib.fp8ws_selftest_bounded_wait(1000, 2, ctypes.byref(out), None) == fw.ERR_SHAPE
