@@ -569,3 +569,25 @@ def test_silu_mul_rows_uses_each_rows_maximum():
         assert np.array_equal(h[r], oracle.silu_mul_2in(np.ascontiguousarray(g[r]),
                                                         np.ascontiguousarray(u[r]), float(s[r])))
         assert (h[r] & 0x7F).max() == 0x7E
+
+
+def test_gated_mlp_per_token_rows_and_weight_channels():
+    """Per-token scales make every output row depend on its own input row only
+    (a row keeps its result when computed alone or beside other rows), and a
+    weight channel's scale multiplies that channel's output exactly: doubling
+    the down projection's scale of one output channel doubles that column and
+    leaves the others."""
+    d = synth.c0_mlp()
+    wg, swg = oracle.quantize_rows(bits_of(d["wg"]))
+    wu, swu = oracle.quantize_rows(bits_of(d["wu"]))
+    wd, swd = oracle.quantize_rows(bits_of(d["wd"]))
+    x = bits_of(d["x"])
+    y = oracle.gated_mlp_per_token(x, wg, swg, wu, swu, wd, swd)
+    rows = [2, 9, 40]
+    y_rows = oracle.gated_mlp_per_token(np.ascontiguousarray(x[rows]), wg, swg, wu, swu, wd, swd)
+    assert np.array_equal(y[rows], y_rows)
+    swd2 = swd.copy()
+    swd2[7] *= 2
+    y2 = oracle.gated_mlp_per_token(x, wg, swg, wu, swu, wd, swd2)
+    assert np.array_equal(oracle.bf16_to_f64(y2[:, 7]), 2 * oracle.bf16_to_f64(y[:, 7]))
+    assert np.array_equal(np.delete(y2, 7, axis=1), np.delete(y, 7, axis=1))
