@@ -705,6 +705,33 @@ def kernel_bench(fw, kind, shape, steps, warmup, device, sustain_s=0.0):
         fn = lambda: fw.fp8_gate_up_swiglu_static(xq, wg, wu, s_in, s_wg, s_wu, s_down, out=h)  # noqa: E731
         work = 4.0 * M * N * K
         nbytes = M * K + 2 * N * K + M * N
+    elif kind == "mlp":
+        M, dm, Ii = shape
+        x = synth.activation_with_outliers(M, dm, 0, 0, 0, device)
+        s_in = fw.fp8_observer_scale(fw.fp8_absmax_bf16(x))
+        wts = [fw.fp8_rtn_quantize_weight(synth.normal(shp, synth.W_STD, synth.seed(0, 90, k), device))
+               for k, shp in enumerate(((Ii, dm), (Ii, dm), (dm, Ii)))]
+        s_down = torch.tensor([0.003], dtype=torch.float32, device=device)
+        wsb = torch.empty(fw.gated_mlp_static_fp8_fused_workspace(M, dm, Ii), dtype=torch.uint8,
+                          device=device)
+        y = torch.empty((M, dm), dtype=torch.bfloat16, device=device)
+        fn = lambda: fw.gated_mlp_static_fp8_fused(x, s_in, *wts[0], *wts[1], s_down, *wts[2],  # noqa: E731
+                                                   workspace=wsb, out=y)
+        work = 6.0 * M * dm * Ii
+        nbytes = 2 * M * dm + 3 * dm * Ii + 2 * M * dm
+    elif kind == "qkv":
+        M, dm, Nq, Nkv = shape
+        x = synth.activation_with_outliers(M, dm, 3, 90, 0, device, heavy_tailed_outliers=True)
+        s_in = fw.fp8_observer_scale(fw.fp8_absmax_bf16(x))
+        wts = [fw.fp8_rtn_quantize_weight(synth.normal((n, dm), synth.W_STD, synth.seed(3, 90, k),
+                                                       device))
+               for k, n in enumerate((Nq, Nkv, Nkv))]
+        wsb = torch.empty(fw.qkv_shared_quant_workspace(M, dm), dtype=torch.uint8, device=device)
+        outs = tuple(torch.empty((M, n), dtype=torch.bfloat16, device=device) for n in (Nq, Nkv, Nkv))
+        fn = lambda: fw.qkv_shared_quant(x, s_in, *wts[0], *wts[1], *wts[2], workspace=wsb,  # noqa: E731
+                                         out=outs)
+        work = 2.0 * M * dm * (Nq + 2 * Nkv)
+        nbytes = 2 * M * dm + dm * (Nq + 2 * Nkv) + 2 * M * (Nq + 2 * Nkv)
     elif kind == "scaled_mm":
         M, N, K = shape
         x = synth.student_t((M, K), 4, synth.seed(1, 92, 0), device)
@@ -825,13 +852,15 @@ def kernel_bench(fw, kind, shape, steps, warmup, device, sustain_s=0.0):
 SWEEPS = {
     "c1": [("gemm", (m, n, synth.C1_K)) for m in synth.C1_M for n in synth.C1_N],
     "c2": [("swiglu", (m, i)) for m in synth.C2_M for i in synth.C2_I],
-    "c3": [("quant", (synth.C3["M"], synth.C3["d"]))] +
+    "c3": [("qkv", (synth.C3["M"], synth.C3["d"], synth.C3["Nq"], synth.C3["Nk"])),
+           ("quant", (synth.C3["M"], synth.C3["d"]))] +
           [("gemm", (synth.C3["M"], n, synth.C3["d"])) for n in (synth.C3["Nq"], synth.C3["Nk"], synth.C3["Nv"])],
     "c4": [("dual", (m, synth.C4["I"], synth.C4["d"])) for m in (1024, 4096)] +
           [("gemm", (m, synth.C4["I"], synth.C4["d"])) for m in (1024, 4096)] +
           [("gemm", (m, synth.C4["d"], synth.C4["I"])) for m in (1024, 4096)] +
           [("swiglu", (m, synth.C4["I"])) for m in (1024, 4096)] +
           [("quant", (m, synth.C4["d"])) for m in (1024, 4096)],
+    "c0": [("mlp", (synth.C0["M"], synth.C0["d"], synth.C0["I"]))],
     # our FP8 GEMM against cuBLASLt FP8 (torch._scaled_mm) at the same shapes
     "fp8ceil": [(k, shp) for shp in ((8192, 8192, 8192), (4096, 12288, 3072), (4096, 3072, 12288))
                 for k in ("gemm", "scaled_mm")],
@@ -908,10 +937,13 @@ def main():
     ap.add_argument("--unfused", action="store_true",
                     help="time the five-kernel composition (separate gate/up GEMMs and SwiGLU-quant)")
     ap.add_argument("--kernel", choices=("gemm", "gemm_ws", "dual", "swiglu", "quant", "gemm_group",
-                                         "gemm_group_ws", "dual_group", "quant_group", "scaled_mm"),
+                                         "gemm_group_ws", "dual_group", "quant_group", "scaled_mm",
+                                         "mlp", "qkv"),
                     help="time one kernel on one shape instead of the pass")
     ap.add_argument("--shape", help="M,N,K for gemm; M,I,K for dual; M,I for swiglu; M,K for quant; "
-                                    "M0,M1,N,K / M0,M1,I,K / M0,M1,K for the group kinds")
+                                    "M0,M1,N,K / M0,M1,I,K / M0,M1,K for the group kinds; "
+                                    "M,d,I for mlp (the fused gated MLP, three launches); "
+                                    "M,d,Nq,Nkv for qkv (shared quantize + grouped Q/K/V GEMM)")
     ap.add_argument("--mode", choices=("group", "towers"), default="group",
                     help="group: one grouped launch per step covers both towers of a layer; "
                          "towers: one launch per tower (see --streams)")

@@ -82,7 +82,7 @@ def _act(act):
 
 
 class LaunchRecord(ctypes.Structure):
-    _fields_ = [("kind", ctypes.c_int32), ("pad", ctypes.c_int32), ("in0", ctypes.c_void_p),
+    _fields_ = [("kind", ctypes.c_int32), ("member", ctypes.c_int32), ("in0", ctypes.c_void_p),
                 ("in1", ctypes.c_void_p), ("out", ctypes.c_void_p)]
 
 
@@ -830,9 +830,11 @@ def launch_count() -> int:
 
 
 def launch_log(max_records: int = 64):
+    """The most recent launch records as (kind, in0, in1, out, member) tuples;
+    a grouped launch has one record per problem (member 0, 1, ...)."""
     buf = (LaunchRecord * max_records)()
     n = load().fp8ws_launch_log(buf, max_records)
-    return [(r.kind, r.in0 or 0, r.in1 or 0, r.out or 0) for r in buf[:n]]
+    return [(r.kind, r.in0 or 0, r.in1 or 0, r.out or 0, r.member) for r in buf[:n]]
 
 
 def launch_log_clear() -> None:

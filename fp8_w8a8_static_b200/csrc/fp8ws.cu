@@ -34,16 +34,18 @@ fp8ws_launch_record g_log[FP8WS_LOG_CAPACITY];
 int64_t g_log_head = 0;  // records written since the last clear
 int64_t g_launch_total = 0;
 
-void log_launch(int kind, const void *in0, const void *in1, const void *out) {
+// One record per problem of a launch (member 0, 1, ... of a grouped launch);
+// the launch itself is counted once, with member 0.
+void log_launch(int kind, const void *in0, const void *in1, const void *out, int member = 0) {
   std::lock_guard<std::mutex> lk(g_log_mu);
   fp8ws_launch_record &r = g_log[g_log_head % FP8WS_LOG_CAPACITY];
   r.kind = kind;
-  r.pad = 0;
+  r.member = member;
   r.in0 = in0;
   r.in1 = in1;
   r.out = out;
   ++g_log_head;
-  ++g_launch_total;
+  if (member == 0) ++g_launch_total;
 }
 
 enum { kKindQuant = 1, kKindGemm = 2, kKindSwiglu = 3, kKindCalib = 4, kKindDual = 5 };
@@ -271,15 +273,17 @@ SplitPlan make_split_plan(int tiles, int pairs, int num_kb, float *partials, int
   return p;
 }
 
-// One problem of a grouped CTA-pair launch.  b2 and s_w2 (the up weight) and
-// s_down are read by the dual gate/up kernel only; out is Y (BF16) for the
-// GEMM and H (FP8) for the dual kernel.  Every problem has M >= 1.
+// One problem of a grouped CTA-pair launch: Y[M,N] from A[M,K] and B[N,K].
+// b2 and s_w2 (the up weight) and s_down are read by the dual gate/up kernel
+// only; out is Y (BF16) for the GEMM and H (FP8) for the dual kernel.  Every
+// problem has M >= 1.
 struct PairProblem {
   const uint8_t *a;
   const uint8_t *b;
   const uint8_t *b2;
   void *out;
   int M;
+  int N;
   const float *s_in;
   const float *s_w;
   const float *s_w2;
@@ -287,25 +291,25 @@ struct PairProblem {
 };
 
 // Kernel-side description of a group whose tiles are tile_m x tile_n.
-PairGroup make_pair_group(const PairProblem *pp, int np, int N, int tile_m, int tile_n,
-                          int *tiles) {
+PairGroup make_pair_group(const PairProblem *pp, int np, int tile_m, int tile_n) {
   PairGroup G = {};
   G.n = np;
-  const int num_n = (N + tile_n - 1) / tile_n;
   int total = 0;
   for (int p = 0; p < kMaxGroup; ++p) {
     const PairProblem &q = pp[p < np ? p : 0];
     G.M[p] = q.M;
+    G.N[p] = q.N;
     G.num_m[p] = (q.M + tile_m - 1) / tile_m;
+    G.num_n[p] = (q.N + tile_n - 1) / tile_n;
     G.s_in[p] = q.s_in;
     G.s_w[p] = q.s_w;
     G.s_w2[p] = q.s_w2;
     G.s_down[p] = q.s_down;
     G.out[p] = q.out;
-    if (p == 1) G.tile_start1 = total;
-    if (p < np) total += G.num_m[p] * num_n;
+    G.tile_start[p] = p < np ? total : INT_MAX;
+    if (p < np) total += G.num_m[p] * G.num_n[p];
   }
-  *tiles = total;
+  G.tiles = total;
   return G;
 }
 
@@ -338,8 +342,8 @@ int pair_clusters(DeviceInfo *d, Kernel kern, int smem, int bit, int *clusters_o
 }
 
 template <int STAGES, int BIT, int SCALE_MODE = 0, bool DIRECT = false>
-int launch_gemm_pair_cfg(DeviceInfo *d, const PairProblem *pp, int np, int N, int K,
-                         cudaStream_t st, void *splitk = nullptr) {
+int launch_gemm_pair_cfg(DeviceInfo *d, const PairProblem *pp, int np, int K, cudaStream_t st,
+                         void *splitk = nullptr) {
   using C = PairCfg<STAGES, DIRECT>;
   auto kern = fp8_gemm_pair_kernel<STAGES, SCALE_MODE, DIRECT>;
   int rc = pair_clusters(d, kern, C::SMEM_BYTES, BIT, &d->pair_clusters);
@@ -348,19 +352,20 @@ int launch_gemm_pair_cfg(DeviceInfo *d, const PairProblem *pp, int np, int N, in
   for (int p = 0; p < np && !rc; ++p) {
     const PairProblem &q = pp[p];
     rc = make_map_2d(&ma[p], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.a, q.M, K, kGemmBK, 128, true);
-    if (!rc) rc = make_map_2d(&mb[p], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.b, N, K, kGemmBK, 128, true);
     if (!rc)
-      rc = make_map_2d(&md[p], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q.out, q.M, N, C::EPI_COLS, 32,
-                       false);
+      rc = make_map_2d(&mb[p], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.b, q.N, K, kGemmBK, 128, true);
+    if (!rc)
+      rc = make_map_2d(&md[p], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q.out, q.M, q.N, C::EPI_COLS,
+                       32, false);
   }
   if (rc) return rc;
-  if (np == 1) {
-    ma[1] = ma[0];
-    mb[1] = mb[0];
-    md[1] = md[0];
+  for (int p = np; p < kMaxGroup; ++p) {  // absent problems: copies, never used
+    ma[p] = ma[0];
+    mb[p] = mb[0];
+    md[p] = md[0];
   }
-  int tiles = 0;
-  const PairGroup G = make_pair_group(pp, np, N, kPairTile, kPairTile, &tiles);
+  const PairGroup G = make_pair_group(pp, np, kPairTile, kPairTile);
+  const int tiles = G.tiles;
   float *partials = static_cast<float *>(splitk);
   int *counters = splitk ? splitk_counters(splitk) : nullptr;
   const SplitPlan plan =
@@ -368,9 +373,10 @@ int launch_gemm_pair_cfg(DeviceInfo *d, const PairProblem *pp, int np, int N, in
   const int units = plan.dp_tiles + plan.split_tiles * plan.splits;
   const int clusters = units < d->pair_clusters ? units : d->pair_clusters;
   if (launch_ex(kern, dim3(2 * clusters), dim3(kGemmThreads), C::SMEM_BYTES, st, 2, ma[0], ma[1],
-                mb[0], mb[1], md[0], md[1], G, N, K, kWaitLimitNs, plan) != cudaSuccess)
+                ma[2], mb[0], mb[1], mb[2], md[0], md[1], md[2], G, K, kWaitLimitNs,
+                plan) != cudaSuccess)
     return FP8WS_ERR_CUDA;
-  log_launch(kKindGemm, pp[0].a, pp[0].b, pp[0].out);
+  for (int p = 0; p < np; ++p) log_launch(kKindGemm, pp[p].a, pp[p].b, pp[p].out, p);
   return launch_status();
 }
 
@@ -387,19 +393,19 @@ bool direct_epilogue() {
 }
 
 template <int BIT, int SCALE_MODE = 0>
-int launch_gemm_pair(DeviceInfo *d, const PairProblem *pp, int np, int N, int K, cudaStream_t st,
+int launch_gemm_pair(DeviceInfo *d, const PairProblem *pp, int np, int K, cudaStream_t st,
                      void *splitk = nullptr) {
   if (direct_epilogue())
-    return launch_gemm_pair_cfg<7, BIT + 16, SCALE_MODE, true>(d, pp, np, N, K, st, splitk);
-  return launch_gemm_pair_cfg<6, BIT, SCALE_MODE, false>(d, pp, np, N, K, st, splitk);
+    return launch_gemm_pair_cfg<7, BIT + 16, SCALE_MODE, true>(d, pp, np, K, st, splitk);
+  return launch_gemm_pair_cfg<6, BIT, SCALE_MODE, false>(d, pp, np, K, st, splitk);
 }
 
 template <int BIT, int SCALE_MODE = 0>
 int launch_gemm_pair(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int M, int N, int K,
                      const float *s_in, const float *s_w, uint16_t *y, cudaStream_t st,
                      void *splitk = nullptr) {
-  const PairProblem p = {xq, wq, nullptr, y, M, s_in, s_w, nullptr, nullptr};
-  return launch_gemm_pair<BIT, SCALE_MODE>(d, &p, 1, N, K, st, splitk);
+  const PairProblem p = {xq, wq, nullptr, y, M, N, s_in, s_w, nullptr, nullptr};
+  return launch_gemm_pair<BIT, SCALE_MODE>(d, &p, 1, K, st, splitk);
 }
 
 // Gate/up dual GEMM with the SwiGLU-quant epilogue, on CTA pairs.
@@ -410,7 +416,7 @@ int launch_dual_swiglu_cfg(DeviceInfo *d, const PairProblem *pp, int np, int N, 
   auto kern = fp8_dual_swiglu_pair_kernel<STAGES, DIRECT, VARIANT>;
   int rc = pair_clusters(d, kern, C::SMEM_BYTES, BIT, &d->dual_clusters);
   if (rc) return rc;
-  CUtensorMap ma[kMaxGroup], mg[kMaxGroup], mu[kMaxGroup], mh[kMaxGroup];
+  CUtensorMap ma[kMaxDualGroup], mg[kMaxDualGroup], mu[kMaxDualGroup], mh[kMaxDualGroup];
   for (int p = 0; p < np && !rc; ++p) {
     const PairProblem &q = pp[p];
     rc = make_map_2d(&ma[p], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.a, q.M, K, kGemmBK, 128, true);
@@ -426,14 +432,14 @@ int launch_dual_swiglu_cfg(DeviceInfo *d, const PairProblem *pp, int np, int N, 
     mu[1] = mu[0];
     mh[1] = mh[0];
   }
-  int tiles = 0;
-  const PairGroup G = make_pair_group(pp, np, N, kDualTileM, kDualTileN, &tiles);
+  const PairGroup G = make_pair_group(pp, np, kDualTileM, kDualTileN);
+  const int tiles = G.tiles;
   const int clusters = tiles < d->dual_clusters ? tiles : d->dual_clusters;
   if (launch_ex(kern, dim3(2 * clusters), dim3(kGemmThreads), C::SMEM_BYTES, st, 2, ma[0], mg[0],
                 mu[0], mh[0], ma[1], mg[1], mu[1], mh[1], G, act, N, K,
                 kWaitLimitNs) != cudaSuccess)
     return FP8WS_ERR_CUDA;
-  log_launch(kKindDual, pp[0].a, pp[0].b, pp[0].out);
+  for (int p = 0; p < np; ++p) log_launch(kKindDual, pp[p].a, pp[p].b, pp[p].out, p);
   return launch_status();
 }
 
@@ -455,7 +461,7 @@ int launch_dual_swiglu(DeviceInfo *d, const uint8_t *xq, const uint8_t *wg, cons
                        int M, int N, int K, const float *s_in, const float *s_wg,
                        const float *s_wu, const float *s_down, SwigluParams act, uint8_t *h,
                        cudaStream_t st) {
-  const PairProblem p = {xq, wg, wu, h, M, s_in, s_wg, s_wu, s_down};
+  const PairProblem p = {xq, wg, wu, h, M, N, s_in, s_wg, s_wu, s_down};
   return launch_dual_swiglu(d, &p, 1, N, K, act, st);
 }
 
@@ -477,20 +483,23 @@ int check_gemm_args(const void *xq, const void *wq, int64_t M, int64_t N, int64_
 int g_forced_gemm_config = 0;  // fp8ws_set_gemm_config: 0 = cost model
 
 // 1 = CTA pair 256 x 256, 2 = one CTA 128 x 256, 3 = 128 x 128, 4 = 128 x 64,
-// for the np problems of rows M[p] sharing N that one launch would cover.
-int gemm_choice(const DeviceInfo *d, const int64_t *M, int np, int64_t N) {
+// for the np problems M[p] x N[p] that one launch would cover.
+int gemm_choice(const DeviceInfo *d, const int64_t *M, const int64_t *N, int np) {
   if (g_forced_gemm_config) return g_forced_gemm_config;
   const int pairs = d->pair_clusters > 0 ? d->pair_clusters : d->sms / 2;
   auto waves = [](int64_t tiles, int64_t slots) { return (tiles + slots - 1) / slots; };
-  int64_t m128 = 0, m256 = 0;
+  int64_t t_pair = 0, t_256 = 0, t_128 = 0, t_64 = 0;
   for (int p = 0; p < np; ++p) {
-    m128 += (M[p] + 127) / 128;
-    m256 += (M[p] + 255) / 256;
+    const int64_t m128 = (M[p] + 127) / 128, m256 = (M[p] + 255) / 256;
+    t_pair += m256 * ((N[p] + 255) / 256);
+    t_256 += m128 * ((N[p] + 255) / 256);
+    t_128 += m128 * ((N[p] + 127) / 128);
+    t_64 += m128 * ((N[p] + 63) / 64);
   }
-  const double est_pair = waves(m256 * ((N + 255) / 256), pairs) * (128.0 * 256) / 1.0;
-  const double est_256 = waves(m128 * ((N + 255) / 256), d->sms) * (128.0 * 256) / 0.85;
-  const double est_128 = waves(m128 * ((N + 127) / 128), d->sms) * (128.0 * 128) / 0.45;
-  const double est_64 = waves(m128 * ((N + 63) / 64), d->sms) * (128.0 * 64) / 0.25;
+  const double est_pair = waves(t_pair, pairs) * (128.0 * 256) / 1.0;
+  const double est_256 = waves(t_256, d->sms) * (128.0 * 256) / 0.85;
+  const double est_128 = waves(t_128, d->sms) * (128.0 * 128) / 0.45;
+  const double est_64 = waves(t_64, d->sms) * (128.0 * 64) / 0.25;
   const double best = fmin(fmin(est_pair, est_256), fmin(est_128, est_64));
   if (est_pair == best) return 1;
   if (est_256 == best) return 2;
@@ -503,7 +512,7 @@ int gemm_dispatch(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int64_t M
                   void *splitk = nullptr) {
   if (M == 0) return FP8WS_OK;
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
-  switch (gemm_choice(d, &M, 1, N)) {
+  switch (gemm_choice(d, &M, &N, 1)) {
     case 1: return launch_gemm_pair<3>(d, xq, wq, m, n, k, s_in, s_w, y, st, splitk);
     case 2: return launch_gemm_cfg<256, 4, 0>(d, xq, wq, m, n, k, s_in, s_w, y, st);
     case 3: return launch_gemm_cfg<128, 6, 1>(d, xq, wq, m, n, k, s_in, s_w, y, st);
@@ -511,25 +520,35 @@ int gemm_dispatch(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int64_t M
   }
 }
 
-// A group of GEMMs sharing N and K: one CTA-pair launch over all their tiles
-// when the cost model picks CTA pairs for the group, else one launch each.
-// Problems with M == 0 are skipped.
-int gemm_group_dispatch(DeviceInfo *d, const PairProblem *pp, int np, int N, int K,
-                        cudaStream_t st, void *splitk = nullptr) {
+// A group of up to kMaxGroup GEMMs sharing K: one CTA-pair launch over all
+// their tiles when the cost model picks CTA pairs for the group, else one
+// launch each.  Problems with M == 0 are skipped.
+int gemm_group_dispatch(DeviceInfo *d, const PairProblem *pp, int np, int K, cudaStream_t st,
+                        void *splitk = nullptr) {
   PairProblem live[kMaxGroup];
-  int64_t rows[kMaxGroup];
+  int64_t rows[kMaxGroup], cols[kMaxGroup];
   int n = 0;
   for (int p = 0; p < np; ++p)
     if (pp[p].M > 0) {
       live[n] = pp[p];
-      rows[n++] = pp[p].M;
+      rows[n] = pp[p].M;
+      cols[n++] = pp[p].N;
     }
   if (n == 0) return FP8WS_OK;
-  if (gemm_choice(d, rows, n, N) == 1) return launch_gemm_pair<3>(d, live, n, N, K, st, splitk);
+  if (gemm_choice(d, rows, cols, n) == 1) return launch_gemm_pair<3>(d, live, n, K, st, splitk);
   int rc = FP8WS_OK;
   for (int p = 0; p < n && !rc; ++p)
-    rc = gemm_dispatch(d, live[p].a, live[p].b, live[p].M, N, K, live[p].s_in, live[p].s_w,
-                       static_cast<uint16_t *>(live[p].out), st, splitk);
+    rc = gemm_dispatch(d, live[p].a, live[p].b, live[p].M, live[p].N, K, live[p].s_in,
+                       live[p].s_w, static_cast<uint16_t *>(live[p].out), st, splitk);
+  return rc;
+}
+
+// Any number of GEMMs sharing K, in grouped launches of up to kMaxGroup.
+int gemm_groups(DeviceInfo *d, const PairProblem *pp, int np, int K, cudaStream_t st,
+                void *splitk) {
+  int rc = FP8WS_OK;
+  for (int p = 0; p < np && !rc; p += kMaxGroup)
+    rc = gemm_group_dispatch(d, pp + p, np - p < kMaxGroup ? np - p : kMaxGroup, K, st, splitk);
   return rc;
 }
 
@@ -564,7 +583,8 @@ int quant_pair_launch(DeviceInfo *d, const QuantSeg *q, int nq, cudaStream_t st,
   if (launch_ex(quant_static_pair_kernel, dim3(grid), dim3(kEwThreads), 0, st, 1, live[0],
                 live[1], split, zero_words, n_zero) != cudaSuccess)
     return FP8WS_ERR_CUDA;
-  log_launch(kKindQuant, live[0].x, live[1].x, live[0].xq);
+  log_launch(kKindQuant, live[0].x, nullptr, live[0].xq, 0);
+  log_launch(kKindQuant, live[1].x, nullptr, live[1].xq, 1);
   return launch_status();
 }
 
@@ -728,8 +748,7 @@ int gated_mlp_static_fp8(const uint16_t *x, int64_t M, int64_t dm, int64_t I, co
 }
 
 size_t qkv_shared_quant_workspace(int64_t M, int64_t d) {
-  if (M < 0 || d < 0) return 0;
-  return round256(static_cast<size_t>(M) * static_cast<size_t>(d));
+  return fp8_shared_quant_linears_workspace(M, d);
 }
 
 int qkv_shared_quant(const uint16_t *x, int64_t M, int64_t dm, const float *s_in,
@@ -737,24 +756,11 @@ int qkv_shared_quant(const uint16_t *x, int64_t M, int64_t dm, const float *s_in
                      int64_t Nk, const float *s_wk, const uint8_t *Wv, int64_t Nv,
                      const float *s_wv, void *workspace, uint16_t *q, uint16_t *k, uint16_t *v,
                      void *stream) {
-  if (!s_in || (M != 0 && !x)) return FP8WS_ERR_NULL;
-  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FP8WS_ERR_WORKSPACE;
-  if (!aligned16(x)) return FP8WS_ERR_ALIGN;
-  uint8_t *xq = static_cast<uint8_t *>(workspace);
-  int rc = check_gemm_args(xq, Wq, M, Nq, dm, s_in, s_wq, q);
-  if (!rc) rc = check_gemm_args(xq, Wk, M, Nk, dm, s_in, s_wk, k);
-  if (!rc) rc = check_gemm_args(xq, Wv, M, Nv, dm, s_in, s_wv, v);
-  if (rc) return rc;
-  DeviceInfo *d;
-  rc = device_info(&d);
-  if (rc) return rc;
-  if (M == 0) return FP8WS_OK;
-  cudaStream_t st = as_stream(stream);
-  rc = quant_launch(d, x, M * dm, s_in, xq, st);
-  if (!rc) rc = gemm_dispatch(d, xq, Wq, M, Nq, dm, s_in, s_wq, q, st);
-  if (!rc) rc = gemm_dispatch(d, xq, Wk, M, Nk, dm, s_in, s_wk, k, st);
-  if (!rc) rc = gemm_dispatch(d, xq, Wv, M, Nv, dm, s_in, s_wv, v, st);
-  return rc;
+  const uint8_t *W[3] = {Wq, Wk, Wv};
+  const int64_t N[3] = {Nq, Nk, Nv};
+  const float *s_w[3] = {s_wq, s_wk, s_wv};
+  uint16_t *y[3] = {q, k, v};
+  return fp8_shared_quant_linears(x, M, dm, s_in, 3, W, N, s_w, y, workspace, stream);
 }
 
 int fp8_gate_up_swiglu_static(const uint8_t *xq, const uint8_t *Wg, const uint8_t *Wu,
@@ -869,8 +875,8 @@ int fp8_linear_static_group(const fp8ws_linear_problem *problems, int count, int
     const fp8ws_linear_problem &q = problems[p];
     const int rc = check_gemm_args(q.xq, q.wq, q.M, N, K, q.s_in, q.s_w, q.y);
     if (rc) return rc;
-    pp[p] = PairProblem{q.xq, q.wq, nullptr, q.y, static_cast<int>(q.M), q.s_in, q.s_w,
-                        nullptr, nullptr};
+    pp[p] = PairProblem{q.xq, q.wq, nullptr, q.y, static_cast<int>(q.M), static_cast<int>(N),
+                        q.s_in, q.s_w, nullptr, nullptr};
     rows += q.M;
   }
   if (workspace && ((reinterpret_cast<uintptr_t>(workspace) & 255u) ||
@@ -885,8 +891,7 @@ int fp8_linear_static_group(const fp8ws_linear_problem *problems, int count, int
       cudaMemsetAsync(splitk_counters(workspace), 0, kSplitkCounterWords * sizeof(int), st) !=
           cudaSuccess)
     return FP8WS_ERR_CUDA;
-  return gemm_group_dispatch(d, pp, count, static_cast<int>(N), static_cast<int>(K), st,
-                             workspace);
+  return gemm_group_dispatch(d, pp, count, static_cast<int>(K), st, workspace);
 }
 
 int fp8_gate_up_swiglu_static_group(const fp8ws_gate_up_problem *problems, int count,
@@ -906,8 +911,8 @@ int fp8_gate_up_swiglu_static_group(const fp8ws_gate_up_problem *problems, int c
     if (rc) return rc;
     if (!aligned16(q.Wu)) return FP8WS_ERR_ALIGN;
     if (q.M > 0)
-      live[n++] = PairProblem{q.xq, q.Wg, q.Wu, q.h, static_cast<int>(q.M), q.s_in, q.s_wg,
-                              q.s_wu, q.s_down};
+      live[n++] = PairProblem{q.xq, q.Wg, q.Wu, q.h, static_cast<int>(q.M), static_cast<int>(I),
+                              q.s_in, q.s_wg, q.s_wu, q.s_down};
   }
   if (I % 16 != 0) return FP8WS_ERR_SHAPE;  // FP8 rows of H must be 16-byte multiples
   if (n == 0) return FP8WS_OK;
@@ -965,10 +970,10 @@ int gated_mlp_static_fp8_group(const fp8ws_mlp_tower *towers, int count, int64_t
     if (rc) return rc;
     if (t.M == 0) continue;
     qs[n] = QuantSeg{t.x, t.M * dm, t.s_in, xq};
-    up[n] = PairProblem{xq, t.Wg, t.Wu, H, static_cast<int>(t.M), t.s_in, t.s_wg, t.s_wu,
-                        t.s_down};
-    down[n] = PairProblem{H, t.Wd, nullptr, t.y, static_cast<int>(t.M), t.s_down, t.s_wd,
-                          nullptr, nullptr};
+    up[n] = PairProblem{xq, t.Wg, t.Wu, H, static_cast<int>(t.M), static_cast<int>(I), t.s_in,
+                        t.s_wg, t.s_wu, t.s_down};
+    down[n] = PairProblem{H, t.Wd, nullptr, t.y, static_cast<int>(t.M), static_cast<int>(dm),
+                          t.s_down, t.s_wd, nullptr, nullptr};
     ++n;
   }
   if (I % 16 != 0) return FP8WS_ERR_SHAPE;
@@ -981,7 +986,7 @@ int gated_mlp_static_fp8_group(const fp8ws_mlp_tower *towers, int count, int64_t
   rc = quant_pair_launch(d, qs, n, st, splitk_counters(splitk), kSplitkCounterWords);
   if (!rc) rc = launch_dual_swiglu(d, up, n, static_cast<int>(I), static_cast<int>(dm), ap, st);
   if (!rc)
-    rc = gemm_group_dispatch(d, down, n, static_cast<int>(dm), static_cast<int>(I), st, splitk);
+    rc = gemm_group_dispatch(d, down, n, static_cast<int>(I), st, splitk);
   return rc;
 }
 
@@ -1032,7 +1037,7 @@ int gated_mlp_static_fp8_noalloc(const uint16_t *x, int64_t M, int64_t d, int64_
 
 size_t fp8_shared_quant_linears_workspace(int64_t M, int64_t d) {
   if (M < 0 || d < 0) return 0;
-  return round256(static_cast<size_t>(M) * static_cast<size_t>(d));
+  return round256(static_cast<size_t>(M) * static_cast<size_t>(d)) + splitk_bytes();
 }
 
 int fp8_shared_quant_linears(const uint16_t *x, int64_t M, int64_t dm, const float *s_in, int n,
@@ -1043,22 +1048,30 @@ int fp8_shared_quant_linears(const uint16_t *x, int64_t M, int64_t dm, const flo
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FP8WS_ERR_WORKSPACE;
   if (!aligned16(x)) return FP8WS_ERR_ALIGN;
   uint8_t *xq = static_cast<uint8_t *>(workspace);
+  void *splitk = xq + round256(static_cast<size_t>(M < 0 ? 0 : M) * static_cast<size_t>(dm));
   int rc = FP8WS_OK;
-  for (int i = 0; i < n && !rc; ++i) rc = check_gemm_args(xq, W[i], M, N[i], dm, s_in, s_w[i], y[i]);
+  PairProblem pp[FP8WS_MAX_PROJECTIONS];
+  for (int i = 0; i < n && !rc; ++i) {
+    rc = check_gemm_args(xq, W[i], M, N[i], dm, s_in, s_w[i], y[i]);
+    pp[i] = PairProblem{xq, W[i], nullptr, y[i], static_cast<int>(M), static_cast<int>(N[i]),
+                        s_in, s_w[i], nullptr, nullptr};
+  }
   if (rc) return rc;
   DeviceInfo *d;
   rc = device_info(&d);
   if (rc) return rc;
   if (M == 0) return FP8WS_OK;
   cudaStream_t st = as_stream(stream);
-  rc = quant_launch(d, x, M * dm, s_in, xq, st);
-  for (int i = 0; i < n && !rc; ++i) rc = gemm_dispatch(d, xq, W[i], M, N[i], dm, s_in, s_w[i], y[i], st);
+  // the quantizer also clears the split-K counters of the GEMMs that follow
+  rc = quant_launch(d, x, M * dm, s_in, xq, st, splitk_counters(splitk), kSplitkCounterWords);
+  if (!rc) rc = gemm_groups(d, pp, n, static_cast<int>(dm), st, splitk);
   return rc;
 }
 
 size_t cross_attention_qkv_static_fp8_workspace(int64_t Mq, int64_t Mkv, int64_t d) {
   if (Mq < 0 || Mkv < 0 || d < 0) return 0;
-  return round256(static_cast<size_t>(Mq) * d) + round256(static_cast<size_t>(Mkv) * d);
+  return round256(static_cast<size_t>(Mq) * d) + round256(static_cast<size_t>(Mkv) * d) +
+         splitk_bytes();
 }
 
 int cross_attention_qkv_static_fp8(const uint16_t *x, int64_t Mq, const uint16_t *ctx,
@@ -1079,17 +1092,25 @@ int cross_attention_qkv_static_fp8(const uint16_t *x, int64_t Mq, const uint16_t
   if (!rc && ((Mq != 0 && !x) || (Mkv != 0 && !ctx))) rc = FP8WS_ERR_NULL;
   if (!rc && (!aligned16(x) || !aligned16(ctx))) rc = FP8WS_ERR_ALIGN;
   if (rc) return rc;
-  const uint8_t *wq1[1] = {Wq};
-  const int64_t nq1[1] = {Nq};
-  const float *sq1[1] = {s_wq};
-  uint16_t *yq1[1] = {q};
-  rc = fp8_shared_quant_linears(x, Mq, dm, s_q, 1, wq1, nq1, sq1, yq1, workspace, stream);
+  DeviceInfo *d;
+  rc = device_info(&d);
   if (rc) return rc;
-  const uint8_t *wkv[2] = {Wk, Wv};
-  const int64_t nkv[2] = {Nk, Nv};
-  const float *skv[2] = {s_wk, s_wv};
-  uint16_t *ykv[2] = {k, v};
-  return fp8_shared_quant_linears(ctx, Mkv, dm, s_kv, 2, wkv, nkv, skv, ykv, ws_kv, stream);
+  if (Mq == 0 && Mkv == 0) return FP8WS_OK;
+  cudaStream_t st = as_stream(stream);
+  // Q quantized from x at s_q; K and V share one quantization of ctx at s_kv
+  // (sharing between Q and K/V must not engage: they read different tensors)
+  void *splitk = ws_kv + round256(static_cast<size_t>(Mkv) * dm);
+  const QuantSeg qs[2] = {QuantSeg{x, Mq * dm, s_q, probe}, QuantSeg{ctx, Mkv * dm, s_kv, ws_kv}};
+  rc = quant_pair_launch(d, qs, 2, st, splitk_counters(splitk), kSplitkCounterWords);
+  const PairProblem pp[3] = {
+      PairProblem{probe, Wq, nullptr, q, static_cast<int>(Mq), static_cast<int>(Nq), s_q, s_wq,
+                  nullptr, nullptr},
+      PairProblem{ws_kv, Wk, nullptr, k, static_cast<int>(Mkv), static_cast<int>(Nk), s_kv, s_wk,
+                  nullptr, nullptr},
+      PairProblem{ws_kv, Wv, nullptr, v, static_cast<int>(Mkv), static_cast<int>(Nv), s_kv, s_wv,
+                  nullptr, nullptr}};
+  if (!rc) rc = gemm_groups(d, pp, 3, static_cast<int>(dm), st, splitk);
+  return rc;
 }
 
 int fp8_quant_per_token(const uint16_t *x, int64_t rows, int64_t K, float *s, uint8_t *xq,

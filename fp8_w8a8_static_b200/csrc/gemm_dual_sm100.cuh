@@ -33,6 +33,7 @@ namespace fp8ws {
 
 constexpr int kDualTileM = 256;  // rows per CTA pair
 constexpr int kDualTileN = 128;  // columns of G and of U per tile
+constexpr int kMaxDualGroup = 2; // problems per grouped launch (the two towers)
 
 // DIRECT_: H written with 16-byte global stores from registers instead of
 // TMA stores of shared-memory tiles; the freed 32 KB hold a seventh stage.
@@ -88,8 +89,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const bool leader = rank == 0;
   const int cluster = blockIdx.x >> 1;
   const int nclusters = gridDim.x >> 1;
-  const int num_n = (N + kDualTileN - 1) / kDualTileN;
-  const int num_tiles = G.n > 1 ? G.tile_start1 + G.num_m[1] * num_n : G.num_m[0] * num_n;
+  const int num_tiles = G.tiles;
   const int num_kb = (K + kGemmBK - 1) / kGemmBK;
 
   if (threadIdx.x == 0) {
@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t issued_mask = 0, issued_parity = 0;
       bool ok = true;
       for (int t = cluster; t < num_tiles && ok; t += nclusters) {
-        const GroupTile gt = group_tile(t, G, num_n);
+        const GroupTile gt = group_tile(t, G);
         const int a_row = gt.tc.m * kDualTileM + static_cast<int>(rank) * 128;
         const int b_row = gt.tc.n * kDualTileN;
         const CUtensorMap *tm_a = gt.p ? &tm_a1 : &tm_a0;
@@ -213,9 +213,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------ epilogue (both CTAs)
     const int ew = warp - 2;
     const int quarter = warp & 3;
-    float scale_g[kMaxGroup], scale_u[kMaxGroup], inv_s[kMaxGroup];
+    float scale_g[kMaxDualGroup], scale_u[kMaxDualGroup], inv_s[kMaxDualGroup];
 #pragma unroll
-    for (int p = 0; p < kMaxGroup; ++p) {
+    for (int p = 0; p < kMaxDualGroup; ++p) {
       const int q = p < G.n ? p : 0;
       scale_g[p] = __ldg(pick(G.s_in, q)) * __ldg(pick(G.s_w, q));
       scale_u[p] = __ldg(pick(G.s_in, q)) * __ldg(pick(G.s_w2, q));
@@ -223,7 +223,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     uint32_t it = 0;
     for (int t = cluster; t < num_tiles; t += nclusters, ++it) {
-      const GroupTile gt = group_tile(t, G, num_n);
+      const GroupTile gt = group_tile(t, G);
       const TileCoord tc = gt.tc;
       const int M = pick(G.M, gt.p);
       const float sg = gt.p ? scale_g[1] : scale_g[0];

@@ -1,9 +1,10 @@
 // FP8 E4M3 W8A8 GEMM on CTA pairs (tcgen05 cta_group::2), for sm_100a.
 //
-//   Y_p[M_p,N] = bf16( (s_in_p * s_w_p) * Xq_p[M_p,K] . Wq_p[N,K]^T ),  fp32 accumulation
+//   Y_p[M_p,N_p] = bf16( (s_in_p * s_w_p) * Xq_p[M_p,K] . Wq_p[N_p,K]^T ),  fp32 accumulation
 //
-// for a group of one or two problems p that share N and K (the two towers of a
-// Mixture-of-Transformers layer), in one persistent launch.  256 x 256 output
+// for a group of up to three problems p that share K (the two towers of a
+// Mixture-of-Transformers layer; the Q, K and V projections of one shared
+// quantized activation), in one persistent launch.  256 x 256 output
 // tiles are computed by a cluster of two CTAs on the two SMs of a TPC.  Each
 // CTA loads 128 rows of A and 128 rows of B per 128-byte K step (32 KB instead
 // of 48 KB per SM for the same tensor work), both CTAs' loads count on the
@@ -13,9 +14,9 @@
 //   warp 0      TMA producer (both CTAs; no cluster multicast)
 //   warp 1      TMEM allocation (both CTAs, cta_group::2); MMA issue (leader)
 //   warps 2..5  epilogue (both CTAs)
-// The tiles of the group form one sequence (problem 0's, then problem 1's),
-// dealt round-robin to the clusters, so the second problem fills the ragged
-// last wave of the first.  Bounded waits as in fp8_gemm_kernel.  Both CTAs always reach the final
+// The tiles of the group form one sequence (problem 0's, then problem 1's,
+// ...), dealt round-robin to the clusters, so each problem fills the ragged
+// last wave of the one before.  Bounded waits as in fp8_gemm_kernel.  Both CTAs always reach the final
 // cluster barrier, so neither leaves while its peer may still touch its
 // shared memory or TMEM.
 #pragma once
@@ -26,16 +27,20 @@
 namespace fp8ws {
 
 constexpr int kPairTile = 256;  // output rows and columns per CTA pair
-constexpr int kMaxGroup = 2;    // problems per grouped launch
+constexpr int kMaxGroup = 3;    // problems per grouped launch
 
-// The problems of one launch.  Global tile g belongs to problem 1 when n == 2
-// and g >= tile_start1.  s_w2 and s_down are read by the dual gate/up kernel
-// only; out[p] is Y_p (BF16) or H_p (FP8) for the register-store epilogues.
+// The problems of one launch.  Problem p owns global tiles tile_start[p] ..
+// tile_start[p + 1] - 1 (tile_start of absent problems: INT_MAX); tiles is
+// the total.  s_w2 and s_down are read by the dual gate/up kernel only; out[p]
+// is Y_p (BF16) or H_p (FP8) for the register-store epilogues.
 struct PairGroup {
   int n;
-  int tile_start1;
+  int tiles;
+  int tile_start[kMaxGroup];
   int M[kMaxGroup];
+  int N[kMaxGroup];
   int num_m[kMaxGroup];
+  int num_n[kMaxGroup];
   const float *s_in[kMaxGroup];
   const float *s_w[kMaxGroup];
   const float *s_w2[kMaxGroup];
@@ -52,13 +57,12 @@ struct GroupTile {
 // kernel parameter block is not copied to local memory.
 template <typename T>
 __device__ __forceinline__ T pick(const T (&a)[kMaxGroup], int p) {
-  return p ? a[1] : a[0];
+  return p == 2 ? a[2] : (p == 1 ? a[1] : a[0]);
 }
 
-__device__ __forceinline__ GroupTile group_tile(int g, const PairGroup &G, int num_n) {
-  const int p = (G.n > 1 && g >= G.tile_start1) ? 1 : 0;
-  const int local = p ? g - G.tile_start1 : g;
-  return GroupTile{p, tile_coord(local, pick(G.num_m, p), num_n)};
+__device__ __forceinline__ GroupTile group_tile(int g, const PairGroup &G) {
+  const int p = (g >= G.tile_start[1]) + (g >= G.tile_start[2]);
+  return GroupTile{p, tile_coord(g - pick(G.tile_start, p), pick(G.num_m, p), pick(G.num_n, p))};
 }
 
 // Split-K of the remainder tiles.  Units 0 .. dp_tiles-1 are whole tiles (the
@@ -128,11 +132,14 @@ template <int STAGES, int SCALE_MODE, bool DIRECT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a0,
                          const __grid_constant__ CUtensorMap tm_a1,
+                         const __grid_constant__ CUtensorMap tm_a2,
                          const __grid_constant__ CUtensorMap tm_b0,
                          const __grid_constant__ CUtensorMap tm_b1,
+                         const __grid_constant__ CUtensorMap tm_b2,
                          const __grid_constant__ CUtensorMap tm_d0,
-                         const __grid_constant__ CUtensorMap tm_d1, const PairGroup G, int N,
-                         int K, uint64_t timeout_ns, SplitPlan plan) {
+                         const __grid_constant__ CUtensorMap tm_d1,
+                         const __grid_constant__ CUtensorMap tm_d2, const PairGroup G, int K,
+                         uint64_t timeout_ns, SplitPlan plan) {
   using C = PairCfg<STAGES, DIRECT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -155,7 +162,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const bool leader = rank == 0;
   const int cluster = blockIdx.x >> 1;
   const int nclusters = gridDim.x >> 1;
-  const int num_n = (N + kPairTile - 1) / kPairTile;
   const int num_kb = (K + kGemmBK - 1) / kGemmBK;
   const int num_units = plan.dp_tiles + plan.split_tiles * plan.splits;
 
@@ -179,6 +185,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tma_prefetch_desc(&tm_b1);
       tma_prefetch_desc(&tm_d1);
     }
+    if (G.n > 2) {
+      tma_prefetch_desc(&tm_a2);
+      tma_prefetch_desc(&tm_b2);
+      tma_prefetch_desc(&tm_d2);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
@@ -199,9 +210,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       for (int u = cluster; u < num_units && ok; u += nclusters) {
         const UnitRange ur = unit_range(u, plan, num_kb);
-        const GroupTile gt = group_tile(ur.tile, G, num_n);
-        const CUtensorMap *tm_a = gt.p ? &tm_a1 : &tm_a0;
-        const CUtensorMap *tm_b = gt.p ? &tm_b1 : &tm_b0;
+        const GroupTile gt = group_tile(ur.tile, G);
+        const CUtensorMap *tm_a = gt.p == 2 ? &tm_a2 : (gt.p ? &tm_a1 : &tm_a0);
+        const CUtensorMap *tm_b = gt.p == 2 ? &tm_b2 : (gt.p ? &tm_b1 : &tm_b0);
         const int a_row = gt.tc.m * kPairTile + static_cast<int>(rank) * 128;
         const int b_row = gt.tc.n * kPairTile + static_cast<int>(rank) * 128;
         for (int kb = ur.kb0; kb < ur.kb1; ++kb) {
@@ -286,10 +297,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t it = 0, chunk = 0;
     for (int u = cluster; u < num_units; u += nclusters, ++it) {
       const UnitRange ur = unit_range(u, plan, num_kb);
-      const GroupTile gt = group_tile(ur.tile, G, num_n);
+      const GroupTile gt = group_tile(ur.tile, G);
       const TileCoord tc = gt.tc;
       const int M = pick(G.M, gt.p);
-      const CUtensorMap *tm_d = gt.p ? &tm_d1 : &tm_d0;
+      const int N = pick(G.N, gt.p);
+      const CUtensorMap *tm_d = gt.p == 2 ? &tm_d2 : (gt.p ? &tm_d1 : &tm_d0);
       const float *s_in = pick(G.s_in, gt.p);
       const float *s_w = pick(G.s_w, gt.p);
       uint16_t *y_out = static_cast<uint16_t *>(pick(G.out, gt.p));

@@ -348,8 +348,12 @@ FP8WS_API int gated_mlp_static_fp8_group(const fp8ws_mlp_tower *towers, int coun
  *
  * x: device [M,d] BF16.  Wq [Nq,d], Wk [Nk,d], Wv [Nv,d]: device FP8.
  * workspace: device, at least qkv_shared_quant_workspace(M,d) bytes, 256-byte
- * aligned (holds Xq).  q [M,Nq], k [M,Nk], v [M,Nv]: device BF16, contiguous.
- * Cross-attention, where K/V come from another tensor, must not use this call.
+ * aligned: Xq [M,d], then scratch for splitting the ragged last wave of the
+ * projection GEMMs over K (as fp8_linear_static_ws).  q [M,Nq], k [M,Nk],
+ * v [M,Nv]: device BF16, contiguous.  The three projections run as one
+ * grouped GEMM launch (their tiles dealt as one sequence, each projection
+ * with its own weight, scale and output).  Cross-attention, where K/V come
+ * from another tensor, must not use this call.
  */
 FP8WS_API size_t qkv_shared_quant_workspace(int64_t M, int64_t d);
 FP8WS_API int qkv_shared_quant(const uint16_t *x, int64_t M, int64_t d, const float *s_in,
@@ -410,7 +414,8 @@ FP8WS_API int gated_mlp_static_fp8_noalloc(const uint16_t *x, int64_t M, int64_t
  * arrays of n entries: device [N[i],d] FP8 weights, output widths, device fp32
  * weight scales and device [M,N[i]] BF16 outputs (each contiguous).
  * workspace: device, fp8_shared_quant_linears_workspace(M,d) bytes, 256-byte
- * aligned (holds Xq).
+ * aligned: Xq [M,d], then the split-K scratch of the projection GEMMs.  The
+ * projections run in grouped GEMM launches of up to three.
  */
 #define FP8WS_MAX_PROJECTIONS 16
 FP8WS_API size_t fp8_shared_quant_linears_workspace(int64_t M, int64_t d);
@@ -429,7 +434,9 @@ FP8WS_API int fp8_shared_quant_linears(const uint16_t *x, int64_t M, int64_t d, 
  * x: device [Mq,d] BF16; ctx: device [Mkv,d] BF16; Wq [Nq,d], Wk [Nk,d],
  * Wv [Nv,d] FP8; q [Mq,Nq], k [Mkv,Nk], v [Mkv,Nv] BF16, contiguous.
  * workspace: cross_attention_qkv_static_fp8_workspace(Mq,Mkv,d) bytes,
- * 256-byte aligned: Xq [Mq,d] then the quantized context [Mkv,d].
+ * 256-byte aligned: Xq [Mq,d], the quantized context [Mkv,d], then the
+ * split-K scratch.  Two launches: one quantize for both inputs, one grouped
+ * GEMM for Q, K and V.
  */
 FP8WS_API size_t cross_attention_qkv_static_fp8_workspace(int64_t Mq, int64_t Mkv, int64_t d);
 FP8WS_API int cross_attention_qkv_static_fp8(const uint16_t *x, int64_t Mq, const uint16_t *ctx,
@@ -548,13 +555,15 @@ FP8WS_API int fp8ws_selftest_bounded_wait(int64_t limit_ns, int mode, int64_t *e
 FP8WS_API int fp8ws_set_gemm_config(int config);
 
 /* Launch log.  Every kernel the library enqueues is counted and recorded in a
- * small ring (the most recent FP8WS_LOG_CAPACITY launches).  kind: 1 quant,
- * 2 GEMM, 3 SwiGLU-quant, 4 calibration, 5 fused gate/up SwiGLU-quant.  in0/in1 are the primary input
- * pointers (for a GEMM: activation and weight), out the output pointer. */
+ * small ring (the most recent FP8WS_LOG_CAPACITY records).  kind: 1 quant,
+ * 2 GEMM, 3 SwiGLU-quant, 4 calibration, 5 fused gate/up SwiGLU-quant.
+ * in0/in1 are the primary input pointers (for a GEMM: activation and weight),
+ * out the output pointer.  A grouped launch writes one record per problem,
+ * member 0, 1, ... in group order, and counts as one launch. */
 #define FP8WS_LOG_CAPACITY 64
 typedef struct {
   int32_t kind;
-  int32_t pad;
+  int32_t member;
   const void *in0;
   const void *in1;
   const void *out;

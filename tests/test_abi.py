@@ -54,7 +54,8 @@ def test_workspace_sizes(lib):
     def r256(v):
         return (v + 255) // 256 * 256
     assert lib.gated_mlp_static_fp8_workspace(64, 256, 704) == r256(64 * 256) + 2 * r256(64 * 704 * 2) + r256(64 * 704)
-    assert lib.qkv_shared_quant_workspace(2048, 3072) == 2048 * 3072
+    # Xq, then the split-K scratch of the grouped projection GEMMs
+    assert lib.qkv_shared_quant_workspace(2048, 3072) == 2048 * 3072 + lib.fp8_linear_static_ws_bytes()
     assert lib.gated_mlp_static_fp8_workspace(-1, 1, 1) == 0
 
 
@@ -129,7 +130,7 @@ def _header_struct_fields(name):
 @pytest.mark.parametrize("cname,pyname", [
     ("fp8ws_quant_problem", "QuantProblem"), ("fp8ws_linear_problem", "LinearProblem"),
     ("fp8ws_gate_up_problem", "GateUpProblem"), ("fp8ws_mlp_tower", "MlpTower"),
-    ("fp8ws_swiglu", "Swiglu")])
+    ("fp8ws_swiglu", "Swiglu"), ("fp8ws_launch_record", "LaunchRecord")])
 def test_group_structs_match_header(cname, pyname):
     """The ctypes layouts follow the header's fields in order.  The group
     structs hold only pointers and 64-bit integers, and the SwiGLU descriptor

@@ -58,13 +58,15 @@ def test_cross_attention_projections():
     q, k, v = fw.cross_attention_qkv_static_fp8(x, ctx, scalar(s_q, DEV), *wq, scalar(s_kv, DEV),
                                                 *wk, *wv, workspace=ws)
     log = fw.launch_log()
-    kinds = [r[0] for r in log]
-    assert kinds == [fw.KIND_QUANT, fw.KIND_GEMM, fw.KIND_QUANT, fw.KIND_GEMM, fw.KIND_GEMM]
-    xq_ptr, ctxq_ptr = log[0][3], log[2][3]
-    assert log[0][1] == x.data_ptr() and log[2][1] == ctx.data_ptr()
+    # one quantize launch for both inputs, one grouped GEMM launch for Q, K, V
+    assert [(r[0], r[4]) for r in log] == [(fw.KIND_QUANT, 0), (fw.KIND_QUANT, 1),
+                                           (fw.KIND_GEMM, 0), (fw.KIND_GEMM, 1), (fw.KIND_GEMM, 2)]
+    xq_ptr, ctxq_ptr = log[0][3], log[1][3]
+    assert log[0][1] == x.data_ptr() and log[1][1] == ctx.data_ptr()
     assert xq_ptr != ctxq_ptr                        # Q does not share K/V's quantization
-    assert log[1][1] == xq_ptr
+    assert log[2][1] == xq_ptr and log[2][3] == q.data_ptr()
     assert log[3][1] == ctxq_ptr and log[4][1] == ctxq_ptr   # K and V share one
+    assert log[3][3] == k.data_ptr() and log[4][3] == v.data_ptr()
     rq = np.random.default_rng(6).choice(Mq, 6, replace=False)
     rk = np.random.default_rng(7).choice(Mkv, 6, replace=False)
     ref_q = oracle.qkv_shared_quant(bits(x[rq]), s_q, [_ref(wq)])[0]

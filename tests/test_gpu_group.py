@@ -218,7 +218,13 @@ def test_mlp_group_matches_single_towers(M0, M1, d, I):
     ys = fw.gated_mlp_static_fp8_group(towers, workspace=ws)
     log = fw.launch_log()
     torch.cuda.synchronize()
-    assert [r[0] for r in log] == [fw.KIND_QUANT, fw.KIND_DUAL, fw.KIND_GEMM]
+    # three launches, each with one record per tower
+    assert [(r[0], r[4]) for r in log] == [(fw.KIND_QUANT, 0), (fw.KIND_QUANT, 1),
+                                           (fw.KIND_DUAL, 0), (fw.KIND_DUAL, 1),
+                                           (fw.KIND_GEMM, 0), (fw.KIND_GEMM, 1)]
+    xq0, xq1 = log[0][3], log[1][3]
+    assert log[2][1] == xq0 and log[3][1] == xq1     # gate/up read each tower's Xq
+    assert log[4][1] == log[2][3] and log[5][1] == log[3][3]   # down reads each H
     views = fw.group_workspace_views(ws, [M0, M1], d, I)
     for p, t in enumerate(towers):
         y1, v1 = _single(t)
