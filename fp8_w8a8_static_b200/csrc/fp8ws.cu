@@ -14,6 +14,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -51,19 +52,33 @@ void log_launch(int kind, const void *in0, const void *in1, const void *out, int
 enum { kKindQuant = 1, kKindGemm = 2, kKindSwiglu = 3, kKindCalib = 4, kKindDual = 5 };
 
 // --------------------------------------------------------------- device info
+// Per-device state, written once under g_dev_mu and read without it: the
+// flags are atomics released after the values they publish.
 struct DeviceInfo {
-  int checked = 0;  // 0 unknown, 1 sm_100, -1 other
-  int sms = 0;
+  std::atomic<int> checked{0};  // 0 unknown, 1 sm_100, -1 other
+  int sms = 0;                  // set before `checked` is released
   // bit per kernel whose attributes were set on this device: 0-2 one-CTA GEMMs,
   // 3/5/6/7 pair GEMM scale modes (+16 direct-store), 4 dual (+8 variant,
   // +16 direct variant, +24 direct plain), 8 per-token SwiGLU
-  unsigned gemm_attr_set = 0;
-  int pair_clusters = 0;       // CTA pairs of the pair GEMM resident at once
-  int dual_clusters = 0;       // CTA pairs of the gate/up dual GEMM resident at once
+  std::atomic<unsigned> gemm_attr_set{0};
+  std::atomic<int> pair_clusters{0};  // CTA pairs of the pair GEMM resident at once
+  std::atomic<int> dual_clusters{0};  // CTA pairs of the gate/up dual GEMM resident at once
   // (the same for every epilogue variant: one CTA per SM either way)
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
+
+// First-use set-up of kernel `bit` on this device, once across threads:
+// `setup` runs under g_dev_mu, and the bit is published after it succeeded.
+template <typename F>
+int once_per_device(DeviceInfo *d, int bit, F setup) {
+  if (d->gemm_attr_set.load(std::memory_order_acquire) & (1u << bit)) return 0;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (d->gemm_attr_set.load(std::memory_order_relaxed) & (1u << bit)) return 0;
+  const int rc = setup();
+  if (rc == 0) d->gemm_attr_set.fetch_or(1u << bit, std::memory_order_release);
+  return rc;
+}
 
 int current_device(int *dev) {
   if (cudaGetDevice(dev) != cudaSuccess) return FP8WS_ERR_CUDA;
@@ -76,19 +91,19 @@ int device_info(DeviceInfo **out) {
   int st = current_device(&dev);
   if (st) return st;
   DeviceInfo &d = g_dev[dev];
-  if (d.checked == 0) {
+  if (d.checked.load(std::memory_order_acquire) == 0) {
     std::lock_guard<std::mutex> lk(g_dev_mu);
-    if (d.checked == 0) {
+    if (d.checked.load(std::memory_order_relaxed) == 0) {
       int major = 0, minor = 0, sms = 0;
       if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
           cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
           cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return FP8WS_ERR_CUDA;
       d.sms = sms;
-      d.checked = (major == 10 && minor == 0) ? 1 : -1;
+      d.checked.store((major == 10 && minor == 0) ? 1 : -1, std::memory_order_release);
     }
   }
-  if (d.checked != 1) return FP8WS_ERR_UNSUPPORTED;
+  if (d.checked.load(std::memory_order_acquire) != 1) return FP8WS_ERR_UNSUPPORTED;
   *out = &d;
   return FP8WS_OK;
 }
@@ -106,14 +121,15 @@ cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
 // kernels loop over the rest with a grid stride).
 template <typename Kernel>
 int ew_grid(const DeviceInfo *d, Kernel kern, int64_t nvec) {
-  static int resident = 0;  // blocks per SM; same on every B200
-  if (resident == 0) {
+  // blocks per SM, the same on every B200; found once per kernel (thread-safe
+  // initialisation of a function-local static)
+  static const int resident = [kern] {
     int r = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&r, kern, kEwThreads, 0) != cudaSuccess ||
         r < 1)
       r = 1;
-    resident = r;
-  }
+    return r;
+  }();
   int64_t per_block = static_cast<int64_t>(kEwThreads) * kEwUnroll;
   int64_t want = (nvec + per_block - 1) / per_block;
   int64_t cap = static_cast<int64_t>(d->sms) * resident;
@@ -126,12 +142,11 @@ int ew_grid(const DeviceInfo *d, Kernel kern, int64_t nvec) {
 // kernel on the stream may be scheduled while this one finishes, and waits in
 // griddepcontrol.wait before touching memory.  FP8WS_PDL=0 turns it off.
 bool use_pdl() {
-  static int v = -1;
-  if (v < 0) {
+  static const bool v = [] {
     const char *e = getenv("FP8WS_PDL");
-    v = (e && e[0] == '0') ? 0 : 1;
-  }
-  return v == 1;
+    return !(e && e[0] == '0');
+  }();
+  return v;
 }
 
 template <typename... KArgs, typename... Args>
@@ -203,12 +218,13 @@ int launch_gemm_cfg(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int M, 
                     const float *s_in, const float *s_w, uint16_t *y, cudaStream_t st) {
   using C = GemmCfg<BN, STAGES>;
   auto kern = fp8_gemm_kernel<BN, STAGES>;
-  if (!(d->gemm_attr_set & (1u << BIT))) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
-        cudaSuccess)
-      return FP8WS_ERR_CUDA;
-    d->gemm_attr_set |= 1u << BIT;
-  }
+  int rc0 = once_per_device(d, BIT, [&] {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                C::SMEM_BYTES) == cudaSuccess
+               ? FP8WS_OK
+               : FP8WS_ERR_CUDA;
+  });
+  if (rc0) return rc0;
   CUtensorMap ma, mb, md;
   int rc = make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, xq, M, K, kGemmBK, kGemmBM, true);
   if (!rc) rc = make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, wq, N, K, kGemmBK, BN, true);
@@ -316,8 +332,8 @@ PairGroup make_pair_group(const PairProblem *pp, int np, int tile_m, int tile_n)
 // Grid of a CTA-pair kernel: as many clusters of two as can be resident at
 // once, found by the occupancy query on the first launch of each variant.
 template <typename Kernel>
-int pair_clusters(DeviceInfo *d, Kernel kern, int smem, int bit, int *clusters_out) {
-  if (!(d->gemm_attr_set & (1u << bit))) {
+int pair_clusters(DeviceInfo *d, Kernel kern, int smem, int bit, std::atomic<int> *clusters_out) {
+  return once_per_device(d, bit, [&] {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)
       return FP8WS_ERR_CUDA;
@@ -335,10 +351,9 @@ int pair_clusters(DeviceInfo *d, Kernel kern, int smem, int bit, int *clusters_o
     int clusters = 0;
     if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1)
       return FP8WS_ERR_CUDA;
-    *clusters_out = clusters;
-    d->gemm_attr_set |= 1u << bit;
-  }
-  return FP8WS_OK;
+    clusters_out->store(clusters, std::memory_order_relaxed);
+    return FP8WS_OK;
+  });
 }
 
 template <int STAGES, int BIT, int SCALE_MODE = 0, bool DIRECT = false>
@@ -369,9 +384,11 @@ int launch_gemm_pair_cfg(DeviceInfo *d, const PairProblem *pp, int np, int K, cu
   float *partials = static_cast<float *>(splitk);
   int *counters = splitk ? splitk_counters(splitk) : nullptr;
   const SplitPlan plan =
-      make_split_plan(tiles, d->pair_clusters, (K + kGemmBK - 1) / kGemmBK, partials, counters);
+      make_split_plan(tiles, d->pair_clusters.load(std::memory_order_relaxed),
+                      (K + kGemmBK - 1) / kGemmBK, partials, counters);
   const int units = plan.dp_tiles + plan.split_tiles * plan.splits;
-  const int clusters = units < d->pair_clusters ? units : d->pair_clusters;
+  const int resident = d->pair_clusters.load(std::memory_order_relaxed);
+  const int clusters = units < resident ? units : resident;
   if (launch_ex(kern, dim3(2 * clusters), dim3(kGemmThreads), C::SMEM_BYTES, st, 2, ma[0], ma[1],
                 ma[2], mb[0], mb[1], mb[2], md[0], md[1], md[2], G, K, kWaitLimitNs,
                 plan) != cudaSuccess)
@@ -384,12 +401,11 @@ int launch_gemm_pair_cfg(DeviceInfo *d, const PairProblem *pp, int np, int K, cu
 // six pipeline stages (default), or 16-byte global stores from registers with
 // seven stages (FP8WS_EPILOGUE=direct).
 bool direct_epilogue() {
-  static int v = -1;
-  if (v < 0) {
+  static const bool v = [] {
     const char *e = getenv("FP8WS_EPILOGUE");
-    v = (e && e[0] == 'd') ? 1 : 0;
-  }
-  return v == 1;
+    return e && e[0] == 'd';
+  }();
+  return v;
 }
 
 template <int BIT, int SCALE_MODE = 0>
@@ -434,7 +450,8 @@ int launch_dual_swiglu_cfg(DeviceInfo *d, const PairProblem *pp, int np, int N, 
   }
   const PairGroup G = make_pair_group(pp, np, kDualTileM, kDualTileN);
   const int tiles = G.tiles;
-  const int clusters = tiles < d->dual_clusters ? tiles : d->dual_clusters;
+  const int resident = d->dual_clusters.load(std::memory_order_relaxed);
+  const int clusters = tiles < resident ? tiles : resident;
   if (launch_ex(kern, dim3(2 * clusters), dim3(kGemmThreads), C::SMEM_BYTES, st, 2, ma[0], mg[0],
                 mu[0], mh[0], ma[1], mg[1], mu[1], mh[1], G, act, N, K,
                 kWaitLimitNs) != cudaSuccess)
@@ -480,13 +497,15 @@ int check_gemm_args(const void *xq, const void *wq, int64_t M, int64_t N, int64_
 // efficiencies are the measured throughput of each configuration on large
 // problems relative to the CTA-pair kernel: narrower one-CTA tiles move more
 // operand bytes per tensor cycle and become L2-bandwidth bound.
-int g_forced_gemm_config = 0;  // fp8ws_set_gemm_config: 0 = cost model
+std::atomic<int> g_forced_gemm_config{0};  // fp8ws_set_gemm_config: 0 = cost model
 
 // 1 = CTA pair 256 x 256, 2 = one CTA 128 x 256, 3 = 128 x 128, 4 = 128 x 64,
 // for the np problems M[p] x N[p] that one launch would cover.
 int gemm_choice(const DeviceInfo *d, const int64_t *M, const int64_t *N, int np) {
-  if (g_forced_gemm_config) return g_forced_gemm_config;
-  const int pairs = d->pair_clusters > 0 ? d->pair_clusters : d->sms / 2;
+  const int forced = g_forced_gemm_config.load(std::memory_order_relaxed);
+  if (forced) return forced;
+  const int resident = d->pair_clusters.load(std::memory_order_relaxed);
+  const int pairs = resident > 0 ? resident : d->sms / 2;
   auto waves = [](int64_t tiles, int64_t slots) { return (tiles + slots - 1) / slots; };
   int64_t t_pair = 0, t_256 = 0, t_128 = 0, t_64 = 0;
   for (int p = 0; p < np; ++p) {
@@ -1162,12 +1181,13 @@ int silu_mul_2in_fp8_per_token(const uint16_t *g, const uint16_t *u, int64_t row
   int rc = device_info(&d);
   if (rc) return rc;
   const size_t smem = static_cast<size_t>(I) * sizeof(float);
-  if (!(d->gemm_attr_set & (1u << 8))) {
-    if (cudaFuncSetAttribute(silu_mul_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kMaxRowI * sizeof(float)) != cudaSuccess)
-      return FP8WS_ERR_CUDA;
-    d->gemm_attr_set |= 1u << 8;
-  }
+  rc = once_per_device(d, 8, [] {
+    return cudaFuncSetAttribute(silu_mul_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kMaxRowI * sizeof(float)) == cudaSuccess
+               ? FP8WS_OK
+               : FP8WS_ERR_CUDA;
+  });
+  if (rc) return rc;
   cudaStream_t st = as_stream(stream);
   if (launch_ex(silu_mul_rows_kernel, dim3(static_cast<unsigned>(rows)), dim3(kRowThreads), smem,
                 st, 1, g, u, static_cast<int>(I), s, h) != cudaSuccess)
@@ -1348,7 +1368,7 @@ int fp8ws_device_status(int *status, int *where) {
 
 int fp8ws_set_gemm_config(int config) {
   if (config < 0 || config > 4) return FP8WS_ERR_SHAPE;
-  g_forced_gemm_config = config;
+  g_forced_gemm_config.store(config, std::memory_order_relaxed);
   return FP8WS_OK;
 }
 
