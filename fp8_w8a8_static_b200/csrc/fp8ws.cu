@@ -196,9 +196,11 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Row-major [rows, cols] matrix, 128-byte swizzled boxes of box_cols x box_rows.
+// Row-major [rows, cols] matrix, swizzled boxes of box_cols x box_rows (the
+// box's rows are 128 bytes for the 128-byte swizzle, 64 for the 64-byte one).
 int make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, int elem_bytes, const void *base,
-                int64_t rows, int64_t cols, int box_cols, int box_rows, bool for_load) {
+                int64_t rows, int64_t cols, int box_cols, int box_rows, bool for_load,
+                CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return FP8WS_ERR_CUDA;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
@@ -206,7 +208,7 @@ int make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, int elem_bytes, const 
   cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                   for_load ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_NONE,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? FP8WS_OK : FP8WS_ERR_CUDA;
@@ -332,7 +334,8 @@ PairGroup make_pair_group(const PairProblem *pp, int np, int tile_m, int tile_n)
 // Grid of a CTA-pair kernel: as many clusters of two as can be resident at
 // once, found by the occupancy query on the first launch of each variant.
 template <typename Kernel>
-int pair_clusters(DeviceInfo *d, Kernel kern, int smem, int bit, std::atomic<int> *clusters_out) {
+int pair_clusters(DeviceInfo *d, Kernel kern, int threads, int smem, int bit,
+                  std::atomic<int> *clusters_out) {
   return once_per_device(d, bit, [&] {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)
@@ -344,7 +347,7 @@ int pair_clusters(DeviceInfo *d, Kernel kern, int smem, int bit, std::atomic<int
     attr[0].val.clusterDim.z = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (d->sms / 2));
-    cfg.blockDim = dim3(kGemmThreads);
+    cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = smem;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
@@ -361,7 +364,7 @@ int launch_gemm_pair_cfg(DeviceInfo *d, const PairProblem *pp, int np, int K, cu
                          void *splitk = nullptr) {
   using C = PairCfg<STAGES, DIRECT>;
   auto kern = fp8_gemm_pair_kernel<STAGES, SCALE_MODE, DIRECT>;
-  int rc = pair_clusters(d, kern, C::SMEM_BYTES, BIT, &d->pair_clusters);
+  int rc = pair_clusters(d, kern, kGemmThreads, C::SMEM_BYTES, BIT, &d->pair_clusters);
   if (rc) return rc;
   CUtensorMap ma[kMaxGroup], mb[kMaxGroup], md[kMaxGroup];
   for (int p = 0; p < np && !rc; ++p) {
@@ -430,7 +433,7 @@ int launch_dual_swiglu_cfg(DeviceInfo *d, const PairProblem *pp, int np, int N, 
                            SwigluParams act, cudaStream_t st) {
   using C = DualCfg<STAGES, DIRECT>;
   auto kern = fp8_dual_swiglu_pair_kernel<STAGES, DIRECT, VARIANT>;
-  int rc = pair_clusters(d, kern, C::SMEM_BYTES, BIT, &d->dual_clusters);
+  int rc = pair_clusters(d, kern, kDualThreads, C::SMEM_BYTES, BIT, &d->dual_clusters);
   if (rc) return rc;
   CUtensorMap ma[kMaxDualGroup], mg[kMaxDualGroup], mu[kMaxDualGroup], mh[kMaxDualGroup];
   for (int p = 0; p < np && !rc; ++p) {
@@ -439,7 +442,9 @@ int launch_dual_swiglu_cfg(DeviceInfo *d, const PairProblem *pp, int np, int N, 
     if (!rc) rc = make_map_2d(&mg[p], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.b, N, K, kGemmBK, 128, true);
     if (!rc)
       rc = make_map_2d(&mu[p], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.b2, N, K, kGemmBK, 128, true);
-    if (!rc) rc = make_map_2d(&mh[p], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.out, q.M, N, 128, 32, false);
+    if (!rc)
+      rc = make_map_2d(&mh[p], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.out, q.M, N, C::EPI_COLS, 32,
+                       false, CU_TENSOR_MAP_SWIZZLE_64B);
   }
   if (rc) return rc;
   if (np == 1) {
@@ -452,7 +457,7 @@ int launch_dual_swiglu_cfg(DeviceInfo *d, const PairProblem *pp, int np, int N, 
   const int tiles = G.tiles;
   const int resident = d->dual_clusters.load(std::memory_order_relaxed);
   const int clusters = tiles < resident ? tiles : resident;
-  if (launch_ex(kern, dim3(2 * clusters), dim3(kGemmThreads), C::SMEM_BYTES, st, 2, ma[0], mg[0],
+  if (launch_ex(kern, dim3(2 * clusters), dim3(kDualThreads), C::SMEM_BYTES, st, 2, ma[0], mg[0],
                 mu[0], mh[0], ma[1], mg[1], mu[1], mh[1], G, act, N, K,
                 kWaitLimitNs) != cudaSuccess)
     return FP8WS_ERR_CUDA;

@@ -16,9 +16,12 @@
 // rows of Xq and 128 rows of its weight per 128-byte K step (32 KB per SM, the
 // same operand traffic per flop as the plain CTA-pair GEMM).  TMEM per CTA
 // holds two buffers of (G 128 columns | U 128 columns), so the epilogue of a
-// tile overlaps the main loop of the next.  Epilogue warps read 32 columns of
-// G and of U per step, write 32 FP8 codes of each row into a 128-byte swizzled
-// row and TMA-store 32 x 128-byte boxes.  Roles, bounded waits and teardown
+// tile overlaps the main loop of the next.  Eight warps share the epilogue:
+// two per TMEM lane quarter (a warp may only read the 32 lanes of quarter
+// warp % 4), each taking 64 of the tile's 128 columns, which keeps each
+// warp's share of the SwiGLU work per tile small beside the main loop.  A warp reads 32 columns of G and of U per
+// step, writes 32 FP8 codes of each row into a 64-byte swizzled row and
+// TMA-stores 32 x 64-byte boxes.  Roles, bounded waits and teardown
 // follow fp8_gemm_pair_kernel, and so does the problem group: one launch can
 // cover the gate/up projections of both towers of a Mixture-of-Transformers
 // layer (shared d and I, per-tower rows, weights and scales), their tiles
@@ -34,6 +37,8 @@ namespace fp8ws {
 constexpr int kDualTileM = 256;  // rows per CTA pair
 constexpr int kDualTileN = 128;  // columns of G and of U per tile
 constexpr int kMaxDualGroup = 2; // problems per grouped launch (the two towers)
+constexpr int kDualEpiWarps = 8;                        // two per TMEM lane quarter
+constexpr int kDualThreads = (2 + kDualEpiWarps) * 32;  // producer, MMA, epilogue
 
 // DIRECT_: H written with 16-byte global stores from registers instead of
 // TMA stores of shared-memory tiles; the freed 32 KB hold a seventh stage.
@@ -45,8 +50,9 @@ struct DualCfg {
   static constexpr int B_BYTES = 128 * kGemmBK;   // 128 rows of Wg (leader) or Wu (peer)
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TX_BYTES = 2 * STAGE_BYTES;
-  static constexpr int EPI_BUF_BYTES = 32 * 128;   // 32 rows x 128 FP8 codes
-  static constexpr int EPI_BYTES = DIRECT ? 0 : 4 * 2 * EPI_BUF_BYTES;
+  static constexpr int EPI_COLS = kDualTileN / 2;      // columns of H per epilogue warp
+  static constexpr int EPI_BUF_BYTES = 32 * EPI_COLS;  // 32 rows x 64 FP8 codes
+  static constexpr int EPI_BYTES = DIRECT ? 0 : kDualEpiWarps * 2 * EPI_BUF_BYTES;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
   static constexpr uint32_t ACC_COLS = 2 * kDualTileN;  // G | U
@@ -57,7 +63,7 @@ struct DualCfg {
 };
 
 template <int STAGES, bool DIRECT, bool VARIANT>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kDualThreads, 1)
     fp8_dual_swiglu_pair_kernel(const __grid_constant__ CUtensorMap tm_a0,
                                 const __grid_constant__ CUtensorMap tm_bg0,
                                 const __grid_constant__ CUtensorMap tm_bu0,
@@ -99,7 +105,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 8);
+      mbar_init(&tempty[i], 2 * kDualEpiWarps);  // every epilogue warp of both CTAs
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -211,8 +217,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------ epilogue (both CTAs)
-    const int ew = warp - 2;
-    const int quarter = warp & 3;
+    const int ew = warp - 2;                      // 0 .. kDualEpiWarps - 1
+    const int quarter = warp & 3;                 // the TMEM lanes this warp may read
+    const int cbase = (ew >> 2) * C::EPI_COLS;    // this warp's 64 of the tile's columns
     float scale_g[kMaxDualGroup], scale_u[kMaxDualGroup], inv_s[kMaxDualGroup];
 #pragma unroll
     for (int p = 0; p < kMaxDualGroup; ++p) {
@@ -242,25 +249,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_after();
       const int row0 = tc.m * kDualTileM + static_cast<int>(rank) * 128 + quarter * 32;
-      const int col0 = tc.n * kDualTileN;
+      const int col0 = tc.n * kDualTileN + cbase;
       const bool store = row0 < M && col0 < N;
       const uint32_t t_g =
-          tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * C::ACC_COLS;
+          tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * C::ACC_COLS + cbase;
       uint8_t *buf = sEpi + (ew * 2 + (it & 1u)) * C::EPI_BUF_BYTES;
       if (!DIRECT) {
         if (lane == 0) tma_store_wait_read<1>();  // this buffer's previous store has read it
         __syncwarp();
       }
-      uint8_t *row = buf + lane * 128;
+      uint8_t *row = buf + lane * C::EPI_COLS;
       uint8_t *hrow = h_out + static_cast<int64_t>(row0 + lane) * N + col0;
       const bool row_ok = row0 + lane < M;
 #pragma unroll 1
-      for (int c = 0; c < kDualTileN / 32; ++c) {
+      for (int c = 0; c < C::EPI_COLS / 32; ++c) {
         uint32_t g[32], u[32];
         tmem_ld_32x32b_x32(t_g + c * 32, g);
         tmem_ld_32x32b_x32(t_g + kDualTileN + c * 32, u);
         tmem_ld_wait();
-        if (c == kDualTileN / 32 - 1) {
+        if (c == C::EPI_COLS / 32 - 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(map_shared_rank(smem_u32(&tempty[acc]), 0));
@@ -284,10 +291,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (row_ok && col0 + 32 * c + 16 < N)
             *reinterpret_cast<uint4 *>(hrow + 32 * c + 16) = make_uint4(q[4], q[5], q[6], q[7]);
         } else {
-          // 32 codes = two 16-byte units (2c, 2c+1) of this row, swizzled
-          *reinterpret_cast<uint4 *>(row + (((2 * c) ^ (lane & 7)) << 4)) =
+          // 32 codes = 16-byte units 2c and 2c + 1 of this 64-byte row, placed
+          // as the 64-byte swizzle of the store map expects: unit k of row r
+          // at ((k ^ ((r >> 1) & 3)) << 4)
+          const int sw = (lane >> 1) & 3;
+          *reinterpret_cast<uint4 *>(row + (((2 * c) ^ sw) << 4)) =
               make_uint4(q[0], q[1], q[2], q[3]);
-          *reinterpret_cast<uint4 *>(row + (((2 * c + 1) ^ (lane & 7)) << 4)) =
+          *reinterpret_cast<uint4 *>(row + (((2 * c + 1) ^ sw) << 4)) =
               make_uint4(q[4], q[5], q[6], q[7]);
         }
       }
