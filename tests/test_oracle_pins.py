@@ -591,3 +591,24 @@ def test_gated_mlp_per_token_rows_and_weight_channels():
     y2 = oracle.gated_mlp_per_token(x, wg, swg, wu, swu, wd, swd2)
     assert np.array_equal(oracle.bf16_to_f64(y2[:, 7]), 2 * oracle.bf16_to_f64(y[:, 7]))
     assert np.array_equal(np.delete(y2, 7, axis=1), np.delete(y, 7, axis=1))
+
+
+def test_down_scales_match_an_independent_composition():
+    """With one calibration batch the moving average is that batch's maximum,
+    so the down_proj scale is fp32(max|SiLU(X Wg^T) * (X Wu^T)| / 448): checked
+    against torch's fp64 matmul and the x * sigmoid(x) form of SiLU.  Swapping
+    gate and up changes it (SiLU belongs to the gate)."""
+    d = synth.c0_mlp()
+    x, wg, wu = d["calib"][0], d["wg"], d["wu"]
+    s = oracle.down_scale([bits_of(x)], bits_of(wg), bits_of(wu))
+    g = x.double() @ wg.double().T
+    u = x.double() @ wu.double().T
+    want = float((g * torch.sigmoid(g) * u).abs().max()) / 448.0
+    assert abs(s - want) <= 2.0 ** -22 * want          # one fp32 rounding of the same value
+    swapped = oracle.down_scale([bits_of(x)], bits_of(wu), bits_of(wg))
+    assert swapped != s
+    gg = synth.normal((64, 300), 2.0, 71)
+    uu = synth.normal((64, 300), 1.0, 72)
+    s2 = oracle.swiglu_down_scale([(bits_of(gg), bits_of(uu))])
+    want2 = float((gg.double() * torch.sigmoid(gg.double()) * uu.double()).abs().max()) / 448.0
+    assert abs(s2 - want2) <= 2.0 ** -22 * want2
