@@ -83,3 +83,43 @@ def test_kv_input_scales_checked_at_load():
     assert fw.fp8_check_shared_input_scale([s, s.clone()]) == fw.OK
     other = scalar(0.031, DEV)
     assert fw.fp8_check_shared_input_scale([s, other]) == fw.ERR_SCALE_MISMATCH
+
+
+def test_many_projections_in_groups_of_three():
+    """Seven projections of one shared quantization (two full groups of three
+    and a remainder, ragged widths) against the oracle; one launch per group."""
+    M, d = 300, 512
+    x = synth.activation_with_outliers(M, d, 5, 8, 0, DEV)
+    s = oracle.f32(0.029)
+    widths = (264, 1024, 8, 520, 256, 3072, 128)
+    projs = [_proj(n, d, 530 + i) for i, n in enumerate(widths)]
+    fw.launch_log_clear()
+    ys = fw.fp8_shared_quant_linears(x, scalar(s, DEV), projs)
+    log = fw.launch_log()
+    assert [(r[0], r[4]) for r in log] == [(fw.KIND_QUANT, 0)] + [
+        (fw.KIND_GEMM, m) for m in (0, 1, 2, 0, 1, 2, 0)]
+    assert all(r[1] == log[0][3] for r in log[1:])          # every GEMM reads the one Xq
+    refs = oracle.qkv_shared_quant(bits(x), s, [_ref(p) for p in projs])
+    for y, r, n in zip(ys, refs, widths):
+        assert y.shape == (M, n) and y.is_contiguous()
+        assert rel_fro(bits(y), r) <= GEMM_REL_FRO
+    assert fw.device_status()[0] == fw.OK
+
+
+@pytest.mark.parametrize("Mq,Mkv", [(0, 256), (256, 0)])
+def test_cross_attention_with_an_empty_side(Mq, Mkv):
+    d = 512
+    x = synth.activation_with_outliers(max(Mq, 1), d, 5, 9, 0, DEV)[:Mq]
+    ctx = synth.activation_with_outliers(max(Mkv, 1), d, 5, 10, 0, DEV)[:Mkv]
+    s_q, s_kv = oracle.f32(0.031), oracle.f32(0.027)
+    wq, wk, wv = _proj(512, d, 541), _proj(256, d, 542), _proj(256, d, 543)
+    q, k, v = fw.cross_attention_qkv_static_fp8(x, ctx, scalar(s_q, DEV), *wq, scalar(s_kv, DEV),
+                                                *wk, *wv)
+    assert q.shape == (Mq, 512) and k.shape == (Mkv, 256) and v.shape == (Mkv, 256)
+    if Mq:
+        ref_q = oracle.qkv_shared_quant(bits(x), s_q, [_ref(wq)])[0]
+        assert rel_fro(bits(q), ref_q) <= GEMM_REL_FRO
+    if Mkv:
+        ref_k, ref_v = oracle.qkv_shared_quant(bits(ctx), s_kv, [_ref(wk), _ref(wv)])
+        assert rel_fro(bits(k), ref_k) <= GEMM_REL_FRO and rel_fro(bits(v), ref_v) <= GEMM_REL_FRO
+    assert fw.device_status()[0] == fw.OK
