@@ -269,3 +269,21 @@ def test_mlp_group_one_tower_empty():
     y1, _ = _single(t0)
     assert ys[1].shape == (0, d)
     assert rel_fro(bits(ys[0]), bits(y1)) <= 1e-3
+
+
+def test_mlp_group_large_sizes_sampled_rows():
+    """Beyond the benchmark's shapes: towers of 16384 and 8192 tokens, d=4096,
+    I=16384 (6,144 gate/up tiles and 384 down tiles per launch, K up to
+    16384); the oracle checks sampled rows of each tower."""
+    d, I = 4096, 16384
+    towers = [_tower(16384, d, I, 61, 0.0025), _tower(8192, d, I, 62, 0.0027)]
+    ys = fw.gated_mlp_static_fp8_group(towers)
+    for p, (t, y) in enumerate(zip(towers, ys)):
+        rows = np.random.default_rng(p + 90).choice(t["x"].shape[0], 3, replace=False)
+        ref = oracle.gated_mlp(np.ascontiguousarray(bits(t["x"])[rows]), t["s_in"].item(),
+                               codes(t["wg"]), t["s_wg"].item(), codes(t["wu"]), t["s_wu"].item(),
+                               t["s_down"].item(), codes(t["wd"]), t["s_wd"].item())
+        assert rel_fro(bits(y)[rows], ref) <= GEMM_REL_FRO
+    assert fw.device_status()[0] == fw.OK
+    del towers, ys
+    torch.cuda.empty_cache()
