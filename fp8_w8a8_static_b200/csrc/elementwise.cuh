@@ -4,7 +4,11 @@
 // All of them stream flat contiguous runs: each thread moves 16-byte vectors
 // (8 BF16 values) with several vectors in flight, grids are sized to fill every
 // SM, and the ragged tail (numel not a multiple of 8) is finished by the first
-// threads of the grid one element at a time.
+// threads of the grid one element at a time.  The hot ones (the quantizer and
+// the two-input SwiGLU) also have a wide form: 32-byte loads (16 values) and
+// 16-byte stores of the codes, half the memory instructions per byte.  The host
+// chooses it for 32-byte-aligned inputs (for the SwiGLU kernels also by length:
+// swiglu_wide_form in fp8ws.cu).
 #pragma once
 
 #include "common.cuh"
@@ -13,6 +17,7 @@ namespace fp8ws {
 
 constexpr int kEwThreads = 256;  // threads per block of the streaming kernels
 constexpr int kEwUnroll = 4;     // 16-byte vectors in flight per thread and input
+constexpr int kEwWideUnroll = 2; // 32-byte vectors in flight per thread and input (wide form)
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
@@ -31,6 +36,111 @@ __device__ __forceinline__ uint32_t pack4(uint32_t p01, uint32_t p23) {
 // Streaming loads/stores: every byte is touched once.
 __device__ __forceinline__ uint4 ld_stream(const uint4 *p) { return __ldcs(p); }
 __device__ __forceinline__ void st_stream(uint2 *p, uint2 v) { __stcs(p, v); }
+__device__ __forceinline__ void st_stream(uint4 *p, uint4 v) { __stcs(p, v); }
+
+// 32-byte streaming load (the 8 x 32-bit vector form of ld.global on
+// sm_100): 16 BF16 values, the first 8 in lo.  p must be 32-byte aligned.
+__device__ __forceinline__ void ld_stream_wide(const uint16_t *p, uint4 &lo, uint4 &hi) {
+  asm volatile("ld.global.cs.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y),
+                 "=r"(hi.z), "=r"(hi.w)
+               : "l"(p));
+}
+
+__device__ __forceinline__ uint4 join(uint2 a, uint2 b) { return make_uint4(a.x, a.y, b.x, b.y); }
+
+// The streaming loops.  Threads tid = 0 .. nthreads - 1 of a range visit its
+// vectors with a stride of nthreads, kEwUnroll (kEwWideUnroll) vectors per
+// input in flight; op8(v...) maps 8 BF16 values per input to 8 codes.  The
+// return value is the number of leading elements covered by whole vectors; the
+// caller finishes the rest (fewer than 16) one element per thread.
+template <bool WIDE, typename Op8>
+__device__ __forceinline__ int64_t stream1(const uint16_t *__restrict__ x, int64_t numel,
+                                           uint8_t *__restrict__ out, int64_t tid,
+                                           int64_t nthreads, Op8 op8) {
+  if constexpr (WIDE) {
+    const int64_t nw = numel >> 4;
+    uint4 *ov = reinterpret_cast<uint4 *>(out);
+    int64_t i = tid;
+    for (; i + (kEwWideUnroll - 1) * nthreads < nw; i += kEwWideUnroll * nthreads) {
+      uint4 lo[kEwWideUnroll], hi[kEwWideUnroll];
+#pragma unroll
+      for (int k = 0; k < kEwWideUnroll; ++k)
+        ld_stream_wide(x + (i + k * nthreads) * 16, lo[k], hi[k]);
+#pragma unroll
+      for (int k = 0; k < kEwWideUnroll; ++k)
+        st_stream(ov + i + k * nthreads, join(op8(lo[k]), op8(hi[k])));
+    }
+    for (; i < nw; i += nthreads) {
+      uint4 lo, hi;
+      ld_stream_wide(x + i * 16, lo, hi);
+      st_stream(ov + i, join(op8(lo), op8(hi)));
+    }
+    return nw << 4;
+  } else {
+    const int64_t nvec = numel >> 3;
+    const uint4 *xv = reinterpret_cast<const uint4 *>(x);
+    uint2 *ov = reinterpret_cast<uint2 *>(out);
+    int64_t i = tid;
+    for (; i + (kEwUnroll - 1) * nthreads < nvec; i += kEwUnroll * nthreads) {
+      uint4 v[kEwUnroll];
+#pragma unroll
+      for (int k = 0; k < kEwUnroll; ++k) v[k] = ld_stream(xv + i + k * nthreads);
+#pragma unroll
+      for (int k = 0; k < kEwUnroll; ++k) st_stream(ov + i + k * nthreads, op8(v[k]));
+    }
+    for (; i < nvec; i += nthreads) st_stream(ov + i, op8(ld_stream(xv + i)));
+    return nvec << 3;
+  }
+}
+
+template <bool WIDE, typename Op8>
+__device__ __forceinline__ int64_t stream2(const uint16_t *__restrict__ a,
+                                           const uint16_t *__restrict__ b, int64_t numel,
+                                           uint8_t *__restrict__ out, int64_t tid,
+                                           int64_t nthreads, Op8 op8) {
+  if constexpr (WIDE) {
+    const int64_t nw = numel >> 4;
+    uint4 *ov = reinterpret_cast<uint4 *>(out);
+    int64_t i = tid;
+    for (; i + (kEwWideUnroll - 1) * nthreads < nw; i += kEwWideUnroll * nthreads) {
+      uint4 a0[kEwWideUnroll], a1[kEwWideUnroll], b0[kEwWideUnroll], b1[kEwWideUnroll];
+#pragma unroll
+      for (int k = 0; k < kEwWideUnroll; ++k) {
+        ld_stream_wide(a + (i + k * nthreads) * 16, a0[k], a1[k]);
+        ld_stream_wide(b + (i + k * nthreads) * 16, b0[k], b1[k]);
+      }
+#pragma unroll
+      for (int k = 0; k < kEwWideUnroll; ++k)
+        st_stream(ov + i + k * nthreads, join(op8(a0[k], b0[k]), op8(a1[k], b1[k])));
+    }
+    for (; i < nw; i += nthreads) {
+      uint4 a0, a1, b0, b1;
+      ld_stream_wide(a + i * 16, a0, a1);
+      ld_stream_wide(b + i * 16, b0, b1);
+      st_stream(ov + i, join(op8(a0, b0), op8(a1, b1)));
+    }
+    return nw << 4;
+  } else {
+    const int64_t nvec = numel >> 3;
+    const uint4 *av = reinterpret_cast<const uint4 *>(a);
+    const uint4 *bv = reinterpret_cast<const uint4 *>(b);
+    uint2 *ov = reinterpret_cast<uint2 *>(out);
+    int64_t i = tid;
+    for (; i + (kEwUnroll - 1) * nthreads < nvec; i += kEwUnroll * nthreads) {
+      uint4 va[kEwUnroll], vb[kEwUnroll];
+#pragma unroll
+      for (int k = 0; k < kEwUnroll; ++k) {
+        va[k] = ld_stream(av + i + k * nthreads);
+        vb[k] = ld_stream(bv + i + k * nthreads);
+      }
+#pragma unroll
+      for (int k = 0; k < kEwUnroll; ++k) st_stream(ov + i + k * nthreads, op8(va[k], vb[k]));
+    }
+    for (; i < nvec; i += nthreads) st_stream(ov + i, op8(ld_stream(av + i), ld_stream(bv + i)));
+    return nvec << 3;
+  }
+}
 
 // ------------------------------------------------------------- quantize
 // q = E4M3_satRNE(fl32(x / s)), the code of the IEEE fp32 quotient.
@@ -78,6 +188,7 @@ __device__ __forceinline__ uint2 quant8(uint4 v, float s, float r) {
 // counters of the GEMMs that follow on the stream).
 // The blocks block0 .. block0 + nblocks - 1 of a launch quantize x, each
 // vector visited by one thread with a stride of the blocks' thread count.
+template <bool WIDE>
 __device__ __forceinline__ void quant_static_range(const uint16_t *__restrict__ x, int64_t numel,
                                                    const float *__restrict__ s_in,
                                                    uint8_t *__restrict__ xq, int block,
@@ -85,27 +196,18 @@ __device__ __forceinline__ void quant_static_range(const uint16_t *__restrict__ 
   if (numel <= 0) return;
   const float s = __ldg(s_in);
   const float r = __frcp_rn(s);
-  const int64_t nvec = numel >> 3;
-  const uint4 *xv = reinterpret_cast<const uint4 *>(x);
-  uint2 *qv = reinterpret_cast<uint2 *>(xq);
   const int64_t tid = static_cast<int64_t>(block) * blockDim.x + threadIdx.x;
-  const int64_t stride = static_cast<int64_t>(nblocks) * blockDim.x;
-  int64_t i = tid;
-  for (; i + (kEwUnroll - 1) * stride < nvec; i += kEwUnroll * stride) {
-    uint4 v[kEwUnroll];
-#pragma unroll
-    for (int u = 0; u < kEwUnroll; ++u) v[u] = ld_stream(xv + i + u * stride);
-#pragma unroll
-    for (int u = 0; u < kEwUnroll; ++u) st_stream(qv + i + u * stride, quant8(v[u], s, r));
-  }
-  for (; i < nvec; i += stride) st_stream(qv + i, quant8(ld_stream(xv + i), s, r));
-  const int64_t t = (nvec << 3) + tid;
+  const int64_t nthreads = static_cast<int64_t>(nblocks) * blockDim.x;
+  const int64_t done =
+      stream1<WIDE>(x, numel, xq, tid, nthreads, [s, r](uint4 v) { return quant8(v, s, r); });
+  const int64_t t = done + tid;
   if (t < numel) {
     float a = __uint_as_float(static_cast<uint32_t>(x[t]) << 16);
     xq[t] = static_cast<uint8_t>(quant1(a, s, r));
   }
 }
 
+template <bool WIDE>
 __global__ void __launch_bounds__(kEwThreads) quant_static_kernel(
     const uint16_t *__restrict__ x, int64_t numel, const float *__restrict__ s_in,
     uint8_t *__restrict__ xq, int *__restrict__ zero_words, int n_zero) {
@@ -113,7 +215,7 @@ __global__ void __launch_bounds__(kEwThreads) quant_static_kernel(
   pdl_wait();
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero_words[i] = 0;
-  quant_static_range(x, numel, s_in, xq, blockIdx.x, gridDim.x);
+  quant_static_range<WIDE>(x, numel, s_in, xq, blockIdx.x, gridDim.x);
 }
 
 // Two activations, each with its own scale, quantized by one launch (the two
@@ -127,6 +229,7 @@ struct QuantSeg {
   uint8_t *xq;
 };
 
+template <bool WIDE>
 __global__ void __launch_bounds__(kEwThreads)
     quant_static_pair_kernel(const QuantSeg a, const QuantSeg b, int split,
                              int *__restrict__ zero_words, int n_zero) {
@@ -135,9 +238,9 @@ __global__ void __launch_bounds__(kEwThreads)
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero_words[i] = 0;
   if (static_cast<int>(blockIdx.x) < split)
-    quant_static_range(a.x, a.numel, a.s_in, a.xq, blockIdx.x, split);
+    quant_static_range<WIDE>(a.x, a.numel, a.s_in, a.xq, blockIdx.x, split);
   else
-    quant_static_range(b.x, b.numel, b.s_in, b.xq, blockIdx.x - split, gridDim.x - split);
+    quant_static_range<WIDE>(b.x, b.numel, b.s_in, b.xq, blockIdx.x - split, gridDim.x - split);
 }
 
 // ------------------------------------------------------ SwiGLU -> FP8
@@ -197,33 +300,19 @@ __device__ __forceinline__ uint2 swiglu_quant8(uint4 g, uint4 u, float inv_s,
   return o;
 }
 
+template <bool WIDE>
 __global__ void __launch_bounds__(kEwThreads) swiglu_2in_kernel(
     const uint16_t *__restrict__ g, const uint16_t *__restrict__ u, int64_t numel,
     const float *__restrict__ s_down, SwigluParams p, uint8_t *__restrict__ h) {
   pdl_launch_dependents();
   pdl_wait();
   const float inv_s = __frcp_rn(__ldg(s_down));
-  const int64_t nvec = numel >> 3;
-  const uint4 *gv = reinterpret_cast<const uint4 *>(g);
-  const uint4 *uv = reinterpret_cast<const uint4 *>(u);
-  uint2 *hv = reinterpret_cast<uint2 *>(h);
   const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  int64_t i = tid;
-  for (; i + (kEwUnroll - 1) * stride < nvec; i += kEwUnroll * stride) {
-    uint4 a[kEwUnroll], b[kEwUnroll];
-#pragma unroll
-    for (int k = 0; k < kEwUnroll; ++k) {
-      a[k] = ld_stream(gv + i + k * stride);
-      b[k] = ld_stream(uv + i + k * stride);
-    }
-#pragma unroll
-    for (int k = 0; k < kEwUnroll; ++k)
-      st_stream(hv + i + k * stride, swiglu_quant8(a[k], b[k], inv_s, p));
-  }
-  for (; i < nvec; i += stride)
-    st_stream(hv + i, swiglu_quant8(ld_stream(gv + i), ld_stream(uv + i), inv_s, p));
-  const int64_t t = (nvec << 3) + tid;
+  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t done = stream2<WIDE>(g, u, numel, h, tid, nthreads, [inv_s, p](uint4 a, uint4 b) {
+    return swiglu_quant8(a, b, inv_s, p);
+  });
+  const int64_t t = done + tid;
   if (t < numel) {
     float a = __uint_as_float(static_cast<uint32_t>(g[t]) << 16);
     float b = __uint_as_float(static_cast<uint32_t>(u[t]) << 16);
@@ -245,31 +334,19 @@ __device__ __forceinline__ uint2 silu_mul_quant8(uint4 g, uint4 u, float inv_s) 
   return o;
 }
 
+template <bool WIDE>
 __global__ void __launch_bounds__(kEwThreads) silu_mul_2in_kernel(
     const uint16_t *__restrict__ g, const uint16_t *__restrict__ u, int64_t numel,
     const float *__restrict__ s_down, uint8_t *__restrict__ h) {
   pdl_launch_dependents();
   pdl_wait();
   const float inv_s = __frcp_rn(__ldg(s_down));
-  const int64_t nvec = numel >> 3;
-  const uint4 *gv = reinterpret_cast<const uint4 *>(g);
-  const uint4 *uv = reinterpret_cast<const uint4 *>(u);
-  uint2 *hv = reinterpret_cast<uint2 *>(h);
   const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  int64_t i = tid;
-  for (; i + (kEwUnroll - 1) * stride < nvec; i += kEwUnroll * stride) {
-    uint4 a[kEwUnroll], b[kEwUnroll];
-#pragma unroll
-    for (int k = 0; k < kEwUnroll; ++k) {
-      a[k] = ld_stream(gv + i + k * stride);
-      b[k] = ld_stream(uv + i + k * stride);
-    }
-#pragma unroll
-    for (int k = 0; k < kEwUnroll; ++k) st_stream(hv + i + k * stride, silu_mul_quant8(a[k], b[k], inv_s));
-  }
-  for (; i < nvec; i += stride) st_stream(hv + i, silu_mul_quant8(ld_stream(gv + i), ld_stream(uv + i), inv_s));
-  const int64_t t = (nvec << 3) + tid;
+  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t done = stream2<WIDE>(g, u, numel, h, tid, nthreads, [inv_s](uint4 a, uint4 b) {
+    return silu_mul_quant8(a, b, inv_s);
+  });
+  const int64_t t = done + tid;
   if (t < numel) {
     float a = __uint_as_float(static_cast<uint32_t>(g[t]) << 16);
     float b = __uint_as_float(static_cast<uint32_t>(u[t]) << 16);
