@@ -922,8 +922,11 @@ def aggregate_value(tokens_per_rank: int, world: int, max_seconds: float) -> flo
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=40)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default 40 for the pass; 50 launches for --kernel/--sweep)")
+    ap.add_argument("--warmup", type=int, default=None,
+                    help="untimed warm-up steps (default 3 for the pass; 10 launches for "
+                         "--kernel/--sweep)")
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--no-e2e", action="store_true")
@@ -952,6 +955,11 @@ def main():
                     help="with --kernel/--sweep: also run each kernel back to back for this many "
                          "seconds and report the power-capped rate")
     args = ap.parse_args()
+    single = bool(args.kernel or args.sweep)
+    if args.steps is None:
+        args.steps = 50 if single else 40
+    if args.warmup is None:
+        args.warmup = 10 if single else 3
     log = lambda m: print(m, file=sys.stderr, flush=True)  # noqa: E731
 
     if args.kernel or args.sweep:
