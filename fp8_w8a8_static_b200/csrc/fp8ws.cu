@@ -350,6 +350,13 @@ PairGroup make_pair_group(const PairProblem *pp, int np, int tile_m, int tile_n)
     G.N[p] = q.N;
     G.num_m[p] = (q.M + tile_m - 1) / tile_m;
     G.num_n[p] = (q.N + tile_n - 1) / tile_n;
+    // Tile order.  When A (M x K) is larger than B (N x K; both weights for
+    // the gate/up kernel), the tiles run row by row: a wave sweeps every
+    // column of a few row blocks, so each A row block leaves DRAM once and B,
+    // the smaller operand, is re-read from L2.  Otherwise they run column by
+    // column within groups of kGroupM row blocks: each B column block is read
+    // once per group and A is re-read from L2.
+    G.group_m[p] = q.M > static_cast<int64_t>(q.N) * (q.b2 ? 2 : 1) ? 1 : kGroupM;
     G.s_in[p] = q.s_in;
     G.s_w[p] = q.s_w;
     G.s_w2[p] = q.s_w2;

@@ -41,6 +41,7 @@ struct PairGroup {
   int N[kMaxGroup];
   int num_m[kMaxGroup];
   int num_n[kMaxGroup];
+  int group_m[kMaxGroup];  // raster: row blocks per column-major group (1 = row-major)
   const float *s_in[kMaxGroup];
   const float *s_w[kMaxGroup];
   const float *s_w2[kMaxGroup];
@@ -62,7 +63,8 @@ __device__ __forceinline__ T pick(const T (&a)[kMaxGroup], int p) {
 
 __device__ __forceinline__ GroupTile group_tile(int g, const PairGroup &G) {
   const int p = (g >= G.tile_start[1]) + (g >= G.tile_start[2]);
-  return GroupTile{p, tile_coord(g - pick(G.tile_start, p), pick(G.num_m, p), pick(G.num_n, p))};
+  return GroupTile{p, tile_coord(g - pick(G.tile_start, p), pick(G.num_m, p), pick(G.num_n, p),
+                                 pick(G.group_m, p))};
 }
 
 // Split-K of the remainder tiles.  Units 0 .. dp_tiles-1 are whole tiles (the

@@ -51,11 +51,14 @@ struct TileCoord {
   int m, n;
 };
 
-__device__ __forceinline__ TileCoord tile_coord(int t, int num_m, int num_n) {
-  const int per_group = kGroupM * num_n;
+// Tile t of a num_m x num_n grid: column by column within groups of group_m
+// row blocks (group_m = 1: row by row).
+__device__ __forceinline__ TileCoord tile_coord(int t, int num_m, int num_n,
+                                                int group_m = kGroupM) {
+  const int per_group = group_m * num_n;
   const int group = t / per_group;
-  const int first_m = group * kGroupM;
-  const int gsize = min(num_m - first_m, kGroupM);
+  const int first_m = group * group_m;
+  const int gsize = min(num_m - first_m, group_m);
   const int r = t - group * per_group;
   return TileCoord{first_m + r % gsize, r / gsize};
 }
