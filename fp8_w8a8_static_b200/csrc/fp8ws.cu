@@ -296,9 +296,15 @@ int *splitk_counters(void *splitk) {
 // Remainder tiles (those past the last full wave) split over S K ranges, S in
 // 1..4 minimising waves-of-units x (1/S) of a tile's time, with at most two
 // waves of units and at least two K steps per range.  No scratch: no split.
+// A split pays only when it takes enough K steps off the critical path to cover
+// its fixed cost (the fp32 partial stores, the wait for the last split, its
+// reduction).  Timed on B200: splitting the ragged wave 4 ways saved 9 us at
+// K = 12288 (96 K steps per tile) and cost 6 us at K = 3072 (24 K steps).
+constexpr int kSplitkMinKb = 64;
+
 SplitPlan make_split_plan(int tiles, int pairs, int num_kb, float *partials, int *counters) {
   SplitPlan p{tiles, 0, 1, num_kb, nullptr, nullptr};
-  if (!partials || pairs < 1 || tiles % pairs == 0) return p;
+  if (!partials || pairs < 1 || tiles % pairs == 0 || num_kb < kSplitkMinKb) return p;
   const int R = tiles % pairs;
   if (R > kSplitkTiles) return p;
   int best_s = 1;

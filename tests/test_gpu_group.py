@@ -111,7 +111,8 @@ def test_linear_group_auto_config():
         _check_gemm(ys[p], xq[p], wq[p], oracle.f32(0.01), oracle.f32(0.002))
 
 
-@pytest.mark.parametrize("M0,M1,N,K", [(4096, 1024, 3072, 12288), (300, 520, 264, 1040)])
+@pytest.mark.parametrize("M0,M1,N,K", [(4096, 1024, 3072, 12288), (300, 520, 264, 8208),
+                                       (300, 520, 264, 1040)])
 def test_linear_group_split_k(M0, M1, N, K):
     rng = np.random.default_rng(M0 + M1)
     xq = [_random_codes(rng, (M, K)) for M in (M0, M1)]

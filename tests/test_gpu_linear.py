@@ -110,8 +110,9 @@ def test_linear_sweep_full_size(M, N):
 @pytest.mark.parametrize("M,N,K", [
     (1024, 3072, 12288),   # understanding-tower down projection: 48 tiles, all split
     (4096, 3072, 12288),   # generation-tower down projection: 2 full waves + 44 split tiles
-    (2048, 1024, 3072),    # K/V projection shape
-    (300, 520, 1040),      # ragged, 9 K steps (a 4-way split would leave one empty)
+    (300, 520, 8208),      # ragged M, N and K (65 K steps, the last partial): split 4 ways
+    (2048, 1024, 3072),    # K/V projection shape: 24 K steps, too few to split
+    (300, 520, 1040),      # ragged, 9 K steps: not split
     (64, 256, 704),
 ])
 def test_split_k_against_oracle(M, N, K):

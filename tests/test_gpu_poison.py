@@ -54,7 +54,7 @@ def test_quant_and_linear(M, N, K, gemm_config):
     _assert_written(xq, y)
 
 
-@pytest.mark.parametrize("M,N,K", SHAPES)
+@pytest.mark.parametrize("M,N,K", SHAPES + [(300, 520, 8208)])  # the last: long enough to split
 def test_linear_split_k_and_group(M, N, K):
     x = synth.normal((M, K), 1.0, M + 2 * K, DEV)
     xq = fw.fp8_quant_static(x, scalar(0.01, DEV))
