@@ -135,6 +135,28 @@ def test_split_k_against_oracle(M, N, K):
     assert fw.device_status()[0] == fw.OK
 
 
+@pytest.mark.parametrize("split", [False, True])
+def test_long_k(split):
+    """K = 65536, 512 K steps per tile: the K coordinates and, with the
+    workspace, a 4-way split at the far end of the allowed range.  The oracle's
+    fp64 sum stays exact (448^2 * 2^16 < 2^35 at a granularity of 2^-18)."""
+    M, N, K = 300, 264, 65536
+    rng = np.random.default_rng(K)
+    xq = _random_codes(rng, (M, K))
+    wq = _random_codes(rng, (N, K), 0.5)
+    s_in, s_w = oracle.f32(0.013), oracle.f32(0.0021)
+    args = (from_codes(xq, DEV), from_codes(wq, DEV), scalar(s_in, DEV), scalar(s_w, DEV))
+    y = fw.fp8_linear_static_ws(*args) if split else fw.fp8_linear_static(*args)
+    rows = np.random.default_rng(5).choice(M, 16, replace=False)
+    yb = bits(y)[rows]
+    xr = np.ascontiguousarray(xq[rows])
+    ref = oracle.linear(xr, wq, s_in, s_w)
+    absref = oracle.linear(xr & 0x7F, wq & 0x7F, s_in, s_w)
+    assert rel_fro(yb, ref) <= GEMM_REL_FRO
+    assert gemm_elementwise_bound_ok(yb, ref, absref, K).all()
+    assert fw.device_status()[0] == fw.OK
+
+
 def test_split_k_short_workspace_refused():
     xq = torch.zeros((256, 256), dtype=fw.FP8, device=DEV)
     ws = torch.empty(1024, dtype=torch.uint8, device=DEV)
