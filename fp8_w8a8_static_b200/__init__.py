@@ -37,6 +37,7 @@ __all__ = [
     "fp8_check_shared_input_scale", "fp8_absmax_bf16", "fp8_silu_mul_absmax",
     "fp8_observer_scale", "fp8_rtn_quantize_weight",
     "device_check", "device_status", "launch_count", "launch_log", "launch_log_clear",
+    "split_plan",
     "selftest_bounded_wait", "SITE_SELFTEST",
     "FP8", "OBSERVER_CONSTANT", "EXPORTED_SYMBOLS",
 ]
@@ -167,6 +168,8 @@ _SIGS = {
     "fp8ws_set_gemm_config": (ctypes.c_int, [ctypes.c_int]),
     "fp8ws_selftest_bounded_wait": (ctypes.c_int, [_I64, ctypes.c_int,
                                                    ctypes.POINTER(ctypes.c_int64), _P]),
+    "fp8ws_split_plan": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int]
+                         + [ctypes.POINTER(ctypes.c_int)] * 4),
     "fp8ws_launch_count": (ctypes.c_int64, []),
     "fp8ws_launch_log": (ctypes.c_int, [ctypes.POINTER(LaunchRecord), ctypes.c_int]),
     "fp8ws_launch_log_clear": (None, []),
@@ -823,6 +826,15 @@ def selftest_bounded_wait(limit_ns: int, mode: int = 0, stream=None) -> int:
 def set_gemm_config(name: str = "auto") -> None:
     """Force a GEMM tile configuration (see GEMM_CONFIGS); "auto" = cost model."""
     _check(load().fp8ws_set_gemm_config(GEMM_CONFIGS[name]), "fp8ws_set_gemm_config")
+
+
+def split_plan(tiles: int, pairs: int, num_kb: int) -> dict:
+    """The CTA-pair GEMM's split-K plan (host only): dp_tiles whole tiles, then
+    split_tiles tiles cut into `splits` K ranges of kb_per_split steps."""
+    out = [ctypes.c_int() for _ in range(4)]
+    _check(load().fp8ws_split_plan(tiles, pairs, num_kb, *[ctypes.byref(o) for o in out]),
+           "fp8ws_split_plan")
+    return dict(zip(("dp_tiles", "split_tiles", "splits", "kb_per_split"), (o.value for o in out)))
 
 
 def launch_count() -> int:

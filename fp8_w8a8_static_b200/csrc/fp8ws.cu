@@ -1428,6 +1428,20 @@ int fp8ws_set_gemm_config(int config) {
   return FP8WS_OK;
 }
 
+int fp8ws_split_plan(int tiles, int pairs, int num_kb, int *dp_tiles, int *split_tiles,
+                     int *splits, int *kb_per_split) {
+  if (!dp_tiles || !split_tiles || !splits || !kb_per_split) return FP8WS_ERR_NULL;
+  if (tiles < 0 || pairs < 1 || num_kb < 1) return FP8WS_ERR_SHAPE;
+  // the plan only needs to know that scratch exists; it is not dereferenced here
+  float scratch_tag = 0.0f;
+  const SplitPlan p = make_split_plan(tiles, pairs, num_kb, &scratch_tag, nullptr);
+  *dp_tiles = p.dp_tiles;
+  *split_tiles = p.split_tiles;
+  *splits = p.splits;
+  *kb_per_split = p.kb_per_split;
+  return FP8WS_OK;
+}
+
 int64_t fp8ws_launch_count(void) {
   std::lock_guard<std::mutex> lk(g_log_mu);
   return g_launch_total;

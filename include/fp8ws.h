@@ -557,6 +557,17 @@ FP8WS_API int fp8ws_selftest_bounded_wait(int64_t limit_ns, int mode, int64_t *e
  * FP8WS_ERR_SHAPE for other values. */
 FP8WS_API int fp8ws_set_gemm_config(int config);
 
+/* The split-K plan of the CTA-pair GEMM (fp8_linear_static_ws and the
+ * grouped projection GEMMs that receive split-K scratch), for tests and
+ * tuning; host only, touches no device.  For `tiles` 256x256 tiles on `pairs`
+ * resident CTA pairs with `num_kb` 128-byte K steps per tile: the first
+ * *dp_tiles tiles run whole, and the last *split_tiles are each cut into
+ * *splits K ranges of *kb_per_split steps (*splits == 1: no split).  Tiles of
+ * fewer than 64 K steps are never split.  FP8WS_ERR_NULL for a NULL output,
+ * FP8WS_ERR_SHAPE for tiles < 0, pairs < 1 or num_kb < 1. */
+FP8WS_API int fp8ws_split_plan(int tiles, int pairs, int num_kb, int *dp_tiles, int *split_tiles,
+                               int *splits, int *kb_per_split);
+
 /* Launch log.  Every kernel the library enqueues is counted and recorded in a
  * small ring (the most recent FP8WS_LOG_CAPACITY records).  kind: 1 quant,
  * 2 GEMM, 3 SwiGLU-quant, 4 calibration, 5 fused gate/up SwiGLU-quant.

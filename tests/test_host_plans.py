@@ -1,0 +1,70 @@
+"""Host logic of the CTA-pair GEMM's split-K plan, on the CPU (no device is
+touched): the decisions for the workloads' shapes, and the invariants every
+plan keeps (the split ranges cover K with none empty, only the ragged last
+wave is split, the scratch slots and counters suffice)."""
+
+import ctypes
+
+import pytest
+
+import fp8_w8a8_static_b200 as fw
+
+PAIRS = 74  # CTA pairs resident at once on a 148-SM B200
+
+
+def test_two_tower_down_projection():
+    """Both towers' down projections (192 + 48 tiles, K = 12288): three full
+    waves, then the 18 remaining tiles split four ways."""
+    assert fw.split_plan(240, PAIRS, 96) == dict(dp_tiles=222, split_tiles=18, splits=4,
+                                                 kb_per_split=24)
+
+
+def test_short_k_is_not_split():
+    """The shared-quant Q/K/V launch (160 tiles, K = 3072, 24 K steps): no split."""
+    assert fw.split_plan(160, PAIRS, 24) == dict(dp_tiles=160, split_tiles=0, splits=1,
+                                                 kb_per_split=24)
+
+
+def test_threshold_at_64_k_steps():
+    assert fw.split_plan(10, PAIRS, 63)["splits"] == 1
+    assert fw.split_plan(10, PAIRS, 64)["splits"] > 1
+
+
+def test_ragged_k_case_of_the_gpu_tests():
+    """M=300, N=520, K=8208: 6 tiles, 65 K steps (the last one partial)."""
+    assert fw.split_plan(6, PAIRS, 65) == dict(dp_tiles=0, split_tiles=6, splits=4,
+                                               kb_per_split=17)
+
+
+def test_full_waves_are_not_split():
+    for waves in (1, 2, 3):
+        p = fw.split_plan(waves * PAIRS, PAIRS, 96)
+        assert p["splits"] == 1 and p["dp_tiles"] == waves * PAIRS
+
+
+@pytest.mark.parametrize("pairs", [1, 2, 37, PAIRS])
+def test_plan_invariants(pairs):
+    for tiles in range(0, 400, 7):
+        for num_kb in (1, 2, 9, 24, 63, 64, 65, 96, 97, 512):
+            p = fw.split_plan(tiles, pairs, num_kb)
+            dp, st, s, kbs = p["dp_tiles"], p["split_tiles"], p["splits"], p["kb_per_split"]
+            assert dp + st == tiles and 1 <= s <= 4
+            if s == 1:
+                assert st == 0 and kbs == num_kb
+                continue
+            assert num_kb >= 64
+            assert dp % pairs == 0 and st == tiles % pairs    # only the ragged last wave
+            assert (s - 1) * kbs < num_kb <= s * kbs           # covers K, no empty range
+            assert kbs >= 2
+            assert st * s <= min(2 * pairs, 148)               # scratch slots
+            assert st <= 128                                   # split-K counters
+
+
+def test_argument_errors():
+    lib = fw.load()
+    out = [ctypes.c_int() for _ in range(4)]
+    refs = [ctypes.byref(o) for o in out]
+    assert lib.fp8ws_split_plan(10, PAIRS, 96, None, *refs[1:]) == fw.ERR_NULL
+    assert lib.fp8ws_split_plan(-1, PAIRS, 96, *refs) == fw.ERR_SHAPE
+    assert lib.fp8ws_split_plan(10, 0, 96, *refs) == fw.ERR_SHAPE
+    assert lib.fp8ws_split_plan(10, PAIRS, 0, *refs) == fw.ERR_SHAPE
