@@ -37,7 +37,7 @@ __all__ = [
     "fp8_check_shared_input_scale", "fp8_absmax_bf16", "fp8_silu_mul_absmax",
     "fp8_observer_scale", "fp8_rtn_quantize_weight",
     "device_check", "device_status", "launch_count", "launch_log", "launch_log_clear",
-    "split_plan",
+    "split_plan", "gemm_plan",
     "selftest_bounded_wait", "SITE_SELFTEST",
     "FP8", "OBSERVER_CONSTANT", "EXPORTED_SYMBOLS",
 ]
@@ -168,6 +168,9 @@ _SIGS = {
     "fp8ws_set_gemm_config": (ctypes.c_int, [ctypes.c_int]),
     "fp8ws_selftest_bounded_wait": (ctypes.c_int, [_I64, ctypes.c_int,
                                                    ctypes.POINTER(ctypes.c_int64), _P]),
+    "fp8ws_gemm_plan": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int64),
+                                       ctypes.POINTER(ctypes.c_int64), ctypes.c_int,
+                                       ctypes.POINTER(ctypes.c_int)]),
     "fp8ws_split_plan": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int]
                          + [ctypes.POINTER(ctypes.c_int)] * 4),
     "fp8ws_launch_count": (ctypes.c_int64, []),
@@ -826,6 +829,17 @@ def selftest_bounded_wait(limit_ns: int, mode: int = 0, stream=None) -> int:
 def set_gemm_config(name: str = "auto") -> None:
     """Force a GEMM tile configuration (see GEMM_CONFIGS); "auto" = cost model."""
     _check(load().fp8ws_set_gemm_config(GEMM_CONFIGS[name]), "fp8ws_set_gemm_config")
+
+
+def gemm_plan(shapes, sms: int = 148, pairs: int = 74) -> str:
+    """The tile configuration the cost model picks for [(M, N), ...] (host
+    only): one of the GEMM_CONFIGS names other than "auto"."""
+    n = len(shapes)
+    M = (ctypes.c_int64 * n)(*[m for m, _ in shapes])
+    N = (ctypes.c_int64 * n)(*[c for _, c in shapes])
+    cfg = ctypes.c_int()
+    _check(load().fp8ws_gemm_plan(sms, pairs, M, N, n, ctypes.byref(cfg)), "fp8ws_gemm_plan")
+    return {v: k for k, v in GEMM_CONFIGS.items()}[cfg.value]
 
 
 def split_plan(tiles: int, pairs: int, num_kb: int) -> dict:

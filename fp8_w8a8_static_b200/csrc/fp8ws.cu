@@ -550,11 +550,10 @@ std::atomic<int> g_forced_gemm_config{0};  // fp8ws_set_gemm_config: 0 = cost mo
 
 // 1 = CTA pair 256 x 256, 2 = one CTA 128 x 256, 3 = 128 x 128, 4 = 128 x 64,
 // for the np problems M[p] x N[p] that one launch would cover.
-int gemm_choice(const DeviceInfo *d, const int64_t *M, const int64_t *N, int np) {
-  const int forced = g_forced_gemm_config.load(std::memory_order_relaxed);
-  if (forced) return forced;
-  const int resident = d->pair_clusters.load(std::memory_order_relaxed);
-  const int pairs = resident > 0 ? resident : d->sms / 2;
+// The cost model alone: the configuration (1 CTA pairs, 2/3/4 one CTA with
+// 128x256, 128x128, 128x64 tiles) for np problems on `sms` SMs holding `pairs`
+// CTA pairs at once.
+int gemm_cost_choice(int sms, int pairs, const int64_t *M, const int64_t *N, int np) {
   auto waves = [](int64_t tiles, int64_t slots) { return (tiles + slots - 1) / slots; };
   int64_t t_pair = 0, t_256 = 0, t_128 = 0, t_64 = 0;
   for (int p = 0; p < np; ++p) {
@@ -565,14 +564,21 @@ int gemm_choice(const DeviceInfo *d, const int64_t *M, const int64_t *N, int np)
     t_64 += m128 * ((N[p] + 63) / 64);
   }
   const double est_pair = waves(t_pair, pairs) * (128.0 * 256) / 1.0;
-  const double est_256 = waves(t_256, d->sms) * (128.0 * 256) / 0.85;
-  const double est_128 = waves(t_128, d->sms) * (128.0 * 128) / 0.45;
-  const double est_64 = waves(t_64, d->sms) * (128.0 * 64) / 0.25;
+  const double est_256 = waves(t_256, sms) * (128.0 * 256) / 0.85;
+  const double est_128 = waves(t_128, sms) * (128.0 * 128) / 0.45;
+  const double est_64 = waves(t_64, sms) * (128.0 * 64) / 0.25;
   const double best = fmin(fmin(est_pair, est_256), fmin(est_128, est_64));
   if (est_pair == best) return 1;
   if (est_256 == best) return 2;
   if (est_128 == best) return 3;
   return 4;
+}
+
+int gemm_choice(const DeviceInfo *d, const int64_t *M, const int64_t *N, int np) {
+  const int forced = g_forced_gemm_config.load(std::memory_order_relaxed);
+  if (forced) return forced;
+  const int resident = d->pair_clusters.load(std::memory_order_relaxed);
+  return gemm_cost_choice(d->sms, resident > 0 ? resident : d->sms / 2, M, N, np);
 }
 
 int gemm_dispatch(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int64_t M, int64_t N,
@@ -1425,6 +1431,16 @@ int fp8ws_device_status(int *status, int *where) {
 int fp8ws_set_gemm_config(int config) {
   if (config < 0 || config > 4) return FP8WS_ERR_SHAPE;
   g_forced_gemm_config.store(config, std::memory_order_relaxed);
+  return FP8WS_OK;
+}
+
+int fp8ws_gemm_plan(int sms, int pairs, const int64_t *M, const int64_t *N, int count,
+                    int *config) {
+  if (!M || !N || !config) return FP8WS_ERR_NULL;
+  if (sms < 1 || pairs < 1 || count < 1 || count > kMaxGroup) return FP8WS_ERR_SHAPE;
+  for (int p = 0; p < count; ++p)
+    if (M[p] < 0 || N[p] < 1) return FP8WS_ERR_SHAPE;
+  *config = gemm_cost_choice(sms, pairs, M, N, count);
   return FP8WS_OK;
 }
 

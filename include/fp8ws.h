@@ -557,6 +557,17 @@ FP8WS_API int fp8ws_selftest_bounded_wait(int64_t limit_ns, int mode, int64_t *e
  * FP8WS_ERR_SHAPE for other values. */
 FP8WS_API int fp8ws_set_gemm_config(int config);
 
+/* The tile configuration the GEMM cost model picks, for tests and tuning;
+ * host only, touches no device, ignores a configuration forced by
+ * fp8ws_set_gemm_config.  Problems: M[p] x N[p] outputs for p < count (1..3,
+ * the most one launch groups: the projections of one shared quantization), on
+ * a GPU with `sms` SMs holding `pairs` CTA pairs at once.  *config receives
+ * fp8ws_set_gemm_config's numbering: 1 CTA-pair 256x256 tiles, 2/3/4 one CTA
+ * with 128x256, 128x128 or 128x64 tiles.  FP8WS_ERR_NULL for a NULL pointer,
+ * FP8WS_ERR_SHAPE for sms < 1, pairs < 1, count outside 1..3, M < 0 or N < 1. */
+FP8WS_API int fp8ws_gemm_plan(int sms, int pairs, const int64_t *M, const int64_t *N, int count,
+                              int *config);
+
 /* The split-K plan of the CTA-pair GEMM (fp8_linear_static_ws and the
  * grouped projection GEMMs that receive split-K scratch), for tests and
  * tuning; host only, touches no device.  For `tiles` 256x256 tiles on `pairs`

@@ -1,7 +1,8 @@
-"""Host logic of the CTA-pair GEMM's split-K plan, on the CPU (no device is
-touched): the decisions for the workloads' shapes, and the invariants every
-plan keeps (the split ranges cover K with none empty, only the ragged last
-wave is split, the scratch slots and counters suffice)."""
+"""Host logic of the GEMM dispatch, on the CPU (no device is touched): the
+tile configuration the cost model picks, and the CTA-pair GEMM's split-K plan
+(the decisions for the workloads' shapes, and the invariants every plan
+keeps: the split ranges cover K with none empty, only the ragged last wave is
+split, the scratch slots and counters suffice)."""
 
 import ctypes
 
@@ -68,3 +69,43 @@ def test_argument_errors():
     assert lib.fp8ws_split_plan(-1, PAIRS, 96, *refs) == fw.ERR_SHAPE
     assert lib.fp8ws_split_plan(10, 0, 96, *refs) == fw.ERR_SHAPE
     assert lib.fp8ws_split_plan(10, PAIRS, 0, *refs) == fw.ERR_SHAPE
+
+
+# ------------------------------------------------------- GEMM tile choice
+
+
+def test_gemm_plan_workload_shapes_use_cta_pairs():
+    """Every GEMM of the workloads runs on CTA pairs (c0, c1, c3 grouped, c4)."""
+    shapes = [[(64, 704)], [(64, 256)]]
+    shapes += [[(m, n)] for m in (256, 1024, 4096) for n in (2048, 8192)]
+    shapes += [[(2048, 3072), (2048, 1024), (2048, 1024)]]
+    shapes += [[(4096, 12288), (1024, 12288)], [(4096, 3072), (1024, 3072)]]
+    for s in shapes:
+        assert fw.gemm_plan(s) == "pair256", s
+
+
+def test_gemm_plan_one_cta_tiles_when_pairs_need_an_extra_wave():
+    """Model (per-SM output area per wave / efficiency): M=1, N=19008 is 75
+    pair tiles, two waves on 74 pairs: 2 * 128*256 / 1.0 = 65536; as 75 one-CTA
+    128x256 tiles it is one wave on 148 SMs: 128*256 / 0.85 = 38550, the
+    smallest (128x128: 149 tiles, 2 * 16384 / 0.45 = 72818; 128x64: 297 tiles,
+    3 * 8192 / 0.25 = 98304).  At N=18944 (74 pair tiles, one wave) the pair
+    kernel's 32768 wins."""
+    assert fw.gemm_plan([(1, 19008)]) == "cta256"
+    assert fw.gemm_plan([(1, 18944)]) == "pair256"
+
+
+def test_gemm_plan_argument_errors():
+    lib = fw.load()
+    M = (ctypes.c_int64 * 3)(64, 64, 64)
+    N = (ctypes.c_int64 * 3)(256, 256, 256)
+    cfg = ctypes.c_int()
+    assert lib.fp8ws_gemm_plan(148, PAIRS, M, N, 1, None) == fw.ERR_NULL
+    assert lib.fp8ws_gemm_plan(148, PAIRS, None, N, 1, ctypes.byref(cfg)) == fw.ERR_NULL
+    for args in ((0, PAIRS, 1), (148, 0, 1), (148, PAIRS, 0), (148, PAIRS, 4)):
+        sms, pairs, count = args
+        assert lib.fp8ws_gemm_plan(sms, pairs, M, N, count, ctypes.byref(cfg)) == fw.ERR_SHAPE
+    bad = (ctypes.c_int64 * 1)(0)
+    assert lib.fp8ws_gemm_plan(148, PAIRS, M, bad, 1, ctypes.byref(cfg)) == fw.ERR_SHAPE
+    assert lib.fp8ws_gemm_plan(148, PAIRS, M, N, 3, ctypes.byref(cfg)) == fw.OK
+    assert cfg.value == 1
