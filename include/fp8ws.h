@@ -107,15 +107,19 @@ FP8WS_API int fp8_linear_static(const uint8_t *xq, const uint8_t *wq, int64_t M,
  * fp8_linear_static_ws -- fp8_linear_static with a scratch workspace that lets
  * the tiles past the last full wave of CTA pairs be split over K (2..4 ranges,
  * chosen from the shape and the number of resident CTA pairs), so the GPU is
- * not left partly idle by a ragged last wave.  Each split stores an fp32
- * partial in the workspace; the last split of a tile to finish adds the
- * partials in split order (deterministic: the same inputs give the same bits
- * on every call) and applies the epilogue.  The sum may differ from the
- * unsplit kernel's in the last bits of fp32, well inside the GEMM tolerance.
- * It pays only when the tile count is far below one wave and K is long: on
- * the two-tower down projections (48 and 192 tiles of 256 x 256 for 74 CTA
- * pairs, K = 12288) the partial traffic and reduction cost more than the idle
- * tail they remove, so the composite calls do not use it.
+ * not left partly idle by a ragged last wave.  Tiles of fewer than 64 K steps
+ * (K < 8192) are never split: there the split's fixed cost exceeds the time
+ * it saves.  Each split stores an fp32 partial in the workspace; the last
+ * split of a tile to finish adds the partials in split order (deterministic:
+ * the same inputs give the same bits on every call) and applies the epilogue.
+ * The sum may differ from the unsplit kernel's in the last bits of fp32, well
+ * inside the GEMM tolerance.  It pays only when few tiles remain past the last
+ * full wave and K is long: on a single tower's down projection (48 or 192
+ * tiles of 256 x 256 for 74 CTA pairs, K = 12288) the partial traffic and
+ * reduction cost more than the idle tail they remove, so the single-tower
+ * composite calls do not use it; the grouped down projection of both towers
+ * (240 tiles, 18 past the third wave) does.  fp8ws_split_plan reports the
+ * plan for a shape.
  * workspace: device, >= fp8_linear_static_ws_bytes() bytes, 256-byte aligned;
  * overwritten (the call clears its counters first).  Other arguments and
  * errors as fp8_linear_static; FP8WS_ERR_WORKSPACE for a missing, misaligned
