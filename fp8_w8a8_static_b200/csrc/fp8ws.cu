@@ -679,6 +679,21 @@ int silu_launch(DeviceInfo *d, const uint16_t *g, const uint16_t *u, int64_t num
 
 size_t round256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
+// Workspace byte counts are formed in 128 bits from sizes below 2^63 and
+// saturate at SIZE_MAX, so that no shape wraps a count into a small number (a
+// SIZE_MAX workspace cannot be allocated).  ws_region(a, b, c) is one region of
+// a * b * c bytes (c: element size, at most 4) rounded up to 256.
+using u128 = unsigned __int128;
+// Factors are clamped at 2^40 (a region that large saturates anyway), so a
+// sum of a few regions stays far below 2^128.
+u128 ws_region(int64_t a, int64_t b, int c = 1) {
+  const int64_t cap = int64_t(1) << 40;
+  const u128 x = static_cast<u128>(a < cap ? a : cap) * static_cast<u128>(b < cap ? b : cap) *
+                 static_cast<u128>(c);
+  return (x + 255) & ~static_cast<u128>(255);
+}
+size_t ws_saturate(u128 v) { return v > SIZE_MAX ? SIZE_MAX : static_cast<size_t>(v); }
+
 // Self-test of the bounded wait (fp8ws_selftest_bounded_wait): lane 0 of warp 0
 // waits on an mbarrier that nothing arrives at.  Mode 0: the wait runs out
 // after limit_ns and records kSiteSelfTest in the status word.  Mode 1: warp 1
@@ -792,8 +807,7 @@ int swiglu_2in_fp8(const uint16_t *g, const uint16_t *u, int64_t numel, const fl
 
 size_t gated_mlp_static_fp8_workspace(int64_t M, int64_t d, int64_t I) {
   if (M < 0 || d < 0 || I < 0) return 0;
-  const size_t m = static_cast<size_t>(M), dd = static_cast<size_t>(d), ii = static_cast<size_t>(I);
-  return round256(m * dd) + 2 * round256(m * ii * 2) + round256(m * ii);
+  return ws_saturate(ws_region(M, d) + 2 * ws_region(M, I, 2) + ws_region(M, I));
 }
 
 int gated_mlp_static_fp8(const uint16_t *x, int64_t M, int64_t dm, int64_t I, const float *s_in,
@@ -867,8 +881,7 @@ int fp8_gate_up_swiglu_static(const uint8_t *xq, const uint8_t *Wg, const uint8_
 
 size_t gated_mlp_static_fp8_fused_workspace(int64_t M, int64_t d, int64_t I) {
   if (M < 0 || d < 0 || I < 0) return 0;
-  const size_t m = static_cast<size_t>(M);
-  return round256(m * static_cast<size_t>(d)) + round256(m * static_cast<size_t>(I));
+  return ws_saturate(ws_region(M, d) + ws_region(M, I));
 }
 
 int gated_mlp_static_fp8_fused(const uint16_t *x, int64_t M, int64_t dm, int64_t I,
@@ -1006,12 +1019,12 @@ int fp8_gate_up_swiglu_static_group(const fp8ws_gate_up_problem *problems, int c
 
 size_t gated_mlp_static_fp8_group_workspace(const int64_t *M, int count, int64_t d, int64_t I) {
   if (!M || count < 1 || count > FP8WS_MAX_GROUP || d < 0 || I < 0) return 0;
-  size_t total = 0;
+  u128 total = splitk_bytes();
   for (int p = 0; p < count; ++p) {
     if (M[p] < 0) return 0;
-    total += gated_mlp_static_fp8_fused_workspace(M[p], d, I);
+    total += ws_region(M[p], d) + ws_region(M[p], I);
   }
-  return total + splitk_bytes();
+  return ws_saturate(total);
 }
 
 int gated_mlp_static_fp8_group(const fp8ws_mlp_tower *towers, int count, int64_t dm, int64_t I,
@@ -1084,6 +1097,18 @@ namespace {
 std::mutex g_noalloc_mu;
 void *g_noalloc_ptr[fp8ws::kMaxDevices];  // device address per device, looked up once
 
+// Bytes of scratch gated_mlp_static_fp8 would use for this shape, or SIZE_MAX
+// for a shape it refuses (d or I not a positive multiple of 16, or a size of
+// 2^31 or more), checked before the size is formed.  The size itself
+// saturates rather than wraps (gated_mlp_static_fp8_workspace).
+size_t noalloc_bytes(int64_t M, int64_t d, int64_t I) {
+  const int64_t lim = int64_t(1) << 31;
+  if (M < 0 || d < 16 || I < 16 || d % 16 != 0 || I % 16 != 0 || M >= lim || d >= lim ||
+      I >= lim)
+    return SIZE_MAX;
+  return gated_mlp_static_fp8_workspace(M, d, I);
+}
+
 // Device address of the scratch area on the current device; the first call
 // per device looks it up with that device current.
 int noalloc_scratch(void **out) {
@@ -1107,8 +1132,7 @@ int gated_mlp_static_fp8_noalloc(const uint16_t *x, int64_t M, int64_t d, int64_
                                  const float *s_in, const uint8_t *Wg, const float *s_wg,
                                  const uint8_t *Wu, const float *s_wu, const float *s_down,
                                  const uint8_t *Wd, const float *s_wd, uint16_t *y, void *stream) {
-  if (M < 0 || d < 0 || I < 0) return FP8WS_ERR_SHAPE;
-  if (gated_mlp_static_fp8_workspace(M, d, I) > FP8WS_NOALLOC_SCRATCH_BYTES) return FP8WS_ERR_SHAPE;
+  if (noalloc_bytes(M, d, I) > FP8WS_NOALLOC_SCRATCH_BYTES) return FP8WS_ERR_SHAPE;
   void *scratch = nullptr;
   int rc = noalloc_scratch(&scratch);
   if (rc) return rc;
@@ -1118,7 +1142,7 @@ int gated_mlp_static_fp8_noalloc(const uint16_t *x, int64_t M, int64_t d, int64_
 
 size_t fp8_shared_quant_linears_workspace(int64_t M, int64_t d) {
   if (M < 0 || d < 0) return 0;
-  return round256(static_cast<size_t>(M) * static_cast<size_t>(d)) + splitk_bytes();
+  return ws_saturate(ws_region(M, d) + splitk_bytes());
 }
 
 int fp8_shared_quant_linears(const uint16_t *x, int64_t M, int64_t dm, const float *s_in, int n,
@@ -1151,8 +1175,7 @@ int fp8_shared_quant_linears(const uint16_t *x, int64_t M, int64_t dm, const flo
 
 size_t cross_attention_qkv_static_fp8_workspace(int64_t Mq, int64_t Mkv, int64_t d) {
   if (Mq < 0 || Mkv < 0 || d < 0) return 0;
-  return round256(static_cast<size_t>(Mq) * d) + round256(static_cast<size_t>(Mkv) * d) +
-         splitk_bytes();
+  return ws_saturate(ws_region(Mq, d) + ws_region(Mkv, d) + splitk_bytes());
 }
 
 int cross_attention_qkv_static_fp8(const uint16_t *x, int64_t Mq, const uint16_t *ctx,
@@ -1260,9 +1283,8 @@ int silu_mul_2in_fp8_per_token(const uint16_t *g, const uint16_t *u, int64_t row
 
 size_t gated_mlp_per_token_fp8_workspace(int64_t M, int64_t d, int64_t I) {
   if (M < 0 || d < 0 || I < 0) return 0;
-  const size_t m = static_cast<size_t>(M);
-  return round256(m * d) + round256(m * 4) + 2 * round256(m * I * 2) + round256(m * I) +
-         round256(m * 4);
+  return ws_saturate(ws_region(M, d) + ws_region(M, 4) + 2 * ws_region(M, I, 2) +
+                     ws_region(M, I) + ws_region(M, 4));
 }
 
 int gated_mlp_per_token_fp8(const uint16_t *x, int64_t M, int64_t dm, int64_t I,

@@ -26,6 +26,9 @@
  *    rounds to nearest, ties to even.
  *  - Errors found inside a kernel (a bounded wait that ran out) are recorded
  *    in a device status word; fp8ws_device_status() reads and clears it.
+ *  - The *_workspace functions return 0 for a negative size, and SIZE_MAX
+ *    (which cannot be allocated) when the byte count does not fit in size_t:
+ *    the count is formed without wrap-around, so no shape yields a small one.
  *
  * Sources of the operations (the pages this library implements):
  *  [MC] Hugging Face model card "Cosmos3-Nano-Policy-DROID, FP8 + RTN +
@@ -108,8 +111,9 @@ FP8WS_API int fp8_linear_static(const uint8_t *xq, const uint8_t *wq, int64_t M,
  * the tiles past the last full wave of CTA pairs be split over K (2..4 ranges,
  * chosen from the shape and the number of resident CTA pairs), so the GPU is
  * not left partly idle by a ragged last wave.  Tiles of fewer than 64 K steps
- * (K < 8192) are never split: there the split's fixed cost exceeds the time
- * it saves.  Each split stores an fp32 partial in the workspace; the last
+ * of 128 bytes (ceil(K / 128) < 64, i.e. K <= 8064 for the multiples of 16
+ * allowed here) are never split: there the split's fixed cost exceeds the
+ * time it saves.  Each split stores an fp32 partial in the workspace; the last
  * split of a tile to finish adds the partials in split order (deterministic:
  * the same inputs give the same bits on every call) and applies the epilogue.
  * The sum may differ from the unsplit kernel's in the last bits of fp32, well
@@ -388,12 +392,28 @@ FP8WS_API int qkv_shared_quant(const uint16_t *x, int64_t M, int64_t d, const fl
  * cudaMalloc, no cudaFree, no allocating library routine.
  *
  * Limits and behaviour:
- *  - Sizes whose gated_mlp_static_fp8_workspace(M, d, I) exceeds
- *    FP8WS_NOALLOC_SCRATCH_BYTES are refused with FP8WS_ERR_SHAPE before any
- *    launch (for d = 3072, I = 12288 this allows up to M = 1024 rows).
+ *  - The rule is gated_mlp_static_fp8_workspace(M, d, I) <=
+ *    FP8WS_NOALLOC_SCRATCH_BYTES; larger shapes are refused with
+ *    FP8WS_ERR_SHAPE before any launch.  That workspace is
+ *    M * (d + 5 I) bytes, each of its four regions rounded up to 256 bytes,
+ *    so for d = 3072, I = 12288 it allows up to M = 1040 rows (1040 * 64512 =
+ *    67,092,480 bytes).  Shapes gated_mlp_static_fp8 refuses (d or I not a
+ *    positive multiple of 16, a size of 2^31 or more) are refused here with
+ *    FP8WS_ERR_SHAPE too, before the size is formed, so no shape can wrap the
+ *    byte count into the limit.
  *  - The first call on each device looks up the scratch area's device
  *    address on that device (cudaGetSymbolAddress, with the device current);
  *    make that first call before any stream capture.
+ *  - When the array is reserved: under CUDA's lazy module loading (the
+ *    default), the library's module -- its kernels and this 64 MiB array --
+ *    is loaded onto a device at the library's first use of that device, and
+ *    that may be this entry point's first call.  A caller that hands all
+ *    device memory to its own pool at start-up must therefore make one call
+ *    on each device before it builds the pool (a call with M = 0 and the
+ *    weight and scale pointers of the later calls does the set-up and
+ *    launches nothing), or run with CUDA_MODULE_LOADING=EAGER so that the
+ *    array is reserved when the library is loaded; otherwise that first call
+ *    can fail with FP8WS_ERR_CUDA (out of memory).
  *  - Every call on a device shares the one scratch area, which keeps the
  *    previous call's contents.  Each call overwrites every byte it reads, so
  *    nothing needs clearing, but calls that overlap on the GPU (different

@@ -65,3 +65,23 @@ def gemm_elementwise_bound_ok(y_bits, ref_bits, abssum_bits, K):
 GEMM_REL_FRO = 1e-2          # GEMM and MLP BF16 outputs, relative Frobenius
 SWIGLU_MAX_STEP = 1          # SwiGLU-quant codes: at most one E4M3 step apart ...
 SWIGLU_MAX_FRAC = 1e-4       # ... on at most this fraction of elements
+
+
+def stratified_rows(M: int, seed: int, block: int = 128, extra: int = 4) -> np.ndarray:
+    """Rows of an [M, ...] output for a sampled oracle check that reach every
+    place a tile-level fault could hide: one row in every `block`-row slab
+    (128 = one CTA's half of a CTA-pair tile, so both CTAs of every pair tile
+    are covered), cycling through the four 32-row epilogue-warp quarters of
+    the slab from one slab to the next, plus the first and last rows (the last
+    one lies in the ragged final tile when M is not a multiple of the tile)
+    and `extra` uniformly drawn rows.  Sorted, without repeats."""
+    rng = np.random.default_rng(seed)
+    rows = {0, M - 1}
+    for i, b0 in enumerate(range(0, M, block)):
+        lo = b0 + (i % 4) * 32
+        hi = min(lo + 32, M)
+        if lo >= M:
+            lo, hi = b0, min(b0 + block, M)
+        rows.add(int(rng.integers(lo, hi)))
+    rows.update(int(r) for r in rng.choice(M, min(extra, M), replace=False))
+    return np.array(sorted(rows), dtype=np.int64)

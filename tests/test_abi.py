@@ -3,6 +3,7 @@ symbol the header declares, and rejects bad arguments before it touches CUDA.
 Also checks that the product path never reaches the oracle."""
 
 import ast
+import ctypes
 import os
 import re
 
@@ -57,6 +58,42 @@ def test_workspace_sizes(lib):
     # Xq, then the split-K scratch of the grouped projection GEMMs
     assert lib.qkv_shared_quant_workspace(2048, 3072) == 2048 * 3072 + lib.fp8_linear_static_ws_bytes()
     assert lib.gated_mlp_static_fp8_workspace(-1, 1, 1) == 0
+
+
+def test_workspace_sizes_saturate(lib):
+    """Byte counts that do not fit in 64 bits give SIZE_MAX, never a wrapped
+    small number: M = 2147391056, d = 2147483616, I = 1288564272 (each below
+    2^31) would sum to 2^64 + 65,143,040 bytes for the gated MLP."""
+    size_max = 2 ** 64 - 1
+    M, d, I = 2147391056, 2147483616, 1288564272
+    assert lib.gated_mlp_static_fp8_workspace(M, d, I) == size_max
+    big = 2 ** 62
+    assert lib.gated_mlp_static_fp8_fused_workspace(big, big, big) == size_max
+    assert lib.gated_mlp_per_token_fp8_workspace(big, big, big) == size_max
+    assert lib.fp8_shared_quant_linears_workspace(big, big) == size_max
+    assert lib.cross_attention_qkv_static_fp8_workspace(big, big, big) == size_max
+    rows = (ctypes.c_int64 * 2)(big, big)
+    assert lib.gated_mlp_static_fp8_group_workspace(rows, 2, big, big) == size_max
+    # ordinary sizes are unchanged
+    assert lib.gated_mlp_static_fp8_workspace(1040, 3072, 12288) == 1040 * 64512
+
+
+@pytest.mark.parametrize("M,d,I", [
+    (2147391056, 2147483616, 1288564272),  # wrapped to 65 MB under a 64-bit sum
+    (1041, 3072, 12288),                    # the first M past the 64 MiB area
+    (1, 100, 704),                          # d not a multiple of 16
+    (1, 256, 8),                            # I below 16
+    (2 ** 31, 256, 704),                    # M of 2^31
+    (-1, 256, 704),
+])
+def test_noalloc_refuses_before_cuda(lib, M, d, I):
+    """The no-alloc gated MLP validates the shape and the scratch size before
+    any CUDA call (here, with no GPU, any CUDA call would fail differently)."""
+    n0 = lib.fp8ws_launch_count()
+    a = 1 << 20  # never dereferenced
+    assert lib.gated_mlp_static_fp8_noalloc(a, M, d, I, a, a, a, a, a, a, a, a, a, None) == \
+        fw.ERR_SHAPE
+    assert lib.fp8ws_launch_count() == n0
 
 
 def test_argument_checks_before_cuda(lib):

@@ -19,7 +19,10 @@ def _run(extra_env=None):
 
 
 def test_reference_arm_json_line():
+    import time
+    t0 = time.perf_counter()
     r = _run()
+    wall = time.perf_counter() - t0
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
     assert len(lines) == 1
@@ -32,6 +35,10 @@ def test_reference_arm_json_line():
                         "d2h_bytes_per_step": 0}
     assert d["vs_baseline"] is None and d["data"] == "synthetic"
     assert "workload" in d["config"]
+    # the step time is the wall time the timed step really took (it fits in
+    # this run); the pass time implied by the sample is under its own key
+    assert 0 < d["ms_per_step"] * d["steps"] / 1e3 < wall
+    assert d["extrapolated_ms_per_pass"] > d["ms_per_step"]
 
 
 def test_reference_arm_other_ranks_exit_without_work():

@@ -10,7 +10,7 @@ import torch
 import fp8_w8a8_static_b200 as fw
 import oracle
 import synth
-from _util import GEMM_REL_FRO, bits, codes, rel_fro, scalar
+from _util import GEMM_REL_FRO, bits, codes, rel_fro, scalar, stratified_rows
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -30,7 +30,7 @@ def test_o_proj_single_linear():
     s = oracle.f32(0.03)
     wo = _proj(d, d, 501)
     (y,) = fw.fp8_shared_quant_linears(x, scalar(s, DEV), [wo])
-    rows = np.random.default_rng(5).choice(M, 8, replace=False)
+    rows = stratified_rows(M, 5)
     ref = oracle.qkv_shared_quant(bits(x[rows]), s, [_ref(wo)])[0]
     assert rel_fro(bits(y[rows]), ref) <= GEMM_REL_FRO
 
@@ -67,8 +67,8 @@ def test_cross_attention_projections():
     assert log[2][1] == xq_ptr and log[2][3] == q.data_ptr()
     assert log[3][1] == ctxq_ptr and log[4][1] == ctxq_ptr   # K and V share one
     assert log[3][3] == k.data_ptr() and log[4][3] == v.data_ptr()
-    rq = np.random.default_rng(6).choice(Mq, 6, replace=False)
-    rk = np.random.default_rng(7).choice(Mkv, 6, replace=False)
+    rq = stratified_rows(Mq, 6)
+    rk = stratified_rows(Mkv, 7)
     ref_q = oracle.qkv_shared_quant(bits(x[rq]), s_q, [_ref(wq)])[0]
     ref_k, ref_v = oracle.qkv_shared_quant(bits(ctx[rk]), s_kv, [_ref(wk), _ref(wv)])
     assert rel_fro(bits(q[rq]), ref_q) <= GEMM_REL_FRO

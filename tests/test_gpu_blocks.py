@@ -9,7 +9,8 @@ import torch
 import fp8_w8a8_static_b200 as fw
 import oracle
 import synth
-from _util import (GEMM_REL_FRO, SWIGLU_MAX_FRAC, bits, code_step_diff, codes, rel_fro, scalar)
+from _util import (GEMM_REL_FRO, SWIGLU_MAX_FRAC, bits, code_step_diff, codes, rel_fro, scalar,
+                   stratified_rows)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -125,7 +126,7 @@ def test_gated_mlp_two_tower_layer_sampled_rows(tower):
     s_down = oracle.down_scale(calib, bits(L["wg"]), bits(L["wu"]))
     y = fw.gated_mlp_static_fp8(L["x"], scalar(s_in, DEV), *w["wg"], *w["wu"],
                                 scalar(s_down, DEV), *w["wd"])
-    rows = np.random.default_rng(7).choice(L["M"], 6, replace=False)
+    rows = stratified_rows(L["M"], 7)
     ref = oracle.gated_mlp(bits(L["x"][rows]), s_in, codes(w["wg"][0]), w["wg"][1].item(),
                            codes(w["wu"][0]), w["wu"][1].item(), s_down, codes(w["wd"][0]),
                            w["wd"][1].item())
@@ -150,7 +151,7 @@ def test_qkv_shared_quant_c3_sampled_rows():
     assert all(r[1] == ws.data_ptr() for r in log[1:])
     for t, n in ((q, 3072), (k, 1024), (v, 1024)):
         assert t.shape == (2048, n) and t.is_contiguous()
-    rows = np.random.default_rng(1).choice(2048, 16, replace=False)
+    rows = stratified_rows(2048, 1)
     refs = oracle.qkv_shared_quant(bits(d["x"][rows]), s_in,
                                    [(codes(w[n][0]), w[n][1].item()) for n in ("wq", "wk", "wv")])
     for t, r in zip((q, k, v), refs):

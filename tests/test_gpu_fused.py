@@ -15,7 +15,7 @@ import fp8_w8a8_static_b200 as fw
 import oracle
 import synth
 from _util import (GEMM_REL_FRO, SWIGLU_MAX_FRAC, bits, code_step_diff, codes, from_codes,
-                   rel_fro, scalar)
+                   rel_fro, scalar, stratified_rows)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -59,7 +59,7 @@ def test_fused_against_oracle_sampled_rows():
     x, s_in, xq, wg, s_wg, wu, s_wu = _inputs(M, K, I, 5)
     s_down = scalar(0.0031, DEV)
     h = fw.fp8_gate_up_swiglu_static(xq, wg, wu, s_in, s_wg, s_wu, s_down)
-    rows = np.random.default_rng(2).choice(M, 8, replace=False)
+    rows = stratified_rows(M, 2)
     xr = np.ascontiguousarray(codes(xq)[rows])
     g = oracle.linear(xr, codes(wg), s_in.item(), s_wg.item())
     u = oracle.linear(xr, codes(wu), s_in.item(), s_wu.item())

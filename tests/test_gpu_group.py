@@ -16,7 +16,7 @@ import fp8_w8a8_static_b200 as fw
 import oracle
 import synth
 from _util import (GEMM_REL_FRO, SWIGLU_MAX_FRAC, bits, code_step_diff, codes, from_codes,
-                   gemm_elementwise_bound_ok, rel_fro, scalar)
+                   gemm_elementwise_bound_ok, rel_fro, scalar, stratified_rows)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -93,7 +93,7 @@ def test_linear_group_equals_single(M0, M1, N, K, pair_config):
         assert torch.equal(ys[p], single)
         rows = None
         if xq[p].shape[0] > 64:
-            rows = np.random.default_rng(p).choice(xq[p].shape[0], 16, replace=False)
+            rows = stratified_rows(xq[p].shape[0], p)
         _check_gemm(ys[p], xq[p], wq[p], s_in[p], s_w[p], rows)
     assert fw.device_status()[0] == fw.OK
 
@@ -124,7 +124,7 @@ def test_linear_group_split_k(M0, M1, N, K):
     ys2 = fw.fp8_linear_static_group(probs, split_k=True, workspace=ws)
     for p in range(2):
         assert torch.equal(ys[p], ys2[p])
-        rows = np.random.default_rng(p + 7).choice(xq[p].shape[0], 16, replace=False)
+        rows = stratified_rows(xq[p].shape[0], p + 7)
         _check_gemm(ys[p], xq[p], wq[p], oracle.f32(0.013), oracle.f32(0.0021), rows)
     assert fw.device_status()[0] == fw.OK
 
@@ -167,7 +167,7 @@ def test_gate_up_group_against_oracle_sampled_rows():
              for p, (M, sd) in enumerate(((M0, 0.0031), (M1, 0.0027)))]
     hs = fw.fp8_gate_up_swiglu_static_group(probs)
     for p, (xq, wg, wu, s_in, s_wg, s_wu, s_down) in enumerate(probs):
-        rows = np.random.default_rng(p).choice(xq.shape[0], 6, replace=False)
+        rows = stratified_rows(xq.shape[0], p)
         xr = np.ascontiguousarray(codes(xq)[rows])
         g = oracle.linear(xr, codes(wg), s_in.item(), s_wg.item())
         u = oracle.linear(xr, codes(wu), s_in.item(), s_wu.item())
@@ -254,7 +254,7 @@ def test_mlp_group_full_size_sampled_rows_against_oracle():
     towers = [_tower(4096, d, I, 21, 0.0031), _tower(1024, d, I, 22, 0.0033)]
     ys = fw.gated_mlp_static_fp8_group(towers)
     for p, (t, y) in enumerate(zip(towers, ys)):
-        rows = np.random.default_rng(p + 40).choice(t["x"].shape[0], 4, replace=False)
+        rows = stratified_rows(t["x"].shape[0], p + 40)
         xr = np.ascontiguousarray(bits(t["x"])[rows])
         ref = oracle.gated_mlp(xr, t["s_in"].item(), codes(t["wg"]), t["s_wg"].item(),
                                codes(t["wu"]), t["s_wu"].item(), t["s_down"].item(),
@@ -280,7 +280,7 @@ def test_mlp_group_large_sizes_sampled_rows():
     towers = [_tower(16384, d, I, 61, 0.0025), _tower(8192, d, I, 62, 0.0027)]
     ys = fw.gated_mlp_static_fp8_group(towers)
     for p, (t, y) in enumerate(zip(towers, ys)):
-        rows = np.random.default_rng(p + 90).choice(t["x"].shape[0], 3, replace=False)
+        rows = stratified_rows(t["x"].shape[0], p + 90)
         ref = oracle.gated_mlp(np.ascontiguousarray(bits(t["x"])[rows]), t["s_in"].item(),
                                codes(t["wg"]), t["s_wg"].item(), codes(t["wu"]), t["s_wu"].item(),
                                t["s_down"].item(), codes(t["wd"]), t["s_wd"].item())

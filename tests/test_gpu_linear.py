@@ -11,7 +11,7 @@ import fp8_w8a8_static_b200 as fw
 import oracle
 import synth
 from _util import (GEMM_REL_FRO, bits, codes, from_codes, gemm_elementwise_bound_ok, rel_fro,
-                   scalar)
+                   scalar, stratified_rows)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -99,7 +99,7 @@ def test_linear_sweep_full_size(M, N):
     s_in = oracle.observer_scale([bits(b) for b in d["calib"]])
     wq, s_w = oracle.rtn_weight(bits(d["w"]))
     xq = oracle.quantize(bits(d["x"]), s_in)
-    rows = np.random.default_rng(M + N).choice(M, 24, replace=False)
+    rows = stratified_rows(M, M + N)
     _run(xq, wq, s_in, s_w, rows=rows)
 
 
@@ -122,7 +122,7 @@ def test_split_k_against_oracle(M, N, K):
     s_in, s_w = oracle.f32(0.013), oracle.f32(0.0021)
     y = fw.fp8_linear_static_ws(from_codes(xq, DEV), from_codes(wq, DEV), scalar(s_in, DEV),
                                 scalar(s_w, DEV))
-    rows = np.random.default_rng(1).choice(M, min(M, 16), replace=False)
+    rows = stratified_rows(M, 1)
     yb = bits(y)[rows]
     ref = oracle.linear(np.ascontiguousarray(xq[rows]), wq, s_in, s_w)
     absref = oracle.linear(np.ascontiguousarray(xq[rows]) & 0x7F, wq & 0x7F, s_in, s_w)
@@ -147,7 +147,7 @@ def test_long_k(split):
     s_in, s_w = oracle.f32(0.013), oracle.f32(0.0021)
     args = (from_codes(xq, DEV), from_codes(wq, DEV), scalar(s_in, DEV), scalar(s_w, DEV))
     y = fw.fp8_linear_static_ws(*args) if split else fw.fp8_linear_static(*args)
-    rows = np.random.default_rng(5).choice(M, 16, replace=False)
+    rows = stratified_rows(M, 5)
     yb = bits(y)[rows]
     xr = np.ascontiguousarray(xq[rows])
     ref = oracle.linear(xr, wq, s_in, s_w)

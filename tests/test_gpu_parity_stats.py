@@ -16,7 +16,7 @@ import fp8_w8a8_static_b200 as fw
 import oracle
 import synth
 from _util import (GEMM_REL_FRO, SWIGLU_MAX_FRAC, SWIGLU_MAX_STEP, bits, code_step_diff, codes,
-                   rel_fro, scalar)
+                   rel_fro, scalar, stratified_rows)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -70,7 +70,7 @@ def test_c1_linear(M, N):
     mismatch = int((codes(xq) != ref_q).sum())
     saturated = int(((ref_q & 0x7F) == 0x7E).sum())
     y = fw.fp8_linear_static(xq, wq, scalar(s_in, DEV), s_w)
-    rows = np.random.default_rng(M + N).choice(M, min(M, 32), replace=False)
+    rows = stratified_rows(M, M + N)
     ref_y = oracle.linear(np.ascontiguousarray(ref_q[rows]), codes(wq), s_in, s_w.item())
     rf = rel_fro(bits(y)[rows], ref_y)
     _report(config="c1", M=M, N=N, K=synth.C1_K, xq_mismatch=mismatch,
@@ -87,7 +87,7 @@ def test_c2_swiglu(M, I):
     d = synth.c2_swiglu(M, I, device=DEV, n_calib=4, calib_rows=8)
     s = oracle.swiglu_down_scale([(bits(a), bits(b)) for a, b in d["calib"]])
     h = fw.silu_mul_2in_fp8(d["g"], d["u"], scalar(s, DEV))
-    rows = np.random.default_rng(M * 3 + I).choice(M, min(M, 64), replace=False)
+    rows = stratified_rows(M, M * 3 + I)
     diff = code_step_diff(codes(h[rows]),
                           oracle.silu_mul_2in(bits(d["g"][rows]), bits(d["u"][rows]), s))
     _report(config="c2", M=M, I=I, rows=len(rows), elements=int(diff.size),
@@ -103,7 +103,7 @@ def test_c3_qkv():
     s_in = oracle.observer_scale([bits(b) for b in d["calib"]])
     w = {n: _rtn(d[n]) for n in ("wq", "wk", "wv")}
     q, k, v = fw.qkv_shared_quant(d["x"], scalar(s_in, DEV), *w["wq"], *w["wk"], *w["wv"])
-    rows = np.random.default_rng(1).choice(2048, 32, replace=False)
+    rows = stratified_rows(2048, 1)
     refs = oracle.qkv_shared_quant(bits(d["x"][rows]), s_in,
                                    [(codes(w[n][0]), w[n][1].item()) for n in ("wq", "wk", "wv")])
     rf = [rel_fro(bits(t[rows]), r) for t, r in zip((q, k, v), refs)]
@@ -127,7 +127,7 @@ def test_c4_two_tower_layer_grouped():
     ys = fw.gated_mlp_static_fp8_group(towers)
     stats = dict(config="c4", layer=0)
     for (name, t, y, args) in zip(("gen", "und"), towers, ys, refs_args):
-        rows = np.random.default_rng(len(name)).choice(t["x"].shape[0], 8, replace=False)
+        rows = stratified_rows(t["x"].shape[0], len(name))
         ref = oracle.gated_mlp(bits(t["x"][rows]), *args)
         stats[f"{name}_rows"] = len(rows)
         stats[f"{name}_y_rel_fro"] = rel_fro(bits(y[rows]), ref)

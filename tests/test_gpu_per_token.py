@@ -11,7 +11,7 @@ import fp8_w8a8_static_b200 as fw
 import oracle
 import synth
 from _util import (GEMM_REL_FRO, SWIGLU_MAX_FRAC, bits, code_step_diff, codes, from_codes,
-                   rel_fro, scalar)
+                   rel_fro, scalar, stratified_rows)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -23,7 +23,7 @@ def test_quant_rows_bitexact(rows, K):
     if rows > 3:
         x[2] = 0  # an all-zero row
     q, s = fw.fp8_quant_per_token(x)
-    sample = np.arange(rows) if rows <= 300 else np.random.default_rng(1).choice(rows, 64, replace=False)
+    sample = np.arange(rows) if rows <= 300 else stratified_rows(rows, 1)
     rq, rs = oracle.quantize_rows(bits(x[sample]))
     assert np.array_equal(s.cpu().numpy()[sample], rs)
     assert np.array_equal(codes(q[sample]), rq)
@@ -77,7 +77,7 @@ def test_gated_mlp_per_token(M):
     wu, s_wu = fw.fp8_quant_per_token(synth.normal((I, d), 0.02, 76, DEV))
     wd, s_wd = fw.fp8_quant_per_token(synth.normal((d, I), 0.02, 77, DEV))
     y = fw.gated_mlp_per_token_fp8(x, wg, s_wg, wu, s_wu, wd, s_wd)
-    rows = np.arange(M) if M <= 64 else np.random.default_rng(3).choice(M, 4, replace=False)
+    rows = np.arange(M) if M <= 64 else stratified_rows(M, 3)
     ref = oracle.gated_mlp_per_token(bits(x[rows]), codes(wg), s_wg.cpu().numpy(), codes(wu),
                                      s_wu.cpu().numpy(), codes(wd), s_wd.cpu().numpy())
     assert rel_fro(bits(y[rows]), ref) <= GEMM_REL_FRO

@@ -7,7 +7,7 @@ import torch
 import fp8_w8a8_static_b200 as fw
 import oracle
 import synth
-from _util import bits, codes, from_bits, is_nan_code, scalar
+from _util import bits, codes, from_bits, is_nan_code, scalar, stratified_rows
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -78,6 +78,6 @@ def test_large_bench_size():
     s = oracle.f32(0.0417)
     q = codes(fw.fp8_quant_static(x, scalar(s, DEV)))
     xb = bits(x)
-    rows = np.random.default_rng(0).choice(4096, 64, replace=False)
+    rows = stratified_rows(4096, 0)
     for r in rows:
         assert np.array_equal(q[r], oracle.quantize(np.ascontiguousarray(xb[r]), s))

@@ -12,7 +12,7 @@ import fp8_w8a8_static_b200 as fw
 import oracle
 import synth
 from _util import (SWIGLU_MAX_FRAC, SWIGLU_MAX_STEP, bits, code_step_diff, codes, from_bits,
-                   scalar)
+                   scalar, stratified_rows)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -50,7 +50,7 @@ def test_sweep_full_size(M, I):
     d = synth.c2_swiglu(M, I, device=DEV, n_calib=4, calib_rows=8)
     s = oracle.swiglu_down_scale([(bits(a), bits(b)) for a, b in d["calib"]])
     h = fw.silu_mul_2in_fp8(d["g"], d["u"], scalar(s, DEV))
-    rows = np.random.default_rng(M * I).choice(M, 12, replace=False)
+    rows = stratified_rows(M, M * I)
     hc = codes(h[rows])
     ref = oracle.silu_mul_2in(bits(d["g"][rows]), bits(d["u"][rows]), s)
     _compare(hc, ref)

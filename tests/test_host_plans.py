@@ -31,6 +31,16 @@ def test_threshold_at_64_k_steps():
     assert fw.split_plan(10, PAIRS, 64)["splits"] > 1
 
 
+def test_threshold_at_ragged_k():
+    """The threshold counts 128-byte K steps, ceil(K / 128): K = 8064 is 63
+    steps (not split), K = 8080 (a multiple of 16 below 8192) is already 64
+    steps and splits like K = 8192."""
+    assert fw.split_plan(10, PAIRS, -(-8064 // 128))["splits"] == 1
+    assert -(-8080 // 128) == 64
+    p = fw.split_plan(10, PAIRS, -(-8080 // 128))
+    assert p == fw.split_plan(10, PAIRS, 8192 // 128) and p["splits"] > 1
+
+
 def test_ragged_k_case_of_the_gpu_tests():
     """M=300, N=520, K=8208: 6 tiles, 65 K steps (the last one partial)."""
     assert fw.split_plan(6, PAIRS, 65) == dict(dp_tiles=0, split_tiles=6, splits=4,

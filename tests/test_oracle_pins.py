@@ -378,6 +378,18 @@ def test_shared_scale_invariant():
     assert not oracle.shared_scales_equal([-s, -s])
 
 
+def test_golden_requant():
+    """Hand-derived values of the fused loader's re-quantization
+    qW' = q(s_i * deq(qW) / s_max) (pull request "Load static FP8 Cosmos3
+    Nano/Super checkpoints without re-quantizing them", Description).  Each
+    case's inverted ratio s_max * deq / s_i gives another code, so a swapped
+    operand fails here."""
+    for code, s_i, s_max, want in _golden("requant"):
+        q = np.array([int(code, 16)], np.uint8)
+        got = oracle.requant_group_member(q, float(s_i), float(s_max))
+        assert int(got[0]) == int(want, 16), (code, s_i, s_max)
+
+
 def test_fused_group_requant_changes_codes_split_keeps_them():
     """Group with genuinely different weight scales (asserted first): the
     fused loader's second rounding changes codes; the split path keeps the
