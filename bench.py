@@ -11,12 +11,16 @@ the whole pass, (1024 + 4096) tokens per step per GPU.
 
 Under torchrun with N>1 every rank runs an independent replica of the pass on
 its own GPU (no data-path collective; weak scaling).  Rank 0 prints one JSON
-line.  The timed region issues the path's kernels through the C ABI with CUDA
-events between them, so the same run yields the pass time and each kernel's
-average duration (for the roofline of the dominant kernel).  The end-to-end
-number goes through the composite gated-MLP call with host buffers: every
-layer's input is copied from pinned host memory and its output copied back
-inside the timed region.
+line.  The timed region replays the pass (one grouped composite C-ABI call per
+layer) as a CUDA graph, with CUDA events around the region only.  Afterwards
+each kind of launch of the step is replayed back to back on its own, which
+gives each kernel's average launch duration (for the roofline of the
+dominant kernel).  The end-to-end number goes through the composite call with
+host buffers: every layer's input is copied from pinned host memory and its
+output copied back inside the timed region.  At N=1 the line also carries the
+per-workload kernel figures ("configs": the Linear sweep, the SwiGLU sweep, the
+shared-quant Q/K/V block, the tiny MLP, the per-token path and the
+cross-attention projections) with their roofline fractions.
 
 `--impl reference` times the CPU oracle (the only other implementation there
 is) on a bounded sample of rows of the same pass on the host cores.
@@ -126,6 +130,75 @@ class ClockSampler:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+class NvmlClockSampler:
+    """SM clock, power and clock-event reasons read through NVML every 20 ms
+    on a host thread while the timed region runs (a 200 ms nvidia-smi loop
+    sees only a couple of samples in a sub-second region).  Reads only."""
+
+    INTERVAL_S = 0.02
+
+    def __init__(self, device_index: int):
+        import pynvml
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(device_index)
+        uuid = getattr(props, "uuid", None)
+        self.h = None
+        if uuid is not None:
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(uuid))
+            except Exception:
+                self.h = None
+        if self.h is None:
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+        self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        self.names = (("hw_slowdown", pynvml.nvmlClocksEventReasonHwSlowdown),
+                      ("hw_thermal_slowdown", pynvml.nvmlClocksEventReasonHwThermalSlowdown),
+                      ("sw_thermal_slowdown", pynvml.nvmlClocksEventReasonSwThermalSlowdown),
+                      ("hw_power_brake_slowdown", pynvml.nvmlClocksEventReasonHwPowerBrakeSlowdown),
+                      ("sw_power_cap", pynvml.nvmlClocksEventReasonSwPowerCap))
+        self.samples = []
+        self.stop_flag = threading.Event()
+        self.thread = None
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_flag.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                pw = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                self.samples.append((float(sm), int(rs), pw))
+            except Exception:
+                pass
+            self.stop_flag.wait(self.INTERVAL_S)
+
+    def start(self):
+        self.samples = []
+        self.stop_flag.clear()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def stop(self):
+        self.stop_flag.set()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+        if not self.samples:
+            return None
+        reasons = sorted({n for _, rs, _ in self.samples for n, bit in self.names if rs & bit})
+        return {"sm_mhz": statistics.median(s[0] for s in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples),
+                "power_w_max": max(s[2] for s in self.samples),
+                "source": f"NVML every {int(self.INTERVAL_S * 1000)} ms during the timed region"}
+
+
+def clock_sampler(device_index: int):
+    try:
+        return NvmlClockSampler(device_index)
+    except Exception:
+        return ClockSampler(device_index)
 
 
 # ---------------------------------------------------------------- set-up
@@ -392,12 +465,11 @@ def capture_graph(run):
     return g
 
 
-def time_device(plan, steps, warmup, dist_ctx, sampler=None, runner=None, instr_plan=None):
+def time_device(plan, steps, warmup, dist_ctx, sampler=None, runner=None):
     """W untimed steps, then K timed steps between a barrier + synchronize on
     both sides, with CUDA events on the launching stream around the region
     only (an event between two kernels would stop the next kernel from being
-    scheduled early).  Then K more steps with events between every launch,
-    for each kernel's average duration."""
+    scheduled early)."""
     run = runner if runner is not None else (lambda: run_plan(plan))
     for _ in range(warmup):
         run()
@@ -414,25 +486,50 @@ def time_device(plan, steps, warmup, dist_ctx, sampler=None, runner=None, instr_
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
     dist_ctx.barrier()
-    total_ms = start.elapsed_time(stop)
+    return start.elapsed_time(stop), clocks
 
-    plan = instr_plan if instr_plan is not None else plan
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(plan) + 1)]
-          for _ in range(steps)]
-    for k in range(steps):
-        run_plan(plan, ev[k])
-    torch.cuda.synchronize()
-    per_kind = {}
-    for k in range(steps):
-        for i, (kind, _, _, nbytes, flops) in enumerate(plan):
-            dt = ev[k][i].elapsed_time(ev[k][i + 1])
-            acc = per_kind.setdefault(kind, [0.0, 0, 0, 0])
-            acc[0] += dt
-            acc[1] += 1
-            acc[2] += nbytes
-            acc[3] += flops
-    instrumented_ms = sum(ev[k][0].elapsed_time(ev[k][-1]) for k in range(steps))
-    return total_ms, per_kind, clocks, instrumented_ms
+
+def time_kinds(plan, steps):
+    """Average launch duration of each kind of launch in the step.  The
+    step's launches of one kind (36 of each in the grouped pass, every one on
+    its own layer's buffers) are captured into a CUDA graph that issues them
+    back to back on one stream, as the step does; the graph is replayed
+    `steps` times, each replay timed by its own event pair, and the median
+    replay time is divided by its launch count.  No event sits between two
+    launches, so programmatic launch overlap is kept, as in the step.
+    Returns {kind: (ms per launch, launches per step, bytes, flops per launch)}."""
+    kinds = []
+    for e in plan:
+        if e[0] not in kinds:
+            kinds.append(e[0])
+    out = {}
+    for kind in kinds:
+        entries = [e for e in plan if e[0] == kind]
+
+        def run_current(entries=entries):
+            h = torch.cuda.current_stream().cuda_stream
+            for _, fn, a, _, _ in entries:
+                if fn(*(a[:-1] + (h,))) != 0:
+                    raise RuntimeError("launch failed")
+        run_current()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            run_current()
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        times = []
+        for _ in range(steps):
+            a.record()
+            g.replay()
+            b.record()
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+        del g
+        n = len(entries)
+        out[kind] = (statistics.median(times) / n, n, entries[0][3], entries[0][4])
+    return out
 
 
 def time_e2e(fw, layers, steps, warmup, device, dist_ctx, fused):
@@ -662,190 +759,302 @@ def cpu_baseline(rows_per_tower: int = 1024):
 
 
 L2_FLUSH_BYTES = 256 * 1024 * 1024  # twice the 126 MB L2
+ROTATE_BYTES = 256 * 1024 * 1024    # buffer sets are rotated until they span twice the L2
+MAX_SETS = 64
+MIN_PER_REPLAY = 20                 # launches per replay of a back-to-back graph
 
 
-def kernel_bench(fw, kind, shape, steps, warmup, device, sustain_s=0.0):
-    """One kernel on synthetic data shaped like the pages' workloads, timed
-    launch by launch with CUDA events.  Between launches, outside the timed
-    interval, L2 is flushed by reading a 256 MB buffer (a read leaves no dirty
-    lines to be written back inside the next timed launch).  With sustain_s >
-    0 the kernel also runs back to back for that many seconds (no flush), the
-    power-capped figure.  Kind "scaled_mm" is torch._scaled_mm (cuBLASLt FP8
-    with per-tensor scales, BF16 out): the library ceiling our FP8 GEMM is
-    compared with, not part of the path.  Returns a dict for one JSON line."""
-    flush = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
-    pk = peaks()
-    if kind in ("gemm", "gemm_ws"):
+def _scalar(v, device):
+    return torch.tensor([v], dtype=torch.float32, device=device)
+
+
+def _static_linear_inputs(fw, M, N, K, cfg, seed, device):
+    x = synth.student_t((M, K), 4, synth.seed(cfg, seed, 0), device)
+    w = synth.normal((N, K), synth.W_STD, synth.seed(cfg, seed, 10), device)
+    s_in = fw.fp8_observer_scale(fw.fp8_absmax_bf16(x))
+    xq = fw.fp8_quant_static(x, s_in)
+    wq, s_w = fw.fp8_rtn_quantize_weight(w)
+    return xq, wq, s_in, s_w
+
+
+def make_kernel(fw, kind, shape, device):
+    """One call of a kernel kind on one shape, with synthetic inputs shaped
+    like the pages' workloads.  Returns (t, call, work, nbytes): t holds every
+    device buffer the call reads or writes (cloning t gives an independent
+    set), call(t) issues the call on the current stream, work is its
+    algorithmic flops (None for the streaming kernels), nbytes its algorithmic
+    bytes (every operand read once, every output written once).  Kind
+    "scaled_mm" is torch._scaled_mm (cuBLASLt FP8 with per-tensor scales, BF16
+    out): the library ceiling our GEMM is compared with, not part of the path."""
+    bf, f8 = torch.bfloat16, fw.FP8
+    emp = lambda shp, dt: torch.empty(shp, dtype=dt, device=device)  # noqa: E731
+    if kind in ("gemm", "gemm_ws", "scaled_mm"):
         M, N, K = shape
-        x = synth.student_t((M, K), 4, synth.seed(1, 90, 0), device)
-        w = synth.normal((N, K), synth.W_STD, synth.seed(1, 90, 10), device)
-        s_in = fw.fp8_observer_scale(fw.fp8_absmax_bf16(x))
-        xq = fw.fp8_quant_static(x, s_in)
-        wq, s_w = fw.fp8_rtn_quantize_weight(w)
-        del x, w
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        xq, wq, s_in, s_w = _static_linear_inputs(fw, M, N, K, 1, 90 if kind != "scaled_mm" else 92,
+                                                  device)
+        t = dict(xq=xq, wq=wq, s_in=s_in, s_w=s_w, y=emp((M, N), bf))
         if kind == "gemm_ws":
-            wsb = torch.zeros(fw.load().fp8_linear_static_ws_bytes(), dtype=torch.uint8,
-                              device=device)
-            fn = lambda: fw.fp8_linear_static_ws(xq, wq, s_in, s_w, workspace=wsb, out=y)  # noqa: E731
+            t["ws"] = torch.zeros(fw.load().fp8_linear_static_ws_bytes(), dtype=torch.uint8,
+                                  device=device)
+            call = lambda t: fw.fp8_linear_static_ws(t["xq"], t["wq"], t["s_in"], t["s_w"],  # noqa: E731
+                                                     workspace=t["ws"], out=t["y"])
+        elif kind == "gemm":
+            call = lambda t: fw.fp8_linear_static(t["xq"], t["wq"], t["s_in"], t["s_w"],  # noqa: E731
+                                                  out=t["y"])
         else:
-            fn = lambda: fw.fp8_linear_static(xq, wq, s_in, s_w, out=y)  # noqa: E731
-        work = 2.0 * M * N * K
-        nbytes = M * K + N * K + 2 * M * N
-    elif kind == "dual":
+            del t["y"]
+            call = lambda t: torch._scaled_mm(t["xq"], t["wq"].t(), scale_a=t["s_in"],  # noqa: E731
+                                              scale_b=t["s_w"], out_dtype=bf)
+        return t, call, 2.0 * M * N * K, M * K + N * K + 2 * M * N
+    if kind == "gemm_scaled":  # per-token activation and per-channel weight scales
+        M, N, K = shape
+        x = synth.activation_with_outliers(M, K, 9, 6, 0, device)
+        xq, sx = fw.fp8_quant_per_token(x)
+        wq, sw = fw.fp8_quant_per_token(synth.normal((N, K), synth.W_STD, synth.seed(6, 90, 1),
+                                                     device))
+        t = dict(xq=xq, wq=wq, sx=sx, sw=sw, y=emp((M, N), bf))
+        call = lambda t: fw.fp8_linear_scaled(t["xq"], t["wq"], t["sx"], t["sw"], out=t["y"])  # noqa: E731
+        return t, call, 2.0 * M * N * K, M * K + N * K + 2 * M * N + 4 * (M + N)
+    if kind == "dual":
         M, N, K = shape
         x = synth.activation_with_outliers(M, K, 9, 1, 0, device)
         s_in = fw.fp8_observer_scale(fw.fp8_absmax_bf16(x))
         xq = fw.fp8_quant_static(x, s_in)
         wg, s_wg = fw.fp8_rtn_quantize_weight(synth.normal((N, K), synth.W_STD, synth.seed(4, 90, 1), device))
         wu, s_wu = fw.fp8_rtn_quantize_weight(synth.normal((N, K), synth.W_STD, synth.seed(4, 90, 2), device))
-        s_down = torch.tensor([0.003], dtype=torch.float32, device=device)
-        del x
-        h = torch.empty((M, N), dtype=fw.FP8, device=device)
-        fn = lambda: fw.fp8_gate_up_swiglu_static(xq, wg, wu, s_in, s_wg, s_wu, s_down, out=h)  # noqa: E731
-        work = 4.0 * M * N * K
-        nbytes = M * K + 2 * N * K + M * N
-    elif kind == "mlp":
+        t = dict(xq=xq, wg=wg, wu=wu, s_in=s_in, s_wg=s_wg, s_wu=s_wu, s_down=_scalar(0.003, device),
+                 h=emp((M, N), f8))
+        call = lambda t: fw.fp8_gate_up_swiglu_static(t["xq"], t["wg"], t["wu"], t["s_in"],  # noqa: E731
+                                                      t["s_wg"], t["s_wu"], t["s_down"], out=t["h"])
+        return t, call, 4.0 * M * N * K, M * K + 2 * N * K + M * N
+    if kind in ("mlp", "mlp_tok"):
         M, dm, Ii = shape
         x = synth.activation_with_outliers(M, dm, 0, 0, 0, device)
-        s_in = fw.fp8_observer_scale(fw.fp8_absmax_bf16(x))
-        wts = [fw.fp8_rtn_quantize_weight(synth.normal(shp, synth.W_STD, synth.seed(0, 90, k), device))
+        ws_ = [synth.normal(shp, synth.W_STD, synth.seed(0, 90, k), device)
                for k, shp in enumerate(((Ii, dm), (Ii, dm), (dm, Ii)))]
-        s_down = torch.tensor([0.003], dtype=torch.float32, device=device)
-        wsb = torch.empty(fw.gated_mlp_static_fp8_fused_workspace(M, dm, Ii), dtype=torch.uint8,
-                          device=device)
-        y = torch.empty((M, dm), dtype=torch.bfloat16, device=device)
-        fn = lambda: fw.gated_mlp_static_fp8_fused(x, s_in, *wts[0], *wts[1], s_down, *wts[2],  # noqa: E731
-                                                   workspace=wsb, out=y)
-        work = 6.0 * M * dm * Ii
-        nbytes = 2 * M * dm + 3 * dm * Ii + 2 * M * dm
-    elif kind == "qkv":
+        if kind == "mlp":
+            t = dict(x=x, s_in=fw.fp8_observer_scale(fw.fp8_absmax_bf16(x)),
+                     s_down=_scalar(0.003, device), y=emp((M, dm), bf),
+                     ws=emp(fw.gated_mlp_static_fp8_fused_workspace(M, dm, Ii), torch.uint8))
+            for name, w in zip(("g", "u", "d"), ws_):
+                t["w" + name], t["s_w" + name] = fw.fp8_rtn_quantize_weight(w)
+            call = lambda t: fw.gated_mlp_static_fp8_fused(  # noqa: E731
+                t["x"], t["s_in"], t["wg"], t["s_wg"], t["wu"], t["s_wu"], t["s_down"], t["wd"],
+                t["s_wd"], workspace=t["ws"], out=t["y"])
+        else:  # per-channel weight scales, per-token activation scales computed at run time
+            t = dict(x=x, y=emp((M, dm), bf),
+                     ws=emp(fw.load().gated_mlp_per_token_fp8_workspace(M, dm, Ii), torch.uint8))
+            for name, w in zip(("g", "u", "d"), ws_):
+                t["w" + name], t["s_w" + name] = fw.fp8_quant_per_token(w)
+            call = lambda t: fw.gated_mlp_per_token_fp8(  # noqa: E731
+                t["x"], t["wg"], t["s_wg"], t["wu"], t["s_wu"], t["wd"], t["s_wd"],
+                workspace=t["ws"], out=t["y"])
+        return t, call, 6.0 * M * dm * Ii, 2 * M * dm + 3 * dm * Ii + 2 * M * dm
+    if kind in ("qkv", "qkv_gemm"):
         M, dm, Nq, Nkv = shape
         x = synth.activation_with_outliers(M, dm, 3, 90, 0, device, heavy_tailed_outliers=True)
         s_in = fw.fp8_observer_scale(fw.fp8_absmax_bf16(x))
-        wts = [fw.fp8_rtn_quantize_weight(synth.normal((n, dm), synth.W_STD, synth.seed(3, 90, k),
-                                                       device))
-               for k, n in enumerate((Nq, Nkv, Nkv))]
-        wsb = torch.empty(fw.qkv_shared_quant_workspace(M, dm), dtype=torch.uint8, device=device)
-        outs = tuple(torch.empty((M, n), dtype=torch.bfloat16, device=device) for n in (Nq, Nkv, Nkv))
-        fn = lambda: fw.qkv_shared_quant(x, s_in, *wts[0], *wts[1], *wts[2], workspace=wsb,  # noqa: E731
-                                         out=outs)
-        work = 2.0 * M * dm * (Nq + 2 * Nkv)
-        nbytes = 2 * M * dm + dm * (Nq + 2 * Nkv) + 2 * M * (Nq + 2 * Nkv)
-    elif kind == "scaled_mm":
-        M, N, K = shape
-        x = synth.student_t((M, K), 4, synth.seed(1, 92, 0), device)
-        w = synth.normal((N, K), synth.W_STD, synth.seed(1, 92, 10), device)
-        s_in = fw.fp8_observer_scale(fw.fp8_absmax_bf16(x))
-        xq = fw.fp8_quant_static(x, s_in)
-        wq, s_w = fw.fp8_rtn_quantize_weight(w)
-        del x, w
-        fn = lambda: torch._scaled_mm(xq, wq.t(), scale_a=s_in, scale_b=s_w,  # noqa: E731
-                                      out_dtype=torch.bfloat16)
-        work = 2.0 * M * N * K
-        nbytes = M * K + N * K + 2 * M * N
-    elif kind in ("gemm_group", "gemm_group_ws"):
+        t = dict(s_in=s_in)
+        for k, (name, n) in enumerate((("q", Nq), ("k", Nkv), ("v", Nkv))):
+            t["w" + name], t["s_w" + name] = fw.fp8_rtn_quantize_weight(
+                synth.normal((n, dm), synth.W_STD, synth.seed(3, 90, k), device))
+            t["y" + name] = emp((M, n), bf)
+        proj = lambda t: [(t["wq"], t["s_wq"]), (t["wk"], t["s_wk"]), (t["wv"], t["s_wv"])]  # noqa: E731
+        outs = lambda t: [t["yq"], t["yk"], t["yv"]]  # noqa: E731
+        nsum = Nq + 2 * Nkv
+        if kind == "qkv":
+            t["x"] = x
+            t["ws"] = emp(fw.qkv_shared_quant_workspace(M, dm), torch.uint8)
+            call = lambda t: fw.fp8_shared_quant_linears(t["x"], t["s_in"], proj(t),  # noqa: E731
+                                                         workspace=t["ws"], out=outs(t))
+            return t, call, 2.0 * M * dm * nsum, 2 * M * dm + dm * nsum + 2 * M * nsum
+        t["xq"] = fw.fp8_quant_static(x, s_in)
+        call = lambda t: fw.fp8_linears_static(t["xq"], t["s_in"], proj(t), out=outs(t))  # noqa: E731
+        return t, call, 2.0 * M * dm * nsum, M * dm + dm * nsum + 2 * M * nsum
+    if kind == "xattn":  # cross-attention: Q from x, K and V from a context tensor
+        Mq, Mkv, dm, Nq, Nkv = shape
+        x = synth.activation_with_outliers(Mq, dm, 5, 5, 0, device)
+        ctx = synth.activation_with_outliers(Mkv, dm, 5, 6, 0, device)
+        t = dict(x=x, ctx=ctx, s_q=fw.fp8_observer_scale(fw.fp8_absmax_bf16(x)),
+                 s_kv=fw.fp8_observer_scale(fw.fp8_absmax_bf16(ctx)),
+                 ws=emp(fw.load().cross_attention_qkv_static_fp8_workspace(Mq, Mkv, dm),
+                        torch.uint8),
+                 yq=emp((Mq, Nq), bf), yk=emp((Mkv, Nkv), bf), yv=emp((Mkv, Nkv), bf))
+        for k, (name, n) in enumerate((("q", Nq), ("k", Nkv), ("v", Nkv))):
+            t["w" + name], t["s_w" + name] = fw.fp8_rtn_quantize_weight(
+                synth.normal((n, dm), synth.W_STD, synth.seed(5, 90, k), device))
+        call = lambda t: fw.cross_attention_qkv_static_fp8(  # noqa: E731
+            t["x"], t["ctx"], t["s_q"], t["wq"], t["s_wq"], t["s_kv"], t["wk"], t["s_wk"],
+            t["wv"], t["s_wv"], workspace=t["ws"], out=(t["yq"], t["yk"], t["yv"]))
+        work = 2.0 * dm * (Mq * Nq + 2 * Mkv * Nkv)
+        return t, call, work, 2 * (Mq + Mkv) * dm + dm * (Nq + 2 * Nkv) + 2 * (Mq * Nq + 2 * Mkv * Nkv)
+    if kind in ("gemm_group", "gemm_group_ws", "dual_group", "quant_group"):
+        if kind == "quant_group":
+            M0, M1, K = shape
+            t = {}
+            for p, M in enumerate((M0, M1)):
+                t[f"x{p}"] = synth.activation_with_outliers(M, K, 9, p, 0, device)
+                t[f"s{p}"] = fw.fp8_observer_scale(fw.fp8_absmax_bf16(t[f"x{p}"]))
+                t[f"q{p}"] = emp((M, K), f8)
+            call = lambda t: fw.fp8_quant_static_group([t["x0"], t["x1"]], [t["s0"], t["s1"]],  # noqa: E731
+                                                       outs=[t["q0"], t["q1"]])
+            return t, call, None, 3 * (M0 + M1) * K
         M0, M1, N, K = shape
-        probs = []
+        t = {}
         for p, M in enumerate((M0, M1)):
-            x = synth.student_t((M, K), 4, synth.seed(1, 91, p), device)
-            s_in = fw.fp8_observer_scale(fw.fp8_absmax_bf16(x))
-            xq = fw.fp8_quant_static(x, s_in)
-            wq, s_w = fw.fp8_rtn_quantize_weight(
-                synth.normal((N, K), synth.W_STD, synth.seed(1, 91, 10 + p), device))
-            probs.append((xq, wq, s_in, s_w))
-            del x
-        ys = [torch.empty((M, N), dtype=torch.bfloat16, device=device) for M in (M0, M1)]
-        wsb = torch.zeros(fw.load().fp8_linear_static_ws_bytes(), dtype=torch.uint8, device=device)
+            if kind == "dual_group":
+                x = synth.activation_with_outliers(M, K, 9, 2 + p, 0, device)
+                t[f"s_in{p}"] = fw.fp8_observer_scale(fw.fp8_absmax_bf16(x))
+                t[f"xq{p}"] = fw.fp8_quant_static(x, t[f"s_in{p}"])
+                for j, nm in enumerate(("wg", "wu")):
+                    t[f"{nm}{p}"], t[f"s_{nm}{p}"] = fw.fp8_rtn_quantize_weight(
+                        synth.normal((N, K), synth.W_STD, synth.seed(4, 91, 1 + j + 2 * p), device))
+                t[f"s_down{p}"] = _scalar(0.003, device)
+                t[f"h{p}"] = emp((M, N), f8)
+            else:
+                t[f"xq{p}"], t[f"wq{p}"], t[f"s_in{p}"], t[f"s_w{p}"] = _static_linear_inputs(
+                    fw, M, N, K, 1, 91 + 2 * p, device)
+                t[f"y{p}"] = emp((M, N), bf)
+        if kind == "dual_group":
+            probs = lambda t: [tuple(t[f"{k}{p}"] for k in ("xq", "wg", "wu", "s_in", "s_wg",  # noqa: E731
+                                                           "s_wu", "s_down")) for p in range(2)]
+            call = lambda t: fw.fp8_gate_up_swiglu_static_group(probs(t), outs=[t["h0"], t["h1"]])  # noqa: E731
+            return t, call, 4.0 * (M0 + M1) * N * K, (M0 + M1) * K + 4 * N * K + (M0 + M1) * N
+        t["ws"] = torch.zeros(fw.load().fp8_linear_static_ws_bytes(), dtype=torch.uint8, device=device)
         split = kind == "gemm_group_ws"
-        fn = lambda: fw.fp8_linear_static_group(probs, outs=ys, split_k=split, workspace=wsb)  # noqa: E731
-        work = 2.0 * (M0 + M1) * N * K
-        nbytes = (M0 + M1) * K + 2 * N * K + 2 * (M0 + M1) * N
-    elif kind == "dual_group":
-        M0, M1, N, K = shape
-        probs = []
-        for p, M in enumerate((M0, M1)):
-            x = synth.activation_with_outliers(M, K, 9, 2 + p, 0, device)
-            s_in = fw.fp8_observer_scale(fw.fp8_absmax_bf16(x))
-            xq = fw.fp8_quant_static(x, s_in)
-            wg, s_wg = fw.fp8_rtn_quantize_weight(
-                synth.normal((N, K), synth.W_STD, synth.seed(4, 91, 1 + 2 * p), device))
-            wu, s_wu = fw.fp8_rtn_quantize_weight(
-                synth.normal((N, K), synth.W_STD, synth.seed(4, 91, 2 + 2 * p), device))
-            s_down = torch.tensor([0.003], dtype=torch.float32, device=device)
-            probs.append((xq, wg, wu, s_in, s_wg, s_wu, s_down))
-            del x
-        hs = [torch.empty((M, N), dtype=fw.FP8, device=device) for M in (M0, M1)]
-        fn = lambda: fw.fp8_gate_up_swiglu_static_group(probs, outs=hs)  # noqa: E731
-        work = 4.0 * (M0 + M1) * N * K
-        nbytes = (M0 + M1) * K + 4 * N * K + (M0 + M1) * N
-    elif kind == "quant_group":
-        M0, M1, K = shape
-        xs = [synth.activation_with_outliers(M, K, 9, p, 0, device) for p, M in enumerate((M0, M1))]
-        ss = [fw.fp8_observer_scale(fw.fp8_absmax_bf16(x)) for x in xs]
-        qs = [torch.empty((M, K), dtype=fw.FP8, device=device) for M in (M0, M1)]
-        fn = lambda: fw.fp8_quant_static_group(xs, ss, outs=qs)  # noqa: E731
-        work = None
-        nbytes = 3 * (M0 + M1) * K
-    elif kind == "swiglu":
+        probs = lambda t: [tuple(t[f"{k}{p}"] for k in ("xq", "wq", "s_in", "s_w")) for p in range(2)]  # noqa: E731
+        call = lambda t: fw.fp8_linear_static_group(probs(t), outs=[t["y0"], t["y1"]],  # noqa: E731
+                                                    split_k=split, workspace=t["ws"])
+        return t, call, 2.0 * (M0 + M1) * N * K, (M0 + M1) * K + 2 * N * K + 2 * (M0 + M1) * N
+    if kind in ("swiglu", "swiglu_tok"):
         M, Ii = shape
-        g = synth.normal((M, Ii), 2.0, synth.seed(2, 90, 7), device)
-        u = synth.normal((M, Ii), 1.0, synth.seed(2, 90, 8), device)
-        s = fw.fp8_observer_scale(fw.fp8_silu_mul_absmax(g, u))
-        h = torch.empty((M, Ii), dtype=fw.FP8, device=device)
-        fn = lambda: fw.silu_mul_2in_fp8(g, u, s, out=h)  # noqa: E731
-        work = None
-        nbytes = 5 * M * Ii
-    elif kind == "quant":
+        t = dict(g=synth.normal((M, Ii), 2.0, synth.seed(2, 90, 7), device),
+                 u=synth.normal((M, Ii), 1.0, synth.seed(2, 90, 8), device), h=emp((M, Ii), f8))
+        if kind == "swiglu":
+            t["s"] = fw.fp8_observer_scale(fw.fp8_silu_mul_absmax(t["g"], t["u"]))
+            call = lambda t: fw.silu_mul_2in_fp8(t["g"], t["u"], t["s"], out=t["h"])  # noqa: E731
+            return t, call, None, 5 * M * Ii
+        t["s"] = emp((M,), torch.float32)
+        call = lambda t: fw.silu_mul_2in_fp8_per_token(t["g"], t["u"], out=t["h"], scales=t["s"])  # noqa: E731
+        return t, call, None, 5 * M * Ii + 4 * M
+    if kind in ("quant", "quant_tok"):
         M, K = shape
-        x = synth.activation_with_outliers(M, K, 9, 0, 0, device)
-        s = fw.fp8_observer_scale(fw.fp8_absmax_bf16(x))
-        xq = torch.empty((M, K), dtype=fw.FP8, device=device)
-        fn = lambda: fw.fp8_quant_static(x, s, out=xq)  # noqa: E731
-        work = None
-        nbytes = 3 * M * K
-    else:
-        raise ValueError(kind)
+        t = dict(x=synth.activation_with_outliers(M, K, 9, 0, 0, device), q=emp((M, K), f8))
+        if kind == "quant":
+            t["s"] = fw.fp8_observer_scale(fw.fp8_absmax_bf16(t["x"]))
+            call = lambda t: fw.fp8_quant_static(t["x"], t["s"], out=t["q"])  # noqa: E731
+            return t, call, None, 3 * M * K
+        t["s"] = emp((M,), torch.float32)
+        call = lambda t: fw.fp8_quant_per_token(t["x"], out=t["q"], scales=t["s"])  # noqa: E731
+        return t, call, None, 3 * M * K + 4 * M
+    raise ValueError(kind)
+
+
+def _set_bytes(t):
+    return sum(v.numel() * v.element_size() for v in t.values())
+
+
+def time_back_to_back(calls, steps, warmup):
+    """Per-launch time of calls issued back to back, as a layer stack issues
+    them: the calls (one per buffer set, repeated to at least MIN_PER_REPLAY)
+    are captured once into a CUDA graph, so that host issue cannot starve the
+    GPU, and the graph is replayed; each replay is timed by its own event pair
+    and the median replay time is divided by its launch count.  Returns (ms
+    per call, calls per replay)."""
+    seq = calls * max(1, -(-MIN_PER_REPLAY // len(calls)))
+    for c in calls:  # eager once: the library's per-device set-up stays out of the capture
+        c()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for c in seq:
+            c()
     for _ in range(warmup):
-        fn()
+        g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     times = []
     for _ in range(steps):
-        flush.sum()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        fn()
+        g.replay()
+        b.record()
+        b.synchronize()
+        times.append(a.elapsed_time(b) / len(seq))
+    del g
+    return statistics.median(times), len(seq)
+
+
+def time_isolated(call, steps, warmup, flush):
+    """One launch at a time with L2 flushed before it (a 256 MB read, which
+    leaves no dirty lines), timed by an event pair around the launch.  The
+    figure includes the launch latency between the event and the kernel."""
+    for _ in range(warmup):
+        call()
+    times = []
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(steps):
+        flush.sum()
+        a.record()
+        call()
         b.record()
         b.synchronize()
         times.append(a.elapsed_time(b))
-    ms = statistics.median(times)
-    out = {"kernel": kind, "shape": list(shape), "us": ms * 1e3, "steps": steps,
+    return statistics.median(times)
+
+
+def kernel_bench(fw, kind, shape, steps, warmup, device, sustain_s=0.0, isolated=True):
+    """One kernel kind on one shape.  The headline "us" is the back-to-back
+    per-launch time over buffer sets rotated until they span twice the L2
+    (so every launch reads its operands from DRAM, as a layer stack does);
+    "us_isolated" is the same launch alone after an L2 flush.  Fractions use
+    the burst peaks (these kernels are timed in short runs).  With sustain_s >
+    0 the back-to-back graph also replays for that many seconds, the
+    power-capped rate.  Returns a dict for one JSON line."""
+    pk = peaks()
+    t0, call, work, nbytes = make_kernel(fw, kind, shape, device)
+    nsets = int(min(MAX_SETS, max(1, -(-ROTATE_BYTES // max(_set_bytes(t0), 1)))))
+    sets = [t0] + [{k: v.clone() for k, v in t0.items()} for _ in range(nsets - 1)]
+    calls = [(lambda t=t: call(t)) for t in sets]
+    ms, per_replay = time_back_to_back(calls, steps, max(warmup // 5, 2))
+    out = {"kernel": kind, "shape": list(shape), "us": ms * 1e3,
            "gbs": nbytes / (ms / 1e3) / 1e9, "hbm_frac": nbytes / (ms / 1e3) / 1e9 / pk["hbm"],
-           "l2": "flushed between launches"}
+           "timing": f"back to back, {nsets} buffer set(s) of {_set_bytes(t0) / 1e6:.1f} MB rotated, "
+                     f"median of {steps} graph replays of {per_replay} launches"}
+    if isolated:
+        flush = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+        ms_iso = time_isolated(calls[0], steps, warmup, flush)
+        out["us_isolated"] = ms_iso * 1e3
+        del flush
     if work:
         out["tflops"] = work / (ms / 1e3) / 1e12
         out["fp8_peak_frac"] = out["tflops"] / (2.0 * pk["bf16"])
-        out["fp8_peak"] = f"{2.0 * pk['bf16']:.0f} TFLOP/s ({pk['source']} bf16 burst x 2)"
     if sustain_s > 0:
-        fn()
+        seq = calls * max(1, -(-MIN_PER_REPLAY // len(calls)))
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for c in seq:
+                c()
+        g.replay()
         torch.cuda.synchronize()
-        n, t0 = 0, time.perf_counter()
+        n, t_start = 0, time.perf_counter()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        while time.perf_counter() - t0 < sustain_s:
-            for _ in range(20):
-                fn()
-            n += 20
+        while time.perf_counter() - t_start < sustain_s:
+            g.replay()
+            n += len(seq)
             torch.cuda.synchronize()
         b.record()
         b.synchronize()
         sus_ms = a.elapsed_time(b) / n
         out["sustained_us"] = sus_ms * 1e3
-        out["sustained_launches"] = n
         if work:
             out["sustained_tflops"] = work / (sus_ms / 1e3) / 1e12
+        del g
     st, where = fw.device_status()
     if st != 0:
         raise RuntimeError(f"device status {st} at wait site {where}")
+    del sets, calls, t0
+    torch.cuda.empty_cache()
     return out
 
 
@@ -853,8 +1062,9 @@ SWEEPS = {
     "c1": [("gemm", (m, n, synth.C1_K)) for m in synth.C1_M for n in synth.C1_N],
     "c2": [("swiglu", (m, i)) for m in synth.C2_M for i in synth.C2_I],
     "c3": [("qkv", (synth.C3["M"], synth.C3["d"], synth.C3["Nq"], synth.C3["Nk"])),
+           ("qkv_gemm", (synth.C3["M"], synth.C3["d"], synth.C3["Nq"], synth.C3["Nk"])),
            ("quant", (synth.C3["M"], synth.C3["d"]))] +
-          [("gemm", (synth.C3["M"], n, synth.C3["d"])) for n in (synth.C3["Nq"], synth.C3["Nk"], synth.C3["Nv"])],
+          [("gemm", (synth.C3["M"], n, synth.C3["d"])) for n in (synth.C3["Nq"], synth.C3["Nk"])],
     "c4": [("dual", (m, synth.C4["I"], synth.C4["d"])) for m in (1024, 4096)] +
           [("gemm", (m, synth.C4["I"], synth.C4["d"])) for m in (1024, 4096)] +
           [("gemm", (m, synth.C4["d"], synth.C4["I"])) for m in (1024, 4096)] +
@@ -869,7 +1079,46 @@ SWEEPS = {
             ("gemm_group", (4096, 1024, synth.C4["d"], synth.C4["I"])),
             ("gemm_group_ws", (4096, 1024, synth.C4["d"], synth.C4["I"])),
             ("quant_group", (4096, 1024, synth.C4["d"]))],
+    # per-token activation / per-channel weight scales at the generation tower's size
+    "per_token": [("mlp_tok", (4096, synth.C4["d"], synth.C4["I"])),
+                  ("quant_tok", (4096, synth.C4["d"])),
+                  ("swiglu_tok", (4096, synth.C4["I"])),
+                  ("gemm_scaled", (4096, synth.C4["I"], synth.C4["d"]))],
+    # cross-attention projections: generation-tower queries over understanding-tower context
+    "xattn": [("xattn", (4096, 1024, synth.C3["d"], synth.C3["Nq"], synth.C3["Nk"]))],
 }
+
+# the workloads whose figures go into the default run's line (key "configs")
+CONFIG_REPLAYS = 20
+LINE_CONFIGS = ("c0", "c1", "c2", "c3", "per_token", "xattn")
+
+
+def config_figures(fw, device, steps, warmup, log):
+    """The default run's per-workload kernel figures: every shape of the
+    Linear sweep (c1), the SwiGLU sweep (c2), the shared-quant Q/K/V block
+    (c3, whole call and its grouped GEMM alone), the tiny MLP (c0), the
+    per-token path and the cross-attention projections, each timed back to
+    back with rotating buffers and alone after an L2 flush."""
+    pk = peaks()
+    out = {"timing": f"back to back over buffer sets spanning >= {ROTATE_BYTES >> 20} MB (twice "
+                     f"the L2), median of {steps} CUDA-graph replays of >= {MIN_PER_REPLAY} "
+                     f"launches; us_isolated: one launch after a 256 MB L2 flush (includes the "
+                     f"launch latency); fractions of the measured burst peaks",
+           "peaks": {"fp8_tflops": 2.0 * pk["bf16"], "hbm_gbs": pk["hbm"],
+                     "source": f"{pk['source']}: bf16 burst x 2 for FP8; copy bandwidth"}}
+    for name in LINE_CONFIGS:
+        rows = []
+        for kind, shape in SWEEPS[name]:
+            r = kernel_bench(fw, kind, shape, steps, warmup, device)
+            keep = {k: (round(v, 4) if isinstance(v, float) else v) for k, v in r.items()
+                    if k not in ("timing",)}
+            if kind in ("swiglu", "swiglu_tok", "quant", "quant_tok"):
+                keep["hbm_nominal_frac"] = round(r["gbs"] / 8000.0, 4)
+            rows.append(keep)
+            log(f"{name} {kind} {shape}: {r['us']:.1f} us"
+                + (f", {r['tflops']:.0f} TFLOP/s" if "tflops" in r else f", {r['gbs']:.0f} GB/s"))
+        out[name] = rows
+    return out
 
 
 # -------------------------------------------------------------- dist glue
@@ -923,7 +1172,8 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None,
-                    help="timed steps (default 40 for the pass; 50 launches for --kernel/--sweep)")
+                    help="timed steps (default 120 for the pass, about 2 s; 50 graph replays "
+                         "for --kernel/--sweep)")
     ap.add_argument("--warmup", type=int, default=None,
                     help="untimed warm-up steps (default 3 for the pass; 10 launches for "
                          "--kernel/--sweep)")
@@ -931,6 +1181,8 @@ def main():
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-workload kernel figures (c0-c3, per-token, cross-attention)")
     ap.add_argument("--streams", type=int, choices=(1, 2), default=2,
                     help="towers mode: 2 runs the two towers of each layer on two streams, "
                          "joined per layer")
@@ -941,12 +1193,15 @@ def main():
                     help="time the five-kernel composition (separate gate/up GEMMs and SwiGLU-quant)")
     ap.add_argument("--kernel", choices=("gemm", "gemm_ws", "dual", "swiglu", "quant", "gemm_group",
                                          "gemm_group_ws", "dual_group", "quant_group", "scaled_mm",
-                                         "mlp", "qkv"),
+                                         "mlp", "qkv", "qkv_gemm", "mlp_tok", "quant_tok",
+                                         "swiglu_tok", "gemm_scaled", "xattn"),
                     help="time one kernel on one shape instead of the pass")
     ap.add_argument("--shape", help="M,N,K for gemm; M,I,K for dual; M,I for swiglu; M,K for quant; "
                                     "M0,M1,N,K / M0,M1,I,K / M0,M1,K for the group kinds; "
                                     "M,d,I for mlp (the fused gated MLP, three launches); "
-                                    "M,d,Nq,Nkv for qkv (shared quantize + grouped Q/K/V GEMM)")
+                                    "M,d,Nq,Nkv for qkv (shared quantize + grouped Q/K/V GEMM) "
+                                    "and qkv_gemm (the grouped GEMM alone); M,d,I for mlp_tok; "
+                                    "M,N,K for gemm_scaled; Mq,Mkv,d,Nq,Nkv for xattn")
     ap.add_argument("--mode", choices=("group", "towers"), default="group",
                     help="group: one grouped launch per step covers both towers of a layer; "
                          "towers: one launch per tower (see --streams)")
@@ -957,7 +1212,7 @@ def main():
     args = ap.parse_args()
     single = bool(args.kernel or args.sweep)
     if args.steps is None:
-        args.steps = 50 if single else 40
+        args.steps = 50 if single else 120
     if args.warmup is None:
         args.warmup = 10 if single else 3
     log = lambda m: print(m, file=sys.stderr, flush=True)  # noqa: E731
@@ -1034,7 +1289,7 @@ def main():
 
     launches_before = fw.launch_count()
     launches_per_step = sum(3 if fused else 5 for _ in value_plan)
-    sampler = ClockSampler(device.index if device.index is not None else 0)
+    sampler = clock_sampler(device.index if device.index is not None else 0)
     runner = make_stream_runner(value_plan, device) if (args.streams == 2 and not grouped) else None
     graph = None
     if grouped and not args.eager:
@@ -1047,16 +1302,18 @@ def main():
                     raise RuntimeError("launch failed")
         graph = capture_graph(run_current)
         runner = graph.replay
-    total_ms, per_kind, clocks, instrumented_ms = time_device(value_plan, args.steps,
-                                                              max(args.warmup, 3), ctx, sampler,
-                                                              runner, instr_plan=plan)
+    total_ms, clocks = time_device(value_plan, args.steps, max(args.warmup, 3), ctx, sampler,
+                                   runner)
+    # each kind's launches of the step replayed back to back (after the timed region)
+    per_kind = time_kinds(plan, args.steps)
     launches = launches_per_step * args.steps
     counted = fw.launch_count() - launches_before
-    if graph is not None:  # launches are counted when issued: the eager step and the capture
-        expect = 2 * launches_per_step + sum(1 for _ in plan) * args.steps
+    # launches are counted when issued: eager calls and captures, not graph replays
+    kinds_issued = 2 * len(plan)  # time_kinds: one eager pass and one capture of each kind
+    if graph is not None:  # the eager step before the capture, and the capture
+        expect = 2 * launches_per_step + kinds_issued
     else:
-        expect = launches_per_step * (args.steps + max(args.warmup, 3)) + \
-            sum(1 for _ in plan) * args.steps
+        expect = launches_per_step * (args.steps + max(args.warmup, 3)) + kinds_issued
     if counted != expect:
         raise RuntimeError(f"launch count {counted} != expected {expect}")
     st, where = fw.device_status()
@@ -1067,22 +1324,26 @@ def main():
     tokens = TOKENS_PER_STEP * args.steps * args.layers / LAYERS
     value = aggregate_value(tokens, ctx.world, max_ms / 1e3)
 
-    # per-kernel achieved rates from the events inside the timed region
-    comp = {"note": "per-kernel figures from a second run of the same steps with an event "
-                    "between every launch (ms_per_step there: %.3f)" % (instrumented_ms / args.steps)}
+    # per-kernel achieved rates: each kind's launches of one step replayed back to back
+    step_ms = {k: ms * n for k, (ms, n, _, _) in per_kind.items()}
+    comp = {"note": "per-kernel figures: each kind's launches of one step (one per layer, on "
+                    "that layer's buffers) captured as a CUDA graph and replayed back to back, "
+                    f"median of {args.steps} replays; no event between launches. The kinds' sum "
+                    f"is {sum(step_ms.values()):.3f} ms per step against the pass's "
+                    f"{max_ms / args.steps:.3f} ms"}
     for kind, (ms, n, nbytes, flops) in per_kind.items():
-        d = {"launches_per_step": n // args.steps, "ms_per_step": ms / args.steps,
-             "share": ms / sum(v[0] for v in per_kind.values())}
+        d = {"launches_per_step": n, "us_per_launch": ms * 1e3, "ms_per_step": step_ms[kind],
+             "share": step_ms[kind] / sum(step_ms.values())}
         if flops:
             d["tflops"] = flops / (ms / 1e3) / 1e12
         d["gbs"] = nbytes / (ms / 1e3) / 1e9
         comp[kind] = d
     # the dominant kernel: the launch shape with the largest share of the pass
     tensor_kinds = [k for k in per_kind if per_kind[k][3]]
-    dom = max(tensor_kinds, key=lambda k: per_kind[k][0])
+    dom = max(tensor_kinds, key=lambda k: step_ms[k])
     fp8_peak = 2.0 * pk["bf16_sustained"]
-    ms, n, _, flops = per_kind[dom]
-    achieved = (flops / n) / (ms / n / 1e3) / 1e12
+    ms, n, nbytes, flops = per_kind[dom]
+    achieved = flops / (ms / 1e3) / 1e12
     kind, tower = dom.split("@")
     if tower == "group":
         mrows = "+".join(f"{M} ({t})" for t, M in GROUP_ORDER)
@@ -1098,16 +1359,15 @@ def main():
     roofline = {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
                 "frac": achieved / fp8_peak, "traffic": TRAFFIC.get(dom),
                 "traffic_unit": "DRAM bytes per launch (ncu)",
-                "kernel": f"{names[kind]}, {tower_desc}, {n // args.steps} launches per step, "
-                          f"{flops / n / 1e9:.1f} GFLOP and {per_kind[dom][2] / n / 1e6:.1f} MB "
-                          "algorithmic per launch",
-                "launch_us": ms / n * 1e3,
+                "kernel": f"{names[kind]}, {tower_desc}, {n} launches per step, "
+                          f"{flops / 1e9:.1f} GFLOP and {nbytes / 1e6:.1f} MB algorithmic per launch",
+                "launch_us": ms * 1e3,
                 "peak_source": f"{pk['source']}: bf16 sustained {pk['bf16_sustained']} TFLOP/s x 2 (nominal fp8/bf16 ratio)"}
     for k in list(comp):
         if k.startswith(("swiglu", "quant")) and isinstance(comp[k], dict):
             comp[k]["hbm_frac"] = comp[k]["gbs"] / pk["hbm"]
-    all_flops = sum(v[3] for v in per_kind.values())
-    all_tensor_ms = sum(per_kind[k][0] for k in tensor_kinds)
+    all_flops = sum(v[3] * v[1] for v in per_kind.values())
+    all_tensor_ms = sum(step_ms[k] for k in tensor_kinds)
     comp["all_tensor_kernels_tflops"] = all_flops / (all_tensor_ms / 1e3) / 1e12
 
     e2e = None
@@ -1131,6 +1391,13 @@ def main():
         tps, cores, sample = cpu_baseline()
         cpu = {"value": tps, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
 
+    configs = None
+    if ctx.world == 1 and not args.no_configs:
+        del graph
+        graph = None
+        torch.cuda.empty_cache()
+        configs = config_figures(fw, device, CONFIG_REPLAYS, 10, log)
+
     if ctx.rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ctx.world,
@@ -1148,7 +1415,7 @@ def main():
                        "parallelism": f"replicas x{ctx.world}",
                        "l2": "inputs larger than L2 (8.15 GB of FP8 weights per pass)"},
             "roofline": roofline, "components": comp, "e2e": e2e, "cpu_baseline": cpu,
-            "gpu_launches": launches, "clocks": clocks,
+            "gpu_launches": launches, "clocks": clocks, "configs": configs,
         }
         print(json.dumps(line), flush=True)
     del graph

@@ -32,6 +32,7 @@ __all__ = [
     "fp8_quant_static_group", "fp8_linear_static_group", "fp8_gate_up_swiglu_static_group",
     "gated_mlp_static_fp8_group", "gated_mlp_static_fp8_group_workspace", "group_workspace_views",
     "qkv_shared_quant", "qkv_shared_quant_workspace", "fp8_shared_quant_linears",
+    "fp8_linears_static",
     "cross_attention_qkv_static_fp8", "fp8_quant_per_token", "fp8_linear_scaled",
     "silu_mul_2in_fp8_per_token", "gated_mlp_per_token_fp8",
     "fp8_check_shared_input_scale", "fp8_absmax_bf16", "fp8_silu_mul_absmax",
@@ -142,6 +143,12 @@ _SIGS = {
                                                 ctypes.POINTER(ctypes.c_int64),
                                                 ctypes.POINTER(ctypes.c_void_p),
                                                 ctypes.POINTER(ctypes.c_void_p), _P, _P]),
+    "fp8_linears_static": (ctypes.c_int, [_P, _I64, _I64, _P, ctypes.c_int,
+                                          ctypes.POINTER(ctypes.c_void_p),
+                                          ctypes.POINTER(ctypes.c_int64),
+                                          ctypes.POINTER(ctypes.c_void_p),
+                                          ctypes.POINTER(ctypes.c_void_p), _P, ctypes.c_size_t,
+                                          _P]),
     "cross_attention_qkv_static_fp8_workspace": (ctypes.c_size_t, [_I64, _I64, _I64]),
     "cross_attention_qkv_static_fp8": (ctypes.c_int, [_P, _I64, _P, _I64, _I64, _P, _P, _I64, _P,
                                                       _P, _P, _I64, _P, _P, _I64, _P, _P, _P, _P,
@@ -641,6 +648,33 @@ def fp8_shared_quant_linears(x, s_in, projections, workspace=None, out=None, str
         _check(lib.fp8_shared_quant_linears(_bf16(x, "x"), M, d, _f32(s_in, "s_in"), n, W, N, S, Y,
                                             _dev_ptr(workspace, "workspace", (torch.uint8,)),
                                             _stream(stream)), "fp8_shared_quant_linears")
+    return out
+
+
+def fp8_linears_static(xq, s_in, projections, out=None, workspace=None, stream=None):
+    """One Linear per (W [N,K] FP8, s_w) in projections over an activation
+    xq [M,K] already quantized at s_in; grouped launches of up to three.
+    workspace (optional, fp8_linear_static_ws_bytes()) lets long-K tails split."""
+    lib = load()
+    M, K = xq.shape
+    n = len(projections)
+    for i, (w, _) in enumerate(projections):
+        if w.dim() != 2 or w.shape[1] != K:
+            raise ValueError(f"projection {i} must be [N, {K}]")
+    if out is None:
+        out = [torch.empty((M, w.shape[0]), dtype=torch.bfloat16, device=xq.device)
+               for w, _ in projections]
+    W = (ctypes.c_void_p * n)(*[_fp8(w, f"W[{i}]") for i, (w, _) in enumerate(projections)])
+    N = (ctypes.c_int64 * n)(*[w.shape[0] for w, _ in projections])
+    S = (ctypes.c_void_p * n)(*[_f32(sw, f"s_w[{i}]") for i, (_, sw) in enumerate(projections)])
+    Y = (ctypes.c_void_p * n)(*[_bf16(y, f"y[{i}]") for i, y in enumerate(out)])
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr = _dev_ptr(workspace, "workspace", (torch.uint8,))
+        ws_bytes = workspace.numel()
+    with _device_of(xq):
+        _check(lib.fp8_linears_static(_fp8(xq, "xq"), M, K, _f32(s_in, "s_in"), n, W, N, S, Y,
+                                      ws_ptr, ws_bytes, _stream(stream)), "fp8_linears_static")
     return out
 
 

@@ -1173,6 +1173,34 @@ int fp8_shared_quant_linears(const uint16_t *x, int64_t M, int64_t dm, const flo
   return rc;
 }
 
+int fp8_linears_static(const uint8_t *xq, int64_t M, int64_t K, const float *s_in, int n,
+                       const uint8_t *const *W, const int64_t *N, const float *const *s_w,
+                       uint16_t *const *y, void *workspace, size_t workspace_bytes,
+                       void *stream) {
+  if (n < 1 || n > FP8WS_MAX_PROJECTIONS) return FP8WS_ERR_SHAPE;
+  if (!W || !N || !s_w || !y) return FP8WS_ERR_NULL;
+  if (workspace && ((reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+                    workspace_bytes < splitk_bytes()))
+    return FP8WS_ERR_WORKSPACE;
+  PairProblem pp[FP8WS_MAX_PROJECTIONS];
+  for (int i = 0; i < n; ++i) {
+    const int rc = check_gemm_args(xq, W[i], M, N[i], K, s_in, s_w[i], y[i]);
+    if (rc) return rc;
+    pp[i] = PairProblem{xq, W[i], nullptr, y[i], static_cast<int>(M), static_cast<int>(N[i]), s_in,
+                        s_w[i], nullptr, nullptr};
+  }
+  DeviceInfo *d;
+  int rc = device_info(&d);
+  if (rc) return rc;
+  if (M == 0) return FP8WS_OK;
+  cudaStream_t st = as_stream(stream);
+  if (workspace &&
+      cudaMemsetAsync(splitk_counters(workspace), 0, kSplitkCounterWords * sizeof(int), st) !=
+          cudaSuccess)
+    return FP8WS_ERR_CUDA;
+  return gemm_groups(d, pp, n, static_cast<int>(K), st, workspace);
+}
+
 size_t cross_attention_qkv_static_fp8_workspace(int64_t Mq, int64_t Mkv, int64_t d) {
   if (Mq < 0 || Mkv < 0 || d < 0) return 0;
   return ws_saturate(ws_region(Mq, d) + ws_region(Mkv, d) + splitk_bytes());

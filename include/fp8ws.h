@@ -452,6 +452,30 @@ FP8WS_API int fp8_shared_quant_linears(const uint16_t *x, int64_t M, int64_t d, 
                                        void *workspace, void *stream);
 
 /*
+ * fp8_linears_static -- n Linears over one activation that the caller has
+ * already quantized at s_in (with fp8_quant_static, or with a kernel of its
+ * own that writes the same codes): fp8_shared_quant_linears without its
+ * quantize launch.  [PR] What changed: the members of a formerly fused group
+ * consume one quantized activation; their calibrated input scales must agree
+ * (fp8_check_shared_input_scale).  The projections run in grouped GEMM
+ * launches of up to three (Q, K and V in one launch).
+ * xq: device [M,K] FP8.  s_in: device fp32.  W, N, s_w, y: host arrays of n
+ * (1..FP8WS_MAX_PROJECTIONS): W[i] device [N[i],K] FP8, s_w[i] device fp32,
+ * y[i] device [M,N[i]] BF16, contiguous.
+ * workspace: NULL (no split over K), or device, >= fp8_linear_static_ws_bytes()
+ * bytes, 256-byte aligned, which lets the tiles past the last full wave of a
+ * long-K launch split over K as in fp8_linear_static_ws (the call clears its
+ * counters first).
+ * Errors: those of fp8_linear_static for each projection, FP8WS_ERR_SHAPE for
+ * n out of range, FP8WS_ERR_NULL for a NULL host array, FP8WS_ERR_WORKSPACE
+ * for a misaligned or short workspace; all found before anything is enqueued.
+ */
+FP8WS_API int fp8_linears_static(const uint8_t *xq, int64_t M, int64_t K, const float *s_in,
+                                 int n, const uint8_t *const *W, const int64_t *N,
+                                 const float *const *s_w, uint16_t *const *y, void *workspace,
+                                 size_t workspace_bytes, void *stream);
+
+/*
  * cross_attention_qkv_static_fp8 -- projections of a cross-attention: Q from
  * the query-side activation x, K and V from a different tensor ctx.  [PR] Test
  * Coverage: where K/V come from another tensor, sharing must not engage

@@ -96,6 +96,24 @@ def test_noalloc_refuses_before_cuda(lib, M, d, I):
     assert lib.fp8ws_launch_count() == n0
 
 
+def test_linears_static_argument_checks(lib):
+    """fp8_linears_static refuses bad arguments before any CUDA call."""
+    import ctypes as C
+    a = 1 << 20
+    W = (C.c_void_p * 2)(a, a)
+    N = (C.c_int64 * 2)(256, 256)
+    S = (C.c_void_p * 2)(a, a)
+    Y = (C.c_void_p * 2)(a, a)
+    assert lib.fp8_linears_static(a, 64, 256, a, 0, W, N, S, Y, None, 0, None) == fw.ERR_SHAPE
+    assert lib.fp8_linears_static(a, 64, 256, a, 17, W, N, S, Y, None, 0, None) == fw.ERR_SHAPE
+    assert lib.fp8_linears_static(a, 64, 256, a, 2, None, N, S, Y, None, 0, None) == fw.ERR_NULL
+    bad_n = (C.c_int64 * 2)(256, 100)  # N % 8 != 0
+    assert lib.fp8_linears_static(a, 64, 256, a, 2, W, bad_n, S, Y, None, 0, None) == fw.ERR_SHAPE
+    assert lib.fp8_linears_static(a + 8, 64, 256, a, 2, W, N, S, Y, None, 0, None) == fw.ERR_ALIGN
+    assert lib.fp8_linears_static(a, 64, 256, a, 2, W, N, S, Y, a + 16, 1 << 30, None) == \
+        fw.ERR_WORKSPACE
+
+
 def test_argument_checks_before_cuda(lib):
     """Null pointers, bad sizes and misaligned pointers are refused before any
     CUDA call, so these run without a GPU."""

@@ -123,3 +123,29 @@ def test_cross_attention_with_an_empty_side(Mq, Mkv):
         ref_k, ref_v = oracle.qkv_shared_quant(bits(ctx), s_kv, [_ref(wk), _ref(wv)])
         assert rel_fro(bits(k), ref_k) <= GEMM_REL_FRO and rel_fro(bits(v), ref_v) <= GEMM_REL_FRO
     assert fw.device_status()[0] == fw.OK
+
+
+@pytest.mark.parametrize("M,Ns", [(2048, (3072, 1024, 1024)),          # the c3 projections
+                                  (300, (512, 256, 768, 128, 1024, 64, 320))])
+def test_linears_over_a_prequantized_activation(M, Ns):
+    """fp8_linears_static on the caller's own Xq gives the outputs of the
+    shared-quant call (which quantizes first) bit for bit, and the oracle's
+    on sampled rows."""
+    d = 3072 if M == 2048 else 272
+    x = synth.activation_with_outliers(M, d, 5, 8, 0, DEV)
+    s = oracle.f32(0.029)
+    ws = [_proj(n, d, 600 + i) for i, n in enumerate(Ns)]
+    ref = fw.fp8_shared_quant_linears(x, scalar(s, DEV), ws)
+    xq = fw.fp8_quant_static(x, scalar(s, DEV))
+    fw.launch_log_clear()
+    got = fw.fp8_linears_static(xq, scalar(s, DEV), ws)
+    log = fw.launch_log()
+    assert all(r[0] == fw.KIND_GEMM and r[1] == xq.data_ptr() for r in log)
+    assert len(log) == len(Ns)
+    for g, r in zip(got, ref):
+        assert torch.equal(g.view(torch.int16), r.view(torch.int16))
+    rows = stratified_rows(M, 9)
+    refs = oracle.qkv_shared_quant(bits(x[rows]), s, [_ref(w) for w in ws])
+    for g, r in zip(got, refs):
+        assert rel_fro(bits(g[rows]), r) <= GEMM_REL_FRO
+    assert fw.device_status()[0] == fw.OK
