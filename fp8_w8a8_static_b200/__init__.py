@@ -178,8 +178,8 @@ _SIGS = {
     "fp8ws_gemm_plan": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int64),
                                        ctypes.POINTER(ctypes.c_int64), ctypes.c_int,
                                        ctypes.POINTER(ctypes.c_int)]),
-    "fp8ws_split_plan": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int]
-                         + [ctypes.POINTER(ctypes.c_int)] * 4),
+    "fp8ws_split_plan": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+                         + [ctypes.POINTER(ctypes.c_int)] * 5),
     "fp8ws_launch_count": (ctypes.c_int64, []),
     "fp8ws_launch_log": (ctypes.c_int, [ctypes.POINTER(LaunchRecord), ctypes.c_int]),
     "fp8ws_launch_log_clear": (None, []),
@@ -876,13 +876,16 @@ def gemm_plan(shapes, sms: int = 148, pairs: int = 74) -> str:
     return {v: k for k, v in GEMM_CONFIGS.items()}[cfg.value]
 
 
-def split_plan(tiles: int, pairs: int, num_kb: int) -> dict:
-    """The CTA-pair GEMM's split-K plan (host only): dp_tiles whole tiles, then
-    split_tiles tiles cut into `splits` K ranges of kb_per_split steps."""
-    out = [ctypes.c_int() for _ in range(4)]
-    _check(load().fp8ws_split_plan(tiles, pairs, num_kb, *[ctypes.byref(o) for o in out]),
-           "fp8ws_split_plan")
-    return dict(zip(("dp_tiles", "split_tiles", "splits", "kb_per_split"), (o.value for o in out)))
+def split_plan(tiles: int, pairs: int, num_kb: int, scratch: bool = True) -> dict:
+    """The CTA-pair GEMM's plan past its last full wave (host only): dp_tiles
+    whole tiles, then split_tiles tiles each cut into `splits` K ranges of
+    kb_per_split steps (needs scratch), or run as two 256x128 halves when
+    halves == 2."""
+    out = [ctypes.c_int() for _ in range(5)]
+    _check(load().fp8ws_split_plan(tiles, pairs, num_kb, int(scratch),
+                                   *[ctypes.byref(o) for o in out]), "fp8ws_split_plan")
+    return dict(zip(("dp_tiles", "split_tiles", "splits", "kb_per_split", "halves"),
+                    (o.value for o in out)))
 
 
 def launch_count() -> int:

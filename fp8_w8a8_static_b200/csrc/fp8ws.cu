@@ -300,13 +300,24 @@ int *splitk_counters(void *splitk) {
 // its fixed cost (the fp32 partial stores, the wait for the last split, its
 // reduction).  Timed on B200: splitting the ragged wave 4 ways saved 9 us at
 // K = 12288 (96 K steps per tile) and cost 6 us at K = 3072 (24 K steps).
+// Otherwise, when the remainder would fill at most half a wave, each of its
+// tiles runs as two 256 x 128 halves instead (no scratch needed): the last
+// wave then takes a half tile's time, not a whole one's.
 constexpr int kSplitkMinKb = 64;
 
 SplitPlan make_split_plan(int tiles, int pairs, int num_kb, float *partials, int *counters) {
-  SplitPlan p{tiles, 0, 1, num_kb, nullptr, nullptr};
-  if (!partials || pairs < 1 || tiles % pairs == 0 || num_kb < kSplitkMinKb) return p;
+  SplitPlan p{tiles, 0, 1, num_kb, nullptr, nullptr, 1};
+  if (pairs < 1 || tiles % pairs == 0) return p;
   const int R = tiles % pairs;
-  if (R > kSplitkTiles) return p;
+  const bool k_split_possible = partials && num_kb >= kSplitkMinKb && R <= kSplitkTiles;
+  if (!k_split_possible) {
+    if (2 * R <= pairs) {
+      p.dp_tiles = tiles - R;
+      p.split_tiles = R;
+      p.halves = 2;
+    }
+    return p;
+  }
   int best_s = 1;
   double best = 1.0;
   for (int S = 2; S <= 4; ++S) {
@@ -363,6 +374,10 @@ PairGroup make_pair_group(const PairProblem *pp, int np, int tile_m, int tile_n)
     // column within groups of kGroupM row blocks: each B column block is read
     // once per group and A is re-read from L2.
     G.group_m[p] = q.M > static_cast<int64_t>(q.N) * (q.b2 ? 2 : 1) ? 1 : kGroupM;
+    // Row by row, each A row block is consumed within a wave and B is read
+    // again by every wave; column by column within row groups, the other way
+    // round.  The operand consumed within a wave is loaded evict-first.
+    G.hint[p] = G.group_m[p] == 1 ? kHintAFirst : kHintBFirst;
     G.s_in[p] = q.s_in;
     G.s_w[p] = q.s_w;
     G.s_w2[p] = q.s_w2;
@@ -410,12 +425,16 @@ int launch_gemm_pair_cfg(DeviceInfo *d, const PairProblem *pp, int np, int K, cu
   auto kern = fp8_gemm_pair_kernel<STAGES, SCALE_MODE, DIRECT>;
   int rc = pair_clusters(d, kern, kGemmThreads, C::SMEM_BYTES, BIT, &d->pair_clusters);
   if (rc) return rc;
-  CUtensorMap ma[kMaxGroup], mb[kMaxGroup], md[kMaxGroup];
+  // B is mapped twice: 128-row boxes for whole tiles, 64-row boxes for the
+  // 256 x 128 halves of a ragged last wave
+  CUtensorMap ma[kMaxGroup], mb[kMaxGroup], mbh[kMaxGroup], md[kMaxGroup];
   for (int p = 0; p < np && !rc; ++p) {
     const PairProblem &q = pp[p];
     rc = make_map_2d(&ma[p], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.a, q.M, K, kGemmBK, 128, true);
     if (!rc)
       rc = make_map_2d(&mb[p], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.b, q.N, K, kGemmBK, 128, true);
+    if (!rc)
+      rc = make_map_2d(&mbh[p], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.b, q.N, K, kGemmBK, 64, true);
     if (!rc)
       rc = make_map_2d(&md[p], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q.out, q.M, q.N, C::EPI_COLS,
                        32, false);
@@ -424,6 +443,7 @@ int launch_gemm_pair_cfg(DeviceInfo *d, const PairProblem *pp, int np, int K, cu
   for (int p = np; p < kMaxGroup; ++p) {  // absent problems: copies, never used
     ma[p] = ma[0];
     mb[p] = mb[0];
+    mbh[p] = mbh[0];
     md[p] = md[0];
   }
   const PairGroup G = make_pair_group(pp, np, kPairTile, kPairTile);
@@ -433,12 +453,12 @@ int launch_gemm_pair_cfg(DeviceInfo *d, const PairProblem *pp, int np, int K, cu
   const SplitPlan plan =
       make_split_plan(tiles, d->pair_clusters.load(std::memory_order_relaxed),
                       (K + kGemmBK - 1) / kGemmBK, partials, counters);
-  const int units = plan.dp_tiles + plan.split_tiles * plan.splits;
+  const int units = plan.dp_tiles + plan.split_tiles * plan.splits * plan.halves;
   const int resident = d->pair_clusters.load(std::memory_order_relaxed);
   const int clusters = units < resident ? units : resident;
   if (launch_ex(kern, dim3(2 * clusters), dim3(kGemmThreads), C::SMEM_BYTES, st, 2, ma[0], ma[1],
-                ma[2], mb[0], mb[1], mb[2], md[0], md[1], md[2], G, K, kWaitLimitNs,
-                plan) != cudaSuccess)
+                ma[2], mb[0], mb[1], mb[2], mbh[0], mbh[1], mbh[2], md[0], md[1], md[2], G, K,
+                kWaitLimitNs, plan) != cudaSuccess)
     return FP8WS_ERR_CUDA;
   for (int p = 0; p < np; ++p) log_launch(kKindGemm, pp[p].a, pp[p].b, pp[p].out, p);
   return launch_status();
@@ -563,7 +583,13 @@ int gemm_cost_choice(int sms, int pairs, const int64_t *M, const int64_t *N, int
     t_128 += m128 * ((N[p] + 127) / 128);
     t_64 += m128 * ((N[p] + 63) / 64);
   }
-  const double est_pair = waves(t_pair, pairs) * (128.0 * 256) / 1.0;
+  // CTA pairs: the full waves, then a ragged remainder that fills at most half
+  // a wave runs as 256 x 128 halves, taken at 0.7 of a whole tile's time (a
+  // half tile moves 3/4 of a whole tile's operand bytes per K step)
+  const int64_t rem = t_pair % pairs;
+  const double pair_waves = static_cast<double>(t_pair / pairs) +
+                            (rem == 0 ? 0.0 : (2 * rem <= pairs ? 0.7 : 1.0));
+  const double est_pair = pair_waves * (128.0 * 256) / 1.0;
   const double est_256 = waves(t_256, sms) * (128.0 * 256) / 0.85;
   const double est_128 = waves(t_128, sms) * (128.0 * 128) / 0.45;
   const double est_64 = waves(t_64, sms) * (128.0 * 64) / 0.25;
@@ -1494,17 +1520,19 @@ int fp8ws_gemm_plan(int sms, int pairs, const int64_t *M, const int64_t *N, int 
   return FP8WS_OK;
 }
 
-int fp8ws_split_plan(int tiles, int pairs, int num_kb, int *dp_tiles, int *split_tiles,
-                     int *splits, int *kb_per_split) {
-  if (!dp_tiles || !split_tiles || !splits || !kb_per_split) return FP8WS_ERR_NULL;
+int fp8ws_split_plan(int tiles, int pairs, int num_kb, int has_scratch, int *dp_tiles,
+                     int *split_tiles, int *splits, int *kb_per_split, int *halves) {
+  if (!dp_tiles || !split_tiles || !splits || !kb_per_split || !halves) return FP8WS_ERR_NULL;
   if (tiles < 0 || pairs < 1 || num_kb < 1) return FP8WS_ERR_SHAPE;
-  // the plan only needs to know that scratch exists; it is not dereferenced here
+  // the plan only needs to know whether scratch exists; it is not dereferenced here
   float scratch_tag = 0.0f;
-  const SplitPlan p = make_split_plan(tiles, pairs, num_kb, &scratch_tag, nullptr);
+  const SplitPlan p =
+      make_split_plan(tiles, pairs, num_kb, has_scratch ? &scratch_tag : nullptr, nullptr);
   *dp_tiles = p.dp_tiles;
   *split_tiles = p.split_tiles;
   *splits = p.splits;
   *kb_per_split = p.kb_per_split;
+  *halves = p.halves;
   return FP8WS_OK;
 }
 

@@ -16,9 +16,12 @@
 //   warps 2..5  epilogue (both CTAs)
 // The tiles of the group form one sequence (problem 0's, then problem 1's,
 // ...), dealt round-robin to the clusters, so each problem fills the ragged
-// last wave of the one before.  Bounded waits as in fp8_gemm_kernel.  Both CTAs always reach the final
-// cluster barrier, so neither leaves while its peer may still touch its
-// shared memory or TMEM.
+// last wave of the one before.  What remains past the last full wave may be
+// split over K (SplitPlan) or, when it would fill at most half a wave, cut
+// into 256 x 128 halves (an N = 128 MMA over 64 rows of B per CTA), so that
+// the last wave runs twice as many, shorter, units.  Bounded waits as in
+// fp8_gemm_kernel.  Both CTAs always reach the final cluster barrier, so
+// neither leaves while its peer may still touch its shared memory or TMEM.
 #pragma once
 
 #include "common.cuh"
@@ -42,12 +45,21 @@ struct PairGroup {
   int num_m[kMaxGroup];
   int num_n[kMaxGroup];
   int group_m[kMaxGroup];  // raster: row blocks per column-major group (1 = row-major)
+  int hint[kMaxGroup];     // L2 policy of the loads: kHintNone, kHintAFirst or kHintBFirst
   const float *s_in[kMaxGroup];
   const float *s_w[kMaxGroup];
   const float *s_w2[kMaxGroup];
   const float *s_down[kMaxGroup];
   void *out[kMaxGroup];
 };
+
+// L2 eviction priority of a problem's operand loads.  The operand that the
+// tile order consumes within one wave (A when the tiles run row by row, B
+// when they run column by column within row groups) is loaded evict-first,
+// so that it leaves L2 before the operand the next waves read again.
+constexpr int kHintNone = 0;
+constexpr int kHintAFirst = 1;
+constexpr int kHintBFirst = 2;
 
 struct GroupTile {
   int p;
@@ -74,6 +86,8 @@ __device__ __forceinline__ GroupTile group_tile(int g, const PairGroup &G) {
 // last split of a tile to finish, told apart by a per-warp counter in
 // `counters` (zero before the launch, reset to zero by that last split), adds
 // the partials in split order and runs the epilogue.  splits == 1: no split.
+// halves == 2 (then splits == 1): the last split_tiles tiles are each cut
+// into two 256 x 128 units over the full K instead (no partials).
 struct SplitPlan {
   int dp_tiles;
   int split_tiles;
@@ -81,10 +95,12 @@ struct SplitPlan {
   int kb_per_split;
   float *partials;  // [split_tiles * splits] slots, see partial_index
   int *counters;    // [split_tiles][2][4]
+  int halves;       // 1, or 2: the remainder tiles run as 256 x 128 halves
 };
 
 struct UnitRange {
   int tile, kb0, kb1, split, slot;  // split < 0: a whole tile
+  int half;                         // -1: all 256 columns; 0 / 1: columns 0-127 / 128-255
 };
 
 // A slot holds one CTA pair's 2 x 128 x 256 fp32 partial as float4s indexed
@@ -95,12 +111,28 @@ __device__ __forceinline__ size_t partial_index(int slot, int rank, int chunk, i
 }
 
 __device__ __forceinline__ UnitRange unit_range(int u, const SplitPlan &p, int num_kb) {
-  if (u < p.dp_tiles) return UnitRange{u, 0, num_kb, -1, -1};
+  if (u < p.dp_tiles) return UnitRange{u, 0, num_kb, -1, -1, -1};
   const int j = u - p.dp_tiles;
+  if (p.halves == 2) return UnitRange{p.dp_tiles + (j >> 1), 0, num_kb, -1, -1, j & 1};
   const int sp = j % p.splits;
   const int kb0 = sp * p.kb_per_split;
   const int kb1 = min(kb0 + p.kb_per_split, num_kb);
-  return UnitRange{p.dp_tiles + j / p.splits, kb0, kb1, sp, j};
+  return UnitRange{p.dp_tiles + j / p.splits, kb0, kb1, sp, j, -1};
+}
+
+__device__ __forceinline__ int plan_units(const SplitPlan &p) {
+  return p.dp_tiles + p.split_tiles * p.splits * p.halves;
+}
+
+// First output column of a unit, and whether it has any column inside N (the
+// second half of a tile in the last, ragged column block may have none; every
+// role skips such a unit alike).
+__device__ __forceinline__ int unit_col0(const UnitRange &ur, const GroupTile &gt) {
+  return gt.tc.n * kPairTile + (ur.half > 0 ? kPairTile / 2 : 0);
+}
+__device__ __forceinline__ bool unit_live(const UnitRange &ur, const GroupTile &gt,
+                                          const PairGroup &G) {
+  return ur.half <= 0 || unit_col0(ur, gt) < pick(G.N, gt.p);
 }
 
 // Scale modes of the epilogue: bit 0 = one activation scale per row
@@ -120,6 +152,7 @@ struct PairCfg {
   static constexpr int B_BYTES = 128 * kGemmBK;   // this CTA's half of B
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TX_BYTES = 2 * STAGE_BYTES;  // both CTAs, counted at the leader
+  static constexpr int TX_HALF_BYTES = 2 * (A_BYTES + B_BYTES / 2);  // a 256 x 128 unit
   static constexpr int EPI_COLS = 64;
   static constexpr int EPI_BUF_BYTES = 32 * EPI_COLS * 2;
   static constexpr int EPI_BYTES = DIRECT ? 0 : 4 * 2 * EPI_BUF_BYTES;
@@ -138,6 +171,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                          const __grid_constant__ CUtensorMap tm_b0,
                          const __grid_constant__ CUtensorMap tm_b1,
                          const __grid_constant__ CUtensorMap tm_b2,
+                         const __grid_constant__ CUtensorMap tm_bh0,
+                         const __grid_constant__ CUtensorMap tm_bh1,
+                         const __grid_constant__ CUtensorMap tm_bh2,
                          const __grid_constant__ CUtensorMap tm_d0,
                          const __grid_constant__ CUtensorMap tm_d1,
                          const __grid_constant__ CUtensorMap tm_d2, const PairGroup G, int K,
@@ -165,7 +201,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int cluster = blockIdx.x >> 1;
   const int nclusters = gridDim.x >> 1;
   const int num_kb = (K + kGemmBK - 1) / kGemmBK;
-  const int num_units = plan.dp_tiles + plan.split_tiles * plan.splits;
+  const int num_units = plan_units(plan);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -192,6 +228,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tma_prefetch_desc(&tm_b2);
       tma_prefetch_desc(&tm_d2);
     }
+    if (plan.halves == 2) {
+      tma_prefetch_desc(&tm_bh0);
+      if (G.n > 1) tma_prefetch_desc(&tm_bh1);
+      if (G.n > 2) tma_prefetch_desc(&tm_bh2);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
@@ -210,13 +251,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t stage = 0, phase = 0;
       uint32_t issued_mask = 0, issued_parity = 0;
       bool ok = true;
+      const uint64_t pol_first = l2_policy_evict_first();
+      const uint64_t pol_normal = l2_policy_evict_normal();
       for (int u = cluster; u < num_units && ok; u += nclusters) {
         const UnitRange ur = unit_range(u, plan, num_kb);
         const GroupTile gt = group_tile(ur.tile, G);
+        if (!unit_live(ur, gt, G)) continue;
+        const bool half = ur.half >= 0;
         const CUtensorMap *tm_a = gt.p == 2 ? &tm_a2 : (gt.p ? &tm_a1 : &tm_a0);
-        const CUtensorMap *tm_b = gt.p == 2 ? &tm_b2 : (gt.p ? &tm_b1 : &tm_b0);
+        const CUtensorMap *tm_b = half ? (gt.p == 2 ? &tm_bh2 : (gt.p ? &tm_bh1 : &tm_bh0))
+                                       : (gt.p == 2 ? &tm_b2 : (gt.p ? &tm_b1 : &tm_b0));
+        const int hint = pick(G.hint, gt.p);
+        const uint64_t pol_a = hint == kHintAFirst ? pol_first : pol_normal;
+        const uint64_t pol_b = hint == kHintBFirst ? pol_first : pol_normal;
         const int a_row = gt.tc.m * kPairTile + static_cast<int>(rank) * 128;
-        const int b_row = gt.tc.n * kPairTile + static_cast<int>(rank) * 128;
+        // a half unit: 64 rows of B per CTA (N = 128 over the pair)
+        const int b_row = unit_col0(ur, gt) + static_cast<int>(rank) * (half ? 64 : 128);
+        const uint32_t tx = half ? C::TX_HALF_BYTES : C::TX_BYTES;
         for (int kb = ur.kb0; kb < ur.kb1; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, timeout_ns)) {
             record_timeout(kSiteProducerEmpty);
@@ -225,9 +276,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           const uint32_t full_leader = map_shared_rank(smem_u32(&full[stage]), 0);
-          if (leader) mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
-          tma_load_2d_pair(sA + stage * C::A_BYTES, tm_a, full_leader, kb * kGemmBK, a_row);
-          tma_load_2d_pair(sB + stage * C::B_BYTES, tm_b, full_leader, kb * kGemmBK, b_row);
+          if (leader) mbar_arrive_expect_tx(&full[stage], tx);
+          tma_load_2d_pair_hint(sA + stage * C::A_BYTES, tm_a, full_leader, kb * kGemmBK, a_row,
+                                pol_a);
+          tma_load_2d_pair_hint(sB + stage * C::B_BYTES, tm_b, full_leader, kb * kGemmBK, b_row,
+                                pol_b);
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -248,12 +301,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------- MMA issue (leader)
     if (lane == 0 && leader) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(kPairTile, kPairTile);
+      constexpr uint32_t idesc_full = idesc_e4m3_f32(kPairTile, kPairTile);
+      constexpr uint32_t idesc_half = idesc_e4m3_f32(kPairTile, kPairTile / 2);
       uint32_t stage = 0, phase = 0;
       uint32_t it = 0;
       bool ok = true;
-      for (int u = cluster; u < num_units && ok; u += nclusters, ++it) {
+      for (int u = cluster; u < num_units && ok; u += nclusters) {
         const UnitRange ur = unit_range(u, plan, num_kb);
+        if (!unit_live(ur, group_tile(ur.tile, G), G)) continue;
+        const uint32_t idesc = ur.half >= 0 ? idesc_half : idesc_full;
         const uint32_t acc = it & 1u;
         const uint32_t acc_phase = (it >> 1) & 1u;
         if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, timeout_ns)) {
@@ -286,6 +342,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
         if (ok) umma_commit_pair(&tfull[acc], 0x3);
+        ++it;
       }
       umma_commit_pair(drain, 0x1);
       int zero = 0;
@@ -297,9 +354,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int ew = warp - 2;
     const int quarter = warp & 3;
     uint32_t it = 0, chunk = 0;
-    for (int u = cluster; u < num_units; u += nclusters, ++it) {
+    for (int u = cluster; u < num_units; u += nclusters) {
       const UnitRange ur = unit_range(u, plan, num_kb);
       const GroupTile gt = group_tile(ur.tile, G);
+      if (!unit_live(ur, gt, G)) continue;
       const TileCoord tc = gt.tc;
       const int M = pick(G.M, gt.p);
       const int N = pick(G.N, gt.p);
@@ -309,6 +367,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint16_t *y_out = static_cast<uint16_t *>(pick(G.out, gt.p));
       const uint32_t acc = it & 1u;
       const uint32_t acc_phase = (it >> 1) & 1u;
+      ++it;
       if (!mbar_wait_bounded_warp(&tfull[acc], acc_phase, abort_flag, timeout_ns)) {
         if (lane == 0) {
           record_timeout(kSiteEpiTmemFull);
@@ -363,9 +422,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       const uint32_t t_row =
           tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kPairTile;
-      constexpr int NCHUNK = kPairTile / C::EPI_COLS;
+      // 64-column chunks of this unit: 4 for a whole tile, 2 for a half
+      const int nchunk = (ur.half >= 0 ? kPairTile / 2 : kPairTile) / C::EPI_COLS;
 #pragma unroll 1
-      for (int c = 0; c < NCHUNK; ++c) {
+      for (int c = 0; c < nchunk; ++c) {
         uint32_t r0[32], r1[32];
         tmem_ld_32x32b_x32(t_row + c * C::EPI_COLS, r0);
         tmem_ld_32x32b_x32(t_row + c * C::EPI_COLS + 32, r1);
@@ -405,12 +465,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             r1[e] = __float_as_uint(v[32 + e]);
           }
         }
-        if (c == NCHUNK - 1) {
+        if (c == nchunk - 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(map_shared_rank(smem_u32(&tempty[acc]), 0));
         }
-        const int col0 = tc.n * kPairTile + c * C::EPI_COLS;
+        const int col0 = unit_col0(ur, gt) + c * C::EPI_COLS;
         if (col0 >= N || row0 >= M) continue;  // whole chunk outside Y
         // per-column scales of this chunk: lane l holds columns l and 32 + l
         float cs0 = 0.0f, cs1 = 0.0f;

@@ -616,16 +616,20 @@ FP8WS_API int fp8ws_set_gemm_config(int config);
 FP8WS_API int fp8ws_gemm_plan(int sms, int pairs, const int64_t *M, const int64_t *N, int count,
                               int *config);
 
-/* The split-K plan of the CTA-pair GEMM (fp8_linear_static_ws and the
- * grouped projection GEMMs that receive split-K scratch), for tests and
- * tuning; host only, touches no device.  For `tiles` 256x256 tiles on `pairs`
- * resident CTA pairs with `num_kb` 128-byte K steps per tile: the first
- * *dp_tiles tiles run whole, and the last *split_tiles are each cut into
- * *splits K ranges of *kb_per_split steps (*splits == 1: no split).  Tiles of
- * fewer than 64 K steps are never split.  FP8WS_ERR_NULL for a NULL output,
- * FP8WS_ERR_SHAPE for tiles < 0, pairs < 1 or num_kb < 1. */
-FP8WS_API int fp8ws_split_plan(int tiles, int pairs, int num_kb, int *dp_tiles, int *split_tiles,
-                               int *splits, int *kb_per_split);
+/* The plan of the CTA-pair GEMM for the tiles past its last full wave, for
+ * tests and tuning; host only, touches no device.  For `tiles` 256x256 tiles
+ * on `pairs` resident CTA pairs with `num_kb` 128-byte K steps per tile, with
+ * split-K scratch (has_scratch != 0: fp8_linear_static_ws and the composite
+ * calls that carry scratch) or without: the first *dp_tiles tiles run whole,
+ * and each of the last *split_tiles is either cut into *splits K ranges of
+ * *kb_per_split steps (needs scratch; tiles of fewer than 64 K steps are
+ * never split), or, when *halves == 2, run as two 256x128 halves over the
+ * full K (chosen when no K split is made and the remainder fills at most half
+ * a wave).  *splits == 1 and *halves == 1: every tile runs whole.
+ * FP8WS_ERR_NULL for a NULL output, FP8WS_ERR_SHAPE for tiles < 0, pairs < 1
+ * or num_kb < 1. */
+FP8WS_API int fp8ws_split_plan(int tiles, int pairs, int num_kb, int has_scratch, int *dp_tiles,
+                               int *split_tiles, int *splits, int *kb_per_split, int *halves);
 
 /* Launch log.  Every kernel the library enqueues is counted and recorded in a
  * small ring (the most recent FP8WS_LOG_CAPACITY records).  kind: 1 quant,

@@ -162,3 +162,50 @@ def test_split_k_short_workspace_refused():
     ws = torch.empty(1024, dtype=torch.uint8, device=DEV)
     with pytest.raises(fw.FP8WSError):
         fw.fp8_linear_static_ws(xq, xq, scalar(1.0, DEV), scalar(1.0, DEV), workspace=ws)
+
+
+# ----------------------------------------------------- ragged last wave: halves
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (256, 19008, 256),   # 75 tiles: the 75th (64 columns) runs as halves, its second one empty
+    (512, 19200, 512),   # 150 tiles: the last 2 run as halves, both halves full
+    (2048, 3072, 3072),  # 96 tiles: 22 past the first wave, 44 halves (the c3 Q projection)
+    (300, 520, 1040),    # 6 tiles, one partial wave: 12 units; the 8-column block's second half empty
+    (96, 4104, 512),     # ragged M and N: 17 tiles, the last one 8 columns wide
+])
+def test_tail_halves_against_oracle(M, N, K):
+    """Shapes whose tiles past the last full wave run as 256x128 halves (the
+    plan is checked on the host first), against the oracle on every row or
+    on stratified rows, under the per-element bound."""
+    fw.set_gemm_config("pair256")
+    try:
+        tiles = -(-M // 256) * -(-N // 256)
+        assert fw.split_plan(tiles, 74, -(-K // 128), scratch=False)["halves"] == 2
+        rng = np.random.default_rng(M + N + K)
+        xq = _random_codes(rng, (M, K))
+        wq = _random_codes(rng, (N, K), 0.5)
+        rows = stratified_rows(M, 3) if M * N * K > 2 ** 31 else None
+        _run(xq, wq, oracle.f32(0.011), oracle.f32(0.0023), rows=rows)
+    finally:
+        fw.set_gemm_config("auto")
+    assert fw.device_status()[0] == fw.OK
+
+
+@pytest.mark.parametrize("x_rows,w_cols", [(False, False), (True, False), (False, True),
+                                           (True, True)])
+def test_tail_halves_vector_scales(x_rows, w_cols):
+    """The four scale modes of the epilogue on half units: 300 x 520 (6 tiles,
+    one partial wave, all run as halves), per-row and per-column scales
+    checked against the oracle's fp64 sum on every element."""
+    M, N, K = 300, 520, 272
+    rng = np.random.default_rng(17 + 2 * x_rows + w_cols)
+    xq = _random_codes(rng, (M, K))
+    wq = _random_codes(rng, (N, K), 0.5)
+    sx = (rng.uniform(0.5, 2.0, M if x_rows else 1) * 0.01).astype(np.float32)
+    sw = (rng.uniform(0.5, 2.0, N if w_cols else 1) * 0.002).astype(np.float32)
+    y = fw.fp8_linear_scaled(from_codes(xq, DEV), from_codes(wq, DEV),
+                             torch.from_numpy(sx).to(DEV), torch.from_numpy(sw).to(DEV))
+    ref = oracle.linear_scaled(xq, wq, sx, sw)
+    assert rel_fro(bits(y), ref) <= GEMM_REL_FRO
+    assert fw.device_status()[0] == fw.OK
