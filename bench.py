@@ -1002,7 +1002,8 @@ def time_isolated(call, steps, warmup, flush):
     return statistics.median(times)
 
 
-def kernel_bench(fw, kind, shape, steps, warmup, device, sustain_s=0.0, isolated=True):
+def kernel_bench(fw, kind, shape, steps, warmup, device, sustain_s=0.0, isolated=True,
+                 clocks=True):
     """One kernel kind on one shape.  The headline "us" is the back-to-back
     per-launch time over buffer sets rotated until they span twice the L2
     (so every launch reads its operands from DRAM, as a layer stack does);
@@ -1012,14 +1013,22 @@ def kernel_bench(fw, kind, shape, steps, warmup, device, sustain_s=0.0, isolated
     power-capped rate.  Returns a dict for one JSON line."""
     pk = peaks()
     t0, call, work, nbytes = make_kernel(fw, kind, shape, device)
-    nsets = int(min(MAX_SETS, max(1, -(-ROTATE_BYTES // max(_set_bytes(t0), 1)))))
+    # at least two sets, so that consecutive launches never share buffers
+    nsets = int(min(MAX_SETS, max(2, -(-ROTATE_BYTES // max(_set_bytes(t0), 1)))))
     sets = [t0] + [{k: v.clone() for k, v in t0.items()} for _ in range(nsets - 1)]
     calls = [(lambda t=t: call(t)) for t in sets]
+    sampler = clock_sampler(device.index if device.index is not None else 0) if clocks else None
+    if sampler:
+        sampler.start()
     ms, per_replay = time_back_to_back(calls, steps, max(warmup // 5, 2))
+    clk = sampler.stop() if sampler else None
     out = {"kernel": kind, "shape": list(shape), "us": ms * 1e3,
            "gbs": nbytes / (ms / 1e3) / 1e9, "hbm_frac": nbytes / (ms / 1e3) / 1e9 / pk["hbm"],
            "timing": f"back to back, {nsets} buffer set(s) of {_set_bytes(t0) / 1e6:.1f} MB rotated, "
                      f"median of {steps} graph replays of {per_replay} launches"}
+    if clk:
+        out["sm_mhz"] = clk["sm_mhz"]
+        out["clock_reasons"] = clk["reasons"]
     if isolated:
         flush = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
         ms_iso = time_isolated(calls[0], steps, warmup, flush)

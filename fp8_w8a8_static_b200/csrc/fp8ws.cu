@@ -356,6 +356,16 @@ struct PairProblem {
   const float *s_down;
 };
 
+// L2 eviction hints on the GEMM operand loads; FP8WS_L2_HINTS=0 turns them off
+// (every load then takes the normal policy).
+bool use_l2_hints() {
+  static const bool v = [] {
+    const char *e = getenv("FP8WS_L2_HINTS");
+    return !(e && e[0] == '0');
+  }();
+  return v;
+}
+
 // Kernel-side description of a group whose tiles are tile_m x tile_n.
 PairGroup make_pair_group(const PairProblem *pp, int np, int tile_m, int tile_n) {
   PairGroup G = {};
@@ -377,7 +387,7 @@ PairGroup make_pair_group(const PairProblem *pp, int np, int tile_m, int tile_n)
     // Row by row, each A row block is consumed within a wave and B is read
     // again by every wave; column by column within row groups, the other way
     // round.  The operand consumed within a wave is loaded evict-first.
-    G.hint[p] = G.group_m[p] == 1 ? kHintAFirst : kHintBFirst;
+    G.hint[p] = !use_l2_hints() ? kHintNone : (G.group_m[p] == 1 ? kHintAFirst : kHintBFirst);
     G.s_in[p] = q.s_in;
     G.s_w[p] = q.s_w;
     G.s_w2[p] = q.s_w2;
