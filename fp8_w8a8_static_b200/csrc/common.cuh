@@ -122,6 +122,16 @@ __device__ __forceinline__ bool mbar_wait_bounded_warp(uint64_t *bar, uint32_t p
   }
 }
 
+// Bring `bytes` bytes at p (16-byte aligned, a multiple of 16) into L2
+// without reading them into the SM.  L2 is the point of coherence, so a
+// prefetch issued before the data's producer has finished cannot make a later
+// load see stale values: at worst it fetches lines that are then overwritten.
+__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)),
+               "r"(bytes)
+               : "memory");
+}
+
 // ------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

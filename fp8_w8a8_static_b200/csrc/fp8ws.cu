@@ -305,13 +305,23 @@ int *splitk_counters(void *splitk) {
 // wave then takes a half tile's time, not a whole one's.
 constexpr int kSplitkMinKb = 64;
 
-SplitPlan make_split_plan(int tiles, int pairs, int num_kb, float *partials, int *counters) {
+// FP8WS_TAIL_HALVES=0 keeps ragged last waves whole (timing comparisons).
+bool tail_halves_enabled() {
+  static const bool v = [] {
+    const char *e = getenv("FP8WS_TAIL_HALVES");
+    return !(e && e[0] == '0');
+  }();
+  return v;
+}
+
+SplitPlan make_split_plan(int tiles, int pairs, int num_kb, float *partials, int *counters,
+                          bool halves_allowed = true) {
   SplitPlan p{tiles, 0, 1, num_kb, nullptr, nullptr, 1};
   if (pairs < 1 || tiles % pairs == 0) return p;
   const int R = tiles % pairs;
   const bool k_split_possible = partials && num_kb >= kSplitkMinKb && R <= kSplitkTiles;
   if (!k_split_possible) {
-    if (2 * R <= pairs) {
+    if (halves_allowed && 2 * R <= pairs) {
       p.dp_tiles = tiles - R;
       p.split_tiles = R;
       p.halves = 2;
@@ -355,6 +365,17 @@ struct PairProblem {
   const float *s_w2;
   const float *s_down;
 };
+
+// The grouped gated MLP's overlap of the next call's input prefetch with its
+// down GEMM's tail (late dependent launch + L2 prefetch); FP8WS_LATE_TRIGGER=0
+// turns it off.
+bool late_trigger_enabled() {
+  static const bool v = [] {
+    const char *e = getenv("FP8WS_LATE_TRIGGER");
+    return !(e && e[0] == '0');
+  }();
+  return v;
+}
 
 // L2 eviction hints on the GEMM operand loads; FP8WS_L2_HINTS=0 turns them off
 // (every load then takes the normal policy).
@@ -430,7 +451,7 @@ int pair_clusters(DeviceInfo *d, Kernel kern, int threads, int smem, int bit,
 
 template <int STAGES, int BIT, int SCALE_MODE = 0, bool DIRECT = false>
 int launch_gemm_pair_cfg(DeviceInfo *d, const PairProblem *pp, int np, int K, cudaStream_t st,
-                         void *splitk = nullptr) {
+                         void *splitk = nullptr, bool late_trigger = false) {
   using C = PairCfg<STAGES, DIRECT>;
   auto kern = fp8_gemm_pair_kernel<STAGES, SCALE_MODE, DIRECT>;
   int rc = pair_clusters(d, kern, kGemmThreads, C::SMEM_BYTES, BIT, &d->pair_clusters);
@@ -460,9 +481,10 @@ int launch_gemm_pair_cfg(DeviceInfo *d, const PairProblem *pp, int np, int K, cu
   const int tiles = G.tiles;
   float *partials = static_cast<float *>(splitk);
   int *counters = splitk ? splitk_counters(splitk) : nullptr;
-  const SplitPlan plan =
-      make_split_plan(tiles, d->pair_clusters.load(std::memory_order_relaxed),
-                      (K + kGemmBK - 1) / kGemmBK, partials, counters);
+  SplitPlan plan = make_split_plan(tiles, d->pair_clusters.load(std::memory_order_relaxed),
+                                   (K + kGemmBK - 1) / kGemmBK, partials, counters,
+                                   tail_halves_enabled());
+  plan.late_trigger = late_trigger ? 1 : 0;
   const int units = plan.dp_tiles + plan.split_tiles * plan.splits * plan.halves;
   const int resident = d->pair_clusters.load(std::memory_order_relaxed);
   const int clusters = units < resident ? units : resident;
@@ -487,10 +509,12 @@ bool direct_epilogue() {
 
 template <int BIT, int SCALE_MODE = 0>
 int launch_gemm_pair(DeviceInfo *d, const PairProblem *pp, int np, int K, cudaStream_t st,
-                     void *splitk = nullptr) {
+                     void *splitk = nullptr, bool late_trigger = false) {
   if (direct_epilogue())
-    return launch_gemm_pair_cfg<7, BIT + 16, SCALE_MODE, true>(d, pp, np, K, st, splitk);
-  return launch_gemm_pair_cfg<6, BIT, SCALE_MODE, false>(d, pp, np, K, st, splitk);
+    return launch_gemm_pair_cfg<7, BIT + 16, SCALE_MODE, true>(d, pp, np, K, st, splitk,
+                                                                late_trigger);
+  return launch_gemm_pair_cfg<6, BIT, SCALE_MODE, false>(d, pp, np, K, st, splitk,
+                                                         late_trigger);
 }
 
 template <int BIT, int SCALE_MODE = 0>
@@ -634,7 +658,7 @@ int gemm_dispatch(DeviceInfo *d, const uint8_t *xq, const uint8_t *wq, int64_t M
 // their tiles when the cost model picks CTA pairs for the group, else one
 // launch each.  Problems with M == 0 are skipped.
 int gemm_group_dispatch(DeviceInfo *d, const PairProblem *pp, int np, int K, cudaStream_t st,
-                        void *splitk = nullptr) {
+                        void *splitk = nullptr, bool late_trigger = false) {
   PairProblem live[kMaxGroup];
   int64_t rows[kMaxGroup], cols[kMaxGroup];
   int n = 0;
@@ -645,7 +669,8 @@ int gemm_group_dispatch(DeviceInfo *d, const PairProblem *pp, int np, int K, cud
       cols[n++] = pp[p].N;
     }
   if (n == 0) return FP8WS_OK;
-  if (gemm_choice(d, rows, cols, n) == 1) return launch_gemm_pair<3>(d, live, n, K, st, splitk);
+  if (gemm_choice(d, rows, cols, n) == 1)
+    return launch_gemm_pair<3>(d, live, n, K, st, splitk, late_trigger);
   int rc = FP8WS_OK;
   for (int p = 0; p < n && !rc; ++p)
     rc = gemm_dispatch(d, live[p].a, live[p].b, live[p].M, live[p].N, K, live[p].s_in,
@@ -675,8 +700,9 @@ int quant_launch(DeviceInfo *d, const uint16_t *x, int64_t numel, const float *s
 
 // Two activations in one launch, the blocks shared in proportion to their
 // sizes; a single non-empty one goes to quant_launch.
+// prefetch_blocks: see quant_static_pair_kernel (0: no prefetch).
 int quant_pair_launch(DeviceInfo *d, const QuantSeg *q, int nq, cudaStream_t st,
-                      int *zero_words = nullptr, int n_zero = 0) {
+                      int *zero_words = nullptr, int n_zero = 0, int prefetch_blocks = 0) {
   QuantSeg live[2];
   int n = 0;
   for (int i = 0; i < nq; ++i)
@@ -694,7 +720,7 @@ int quant_pair_launch(DeviceInfo *d, const QuantSeg *q, int nq, cudaStream_t st,
   split = split < 1 ? 1 : (split > grid - 1 ? grid - 1 : split);
   if (launch_ex(wide ? quant_static_pair_kernel<true> : quant_static_pair_kernel<false>,
                 dim3(grid), dim3(kEwThreads), 0, st, 1, live[0], live[1], split, zero_words,
-                n_zero) != cudaSuccess)
+                n_zero, prefetch_blocks) != cudaSuccess)
     return FP8WS_ERR_CUDA;
   log_launch(kKindQuant, live[0].x, nullptr, live[0].xq, 0);
   log_launch(kKindQuant, live[1].x, nullptr, live[1].xq, 1);
@@ -1113,10 +1139,16 @@ int gated_mlp_static_fp8_group(const fp8ws_mlp_tower *towers, int count, int64_t
   if (rc) return rc;
   cudaStream_t st = as_stream(stream);
   void *splitk = ws;  // 256-byte aligned: every region above is a multiple of 256 bytes
-  rc = quant_pair_launch(d, qs, n, st, splitk_counters(splitk), kSplitkCounterWords);
+  // The quantizer prefetches both towers' X into L2 before it waits for the
+  // kernel before it; the down GEMM lets the next kernel on the stream (the
+  // next layer's quantizer, in a stack of these calls) launch only as its CTAs
+  // start their last tiles, so that prefetch overlaps the GEMM's tail.
+  rc = quant_pair_launch(d, qs, n, st, splitk_counters(splitk), kSplitkCounterWords,
+                         late_trigger_enabled() ? d->sms : 0);
   if (!rc) rc = launch_dual_swiglu(d, up, n, static_cast<int>(I), static_cast<int>(dm), ap, st);
   if (!rc)
-    rc = gemm_group_dispatch(d, down, n, static_cast<int>(I), st, splitk);
+    rc = gemm_group_dispatch(d, down, n, static_cast<int>(I), st, splitk,
+                             late_trigger_enabled());
   return rc;
 }
 

@@ -96,6 +96,9 @@ struct SplitPlan {
   float *partials;  // [split_tiles * splits] slots, see partial_index
   int *counters;    // [split_tiles][2][4]
   int halves;       // 1, or 2: the remainder tiles run as 256 x 128 halves
+  // 1: let the next kernel on the stream launch only when this CTA starts its
+  // last unit (the next kernel prefetches its input meanwhile), not at once
+  int late_trigger;
 };
 
 struct UnitRange {
@@ -238,7 +241,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
     tmem_relinquish_pair();
   }
-  pdl_launch_dependents();
+  if (!plan.late_trigger) pdl_launch_dependents();
   pdl_wait();  // the previous kernel's outputs (our inputs) are complete from here on
   tc_fence_before();
   cluster_sync();
@@ -254,6 +257,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint64_t pol_first = l2_policy_evict_first();
       const uint64_t pol_normal = l2_policy_evict_normal();
       for (int u = cluster; u < num_units && ok; u += nclusters) {
+        if (plan.late_trigger && u + nclusters >= num_units) pdl_launch_dependents();
         const UnitRange ur = unit_range(u, plan, num_kb);
         const GroupTile gt = group_tile(ur.tile, G);
         if (!unit_live(ur, gt, G)) continue;
