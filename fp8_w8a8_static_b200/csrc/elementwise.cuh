@@ -474,8 +474,10 @@ __global__ void rtn_scale_kernel(float *__restrict__ s) {
 // --------------------------------------------- per-token / per-channel rows
 namespace fp8ws {
 
-constexpr int kRowThreads = 256;
+constexpr int kRowThreads = 256;       // threads per row of the per-token SwiGLU
+constexpr int kQuantRowThreads = 128;  // threads per row of the per-token quantizer
 
+template <int THREADS = kRowThreads>
 __device__ __forceinline__ float block_max_rows(float m, float *red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
@@ -483,16 +485,19 @@ __device__ __forceinline__ float block_max_rows(float m, float *red) {
   __syncthreads();
   m = red[0];
 #pragma unroll
-  for (int w = 1; w < kRowThreads / 32; ++w) m = fmaxf(m, red[w]);
+  for (int w = 1; w < THREADS / 32; ++w) m = fmaxf(m, red[w]);
   return m;
 }
 
 // One block per row of a [rows, K] BF16 tensor (K % 8 == 0): s[r] = max|x| /
 // 448 (1 for an all-zero row), codes q(x, s[r]) as the static quantizer.
 // Per-token scales for activations, per-channel scales for weights.
-__global__ void __launch_bounds__(kRowThreads) quant_rows_kernel(
+// HELD: 8-element vectors per thread that a row may keep in registers (rows
+// of up to kQuantRowThreads * HELD vectors take the single-read path).
+template <int HELD>
+__global__ void __launch_bounds__(kQuantRowThreads) quant_rows_kernel(
     const uint16_t *__restrict__ x, int K, float *__restrict__ s_out, uint8_t *__restrict__ q) {
-  __shared__ float red[kRowThreads / 32];
+  __shared__ float red[kQuantRowThreads / 32];
   pdl_launch_dependents();
   pdl_wait();
   const int64_t row = blockIdx.x;
@@ -500,18 +505,41 @@ __global__ void __launch_bounds__(kRowThreads) quant_rows_kernel(
   uint2 *qv = reinterpret_cast<uint2 *>(q + row * K);
   const int nvec = K >> 3;
   float m = 0.0f;
-  for (int i = threadIdx.x; i < nvec; i += kRowThreads) m = absmax8(__ldg(xv + i), m);
-  m = block_max_rows(m, red);
+  if (nvec <= kQuantRowThreads * HELD) {
+    // the whole row fits in the threads' registers: every load in flight at
+    // once, and the quantization reuses the values instead of reading again
+    uint4 v[HELD];
+#pragma unroll
+    for (int k = 0; k < HELD; ++k) {
+      const int i = threadIdx.x + k * kQuantRowThreads;
+      v[k] = i < nvec ? ld_stream(xv + i) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int k = 0; k < HELD; ++k) m = absmax8(v[k], m);
+    m = block_max_rows<kQuantRowThreads>(m, red);
+    const float s = m > 0.0f ? __fdiv_rn(m, 448.0f) : 1.0f;
+    const float r = __frcp_rn(s);
+    if (threadIdx.x == 0) s_out[row] = s;
+#pragma unroll
+    for (int k = 0; k < HELD; ++k) {
+      const int i = threadIdx.x + k * kQuantRowThreads;
+      if (i < nvec) st_stream(qv + i, quant8(v[k], s, r));
+    }
+    return;
+  }
+  for (int i = threadIdx.x; i < nvec; i += kQuantRowThreads) m = absmax8(__ldg(xv + i), m);
+  m = block_max_rows<kQuantRowThreads>(m, red);
   const float s = m > 0.0f ? __fdiv_rn(m, 448.0f) : 1.0f;
   const float r = __frcp_rn(s);
   if (threadIdx.x == 0) s_out[row] = s;
-  for (int i = threadIdx.x; i < nvec; i += kRowThreads) qv[i] = quant8(__ldg(xv + i), s, r);
+  for (int i = threadIdx.x; i < nvec; i += kQuantRowThreads) qv[i] = quant8(__ldg(xv + i), s, r);
 }
 
 // One block per row of G, U [rows, I] (I % 8 == 0, I <= kMaxRowI): v =
 // SiLU(g) * u in fp32 kept in shared memory, s[r] = max|v| / 448 (1 for an
 // all-zero row), h = E4M3(v * (1/s)).
 constexpr int kMaxRowI = 16384;
+constexpr int kRowBatch = 4;  // vector pairs a thread loads before using the first
 
 __global__ void __launch_bounds__(kRowThreads) silu_mul_rows_kernel(
     const uint16_t *__restrict__ g, const uint16_t *__restrict__ u, int I,
@@ -525,16 +553,36 @@ __global__ void __launch_bounds__(kRowThreads) silu_mul_rows_kernel(
   const uint4 *uv = reinterpret_cast<const uint4 *>(u + row * I);
   const int nvec = I >> 3;
   float m = 0.0f;
-  for (int i = threadIdx.x; i < nvec; i += kRowThreads) {
-    const uint4 a = ld_stream(gv + i), b = ld_stream(uv + i);
-    float v[8] = {silu_mul(bf16_lo(a.x), bf16_lo(b.x)), silu_mul(bf16_hi(a.x), bf16_hi(b.x)),
-                  silu_mul(bf16_lo(a.y), bf16_lo(b.y)), silu_mul(bf16_hi(a.y), bf16_hi(b.y)),
-                  silu_mul(bf16_lo(a.z), bf16_lo(b.z)), silu_mul(bf16_hi(a.z), bf16_hi(b.z)),
-                  silu_mul(bf16_lo(a.w), bf16_lo(b.w)), silu_mul(bf16_hi(a.w), bf16_hi(b.w))};
+  // kRowBatch vector pairs per thread are loaded before the first is used, so
+  // a row costs one or two memory round trips instead of one per vector
+  for (int base = threadIdx.x; base < nvec; base += kRowThreads * kRowBatch) {
+    uint4 a[kRowBatch], b[kRowBatch];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      vrow[i * 8 + e] = v[e];
-      m = fmaxf(m, fabsf(v[e]));
+    for (int k = 0; k < kRowBatch; ++k) {
+      const int i = base + k * kRowThreads;
+      if (i < nvec) {
+        a[k] = ld_stream(gv + i);
+        b[k] = ld_stream(uv + i);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kRowBatch; ++k) {
+      const int i = base + k * kRowThreads;
+      if (i < nvec) {
+        float v[8] = {silu_mul(bf16_lo(a[k].x), bf16_lo(b[k].x)),
+                      silu_mul(bf16_hi(a[k].x), bf16_hi(b[k].x)),
+                      silu_mul(bf16_lo(a[k].y), bf16_lo(b[k].y)),
+                      silu_mul(bf16_hi(a[k].y), bf16_hi(b[k].y)),
+                      silu_mul(bf16_lo(a[k].z), bf16_lo(b[k].z)),
+                      silu_mul(bf16_hi(a[k].z), bf16_hi(b[k].z)),
+                      silu_mul(bf16_lo(a[k].w), bf16_lo(b[k].w)),
+                      silu_mul(bf16_hi(a[k].w), bf16_hi(b[k].w))};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          vrow[i * 8 + e] = v[e];
+          m = fmaxf(m, fabsf(v[e]));
+        }
+      }
     }
   }
   m = block_max_rows(m, red);

@@ -1324,8 +1324,11 @@ int fp8_quant_per_token(const uint16_t *x, int64_t rows, int64_t K, float *s, ui
   int rc = device_info(&d);
   if (rc) return rc;
   cudaStream_t st = as_stream(stream);
-  if (launch_ex(quant_rows_kernel, dim3(static_cast<unsigned>(rows)), dim3(kRowThreads), 0, st, 1,
-                x, static_cast<int>(K), s, xq) != cudaSuccess)
+  // rows of up to 4096 elements hold 4 vectors per thread (fewer registers,
+  // more rows in flight per SM), up to 8192 hold 8, longer rows are read twice
+  if (launch_ex(K <= 4096 ? quant_rows_kernel<4> : quant_rows_kernel<8>,
+                dim3(static_cast<unsigned>(rows)), dim3(kQuantRowThreads), 0, st, 1, x,
+                static_cast<int>(K), s, xq) != cudaSuccess)
     return FP8WS_ERR_CUDA;
   log_launch(kKindQuant, x, nullptr, xq);
   return launch_status();
