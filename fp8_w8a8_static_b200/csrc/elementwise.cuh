@@ -207,11 +207,16 @@ __device__ __forceinline__ void quant_static_range(const uint16_t *__restrict__ 
   }
 }
 
+// prefetch_share_l2 and the prefetch_blocks argument: see quant_static_pair_kernel.
+__device__ __forceinline__ void prefetch_share_l2(const void *p, int64_t n, int blk, int nblk);
+
 template <bool WIDE>
 __global__ void __launch_bounds__(kEwThreads) quant_static_kernel(
     const uint16_t *__restrict__ x, int64_t numel, const float *__restrict__ s_in,
-    uint8_t *__restrict__ xq, int *__restrict__ zero_words, int n_zero) {
+    uint8_t *__restrict__ xq, int *__restrict__ zero_words, int n_zero, int prefetch_blocks) {
   pdl_launch_dependents();
+  if (threadIdx.x == 0 && prefetch_blocks > 0)
+    prefetch_share_l2(x, numel * 2, blockIdx.x, prefetch_blocks);
   pdl_wait();
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero_words[i] = 0;
@@ -248,7 +253,8 @@ __device__ __forceinline__ void prefetch_share_l2(const void *p, int64_t n, int 
 // each of the first prefetch_blocks blocks (those resident earliest, one per
 // SM) prefetches its share of both inputs into L2, so that their DRAM reads
 // overlap the end of the previous kernel (which, in the grouped gated MLP,
-// lets this grid launch only as it starts its last tiles).
+// lets this grid launch only as it starts its last tiles).  When the previous
+// kernel has already finished, the prefetch merely runs beside the loads.
 template <bool WIDE>
 __global__ void __launch_bounds__(kEwThreads)
     quant_static_pair_kernel(const QuantSeg a, const QuantSeg b, int split,

@@ -59,8 +59,8 @@ struct DeviceInfo {
   int sms = 0;                  // set before `checked` is released
   int64_t l2_bytes = 0;         // likewise
   // bit per kernel whose attributes were set on this device: 0-2 one-CTA GEMMs,
-  // 3/5/6/7 pair GEMM scale modes (+16 direct-store), 4 dual (+8 variant,
-  // +16 direct variant, +24 direct plain), 8 per-token SwiGLU
+  // 3/5/6/7 pair GEMM scale modes (+16 direct-store), 9 five-stage pair GEMM,
+  // 4 dual (+8 variant, +16 direct variant, +24 direct plain), 8 per-token SwiGLU
   std::atomic<unsigned> gemm_attr_set{0};
   std::atomic<int> pair_clusters{0};  // CTA pairs of the pair GEMM resident at once
   std::atomic<int> dual_clusters{0};  // CTA pairs of the gate/up dual GEMM resident at once
@@ -377,6 +377,16 @@ bool late_trigger_enabled() {
   return v;
 }
 
+// L2 prefetch of the quantizers' inputs before they wait for the kernel
+// before them; FP8WS_PREFETCH=0 turns it off (timing comparisons).
+bool prefetch_enabled() {
+  static const bool v = [] {
+    const char *e = getenv("FP8WS_PREFETCH");
+    return !(e && e[0] == '0');
+  }();
+  return v;
+}
+
 // L2 eviction hints on the GEMM operand loads; FP8WS_L2_HINTS=0 turns them off
 // (every load then takes the normal policy).
 bool use_l2_hints() {
@@ -507,9 +517,21 @@ bool direct_epilogue() {
   return v;
 }
 
+// FP8WS_PAIR_STAGES=5: the CTA-pair GEMM with a five-stage ring instead of six
+// (per-tensor scales only), to see how the K step depends on the ring depth.
+bool five_stages() {
+  static const bool v = [] {
+    const char *e = getenv("FP8WS_PAIR_STAGES");
+    return e && e[0] == '5';
+  }();
+  return v;
+}
+
 template <int BIT, int SCALE_MODE = 0>
 int launch_gemm_pair(DeviceInfo *d, const PairProblem *pp, int np, int K, cudaStream_t st,
                      void *splitk = nullptr, bool late_trigger = false) {
+  if (SCALE_MODE == 0 && five_stages())
+    return launch_gemm_pair_cfg<5, 9, 0, false>(d, pp, np, K, st, splitk, late_trigger);
   if (direct_epilogue())
     return launch_gemm_pair_cfg<7, BIT + 16, SCALE_MODE, true>(d, pp, np, K, st, splitk,
                                                                 late_trigger);
@@ -691,8 +713,11 @@ int gemm_groups(DeviceInfo *d, const PairProblem *pp, int np, int K, cudaStream_
 int quant_launch(DeviceInfo *d, const uint16_t *x, int64_t numel, const float *s, uint8_t *xq,
                  cudaStream_t st, int *zero_words = nullptr, int n_zero = 0) {
   if (numel == 0) return FP8WS_OK;
+  // the first blocks prefetch x into L2 while the previous kernel drains
   if (ew_launch<quant_static_kernel<true>, quant_static_kernel<false>>(
-          d, aligned32(x), numel >> 3, st, x, numel, s, xq, zero_words, n_zero) != cudaSuccess)
+          d, aligned32(x), numel >> 3, st, x, numel, s, xq, zero_words, n_zero,
+          prefetch_enabled() ? d->sms : 0) !=
+      cudaSuccess)
     return FP8WS_ERR_CUDA;
   log_launch(kKindQuant, x, nullptr, xq);
   return launch_status();
@@ -700,9 +725,11 @@ int quant_launch(DeviceInfo *d, const uint16_t *x, int64_t numel, const float *s
 
 // Two activations in one launch, the blocks shared in proportion to their
 // sizes; a single non-empty one goes to quant_launch.
-// prefetch_blocks: see quant_static_pair_kernel (0: no prefetch).
+// The first d->sms blocks prefetch both inputs into L2 while the previous
+// kernel drains (see quant_static_pair_kernel).
 int quant_pair_launch(DeviceInfo *d, const QuantSeg *q, int nq, cudaStream_t st,
-                      int *zero_words = nullptr, int n_zero = 0, int prefetch_blocks = 0) {
+                      int *zero_words = nullptr, int n_zero = 0) {
+  const int prefetch_blocks = prefetch_enabled() ? d->sms : 0;
   QuantSeg live[2];
   int n = 0;
   for (int i = 0; i < nq; ++i)
@@ -1142,9 +1169,8 @@ int gated_mlp_static_fp8_group(const fp8ws_mlp_tower *towers, int count, int64_t
   // The quantizer prefetches both towers' X into L2 before it waits for the
   // kernel before it; the down GEMM lets the next kernel on the stream (the
   // next layer's quantizer, in a stack of these calls) launch only as its CTAs
-  // start their last tiles, so that prefetch overlaps the GEMM's tail.
-  rc = quant_pair_launch(d, qs, n, st, splitk_counters(splitk), kSplitkCounterWords,
-                         late_trigger_enabled() ? d->sms : 0);
+  // start their last tiles, so that such a prefetch overlaps the GEMM's tail.
+  rc = quant_pair_launch(d, qs, n, st, splitk_counters(splitk), kSplitkCounterWords);
   if (!rc) rc = launch_dual_swiglu(d, up, n, static_cast<int>(I), static_cast<int>(dm), ap, st);
   if (!rc)
     rc = gemm_group_dispatch(d, down, n, static_cast<int>(I), st, splitk,
