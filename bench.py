@@ -57,8 +57,6 @@ TOKENS_PER_STEP = sum(m for _, m in TOWERS)
 # order of the towers inside a grouped launch: the generation tower's tiles
 # first, the understanding tower's fill the ragged last wave
 GROUP_ORDER = (TOWERS[1], TOWERS[0])
-if os.environ.get("FP8WS_BENCH_UND_FIRST") == "1":  # timing comparison of the tower order
-    GROUP_ORDER = (TOWERS[0], TOWERS[1])
 CALIB_BATCHES = 16
 CALIB_ROWS = 256
 

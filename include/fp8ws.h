@@ -102,6 +102,11 @@ FP8WS_API int fp8_quant_static(const uint16_t *x, int64_t numel, const float *s_
  * y: device [M,N] BF16, row-major, contiguous (row stride N).
  * Sizes: M >= 0 (0 launches nothing), N >= 8 with N % 8 == 0, K >= 16 with
  * K % 16 == 0; M, N, K < 2^31.
+ * Tiling: 256 x 256 tiles on CTA pairs (one-CTA tiles where a cost model finds
+ * them faster); when the tiles past the last full wave of pairs would fill
+ * at most half a wave, each of them runs as two 256 x 128 halves over the
+ * full K, which gives the same result per element.  fp8ws_split_plan reports
+ * the plan for a shape.
  */
 FP8WS_API int fp8_linear_static(const uint8_t *xq, const uint8_t *wq, int64_t M, int64_t N, int64_t K,
                       const float *s_in, const float *s_w, uint16_t *y, void *stream);
