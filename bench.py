@@ -19,8 +19,9 @@ dominant kernel).  The end-to-end number goes through the composite call with
 host buffers: every layer's input is copied from pinned host memory and its
 output copied back inside the timed region.  At N=1 the line also carries the
 per-workload kernel figures ("configs": the Linear sweep, the SwiGLU sweep, the
-shared-quant Q/K/V block, the tiny MLP, the per-token path and the
-cross-attention projections) with their roofline fractions.
+shared-quant Q/K/V block, the tiny MLP, the per-token path, the
+cross-attention projections and the SwiGLU variant) with their roofline
+fractions.
 
 `--impl reference` times the CPU oracle (the only other implementation there
 is) on a bounded sample of rows of the same pass on the host cores.
@@ -777,6 +778,11 @@ def _static_linear_inputs(fw, M, N, K, cfg, seed, device):
     return xq, wq, s_in, s_w
 
 
+# The SwiGLU variant timed by the "variants" workload: alpha 1.702 inside the
+# sigmoid, beta 1 on up, clamp at 7 (the shape the pages' notes name).
+SWIGLU_VARIANT = lambda fw: fw.swiglu(1.702, 1.0, 7.0)  # noqa: E731
+
+
 def make_kernel(fw, kind, shape, device):
     """One call of a kernel kind on one shape, with synthetic inputs shaped
     like the pages' workloads.  Returns (t, call, work, nbytes): t holds every
@@ -815,7 +821,7 @@ def make_kernel(fw, kind, shape, device):
         t = dict(xq=xq, wq=wq, sx=sx, sw=sw, y=emp((M, N), bf))
         call = lambda t: fw.fp8_linear_scaled(t["xq"], t["wq"], t["sx"], t["sw"], out=t["y"])  # noqa: E731
         return t, call, 2.0 * M * N * K, M * K + N * K + 2 * M * N + 4 * (M + N)
-    if kind == "dual":
+    if kind in ("dual", "dual_var"):
         M, N, K = shape
         x = synth.activation_with_outliers(M, K, 9, 1, 0, device)
         s_in = fw.fp8_observer_scale(fw.fp8_absmax_bf16(x))
@@ -824,8 +830,10 @@ def make_kernel(fw, kind, shape, device):
         wu, s_wu = fw.fp8_rtn_quantize_weight(synth.normal((N, K), synth.W_STD, synth.seed(4, 90, 2), device))
         t = dict(xq=xq, wg=wg, wu=wu, s_in=s_in, s_wg=s_wg, s_wu=s_wu, s_down=_scalar(0.003, device),
                  h=emp((M, N), f8))
+        act = SWIGLU_VARIANT(fw) if kind == "dual_var" else None
         call = lambda t: fw.fp8_gate_up_swiglu_static(t["xq"], t["wg"], t["wu"], t["s_in"],  # noqa: E731
-                                                      t["s_wg"], t["s_wu"], t["s_down"], out=t["h"])
+                                                      t["s_wg"], t["s_wu"], t["s_down"], act=act,
+                                                      out=t["h"])
         return t, call, 4.0 * M * N * K, M * K + 2 * N * K + M * N
     if kind in ("mlp", "mlp_tok"):
         M, dm, Ii = shape
@@ -926,13 +934,18 @@ def make_kernel(fw, kind, shape, device):
         call = lambda t: fw.fp8_linear_static_group(probs(t), outs=[t["y0"], t["y1"]],  # noqa: E731
                                                     split_k=split, workspace=t["ws"])
         return t, call, 2.0 * (M0 + M1) * N * K, (M0 + M1) * K + 2 * N * K + 2 * (M0 + M1) * N
-    if kind in ("swiglu", "swiglu_tok"):
+    if kind in ("swiglu", "swiglu_tok", "swiglu_var"):
         M, Ii = shape
         t = dict(g=synth.normal((M, Ii), 2.0, synth.seed(2, 90, 7), device),
                  u=synth.normal((M, Ii), 1.0, synth.seed(2, 90, 8), device), h=emp((M, Ii), f8))
         if kind == "swiglu":
             t["s"] = fw.fp8_observer_scale(fw.fp8_silu_mul_absmax(t["g"], t["u"]))
             call = lambda t: fw.silu_mul_2in_fp8(t["g"], t["u"], t["s"], out=t["h"])  # noqa: E731
+            return t, call, None, 5 * M * Ii
+        if kind == "swiglu_var":
+            t["s"] = _scalar(0.01, device)
+            act = SWIGLU_VARIANT(fw)
+            call = lambda t: fw.swiglu_2in_fp8(t["g"], t["u"], t["s"], act, out=t["h"])  # noqa: E731
             return t, call, None, 5 * M * Ii
         t["s"] = emp((M,), torch.float32)
         call = lambda t: fw.silu_mul_2in_fp8_per_token(t["g"], t["u"], out=t["h"], scales=t["s"])  # noqa: E731
@@ -1095,19 +1108,24 @@ SWEEPS = {
                   ("gemm_scaled", (4096, synth.C4["I"], synth.C4["d"]))],
     # cross-attention projections: generation-tower queries over understanding-tower context
     "xattn": [("xattn", (4096, 1024, synth.C3["d"], synth.C3["Nq"], synth.C3["Nk"]))],
+    # the swiglu_alpha/beta/limit variant: element-wise and in the gate/up epilogue
+    "variants": [("swiglu_var", (4096, synth.C4["I"])),
+                 ("dual_var", (4096, synth.C4["I"], synth.C4["d"])),
+                 ("dual", (4096, synth.C4["I"], synth.C4["d"]))],
 }
 
 # the workloads whose figures go into the default run's line (key "configs")
 CONFIG_REPLAYS = 20
-LINE_CONFIGS = ("c0", "c1", "c2", "c3", "per_token", "xattn")
+LINE_CONFIGS = ("c0", "c1", "c2", "c3", "per_token", "xattn", "variants")
 
 
 def config_figures(fw, device, steps, warmup, log):
     """The default run's per-workload kernel figures: every shape of the
     Linear sweep (c1), the SwiGLU sweep (c2), the shared-quant Q/K/V block
     (c3, whole call and its grouped GEMM alone), the tiny MLP (c0), the
-    per-token path and the cross-attention projections, each timed back to
-    back with rotating buffers and alone after an L2 flush."""
+    per-token path, the cross-attention projections and the SwiGLU variant
+    (element-wise, and in the gate/up epilogue beside the plain one), each
+    timed back to back with rotating buffers and alone after an L2 flush."""
     pk = peaks()
     out = {"timing": f"back to back over buffer sets spanning >= {ROTATE_BYTES >> 20} MB (twice "
                      f"the L2), median of {steps} CUDA-graph replays of >= {MIN_PER_REPLAY} "
@@ -1121,7 +1139,7 @@ def config_figures(fw, device, steps, warmup, log):
             r = kernel_bench(fw, kind, shape, steps, warmup, device)
             keep = {k: (round(v, 4) if isinstance(v, float) else v) for k, v in r.items()
                     if k not in ("timing",)}
-            if kind in ("swiglu", "swiglu_tok", "quant", "quant_tok"):
+            if kind in ("swiglu", "swiglu_tok", "swiglu_var", "quant", "quant_tok"):
                 keep["hbm_nominal_frac"] = round(r["gbs"] / 8000.0, 4)
             rows.append(keep)
             log(f"{name} {kind} {shape}: {r['us']:.1f} us"
@@ -1203,7 +1221,8 @@ def main():
     ap.add_argument("--kernel", choices=("gemm", "gemm_ws", "dual", "swiglu", "quant", "gemm_group",
                                          "gemm_group_ws", "dual_group", "quant_group", "scaled_mm",
                                          "mlp", "qkv", "qkv_gemm", "mlp_tok", "quant_tok",
-                                         "swiglu_tok", "gemm_scaled", "xattn"),
+                                         "swiglu_tok", "gemm_scaled", "xattn", "swiglu_var",
+                                         "dual_var"),
                     help="time one kernel on one shape instead of the pass")
     ap.add_argument("--shape", help="M,N,K for gemm; M,I,K for dual; M,I for swiglu; M,K for quant; "
                                     "M0,M1,N,K / M0,M1,I,K / M0,M1,K for the group kinds; "
