@@ -1115,7 +1115,7 @@ SWEEPS = {
 }
 
 # the workloads whose figures go into the default run's line (key "configs")
-CONFIG_REPLAYS = 20
+CONFIG_REPLAYS = 50
 LINE_CONFIGS = ("c0", "c1", "c2", "c3", "per_token", "xattn", "variants")
 
 
