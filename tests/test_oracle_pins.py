@@ -624,3 +624,23 @@ def test_down_scales_match_an_independent_composition():
     s2 = oracle.swiglu_down_scale([(bits_of(gg), bits_of(uu))])
     want2 = float((gg.double() * torch.sigmoid(gg.double()) * uu.double()).abs().max()) / 448.0
     assert abs(s2 - want2) <= 2.0 ** -22 * want2
+
+
+def test_silu_mul_f64_identities():
+    """The fp64 SiLU(g)*u the per-row SwiGLU scales come from, pinned by two
+    identities of the function: SiLU(x) - SiLU(-x) = x (as sigmoid(x) +
+    sigmoid(-x) = 1), over the full range, and SiLU(x) = (x/2)(1 + tanh(x/2)),
+    evaluated with numpy's tanh rather than the oracle's exp, where that form
+    does not cancel; u scales the product."""
+    rng = np.random.default_rng(71)
+    x = np.concatenate([rng.normal(0.0, 3.0, 500), [0.0, 1e-300, -1e-300, 30.0, -30.0, 700.0]])
+    one = np.ones_like(x)
+    pos = oracle.silu_mul_f64(x, one)
+    neg = oracle.silu_mul_f64(-x, one)
+    assert np.allclose(pos - neg, x, rtol=1e-13, atol=1e-300)
+    # the tanh form cancels for large negative x (1 + tanh(x/2) -> 0): compared where |x| <= 8
+    m = np.abs(x) <= 8.0
+    assert np.allclose(pos[m], 0.5 * x[m] * (1.0 + np.tanh(0.5 * x[m])), rtol=1e-12, atol=1e-300)
+    u = rng.normal(0.0, 1.0, x.size)
+    assert np.allclose(oracle.silu_mul_f64(x, u), pos * u, rtol=1e-15, atol=0.0)
+    assert oracle.silu_mul_f64(np.array([0.0]), np.array([5.0]))[0] == 0.0
