@@ -583,11 +583,12 @@ __global__ void __launch_bounds__(kRowThreads) silu_mul_rows_kernel(
                       silu_mul(bf16_hi(a[k].z), bf16_hi(b[k].z)),
                       silu_mul(bf16_lo(a[k].w), bf16_lo(b[k].w)),
                       silu_mul(bf16_hi(a[k].w), bf16_hi(b[k].w))};
+        // v of vector i as two float4 planes (values 0-3 at i, 4-7 at nvec + i),
+        // so that a warp's 16-byte shared-memory accesses are contiguous
+        reinterpret_cast<float4 *>(vrow)[i] = make_float4(v[0], v[1], v[2], v[3]);
+        reinterpret_cast<float4 *>(vrow)[nvec + i] = make_float4(v[4], v[5], v[6], v[7]);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          vrow[i * 8 + e] = v[e];
-          m = fmaxf(m, fabsf(v[e]));
-        }
+        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[e]));
       }
     }
   }
@@ -597,10 +598,11 @@ __global__ void __launch_bounds__(kRowThreads) silu_mul_rows_kernel(
   if (threadIdx.x == 0) s_out[row] = s;
   uint2 *hv = reinterpret_cast<uint2 *>(h + row * I);
   for (int i = threadIdx.x; i < nvec; i += kRowThreads) {
-    const float *v = vrow + i * 8;
+    const float4 lo = reinterpret_cast<const float4 *>(vrow)[i];
+    const float4 hi = reinterpret_cast<const float4 *>(vrow)[nvec + i];
     uint2 o;
-    o.x = pack4(cvt_e4m3x2(v[0] * inv, v[1] * inv), cvt_e4m3x2(v[2] * inv, v[3] * inv));
-    o.y = pack4(cvt_e4m3x2(v[4] * inv, v[5] * inv), cvt_e4m3x2(v[6] * inv, v[7] * inv));
+    o.x = pack4(cvt_e4m3x2(lo.x * inv, lo.y * inv), cvt_e4m3x2(lo.z * inv, lo.w * inv));
+    o.y = pack4(cvt_e4m3x2(hi.x * inv, hi.y * inv), cvt_e4m3x2(hi.z * inv, hi.w * inv));
     st_stream(hv + i, o);
   }
 }
