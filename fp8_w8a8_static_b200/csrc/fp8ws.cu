@@ -1433,9 +1433,18 @@ int gated_mlp_per_token_fp8(const uint16_t *x, int64_t M, int64_t dm, int64_t I,
   if (!rc) rc = check_gemm_args(H, Wd, M, dm, I, sh, s_wd, y);
   if (rc) return rc;
   if (M == 0) return FP8WS_OK;
+  DeviceInfo *d;
+  rc = device_info(&d);
+  if (rc) return rc;
   rc = fp8_quant_per_token(x, M, dm, sx, xq, stream);
-  if (!rc) rc = fp8_linear_scaled(xq, Wg, M, I, dm, sx, 1, s_wg, 1, G, stream);
-  if (!rc) rc = fp8_linear_scaled(xq, Wu, M, I, dm, sx, 1, s_wu, 1, U, stream);
+  // gate and up share one launch (row and column scale vectors in the epilogue)
+  const PairProblem gu[2] = {
+      PairProblem{xq, Wg, nullptr, G, static_cast<int>(M), static_cast<int>(I), sx, s_wg, nullptr,
+                  nullptr},
+      PairProblem{xq, Wu, nullptr, U, static_cast<int>(M), static_cast<int>(I), sx, s_wu, nullptr,
+                  nullptr}};
+  if (!rc) rc = launch_gemm_pair<7, kScaleRowVec | kScaleColVec>(d, gu, 2, static_cast<int>(dm),
+                                                                as_stream(stream));
   if (!rc) rc = silu_mul_2in_fp8_per_token(G, U, M, I, sh, H, stream);
   if (!rc) rc = fp8_linear_scaled(H, Wd, M, dm, I, sh, 1, s_wd, 1, y, stream);
   return rc;
