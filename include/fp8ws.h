@@ -522,8 +522,9 @@ FP8WS_API int cross_attention_qkv_static_fp8(const uint16_t *x, int64_t Mq, cons
  *   an all-zero row), h = E4M3_satRNE(v / s[r]).  G, U: device [rows,I] BF16,
  *   I % 8 == 0, I <= 16384.  s: device, rows fp32 (written).  h: [rows,I] FP8.
  * gated_mlp_per_token_fp8 -- the gated MLP on this scheme: per-token X
- *   quantization, gate and up GEMMs with (per-token x per-channel) scales,
- *   per-token SwiGLU quantization, down GEMM likewise.  s_wg, s_wu: device [I]
+ *   quantization, gate and up GEMMs with (per-token x per-channel) scales in
+ *   one grouped launch, per-token SwiGLU quantization, down GEMM likewise:
+ *   four launches.  s_wg, s_wu: device [I]
  *   fp32, s_wd: device [d] fp32 (per-channel).  workspace:
  *   gated_mlp_per_token_fp8_workspace(M,d,I) bytes, 256-byte aligned:
  *   Xq [M,d] | s_x [M] | G [M,I] | U [M,I] | H [M,I] | s_h [M], each region
