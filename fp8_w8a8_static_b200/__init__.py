@@ -173,6 +173,7 @@ _SIGS = {
     "fp8ws_device_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int),
                                            ctypes.POINTER(ctypes.c_int)]),
     "fp8ws_set_gemm_config": (ctypes.c_int, [ctypes.c_int]),
+    "fp8ws_set_quant_form": (ctypes.c_int, [ctypes.c_int]),
     "fp8ws_selftest_bounded_wait": (ctypes.c_int, [_I64, ctypes.c_int,
                                                    ctypes.POINTER(ctypes.c_int64), _P]),
     "fp8ws_gemm_plan": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int64),
@@ -863,6 +864,15 @@ def selftest_bounded_wait(limit_ns: int, mode: int = 0, stream=None) -> int:
 def set_gemm_config(name: str = "auto") -> None:
     """Force a GEMM tile configuration (see GEMM_CONFIGS); "auto" = cost model."""
     _check(load().fp8ws_set_gemm_config(GEMM_CONFIGS[name]), "fp8ws_set_gemm_config")
+
+
+QUANT_FORMS = {"auto": 0, "staged": 1, "stream": 2}
+
+
+def set_quant_form(name: str = "auto") -> None:
+    """Force the static quantizer's form (see QUANT_FORMS); "auto" chooses by
+    input size.  The codes are the same in every form."""
+    _check(load().fp8ws_set_quant_form(QUANT_FORMS[name]), "fp8ws_set_quant_form")
 
 
 def gemm_plan(shapes, sms: int = 148, pairs: int = 74) -> str:

@@ -24,6 +24,8 @@ enum WaitSite : int {
   kSiteEpiTmemFull = 4,
   kSiteDrain = 5,
   kSiteSelfTest = 6,  // fp8ws_selftest_bounded_wait
+  kSiteStagedFull = 7,   // staged quantizer: a chunk that did not arrive
+  kSiteStagedEmpty = 8,  // staged quantizer: a ring slot that was not released
 };
 
 __device__ __forceinline__ void record_timeout(int site) {
@@ -130,6 +132,18 @@ __device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes) 
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)),
                "r"(bytes)
                : "memory");
+}
+
+// One contiguous run of `bytes` bytes from global to shared memory by the
+// bulk copy engine, completing `bytes` transaction bytes on the mbarrier.
+// Both addresses 16-byte aligned, bytes a multiple of 16.  No multicast.
+__device__ __forceinline__ void bulk_load_1d(void *dst, const void *src, uint32_t bytes,
+                                             uint64_t *bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
 }
 
 // ------------------------------------------------------------------- TMA

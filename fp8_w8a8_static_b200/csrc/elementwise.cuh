@@ -153,6 +153,15 @@ __device__ __forceinline__ int64_t stream2(const uint16_t *__restrict__ a,
 // patterns, across a binade boundary too) give the same code, that is the
 // code of the quotient.  Otherwise (t near an E4M3 rounding boundary, near
 // zero, or not finite) the quotient is computed with IEEE division.
+// r for the tests below: fl32(1/s) when that is a normal fp32 number, else 0.
+// With r = 0 every test fails (the bits 4 ulp below +-0 are a NaN), so a scale
+// whose reciprocal overflows or is subnormal sends each value to IEEE
+// division: 0 * inf would otherwise give the NaN code for x = 0.
+__device__ __forceinline__ float quant_recip(float s) {
+  const float r = __frcp_rn(s);
+  return (r >= 0x1p-126f && r <= 0x1p126f) ? r : 0.0f;
+}
+
 __device__ __forceinline__ uint32_t quant1(float x, float s, float r) {
   const float t = x * r;
   const uint32_t b = __float_as_uint(t);
@@ -161,27 +170,76 @@ __device__ __forceinline__ uint32_t quant1(float x, float s, float r) {
   return cvt_e4m3x2(__fdiv_rn(x, s), 0.0f) & 0xFFu;
 }
 
-// The same test for the two BF16 values of one 32-bit word at once: one
-// conversion of the pair 4 ulp below, one 4 ulp above; if the two code pairs
-// agree they are the codes of both quotients.
-__device__ __forceinline__ uint32_t quant2(uint32_t w, float s, float r) {
-  const float a = bf16_lo(w), c = bf16_hi(w);
-  const uint32_t ba = __float_as_uint(a * r), bc = __float_as_uint(c * r);
-  const uint32_t lo = cvt_e4m3x2(__uint_as_float(ba - 4u), __uint_as_float(bc - 4u));
-  const uint32_t hi = cvt_e4m3x2(__uint_as_float(ba + 4u), __uint_as_float(bc + 4u));
-  if (lo == hi) return lo;
-  return cvt_e4m3x2(__fdiv_rn(a, s), __fdiv_rn(c, s));
+// The vector kernels test 8 values at once with a cheaper bracket (quant1
+// above serves the values past the last whole vector): with
+// rl = fl32(r (1 - 2^-20)) and rh = fl32(r (1 + 2^-20)) (r = fl32(1/s)
+// normal), the products x rl and x rh bracket the IEEE quotient fl32(x / s)
+// in magnitude while they are normal fp32 numbers: r, rl or rh and the product
+// each add a relative error of at most 2^-24, about 3 * 2^-24 in all, far
+// inside the 2^-20 offset, and fl32(x / s) is within 2^-24 of x / s.  Rounding
+// to E4M3 is monotone, so equal codes at both ends are the quotient's code.
+// Quotients below the fp32 normal range give the code +-0, as do both
+// products; overflowing ones saturate at both ends.  A pair of values takes
+// one packed f32x2 multiply per end.  Any other scale (1/s overflowing,
+// subnormal, zero, negative or NaN) gets rl = 0 and rh = inf, whose codes
+// never agree unless x is a NaN, so every value goes to IEEE division.
+struct QuantBracket {
+  uint64_t lo, hi;  // rl, rh in both halves of an f32x2
+  float s;
+};
+
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
 }
 
-__device__ __forceinline__ uint32_t quant4(uint32_t w0, uint32_t w1, float s, float r) {
-  return pack4(quant2(w0, s, r), quant2(w1, s, r));
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
 }
 
-__device__ __forceinline__ uint2 quant8(uint4 v, float s, float r) {
-  uint2 o;
-  o.x = quant4(v.x, v.y, s, r);
-  o.y = quant4(v.z, v.w, s, r);
-  return o;
+// E4M3 codes of the two halves of an f32x2, the low half in the low byte.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(uint64_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return cvt_e4m3x2(lo, hi);
+}
+
+__device__ __forceinline__ QuantBracket quant_bracket(float s) {
+  const float r = __frcp_rn(s);
+  const bool ok = r >= 0x1p-126f && r <= 0x1p126f;
+  const float rl = ok ? __fmul_rn(r, 1.0f - 0x1p-20f) : 0.0f;
+  const float rh = ok ? __fmul_rn(r, 1.0f + 0x1p-20f) : __int_as_float(0x7F800000);
+  return QuantBracket{f32x2(rl, rl), f32x2(rh, rh), s};
+}
+
+// The pairs whose two ends disagree, by IEEE division; out of line so that
+// the common path keeps few registers.
+__device__ __noinline__ uint2 quant8_divide(uint4 v, float s, uint2 lo, uint2 hi) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t c[4] = {lo.x & 0xFFFFu, lo.x >> 16, lo.y & 0xFFFFu, lo.y >> 16};
+  const uint32_t h[4] = {hi.x & 0xFFFFu, hi.x >> 16, hi.y & 0xFFFFu, hi.y >> 16};
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    if (c[k] != h[k]) c[k] = cvt_e4m3x2(__fdiv_rn(bf16_lo(w[k]), s), __fdiv_rn(bf16_hi(w[k]), s));
+  return make_uint2(pack4(c[0], c[1]), pack4(c[2], c[3]));
+}
+
+__device__ __forceinline__ uint2 quant8_bracket(uint4 v, const QuantBracket &q) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t lo[4], hi[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint64_t x = f32x2(bf16_lo(w[k]), bf16_hi(w[k]));
+    lo[k] = cvt_e4m3x2(mul_f32x2(x, q.lo));
+    hi[k] = cvt_e4m3x2(mul_f32x2(x, q.hi));
+  }
+  const uint2 a = make_uint2(pack4(lo[0], lo[1]), pack4(lo[2], lo[3]));
+  const uint2 b = make_uint2(pack4(hi[0], hi[1]), pack4(hi[2], hi[3]));
+  if (a.x == b.x && a.y == b.y) return a;
+  return quant8_divide(v, q.s, a, b);
 }
 
 // zero_words / n_zero: an optional int array cleared by block 0 (the split-K
@@ -195,15 +253,15 @@ __device__ __forceinline__ void quant_static_range(const uint16_t *__restrict__ 
                                                    int nblocks) {
   if (numel <= 0) return;
   const float s = __ldg(s_in);
-  const float r = __frcp_rn(s);
+  const QuantBracket q = quant_bracket(s);
   const int64_t tid = static_cast<int64_t>(block) * blockDim.x + threadIdx.x;
   const int64_t nthreads = static_cast<int64_t>(nblocks) * blockDim.x;
   const int64_t done =
-      stream1<WIDE>(x, numel, xq, tid, nthreads, [s, r](uint4 v) { return quant8(v, s, r); });
+      stream1<WIDE>(x, numel, xq, tid, nthreads, [&q](uint4 v) { return quant8_bracket(v, q); });
   const int64_t t = done + tid;
   if (t < numel) {
     float a = __uint_as_float(static_cast<uint32_t>(x[t]) << 16);
-    xq[t] = static_cast<uint8_t>(quant1(a, s, r));
+    xq[t] = static_cast<uint8_t>(quant1(a, s, quant_recip(s)));
   }
 }
 
@@ -271,6 +329,163 @@ __global__ void __launch_bounds__(kEwThreads)
     quant_static_range<WIDE>(a.x, a.numel, a.s_in, a.xq, blockIdx.x, split);
   else
     quant_static_range<WIDE>(b.x, b.numel, b.s_in, b.xq, blockIdx.x - split, gridDim.x - split);
+}
+
+// ---------------------------------------------------- quantize, staged form
+// The staged quantizer: one CTA per SM (fewer for short inputs).  The input
+// runs (one or two activations, each with its own scale) are cut into chunks
+// of kStagedChunk bytes of whole 8-value vectors, dealt to the CTAs round
+// robin.  A producer thread streams its CTA's chunks into a ring of
+// kStagedStages shared-memory slots with cp.async.bulk, each completing an
+// mbarrier by its byte count; kStagedConsumerWarps warps convert each chunk
+// and store the codes, then release the slot.  The bytes in flight per SM are
+// set by the ring, not by registers, so reads keep streaming while the
+// consumers work.  With two CTAs' worth of shared memory and threads free on
+// each SM, the next launch's CTA can become resident and wait beside it.
+constexpr int kStagedChunk = 16384;  // input bytes per chunk (8192 BF16 values)
+constexpr int kStagedStages = 6;
+constexpr int kStagedConsumerWarps = 16;
+constexpr int kStagedConsumers = kStagedConsumerWarps * 32;
+constexpr int kStagedThreads = kStagedConsumers + 32;  // + the producer warp
+constexpr int kStagedSmem = kStagedStages * kStagedChunk + 2 * kStagedStages * 8 + 16;
+
+__host__ __device__ __forceinline__ int64_t staged_chunks(int64_t numel) {
+  return ((numel >> 3) * 16 + kStagedChunk - 1) / kStagedChunk;
+}
+
+// Chunk c of the two runs: its run, its byte offset in that run's input and
+// its length in bytes (a multiple of 16).
+__device__ __forceinline__ void staged_chunk(const QuantSeg &a, const QuantSeg &b, int64_t ca,
+                                             int64_t c, bool &second, int64_t &off,
+                                             uint32_t &bytes) {
+  second = c >= ca;
+  const QuantSeg &g = second ? b : a;
+  off = (second ? c - ca : c) * kStagedChunk;
+  const int64_t run = (g.numel >> 3) * 16;
+  bytes = static_cast<uint32_t>(run - off < kStagedChunk ? run - off : kStagedChunk);
+}
+
+// a, b: the two runs (b.numel = 0 for one).  Block 0 also clears n_zero words
+// at zero_words and quantizes the fewer than 8 values past each run's last
+// whole vector.  prefetch: before waiting for the previous kernel, the
+// producer prefetches its CTA's chunks into L2.  Waits give up after
+// timeout_ns (device status word, wait sites 7 and 8).
+__global__ void __launch_bounds__(kStagedThreads, 2)
+    quant_staged_kernel(const QuantSeg a, const QuantSeg b, int *__restrict__ zero_words,
+                        int n_zero, int prefetch, uint64_t timeout_ns) {
+  extern __shared__ __align__(128) uint8_t staged_smem[];
+  uint8_t *ring = staged_smem;
+  uint64_t *full = reinterpret_cast<uint64_t *>(staged_smem + kStagedStages * kStagedChunk);
+  uint64_t *empty = full + kStagedStages;
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + kStagedStages);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t ca = staged_chunks(a.numel);
+  const int64_t total = ca + staged_chunks(b.numel);
+  pdl_launch_dependents();
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStagedStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kStagedConsumerWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kStagedConsumerWarps && lane == 0 && prefetch) {
+    for (int64_t c = blockIdx.x; c < total; c += gridDim.x) {
+      bool second;
+      int64_t off;
+      uint32_t bytes;
+      staged_chunk(a, b, ca, c, second, off, bytes);
+      prefetch_l2_bulk(reinterpret_cast<const uint8_t *>(second ? b.x : a.x) + off, bytes);
+    }
+  }
+  __syncthreads();
+  pdl_wait();
+
+  if (warp == kStagedConsumerWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane != 0) return;
+    const uint64_t pol = l2_policy_evict_first();
+    uint32_t issued = 0, parity = 0;
+    bool ok = true;
+    int j = 0;
+    for (int64_t c = blockIdx.x; c < total; c += gridDim.x, ++j) {
+      const int slot = j % kStagedStages;
+      const uint32_t ph = (j / kStagedStages) & 1u;
+      if (!mbar_wait_bounded(&empty[slot], ph ^ 1u, abort_flag, timeout_ns)) {
+        record_timeout(kSiteStagedEmpty);
+        *abort_flag = 1;
+        ok = false;
+        break;
+      }
+      bool second;
+      int64_t off;
+      uint32_t bytes;
+      staged_chunk(a, b, ca, c, second, off, bytes);
+      mbar_arrive_expect_tx(&full[slot], bytes);
+      bulk_load_1d(ring + slot * kStagedChunk,
+                   reinterpret_cast<const uint8_t *>(second ? b.x : a.x) + off, bytes,
+                   &full[slot], pol);
+      issued |= 1u << slot;
+      parity = (parity & ~(1u << slot)) | (ph << slot);
+    }
+    if (!ok) {
+      // let the copies this CTA started land before it can exit
+      int zero = 0;
+      for (int s = 0; s < kStagedStages; ++s)
+        if (issued & (1u << s)) mbar_wait_bounded(&full[s], (parity >> s) & 1u, &zero, timeout_ns);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int t = threadIdx.x;
+  const QuantBracket qa = quant_bracket(a.numel > 0 ? __ldg(a.s_in) : 1.0f);
+  const QuantBracket qb = quant_bracket(b.numel > 0 ? __ldg(b.s_in) : 1.0f);
+  if (blockIdx.x == 0) {
+    for (int i = t; i < n_zero; i += kStagedConsumers) zero_words[i] = 0;
+    // the values past the last whole vector of each run (fewer than 8 each)
+    const int ra = static_cast<int>(a.numel & 7), rb = static_cast<int>(b.numel & 7);
+    if (t < ra) {
+      const int64_t i = a.numel - ra + t;
+      a.xq[i] = static_cast<uint8_t>(
+          quant1(__uint_as_float(static_cast<uint32_t>(a.x[i]) << 16), qa.s, quant_recip(qa.s)));
+    } else if (t >= 8 && t - 8 < rb) {
+      const int64_t i = b.numel - rb + (t - 8);
+      b.xq[i] = static_cast<uint8_t>(
+          quant1(__uint_as_float(static_cast<uint32_t>(b.x[i]) << 16), qb.s, quant_recip(qb.s)));
+    }
+  }
+  int j = 0;
+  for (int64_t c = blockIdx.x; c < total; c += gridDim.x, ++j) {
+    const int slot = j % kStagedStages;
+    const uint32_t ph = (j / kStagedStages) & 1u;
+    if (!mbar_wait_bounded_warp(&full[slot], ph, abort_flag, timeout_ns)) {
+      if (lane == 0) {
+        record_timeout(kSiteStagedFull);
+        *abort_flag = 1;
+      }
+      break;
+    }
+    bool second;
+    int64_t off;
+    uint32_t bytes;
+    staged_chunk(a, b, ca, c, second, off, bytes);
+    const QuantBracket &q = second ? qb : qa;
+    const uint4 *sv = reinterpret_cast<const uint4 *>(ring + slot * kStagedChunk);
+    uint2 *ov = reinterpret_cast<uint2 *>((second ? b.xq : a.xq) + (off >> 1));
+    const int nv = static_cast<int>(bytes >> 4);
+    if (nv == kStagedChunk / 16) {
+      static_assert(kStagedChunk / 16 == 2 * kStagedConsumers, "two vectors per thread");
+      const uint4 v0 = sv[t], v1 = sv[t + kStagedConsumers];
+      st_stream(ov + t, quant8_bracket(v0, q));
+      st_stream(ov + t + kStagedConsumers, quant8_bracket(v1, q));
+    } else {
+      for (int i = t; i < nv; i += kStagedConsumers) st_stream(ov + i, quant8_bracket(sv[i], q));
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[slot]);
+  }
 }
 
 // ------------------------------------------------------ SwiGLU -> FP8
@@ -524,21 +739,22 @@ __global__ void __launch_bounds__(kQuantRowThreads) quant_rows_kernel(
     for (int k = 0; k < HELD; ++k) m = absmax8(v[k], m);
     m = block_max_rows<kQuantRowThreads>(m, red);
     const float s = m > 0.0f ? __fdiv_rn(m, 448.0f) : 1.0f;
-    const float r = __frcp_rn(s);
+    const QuantBracket qb = quant_bracket(s);
     if (threadIdx.x == 0) s_out[row] = s;
 #pragma unroll
     for (int k = 0; k < HELD; ++k) {
       const int i = threadIdx.x + k * kQuantRowThreads;
-      if (i < nvec) st_stream(qv + i, quant8(v[k], s, r));
+      if (i < nvec) st_stream(qv + i, quant8_bracket(v[k], qb));
     }
     return;
   }
   for (int i = threadIdx.x; i < nvec; i += kQuantRowThreads) m = absmax8(__ldg(xv + i), m);
   m = block_max_rows<kQuantRowThreads>(m, red);
   const float s = m > 0.0f ? __fdiv_rn(m, 448.0f) : 1.0f;
-  const float r = __frcp_rn(s);
+  const QuantBracket qb = quant_bracket(s);
   if (threadIdx.x == 0) s_out[row] = s;
-  for (int i = threadIdx.x; i < nvec; i += kQuantRowThreads) qv[i] = quant8(__ldg(xv + i), s, r);
+  for (int i = threadIdx.x; i < nvec; i += kQuantRowThreads)
+    qv[i] = quant8_bracket(__ldg(xv + i), qb);
 }
 
 // One block per row of G, U [rows, I] (I % 8 == 0, I <= kMaxRowI): v =

@@ -60,7 +60,8 @@ struct DeviceInfo {
   int64_t l2_bytes = 0;         // likewise
   // bit per kernel whose attributes were set on this device: 0-2 one-CTA GEMMs,
   // 3/5/6/7 pair GEMM scale modes (+16 direct-store), 9 five-stage pair GEMM,
-  // 4 dual (+8 variant, +16 direct variant, +24 direct plain), 8 per-token SwiGLU
+  // 4 dual (+8 variant, +16 direct variant, +24 direct plain), 8 per-token SwiGLU,
+  // 10 staged quantizer
   std::atomic<unsigned> gemm_attr_set{0};
   std::atomic<int> pair_clusters{0};  // CTA pairs of the pair GEMM resident at once
   std::atomic<int> dual_clusters{0};  // CTA pairs of the gate/up dual GEMM resident at once
@@ -710,9 +711,59 @@ int gemm_groups(DeviceInfo *d, const PairProblem *pp, int np, int K, cudaStream_
 }
 
 // ----------------------------------------------------------- elementwise
+// The quantizer's form, set by fp8ws_set_quant_form: 0 chooses by size
+// (default), 1 the staged kernel, 2 the streaming kernels; FP8WS_QUANT=staged
+// or =stream sets the starting value (timing comparisons).  All give the same
+// codes.  Timed on B200, back to back: the streaming kernels are faster up to
+// an input about as large as L2 (9.4 against 11.6 us for 4096 + 1024 rows x
+// 3072, 4.6 against 5.7 us for 2048 x 3072, 35.8 against 37.4 us for 8192 x
+// 8192, 134 MB); from 1.5 times L2 up the staged kernel's steady stream of
+// reads wins (56.2 against 64.7 us for 12288 x 8192, 78 against 90 us for
+// 16384 x 8192).
+std::atomic<int> g_quant_form{-1};
+bool staged_quant(const DeviceInfo *d, int64_t numel) {
+  int f = g_quant_form.load(std::memory_order_relaxed);
+  if (f < 0) {
+    const char *e = getenv("FP8WS_QUANT");
+    int want = !e ? 0 : (strcmp(e, "staged") == 0 ? 1 : (strcmp(e, "stream") == 0 ? 2 : 0));
+    // keep a form set meanwhile by fp8ws_set_quant_form
+    if (!g_quant_form.compare_exchange_strong(f, want, std::memory_order_relaxed)) want = f;
+    f = want;
+  }
+  if (f == 0) return numel * 4 >= d->l2_bytes * 3;  // BF16 input >= 1.5 x L2
+  return f == 1;
+}
+
+// One or two runs (b.numel = 0 for one) through quant_staged_kernel: one CTA
+// per SM, or one per chunk when there are fewer chunks than SMs.
+int quant_staged_launch(DeviceInfo *d, const QuantSeg &a, const QuantSeg &b, cudaStream_t st,
+                        int *zero_words, int n_zero) {
+  int rc = once_per_device(d, 10, [] {
+    return cudaFuncSetAttribute(quant_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kStagedSmem) == cudaSuccess
+               ? FP8WS_OK
+               : FP8WS_ERR_CUDA;
+  });
+  if (rc) return rc;
+  const int64_t chunks = staged_chunks(a.numel) + staged_chunks(b.numel);
+  const int grid = chunks >= d->sms ? d->sms : (chunks > 0 ? static_cast<int>(chunks) : 1);
+  if (launch_ex(quant_staged_kernel, dim3(grid), dim3(kStagedThreads), kStagedSmem, st, 1, a, b,
+                zero_words, n_zero, prefetch_enabled() ? 1 : 0, kWaitLimitNs) != cudaSuccess)
+    return FP8WS_ERR_CUDA;
+  return FP8WS_OK;
+}
+
 int quant_launch(DeviceInfo *d, const uint16_t *x, int64_t numel, const float *s, uint8_t *xq,
                  cudaStream_t st, int *zero_words = nullptr, int n_zero = 0) {
   if (numel == 0) return FP8WS_OK;
+  if (staged_quant(d, numel)) {
+    const int rc = quant_staged_launch(d, QuantSeg{x, numel, s, xq},
+                                       QuantSeg{nullptr, 0, nullptr, nullptr}, st, zero_words,
+                                       n_zero);
+    if (rc) return rc;
+    log_launch(kKindQuant, x, nullptr, xq);
+    return launch_status();
+  }
   // the first blocks prefetch x into L2 while the previous kernel drains
   if (ew_launch<quant_static_kernel<true>, quant_static_kernel<false>>(
           d, aligned32(x), numel >> 3, st, x, numel, s, xq, zero_words, n_zero,
@@ -738,6 +789,13 @@ int quant_pair_launch(DeviceInfo *d, const QuantSeg *q, int nq, cudaStream_t st,
   if (n == 1)
     return quant_launch(d, live[0].x, live[0].numel, live[0].s_in, live[0].xq, st, zero_words,
                         n_zero);
+  if (staged_quant(d, live[0].numel + live[1].numel)) {
+    const int rc = quant_staged_launch(d, live[0], live[1], st, zero_words, n_zero);
+    if (rc) return rc;
+    log_launch(kKindQuant, live[0].x, nullptr, live[0].xq, 0);
+    log_launch(kKindQuant, live[1].x, nullptr, live[1].xq, 1);
+    return launch_status();
+  }
   const int64_t total = live[0].numel + live[1].numel;
   const bool wide = aligned32(live[0].x) && aligned32(live[1].x);
   int grid = wide ? ew_grid<quant_static_pair_kernel<true>>(d, total >> 3)
@@ -1587,6 +1645,12 @@ int fp8ws_device_status(int *status, int *where) {
 int fp8ws_set_gemm_config(int config) {
   if (config < 0 || config > 4) return FP8WS_ERR_SHAPE;
   g_forced_gemm_config.store(config, std::memory_order_relaxed);
+  return FP8WS_OK;
+}
+
+int fp8ws_set_quant_form(int form) {
+  if (form < 0 || form > 2) return FP8WS_ERR_SHAPE;
+  g_quant_form.store(form, std::memory_order_relaxed);
   return FP8WS_OK;
 }
 

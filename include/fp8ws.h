@@ -611,6 +611,17 @@ FP8WS_API int fp8ws_selftest_bounded_wait(int64_t limit_ns, int mode, int64_t *e
  * FP8WS_ERR_SHAPE for other values. */
 FP8WS_API int fp8ws_set_gemm_config(int config);
 
+/* Form of the static quantizer (fp8_quant_static and the quantization step
+ * of every composite call), for tests and timing; the codes are the same in
+ * every form.  0 = by size (default): the streaming kernels for BF16 inputs
+ * smaller than 1.5 times L2, the staged kernel from there up.  1 = staged: one CTA per SM,
+ * input chunks streamed into a shared-memory ring by the bulk copy engine.
+ * 2 = streaming: each thread loads its own vectors (32 bytes at a time for
+ * 32-byte-aligned inputs).  FP8WS_QUANT=staged or =stream in the environment
+ * sets the starting value.  Applies to later calls from every thread;
+ * FP8WS_ERR_SHAPE for other values. */
+FP8WS_API int fp8ws_set_quant_form(int form);
+
 /* The tile configuration the GEMM cost model picks, for tests and tuning;
  * host only, touches no device, ignores a configuration forced by
  * fp8ws_set_gemm_config.  Problems: M[p] x N[p] outputs for p < count (1..3,

@@ -252,3 +252,12 @@ def test_selftest_argument_checks(lib):
     assert lib.fp8ws_selftest_bounded_wait(0, 0, ctypes.byref(out), None) == fw.ERR_SHAPE
     assert lib.fp8ws_selftest_bounded_wait(5_000_000_000, 0, ctypes.byref(out), None) == fw.ERR_SHAPE
     assert lib.fp8ws_selftest_bounded_wait(1000, 2, ctypes.byref(out), None) == fw.ERR_SHAPE
+
+
+def test_quant_form_switch(lib):
+    """fp8ws_set_quant_form takes 0 (by size), 1 (staged) or 2 (streaming),
+    nothing else; host only."""
+    for bad in (-1, 3, 7):
+        assert lib.fp8ws_set_quant_form(bad) == fw.ERR_SHAPE
+    for good in (2, 1, 0):
+        assert lib.fp8ws_set_quant_form(good) == fw.OK

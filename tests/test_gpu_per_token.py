@@ -29,6 +29,26 @@ def test_quant_rows_bitexact(rows, K):
     assert np.array_equal(codes(q[sample]), rq)
 
 
+def test_quant_rows_of_tiny_magnitude():
+    """Rows whose max |x| is below 448 * 2^-128, so that the row's scale is a
+    subnormal fp32 number and 1/s overflows: codes still the oracle's (the
+    zeros of the row give 0, not a NaN), scales equal."""
+    K = 3072
+    x = synth.activation_with_outliers(4, K, 6, 9, 0, DEV).float()
+    x = x / x.abs().amax(dim=1, keepdim=True)
+    x[0] *= 1e-37
+    x[1] *= 3e-39
+    x[2] *= 1e-36
+    x[3] *= 1e-30          # an ordinary small row beside them
+    x = x.to(torch.bfloat16)
+    x[:, ::7] = 0
+    q, s = fw.fp8_quant_per_token(x)
+    rq, rs = oracle.quantize_rows(bits(x))
+    assert (rs[:3] < 2.0 ** -126).all()
+    assert np.array_equal(s.cpu().numpy(), rs)
+    assert np.array_equal(codes(q), rq)
+
+
 def test_per_channel_weights_bitexact():
     w = synth.normal((1024, 3072), 0.02, 71, DEV)
     q, s = fw.fp8_quant_per_token(w)

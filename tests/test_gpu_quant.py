@@ -13,6 +13,13 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
+@pytest.fixture(params=["staged", "stream", "auto"])
+def quant_form(request):
+    fw.set_quant_form(request.param)
+    yield request.param
+    fw.set_quant_form("auto")
+
+
 def _check(x_bits, s):
     x = from_bits(x_bits, DEV)
     q = codes(fw.fp8_quant_static(x, scalar(s, DEV)))
@@ -22,10 +29,17 @@ def _check(x_bits, s):
     assert np.array_equal(q[~nan], ref[~nan])
 
 
-@pytest.mark.parametrize("s", [1.0, 2.0 ** -10, 0.0123, 3.7, 1e-6, 1e4])
-def test_every_bf16_pattern(s):
+@pytest.mark.parametrize("s", [1.0, 2.0 ** -10, 0.0123, 3.7, 1e-6, 1e4,
+                               1e-39,        # subnormal: 1/s overflows to inf
+                               2.0 ** -126,  # smallest normal: 1/s = 2^126
+                               2.0 ** 127,   # 1/s subnormal
+                               3e38])
+def test_every_bf16_pattern(s, quant_form):
     """All 65536 BF16 bit patterns (zeros, subnormals, NaN, inf, everything in
-    between) against the oracle at several scales."""
+    between) against the oracle at several scales, in both forms of the
+    quantizer.  At the last four scales the reciprocal-based tests of the
+    kernels cannot be trusted and every value goes to IEEE division; an input
+    of 0 must still give the code 0 (0 * inf would be a NaN)."""
     _check(np.arange(65536, dtype=np.uint32).astype(np.uint16), oracle.f32(s))
 
 
@@ -51,8 +65,11 @@ def test_c3_input():
     _check(bits(d["x"]), s)
 
 
-@pytest.mark.parametrize("n", [1, 7, 8, 9, 15, 17, 4095, 1_000_003])
-def test_ragged_lengths(n):
+@pytest.mark.parametrize("n", [1, 7, 8, 9, 15, 17, 4095, 8191, 8192, 8199, 1_000_003,
+                               148 * 8192 + 13])
+def test_ragged_lengths(n, quant_form):
+    """Lengths around the staged form's 8192-value chunks and one CTA per SM,
+    and tails of fewer than 8 values."""
     rng = np.random.default_rng(n)
     x = torch.from_numpy((rng.standard_t(3, size=n) * 40).astype(np.float32)).to(torch.bfloat16)
     _check(bits(x), oracle.f32(0.071))
@@ -70,6 +87,23 @@ def test_rank3_input_flat():
     q = fw.fp8_quant_static(x, scalar(0.05, DEV))
     assert q.shape == x.shape
     assert np.array_equal(codes(q).ravel(), oracle.quantize(bits(x).ravel(), oracle.f32(0.05)))
+
+
+def test_forms_agree_on_two_tower_group():
+    """The pass's grouped quantization (4096 + 1024 rows x 3072): the staged
+    and the streaming forms write the same codes, byte for byte."""
+    xs = [synth.activation_with_outliers(M, 3072, 4, 2, t, DEV) for t, M in enumerate((4096, 1024))]
+    ss = [scalar(0.0417, DEV), scalar(0.0213, DEV)]
+    out = {}
+    try:
+        for form in ("staged", "stream"):
+            fw.set_quant_form(form)
+            out[form] = [codes(q) for q in fw.fp8_quant_static_group(xs, ss)]
+    finally:
+        fw.set_quant_form("auto")
+    for a, b in zip(out["staged"], out["stream"]):
+        assert np.array_equal(a, b)
+    assert fw.device_status()[0] == fw.OK
 
 
 def test_large_bench_size():

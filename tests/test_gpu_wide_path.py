@@ -6,7 +6,10 @@ size), so the lengths here (all short) run the wide form when aligned and the
 16-byte form when shifted.  Both forms give the oracle's codes and the same codes as each
 other, byte for byte, on lengths that exercise every tail (fewer than 16
 leftover elements).  The long lengths of the workloads' sweeps run in the
-parity tests of each kernel."""
+parity tests of each kernel.  The quantizer also has a staged form (input
+chunks moved by the bulk copy engine; 16-byte alignment is all it needs),
+which it takes by default only for inputs of 1.5 times L2 and more, so the quantizer
+tests here select the streaming form explicitly."""
 
 import numpy as np
 import pytest
@@ -40,6 +43,13 @@ def _aligned(t):
 LENGTHS = [1, 8, 9, 15, 16, 17, 31, 33, 4095, 65_543, 1_000_003]
 
 
+@pytest.fixture
+def stream_form():
+    fw.set_quant_form("stream")
+    yield
+    fw.set_quant_form("auto")
+
+
 def _heavy(n, seed, scale=40.0):
     rng = np.random.default_rng(seed)
     x = (rng.standard_t(3, size=n) * scale).astype(np.float32)
@@ -47,7 +57,7 @@ def _heavy(n, seed, scale=40.0):
 
 
 @pytest.mark.parametrize("n", LENGTHS)
-def test_quant_forms_agree_with_oracle(n):
+def test_quant_forms_agree_with_oracle(n, stream_form):
     x = _aligned(_heavy(n, n))
     s = oracle.f32(0.071)
     q_wide = codes(fw.fp8_quant_static(x, scalar(s, DEV)))
@@ -59,7 +69,7 @@ def test_quant_forms_agree_with_oracle(n):
     assert np.array_equal(q_wide[~nan], ref[~nan])
 
 
-def test_quant_every_bf16_pattern_narrow_form():
+def test_quant_every_bf16_pattern_narrow_form(stream_form):
     """All 65536 BF16 patterns through the 16-byte form."""
     x = torch.from_numpy(np.arange(65536, dtype=np.uint32).astype(np.uint16).view(np.int16))
     x = x.view(torch.bfloat16).to(DEV)
@@ -69,6 +79,29 @@ def test_quant_every_bf16_pattern_narrow_form():
     nan = is_nan_code(ref)
     assert np.array_equal(is_nan_code(q), nan)
     assert np.array_equal(q[~nan], ref[~nan])
+
+
+@pytest.mark.parametrize("n", LENGTHS)
+def test_staged_quant_on_shifted_input(n):
+    """The staged form on an input 16 bytes past a 32-byte boundary gives the
+    codes it gives on the aligned copy, and the oracle's."""
+    fw.set_quant_form("staged")
+    try:
+        _staged_shifted_check(n)
+    finally:
+        fw.set_quant_form("auto")
+
+
+def _staged_shifted_check(n):
+    x = _aligned(_heavy(n, n + 1))
+    s = oracle.f32(0.071)
+    q_aligned = codes(fw.fp8_quant_static(x, scalar(s, DEV)))
+    q_shifted = codes(fw.fp8_quant_static(_shifted(x), scalar(s, DEV)))
+    assert np.array_equal(q_aligned, q_shifted)
+    ref = oracle.quantize(bits(x), s)
+    nan = is_nan_code(ref)
+    assert np.array_equal(is_nan_code(q_aligned), nan)
+    assert np.array_equal(q_aligned[~nan], ref[~nan])
 
 
 def _swiglu_check(h, g, u, s):
@@ -105,7 +138,7 @@ def test_swiglu_variant_forms_agree(n):
 
 
 @pytest.mark.parametrize("M0,M1,K", [(129, 33, 3072), (5, 1, 24), (1000, 64, 272)])
-def test_group_quant_forms(M0, M1, K):
+def test_group_quant_forms(M0, M1, K, stream_form):
     """The grouped quantizer takes the wide form only when both activations are
     32-byte aligned; one shifted activation moves both to the 16-byte form."""
     xs = [synth.normal((M, K), 1.0, M + K, DEV) for M in (M0, M1)]
