@@ -106,6 +106,26 @@ def test_forms_agree_on_two_tower_group():
     assert fw.device_status()[0] == fw.OK
 
 
+def test_default_form_above_l2():
+    """12288 x 8192 (201 MB of BF16, past 1.5 x L2, where the default form is
+    the staged kernel): the same codes as the streaming form, byte for byte,
+    and the oracle's on stratified rows."""
+    M, K = 12288, 8192
+    x = synth.activation_with_outliers(M, K, 4, 3, 0, DEV)
+    s = oracle.f32(0.0389)
+    q_auto = fw.fp8_quant_static(x, scalar(s, DEV))
+    fw.set_quant_form("stream")
+    try:
+        q_stream = fw.fp8_quant_static(x, scalar(s, DEV))
+    finally:
+        fw.set_quant_form("auto")
+    assert torch.equal(q_auto.view(torch.uint8), q_stream.view(torch.uint8))
+    rows = stratified_rows(M, 4)
+    xb = bits(x[rows])
+    assert np.array_equal(codes(q_auto[rows]), oracle.quantize(xb, s))
+    assert fw.device_status()[0] == fw.OK
+
+
 def test_large_bench_size():
     """Full size of the largest activation the two-tower pass quantizes."""
     x = synth.activation_with_outliers(4096, 3072, 4, 1, 0, DEV)
