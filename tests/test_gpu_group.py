@@ -48,12 +48,20 @@ def _check_gemm(y, xq, wq, s_in, s_w, rows=None):
 # ------------------------------------------------------------------ quantize
 
 
+@pytest.mark.parametrize("form", ["stream", "staged"])
 @pytest.mark.parametrize("n0,n1", [(4096 * 3072, 1024 * 3072), (7, 100_003), (1, 1),
-                                   (0, 4097), (4097, 0), (64 * 256, 64 * 256)])
-def test_quant_group_against_oracle(n0, n1):
+                                   (0, 4097), (4097, 0), (64 * 256, 64 * 256), (8195, 13),
+                                   (131_079, 8_189)])
+def test_quant_group_against_oracle(n0, n1, form):
+    """Both forms of the quantizer; ragged runs leave fewer than 8 values past
+    the last whole vector of either run, or of both at once."""
     xs = [synth.normal((max(n0, 1),), 3.0, 1, DEV)[:n0], synth.normal((max(n1, 1),), 0.5, 2, DEV)[:n1]]
     s = [oracle.f32(0.0213), oracle.f32(0.00317)]
-    outs = fw.fp8_quant_static_group(xs, [scalar(v, DEV) for v in s])
+    fw.set_quant_form(form)
+    try:
+        outs = fw.fp8_quant_static_group(xs, [scalar(v, DEV) for v in s])
+    finally:
+        fw.set_quant_form("auto")
     for x, o, sv in zip(xs, outs, s):
         ref = oracle.quantize(bits(x), sv) if x.numel() else np.zeros(0, np.uint8)
         assert np.array_equal(codes(o), ref)
