@@ -748,12 +748,21 @@ class OracleSample:
                 f"time per row extrapolated to the 36-layer pass")
 
 
-def cpu_baseline(rows_per_tower: int = 1024):
+def cpu_baseline(rows_per_tower: int = 1024, single_rows: int = 64):
+    """The oracle on all host cores, and separately on one thread (a smaller
+    sample: about the same wall time)."""
     o = OracleSample()
     t0 = time.perf_counter()
     spt = o.run(rows_per_tower)
     wall = time.perf_counter() - t0
-    return o.tokens_per_s(spt), o.cores, o.describe(rows_per_tower, wall)
+    o.oracle.set_num_threads(1)
+    t0 = time.perf_counter()
+    spt1 = o.run(single_rows)
+    wall1 = time.perf_counter() - t0
+    o.oracle.set_num_threads(o.cores)
+    single = {"value": o.tokens_per_s(spt1), "threads": 1,
+              "sample": f"{single_rows} rows of layer {o.layer} of each tower, {wall1:.1f}s wall"}
+    return o.tokens_per_s(spt), o.cores, o.describe(rows_per_tower, wall), single
 
 
 # ------------------------------------------------------- single kernels
@@ -1416,8 +1425,9 @@ def main():
 
     cpu = None
     if ctx.rank == 0 and ctx.world == 1 and not args.no_cpu_baseline:
-        tps, cores, sample = cpu_baseline()
-        cpu = {"value": tps, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+        tps, cores, sample, single = cpu_baseline()
+        cpu = {"value": tps, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+               "nproc": os.cpu_count(), "single_thread": single}
 
     configs = None
     if ctx.world == 1 and not args.no_configs:
