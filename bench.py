@@ -1125,16 +1125,19 @@ SWEEPS = {
 
 # the workloads whose figures go into the default run's line (key "configs")
 CONFIG_REPLAYS = 50
-LINE_CONFIGS = ("c0", "c1", "c2", "c3", "per_token", "xattn", "variants")
+# fp8ceil: the measured FP8 ceiling, cuBLASLt (torch._scaled_mm) beside our GEMM at the same shapes
+LINE_CONFIGS = ("c0", "c1", "c2", "c3", "per_token", "xattn", "variants", "fp8ceil")
 
 
 def config_figures(fw, device, steps, warmup, log):
     """The default run's per-workload kernel figures: every shape of the
     Linear sweep (c1), the SwiGLU sweep (c2), the shared-quant Q/K/V block
     (c3, whole call and its grouped GEMM alone), the tiny MLP (c0), the
-    per-token path, the cross-attention projections and the SwiGLU variant
-    (element-wise, and in the gate/up epilogue beside the plain one), each
-    timed back to back with rotating buffers and alone after an L2 flush."""
+    per-token path, the cross-attention projections, the SwiGLU variant
+    (element-wise, and in the gate/up epilogue beside the plain one) and the
+    measured FP8 ceiling (cuBLASLt's FP8 GEMM beside ours at 8192^3 and the
+    two-tower shapes), each timed back to back with rotating buffers and alone
+    after an L2 flush."""
     pk = peaks()
     out = {"timing": f"back to back over buffer sets spanning >= {ROTATE_BYTES >> 20} MB (twice "
                      f"the L2), median of {steps} CUDA-graph replays of >= {MIN_PER_REPLAY} "
