@@ -83,6 +83,9 @@ enum {
  * s_in: device, one fp32 value.
  * xq: device, numel FP8 codes (written).
  * numel >= 0 (0 launches nothing).
+ * The codes are those of the IEEE quotient for every value of s_in, a zero or
+ * subnormal scale included, whichever form of the kernel runs
+ * (fp8ws_set_quant_form).
  */
 FP8WS_API int fp8_quant_static(const uint16_t *x, int64_t numel, const float *s_in, uint8_t *xq,
                      void *stream);
