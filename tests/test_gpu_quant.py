@@ -33,13 +33,16 @@ def _check(x_bits, s):
                                1e-39,        # subnormal: 1/s overflows to inf
                                2.0 ** -126,  # smallest normal: 1/s = 2^126
                                2.0 ** 127,   # 1/s subnormal
-                               3e38])
+                               3e38,
+                               0.0, -0.0123, float("inf"), float("nan")])  # outside any calibration
 def test_every_bf16_pattern(s, quant_form):
     """All 65536 BF16 bit patterns (zeros, subnormals, NaN, inf, everything in
     between) against the oracle at several scales, in both forms of the
-    quantizer.  At the last four scales the reciprocal-based tests of the
-    kernels cannot be trusted and every value goes to IEEE division; an input
-    of 0 must still give the code 0 (0 * inf would be a NaN)."""
+    quantizer.  From 1e-39 on, the reciprocal-based tests of the kernels
+    cannot be trusted and every value goes to IEEE division; an input of 0
+    must still give the code 0 at a subnormal scale (0 * inf would be a NaN),
+    and zero, negative, infinite and NaN scales give the IEEE quotient's codes
+    too."""
     _check(np.arange(65536, dtype=np.uint32).astype(np.uint16), oracle.f32(s))
 
 
