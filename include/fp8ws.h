@@ -593,7 +593,11 @@ FP8WS_API int fp8ws_device_check(void);
 
 /* Read and clear the device status word of the current device (synchronizes
  * the device).  *status receives FP8WS_OK or FP8WS_ERR_DEVICE_TIMEOUT;
- * *where receives a code naming the wait that ran out (0 if none). */
+ * *where receives a code naming the wait that ran out (0 if none): in the
+ * GEMMs 1 (producer, free stage), 2 (MMA, loaded stage), 3 (MMA, free
+ * accumulator), 4 (epilogue, finished accumulator), 5 (teardown, last MMAs);
+ * 6 the self-test below; in the staged quantizer 7 (consumers, loaded chunk),
+ * 8 (producer, free slot). */
 FP8WS_API int fp8ws_device_status(int *status, int *where);
 
 /* Self-test of the bounded waits every GEMM kernel uses (failure detection
