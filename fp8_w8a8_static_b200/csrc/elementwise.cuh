@@ -761,8 +761,13 @@ __global__ void __launch_bounds__(kQuantRowThreads) quant_rows_kernel(
 // SiLU(g) * u in fp32 kept in shared memory, s[r] = max|v| / 448 (1 for an
 // all-zero row), h = E4M3(v * (1/s)).
 constexpr int kMaxRowI = 16384;
-constexpr int kRowBatch = 4;  // vector pairs a thread loads before using the first
 
+// BATCH: vector pairs a thread loads before using the first.  The host takes
+// BATCH = 6 for rows of 5 or 6 pairs per thread (8192 < I <= 12288), so that a
+// row costs one memory round trip, and 4 otherwise (72 against 59 registers:
+// three blocks per SM instead of four where one round trip is not reached
+// anyway).
+template <int BATCH>
 __global__ void __launch_bounds__(kRowThreads) silu_mul_rows_kernel(
     const uint16_t *__restrict__ g, const uint16_t *__restrict__ u, int I,
     float *__restrict__ s_out, uint8_t *__restrict__ h) {
@@ -775,12 +780,12 @@ __global__ void __launch_bounds__(kRowThreads) silu_mul_rows_kernel(
   const uint4 *uv = reinterpret_cast<const uint4 *>(u + row * I);
   const int nvec = I >> 3;
   float m = 0.0f;
-  // kRowBatch vector pairs per thread are loaded before the first is used, so
-  // a row costs one or two memory round trips instead of one per vector
-  for (int base = threadIdx.x; base < nvec; base += kRowThreads * kRowBatch) {
-    uint4 a[kRowBatch], b[kRowBatch];
+  // BATCH vector pairs per thread are loaded before the first is used, so a
+  // row costs one or two memory round trips instead of one per vector
+  for (int base = threadIdx.x; base < nvec; base += kRowThreads * BATCH) {
+    uint4 a[BATCH], b[BATCH];
 #pragma unroll
-    for (int k = 0; k < kRowBatch; ++k) {
+    for (int k = 0; k < BATCH; ++k) {
       const int i = base + k * kRowThreads;
       if (i < nvec) {
         a[k] = ld_stream(gv + i);
@@ -788,7 +793,7 @@ __global__ void __launch_bounds__(kRowThreads) silu_mul_rows_kernel(
       }
     }
 #pragma unroll
-    for (int k = 0; k < kRowBatch; ++k) {
+    for (int k = 0; k < BATCH; ++k) {
       const int i = base + k * kRowThreads;
       if (i < nvec) {
         float v[8] = {silu_mul(bf16_lo(a[k].x), bf16_lo(b[k].x)),

@@ -82,9 +82,14 @@ def test_linear_scaled(x_vec, w_vec):
         assert torch.equal(y, fw.fp8_linear_static(xq, wq, sx, sw))
 
 
-def test_silu_mul_per_token():
-    g = synth.normal((256, 12288), 2.0, 73, DEV)
-    u = synth.normal((256, 12288), 1.0, 74, DEV)
+@pytest.mark.parametrize("rows,I", [(256, 12288), (64, 8192), (64, 8200), (64, 12296),
+                                    (32, 16384), (300, 264)])
+def test_silu_mul_per_token(rows, I):
+    """Rows of 4 to 8 vector pairs per thread: 5 or 6 (8192 < I <= 12288) load
+    in one batch of 6, the others in batches of 4; within the SwiGLU bar of
+    the oracle either way, scales within fp32 rounding of its fp64 ones."""
+    g = synth.normal((rows, I), 2.0, 73, DEV)
+    u = synth.normal((rows, I), 1.0, 74, DEV)
     g[5] = 0
     h, s = fw.silu_mul_2in_fp8_per_token(g, u)
     rh, rs = oracle.silu_mul_2in_rows(bits(g), bits(u))
