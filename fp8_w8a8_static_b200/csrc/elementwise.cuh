@@ -764,11 +764,13 @@ constexpr int kMaxRowI = 16384;
 
 // BATCH: vector pairs a thread loads before using the first.  The host takes
 // BATCH = 6 for rows of 5 or 6 pairs per thread (8192 < I <= 12288), so that a
-// row costs one memory round trip, and 4 otherwise (72 against 59 registers:
+// row costs one memory round trip, and 4 otherwise (80 against 64 registers:
 // three blocks per SM instead of four where one round trip is not reached
-// anyway).
+// anyway).  The batch of 4 is held to four blocks' registers (64; 26.9 against
+// 27.5 us at 4096 x 8192 with the compiler's own 59); the batch of 6 to three
+// blocks' (at 64 registers it spills: 56.7 against 41.0 us at 4096 x 12288).
 template <int BATCH>
-__global__ void __launch_bounds__(kRowThreads) silu_mul_rows_kernel(
+__global__ void __launch_bounds__(kRowThreads, BATCH == 4 ? 4 : 3) silu_mul_rows_kernel(
     const uint16_t *__restrict__ g, const uint16_t *__restrict__ u, int I,
     float *__restrict__ s_out, uint8_t *__restrict__ h) {
   extern __shared__ float vrow[];
