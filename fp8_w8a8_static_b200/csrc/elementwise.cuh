@@ -545,8 +545,12 @@ __device__ __forceinline__ uint2 swiglu_quant8(uint4 g, uint4 u, float inv_s,
   return o;
 }
 
+// Register caps (both two-input SwiGLU kernels): the 16-byte form at six blocks
+// per SM (40 registers instead of 64; four blocks before): 26.5 against 27.2 us
+// at 4096 x 8192, the same within 0.3% at 4096 x 12288, on one box.  The wide
+// form keeps the compiler's choice (0: no minimum); six blocks cost it 1-2%.
 template <bool WIDE>
-__global__ void __launch_bounds__(kEwThreads) swiglu_2in_kernel(
+__global__ void __launch_bounds__(kEwThreads, WIDE ? 0 : 6) swiglu_2in_kernel(
     const uint16_t *__restrict__ g, const uint16_t *__restrict__ u, int64_t numel,
     const float *__restrict__ s_down, SwigluParams p, uint8_t *__restrict__ h) {
   pdl_launch_dependents();
@@ -580,7 +584,7 @@ __device__ __forceinline__ uint2 silu_mul_quant8(uint4 g, uint4 u, float inv_s) 
 }
 
 template <bool WIDE>
-__global__ void __launch_bounds__(kEwThreads) silu_mul_2in_kernel(
+__global__ void __launch_bounds__(kEwThreads, WIDE ? 0 : 6) silu_mul_2in_kernel(
     const uint16_t *__restrict__ g, const uint16_t *__restrict__ u, int64_t numel,
     const float *__restrict__ s_down, uint8_t *__restrict__ h) {
   pdl_launch_dependents();
