@@ -3,6 +3,11 @@
 Bar: relative Frobenius error <= 1e-2 (the stated requirement), and every
 element within one BF16 step plus a worst-case fp32 accumulation error."""
 
+import os
+import subprocess
+import sys
+import textwrap
+
 import numpy as np
 import pytest
 import torch
@@ -190,6 +195,48 @@ def test_tail_halves_against_oracle(M, N, K):
     finally:
         fw.set_gemm_config("auto")
     assert fw.device_status()[0] == fw.OK
+
+
+_HALVES_CHILD = textwrap.dedent("""
+    import hashlib, sys
+    import numpy as np, torch
+    sys.path.insert(0, {root!r})
+    sys.path.insert(0, {tests!r})
+    import fp8_w8a8_static_b200 as fw
+    from _util import from_codes, scalar
+    fw.set_gemm_config("pair256")
+    out = []
+    for M, N, K in {shapes!r}:
+        rng = np.random.default_rng(M * 31 + N * 7 + K)
+        xq = rng.integers(0, 0x7F, (M, K), dtype=np.uint8) | (rng.integers(0, 2, (M, K), dtype=np.uint8) << 7)
+        wq = rng.integers(0, 0x7F, (N, K), dtype=np.uint8) | (rng.integers(0, 2, (N, K), dtype=np.uint8) << 7)
+        xq[(xq & 0x7F) == 0x7F] = 0x00   # no NaN codes
+        wq[(wq & 0x7F) == 0x7F] = 0x00
+        y = fw.fp8_linear_static(from_codes(xq, "cuda"), from_codes(wq, "cuda"), scalar(0.011, "cuda"),
+                                 scalar(0.0023, "cuda"))
+        out.append(hashlib.sha256(y.cpu().view(torch.int16).numpy().tobytes()).hexdigest())
+    print(" ".join(out))
+""")
+
+
+def test_tail_halves_bit_identical_to_whole_tiles():
+    """A 256 x 128 half (an N = 128 MMA over 64-row boxes of B) gives every
+    element the bits the whole 256 x 256 tile gives: the same seeded GEMMs,
+    run in a child process with the halves switched off (FP8WS_TAIL_HALVES=0,
+    read once per process), hash to the same bytes."""
+    shapes = [(300, 520, 1040), (2048, 3072, 3072), (256, 19008, 256)]
+    for M, N, K in shapes:
+        assert fw.split_plan(-(-M // 256) * -(-N // 256), 74, -(-K // 128), scratch=False)["halves"] == 2
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = _HALVES_CHILD.format(root=root, tests=os.path.join(root, "tests"), shapes=shapes)
+    hashes = {}
+    for halves in ("1", "0"):
+        env = dict(os.environ, FP8WS_TAIL_HALVES=halves)
+        r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=600,
+                           env=env)
+        assert r.returncode == 0, r.stdout + r.stderr
+        hashes[halves] = r.stdout.split()
+    assert len(hashes["1"]) == len(shapes) and hashes["1"] == hashes["0"]
 
 
 @pytest.mark.parametrize("x_rows,w_cols", [(False, False), (True, False), (False, True),
