@@ -265,26 +265,11 @@ __device__ __forceinline__ void quant_static_range(const uint16_t *__restrict__ 
   }
 }
 
-// prefetch_share_l2 and the prefetch_blocks argument: see quant_static_pair_kernel.
-__device__ __forceinline__ void prefetch_share_l2(const void *p, int64_t n, int blk, int nblk);
-
-template <bool WIDE>
-__global__ void __launch_bounds__(kEwThreads) quant_static_kernel(
-    const uint16_t *__restrict__ x, int64_t numel, const float *__restrict__ s_in,
-    uint8_t *__restrict__ xq, int *__restrict__ zero_words, int n_zero, int prefetch_blocks) {
-  pdl_launch_dependents();
-  if (threadIdx.x == 0 && prefetch_blocks > 0)
-    prefetch_share_l2(x, numel * 2, blockIdx.x, prefetch_blocks);
-  pdl_wait();
-  if (blockIdx.x == 0)
-    for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero_words[i] = 0;
-  quant_static_range<WIDE>(x, numel, s_in, xq, blockIdx.x, gridDim.x);
-}
-
 // Two activations, each with its own scale, quantized by one launch (the two
 // towers of a layer): blocks 0 .. split - 1 take the first, the rest the
-// second.  Block 0 also clears n_zero words at zero_words (split-K counters of
-// a later kernel), as quant_static_kernel does.
+// second; one activation is the case of an empty second one and split equal
+// to the grid.  Block 0 also clears n_zero words at zero_words (split-K
+// counters of a later kernel).
 struct QuantSeg {
   const uint16_t *x;
   int64_t numel;
