@@ -74,3 +74,39 @@ def test_fused_mlp_and_qkv_graph_replay():
     assert torch.equal(y, eager)
     for a, b in zip(qo, q_eager):
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("form", ["staged", "stream"])
+def test_quantizer_forms_graph_replay(form):
+    """Both forms of the quantizer, captured in a graph as the first step of
+    the grouped gated MLP and on their own, replay to the eager codes; the
+    staged form's mbarrier ring and bulk copies are set up anew in every
+    replayed launch."""
+    fw.set_quant_form(form)
+    try:
+        M0, M1, d, I = 300, 96, 512, 1040
+        towers = [_tower(M0, d, I, 11, 0.003), _tower(M1, d, I, 12, 0.0035)]
+        # 6,408,693 values: 783 chunks of 16 KB in the staged form, the last partial, and a
+        # 5-value tail past the last whole vector
+        x = synth.activation_with_outliers(1031, 6216, 4, 13, 0, DEV).flatten()[:-3]
+        s = scalar(0.021, DEV)
+        ws = torch.empty(fw.gated_mlp_static_fp8_group_workspace([M0, M1], d, I),
+                         dtype=torch.uint8, device=DEV)
+        eager = [y.clone() for y in fw.gated_mlp_static_fp8_group(towers, workspace=ws)]
+        q_eager = fw.fp8_quant_static(x, s).clone()
+        torch.cuda.synchronize()
+        outs = [torch.empty_like(y) for y in eager]
+        q = torch.empty_like(q_eager)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fw.gated_mlp_static_fp8_group(towers, workspace=ws, outs=outs)
+            fw.fp8_quant_static(x, s, out=q)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        for o, e in zip(outs, eager):
+            assert torch.equal(o, e)
+        assert torch.equal(q.view(torch.uint8), q_eager.view(torch.uint8))
+        assert fw.device_status()[0] == fw.OK
+    finally:
+        fw.set_quant_form("auto")
