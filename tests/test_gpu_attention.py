@@ -3,7 +3,6 @@ own quantization), the general shared-quant projection call, and
 cross-attention Q/K/V, where Q reads the query-side activation and K/V a
 different tensor, so Q does not share their quantization."""
 
-import numpy as np
 import pytest
 import torch
 

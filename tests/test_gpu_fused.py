@@ -14,8 +14,8 @@ import torch
 import fp8_w8a8_static_b200 as fw
 import oracle
 import synth
-from _util import (GEMM_REL_FRO, SWIGLU_MAX_FRAC, bits, code_step_diff, codes, from_codes,
-                   rel_fro, scalar, stratified_rows)
+from _util import (GEMM_REL_FRO, SWIGLU_MAX_FRAC, bits, code_step_diff, codes, rel_fro,
+                   scalar, stratified_rows)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"

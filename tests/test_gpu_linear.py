@@ -15,8 +15,8 @@ import torch
 import fp8_w8a8_static_b200 as fw
 import oracle
 import synth
-from _util import (GEMM_REL_FRO, bits, codes, from_codes, gemm_elementwise_bound_ok, rel_fro,
-                   scalar, stratified_rows)
+from _util import (GEMM_REL_FRO, bits, from_codes, gemm_elementwise_bound_ok, rel_fro, scalar,
+                   stratified_rows)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"

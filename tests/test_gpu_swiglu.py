@@ -11,8 +11,8 @@ import torch
 import fp8_w8a8_static_b200 as fw
 import oracle
 import synth
-from _util import (SWIGLU_MAX_FRAC, SWIGLU_MAX_STEP, bits, code_step_diff, codes, from_bits,
-                   scalar, stratified_rows)
+from _util import (SWIGLU_MAX_FRAC, SWIGLU_MAX_STEP, bits, code_step_diff, codes, scalar,
+                   stratified_rows)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
