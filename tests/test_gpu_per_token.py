@@ -18,11 +18,12 @@ DEV = "cuda"
 
 
 @pytest.mark.parametrize("rows,K", [(1, 8), (7, 264), (300, 3072), (4096, 3072),
-                                    (9, 1032), (33, 4096), (5, 4104), (3, 8200), (2, 16384)])
+                                    (9, 1032), (17, 3080), (33, 4096), (5, 4104), (3, 8200),
+                                    (2, 16384)])
 def test_quant_rows_bitexact(rows, K):
-    """One block per row: rows of up to 4096 values held in registers (4
-    vectors per thread), up to 8192 (8 per thread), longer ones read twice;
-    codes and scales bit-exact in each regime and at its edges."""
+    """One block per row: rows of up to 3072 values held in registers as 3
+    vectors per thread, up to 4096 as 4, up to 8192 as 8, longer ones read
+    twice; codes and scales bit-exact in each regime and at its edges."""
     x = synth.activation_with_outliers(rows, K, 6, rows, 0, DEV)
     if rows > 3:
         x[2] = 0  # an all-zero row
